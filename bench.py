@@ -1,0 +1,462 @@
+"""Benchmark of the UFP4 hot path on B200.
+
+One step = the whole data-parallel hot path of one linear layer of LLM
+pretraining under the UFP4 recipe: RHT + block-scale + 4-bit quantize of every
+GEMM operand along its reduction dimension (X and W: RTNE; dY: stochastic
+rounding, Philox seed 1234) and the three training GEMMs
+    FPROP Y = X W^T,  DGRAD dX = dY W,  WGRAD dW = dY^T X
+on X [8192, 2048] ~ N(0,1) with 10 outlier channels x30, W [8192, 2048]
+~ N(0, 0.02), dY [8192, 8192] ~ N(0, 1e-3); RHT16, scale block 16, E1M2 grid.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--scale two-level|fp32]
+
+Prints one JSON line (rank 0).  `value` is the effective UFP4 GEMM throughput of
+the whole step: 3 * 2*M*N*K / step time (quantization included).  Multi-GPU
+runs are independent replicas (the path has no exchange step): weak scaling,
+time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from fp4_quantized_gemms_b200 import workloads as wl  # noqa: E402
+
+METRIC = "UFP4 GEMM TFLOPS & % tensor peak; RHT-quantize HBM GB/s & % of 8 TB/s"
+SHAPE = wl.LAYER
+SR_SEED = 1234
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(scale: str) -> dict:
+    s = SHAPE
+    return {
+        "workload": (f"one linear layer, all three GEMMs: X bf16 {s.M}x{s.K} ~N(0,1) with 0.5% "
+                     f"outlier channels x30, W bf16 {s.N}x{s.K} ~N(0,0.02), dY bf16 {s.M}x{s.N} "
+                     f"~N(0,1e-3); RHT16 on every operand along its K, block 16, E1M2; "
+                     f"RTNE X/W, SR (Philox seed {SR_SEED}) dY"),
+        "scales": "E4M3 block x fp32 tensor (two-level)" if scale == "two-level" else "fp32 per block",
+        "M": s.M, "K": s.K, "N": s.N,
+        "gemm_flops_per_step": 3 * 2 * s.M * s.N * s.K,
+        "l2": "inputs larger than L2: one step reads and writes ~0.9 GB (outputs 0.4 GB)",
+    }
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        loaded = [v for v in sm if v > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ device arm
+def to_dev(bits: np.ndarray, device) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+class LayerStep:
+    """Preallocated buffers and one call sequence of the hot path."""
+
+    def __init__(self, device, scale: str):
+        from fp4_quantized_gemms_b200 import ufp4
+        self.u = ufp4
+        self.dev = device
+        two = scale == "two-level"
+        fmt = ufp4.SCALE_E4M3_X_FP32 if two else ufp4.SCALE_FP32
+        base = ufp4.QuantConfig(grid=ufp4.GRID_E1M2, hadamard_n=16, block=16, scale_fmt=fmt)
+        self.two = two
+        self.c_rtne = base
+        self.c_sr0 = base.with_(rounding=ufp4.ROUND_SR, sr_seed=SR_SEED, sr_stream=0)
+        self.c_sr1 = base.with_(rounding=ufp4.ROUND_SR, sr_seed=SR_SEED, sr_stream=1)
+        s = SHAPE
+        X, W, dY = wl.layer_inputs(s)
+        self.X, self.W, self.dY = to_dev(X, device), to_dev(W, device), to_dev(dY, device)
+        C, R = ufp4.ALONG_COLS, ufp4.ALONG_ROWS
+        E = ufp4.empty_qtensor
+        self.qx = E(s.M, s.K, self.c_rtne, device)        # FPROP A
+        self.qw = E(s.N, s.K, self.c_rtne, device)        # FPROP B
+        self.qdy = E(s.M, s.N, self.c_sr0, device)        # DGRAD A
+        self.qwt = E(s.K, s.N, self.c_rtne, device)       # DGRAD B
+        self.qdyt = E(s.N, s.M, self.c_sr1, device)       # WGRAD A
+        self.qxt = E(s.K, s.M, self.c_rtne, device)       # WGRAD B
+        self.jobs = [(self.X, C, self.qx), (self.W, C, self.qw), (self.dY, C, self.qdy),
+                     (self.W, R, self.qwt), (self.dY, R, self.qdyt), (self.X, R, self.qxt)]
+        self.amax = torch.zeros(len(self.jobs), dtype=torch.float32, device=device)
+        self.Y = torch.empty((s.M, s.N), dtype=torch.float32, device=device)
+        self.dX = torch.empty((s.M, s.K), dtype=torch.float32, device=device)
+        self.dW = torch.empty((s.N, s.K), dtype=torch.float32, device=device)
+        self.launches = len(self.jobs) * (2 if two else 1) + 3
+        self.quant_elems = sum(j[0].numel() for j in self.jobs)
+
+    def quantize_all(self):
+        u = self.u
+        for i, (x, axis, q) in enumerate(self.jobs):
+            am = None
+            if self.two:
+                am = self.amax[i:i + 1]
+                u.rht_amax(x, axis, 16, q.cfg.rht_sign_mask, out=am)
+            u.rht_quantize(x, axis, q.cfg, tensor_amax=am, out=q)
+
+    def gemms(self, events=None):
+        u = self.u
+        if events:
+            events[0].record()
+        u.gemm_fprop(self.qx, self.qw, out=self.Y)
+        if events:
+            events[1].record()
+        u.gemm_dgrad(self.qdy, self.qwt, out=self.dX)
+        if events:
+            events[2].record()
+        u.gemm_wgrad(self.qdyt, self.qxt, out=self.dW)
+        if events:
+            events[3].record()
+
+    def step(self, events=None):
+        if events:
+            events[0].record()
+        self.quantize_all()
+        self.gemms(events[1:] if events else None)
+
+
+def quant_bytes(step: LayerStep) -> float:
+    """Algorithmic bytes of the six quantize calls: bf16 in, packed codes,
+    block scales (fp32, or E4M3 + the amax pass re-reading the input)."""
+    n = step.quant_elems
+    per = 2 + 0.5 + (4 / 16 if not step.two else 1 / 16)
+    total = n * per
+    if step.two:
+        total += n * 2   # rotated-amax pass reads the input once more
+    return total
+
+
+def run_device(args, rank, world, device):
+    from fp4_quantized_gemms_b200 import ufp4
+    peaks, peak_kind = load_peaks()
+    s = SHAPE
+    flops = 3 * 2 * s.M * s.N * s.K
+    step = LayerStep(device, args.scale)
+    stream = torch.cuda.current_stream(device)
+
+    for _ in range(args.warmup):
+        step.step()
+    torch.cuda.synchronize(device)
+    if ufp4.check_device_status() != ufp4.OK:
+        raise RuntimeError("device error word set during warm-up")
+
+    nev = 5
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(args.steps):
+            step.step(ev[i])
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    q_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps))
+    g_ms = [statistics.mean(ev[i][1 + j].elapsed_time(ev[i][2 + j]) for i in range(args.steps))
+            for j in range(3)]
+    status = ufp4.check_device_status()
+
+    # ---- end to end through the public API with host buffers (rank-local)
+    e2e = run_e2e(step, args, device)
+
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    gemm_tf = [2 * s.M * s.N * s.K / (g * 1e-3) / 1e12 for g in g_ms]
+    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    qbytes = quant_bytes(step)
+    q_gbs = qbytes / (q_ms * 1e-3) / 1e9
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    dom = int(np.argmax(g_ms))
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e1m2 codes, fp16 tensor-core operands, fp32 accumulate",
+        "data": "synthetic (seeded PCG64 inputs of the workload's shapes and distributions)",
+        "config": {**workload_desc(args.scale), "parallelism": f"replicas x{world}"},
+        "gpu_launches": step.launches * args.steps,
+        "kernels": {
+            "quantize_all_ms": round(q_ms, 4),
+            "quantize_GBps": round(q_gbs, 1),
+            "quantize_frac_of_8TBps": round(q_gbs / 8000.0, 4),
+            "quantize_frac_of_measured_hbm": round(q_gbs / hbm, 4),
+            "gemm_ms": {k: round(v, 4) for k, v in zip(("fprop", "dgrad", "wgrad"), g_ms)},
+            "gemm_TFLOPs": {k: round(v, 1) for k, v in zip(("fprop", "dgrad", "wgrad"), gemm_tf)},
+        },
+        "roofline": {
+            "kernel": f"gemm_tn ({('fprop', 'dgrad', 'wgrad')[dom]}), kind::f16 tcgen05",
+            "bound": "tensor",
+            "achieved": round(gemm_tf[dom], 1),
+            "peak": peak_tf,
+            "peak_source": f"{peak_kind} bf16 dense (fp16 runs at the bf16 rate), burst",
+            "unit": "TFLOP/s",
+            "frac": round(gemm_tf[dom] / peak_tf, 4),
+            "traffic": None,
+        },
+        "e2e": e2e,
+        "device_status": ufp4.status_string(status),
+    }
+    result["clocks"] = clk.summary()
+    return result
+
+
+def run_e2e(step: LayerStep, args, device):
+    """Same step through the public API with HOST inputs and outputs: pinned
+    H2D copies of X, W, dY, the hot path, D2H copies of Y, dX, dW, all inside
+    the timed region."""
+    s = SHAPE
+    X, W, dY = wl.layer_inputs(s)
+    hX = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hW = torch.from_numpy(W.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hdY = torch.from_numpy(dY.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hY = torch.empty(step.Y.shape, dtype=torch.float32).pin_memory()
+    hdX = torch.empty(step.dX.shape, dtype=torch.float32).pin_memory()
+    hdW = torch.empty(step.dW.shape, dtype=torch.float32).pin_memory()
+    h2d = (hX.numel() + hW.numel() + hdY.numel()) * 2
+    d2h = (hY.numel() + hdX.numel() + hdW.numel()) * 4
+
+    def one():
+        step.X.copy_(hX, non_blocking=True)
+        step.W.copy_(hW, non_blocking=True)
+        step.dY.copy_(hdY, non_blocking=True)
+        step.step()
+        hY.copy_(step.Y, non_blocking=True)
+        hdX.copy_(step.dX, non_blocking=True)
+        hdW.copy_(step.dW, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        one()
+    torch.cuda.synchronize(device)
+    n = max(1, min(args.steps, 10))
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(n):
+        one()
+    b.record()
+    torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b) / n
+    flops = 3 * 2 * s.M * s.N * s.K
+    return {"value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": n}
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_sample_step(rng, n_rows=8, n_cols=8):
+    """A bounded sample of one step on the host cores: the oracle quantizes
+    n_rows / n_cols output rows of every operand (full reduction length) and
+    contracts the n_rows x n_cols sampled block of each GEMM.  Returns
+    (effective GEMM flops of the sampled entries, seconds)."""
+    import oracle
+    s = SHAPE
+    X, W, dY = wl.layer_inputs(s)
+    rt = oracle.QuantCfg(grid=0, hadamard_n=16, block=16, sign_mask=0x09F1FD9D03F0A9B4)
+    sr0 = oracle.QuantCfg(grid=0, rounding=1, sr_seed=SR_SEED, sr_stream=0, hadamard_n=16,
+                          block=16, sign_mask=0x09F1FD9D03F0A9B4)
+    sr1 = oracle.QuantCfg(grid=0, rounding=1, sr_seed=SR_SEED, sr_stream=1, hadamard_n=16,
+                          block=16, sign_mask=0x09F1FD9D03F0A9B4)
+    gemms = [((X, 0, rt, s.M), (W, 0, rt, s.N), s.K),
+             ((dY, 0, sr0, s.M), (W, 1, rt, s.K), s.N),
+             ((dY, 1, sr1, s.N), (X, 1, rt, s.K), s.M)]
+    flops = 0.0
+    t0 = time.perf_counter()
+    for (a_bits, a_ax, a_cfg, a_rows), (b_bits, b_ax, b_cfg, b_rows), K in gemms:
+        ia = rng.choice(a_rows, n_rows, replace=False)
+        jb = rng.choice(b_rows, n_cols, replace=False)
+        qa = [oracle.quantize(a_bits, a_ax, a_cfg, r0=int(r), nr=1) for r in ia]
+        qb = [oracle.quantize(b_bits, b_ax, b_cfg, r0=int(r), nr=1) for r in jb]
+        A = np.concatenate([q.dequantize() for q in qa])
+        B = np.concatenate([q.dequantize() for q in qb])
+        out = np.empty(n_rows * n_cols)
+        ii = np.repeat(np.arange(n_rows), n_cols)
+        jj = np.tile(np.arange(n_cols), n_rows)
+        qa[0].codes = np.concatenate([q.codes for q in qa])
+        qa[0].scales = np.concatenate([q.scales for q in qa])
+        qb[0].codes = np.concatenate([q.codes for q in qb])
+        qb[0].scales = np.concatenate([q.scales for q in qb])
+        out = oracle.gemm_tn_entries(qa[0], qb[0], ii, jj)
+        flops += 2.0 * K * out.size
+        del A, B
+    return flops, time.perf_counter() - t0
+
+
+def run_reference(args, world):
+    import oracle
+    oracle.build()
+    rng = np.random.default_rng(0)
+    wl.layer_inputs(SHAPE)   # generate inputs outside the timed region
+    for _ in range(args.warmup):
+        oracle_sample_step(rng)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        f, t = oracle_sample_step(rng)
+        times.append(t)
+        flops += f
+    total = sum(times)
+    value = flops / total / 1e12
+    cores = oracle.num_threads()
+    sample = ("per step: 8 sampled output rows of each of the 6 quantized operands "
+              "(full reduction length) and the 8x8 sampled block of each GEMM")
+    res = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64 oracle (fp32 RHT, exact rounding decisions)", "data": "synthetic",
+        "config": {**workload_desc("fp32"), "parallelism": "host cores"},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    return res
+
+
+def cpu_baseline_quick():
+    """The oracle as it stands, on a bounded sample of the workload (rank 0)."""
+    import oracle
+    oracle.build()
+    rng = np.random.default_rng(1)
+    oracle_sample_step(rng, 4, 4)       # warm caches / page in
+    flops, secs = 0.0, 0.0
+    n = 0
+    while secs < 10.0 and n < 6:
+        f, t = oracle_sample_step(rng)
+        flops += f
+        secs += t
+        n += 1
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": (f"{n} sampled steps: 8 output rows of each of the 6 quantized operands "
+                       f"(full K) and an 8x8 block of each GEMM, {secs:.1f} s of CPU work")}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ufp4", choices=["ufp4", "reference"])
+    ap.add_argument("--scale", default="two-level", choices=["two-level", "fp32"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, world)), flush=True)
+        return
+
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    from fp4_quantized_gemms_b200 import build as ufp4_build
+    ufp4_build.build()
+    res = run_device(args, rank, world, device)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline_quick()
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,334 @@
+// api.cu -- the C ABI of libufp4.so (declared in include/ufp4.h): argument
+// validation on the host, tensor-map encoding, kernel dispatch.  No call
+// allocates, frees or synchronises (ufp4_check_device_status excepted).
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "ufp4.h"
+#include "ufp4_internal.h"
+
+namespace ufp4 {
+
+cudaError_t read_and_clear_error_word(uint32_t *out);   // gemm.cu
+
+namespace {
+
+constexpr int64_t kKAlign = 64;
+constexpr int64_t kScaleLdAlign = 64;
+
+int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool cfg_valid(const ufp4_quant_cfg_t &c) {
+    if (c.grid != UFP4_GRID_E1M2 && c.grid != UFP4_GRID_E2M1) return false;
+    if (c.rounding != UFP4_ROUND_RTNE && c.rounding != UFP4_ROUND_SR) return false;
+    if (!(c.hadamard_n == 0 || c.hadamard_n == 16 || c.hadamard_n == 32 || c.hadamard_n == 64))
+        return false;
+    if (c.block != 16 && c.block != 32) return false;
+    if (c.scale_fmt != UFP4_SCALE_FP32 && c.scale_fmt != UFP4_SCALE_E4M3_X_FP32) return false;
+    return true;
+}
+
+int sm_count() {
+    static int cache[64];
+    static std::once_flag flags[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::call_once(flags[dev], [dev] {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev] = n;
+    });
+    return cache[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Common checks of one quantized operand descriptor.
+ufp4_status_t check_qtensor(const ufp4_qtensor_t *q) {
+    if (q == nullptr) return UFP4_ERR_INVALID_ARG;
+    if (!cfg_valid(q->cfg)) return UFP4_ERR_INVALID_ARG;
+    if (q->rows < 0 || q->k < 0) return UFP4_ERR_INVALID_ARG;
+    if (q->kpad != round_up(q->k, kKAlign)) return UFP4_ERR_INVALID_ARG;
+    if (q->scale_ld < q->rows || q->scale_ld % kScaleLdAlign != 0) return UFP4_ERR_INVALID_ARG;
+    if (q->rows > 0 && q->kpad > 0) {
+        if (q->codes == nullptr || q->scales == nullptr) return UFP4_ERR_INVALID_ARG;
+        if (!aligned16(q->codes) || !aligned16(q->scales)) return UFP4_ERR_ALIGNMENT;
+    }
+    if (q->cfg.scale_fmt == UFP4_SCALE_E4M3_X_FP32 && q->tensor_scale == nullptr)
+        return UFP4_ERR_INVALID_ARG;
+    if (q->rows > (int64_t(1) << 31) || q->kpad > (int64_t(1) << 31)) return UFP4_ERR_UNSUPPORTED;
+    return UFP4_OK;
+}
+
+ufp4_status_t check_pair(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b) {
+    ufp4_status_t s = check_qtensor(a);
+    if (s != UFP4_OK) return s;
+    s = check_qtensor(b);
+    if (s != UFP4_OK) return s;
+    const ufp4_quant_cfg_t &x = a->cfg, &y = b->cfg;
+    if (x.grid != y.grid || x.block != y.block || x.scale_fmt != y.scale_fmt ||
+        x.hadamard_n != y.hadamard_n)
+        return UFP4_ERR_OPERAND_MISMATCH;
+    if (x.hadamard_n > 0) {
+        const uint64_t m = x.hadamard_n == 64 ? ~uint64_t(0) : ((uint64_t(1) << x.hadamard_n) - 1);
+        if ((x.rht_sign_mask & m) != (y.rht_sign_mask & m)) return UFP4_ERR_OPERAND_MISMATCH;
+    }
+    if (a->k != b->k || a->kpad != b->kpad) return UFP4_ERR_OPERAND_MISMATCH;
+    return UFP4_OK;
+}
+
+ufp4_status_t encode_operand_maps(const ufp4_qtensor_t *q, int box_rows, int mode,
+                                  CUtensorMap *codes, CUtensorMap *scales) {
+    const int64_t rows_t = q->rows > 0 ? q->rows : 1;
+    CUresult r = encode_tensor_map_2d(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, q->codes,
+                                      static_cast<uint64_t>(q->kpad / 2),
+                                      static_cast<uint64_t>(rows_t),
+                                      static_cast<uint64_t>(q->kpad / 2), 32,
+                                      static_cast<uint32_t>(box_rows));
+    if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
+    const int nblk_stage = 64 / q->cfg.block;
+    const uint64_t nblk = static_cast<uint64_t>(q->kpad / q->cfg.block);
+    if (mode == 1) {
+        r = encode_tensor_map_2d(scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, q->scales,
+                                 static_cast<uint64_t>(q->scale_ld), nblk,
+                                 static_cast<uint64_t>(q->scale_ld), static_cast<uint32_t>(box_rows),
+                                 static_cast<uint32_t>(nblk_stage));
+    } else {
+        r = encode_tensor_map_2d(scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, q->scales,
+                                 static_cast<uint64_t>(q->scale_ld), nblk,
+                                 static_cast<uint64_t>(q->scale_ld) * 4,
+                                 static_cast<uint32_t>(box_rows), static_cast<uint32_t>(nblk_stage));
+    }
+    return r == CUDA_SUCCESS ? UFP4_OK : UFP4_ERR_CUDA;
+}
+
+ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
+                       const ufp4_group_t *groups_dev, int32_t num_groups, float *c, int64_t ldc,
+                       int64_t m, int64_t n, void *stream) {
+    ufp4_status_t s = check_pair(a, b);
+    if (s != UFP4_OK) return s;
+    if (c == nullptr && (m > 0 && n > 0)) return UFP4_ERR_INVALID_ARG;
+    if (ldc < n || ldc < 1) return UFP4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(c) & 3u) != 0) return UFP4_ERR_ALIGNMENT;
+    if (groups_dev != nullptr && (reinterpret_cast<uintptr_t>(groups_dev) & 7u))
+        return UFP4_ERR_ALIGNMENT;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int mode = a->cfg.scale_fmt == UFP4_SCALE_E4M3_X_FP32 ? 1 : 0;
+    if (groups_dev == nullptr) {
+        if (m == 0 || n == 0) return UFP4_OK;
+        if (a->kpad == 0) {
+            cudaError_t e = cudaMemset2DAsync(c, static_cast<size_t>(ldc) * 4, 0,
+                                              static_cast<size_t>(n) * 4, static_cast<size_t>(m), st);
+            return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
+        }
+    } else if (num_groups == 0 || a->kpad == 0 || a->rows == 0 || b->rows == 0) {
+        return UFP4_OK;
+    }
+    if (encode_fn() == nullptr) return UFP4_ERR_CUDA;
+
+    GemmArgs args;
+    memset(&args, 0, sizeof(args));
+    const int bn = mode == 1 ? 256 : 128;
+    s = encode_operand_maps(a, 128, mode, &args.tm_a_codes, &args.tm_a_scales);
+    if (s != UFP4_OK) return s;
+    s = encode_operand_maps(b, bn, mode, &args.tm_b_codes, &args.tm_b_scales);
+    if (s != UFP4_OK) return s;
+    args.a_S = a->tensor_scale;
+    args.b_S = b->tensor_scale;
+    args.c = c;
+    args.ldc = ldc;
+    args.inv_n = a->cfg.hadamard_n > 0 ? 1.0f / static_cast<float>(a->cfg.hadamard_n) : 1.0f;
+    args.block = a->cfg.block;
+    args.groups = reinterpret_cast<const GemmGroup *>(groups_dev);
+    args.num_groups = num_groups;
+    args.single.m = m;
+    args.single.n = n;
+    args.single.k = a->kpad;
+    cudaError_t e = launch_gemm(args, mode, a->cfg.grid, sm_count(), st);
+    return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
+}
+
+ufp4_status_t check_input(const void *x, int64_t rows, int64_t cols, int64_t ld, int32_t axis) {
+    if (rows < 0 || cols < 0) return UFP4_ERR_INVALID_ARG;
+    if (axis != UFP4_ALONG_COLS && axis != UFP4_ALONG_ROWS) return UFP4_ERR_INVALID_ARG;
+    if (rows > 0 && cols > 0) {
+        if (x == nullptr) return UFP4_ERR_INVALID_ARG;
+        if (ld < cols) return UFP4_ERR_INVALID_ARG;
+        if (!aligned16(x) || ld % 8 != 0 || cols % 8 != 0) return UFP4_ERR_ALIGNMENT;
+    }
+    return UFP4_OK;
+}
+
+}  // namespace
+
+CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
+                              uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                              uint32_t box_inner, uint32_t box_outer) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (fn == nullptr) return CUDA_ERROR_NOT_INITIALIZED;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estride[2] = {1, 1};
+    return fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estride,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+}  // namespace ufp4
+
+using namespace ufp4;
+
+extern "C" {
+
+int32_t ufp4_version(void) { return 100; }
+
+const char *ufp4_status_string(ufp4_status_t s) {
+    switch (s) {
+        case UFP4_OK: return "UFP4_OK";
+        case UFP4_ERR_INVALID_ARG: return "UFP4_ERR_INVALID_ARG";
+        case UFP4_ERR_UNSUPPORTED: return "UFP4_ERR_UNSUPPORTED";
+        case UFP4_ERR_ALIGNMENT: return "UFP4_ERR_ALIGNMENT";
+        case UFP4_ERR_OPERAND_MISMATCH: return "UFP4_ERR_OPERAND_MISMATCH";
+        case UFP4_ERR_CUDA: return "UFP4_ERR_CUDA";
+        case UFP4_ERR_DEVICE_TIMEOUT: return "UFP4_ERR_DEVICE_TIMEOUT";
+    }
+    return "UFP4_ERR_UNKNOWN";
+}
+
+ufp4_status_t ufp4_qtensor_layout(int64_t rows, int64_t k, const ufp4_quant_cfg_t *cfg,
+                                  int64_t *kpad, int64_t *scale_ld, size_t *codes_bytes,
+                                  size_t *scales_bytes) {
+    if (cfg == nullptr || rows < 0 || k < 0 || !cfg_valid(*cfg)) return UFP4_ERR_INVALID_ARG;
+    const int64_t kp = round_up(k, kKAlign);
+    const int64_t sl = round_up(rows > 0 ? rows : 1, kScaleLdAlign);
+    const int64_t elt = cfg->scale_fmt == UFP4_SCALE_FP32 ? 4 : 1;
+    if (kpad) *kpad = kp;
+    if (scale_ld) *scale_ld = sl;
+    if (codes_bytes) *codes_bytes = static_cast<size_t>(rows * (kp / 2));
+    if (scales_bytes) *scales_bytes = static_cast<size_t>((kp / cfg->block) * sl * elt);
+    return UFP4_OK;
+}
+
+ufp4_status_t ufp4_rht_amax(const void *x_dev, int64_t rows, int64_t cols, int64_t ld,
+                            int32_t axis, int32_t hadamard_n, uint64_t rht_sign_mask,
+                            float *amax_dev, void *stream) {
+    ufp4_status_t s = check_input(x_dev, rows, cols, ld, axis);
+    if (s != UFP4_OK) return s;
+    if (amax_dev == nullptr) return UFP4_ERR_INVALID_ARG;
+    if (!(hadamard_n == 0 || hadamard_n == 16 || hadamard_n == 32 || hadamard_n == 64))
+        return UFP4_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    QuantArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x = static_cast<const uint16_t *>(x_dev);
+    a.rows = rows;
+    a.cols = cols;
+    a.ld = ld;
+    a.axis = axis;
+    a.out_rows = axis == UFP4_ALONG_COLS ? rows : cols;
+    a.K = axis == UFP4_ALONG_COLS ? cols : rows;
+    a.kpad = round_up(a.K, kKAlign);
+    a.amax_out = amax_dev;
+    a.sign_mask = rht_sign_mask;
+    if (a.out_rows == 0 || a.kpad == 0) {
+        return cudaMemsetAsync(amax_dev, 0, sizeof(float), st) == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
+    }
+    cudaError_t e = launch_rht_amax(a, hadamard_n, sm_count(), st);
+    return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
+}
+
+ufp4_status_t ufp4_rht_quantize(const void *x_dev, int64_t rows, int64_t cols, int64_t ld,
+                                int32_t axis, const float *tensor_amax_dev, ufp4_qtensor_t *out,
+                                void *stream) {
+    ufp4_status_t s = check_input(x_dev, rows, cols, ld, axis);
+    if (s != UFP4_OK) return s;
+    s = check_qtensor(out);
+    if (s != UFP4_OK) return s;
+    const int64_t out_rows = axis == UFP4_ALONG_COLS ? rows : cols;
+    const int64_t K = axis == UFP4_ALONG_COLS ? cols : rows;
+    if (out->rows != out_rows || out->k != K) return UFP4_ERR_INVALID_ARG;
+    const bool two_level = out->cfg.scale_fmt == UFP4_SCALE_E4M3_X_FP32;
+    if (two_level && tensor_amax_dev == nullptr) return UFP4_ERR_INVALID_ARG;
+    if (out_rows == 0 || out->kpad == 0) return UFP4_OK;
+    QuantArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x = static_cast<const uint16_t *>(x_dev);
+    a.rows = rows;
+    a.cols = cols;
+    a.ld = ld;
+    a.axis = axis;
+    a.out_rows = out_rows;
+    a.K = K;
+    a.kpad = out->kpad;
+    a.scale_ld = out->scale_ld;
+    a.codes = static_cast<uint8_t *>(out->codes);
+    a.scales = out->scales;
+    a.S_out = two_level ? out->tensor_scale : nullptr;
+    a.amax_t = two_level ? tensor_amax_dev : nullptr;
+    a.seed = out->cfg.sr_seed;
+    a.stream = out->cfg.sr_stream;
+    a.sign_mask = out->cfg.rht_sign_mask;
+    a.scale_fmt = out->cfg.scale_fmt;
+    cudaError_t e = launch_rht_quantize(a, out->cfg.hadamard_n, out->cfg.block, out->cfg.grid,
+                                        out->cfg.rounding, sm_count(),
+                                        static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
+}
+
+ufp4_status_t ufp4_gemm_fprop(const ufp4_qtensor_t *xq, const ufp4_qtensor_t *wq, float *y_dev,
+                              int64_t ldy, void *stream) {
+    if (xq == nullptr || wq == nullptr) return UFP4_ERR_INVALID_ARG;
+    return run_gemm(xq, wq, nullptr, 0, y_dev, ldy, xq->rows, wq->rows, stream);
+}
+
+ufp4_status_t ufp4_gemm_dgrad(const ufp4_qtensor_t *dyq, const ufp4_qtensor_t *wtq, float *dx_dev,
+                              int64_t lddx, void *stream) {
+    if (dyq == nullptr || wtq == nullptr) return UFP4_ERR_INVALID_ARG;
+    return run_gemm(dyq, wtq, nullptr, 0, dx_dev, lddx, dyq->rows, wtq->rows, stream);
+}
+
+ufp4_status_t ufp4_gemm_wgrad(const ufp4_qtensor_t *dytq, const ufp4_qtensor_t *xtq,
+                              float *dw_dev, int64_t lddw, void *stream) {
+    if (dytq == nullptr || xtq == nullptr) return UFP4_ERR_INVALID_ARG;
+    return run_gemm(dytq, xtq, nullptr, 0, dw_dev, lddw, dytq->rows, xtq->rows, stream);
+}
+
+ufp4_status_t ufp4_grouped_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
+                                const ufp4_group_t *groups_dev, int32_t num_groups, float *c_dev,
+                                int64_t ldc, void *stream) {
+    if (a == nullptr || b == nullptr || num_groups < 0) return UFP4_ERR_INVALID_ARG;
+    if (num_groups > 0 && groups_dev == nullptr) return UFP4_ERR_INVALID_ARG;
+    if (num_groups == 0) return UFP4_OK;
+    if (c_dev == nullptr) return UFP4_ERR_INVALID_ARG;
+    return run_gemm(a, b, groups_dev, num_groups, c_dev, ldc, 0, 0, stream);
+}
+
+ufp4_status_t ufp4_check_device_status(void) {
+    uint32_t w = 0;
+    if (read_and_clear_error_word(&w) != cudaSuccess) return UFP4_ERR_CUDA;
+    return w == 0 ? UFP4_OK : UFP4_ERR_DEVICE_TIMEOUT;
+}
+
+}  // extern "C"

@@ -1,0 +1,63 @@
+// ufp4_internal.h -- launch interfaces between the C ABI layer and kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ufp4 {
+
+struct QuantArgs {
+    const uint16_t *x;   // bf16 input [rows][ld]
+    int64_t rows, cols, ld;
+    int axis;            // 0: reduce along cols, 1: along rows (transposed out)
+    int64_t out_rows;    // rows of the K-major output
+    int64_t K, kpad, scale_ld;
+    uint8_t *codes;      // [out_rows][kpad/2]
+    void *scales;        // block-major [kpad/B][scale_ld], fp32 or E4M3
+    float *S_out;        // two-level: receives S
+    const float *amax_t; // two-level: rotated tensor amax
+    float *amax_out;     // amax kernel output
+    uint64_t seed;
+    uint32_t stream;
+    uint64_t sign_mask;
+    int scale_fmt;
+    int64_t num_units;   // filled by the launcher
+};
+
+cudaError_t launch_rht_quantize(QuantArgs a, int hadamard_n, int block, int grid_kind,
+                                int rounding, int num_sms, cudaStream_t stream);
+cudaError_t launch_rht_amax(QuantArgs a, int hadamard_n, int num_sms, cudaStream_t stream);
+
+// One contraction problem (a group of the grouped GEMM, or the whole GEMM).
+struct GemmGroup {
+    int64_t m, n, k;
+    int64_t a_row, a_col;
+    int64_t b_row, b_col;
+    int64_t c_row, c_col;
+};
+
+struct GemmArgs {
+    CUtensorMap tm_a_codes, tm_b_codes;   // u8 [rows][kpad/2]
+    CUtensorMap tm_a_scales, tm_b_scales; // [nblk][scale_ld], fp32 or u8
+    const float *a_S, *b_S;               // two-level tensor scales (device)
+    float *c;
+    int64_t ldc;
+    float inv_n;                          // 1/n of the Hadamard size (1 if none)
+    int block;                            // 16 or 32
+    const GemmGroup *groups;              // device table or nullptr
+    int num_groups;
+    GemmGroup single;                     // used when groups == nullptr
+};
+
+// mode 0: fp32 block scales (per-block partial products, CUDA-core scaling)
+// mode 1: E4M3 x fp32 two-level scales (scales folded into fp16 operands)
+cudaError_t launch_gemm(const GemmArgs &args, int mode, int grid_kind, int num_sms,
+                        cudaStream_t stream);
+
+// Driver entry point for tensor-map encoding (resolved once at run time).
+CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
+                              uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                              uint32_t box_inner, uint32_t box_outer);
+
+}  // namespace ufp4

@@ -1,0 +1,251 @@
+"""Thin Python binding of libufp4.so (argument marshalling only).
+
+Every function here maps one-to-one onto an ``extern "C"`` entry point of
+``include/ufp4.h``; tensors are torch CUDA tensors (device memory and streams
+come from PyTorch), results are computed by the library's kernels.  There is
+no CPU path: loading raises if the shared library is missing, and every call
+that launches work raises if the tensors are not on a CUDA device.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, replace
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libufp4.so")
+
+# enums (include/ufp4.h)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_OPERAND_MISMATCH, ERR_CUDA, \
+    ERR_DEVICE_TIMEOUT = range(7)
+GRID_E1M2, GRID_E2M1 = 0, 1
+ROUND_RTNE, ROUND_SR = 0, 1
+SCALE_FP32, SCALE_E4M3_X_FP32 = 0, 1
+ALONG_COLS, ALONG_ROWS = 0, 1
+DEFAULT_SIGN_MASK = 0x09F1FD9D03F0A9B4
+
+EXPORTED = [
+    "ufp4_qtensor_layout", "ufp4_rht_amax", "ufp4_rht_quantize", "ufp4_gemm_fprop",
+    "ufp4_gemm_dgrad", "ufp4_gemm_wgrad", "ufp4_grouped_gemm", "ufp4_check_device_status",
+    "ufp4_status_string", "ufp4_version",
+]
+
+
+class UFP4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+class QuantCfgC(ctypes.Structure):
+    _fields_ = [("grid", ctypes.c_int32), ("rounding", ctypes.c_int32),
+                ("sr_seed", ctypes.c_uint64), ("sr_stream", ctypes.c_uint32),
+                ("hadamard_n", ctypes.c_int32), ("rht_sign_mask", ctypes.c_uint64),
+                ("block", ctypes.c_int32), ("scale_fmt", ctypes.c_int32)]
+
+
+class QTensorC(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("tensor_scale", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("k", ctypes.c_int64), ("kpad", ctypes.c_int64), ("scale_ld", ctypes.c_int64),
+                ("cfg", QuantCfgC)]
+
+
+class GroupC(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in
+                ("m", "n", "k", "a_row", "a_col", "b_row", "b_col", "c_row", "c_col")]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libufp4.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m fp4_quantized_gemms_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i64, i32, u64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_uint64
+        st = ctypes.c_int
+        L.ufp4_status_string.restype = ctypes.c_char_p
+        L.ufp4_status_string.argtypes = [st]
+        L.ufp4_version.restype = i32
+        L.ufp4_qtensor_layout.restype = st
+        L.ufp4_qtensor_layout.argtypes = [i64, i64, ctypes.POINTER(QuantCfgC),
+                                          ctypes.POINTER(i64), ctypes.POINTER(i64),
+                                          ctypes.POINTER(ctypes.c_size_t),
+                                          ctypes.POINTER(ctypes.c_size_t)]
+        L.ufp4_rht_amax.restype = st
+        L.ufp4_rht_amax.argtypes = [P, i64, i64, i64, i32, i32, u64, P, P]
+        L.ufp4_rht_quantize.restype = st
+        L.ufp4_rht_quantize.argtypes = [P, i64, i64, i64, i32, P, ctypes.POINTER(QTensorC), P]
+        for name in ("ufp4_gemm_fprop", "ufp4_gemm_dgrad", "ufp4_gemm_wgrad"):
+            f = getattr(L, name)
+            f.restype = st
+            f.argtypes = [ctypes.POINTER(QTensorC), ctypes.POINTER(QTensorC), P, i64, P]
+        L.ufp4_grouped_gemm.restype = st
+        L.ufp4_grouped_gemm.argtypes = [ctypes.POINTER(QTensorC), ctypes.POINTER(QTensorC), P,
+                                        i32, P, i64, P]
+        L.ufp4_check_device_status.restype = st
+        L.ufp4_check_device_status.argtypes = []
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().ufp4_status_string(status).decode()
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise UFP4Error(status, where)
+
+
+def _stream_ptr(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _require_cuda(*tensors):
+    for t in tensors:
+        if t is not None and not t.is_cuda:
+            raise RuntimeError("ufp4 kernels need CUDA tensors (there is no CPU path)")
+
+
+# ---------------------------------------------------------------- operands
+@dataclass(frozen=True)
+class QuantConfig:
+    grid: int = GRID_E1M2
+    rounding: int = ROUND_RTNE
+    sr_seed: int = 0
+    sr_stream: int = 0
+    hadamard_n: int = 16
+    rht_sign_mask: int = DEFAULT_SIGN_MASK
+    block: int = 16
+    scale_fmt: int = SCALE_FP32
+
+    def c(self) -> QuantCfgC:
+        return QuantCfgC(self.grid, self.rounding, self.sr_seed, self.sr_stream, self.hadamard_n,
+                         self.rht_sign_mask, self.block, self.scale_fmt)
+
+    def with_(self, **kw) -> "QuantConfig":
+        return replace(self, **kw)
+
+
+def layout(rows: int, k: int, cfg: QuantConfig):
+    kpad, sld = ctypes.c_int64(), ctypes.c_int64()
+    cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    c = cfg.c()
+    _check(lib().ufp4_qtensor_layout(rows, k, ctypes.byref(c), ctypes.byref(kpad),
+                                     ctypes.byref(sld), ctypes.byref(cb), ctypes.byref(sb)),
+           "ufp4_qtensor_layout")
+    return kpad.value, sld.value, cb.value, sb.value
+
+
+@dataclass
+class QTensor:
+    """A quantized operand: K-major packed codes + block-major scales."""
+    codes: torch.Tensor          # uint8 [rows, kpad/2]
+    scales: torch.Tensor         # float32 or uint8 [kpad/block, scale_ld]
+    tensor_scale: torch.Tensor | None   # float32 [1] (two-level only)
+    rows: int
+    k: int
+    kpad: int
+    scale_ld: int
+    cfg: QuantConfig
+
+    def c(self) -> QTensorC:
+        return QTensorC(self.codes.data_ptr(), self.scales.data_ptr(),
+                        self.tensor_scale.data_ptr() if self.tensor_scale is not None else None,
+                        self.rows, self.k, self.kpad, self.scale_ld, self.cfg.c())
+
+
+def empty_qtensor(rows: int, k: int, cfg: QuantConfig, device="cuda") -> QTensor:
+    kpad, sld, _, _ = layout(rows, k, cfg)
+    nblk = kpad // cfg.block
+    codes = torch.empty((rows, kpad // 2), dtype=torch.uint8, device=device)
+    if cfg.scale_fmt == SCALE_FP32:
+        scales = torch.empty((nblk, sld), dtype=torch.float32, device=device)
+        ts = None
+    else:
+        scales = torch.empty((nblk, sld), dtype=torch.uint8, device=device)
+        ts = torch.empty(1, dtype=torch.float32, device=device)
+    return QTensor(codes, scales, ts, rows, k, kpad, sld, cfg)
+
+
+# ---------------------------------------------------------------- entry points
+def rht_amax(x: torch.Tensor, axis: int, hadamard_n: int,
+             sign_mask: int = DEFAULT_SIGN_MASK, out: torch.Tensor | None = None) -> torch.Tensor:
+    """max |H_n D x| over the operand's K-major view -> float32 [1] on device."""
+    _require_cuda(x)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    rows, cols = x.shape
+    _check(lib().ufp4_rht_amax(ctypes.c_void_p(x.data_ptr()), rows, cols, x.stride(0), axis,
+                               hadamard_n, sign_mask, ctypes.c_void_p(out.data_ptr()),
+                               _stream_ptr(x.device)), "ufp4_rht_amax")
+    return out
+
+
+def rht_quantize(x: torch.Tensor, axis: int, cfg: QuantConfig,
+                 tensor_amax: torch.Tensor | None = None, out: QTensor | None = None) -> QTensor:
+    """Fused RHT + block scale + 4-bit rounding + packing of a bf16 operand."""
+    _require_cuda(x, tensor_amax)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    orows, k = (rows, cols) if axis == ALONG_COLS else (cols, rows)
+    if out is None:
+        out = empty_qtensor(orows, k, cfg, device=x.device)
+    if cfg.scale_fmt == SCALE_E4M3_X_FP32 and tensor_amax is None:
+        tensor_amax = rht_amax(x, axis, cfg.hadamard_n, cfg.rht_sign_mask)
+    qc = out.c()
+    _check(lib().ufp4_rht_quantize(ctypes.c_void_p(x.data_ptr()), rows, cols, x.stride(0), axis,
+                                   ctypes.c_void_p(tensor_amax.data_ptr()) if tensor_amax is not None else None,
+                                   ctypes.byref(qc), _stream_ptr(x.device)), "ufp4_rht_quantize")
+    return out
+
+
+def _gemm(name: str, a: QTensor, b: QTensor, out: torch.Tensor | None) -> torch.Tensor:
+    _require_cuda(a.codes, b.codes)
+    if out is None:
+        out = torch.empty((a.rows, b.rows), dtype=torch.float32, device=a.codes.device)
+    ac, bc = a.c(), b.c()
+    _check(getattr(lib(), name)(ctypes.byref(ac), ctypes.byref(bc), ctypes.c_void_p(out.data_ptr()),
+                                out.stride(0), _stream_ptr(out.device)), name)
+    return out
+
+
+def gemm_fprop(xq: QTensor, wq: QTensor, out=None) -> torch.Tensor:
+    """Y = X W^T from X, W both quantized ALONG_COLS."""
+    return _gemm("ufp4_gemm_fprop", xq, wq, out)
+
+
+def gemm_dgrad(dyq: QTensor, wtq: QTensor, out=None) -> torch.Tensor:
+    """dX = dY W from dY quantized ALONG_COLS and W quantized ALONG_ROWS."""
+    return _gemm("ufp4_gemm_dgrad", dyq, wtq, out)
+
+
+def gemm_wgrad(dytq: QTensor, xtq: QTensor, out=None) -> torch.Tensor:
+    """dW = dY^T X from dY and X both quantized ALONG_ROWS."""
+    return _gemm("ufp4_gemm_wgrad", dytq, xtq, out)
+
+
+def grouped_gemm(a: QTensor, b: QTensor, groups: torch.Tensor, out: torch.Tensor) -> torch.Tensor:
+    """groups: int64 CUDA tensor [G, 9] rows (m, n, k, a_row, a_col, b_row, b_col, c_row, c_col)."""
+    _require_cuda(a.codes, b.codes, groups, out)
+    assert groups.dtype == torch.int64 and groups.dim() == 2 and groups.shape[1] == 9
+    groups = groups.contiguous()
+    ac, bc = a.c(), b.c()
+    _check(lib().ufp4_grouped_gemm(ctypes.byref(ac), ctypes.byref(bc),
+                                   ctypes.c_void_p(groups.data_ptr()), groups.shape[0],
+                                   ctypes.c_void_p(out.data_ptr()), out.stride(0),
+                                   _stream_ptr(out.device)), "ufp4_grouped_gemm")
+    return out
+
+
+def check_device_status() -> int:
+    """Reads and clears the kernels' device error word (synchronises)."""
+    return lib().ufp4_check_device_status()

@@ -24,8 +24,8 @@ SEED_X, SEED_W, SEED_DY, SEED_OUTLIER, SEED_STUDENT, SEED_ZIPF = 1, 2, 3, 4, 5, 
 def bf16_bits(a: np.ndarray) -> np.ndarray:
     """float32 -> bf16 bit pattern, round to nearest even (finite inputs)."""
     f = np.ascontiguousarray(a, dtype=np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    r = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    u = f.view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
     return r.astype(np.uint16)
 
 
@@ -84,8 +84,23 @@ LARGE = LayerShape(M=16384, K=8192, N=28672, x_outlier_frac=0.01, x_outlier_fact
                    w_std=0.01, dy_std=1e-4)
 
 
-def layer_inputs(shape: LayerShape, want_dy: bool = True, n_outliers: int | None = None):
-    """X [M, K], W [N, K], dY [M, N] as bf16 bit patterns."""
+_LAYER_CACHE: dict = {}
+
+
+def layer_inputs(shape: LayerShape, want_dy: bool = True, n_outliers: int | None = None,
+                 cache: bool = True):
+    """X [M, K], W [N, K], dY [M, N] as bf16 bit patterns (memoised per shape)."""
+    key = (shape.M, shape.K, shape.N, want_dy, n_outliers)
+    if cache and key in _LAYER_CACHE:
+        return _LAYER_CACHE[key]
+    out = _layer_inputs(shape, want_dy, n_outliers)
+    if cache:
+        _LAYER_CACHE.clear()
+        _LAYER_CACHE[key] = out
+    return out
+
+
+def _layer_inputs(shape: LayerShape, want_dy: bool, n_outliers: int | None):
     if n_outliers is None:
         n_outliers = int(round(shape.x_outlier_frac * shape.K))
     if shape is TINY:

@@ -1,0 +1,205 @@
+/*
+ * ufp4.h -- C ABI of libufp4.so: the data-parallel hot path of the UFP4
+ * 4-bit training recipe on NVIDIA B200 (sm_100a).
+ *
+ * Method: arXiv 2606.20381, "Rethinking Shrinkage Bias in LLM FP4 Pretraining:
+ * Geometric Origin, Systemic Impact, and UFP4 Recipe".  Citations name the
+ * paperlayer.ai per-section summary of the paper as [PL], the gist.science
+ * technical summary as [GS] and the author's dreamwings.cn post as [DW].
+ *
+ * What the library computes ([PL] §2 Preliminaries, §4 UFP4):
+ *   1. ufp4_rht_quantize: for each row of an operand's K-major view (K = the
+ *      GEMM's reduction dimension), apply a random sign diagonal D and an
+ *      unnormalised Sylvester Hadamard H_n per n-block, take the absolute
+ *      maximum of each scale block, derive the block scale, round every
+ *      element to the 4-bit grid (RTNE, or stochastic rounding from a
+ *      Philox4x32-10 stream) and pack two codes per byte.
+ *   2. ufp4_gemm_{fprop,dgrad,wgrad}: C[i][j] = (1/n) sum_k A[i][k] B[j][k]
+ *      over the dequantized operands, fp32 accumulation, fp32 output.
+ *   3. ufp4_grouped_gemm: the same contraction for a table of independent
+ *      sub-problems (mixture-of-experts layers).
+ *
+ * Conventions shared by every call:
+ *   - All pointers named *_dev, and every pointer inside ufp4_qtensor_t, are
+ *     device pointers owned by the caller.  The library never allocates,
+ *     frees or synchronises; work is enqueued on `stream` (a cudaStream_t
+ *     passed as void*; NULL = legacy default stream) and returns at once.
+ *   - Arguments are validated on the host before any launch; a failed check
+ *     returns an error status and enqueues nothing.
+ *   - Inputs are assumed finite; NaN/Inf inputs give unspecified codes.
+ *   - Outputs are overwritten (no accumulation into C).
+ *
+ * Quantized operand layout (ufp4_qtensor_t), for `rows` output rows and
+ * reduction length `k`:
+ *   kpad      = k rounded up to a multiple of 64; positions >= k hold zeros.
+ *   codes     u8 [rows][kpad/2], row-major.  Byte j of a row holds element 2j
+ *             in its low nibble and element 2j+1 in its high nibble.  A nibble
+ *             is sign-magnitude: bit 3 = sign, bits 0..2 = magnitude index k
+ *             of the grid (E1M2: k/4; E2M1: {0,.5,1,1.5,2,3,4,6}[k]).  Zero is
+ *             always 0x0, never 0x8.
+ *   scales    block-major: entry (row r, block b) at scales[b*scale_ld + r],
+ *             scale_ld = rows rounded up to a multiple of 64.
+ *             UFP4_SCALE_FP32:         fp32, s = RN(amax_b / gmax).
+ *             UFP4_SCALE_E4M3_X_FP32:  u8 OCP E4M3 e_b; the step of the block
+ *                                      is e_b * S with S = *tensor_scale.
+ *   The dequantized (rotated) value of element (r, t) is s * lvl(code); the
+ *   Hadamard normalisation 1/n is applied once in the GEMM (n = 0: none).
+ */
+#ifndef UFP4_H
+#define UFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    UFP4_OK = 0,
+    UFP4_ERR_INVALID_ARG = 1,      /* null pointer, bad size or enum value       */
+    UFP4_ERR_UNSUPPORTED = 2,      /* valid but not implemented combination      */
+    UFP4_ERR_ALIGNMENT = 3,        /* pointer / leading dimension alignment      */
+    UFP4_ERR_OPERAND_MISMATCH = 4, /* GEMM operands quantized incompatibly       */
+    UFP4_ERR_CUDA = 5,             /* a CUDA runtime/driver call failed          */
+    UFP4_ERR_DEVICE_TIMEOUT = 6    /* a kernel's bounded wait gave up            */
+} ufp4_status_t;
+
+/* 4-bit grids, [PL] §2 "FP4 formats" and §4.  INT4 is the E1M2 grid (same
+ * codes under absmax scaling). */
+typedef enum { UFP4_GRID_E1M2 = 0, UFP4_GRID_E2M1 = 1 } ufp4_grid_t;
+/* Rounding rules, [PL] §2 "Rounding rules": RTNE for X and W, SR on dY. */
+typedef enum { UFP4_ROUND_RTNE = 0, UFP4_ROUND_SR = 1 } ufp4_round_t;
+/* Block scale formats: plain fp32 per block, or the two-level hierarchy of
+ * NVFP4 ([PL] §6 "FP4 formats, block scaling, and scale hierarchy") that UFP4
+ * inherits ([DW]: the NVFP4 recipe with the grid swapped). */
+typedef enum { UFP4_SCALE_FP32 = 0, UFP4_SCALE_E4M3_X_FP32 = 1 } ufp4_scale_fmt_t;
+/* Which input dimension is the GEMM's reduction dimension ([PL] §2: input
+ * channels for fwd_y, output channels for bwd_dx, tokens for bwd_dw).
+ * ALONG_COLS: the contiguous dimension; output row r = input row r.
+ * ALONG_ROWS: the strided dimension; output row r = input column r (the
+ *             quantized operand is the transpose, K-major). */
+typedef enum { UFP4_ALONG_COLS = 0, UFP4_ALONG_ROWS = 1 } ufp4_axis_t;
+
+/* Quantizer configuration.  Fixed-width fields (C ABI stable). */
+typedef struct {
+    int32_t grid;           /* ufp4_grid_t                                   */
+    int32_t rounding;       /* ufp4_round_t                                  */
+    uint64_t sr_seed;       /* Philox4x32-10 key (SR only)                   */
+    uint32_t sr_stream;     /* Philox counter word 2 (SR only)               */
+    int32_t hadamard_n;     /* 0 (no RHT), 16, 32 or 64                      */
+    uint64_t rht_sign_mask; /* bit i set => D_ii = -1, i < hadamard_n        */
+    int32_t block;          /* scale block length along K: 16 or 32          */
+    int32_t scale_fmt;      /* ufp4_scale_fmt_t                              */
+} ufp4_quant_cfg_t;
+
+/* A quantized operand: plain descriptor, owns nothing. */
+typedef struct {
+    void *codes;            /* device u8 [rows][kpad/2]                      */
+    void *scales;           /* device, block-major, see layout above         */
+    float *tensor_scale;    /* device fp32 S (two-level only, else NULL)     */
+    int64_t rows;           /* output rows of the K-major view               */
+    int64_t k;              /* logical reduction length                      */
+    int64_t kpad;           /* k rounded up to 64                            */
+    int64_t scale_ld;       /* rows rounded up to 64                         */
+    ufp4_quant_cfg_t cfg;   /* how it was quantized                          */
+} ufp4_qtensor_t;
+
+/* One sub-problem of ufp4_grouped_gemm:
+ *   C[c_row+i][c_col+j] = (1/n) sum_{t<k} A[a_row+i][a_col+t] * B[b_row+j][b_col+t]
+ * for 0 <= i < m, 0 <= j < n.  k, a_col and b_col are multiples of 64. */
+typedef struct {
+    int64_t m, n, k;
+    int64_t a_row, a_col;
+    int64_t b_row, b_col;
+    int64_t c_row, c_col;
+} ufp4_group_t;
+
+/* Default RHT sign mask: bits of splitmix64(0x5EED), any fixed choice works
+ * as long as both operands of a GEMM use the same one. */
+#define UFP4_DEFAULT_SIGN_MASK 0x09F1FD9D03F0A9B4ull
+
+/* Sizes of a quantized operand.  Fills kpad, scale_ld and the byte counts of
+ * the codes and scales buffers the caller must provide.  Any output pointer
+ * may be NULL.  Errors: UFP4_ERR_INVALID_ARG (rows < 0, k < 0, bad cfg). */
+ufp4_status_t ufp4_qtensor_layout(int64_t rows, int64_t k, const ufp4_quant_cfg_t *cfg,
+                                  int64_t *kpad, int64_t *scale_ld,
+                                  size_t *codes_bytes, size_t *scales_bytes);
+
+/* Absolute maximum of the rotated operand, max |H_n D x| over all elements
+ * (the tensor amax that the two-level scale S is derived from; [PL] §2
+ * "Random Hadamard transforms").  Input x_dev: bf16 [rows][ld] row-major,
+ * 16-byte aligned, ld and (for ALONG_COLS) cols multiples of 8.  Writes one
+ * fp32 to amax_dev (device).  Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED
+ * (hadamard_n not in {0,16,32,64}), CUDA. */
+ufp4_status_t ufp4_rht_amax(const void *x_dev, int64_t rows, int64_t cols, int64_t ld,
+                            int32_t axis, int32_t hadamard_n, uint64_t rht_sign_mask,
+                            float *amax_dev, void *stream);
+
+/* Fused RHT + block absmax + scale + 4-bit rounding + packing ([PL] §2
+ * "Blockwise quantization", "Rounding rules", "Random Hadamard transforms";
+ * [PL] §5 and [GS] "Efficiëntie": RHT fused into the quantizer).
+ *   x_dev       bf16 [rows][ld], row-major, 16-byte aligned, ld % 8 == 0;
+ *               cols % 8 == 0 for ALONG_COLS, rows % 8 == 0 not required.
+ *   axis        ufp4_axis_t, the reduction dimension of the consuming GEMM.
+ *   tensor_amax_dev  device fp32 rotated amax (two-level scale only; from
+ *               ufp4_rht_amax or the caller), else NULL.
+ *   out         descriptor filled by the caller: codes/scales buffers sized by
+ *               ufp4_qtensor_layout, rows = output rows (rows for ALONG_COLS,
+ *               cols for ALONG_ROWS), k = the other dimension, kpad,
+ *               scale_ld, cfg; tensor_scale (two-level) receives S.
+ * SR draws are a pure function of (sr_seed, sr_stream, output row, column):
+ * the same call gives the same bits on any launch configuration.
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED, CUDA. */
+ufp4_status_t ufp4_rht_quantize(const void *x_dev, int64_t rows, int64_t cols, int64_t ld,
+                                int32_t axis, const float *tensor_amax_dev,
+                                ufp4_qtensor_t *out, void *stream);
+
+/* FPROP, fwd_y:  Y[M][N] = X W^T.  xq: X quantized ALONG_COLS ([M][K]);
+ * wq: W quantized ALONG_COLS ([N][K]).  y_dev fp32 [M][ldy], ldy >= N,
+ * 4-byte aligned (rows that are 16-byte aligned get vector stores).
+ * ([PL] §2: rotation along input channels.)
+ * Errors: INVALID_ARG, ALIGNMENT, OPERAND_MISMATCH (grid, block, scale format,
+ * hadamard_n, sign mask or kpad differ), UNSUPPORTED, CUDA. */
+ufp4_status_t ufp4_gemm_fprop(const ufp4_qtensor_t *xq, const ufp4_qtensor_t *wq,
+                              float *y_dev, int64_t ldy, void *stream);
+
+/* DGRAD, bwd_dx:  dX[M][K] = dY W.  dyq: dY [M][N] quantized ALONG_COLS
+ * (usually SR); wtq: W [N][K] quantized ALONG_ROWS, i.e. W^T [K][N] K-major.
+ * dx_dev fp32 [M][lddx].  ([PL] §2: rotation along output channels.) */
+ufp4_status_t ufp4_gemm_dgrad(const ufp4_qtensor_t *dyq, const ufp4_qtensor_t *wtq,
+                              float *dx_dev, int64_t lddx, void *stream);
+
+/* WGRAD, bwd_dw:  dW[N][K] = dY^T X.  dytq: dY [M][N] quantized ALONG_ROWS
+ * (dY^T [N][M]); xtq: X [M][K] quantized ALONG_ROWS (X^T [K][M]).
+ * dw_dev fp32 [N][lddw].  ([PL] §2: rotation along batch tokens.) */
+ufp4_status_t ufp4_gemm_wgrad(const ufp4_qtensor_t *dytq, const ufp4_qtensor_t *xtq,
+                              float *dw_dev, int64_t lddw, void *stream);
+
+/* Grouped contraction for mixture-of-experts layers (the recipe is trained
+ * on MoE 7.9B / 124B models, [PL] §5 Q2-Q3).  groups_dev: device array of
+ * num_groups ufp4_group_t, read by the kernel (the tile schedule is derived on
+ * the device, so the table may be written by earlier kernels on the same
+ * stream without a host round trip).  All groups share the
+ * quantized operands a and b (same constraints as ufp4_gemm_fprop) and the
+ * fp32 output c_dev [..][ldc].  Groups must not write overlapping outputs.
+ * Errors: INVALID_ARG, ALIGNMENT, OPERAND_MISMATCH, UNSUPPORTED, CUDA. */
+ufp4_status_t ufp4_grouped_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
+                                const ufp4_group_t *groups_dev, int32_t num_groups,
+                                float *c_dev, int64_t ldc, void *stream);
+
+/* Reads and clears the device-side error word that kernels set when a
+ * bounded pipeline wait gives up (synchronises the current device).
+ * Returns UFP4_OK or UFP4_ERR_DEVICE_TIMEOUT (or UFP4_ERR_CUDA). */
+ufp4_status_t ufp4_check_device_status(void);
+
+/* Human-readable name of a status code (static string). */
+const char *ufp4_status_string(ufp4_status_t status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int32_t ufp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* UFP4_H */

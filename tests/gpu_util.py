@@ -1,0 +1,68 @@
+"""Helpers for the GPU parity tests: move seeded inputs to the device, read the
+library's packed outputs back in the oracle's logical layout."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp4_quantized_gemms_b200 import ufp4
+
+needs_gpu = [pytest.mark.gpu,
+             pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+GEMM_RTOL = 1e-5   # relative Frobenius error vs the fp64 oracle (the method's bound)
+
+
+def to_dev(bits: np.ndarray) -> torch.Tensor:
+    """bf16 bit pattern (uint16) -> bf16 CUDA tensor with the same bits."""
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.view(torch.bfloat16).cuda()
+
+
+def oracle_cfg(cfg: ufp4.QuantConfig) -> oracle.QuantCfg:
+    return oracle.QuantCfg(grid=cfg.grid, rounding=cfg.rounding, sr_seed=cfg.sr_seed,
+                           sr_stream=cfg.sr_stream, hadamard_n=cfg.hadamard_n,
+                           sign_mask=cfg.rht_sign_mask, block=cfg.block,
+                           scale_fmt=cfg.scale_fmt)
+
+
+def unpack_codes(q: ufp4.QTensor, rows=None) -> np.ndarray:
+    """uint8 [rows, kpad/2] -> int8 nibbles [rows, kpad], low nibble first."""
+    c = q.codes if rows is None else q.codes[torch.as_tensor(rows, device=q.codes.device)]
+    b = c.cpu().numpy()
+    out = np.empty((b.shape[0], b.shape[1] * 2), dtype=np.int8)
+    out[:, 0::2] = b & 0x0F
+    out[:, 1::2] = b >> 4
+    return out
+
+
+def logical_scales(q: ufp4.QTensor, rows=None) -> np.ndarray:
+    """block-major [nblk, scale_ld] -> [rows, nblk]."""
+    s = q.scales.cpu().numpy()[:, :q.rows].T
+    return s if rows is None else s[np.asarray(rows)]
+
+
+def tensor_scale(q: ufp4.QTensor) -> float:
+    return float(q.tensor_scale.cpu().numpy()[0]) if q.tensor_scale is not None else 1.0
+
+
+def assert_quant_equal(q: ufp4.QTensor, ref: oracle.QTensor, rows=None):
+    got = unpack_codes(q, rows)
+    if not np.array_equal(got, ref.codes):
+        bad = np.argwhere(got != ref.codes)
+        r, c = bad[0]
+        raise AssertionError(f"{len(bad)} codes differ; first at ({r},{c}): gpu {got[r, c]} "
+                             f"oracle {ref.codes[r, c]}")
+    sc = logical_scales(q, rows)
+    if ref.scales is not None:
+        assert np.array_equal(sc.view(np.uint32), ref.scales.view(np.uint32)), "fp32 scales differ"
+    else:
+        assert np.array_equal(sc, ref.escales), "E4M3 block scales differ"
+        assert np.float32(tensor_scale(q)) == np.float32(ref.S), "tensor scale differs"
+
+
+def rel_fro(got: np.ndarray, ref: np.ndarray) -> float:
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = np.linalg.norm(ref)
+    return float(np.linalg.norm(got - ref) / (den if den > 0 else 1.0))

@@ -1,0 +1,144 @@
+"""C ABI checks that need no GPU: the library builds and loads, exports every
+function ``include/ufp4.h`` declares, the ctypes mirrors match the C struct
+layouts, and host-side validation rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from fp4_quantized_gemms_b200 import build as ufp4_build
+from fp4_quantized_gemms_b200 import ufp4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ufp4.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    ufp4_build.build()
+    return ufp4.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ufp4_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert set(names) == set(ufp4.EXPORTED)
+    nm = subprocess.run(["nm", "-D", "--defined-only", ufp4.LIB_PATH], capture_output=True,
+                        text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(ufp4_\w+)", nm))
+    for n in names:
+        assert n in exported, n
+        assert hasattr(L, n)
+
+
+def test_struct_layouts_match_header(tmp_path):
+    """sizeof / offsetof from the C compiler == the ctypes mirrors."""
+    src = tmp_path / "layout.c"
+    src.write_text("""
+#include <stdio.h>
+#include <stddef.h>
+#include "ufp4.h"
+int main(void) {
+  printf("%zu %zu %zu %zu %zu\\n", sizeof(ufp4_quant_cfg_t), offsetof(ufp4_quant_cfg_t, sr_seed),
+         offsetof(ufp4_quant_cfg_t, rht_sign_mask), offsetof(ufp4_quant_cfg_t, scale_fmt), 0);
+  printf("%zu %zu %zu %zu\\n", sizeof(ufp4_qtensor_t), offsetof(ufp4_qtensor_t, rows),
+         offsetof(ufp4_qtensor_t, scale_ld), offsetof(ufp4_qtensor_t, cfg));
+  printf("%zu %zu\\n", sizeof(ufp4_group_t), offsetof(ufp4_group_t, c_col));
+  return 0;
+}
+""")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    c1 = list(map(int, out[0].split()))
+    c2 = list(map(int, out[1].split()))
+    c3 = list(map(int, out[2].split()))
+    Q, T, G = ufp4.QuantCfgC, ufp4.QTensorC, ufp4.GroupC
+    assert c1[:4] == [ctypes.sizeof(Q), Q.sr_seed.offset, Q.rht_sign_mask.offset, Q.scale_fmt.offset]
+    assert c2 == [ctypes.sizeof(T), T.rows.offset, T.scale_ld.offset, T.cfg.offset]
+    assert c3 == [ctypes.sizeof(G), G.c_col.offset]
+
+
+def test_status_strings_and_version(L):
+    assert ufp4.status_string(ufp4.OK) == "UFP4_OK"
+    assert ufp4.status_string(ufp4.ERR_OPERAND_MISMATCH) == "UFP4_ERR_OPERAND_MISMATCH"
+    assert L.ufp4_version() >= 100
+
+
+@pytest.mark.parametrize("k,block,fmt,kpad,codes,scales", [
+    (512, 16, ufp4.SCALE_FP32, 512, 256 * 256, 32 * 256 * 4),
+    (500, 16, ufp4.SCALE_FP32, 512, 256 * 256, 32 * 256 * 4),
+    (2048, 32, ufp4.SCALE_E4M3_X_FP32, 2048, 256 * 1024, 64 * 256),
+    (0, 16, ufp4.SCALE_FP32, 0, 0, 0),
+])
+def test_layout(L, k, block, fmt, kpad, codes, scales):
+    cfg = ufp4.QuantConfig(block=block, scale_fmt=fmt)
+    kp, sld, cb, sb = ufp4.layout(256, k, cfg)
+    assert (kp, sld, cb, sb) == (kpad, 256, codes, scales)
+    assert ufp4.layout(300, 64, cfg)[1] == 320
+
+
+def _q(rows=128, k=256, **kw):
+    cfg = ufp4.QuantConfig(**kw).c()
+    kp = (k + 63) // 64 * 64
+    return ufp4.QTensorC(16 * 1024, 32 * 1024, 48 * 1024 if kw.get("scale_fmt") else None,
+                         rows, k, kp, (rows + 63) // 64 * 64, cfg)
+
+
+def _gemm(L, a, b, c_ptr=64 * 1024, ldc=128):
+    return L.ufp4_gemm_fprop(ctypes.byref(a), ctypes.byref(b), ctypes.c_void_p(c_ptr), ldc, None)
+
+
+def test_gemm_validation_rejects_before_launch(L):
+    """Every rejection below happens on the host: no CUDA call is made."""
+    assert _gemm(L, _q(grid=0), _q(grid=1)) == ufp4.ERR_OPERAND_MISMATCH
+    assert _gemm(L, _q(block=16), _q(block=32)) == ufp4.ERR_OPERAND_MISMATCH
+    assert _gemm(L, _q(hadamard_n=16), _q(hadamard_n=32)) == ufp4.ERR_OPERAND_MISMATCH
+    assert _gemm(L, _q(rht_sign_mask=1), _q(rht_sign_mask=2)) == ufp4.ERR_OPERAND_MISMATCH
+    # sign-mask bits beyond n do not matter
+    a, b = _q(hadamard_n=16, rht_sign_mask=0x1_0001), _q(hadamard_n=16, rht_sign_mask=0x2_0001)
+    assert _gemm(L, a, b, c_ptr=64 * 1024 + 2) == ufp4.ERR_ALIGNMENT
+    assert _gemm(L, _q(k=256), _q(k=192)) == ufp4.ERR_OPERAND_MISMATCH
+    assert _gemm(L, _q(scale_fmt=0), _q(scale_fmt=1)) == ufp4.ERR_OPERAND_MISMATCH
+    bad = _q()
+    bad.kpad = 100
+    assert _gemm(L, bad, _q()) == ufp4.ERR_INVALID_ARG
+    bad = _q()
+    bad.codes = 16 * 1024 + 8
+    assert _gemm(L, bad, _q()) == ufp4.ERR_ALIGNMENT
+    bad = _q(scale_fmt=1)
+    bad.tensor_scale = None
+    assert _gemm(L, bad, _q(scale_fmt=1)) == ufp4.ERR_INVALID_ARG
+    assert _gemm(L, _q(), _q(), ldc=64) == ufp4.ERR_INVALID_ARG    # ldc < N
+    assert _gemm(L, _q(), _q(), c_ptr=64 * 1024 + 1) == ufp4.ERR_ALIGNMENT
+    bad_cfg = _q()
+    bad_cfg.cfg.hadamard_n = 8
+    assert _gemm(L, bad_cfg, _q()) == ufp4.ERR_INVALID_ARG
+    assert L.ufp4_gemm_fprop(None, ctypes.byref(_q()), None, 128, None) == ufp4.ERR_INVALID_ARG
+    assert L.ufp4_grouped_gemm(ctypes.byref(_q()), ctypes.byref(_q()), None, 3, None, 128,
+                               None) == ufp4.ERR_INVALID_ARG
+    assert L.ufp4_grouped_gemm(ctypes.byref(_q()), ctypes.byref(_q()), None, -1, None, 128,
+                               None) == ufp4.ERR_INVALID_ARG
+
+
+def test_quantize_validation_rejects_before_launch(L):
+    out = _q(rows=64, k=128)
+    x = ctypes.c_void_p(4096)
+    Q = L.ufp4_rht_quantize
+    assert Q(None, 64, 128, 128, 0, None, ctypes.byref(out), None) == ufp4.ERR_INVALID_ARG
+    assert Q(x, 64, 128, 100, 0, None, ctypes.byref(out), None) == ufp4.ERR_INVALID_ARG   # ld < cols
+    assert Q(x, 64, 120, 124, 0, None, ctypes.byref(_q(rows=64, k=120)), None) == ufp4.ERR_ALIGNMENT
+    assert Q(ctypes.c_void_p(4098), 64, 128, 128, 0, None, ctypes.byref(out), None) == ufp4.ERR_ALIGNMENT
+    assert Q(x, 64, 128, 128, 2, None, ctypes.byref(out), None) == ufp4.ERR_INVALID_ARG   # axis
+    assert Q(x, 64, 128, 128, 1, None, ctypes.byref(out), None) == ufp4.ERR_INVALID_ARG   # shape
+    two = _q(rows=64, k=128, scale_fmt=1)
+    assert Q(x, 64, 128, 128, 0, None, ctypes.byref(two), None) == ufp4.ERR_INVALID_ARG   # no amax
+    assert L.ufp4_rht_amax(x, 64, 128, 128, 0, 8, 0, ctypes.c_void_p(4096), None) == ufp4.ERR_UNSUPPORTED
+    assert L.ufp4_rht_amax(x, 64, 128, 128, 0, 16, 0, None, None) == ufp4.ERR_INVALID_ARG

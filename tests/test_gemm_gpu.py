@@ -1,0 +1,157 @@
+"""Parity of the three training GEMMs with the oracle.
+
+The CUDA path (GPU quantize -> GPU GEMM) and the oracle path (oracle quantize
+-> fp64 contraction of the dequantized operands) start from the same seeded
+bf16 inputs; the GPU's codes are checked bit-exactly and its fp32 output
+within GEMM_RTOL relative Frobenius error of the fp64 result."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp4_quantized_gemms_b200 import ufp4
+from fp4_quantized_gemms_b200 import workloads as wl
+from tests.gpu_util import (GEMM_RTOL, assert_quant_equal, needs_gpu, oracle_cfg, rel_fro,
+                            to_dev)
+
+pytestmark = needs_gpu
+
+C, R = ufp4.ALONG_COLS, ufp4.ALONG_ROWS
+
+
+def _quant_both(bits, axis, cfg, rows=None):
+    """GPU and oracle quantization of the same operand (optionally only some
+    output rows on the oracle side)."""
+    x = to_dev(bits)
+    amax_d, amax_o = None, 0.0
+    if cfg.scale_fmt == ufp4.SCALE_E4M3_X_FP32:
+        amax_d = ufp4.rht_amax(x, axis, cfg.hadamard_n, cfg.rht_sign_mask)
+        amax_o = oracle.rht_amax(bits, axis, cfg.hadamard_n, cfg.rht_sign_mask)
+    q = ufp4.rht_quantize(x, axis, cfg, tensor_amax=amax_d)
+    oc = oracle_cfg(cfg)
+    if rows is None:
+        ref = oracle.quantize(bits, axis, oc, tensor_amax=amax_o)
+    else:
+        parts = [oracle.quantize(bits, axis, oc, tensor_amax=amax_o, r0=int(r), nr=1) for r in rows]
+        ref = parts[0]
+        ref.codes = np.concatenate([p.codes for p in parts])
+        if ref.scales is not None:
+            ref.scales = np.concatenate([p.scales for p in parts])
+        else:
+            ref.escales = np.concatenate([p.escales for p in parts])
+    return q, ref
+
+
+def _check_full(qa, ra, qb, rb, fn):
+    out = fn(qa, qb)
+    torch.cuda.synchronize()
+    assert ufp4.check_device_status() == ufp4.OK
+    assert_quant_equal(qa, ra)
+    assert_quant_equal(qb, rb)
+    ref = oracle.gemm_tn(ra, rb)
+    got = out.cpu().numpy()
+    assert got.shape == ref.shape
+    err = rel_fro(got, ref)
+    assert err <= GEMM_RTOL, err
+    return err
+
+
+def _cfg(grid=0, fmt=0, n=16, block=16, rounding=0, stream=0):
+    return ufp4.QuantConfig(grid=grid, rounding=rounding, sr_seed=1234, sr_stream=stream,
+                            hadamard_n=n, block=block, scale_fmt=fmt)
+
+
+@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1])
+@pytest.mark.parametrize("fmt", [ufp4.SCALE_FP32, ufp4.SCALE_E4M3_X_FP32])
+def test_fprop_tiny_config(grid, fmt):
+    """X 256x512 with 4 outlier columns x20, W 512x512 ~ N(0, 0.02), RHT16, block 16."""
+    X, W, _ = wl.layer_inputs(wl.TINY, want_dy=False)
+    cfg = _cfg(grid=grid, fmt=fmt)
+    qx, rx = _quant_both(X, C, cfg)
+    qw, rw = _quant_both(W, C, cfg)
+    _check_full(qx, rx, qw, rw, ufp4.gemm_fprop)
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 200, 200), (128, 256, 64), (1, 1, 8), (129, 257, 136),
+                                   (640, 520, 1000)])
+@pytest.mark.parametrize("fmt", [ufp4.SCALE_FP32, ufp4.SCALE_E4M3_X_FP32])
+@pytest.mark.parametrize("grid,n,block", [(0, 16, 16), (1, 32, 32), (0, 64, 32), (1, 0, 16),
+                                          (0, 0, 32)])
+def test_fprop_ragged_shapes(M, N, K, fmt, grid, n, block):
+    """Partial M / N tiles, K tails padded inside the quantizer, degenerate sizes."""
+    X = wl.normal_with_outlier_channels(M, K, 1.0, min(2, K), 20.0)
+    W = wl.normal(N, K, 0.02, 2)
+    cfg = _cfg(grid=grid, fmt=fmt, n=n, block=block)
+    qx, rx = _quant_both(X, C, cfg)
+    qw, rw = _quant_both(W, C, cfg)
+    _check_full(qx, rx, qw, rw, ufp4.gemm_fprop)
+
+
+@pytest.mark.parametrize("fmt", [ufp4.SCALE_FP32, ufp4.SCALE_E4M3_X_FP32])
+@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1])
+def test_layer_dgrad_wgrad_small(fmt, grid):
+    """The full recipe on a small layer: RHT on every operand along its GEMM's
+    K, RTNE for X / W, SR on dY (stream 0 for DGRAD, 1 for WGRAD)."""
+    M, K, N = 384, 320, 264
+    X = wl.normal_with_outlier_channels(M, K, 1.0, 3, 30.0)
+    W = wl.normal(N, K, 0.02, 2)
+    dY = wl.normal(M, N, 1e-3, 3)
+    rtne, sr0, sr1 = _cfg(grid=grid, fmt=fmt), _cfg(grid=grid, fmt=fmt, rounding=1, stream=0), \
+        _cfg(grid=grid, fmt=fmt, rounding=1, stream=1)
+    qdy, rdy = _quant_both(dY, C, sr0)          # [M, N], K = N
+    qwt, rwt = _quant_both(W, R, rtne)          # W^T [K, N]
+    _check_full(qdy, rdy, qwt, rwt, ufp4.gemm_dgrad)
+    qdyt, rdyt = _quant_both(dY, R, sr1)        # dY^T [N, M]
+    qxt, rxt = _quant_both(X, R, rtne)          # X^T [K, M]
+    _check_full(qdyt, rdyt, qxt, rxt, ufp4.gemm_wgrad)
+
+
+def _sampled(shape: wl.LayerShape, fmt, grid, gemm, n_rows=96, n_cols=96):
+    """One GEMM of a full-size layer in the production launch; the oracle
+    computes a sampled row x column block of the output."""
+    X, W, dY = wl.layer_inputs(shape, want_dy=gemm != "fprop")
+    rng = np.random.default_rng(17)
+    if gemm == "fprop":
+        a_bits, a_axis, a_cfg = X, C, _cfg(grid=grid, fmt=fmt)
+        b_bits, b_axis, b_cfg = W, C, _cfg(grid=grid, fmt=fmt)
+        fn = ufp4.gemm_fprop
+    elif gemm == "dgrad":
+        a_bits, a_axis, a_cfg = dY, C, _cfg(grid=grid, fmt=fmt, rounding=1, stream=0)
+        b_bits, b_axis, b_cfg = W, R, _cfg(grid=grid, fmt=fmt)
+        fn = ufp4.gemm_dgrad
+    else:
+        a_bits, a_axis, a_cfg = dY, R, _cfg(grid=grid, fmt=fmt, rounding=1, stream=1)
+        b_bits, b_axis, b_cfg = X, R, _cfg(grid=grid, fmt=fmt)
+        fn = ufp4.gemm_wgrad
+    ma = a_bits.shape[0] if a_axis == C else a_bits.shape[1]
+    nb = b_bits.shape[0] if b_axis == C else b_bits.shape[1]
+    ii = np.unique(np.concatenate([[0, ma - 1], rng.choice(ma, n_rows, replace=False)]))
+    jj = np.unique(np.concatenate([[0, nb - 1], rng.choice(nb, n_cols, replace=False)]))
+    qa, ra = _quant_both(a_bits, a_axis, a_cfg, rows=ii)
+    qb, rb = _quant_both(b_bits, b_axis, b_cfg, rows=jj)
+    out = fn(qa, qb)
+    torch.cuda.synchronize()
+    assert ufp4.check_device_status() == ufp4.OK
+    assert_quant_equal(qa, ra, ii)
+    assert_quant_equal(qb, rb, jj)
+    ref = oracle.gemm_tn(ra, rb)                       # [len(ii), len(jj)]
+    got = out[torch.as_tensor(ii, device="cuda")][:, torch.as_tensor(jj, device="cuda")].cpu().numpy()
+    err = rel_fro(got, ref)
+    assert err <= GEMM_RTOL, err
+    return err
+
+
+@pytest.mark.parametrize("gemm", ["fprop", "dgrad", "wgrad"])
+@pytest.mark.parametrize("fmt", [ufp4.SCALE_FP32, ufp4.SCALE_E4M3_X_FP32])
+def test_layer_config_sampled(gemm, fmt):
+    """X 8192x2048 (10 outlier channels x30), W 8192x2048, dY 8192x8192."""
+    _sampled(wl.LAYER, fmt, ufp4.GRID_E1M2, gemm)
+
+
+@pytest.mark.parametrize("gemm", ["fprop", "dgrad", "wgrad"])
+@pytest.mark.parametrize("fmt,grid", [(ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E1M2),
+                                      (ufp4.SCALE_FP32, ufp4.GRID_E1M2),
+                                      (ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E2M1)])
+def test_large_config_sampled(gemm, fmt, grid):
+    """M=16384, K=8192, N=28672 (1% outlier channels x50): the largest layer."""
+    _sampled(wl.LARGE, fmt, grid, gemm, n_rows=64, n_cols=64)

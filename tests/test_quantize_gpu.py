@@ -1,0 +1,116 @@
+"""Parity of the fused RHT + quantize kernel with the oracle: bit-exact codes,
+block scales, tensor scales and SR draws, on shapes that span several work
+units and ragged tails, and on the quantizer-sweep sizes (sampled rows)."""
+import itertools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp4_quantized_gemms_b200 import ufp4
+from fp4_quantized_gemms_b200 import workloads as wl
+from tests.gpu_util import assert_quant_equal, needs_gpu, oracle_cfg, to_dev
+
+pytestmark = needs_gpu
+
+AXES = [ufp4.ALONG_COLS, ufp4.ALONG_ROWS]
+
+
+def _run(x_bits, axis, cfg, rows=None):
+    x = to_dev(x_bits)
+    amax_o = 0.0
+    amax_d = None
+    if cfg.scale_fmt == ufp4.SCALE_E4M3_X_FP32:
+        amax_o = oracle.rht_amax(x_bits, axis, cfg.hadamard_n, cfg.rht_sign_mask)
+        amax_d = ufp4.rht_amax(x, axis, cfg.hadamard_n, cfg.rht_sign_mask)
+        assert np.float32(amax_d.item()) == np.float32(amax_o)
+    q = ufp4.rht_quantize(x, axis, cfg, tensor_amax=amax_d)
+    torch.cuda.synchronize()
+    oc = oracle_cfg(cfg)
+    if rows is None:
+        ref = oracle.quantize(x_bits, axis, oc, tensor_amax=amax_o)
+    else:
+        refs = [oracle.quantize(x_bits, axis, oc, tensor_amax=amax_o, r0=int(r), nr=1) for r in rows]
+        ref = refs[0]
+        ref.codes = np.concatenate([r.codes for r in refs])
+        if ref.scales is not None:
+            ref.scales = np.concatenate([r.scales for r in refs])
+        else:
+            ref.escales = np.concatenate([r.escales for r in refs])
+    assert_quant_equal(q, ref, rows)
+    return q
+
+
+GRID_ROUND_FMT = list(itertools.product([ufp4.GRID_E1M2, ufp4.GRID_E2M1],
+                                        [ufp4.ROUND_RTNE, ufp4.ROUND_SR],
+                                        [ufp4.SCALE_FP32, ufp4.SCALE_E4M3_X_FP32]))
+
+
+@pytest.mark.parametrize("axis", AXES)
+@pytest.mark.parametrize("n,block", [(0, 16), (16, 16), (16, 32), (32, 16), (32, 32), (64, 16),
+                                     (64, 32), (0, 32)])
+@pytest.mark.parametrize("grid,rounding,fmt", GRID_ROUND_FMT)
+def test_quantize_matches_oracle_small(axis, n, block, grid, rounding, fmt):
+    """200 x 136: ragged rows (not a multiple of 8 / 64) and a ragged K tail."""
+    X = wl.student_t(200, 136, seed=11)
+    cfg = ufp4.QuantConfig(grid=grid, rounding=rounding, sr_seed=1234, sr_stream=axis,
+                           hadamard_n=n, block=block, scale_fmt=fmt)
+    _run(X, axis, cfg)
+
+
+@pytest.mark.parametrize("axis", AXES)
+@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1])
+def test_quantize_exact_ties_and_zero_blocks(axis, grid):
+    """n = 0 with values on grid midpoints (exact RTNE ties), level values (SR
+    must not move them), all-zero blocks and a block whose max is tiny."""
+    rng = np.random.default_rng(3)
+    lv = oracle.levels(grid)
+    mids = (lv[:-1] + lv[1:]) / 2
+    vals = np.concatenate([mids, lv, -mids, -lv])
+    X = rng.choice(vals, size=(64, 128)).astype(np.float32) * np.float32(0.5)
+    X[:, 0::16] = np.float32(lv[-1] * 0.5)          # block max = gmax * 0.5 -> s = 0.5 (exact)
+    X[5, :] = 0.0
+    X[9, 32:48] = 0.0
+    X[11, 64:80] = np.float32(1e-30)
+    bits = wl.bf16_bits(X)
+    for rounding in (ufp4.ROUND_RTNE, ufp4.ROUND_SR):
+        cfg = ufp4.QuantConfig(grid=grid, rounding=rounding, sr_seed=7, hadamard_n=0)
+        _run(bits, axis, cfg)
+
+
+@pytest.mark.parametrize("axis", AXES)
+def test_quantize_medium_with_outliers(axis):
+    X = wl.normal_with_outlier_channels(1000, 1000, 1.0, 5, 30.0)
+    for grid, rnd in [(0, 0), (0, 1), (1, 0)]:
+        cfg = ufp4.QuantConfig(grid=grid, rounding=rnd, sr_seed=1234, hadamard_n=16, block=16)
+        _run(X, axis, cfg)
+
+
+def test_sr_draws_independent_of_launch_shape():
+    """SR bits are a function of (seed, stream, row, column) only: quantizing a
+    row block alone gives the same codes as inside the full tensor."""
+    X = wl.student_t(256, 512, seed=12)
+    cfg = ufp4.QuantConfig(rounding=ufp4.ROUND_SR, sr_seed=99, hadamard_n=32)
+    full = ufp4.rht_quantize(to_dev(X), ufp4.ALONG_COLS, cfg)
+    again = ufp4.rht_quantize(to_dev(X), ufp4.ALONG_COLS, cfg)
+    assert torch.equal(full.codes, again.codes)
+    other = ufp4.rht_quantize(to_dev(X), ufp4.ALONG_COLS, cfg.with_(sr_seed=100))
+    assert not torch.equal(full.codes, other.codes)
+
+
+@pytest.mark.parametrize("shape", wl.QUANT_SWEEP_SHAPES)
+@pytest.mark.parametrize("axis", AXES)
+def test_quantize_sweep_sizes_sampled(shape, axis):
+    """Full quantizer-sweep sizes in the production launch; 48 sampled output
+    rows (plus the first and last) checked against the oracle row by row."""
+    rows, cols = shape
+    X = wl.student_t(rows, cols)
+    nout = rows if axis == ufp4.ALONG_COLS else cols
+    rng = np.random.default_rng(rows + axis)
+    sample = np.unique(np.concatenate([[0, nout - 1], rng.choice(nout, 48, replace=False)]))
+    for grid, rnd, n, block in [(0, 0, 16, 16), (0, 1, 64, 32), (1, 0, 32, 16)]:
+        cfg = ufp4.QuantConfig(grid=grid, rounding=rnd, sr_seed=1234, hadamard_n=n, block=block)
+        _run(X, axis, cfg, rows=sample)
+    cfg = ufp4.QuantConfig(hadamard_n=16, block=16, scale_fmt=ufp4.SCALE_E4M3_X_FP32)
+    _run(X, axis, cfg, rows=sample)
