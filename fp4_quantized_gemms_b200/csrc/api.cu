@@ -81,7 +81,7 @@ ufp4_status_t check_qtensor(const ufp4_qtensor_t *q) {
     return UFP4_OK;
 }
 
-ufp4_status_t check_pair(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b) {
+ufp4_status_t check_pair(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b, bool same_k) {
     ufp4_status_t s = check_qtensor(a);
     if (s != UFP4_OK) return s;
     s = check_qtensor(b);
@@ -94,7 +94,7 @@ ufp4_status_t check_pair(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b) {
         const uint64_t m = x.hadamard_n == 64 ? ~uint64_t(0) : ((uint64_t(1) << x.hadamard_n) - 1);
         if ((x.rht_sign_mask & m) != (y.rht_sign_mask & m)) return UFP4_ERR_OPERAND_MISMATCH;
     }
-    if (a->k != b->k || a->kpad != b->kpad) return UFP4_ERR_OPERAND_MISMATCH;
+    if (same_k && (a->k != b->k || a->kpad != b->kpad)) return UFP4_ERR_OPERAND_MISMATCH;
     return UFP4_OK;
 }
 
@@ -126,7 +126,9 @@ ufp4_status_t encode_operand_maps(const ufp4_qtensor_t *q, int box_rows, int mod
 ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
                        const ufp4_group_t *groups_dev, int32_t num_groups, float *c, int64_t ldc,
                        int64_t m, int64_t n, void *stream) {
-    ufp4_status_t s = check_pair(a, b);
+    // Grouped problems pick their own K window of each operand (a_col, b_col,
+    // k per group), so only the quantization settings must agree there.
+    ufp4_status_t s = check_pair(a, b, groups_dev == nullptr);
     if (s != UFP4_OK) return s;
     if (c == nullptr && (m > 0 && n > 0)) return UFP4_ERR_INVALID_ARG;
     if (ldc < n || ldc < 1) return UFP4_ERR_INVALID_ARG;

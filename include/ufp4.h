@@ -180,10 +180,18 @@ ufp4_status_t ufp4_gemm_wgrad(const ufp4_qtensor_t *dytq, const ufp4_qtensor_t *
  * on MoE 7.9B / 124B models, [PL] §5 Q2-Q3).  groups_dev: device array of
  * num_groups ufp4_group_t, read by the kernel (the tile schedule is derived on
  * the device, so the table may be written by earlier kernels on the same
- * stream without a host round trip).  All groups share the
- * quantized operands a and b (same constraints as ufp4_gemm_fprop) and the
- * fp32 output c_dev [..][ldc].  Groups must not write overlapping outputs.
- * Errors: INVALID_ARG, ALIGNMENT, OPERAND_MISMATCH, UNSUPPORTED, CUDA. */
+ * stream without a host round trip).  Each group contracts its own window of
+ * the shared quantized operands a and b: rows [a_row, a_row+m) x columns
+ * [a_col, a_col+k) of a and the same for b, so a and b must agree on grid,
+ * block, scale format, hadamard_n and sign mask but not on k.  Typical uses:
+ * per-expert token segments of a routed activation (FPROP / DGRAD, ragged m),
+ * per-expert K windows of a stacked weight quantized ALONG_ROWS (DGRAD), and
+ * per-expert token windows along K (WGRAD, segments zero-padded to 64).
+ * Requirements checked on the device: k, a_col, b_col multiples of 64; a_row,
+ * b_row multiples of 16; a group that violates them is skipped and writes
+ * nothing.  Reads outside an operand return zeros.  The caller guarantees that
+ * every group's output window lies inside c_dev [..][ldc] and that groups do
+ * not overlap.  Errors: INVALID_ARG, ALIGNMENT, OPERAND_MISMATCH, CUDA. */
 ufp4_status_t ufp4_grouped_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
                                 const ufp4_group_t *groups_dev, int32_t num_groups,
                                 float *c_dev, int64_t ldc, void *stream);

@@ -299,6 +299,17 @@ def gemm_tn(a: QTensor, b: QTensor) -> np.ndarray:
     return C
 
 
+def gemm_dequantized(A: np.ndarray, B: np.ndarray, inv_n: float) -> np.ndarray:
+    """C = inv_n * A B^T for dequantized fp64 operands (rows of A, B along K)."""
+    A = np.ascontiguousarray(A, dtype=np.float64)
+    B = np.ascontiguousarray(B, dtype=np.float64)
+    M, K = A.shape
+    N = B.shape[0]
+    C = np.empty((M, N), dtype=np.float64)
+    lib().uo_gemm_tn_f64(_p(A), _p(B), M, N, K, float(inv_n), _p(C), N)
+    return C
+
+
 def gemm_tn_entries(a: QTensor, b: QTensor, ii, jj) -> np.ndarray:
     """Selected entries; ``ii``/``jj`` index the rows held in ``a``/``b``."""
     A = a.dequantize()

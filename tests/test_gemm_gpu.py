@@ -109,7 +109,7 @@ def test_layer_dgrad_wgrad_small(fmt, grid):
 def _sampled(shape: wl.LayerShape, fmt, grid, gemm, n_rows=96, n_cols=96):
     """One GEMM of a full-size layer in the production launch; the oracle
     computes a sampled row x column block of the output."""
-    X, W, dY = wl.layer_inputs(shape, want_dy=gemm != "fprop")
+    X, W, dY = wl.layer_inputs(shape, want_dy=True)
     rng = np.random.default_rng(17)
     if gemm == "fprop":
         a_bits, a_axis, a_cfg = X, C, _cfg(grid=grid, fmt=fmt)
