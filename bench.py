@@ -409,15 +409,15 @@ def cpu_baseline_quick():
     oracle_sample_step(rng, 4, 4)       # warm caches / page in
     flops, secs = 0.0, 0.0
     n = 0
-    while secs < 10.0 and n < 6:
-        f, t = oracle_sample_step(rng)
+    while secs < 10.0 and n < 200:
+        f, t = oracle_sample_step(rng, 32, 32)
         flops += f
         secs += t
         n += 1
     return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
             "kind": "oracle",
-            "sample": (f"{n} sampled steps: 8 output rows of each of the 6 quantized operands "
-                       f"(full K) and an 8x8 block of each GEMM, {secs:.1f} s of CPU work")}
+            "sample": (f"{n} sampled steps: 32 output rows of each of the 6 quantized operands "
+                       f"(full K) and a 32x32 block of each GEMM, {secs:.1f} s of CPU work")}
 
 
 def main():

@@ -105,11 +105,11 @@ ufp4_status_t encode_operand_maps(const ufp4_qtensor_t *q, int box_rows, int mod
                                       static_cast<uint64_t>(q->kpad / 2),
                                       static_cast<uint64_t>(rows_t),
                                       static_cast<uint64_t>(q->kpad / 2), 32,
-                                      static_cast<uint32_t>(box_rows));
+                                      static_cast<uint32_t>(box_rows), CU_TENSOR_MAP_SWIZZLE_32B);
     if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
     const int nblk_stage = 64 / q->cfg.block;
     const uint64_t nblk = static_cast<uint64_t>(q->kpad / q->cfg.block);
-    if (mode == 1) {
+    if (mode != 0) {
         r = encode_tensor_map_2d(scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, q->scales,
                                  static_cast<uint64_t>(q->scale_ld), nblk,
                                  static_cast<uint64_t>(q->scale_ld), static_cast<uint32_t>(box_rows),
@@ -136,7 +136,11 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
     if (groups_dev != nullptr && (reinterpret_cast<uintptr_t>(groups_dev) & 7u))
         return UFP4_ERR_ALIGNMENT;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int mode = a->cfg.scale_fmt == UFP4_SCALE_E4M3_X_FP32 ? 1 : 0;
+    // fp32 block scales: per-block partials (mode 0).  Two-level scales: the
+    // CTA-pair kernel (256 x 256 tiles, mode 2), or one CTA per 128 x 256 tile
+    // (mode 1) when a single problem has at most 128 rows.
+    int mode = 0;
+    if (a->cfg.scale_fmt == UFP4_SCALE_E4M3_X_FP32) mode = (groups_dev != nullptr || m > 128) ? 2 : 1;
     if (groups_dev == nullptr) {
         if (m == 0 || n == 0) return UFP4_OK;
         if (a->kpad == 0) {
@@ -151,7 +155,7 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
 
     GemmArgs args;
     memset(&args, 0, sizeof(args));
-    const int bn = mode == 1 ? 256 : 128;
+    const int bn = mode == 1 ? 256 : 128;   // B rows staged per CTA
     s = encode_operand_maps(a, 128, mode, &args.tm_a_codes, &args.tm_a_scales);
     if (s != UFP4_OK) return s;
     s = encode_operand_maps(b, bn, mode, &args.tm_b_codes, &args.tm_b_scales);
@@ -186,7 +190,7 @@ ufp4_status_t check_input(const void *x, int64_t rows, int64_t cols, int64_t ld,
 
 CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
                               uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                              uint32_t box_inner, uint32_t box_outer) {
+                              uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
     PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
     if (fn == nullptr) return CUDA_ERROR_NOT_INITIALIZED;
     const cuuint64_t dims[2] = {inner, outer};
@@ -194,7 +198,7 @@ CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, const
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estride[2] = {1, 1};
     return fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estride,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 

@@ -31,6 +31,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 #define UFP4_PIPELINE_KERNELS 1
 #include "ufp4_device.cuh"
@@ -48,27 +49,52 @@ constexpr int kOpRow = BK * 2;     // fp16 bytes per row per stage (= 128)
 template <int MODE>
 struct Cfg;
 
+// mode 1: two-level scales folded into fp16 operands, one CTA per 128 x 256 tile
 template <>
 struct Cfg<1> {
-    static constexpr int BN = 256;
-    static constexpr int NT = 8;   // transform warps
-    static constexpr int NE = 4;   // epilogue warps
-    static constexpr int NC = 4;   // code ring slots
-    static constexpr int NO = 3;   // fp16 operand ring slots
-    static constexpr int NS = 0;   // separate scale ring slots
-    static constexpr int NP = 2;   // TMEM accumulators (BN columns each)
+    static constexpr int BN = 256;  // B rows staged per CTA
+    static constexpr int TM = 128;  // output tile rows
+    static constexpr int TN = 256;  // output tile columns (= accumulator columns)
+    static constexpr int CG = 1;    // CTAs per MMA
+    static constexpr int NT = 12;   // transform warps (one operand row per thread)
+    static constexpr int NE = 4;    // epilogue warps
+    static constexpr int NC = 4;    // code ring slots
+    static constexpr int NO = 3;    // fp16 operand ring slots
+    static constexpr int NS = 0;    // separate scale ring slots
+    static constexpr int NP = 2;    // TMEM accumulators
     static constexpr int kScaleElt = 1;
 };
 
+// mode 2: mode 1 on a CTA pair (cta_group::2): a 256 x 256 tile, each CTA
+// stages 128 rows of A and 128 rows of B and holds 128 accumulator rows.
+template <>
+struct Cfg<2> {
+    static constexpr int BN = 128;
+    static constexpr int TM = 256;
+    static constexpr int TN = 256;
+    static constexpr int CG = 2;
+    static constexpr int NT = 8;
+    static constexpr int NE = 4;
+    static constexpr int NC = 4;
+    static constexpr int NO = 4;
+    static constexpr int NS = 0;
+    static constexpr int NP = 2;
+    static constexpr int kScaleElt = 1;
+};
+
+// mode 0: fp32 block scales, per-block partial products in TMEM
 template <>
 struct Cfg<0> {
     static constexpr int BN = 128;
+    static constexpr int TM = 128;
+    static constexpr int TN = 128;
+    static constexpr int CG = 1;
     static constexpr int NT = 2;
     static constexpr int NE = 8;
     static constexpr int NC = 4;
     static constexpr int NO = 3;
     static constexpr int NS = 4;
-    static constexpr int NP = 4;   // TMEM partial buffers (BN columns each)
+    static constexpr int NP = 4;    // TMEM partial buffers
     static constexpr int kScaleElt = 4;
 };
 
@@ -83,7 +109,9 @@ struct Layout {
     // scales per stage for the smallest block (16): BK/16 = 4 blocks
     static constexpr int kScA = BM * (BK / 16) * C::kScaleElt;
     static constexpr int kScB = BN * (BK / 16) * C::kScaleElt;
-    static constexpr int kCodeSlot = MODE == 1 ? kCodeA + kCodeB + kScA + kScB : kCodeA + kCodeB;
+    // code slots start on 1024-byte boundaries (the 32-byte TMA swizzle)
+    static constexpr int kCodeSlot =
+        ((MODE != 0 ? kCodeA + kCodeB + kScA + kScB : kCodeA + kCodeB) + 1023) / 1024 * 1024;
     static constexpr int kScSlot = MODE == 0 ? kScA + kScB : 0;
 
     static constexpr int off_op = 0;
@@ -98,7 +126,10 @@ struct Layout {
     static constexpr int kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
     static constexpr int kThreads = 32 * (2 + C::NT + C::NE);
     static constexpr int kTmemCols = 512;
-    static_assert(C::NP * BN <= kTmemCols, "TMEM budget");
+    static constexpr int kAccCols = MODE == 0 ? BN : C::TN;
+    static_assert(C::NP * kAccCols <= kTmemCols, "TMEM budget");
+    static_assert(BM + BN <= C::NT * 32 * 4, "transform rows");
+    static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
 struct Tile {
@@ -113,10 +144,10 @@ __device__ __forceinline__ bool group_ok(const GemmGroup &g) {
            g.b_row >= 0 && g.c_row >= 0 && g.c_col >= 0;
 }
 
-template <int BN>
+template <int TM, int TN>
 __device__ __forceinline__ int64_t tiles_of(const GemmGroup &g) {
     if (!group_ok(g)) return 0;
-    return ((g.m + BM - 1) / BM) * ((g.n + BN - 1) / BN);
+    return ((g.m + TM - 1) / TM) * ((g.n + TN - 1) / TN);
 }
 
 __device__ __forceinline__ GemmGroup load_group(const GemmArgs &a, int i) {
@@ -135,27 +166,27 @@ __device__ __forceinline__ GemmGroup load_group(const GemmArgs &a, int i) {
     return g;
 }
 
-template <int BN>
+template <int TM, int TN>
 __device__ int64_t total_tiles(const GemmArgs &a) {
     const int ng = a.groups == nullptr ? 1 : a.num_groups;
     int64_t t = 0;
-    for (int i = 0; i < ng; ++i) t += tiles_of<BN>(load_group(a, i));
+    for (int i = 0; i < ng; ++i) t += tiles_of<TM, TN>(load_group(a, i));
     return t;
 }
 
 // Tile t of the concatenated schedule (groups in order, M fastest inside).
-template <int BN>
+template <int TM, int TN>
 __device__ Tile get_tile(const GemmArgs &a, int64_t t) {
     const int ng = a.groups == nullptr ? 1 : a.num_groups;
     Tile tl;
     for (int i = 0; i < ng; ++i) {
         const GemmGroup g = load_group(a, i);
-        const int64_t nt = tiles_of<BN>(g);
+        const int64_t nt = tiles_of<TM, TN>(g);
         if (t < nt) {
-            const int64_t mt = (g.m + BM - 1) / BM;
+            const int64_t mt = (g.m + TM - 1) / TM;
             tl.g = g;
-            tl.m0 = (t % mt) * BM;
-            tl.n0 = (t / mt) * BN;
+            tl.m0 = (t % mt) * TM;
+            tl.n0 = (t / mt) * TN;
             tl.nks = static_cast<int>(g.k / BK);
             return tl;
         }
@@ -172,41 +203,74 @@ __device__ Tile get_tile(const GemmArgs &a, int64_t t) {
 // index i).  Output word i (i = 0..3) holds the fp16 pair (code i, code i+4):
 // the same K permutation inside every 8-element chunk of both operands, which
 // leaves every dot product (and every 16-block) unchanged.
-__device__ __forceinline__ uint32_t sign_pair(uint32_t t) { return (t << 12) & 0x80008000u; }
+//
+// E1M2 carries the magnitude index k (the level is k/4; the 1/4 moves to the
+// epilogue); E2M1 carries the level itself.  With a block scale e (an E4M3
+// value, fp16-exact) the pair is multiplied in: e*k <= 7*448 and e*lvl <= 6*448
+// have at most 7 significant bits and stay in fp16's normal range, so every
+// operand value is exact.
 
-// E1M2: magnitude index k itself (the level is k/4; the 1/4 goes to the scale).
-__device__ __forceinline__ void expand_e1m2(uint32_t w, uint32_t (&o)[4]) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t t = w >> (4 * i);
-        const uint32_t mag = (t & 0x00070007u) | 0x64006400u;   // fp16 1024 + k
-        const __half2 h = __hsub2(*reinterpret_cast<const __half2 *>(&mag),
-                                  __half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
-        o[i] = *reinterpret_cast<const uint32_t *>(&h) ^ sign_pair(t);
-    }
+// Sign bits of codes i and i+4 (nibble bit 3) moved to fp16 bits 15 and 31.
+template <int I>
+__device__ __forceinline__ uint32_t sign_pair(uint32_t w) {
+    return (w << (12 - 4 * I)) & 0x80008000u;
 }
 
-// E2M1: fp16 of the level {0,.5,1,1.5,2,3,4,6}; only the high byte is nonzero.
-__device__ __forceinline__ void expand_e2m1(uint32_t w, uint32_t (&o)[4]) {
-    const uint32_t m = w & 0x77777777u;
-    const uint32_t lo = __byte_perm(0x3E3C3800u, 0x46444240u, m);
-    const uint32_t hi = __byte_perm(0x3E3C3800u, 0x46444240u, m >> 16);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t sel = ((4u + i) << 12) | (static_cast<uint32_t>(i) << 4);
-        o[i] = (__byte_perm(lo, hi, sel) & 0xFF00FF00u) ^ sign_pair(w >> (4 * i));
-    }
+// k of codes I and I+4 placed in mantissa bits 7..9 of fp16 8.0 (0x4800):
+// the pair (8 + k_I, 8 + k_{I+4}).
+template <int I>
+__device__ __forceinline__ uint32_t eight_plus_k(uint32_t w) {
+    const uint32_t t = (I <= 1) ? (w << (7 - 4 * I)) : (w >> (4 * I - 7));
+    return (t & 0x03800380u) | 0x48004800u;
 }
 
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
+
+// Unscaled expansion (fp32 block-scale mode): k (E1M2) or lvl (E2M1).
 template <int GRID>
-__device__ __forceinline__ void expand(uint32_t w, uint32_t (&o)[4]) {
-    if (GRID == 0) expand_e1m2(w, o);
-    else expand_e2m1(w, o);
+__device__ __forceinline__ void expand_unscaled(uint32_t w, uint32_t (&o)[4]) {
+    if (GRID == 0) {
+        const __half2 eight = __half2(__ushort_as_half(0x4800), __ushort_as_half(0x4800));
+        o[0] = h2_bits(__hsub2(bits_h2(eight_plus_k<0>(w)), eight)) ^ sign_pair<0>(w);
+        o[1] = h2_bits(__hsub2(bits_h2(eight_plus_k<1>(w)), eight)) ^ sign_pair<1>(w);
+        o[2] = h2_bits(__hsub2(bits_h2(eight_plus_k<2>(w)), eight)) ^ sign_pair<2>(w);
+        o[3] = h2_bits(__hsub2(bits_h2(eight_plus_k<3>(w)), eight)) ^ sign_pair<3>(w);
+    } else {
+        // fp16 high byte of {0,.5,1,1.5,2,3,4,6}; the low byte is always 0.
+        const uint32_t m = w & 0x77777777u;
+        const uint32_t lo = __byte_perm(0x3E3C3800u, 0x46444240u, m);
+        const uint32_t hi = __byte_perm(0x3E3C3800u, 0x46444240u, m >> 16);
+        o[0] = (__byte_perm(lo, hi, 0x4000u) & 0xFF00FF00u) ^ sign_pair<0>(w);
+        o[1] = (__byte_perm(lo, hi, 0x5010u) & 0xFF00FF00u) ^ sign_pair<1>(w);
+        o[2] = (__byte_perm(lo, hi, 0x6020u) & 0xFF00FF00u) ^ sign_pair<2>(w);
+        o[3] = (__byte_perm(lo, hi, 0x7030u) & 0xFF00FF00u) ^ sign_pair<3>(w);
+    }
 }
 
-__device__ __forceinline__ uint32_t hmul2_bits(uint32_t x, __half2 s) {
-    const __half2 r = __hmul2(*reinterpret_cast<const __half2 *>(&x), s);
-    return *reinterpret_cast<const uint32_t *>(&r);
+// Scaled expansion (two-level mode): e*k (E1M2) via one fma per pair,
+// (8 + k) * e - 8 * e = k * e (exact), or e*lvl (E2M1).
+template <int GRID>
+__device__ __forceinline__ void expand_scaled(uint32_t w, __half2 e2, __half2 m8e2, uint32_t (&o)[4]) {
+    if (GRID == 0) {
+        o[0] = h2_bits(__hfma2(bits_h2(eight_plus_k<0>(w)), e2, m8e2)) ^ sign_pair<0>(w);
+        o[1] = h2_bits(__hfma2(bits_h2(eight_plus_k<1>(w)), e2, m8e2)) ^ sign_pair<1>(w);
+        o[2] = h2_bits(__hfma2(bits_h2(eight_plus_k<2>(w)), e2, m8e2)) ^ sign_pair<2>(w);
+        o[3] = h2_bits(__hfma2(bits_h2(eight_plus_k<3>(w)), e2, m8e2)) ^ sign_pair<3>(w);
+    } else {
+        uint32_t u[4];
+        expand_unscaled<1>(w, u);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) o[q] = h2_bits(__hmul2(bits_h2(u[q]), e2));
+    }
+}
+
+// E4M3 byte -> fp16 pair (e, e), exact (hardware conversion).
+__device__ __forceinline__ __half2 e4m3_pair(uint32_t byte) {
+    const uint16_t two = static_cast<uint16_t>(byte | (byte << 8));
+    uint32_t out;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(out) : "h"(two));
+    return bits_h2(out);
 }
 
 // ---------------------------------------------------------------------------
@@ -216,6 +280,10 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
     using C = Cfg<MODE>;
     using Lay = Layout<MODE>;
     constexpr int BN = C::BN;
+    constexpr int TM = C::TM;
+    constexpr int TN = C::TN;
+    constexpr bool kPair = C::CG == 2;
+    constexpr bool kFolded = MODE != 0;   // two-level scales folded into the operands
     constexpr int NSr = C::NS > 0 ? C::NS : 1;   // scale-ring modulus (mode 0 only)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -238,15 +306,20 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
     auto op_b = [&](int s) { return op_a(s) + Lay::kOpA; };
     auto code_a = [&](int s) { return smem + Lay::off_code + s * Lay::kCodeSlot; };
     auto code_b = [&](int s) { return code_a(s) + Lay::kCodeA; };
-    // mode 1: scales ride in the code slot; mode 0: separate scale ring
+    // folded modes: scales ride in the code slot; mode 0: separate scale ring
     auto sc_a = [&](int s) {
-        return MODE == 1 ? code_b(s) + Lay::kCodeB : smem + Lay::off_sc + s * Lay::kScSlot;
+        return kFolded ? code_b(s) + Lay::kCodeB : smem + Lay::off_sc + s * Lay::kScSlot;
     };
     auto sc_b = [&](int s) { return sc_a(s) + Lay::kScA; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int nblk_stage = BK / args.block;
+    // CTA pair: rank 0 issues the MMAs; rank r stages rows [128 r, 128 r + 128)
+    // of both the A tile and the B tile and holds accumulator rows 128 r...
+    const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+    const int64_t unit = kPair ? (blockIdx.x >> 1) : blockIdx.x;
+    const int64_t nunits = kPair ? (gridDim.x >> 1) : gridDim.x;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::NC; ++i) {
@@ -254,7 +327,7 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
             mbar_init(&code_empty[i], C::NT);
         }
         for (int i = 0; i < C::NO; ++i) {
-            mbar_init(&op_full[i], C::NT);
+            mbar_init(&op_full[i], C::NT * C::CG);
             mbar_init(&op_empty[i], 1);
         }
         for (int i = 0; i < C::NS; ++i) {
@@ -263,7 +336,7 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
         }
         for (int i = 0; i < C::NP; ++i) {
             mbar_init(&p_full[i], 1);
-            mbar_init(&p_empty[i], C::NE);
+            mbar_init(&p_empty[i], C::NE * C::CG);
         }
         mbar_init(drain, 1);
         *abort_flag = 0u;
@@ -275,22 +348,26 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
         tma_prefetch_desc(&args.tm_a_scales);
         tma_prefetch_desc(&args.tm_b_scales);
     }
-    if (warp == 1) tmem_alloc(tmem_slot, Lay::kTmemCols);
+    if (warp == 1) {
+        if constexpr (kPair) tmem_alloc_pair(tmem_slot, Lay::kTmemCols);
+        else tmem_alloc(tmem_slot, Lay::kTmemCols);
+    }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (kPair) cluster_sync();
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int64_t ntiles = total_tiles<BN>(args);
+    const int64_t ntiles = total_tiles<TM, TN>(args);
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             uint32_t it = 0, sit = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                const Tile tl = get_tile<BN>(args, t);
-                const int32_t arow = static_cast<int32_t>(tl.g.a_row + tl.m0);
-                const int32_t brow = static_cast<int32_t>(tl.g.b_row + tl.n0);
+            for (int64_t t = unit; t < ntiles && ok; t += nunits) {
+                const Tile tl = get_tile<TM, TN>(args, t);
+                const int32_t arow = static_cast<int32_t>(tl.g.a_row + tl.m0 + 128 * rank);
+                const int32_t brow = static_cast<int32_t>(tl.g.b_row + tl.n0 + BN * rank);
                 for (int ks = 0; ks < tl.nks; ++ks, ++it) {
                     const int s = it % C::NC;
                     const uint32_t use = it / C::NC;
@@ -301,11 +378,11 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
                     const int32_t acol = static_cast<int32_t>(tl.g.a_col + ks * BK);
                     const int32_t bcol = static_cast<int32_t>(tl.g.b_col + ks * BK);
                     uint32_t bytes = Lay::kCodeA + Lay::kCodeB;
-                    if (MODE == 1) bytes += (BM + BN) * nblk_stage;
+                    if (kFolded) bytes += (BM + BN) * nblk_stage;
                     mbar_arrive_expect_tx(&code_full[s], bytes);
                     tma_load_2d(code_a(s), &args.tm_a_codes, &code_full[s], acol / 2, arow);
                     tma_load_2d(code_b(s), &args.tm_b_codes, &code_full[s], bcol / 2, brow);
-                    if (MODE == 1) {
+                    if (kFolded) {
                         tma_load_2d(sc_a(s), &args.tm_a_scales, &code_full[s], arow, acol / args.block);
                         tma_load_2d(sc_b(s), &args.tm_b_scales, &code_full[s], brow, bcol / args.block);
                     } else {
@@ -344,44 +421,51 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ UMMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = umma_idesc_f16_f32(BM, BN);
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = umma_idesc_f16_f32(kPair ? 256 : BM, Lay::kAccCols);
             uint32_t it = 0, pq = 0, tcount = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
-                const Tile tl = get_tile<BN>(args, t);
+            auto wait = [&](uint64_t *bar, uint32_t parity) {
+                return kPair ? mbar_wait_cluster(bar, parity, kErrTimeoutMma, abort_flag)
+                             : mbar_wait(bar, parity, kErrTimeoutMma, abort_flag);
+            };
+            for (int64_t t = unit; t < ntiles && ok; t += nunits, ++tcount) {
+                const Tile tl = get_tile<TM, TN>(args, t);
                 uint32_t acc_col = 0;
-                if (MODE == 1) {
+                if (kFolded) {
                     const int b = tcount & 1;
-                    if (!mbar_wait(&p_empty[b], ((tcount >> 1) & 1) ^ 1, kErrTimeoutMma, abort_flag)) {
+                    if (!wait(&p_empty[b], ((tcount >> 1) & 1) ^ 1)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    acc_col = b * BN;
+                    acc_col = b * Lay::kAccCols;
                 }
                 for (int ks = 0; ks < tl.nks && ok; ++ks, ++it) {
                     const int s = it % C::NO;
-                    if (!mbar_wait(&op_full[s], (it / C::NO) & 1, kErrTimeoutMma, abort_flag)) {
+                    if (!wait(&op_full[s], (it / C::NO) & 1)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t a0 = smem_addr(op_a(s));
                     const uint32_t b0 = smem_addr(op_b(s));
-                    if (MODE == 1) {
+                    if (kFolded) {
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk) {
-                            umma_f16(tmem_base + acc_col, umma_desc_sw128(a0 + kk * 32),
-                                     umma_desc_sw128(b0 + kk * 32), idesc,
-                                     (ks > 0 || kk > 0) ? 1u : 0u);
+                            const uint64_t ad = umma_desc_sw128(a0 + kk * 32);
+                            const uint64_t bd = umma_desc_sw128(b0 + kk * 32);
+                            const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
+                            if constexpr (kPair) umma_f16_pair(tmem_base + acc_col, ad, bd, idesc, acc);
+                            else umma_f16(tmem_base + acc_col, ad, bd, idesc, acc);
                         }
+                        if constexpr (kPair) umma_commit_pair_mc(&op_empty[s], 0x3);
+                        else umma_commit(&op_empty[s]);
                     } else {
                         const int slices = args.block / 16;
                         for (int bi = 0; bi < nblk_stage; ++bi, ++pq) {
                             const int p = pq % C::NP;
-                            if (!mbar_wait(&p_empty[p], ((pq / C::NP) & 1) ^ 1, kErrTimeoutMma,
-                                           abort_flag)) {
+                            if (!wait(&p_empty[p], ((pq / C::NP) & 1) ^ 1)) {
                                 ok = false;
                                 break;
                             }
@@ -393,66 +477,85 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
                             }
                             umma_commit(&p_full[p]);
                         }
+                        umma_commit(&op_empty[s]);
                     }
-                    umma_commit(&op_empty[s]);
                 }
-                if (MODE == 1 && ok) umma_commit(&p_full[tcount & 1]);
+                if (kFolded && ok) {
+                    if constexpr (kPair) umma_commit_pair_mc(&p_full[tcount & 1], 0x3);
+                    else umma_commit(&p_full[tcount & 1]);
+                }
             }
             // Drain: every MMA issued by this thread completes before TMEM is freed.
-            umma_commit(drain);
+            if constexpr (kPair) umma_commit_pair(drain);
+            else umma_commit(drain);
             uint32_t dummy = 0;
             mbar_wait(drain, 0, kErrTimeoutDrain, reinterpret_cast<volatile uint32_t *>(&dummy));
         }
     } else if (warp < 2 + C::NT) {
         // ------------------------------------------------------------ transform
+        // One operand row (64 codes, 32 bytes) per thread per stage.  The code
+        // tiles arrive with the 32-byte TMA swizzle: the two 16-byte halves of
+        // row r are swapped when bit 2 of r is set, so the lanes of a quarter
+        // warp read distinct banks.
         const int tt = threadIdx.x - 64;
-        constexpr int kUnits = (BM + BN) * 2;   // (row, 32-code half)
-        const __half2 unit2 = __float2half2_rn(GRID == 0 ? 0.25f : 1.0f);
+        constexpr int kRows = BM + BN;
+        const int blk_shift = args.block == 16 ? 4 : 5;
         uint32_t it = 0;
         bool ok = true;
-        for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const Tile tl = get_tile<BN>(args, t);
+        for (int64_t t = unit; t < ntiles && ok; t += nunits) {
+            const Tile tl = get_tile<TM, TN>(args, t);
             for (int ks = 0; ks < tl.nks; ++ks, ++it) {
                 const int cs = it % C::NC;
                 const int os = it % C::NO;
                 if (!warp_wait(&code_full[cs], (it / C::NC) & 1, kErrTimeoutTransform, abort_flag) ||
-                    !warp_wait(&op_empty[os], ((it / C::NO) & 1) ^ 1, kErrTimeoutTransform,
-                               abort_flag)) {
+                    !warp_wait<kPair>(&op_empty[os], ((it / C::NO) & 1) ^ 1, kErrTimeoutTransform,
+                                      abort_flag)) {
                     ok = false;
                     break;
                 }
                 const uint8_t *ca = code_a(cs);
                 const uint8_t *cb = code_b(cs);
+                const uint8_t *sa = sc_a(cs);
+                const uint8_t *sb = sc_b(cs);
                 uint8_t *oa = op_a(os);
                 uint8_t *ob = op_b(os);
-                for (int u = tt; u < kUnits; u += C::NT * 32) {
-                    const int row = u >> 1;
-                    const int half = u & 1;
+#pragma unroll 1
+                for (int row = tt; row < kRows; row += C::NT * 32) {
                     const bool isA = row < BM;
                     const int r = isA ? row : row - BM;
-                    const uint4 w =
-                        *reinterpret_cast<const uint4 *>((isA ? ca : cb) + r * kCodeRow + half * 16);
-                    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-                    uint8_t *dst = isA ? oa : ob;
+                    const uint8_t *src = (isA ? ca : cb) + r * kCodeRow;
+                    const int flip = (r >> 2) & 1;
+                    const uint4 h0 = *reinterpret_cast<const uint4 *>(src + (flip << 4));
+                    const uint4 h1 = *reinterpret_cast<const uint4 *>(src + ((flip ^ 1) << 4));
+                    const uint32_t words[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+                    uint8_t *dst = (isA ? oa : ob) + r * 128;
+                    const uint32_t sw = static_cast<uint32_t>(r & 7);
+                    __half2 e2[4], n2[4];
+                    if (kFolded) {
+                        const uint8_t *sc = (isA ? sa : sb) + r;
+                        const int ld = isA ? BM : BN;
+                        const __half2 m8 = __float2half2_rn(-8.0f);
 #pragma unroll
-                    for (int wi = 0; wi < 4; ++wi) {
-                        uint32_t o[4];
-                        expand<GRID>(words[wi], o);
-                        if (MODE == 1) {
-                            const int blk = (half * 32 + wi * 8) / args.block;
-                            const uint8_t e8 = isA ? sc_a(cs)[blk * BM + r] : sc_b(cs)[blk * BN + r];
-                            const __half2 s2 = __hmul2(__float2half2_rn(e4m3_to_f32(e8)), unit2);
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) o[q] = hmul2_bits(o[q], s2);
+                        for (int b = 0; b < 4; ++b) {
+                            const int blk = (16 * b) >> blk_shift;
+                            e2[b] = e4m3_pair(sc[blk * ld]);
+                            n2[b] = __hmul2(e2[b], m8);
                         }
-                        *reinterpret_cast<uint4 *>(dst + sw128_offset(r, half * 4 + wi)) =
+                    }
+#pragma unroll
+                    for (int wi = 0; wi < 8; ++wi) {
+                        uint32_t o[4];
+                        if (kFolded) expand_scaled<GRID>(words[wi], e2[wi >> 1], n2[wi >> 1], o);
+                        else expand_unscaled<GRID>(words[wi], o);
+                        *reinterpret_cast<uint4 *>(dst + ((static_cast<uint32_t>(wi) ^ sw) << 4)) =
                             make_uint4(o[0], o[1], o[2], o[3]);
                     }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive(&op_full[os]);
+                    if (kPair && rank != 0) mbar_arrive_remote(&op_full[os], 0);
+                    else mbar_arrive(&op_full[os]);
                     mbar_arrive(&code_empty[cs]);
                 }
             }
@@ -463,26 +566,32 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
         const int q = warp & 3;               // TMEM lane quarter of this warp
         const int row_in_tile = 32 * q + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-        if (MODE == 1) {
-            const float mult = __fmul_rn(__fmul_rn(*args.a_S, *args.b_S), args.inv_n);
+        if (kFolded) {
+            // E1M2 operands carry k = 4 * level on both sides: 1/16 (exact).
+            const float mult = __fmul_rn(__fmul_rn(*args.a_S, *args.b_S),
+                                         args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f));
             uint32_t tcount = 0;
-            for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
-                const Tile tl = get_tile<BN>(args, t);
+            for (int64_t t = unit; t < ntiles; t += nunits, ++tcount) {
+                const Tile tl = get_tile<TM, TN>(args, t);
                 const int b = tcount & 1;
-                if (!warp_wait(&p_full[b], (tcount >> 1) & 1, kErrTimeoutEpilogue, abort_flag)) break;
+                if (!warp_wait<kPair>(&p_full[b], (tcount >> 1) & 1, kErrTimeoutEpilogue, abort_flag))
+                    break;
                 tc_fence_after();
-                const int64_t row = tl.m0 + row_in_tile;
+                const int64_t row = tl.m0 + 128 * rank + row_in_tile;
                 const bool row_ok = row < tl.g.m;
                 float *crow = args.c + (tl.g.c_row + row) * args.ldc + tl.g.c_col + tl.n0;
 #pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
+                for (int c = 0; c < TN / 32; ++c) {
                     uint32_t r[32];
-                    tmem_ld_32x32b_x32(tmem_base + b * BN + 32 * c + lane_addr, r);
+                    tmem_ld_32x32b_x32(tmem_base + b * Lay::kAccCols + 32 * c + lane_addr, r);
                     tmem_wait_ld();
-                    if (c == BN / 32 - 1) {
+                    if (c == TN / 32 - 1) {
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&p_empty[b]);
+                        if (lane == 0) {
+                            if (kPair && rank != 0) mbar_arrive_remote(&p_empty[b], 0);
+                            else mbar_arrive(&p_empty[b]);
+                        }
                     }
                     if (!row_ok) continue;
                     const int64_t col0 = tl.n0 + 32 * c;
@@ -510,8 +619,8 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
             const float mult = args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f);
             uint32_t it = 0, pq = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                const Tile tl = get_tile<BN>(args, t);
+            for (int64_t t = unit; t < ntiles && ok; t += nunits) {
+                const Tile tl = get_tile<TM, TN>(args, t);
                 float acc[64];
 #pragma unroll
                 for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
@@ -581,16 +690,358 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
     }
 
     tc_fence_before();
+    if constexpr (kPair) cluster_sync();
+    else __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        if constexpr (kPair) tmem_dealloc_pair(tmem_base, Lay::kTmemCols);
+        else tmem_dealloc(tmem_base, Lay::kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Native block-scaled FP4 path for two-level scales (mode 3).
+//
+// kind::mxf4nvf4 multiplies E2M1 operands scaled per 16 elements by UE4M3
+// factors, which is exactly an E2M1 operand under the two-level scales (the
+// block scale e_b is a positive E4M3 byte).  E2M1 codes go from TMA straight
+// to the tensor core.  An E1M2 code k splits exactly into two E2M1 values,
+// k = hi + lo with hi in {0,1,2,3,4,4,6,6}[k] and lo = 1 for k in {5,7}, so
+// sum_k k_a k_b e_a e_b = sum over the four plane products, each one native
+// FP4 MMA with the same scale factors.  The split is a per-byte bit
+// operation done in place in shared memory (hi overwrites the code bytes).
+//
+// Tile 128 x 256, 128 K elements (64 bytes of codes per row, 64-byte TMA
+// swizzle) per stage.  A transform group permutes the block-major E4M3 bytes
+// into the 128-row x 4-scale atoms that tcgen05.cp moves to TMEM.
+template <int GRID>
+struct Fp4Cfg {
+    static constexpr int BN = 256;
+    static constexpr int BKE = 128;            // K elements per stage
+    static constexpr int kRow = 64;            // code bytes per row per stage
+    static constexpr int NSTAGE = GRID == 0 ? 3 : 5;
+    static constexpr int NT = 4;               // transform warps
+    static constexpr int NE = 4;               // epilogue warps
+    static constexpr int kCodesA = BM * kRow;
+    static constexpr int kCodesB = BN * kRow;
+    static constexpr int kLoA = GRID == 0 ? kCodesA : 0;
+    static constexpr int kLoB = GRID == 0 ? kCodesB : 0;
+    static constexpr int kRawA = BM * (BKE / 16);
+    static constexpr int kRawB = BN * (BKE / 16);
+    static constexpr int kSfA = 2 * 512;        // 2 K-steps x 1 row tile
+    static constexpr int kSfB = 2 * 2 * 512;    // 2 K-steps x 2 row tiles
+    static constexpr int o_codes_a = 0;
+    static constexpr int o_codes_b = o_codes_a + kCodesA;
+    static constexpr int o_lo_a = o_codes_b + kCodesB;
+    static constexpr int o_lo_b = o_lo_a + kLoA;
+    static constexpr int o_raw_a = o_lo_b + kLoB;
+    static constexpr int o_raw_b = o_raw_a + kRawA;
+    static constexpr int o_sf_a = o_raw_b + kRawB;
+    static constexpr int o_sf_b = o_sf_a + kSfA;
+    static constexpr int kStage = (o_sf_b + kSfB + 1023) / 1024 * 1024;
+    static constexpr int o_bar = NSTAGE * kStage;
+    // barriers: full, ready, empty per stage; acc_full, acc_empty, drain
+    static constexpr int kNumBars = 3 * NSTAGE + 3;
+    static constexpr int o_misc = o_bar + kNumBars * 8;
+    static constexpr int kAlloc = o_misc + 64 + 1024;
+    static constexpr int kThreads = 32 * (2 + NT + NE);
+    static constexpr int kSfColsPerStage = 24;  // SFA 2 x 4, SFB 2 x 8
+    static constexpr int kAccCols = 256;
+    static_assert(kAccCols + NSTAGE * kSfColsPerStage <= 512, "TMEM budget");
+    static_assert(kAlloc <= 232448, "shared memory budget");
+};
+
+// hi / lo E2M1 planes of 8 E1M2 codes (see above); signs copied to both.
+__device__ __forceinline__ void split_e1m2(uint32_t w, uint32_t &hi, uint32_t &lo) {
+    const uint32_t M = 0x11111111u;
+    const uint32_t b0 = w & M, b1 = (w >> 1) & M, b2 = (w >> 2) & M, s = w & 0x88888888u;
+    const uint32_t h2 = b2 | b1;
+    const uint32_t h1 = b2 | (~b1 & b0);
+    const uint32_t h0 = b1 & (b0 | b2);
+    hi = s | (h2 << 2) | (h1 << 1) | h0;
+    lo = s | ((b2 & b0) << 1);
+}
+
+template <int GRID>
+__global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
+    gemm_fp4_kernel(const __grid_constant__ GemmArgs args) {
+    using C = Fp4Cfg<GRID>;
+    constexpr int BN = C::BN;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::o_bar);
+    uint64_t *ready = full + C::NSTAGE;
+    uint64_t *empty = ready + C::NSTAGE;
+    uint64_t *acc_full = empty + C::NSTAGE;
+    uint64_t *acc_empty = acc_full + 1;
+    uint64_t *drain = acc_empty + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::o_misc);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::o_misc + 4);
+    auto stage = [&](int s) { return smem + s * C::kStage; };
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int blk = args.block;                       // 16 or 32
+    const int nraw = C::BKE / blk;                    // raw scale rows per stage
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::NSTAGE; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&ready[i], C::NT);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, C::NE);
+        mbar_init(drain, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&args.tm_a_codes);
+        tma_prefetch_desc(&args.tm_b_codes);
+        tma_prefetch_desc(&args.tm_a_scales);
+        tma_prefetch_desc(&args.tm_b_scales);
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int64_t ntiles = total_tiles<BM, BN>(args);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                const Tile tl = get_tile<BM, BN>(args, t);
+                const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
+                const int32_t arow = static_cast<int32_t>(tl.g.a_row + tl.m0);
+                const int32_t brow = static_cast<int32_t>(tl.g.b_row + tl.n0);
+                for (int ks = 0; ks < nks; ++ks, ++it) {
+                    const int s = it % C::NSTAGE;
+                    if (!mbar_wait(&empty[s], ((it / C::NSTAGE) & 1) ^ 1, kErrTimeoutProducer,
+                                   abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const int32_t acol = static_cast<int32_t>(tl.g.a_col + ks * C::BKE);
+                    const int32_t bcol = static_cast<int32_t>(tl.g.b_col + ks * C::BKE);
+                    uint8_t *st = stage(s);
+                    mbar_arrive_expect_tx(&full[s], C::kCodesA + C::kCodesB + (BM + BN) * nraw);
+                    tma_load_2d(st + C::o_codes_a, &args.tm_a_codes, &full[s], acol / 2, arow);
+                    tma_load_2d(st + C::o_codes_b, &args.tm_b_codes, &full[s], bcol / 2, brow);
+                    tma_load_2d(st + C::o_raw_a, &args.tm_a_scales, &full[s], arow, acol / blk);
+                    tma_load_2d(st + C::o_raw_b, &args.tm_b_scales, &full[s], brow, bcol / blk);
+                }
+            }
+            for (int s = 0; s < C::NSTAGE; ++s) {
+                if (it > static_cast<uint32_t>(s)) {
+                    const uint32_t last = (it - 1 - s) / C::NSTAGE * C::NSTAGE + s;
+                    uint32_t dummy = 0;
+                    mbar_wait(&full[s], (last / C::NSTAGE) & 1, kErrTimeoutDrain,
+                              reinterpret_cast<volatile uint32_t *>(&dummy));
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ UMMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_fp4_bs(BM, BN);
+            uint32_t it = 0, tcount = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
+                const Tile tl = get_tile<BM, BN>(args, t);
+                const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
+                if (!mbar_wait(acc_empty, (tcount & 1) ^ 1, kErrTimeoutMma, abort_flag)) break;
+                tc_fence_after();
+                bool first = true;
+                for (int ks = 0; ks < nks && ok; ++ks, ++it) {
+                    const int s = it % C::NSTAGE;
+                    if (!mbar_wait(&ready[s], (it / C::NSTAGE) & 1, kErrTimeoutMma, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    uint8_t *st = stage(s);
+                    const uint32_t sf0 = tmem_base + C::kAccCols + s * C::kSfColsPerStage;
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        tmem_cp_32x128b_x4(sf0 + 4 * j, sf_atom_desc(smem_addr(st + C::o_sf_a + 512 * j)));
+                        tmem_cp_32x128b_x4(sf0 + 8 + 8 * j,
+                                           sf_atom_desc(smem_addr(st + C::o_sf_b + 1024 * j)));
+                        tmem_cp_32x128b_x4(sf0 + 12 + 8 * j,
+                                           sf_atom_desc(smem_addr(st + C::o_sf_b + 1024 * j + 512)));
+                    }
+                    // a K tail of 64 (k not a multiple of 128) uses only the first half
+                    const int steps = (ks == nks - 1 && (tl.g.k % C::BKE) != 0) ? 1 : 2;
+                    const uint32_t a0 = smem_addr(st + C::o_codes_a), b0 = smem_addr(st + C::o_codes_b);
+                    for (int j = 0; j < steps; ++j) {
+                        const uint32_t sfa = sf0 + 4 * j, sfb = sf0 + 8 + 8 * j;
+                        if (GRID == 1) {
+                            umma_fp4_bs(tmem_base, umma_desc_sw64(a0 + 32 * j), umma_desc_sw64(b0 + 32 * j),
+                                        idesc, sfa, sfb, first ? 0u : 1u);
+                            first = false;
+                        } else {
+                            const uint32_t al = smem_addr(st + C::o_lo_a), bl = smem_addr(st + C::o_lo_b);
+                            const uint32_t as[2] = {a0, al}, bs[2] = {b0, bl};
+#pragma unroll
+                            for (int pa = 0; pa < 2; ++pa)
+#pragma unroll
+                                for (int pb = 0; pb < 2; ++pb) {
+                                    umma_fp4_bs(tmem_base, umma_desc_sw64(as[pa] + 32 * j),
+                                                umma_desc_sw64(bs[pb] + 32 * j), idesc, sfa, sfb,
+                                                first ? 0u : 1u);
+                                    first = false;
+                                }
+                        }
+                    }
+                    umma_commit(&empty[s]);
+                }
+                if (ok) umma_commit(acc_full);
+            }
+            umma_commit(drain);
+            uint32_t dummy = 0;
+            mbar_wait(drain, 0, kErrTimeoutDrain, reinterpret_cast<volatile uint32_t *>(&dummy));
+        }
+    } else if (warp < 2 + C::NT) {
+        // ------------------------------------------------------------ transform
+        const int tt = threadIdx.x - 64;
+        constexpr int kThr = C::NT * 32;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const Tile tl = get_tile<BM, BN>(args, t);
+            const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
+            for (int ks = 0; ks < nks; ++ks, ++it) {
+                const int s = it % C::NSTAGE;
+                if (!warp_wait(&full[s], (it / C::NSTAGE) & 1, kErrTimeoutTransform, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *st = stage(s);
+                // scale atoms: unit = (row, K-step j): 4 scales of 16 elements
+                for (int u = tt; u < 2 * (BM + BN); u += kThr) {
+                    const int j = u & 1;
+                    const int row = u >> 1;
+                    const bool isA = row < BM;
+                    const int r = isA ? row : row - BM;
+                    const uint8_t *raw = st + (isA ? C::o_raw_a : C::o_raw_b);
+                    const int rows = isA ? BM : BN;
+                    uint32_t word = 0;
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb) {
+                        const int b16 = 4 * j + kb;                  // 16-element block in the stage
+                        const int braw = blk == 16 ? b16 : (b16 >> 1);
+                        word |= static_cast<uint32_t>(raw[braw * rows + r]) << (8 * kb);
+                    }
+                    uint8_t *atom = st + (isA ? C::o_sf_a + 512 * j
+                                              : C::o_sf_b + 1024 * j + 512 * (r >> 7));
+                    const int rr = r & 127;
+                    *reinterpret_cast<uint32_t *>(atom + 16 * (rr & 31) + 4 * (rr >> 5)) = word;
+                }
+                if (GRID == 0) {
+                    // E1M2 planes: 16-byte chunks of the code tiles, in place.
+                    for (int c = tt; c < (C::kCodesA + C::kCodesB) / 16; c += kThr) {
+                        const int off = c * 16;
+                        uint8_t *src = st + off;   // codes A then codes B are contiguous
+                        uint8_t *lo_dst = st + C::o_lo_a + off;
+                        uint4 w = *reinterpret_cast<const uint4 *>(src);
+                        uint4 h, l;
+                        split_e1m2(w.x, h.x, l.x);
+                        split_e1m2(w.y, h.y, l.y);
+                        split_e1m2(w.z, h.z, l.z);
+                        split_e1m2(w.w, h.w, l.w);
+                        *reinterpret_cast<uint4 *>(src) = h;
+                        *reinterpret_cast<uint4 *>(lo_dst) = l;
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ready[s]);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;
+        const int row_in_tile = 32 * q + lane;
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+        // E1M2 planes carry k = 4 * level on both sides: 1/16 (exact).
+        const float mult = __fmul_rn(__fmul_rn(*args.a_S, *args.b_S),
+                                     args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f));
+        uint32_t tcount = 0;
+        for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
+            const Tile tl = get_tile<BM, BN>(args, t);
+            if (!warp_wait(acc_full, tcount & 1, kErrTimeoutEpilogue, abort_flag)) break;
+            tc_fence_after();
+            const int64_t row = tl.m0 + row_in_tile;
+            const bool row_ok = row < tl.g.m;
+            float *crow = args.c + (tl.g.c_row + row) * args.ldc + tl.g.c_col + tl.n0;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + 32 * c + lane_addr, r);
+                tmem_wait_ld();
+                if (c == BN / 32 - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(acc_empty);
+                }
+                if (!row_ok) continue;
+                const int64_t col0 = tl.n0 + 32 * c;
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    v[i] = tl.g.k > 0 ? __fmul_rn(__uint_as_float(r[i]), mult) : 0.0f;
+                float *dst = crow + 32 * c;
+                const bool vec = (col0 + 32 <= tl.g.n) && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
+                if (vec) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4 *>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                } else {
+                    for (int i = 0; i < 32; ++i)
+                        if (col0 + i < tl.g.n) dst[i] = v[i];
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, Lay::kTmemCols);
+        tmem_dealloc(tmem_base, 512);
     }
+}
+
+template <int GRID>
+cudaError_t launch_fp4(const GemmArgs &args, int num_sms, cudaStream_t stream) {
+    using C = Fp4Cfg<GRID>;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_fp4_kernel<GRID>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    int units = num_sms;
+    if (args.groups == nullptr) {
+        const GemmGroup &g = args.single;
+        const int64_t tiles = ((g.m + BM - 1) / BM) * ((g.n + C::BN - 1) / C::BN);
+        if (tiles < units) units = static_cast<int>(tiles);
+    }
+    if (units <= 0) return cudaSuccess;
+    gemm_fp4_kernel<GRID><<<units, C::kThreads, C::kAlloc, stream>>>(args);
+    return cudaGetLastError();
 }
 
 template <int MODE, int GRID>
 cudaError_t launch_impl(const GemmArgs &args, int num_sms, cudaStream_t stream) {
     using Lay = Layout<MODE>;
+    using C = Cfg<MODE>;
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(gemm_tn_kernel<MODE, GRID>,
@@ -598,27 +1049,46 @@ cudaError_t launch_impl(const GemmArgs &args, int num_sms, cudaStream_t stream) 
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    int grid = num_sms;
+    int units = num_sms / C::CG;
     if (args.groups == nullptr) {
         const GemmGroup &g = args.single;
-        const int64_t tiles = ((g.m + BM - 1) / BM) * ((g.n + Lay::BN - 1) / Lay::BN);
-        if (tiles < grid) grid = static_cast<int>(tiles);
+        const int64_t tiles = ((g.m + C::TM - 1) / C::TM) * ((g.n + C::TN - 1) / C::TN);
+        if (tiles < units) units = static_cast<int>(tiles);
     }
-    if (grid <= 0) return cudaSuccess;
-    gemm_tn_kernel<MODE, GRID><<<grid, Lay::kThreads, Lay::kAlloc, stream>>>(args);
-    return cudaGetLastError();
+    if (units <= 0) return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(units * C::CG, 1, 1);
+    cfg.blockDim = dim3(Lay::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = Lay::kAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C::CG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_tn_kernel<MODE, GRID>, args);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm(const GemmArgs &args, int mode, int grid_kind, int num_sms,
                         cudaStream_t stream) {
-    if (mode == 1) {
-        return grid_kind == 0 ? launch_impl<1, 0>(args, num_sms, stream)
-                              : launch_impl<1, 1>(args, num_sms, stream);
+    switch (mode) {
+        case 0:
+            return grid_kind == 0 ? launch_impl<0, 0>(args, num_sms, stream)
+                                  : launch_impl<0, 1>(args, num_sms, stream);
+        case 1:
+            return grid_kind == 0 ? launch_impl<1, 0>(args, num_sms, stream)
+                                  : launch_impl<1, 1>(args, num_sms, stream);
+        case 2:
+            return grid_kind == 0 ? launch_impl<2, 0>(args, num_sms, stream)
+                                  : launch_impl<2, 1>(args, num_sms, stream);
+        default:
+            return grid_kind == 0 ? launch_fp4<0>(args, num_sms, stream)
+                                  : launch_fp4<1>(args, num_sms, stream);
     }
-    return grid_kind == 0 ? launch_impl<0, 0>(args, num_sms, stream)
-                          : launch_impl<0, 1>(args, num_sms, stream);
 }
 
 }  // namespace ufp4

@@ -79,6 +79,16 @@ __device__ __forceinline__ float exact_diff(float au, float t, float m1, float b
 // saturating at gmax.  [PL] §2 "Rounding rules".
 template <int GRID>
 __device__ __forceinline__ int round_rtne(float au, float m1, float b, float inv) {
+    if (!(fabsf(inv) < INFINITY)) {
+        // Subnormal step: no usable reciprocal, count the boundaries passed.
+        int k = 0;
+#pragma unroll
+        for (int j = 0; j < 7; ++j) {
+            const float d = exact_diff(au, mid_of<GRID>(j), m1, b);
+            if (d > 0.0f || (d == 0.0f && (j & 1))) k = j + 1;
+        }
+        return k;
+    }
     int k = estimate_nearest<GRID>(au * inv);
     if (k > 0) {
         const float d = exact_diff(au, mid_of<GRID>(k - 1), m1, b);
@@ -95,11 +105,19 @@ __device__ __forceinline__ int round_rtne(float au, float m1, float b, float inv
 // au > (lo + r16 * 2^-16 * (hi - lo)) * s.
 template <int GRID>
 __device__ __forceinline__ int round_sr(float au, float m1, float b, float inv, uint32_t r16) {
-    int lo = estimate_floor<GRID>(au * inv);
-    if (lo > 0 && exact_diff(au, level_of<GRID>(lo), m1, b) < 0.0f) {
-        --lo;
-    } else if (lo < 7 && exact_diff(au, level_of<GRID>(lo + 1), m1, b) >= 0.0f) {
-        ++lo;
+    int lo;
+    if (!(fabsf(inv) < INFINITY)) {
+        lo = 0;
+#pragma unroll
+        for (int j = 1; j < 8; ++j)
+            if (exact_diff(au, level_of<GRID>(j), m1, b) >= 0.0f) lo = j;
+    } else {
+        lo = estimate_floor<GRID>(au * inv);
+        if (lo > 0 && exact_diff(au, level_of<GRID>(lo), m1, b) < 0.0f) {
+            --lo;
+        } else if (lo < 7 && exact_diff(au, level_of<GRID>(lo + 1), m1, b) >= 0.0f) {
+            ++lo;
+        }
     }
     if (lo >= 7) return 7;
     const float l0 = level_of<GRID>(lo);
@@ -184,197 +202,358 @@ __device__ __forceinline__ ScaleOut block_scale(float amax, int scale_fmt, float
     return o;
 }
 
+// Keeps the sign bit of a nibble only when its magnitude is nonzero, for
+// the 8 nibbles of a word at once (mag + 7 sets bit 3 iff mag >= 1, and never
+// carries into the next nibble).  Zero is always coded 0x0.
+__device__ __forceinline__ uint32_t canonical_zero(uint32_t w) {
+    const uint32_t mag = w & 0x77777777u;
+    return w & (0x77777777u | ((mag + 0x77777777u) & 0x88888888u));
+}
+
+// x + 1.5*2^23 rounds x to an integer (ties to even) in the low mantissa bits.
+constexpr float kRound = 12582912.0f;
+// A candidate closer than this (in units of the grid step) to a decision
+// boundary is re-decided by the exact path.  The estimate's error is below
+// 2^-20 steps (two roundings of a quotient below 8).
+constexpr float kMargin = 1.0f / 65536.0f;
+
+// E2M1 RTNE of (b, a) -> one byte, low nibble = a (OCP FP4 encoding, sign kept).
+__device__ __forceinline__ uint32_t cvt_e2m1x4(float a0, float a1, float a2, float a3, float a4,
+                                               float a5, float a6, float a7) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(a0), "f"(a1), "f"(a2), "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7));
+    return out;
+}
+
+// Exact path: every element decided by the fma boundary tests.
+template <int GRID, int RND>
+__device__ __noinline__ uint2 round_pack_exact(const float (&v)[16], const ScaleOut &sc,
+                                               const uint32_t (&rnd)[8]) {
+    uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float u = v[i];
+        const float au = fabsf(u);
+        int k;
+        if (RND == 0) {
+            k = round_rtne<GRID>(au, sc.m1, sc.b, sc.inv);
+        } else {
+            const uint32_t word = rnd[i >> 1];
+            const uint32_t r16 = (i & 1) ? (word >> 16) : (word & 0xFFFFu);
+            k = round_sr<GRID>(au, sc.m1, sc.b, sc.inv, r16);
+        }
+        const uint32_t code = static_cast<uint32_t>(k) | ((__float_as_uint(u) >> 28) & 8u);
+        if (i < 8) w0 |= code << (4 * i);
+        else w1 |= code << (4 * (i - 8));
+    }
+    return make_uint2(canonical_zero(w0), canonical_zero(w1));
+}
+
 // Round the 16 rotated values of one chunk and pack them (2 codes / byte,
-// low nibble = lower K index).  Returns the 8 packed bytes.
+// low nibble = lower K index).  A certified fast path decides each element
+// from an fp32 estimate of |u|/s; when any element of the chunk lies within
+// kMargin of a decision boundary the chunk is re-decided exactly, so the
+// result always equals the exact-quotient rule.
 template <int GRID, int RND>
 __device__ __forceinline__ uint2 round_pack(const float (&v)[16], const ScaleOut &sc,
-                                            uint64_t seed, uint32_t stream, uint64_t L0) {
+                                            const PhiloxKeys &keys, uint32_t stream, uint64_t L0) {
     uint32_t rnd[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (RND == 1) {
-        const uint2 key = make_uint2(static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
         const uint64_t g0 = L0 >> 3;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
             const uint64_t g = g0 + c;
             const uint4 r = philox4x32_10(
-                make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), stream, 0u), key);
+                make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), stream, 0u), keys);
             rnd[4 * c + 0] = r.x;
             rnd[4 * c + 1] = r.y;
             rnd[4 * c + 2] = r.z;
             rnd[4 * c + 3] = r.w;
         }
     }
-    uint32_t w0 = 0, w1 = 0;
+    if (sc.zero) return make_uint2(0u, 0u);
+    uint32_t w[2] = {0u, 0u};
+    bool risky = !(sc.inv * 4.0f < INFINITY);   // tiny (subnormal) step: exact path
+    if (GRID == 0 && RND == 0) {
+        // E1M2 RTNE: k = rint(min(|u| * 4/s, 7)).
+        const float inv4 = sc.inv * 4.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float u = v[i];
-        const float au = fabsf(u);
-        int k = 0;
-        if (!sc.zero) {
-            if (RND == 0) {
-                k = round_rtne<GRID>(au, sc.m1, sc.b, sc.inv);
-            } else {
-                const uint32_t word = rnd[i >> 1];
-                const uint32_t r16 = (i & 1) ? (word >> 16) : (word & 0xFFFFu);
-                k = round_sr<GRID>(au, sc.m1, sc.b, sc.inv, r16);
-            }
+        for (int i = 0; i < 16; ++i) {
+            const float u = v[i];
+            const float y = fminf(fabsf(u) * inv4, 7.0f);
+            const float f = y + kRound;
+            risky |= fabsf(y - (f - kRound)) > 0.5f - kMargin;
+            const uint32_t code = (__float_as_uint(f) & 7u) | ((__float_as_uint(u) >> 28) & 8u);
+            w[i >> 3] |= code << (4 * (i & 7));
         }
-        uint32_t code = static_cast<uint32_t>(k);
-        if (k != 0 && (__float_as_uint(u) >> 31)) code |= 8u;
-        if (i < 8) w0 |= code << (4 * i);
-        else w1 |= code << (4 * (i - 8));
-    }
-    return make_uint2(w0, w1);
-}
-
-struct Loaded {
-    uint4 q[16];
-};
-
-// Row-wise: lane loads elements [k0, k0+16) of its row.
-__device__ __forceinline__ void load_rowwise(const QuantArgs &a, int64_t row, int64_t k0,
-                                             uint4 &q0, uint4 &q1) {
-    q0 = make_uint4(0, 0, 0, 0);
-    q1 = make_uint4(0, 0, 0, 0);
-    if (row >= a.rows) return;
-    const uint16_t *p = a.x + row * a.ld + k0;
-    if (k0 < a.cols) q0 = __ldg(reinterpret_cast<const uint4 *>(p));
-    if (k0 + 8 < a.cols) q1 = __ldg(reinterpret_cast<const uint4 *>(p + 8));
-}
-
-// Column-wise: lane loads input rows [k0, k0+16) x columns [c0, c0+8).
-__device__ __forceinline__ void load_colwise(const QuantArgs &a, int64_t k0, int64_t c0,
-                                             uint4 (&q)[16]) {
-    const bool col_ok = c0 < a.cols;
+    } else if (GRID == 0 && RND == 1) {
+        // E1M2 SR.  With q = |u|/(s/4) and r = r16 * 2^-16, "lo = floor(q), up
+        // iff q > lo + r" is exactly k = ceil(q - r): for q = lo + f the value
+        // q - r lies in (lo, lo+1) when f > r and in (lo-1, lo] otherwise.
+        // q >= 7 gives 7 (clamp first).  ceil(t) = rint(t + 1/2) except when t
+        // is (near) an integer, which the margin test sends to the exact path.
+        const float inv4 = sc.inv * 4.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        q[i] = make_uint4(0, 0, 0, 0);
-        if (col_ok && k0 + i < a.rows)
-            q[i] = __ldg(reinterpret_cast<const uint4 *>(a.x + (k0 + i) * a.ld + c0));
+        for (int i = 0; i < 16; ++i) {
+            const float u = v[i];
+            const float y = fminf(fabsf(u) * inv4, 7.0f);
+            const uint32_t word = rnd[i >> 1];
+            const uint32_t r16 = (i & 1) ? (word >> 16) : (word & 0xFFFFu);
+            const float rf = __uint_as_float(0x4B000000u | r16) - 8388608.0f;   // r16 exactly
+            const float th = __fmaf_rn(rf, -1.0f / 65536.0f, y) + 0.5f;          // q - r + 1/2
+            const float f = th + kRound;
+            risky |= fabsf(th - (f - kRound)) > 0.5f - kMargin;
+            const uint32_t code = (__float_as_uint(f) & 7u) | ((__float_as_uint(u) >> 28) & 8u);
+            w[i >> 3] |= code << (4 * (i & 7));
+        }
+    } else if (GRID == 1 && RND == 0) {
+        // E2M1 RTNE: the hardware E2M1 conversion of u/s (ties to even); the
+        // distance to the nearest midpoint is measured in a scale where the
+        // midpoints are half-integers (x2 below 2, x1 below 4, x0.5 above).
+        float y[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            y[i] = v[i] * sc.inv;
+            const float ay = fminf(fabsf(y[i]), 6.0f);
+            const float scl = ay < 2.0f ? 2.0f : (ay < 4.0f ? 1.0f : 0.5f);
+            const float m = __fmaf_rn(ay, scl, -0.5f);
+            risky |= fabsf(m - ((m + kRound) - kRound)) < kMargin;
+        }
+        w[0] = cvt_e2m1x4(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+        w[1] = cvt_e2m1x4(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
+    } else {
+        risky = true;   // E2M1 SR: exact path only
     }
+    if (risky) return round_pack_exact<GRID, RND>(v, sc, rnd);
+    return make_uint2(canonical_zero(w[0]), canonical_zero(w[1]));
 }
 
-__device__ __forceinline__ uint32_t pick_word(const uint4 &q, int w) {
-    return w == 0 ? q.x : (w == 1 ? q.y : (w == 2 ? q.z : q.w));
-}
+// ---------------------------------------------------------------------------
+// Kernel.  A CTA of 256 threads owns a unit of 256 output rows x 64 elements
+// of K; thread t owns output row r0 + t of the unit (all 64 K elements, so any
+// Hadamard size up to 64 and either block size stays inside the thread).  The
+// unit's bf16 tile is staged in shared memory by TMA with the 128-byte
+// swizzle, double-buffered across the CTA's units:
+//   row-wise    one 64 (K) x 256 (rows) box; thread t reads row t, eight
+//               16-byte chunks (chunk c of row t sits at chunk c ^ (t & 7)).
+//   column-wise four 64 (columns) x 64 (K rows) boxes side by side; thread t
+//               reads column t, one bf16 per K row; a warp reads 32
+//               consecutive columns of one K row (no bank conflicts).
+// Codes (32 bytes per thread) and block-major scales (a warp writes 32
+// consecutive rows of each block) go straight to global memory.
+constexpr int kUnitRows = 256;
+constexpr int kStageBytes = kUnitRows * 64 * 2;   // 32 KB of bf16
+constexpr int kQuantSmem = 2 * kStageBytes + 1024 + 64;
 
 template <int AXIS, int NH, int BLK, int GRID, int RND, bool AMAX_ONLY>
-__global__ void __launch_bounds__(kThreads) rht_quantize_kernel(const QuantArgs a) {
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int j = lane & 3;
-    const int g = lane >> 2;
+__global__ void __launch_bounds__(kThreads) rht_quantize_kernel(const __grid_constant__ QuantArgs a,
+                                                               const __grid_constant__ CUtensorMap tmap) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + 2 * kStageBytes);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + 2 * kStageBytes + 16);
+    const int t = threadIdx.x;
+    const int lane = t & 31;
     const int64_t nseg = a.kpad / 64;
+    const int64_t nrb = (a.out_rows + kUnitRows - 1) / kUnitRows;
+    const int64_t nunits = nseg * nrb;
+
+    auto unit_coords = [&](int64_t u, int64_t &rb, int64_t &seg) {
+        if (AXIS == 0) {
+            rb = u / nseg;
+            seg = u % nseg;
+        } else {
+            seg = u / nrb;
+            rb = u % nrb;
+        }
+    };
+    auto issue = [&](int64_t u, int s) {
+        int64_t rb, seg;
+        unit_coords(u, rb, seg);
+        uint8_t *dst = smem + s * kStageBytes;
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        if (AXIS == 0) {
+            tma_load_2d(dst, &tmap, &full[s], static_cast<int32_t>(seg * 64),
+                              static_cast<int32_t>(rb * kUnitRows));
+        } else {
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                tma_load_2d(dst + b * 8192, &tmap, &full[s],
+                                  static_cast<int32_t>(rb * kUnitRows + 64 * b),
+                                  static_cast<int32_t>(seg * 64));
+        }
+    };
+
+    if (t == 0) {
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    int64_t u0 = blockIdx.x;
+    if (t == 0) {
+        if (u0 < nunits) issue(u0, 0);
+        if (u0 + gridDim.x < nunits) issue(u0 + gridDim.x, 1);
+    }
 
     float S = 1.0f, G = 0.0f;
     if (!AMAX_ONLY && a.scale_fmt == 1) {
         const float amax_t = *a.amax_t;
         S = amax_t > 0.0f ? __fdiv_rn(amax_t, gmax_of<GRID>() * 448.0f) : 1.0f;
         G = __fmul_rn(gmax_of<GRID>(), S);
-        if (blockIdx.x == 0 && threadIdx.x == 0 && a.S_out) *a.S_out = S;
+        if (blockIdx.x == 0 && t == 0 && a.S_out) *a.S_out = S;
     }
-    const uint32_t sgn = lane_sign_bits<NH>(a.sign_mask, j);
+    // D for the 64 positions of a segment (K offsets are multiples of 64).
+    uint64_t pat = 0;
+    if (NH > 0) {
+        const uint64_t m = NH == 64 ? a.sign_mask : (a.sign_mask & ((1ull << NH) - 1));
+#pragma unroll
+        for (int off = 0; off < 64; off += (NH > 0 ? NH : 64)) pat |= m << off;
+    }
+    const uint32_t pat_lo = static_cast<uint32_t>(pat), pat_hi = static_cast<uint32_t>(pat >> 32);
+    PhiloxKeys keys;
+    if (RND == 1) keys = philox_keys(a.seed);
     float amax_acc = 0.0f;
 
-    const int64_t total_warps = static_cast<int64_t>(gridDim.x) * kWarps;
-    for (int64_t unit = static_cast<int64_t>(blockIdx.x) * kWarps + warp; unit < a.num_units;
-         unit += total_warps) {
-        int64_t seg, rbase;
-        if (AXIS == 0) {
-            seg = unit % nseg;
-            rbase = (unit / nseg) * 8;
-        } else {
-            const int64_t ncb = (a.out_rows + 63) / 64;
-            seg = unit / ncb;
-            rbase = (unit % ncb) * 64;
+    uint32_t it = 0;
+    for (int64_t u = u0; u < nunits; u += gridDim.x, ++it) {
+        const int s = it & 1;
+        const uint32_t parity = (it >> 1) & 1;
+        // every thread observes the phase itself (bounded)
+        bool ok = mbar_try_wait(&full[s], parity);
+        if (!ok) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!(ok = mbar_try_wait(&full[s], parity))) {
+                if (*abort_flag) break;
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    *abort_flag = 1u;
+                    break;
+                }
+            }
         }
-        const int64_t k0 = seg * 64 + 16 * j;
+        // one decision for the whole CTA (its barriers must stay matched)
+        if (!__syncthreads_and(ok ? 1 : 0)) break;
+        int64_t rb, seg;
+        unit_coords(u, rb, seg);
+        const int64_t orow = rb * kUnitRows + t;
+        const int64_t k0 = seg * 64;
+        const uint8_t *tile = smem + s * kStageBytes;
 
-        uint4 q[16];
-        if (AXIS == 0) {
-            load_rowwise(a, rbase + g, k0, q[0], q[1]);
-        } else {
-            load_colwise(a, k0, rbase + 8 * g, q);
-        }
-
-        constexpr int kRowsPerLane = AXIS == 0 ? 1 : 8;
-        float col_scales[8];
+        // ---- per group of GS elements (the Hadamard block and the scale block
+        // both lie inside one group): load, D, H, block scales, round, pack.
+        constexpr int GS = (NH > BLK ? NH : BLK) > 16 ? (NH > BLK ? NH : BLK) : 16;
+        uint32_t codes[8];
+        uint32_t stored[4];
 #pragma unroll
-        for (int rr = 0; rr < kRowsPerLane; ++rr) {
-            float v[16];
+        for (int g0 = 0; g0 < 64; g0 += GS) {
+            float v[GS];
             if (AXIS == 0) {
+                const uint8_t *rowp = tile + t * 128;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint32_t w0 = pick_word(q[0], i >> 1);
-                    const uint32_t w1 = pick_word(q[1], i >> 1);
-                    v[i] = (i & 1) ? bf16_hi(w0) : bf16_lo(w0);
-                    v[i + 8] = (i & 1) ? bf16_hi(w1) : bf16_lo(w1);
+                for (int c = 0; c < GS / 8; ++c) {
+                    const int cg = g0 / 8 + c;
+                    const uint4 q = *reinterpret_cast<const uint4 *>(rowp + ((cg ^ (t & 7)) << 4));
+                    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        v[8 * c + 2 * e] = __uint_as_float(w[e] << 16);
+                        v[8 * c + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+                    }
                 }
             } else {
+                const int cc = t & 63;
+                const uint8_t *colp = tile + (t >> 6) * 8192 + (cc & 7) * 2;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint32_t w = pick_word(q[i], rr >> 1);
-                    v[i] = (rr & 1) ? bf16_hi(w) : bf16_lo(w);
+                for (int i = 0; i < GS; ++i) {
+                    const int kr = g0 + i;
+                    const uint16_t b = *reinterpret_cast<const uint16_t *>(
+                        colp + kr * 128 + ((((cc >> 3) ^ kr) & 7) << 4));
+                    v[i] = __uint_as_float(static_cast<uint32_t>(b) << 16);
                 }
             }
-            // D: exact negation where the sign mask bit is set.
+            if (NH > 0) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (((sgn >> i) & 1u) << 31));
-            fwht_chunk<NH>(v, j);
-
-            float amax = 0.0f;
+                for (int i = 0; i < GS; ++i) {
+                    const int p = g0 + i;
+                    const uint32_t bit = p < 32 ? (pat_lo >> p) & 1u : (pat_hi >> (p - 32)) & 1u;
+                    v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (bit << 31));
+                }
 #pragma unroll
-            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+                for (int h = 1; h < NH; h <<= 1) {
+#pragma unroll
+                    for (int i = 0; i < GS; ++i) {
+                        if (i & h) continue;
+                        const float x0 = v[i], x1 = v[i + h];
+                        v[i] = __fadd_rn(x0, x1);
+                        v[i + h] = __fsub_rn(x0, x1);
+                    }
+                }
+            }
             if (AMAX_ONLY) {
-                amax_acc = fmaxf(amax_acc, amax);
+#pragma unroll
+                for (int i = 0; i < GS; ++i) amax_acc = fmaxf(amax_acc, fabsf(v[i]));
                 continue;
             }
-            if (BLK == 32) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-
-            const ScaleOut sc = block_scale<GRID>(amax, a.scale_fmt, S, G);
-            const int64_t orow = AXIS == 0 ? rbase + g : rbase + 8 * g + rr;
-            const uint64_t L0 = static_cast<uint64_t>(orow) * static_cast<uint64_t>(a.kpad) +
-                                static_cast<uint64_t>(k0);
-            const uint2 packed = round_pack<GRID, RND>(v, sc, a.seed, a.stream, L0);
-
-            if (orow < a.out_rows) {
-                *reinterpret_cast<uint2 *>(a.codes + orow * (a.kpad / 2) + k0 / 2) = packed;
-                const int64_t blk = k0 / BLK;
-                const bool writer = (BLK == 16) || ((j & 1) == 0);
-                if (AXIS == 0 && writer) {
-                    if (a.scale_fmt == 0)
-                        reinterpret_cast<uint32_t *>(a.scales)[blk * a.scale_ld + orow] = sc.stored;
-                    else
-                        reinterpret_cast<uint8_t *>(a.scales)[blk * a.scale_ld + orow] =
-                            static_cast<uint8_t>(sc.stored);
-                }
-            }
-            col_scales[rr] = __uint_as_float(sc.stored);
-        }
-        if (!AMAX_ONLY && AXIS == 1) {
-            // 8 consecutive output rows of one block: one 32-byte (fp32) or
-            // 8-byte (E4M3) store per lane.
-            const int64_t c0 = rbase + 8 * g;
-            const int64_t blk = k0 / BLK;
-            const bool writer = (BLK == 16) || ((j & 1) == 0);
-            if (writer && c0 < a.out_rows) {
-                if (a.scale_fmt == 0) {
-                    float4 *dst = reinterpret_cast<float4 *>(
-                        reinterpret_cast<float *>(a.scales) + blk * a.scale_ld + c0);
-                    dst[0] = make_float4(col_scales[0], col_scales[1], col_scales[2], col_scales[3]);
-                    dst[1] = make_float4(col_scales[4], col_scales[5], col_scales[6], col_scales[7]);
-                } else {
-                    uint32_t lo = 0, hi = 0;
 #pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        lo |= (__float_as_uint(col_scales[r]) & 0xFFu) << (8 * r);
-                        hi |= (__float_as_uint(col_scales[r + 4]) & 0xFFu) << (8 * r);
-                    }
-                    *reinterpret_cast<uint2 *>(reinterpret_cast<uint8_t *>(a.scales) +
-                                               blk * a.scale_ld + c0) = make_uint2(lo, hi);
+            for (int b0 = 0; b0 < GS; b0 += BLK) {
+                float am = 0.0f;
+#pragma unroll
+                for (int i = 0; i < BLK; ++i) am = fmaxf(am, fabsf(v[b0 + i]));
+                const ScaleOut sc = block_scale<GRID>(am, a.scale_fmt, S, G);
+                stored[(g0 + b0) / BLK] = sc.stored;
+#pragma unroll
+                for (int c0 = 0; c0 < BLK; c0 += 16) {
+                    float chunk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) chunk[i] = v[b0 + c0 + i];
+                    const int kc = g0 + b0 + c0;
+                    const uint64_t L0 = static_cast<uint64_t>(orow) * static_cast<uint64_t>(a.kpad) +
+                                        static_cast<uint64_t>(k0 + kc);
+                    const uint2 pk = round_pack<GRID, RND>(chunk, sc, keys, a.stream, L0);
+                    codes[kc / 8] = pk.x;
+                    codes[kc / 8 + 1] = pk.y;
                 }
             }
+        }
+        if (!AMAX_ONLY && orow < a.out_rows) {
+            uint4 *dst = reinterpret_cast<uint4 *>(a.codes + orow * (a.kpad / 2) + k0 / 2);
+            dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+            dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+            constexpr int kBlocks = 64 / BLK;
+#pragma unroll
+            for (int b = 0; b < kBlocks; ++b) {
+                const int64_t blk = k0 / BLK + b;
+                if (a.scale_fmt == 0)
+                    reinterpret_cast<uint32_t *>(a.scales)[blk * a.scale_ld + orow] = stored[b];
+                else
+                    reinterpret_cast<uint8_t *>(a.scales)[blk * a.scale_ld + orow] =
+                        static_cast<uint8_t>(stored[b]);
+            }
+        }
+        __syncthreads();   // stage s fully consumed
+        if (t == 0 && u + 2 * static_cast<int64_t>(gridDim.x) < nunits)
+            issue(u + 2 * gridDim.x, s);
+    }
+    // Drain in-flight copies before the CTA exits (time-bounded).
+    if (t == 0) {
+        for (uint32_t k = 0; k < 2; ++k) {
+            // the copies issued for iterations it and it+1 (if any)
+            const int64_t u = u0 + static_cast<int64_t>(it + k) * gridDim.x;
+            if (u >= nunits) break;
+            const int s = (it + k) & 1;
+            const uint32_t parity = ((it + k) >> 1) & 1;
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&full[s], parity))
+                if (globaltimer_ns() - t0 > kWaitLimitNs) break;
         }
     }
     if (AMAX_ONLY) {
@@ -387,33 +566,41 @@ __global__ void __launch_bounds__(kThreads) rht_quantize_kernel(const QuantArgs 
 }
 
 template <int AXIS, int NH, int BLK, int GRID, int RND, bool AMAX_ONLY>
-cudaError_t launch_one(const QuantArgs &a, int num_sms, cudaStream_t stream) {
-    const int64_t blocks_needed = (a.num_units + kWarps - 1) / kWarps;
-    const int64_t cap = static_cast<int64_t>(num_sms) * (AXIS == 0 ? 8 : 4);
-    const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
+cudaError_t launch_one(const QuantArgs &a, const CUtensorMap &tmap, int num_sms,
+                       cudaStream_t stream) {
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(rht_quantize_kernel<AXIS, NH, BLK, GRID, RND, AMAX_ONLY>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    const int64_t nunits = (a.kpad / 64) * ((a.out_rows + kUnitRows - 1) / kUnitRows);
+    const int64_t cap = static_cast<int64_t>(num_sms) * 3;
+    const int grid = static_cast<int>(nunits < cap ? nunits : cap);
     if (grid <= 0) return cudaSuccess;
-    rht_quantize_kernel<AXIS, NH, BLK, GRID, RND, AMAX_ONLY><<<grid, kThreads, 0, stream>>>(a);
+    rht_quantize_kernel<AXIS, NH, BLK, GRID, RND, AMAX_ONLY><<<grid, kThreads, kQuantSmem, stream>>>(a, tmap);
     return cudaGetLastError();
 }
 
 template <int AXIS, int NH, int BLK, bool AMAX_ONLY>
-cudaError_t dispatch_grid_round(const QuantArgs &a, int grid_kind, int rnd, int num_sms,
-                                cudaStream_t stream) {
-    if (AMAX_ONLY) return launch_one<AXIS, NH, BLK, 0, 0, true>(a, num_sms, stream);
+cudaError_t dispatch_grid_round(const QuantArgs &a, const CUtensorMap &m, int grid_kind, int rnd,
+                                int num_sms, cudaStream_t stream) {
+    if (AMAX_ONLY) return launch_one<AXIS, NH, BLK, 0, 0, true>(a, m, num_sms, stream);
     if (grid_kind == 0) {
-        return rnd == 0 ? launch_one<AXIS, NH, BLK, 0, 0, false>(a, num_sms, stream)
-                        : launch_one<AXIS, NH, BLK, 0, 1, false>(a, num_sms, stream);
+        return rnd == 0 ? launch_one<AXIS, NH, BLK, 0, 0, false>(a, m, num_sms, stream)
+                        : launch_one<AXIS, NH, BLK, 0, 1, false>(a, m, num_sms, stream);
     }
-    return rnd == 0 ? launch_one<AXIS, NH, BLK, 1, 0, false>(a, num_sms, stream)
-                    : launch_one<AXIS, NH, BLK, 1, 1, false>(a, num_sms, stream);
+    return rnd == 0 ? launch_one<AXIS, NH, BLK, 1, 0, false>(a, m, num_sms, stream)
+                    : launch_one<AXIS, NH, BLK, 1, 1, false>(a, m, num_sms, stream);
 }
 
 template <int AXIS, bool AMAX_ONLY>
-cudaError_t dispatch_nh_blk(const QuantArgs &a, int nh, int blk, int grid_kind, int rnd,
-                            int num_sms, cudaStream_t stream) {
-#define UFP4_CASE(N, B)                                                                     \
-    if (nh == N && blk == B)                                                                \
-        return dispatch_grid_round<AXIS, N, B, AMAX_ONLY>(a, grid_kind, rnd, num_sms, stream);
+cudaError_t dispatch_nh_blk(const QuantArgs &a, const CUtensorMap &m, int nh, int blk,
+                            int grid_kind, int rnd, int num_sms, cudaStream_t stream) {
+#define UFP4_CASE(N, B)                                                                          \
+    if (nh == N && blk == B)                                                                     \
+        return dispatch_grid_round<AXIS, N, B, AMAX_ONLY>(a, m, grid_kind, rnd, num_sms, stream);
     UFP4_CASE(0, 16)
     UFP4_CASE(0, 32)
     UFP4_CASE(16, 16)
@@ -426,27 +613,37 @@ cudaError_t dispatch_nh_blk(const QuantArgs &a, int nh, int blk, int grid_kind, 
     return cudaErrorInvalidValue;
 }
 
+// bf16 input as a 2-D tensor map: rows x cols, row pitch ld; 128-byte swizzle,
+// box 64 x 256 (row-wise: K x rows) or 64 x 64 (column-wise: columns x K).
+cudaError_t make_input_map(const QuantArgs &a, CUtensorMap *m) {
+    const uint32_t box_outer = a.axis == 0 ? kUnitRows : 64;
+    CUresult r = encode_tensor_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x,
+                                      static_cast<uint64_t>(a.cols), static_cast<uint64_t>(a.rows),
+                                      static_cast<uint64_t>(a.ld) * 2, 64, box_outer,
+                                      CU_TENSOR_MAP_SWIZZLE_128B);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 cudaError_t launch_rht_quantize(QuantArgs a, int hadamard_n, int block, int grid_kind,
                                 int rounding, int num_sms, cudaStream_t stream) {
-    if (a.axis == 0) {
-        a.num_units = ((a.out_rows + 7) / 8) * (a.kpad / 64);
-        return dispatch_nh_blk<0, false>(a, hadamard_n, block, grid_kind, rounding, num_sms, stream);
-    }
-    a.num_units = ((a.out_rows + 63) / 64) * (a.kpad / 64);
-    return dispatch_nh_blk<1, false>(a, hadamard_n, block, grid_kind, rounding, num_sms, stream);
+    CUtensorMap m;
+    cudaError_t e = make_input_map(a, &m);
+    if (e != cudaSuccess) return e;
+    if (a.axis == 0)
+        return dispatch_nh_blk<0, false>(a, m, hadamard_n, block, grid_kind, rounding, num_sms, stream);
+    return dispatch_nh_blk<1, false>(a, m, hadamard_n, block, grid_kind, rounding, num_sms, stream);
 }
 
 cudaError_t launch_rht_amax(QuantArgs a, int hadamard_n, int num_sms, cudaStream_t stream) {
     cudaError_t e = cudaMemsetAsync(a.amax_out, 0, sizeof(float), stream);
     if (e != cudaSuccess) return e;
-    if (a.axis == 0) {
-        a.num_units = ((a.out_rows + 7) / 8) * (a.kpad / 64);
-        return dispatch_nh_blk<0, true>(a, hadamard_n, 16, 0, 0, num_sms, stream);
-    }
-    a.num_units = ((a.out_rows + 63) / 64) * (a.kpad / 64);
-    return dispatch_nh_blk<1, true>(a, hadamard_n, 16, 0, 0, num_sms, stream);
+    CUtensorMap m;
+    e = make_input_map(a, &m);
+    if (e != cudaSuccess) return e;
+    if (a.axis == 0) return dispatch_nh_blk<0, true>(a, m, hadamard_n, 16, 0, 0, num_sms, stream);
+    return dispatch_nh_blk<1, true>(a, m, hadamard_n, 16, 0, 0, num_sms, stream);
 }
 
 }  // namespace ufp4

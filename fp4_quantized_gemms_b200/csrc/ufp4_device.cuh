@@ -8,21 +8,6 @@
 
 namespace ufp4 {
 
-#ifdef UFP4_PIPELINE_KERNELS
-// ---------------------------------------------------------------------------
-// Device error word.  Bounded waits that give up OR a code in here and make
-// their kernel unwind; the host reads it through ufp4_check_device_status().
-// Only the pipelined GEMM translation unit includes this section.
-static __device__ uint32_t g_error_word = 0;
-
-enum : uint32_t {
-    kErrTimeoutProducer = 1u << 0,
-    kErrTimeoutTransform = 1u << 1,
-    kErrTimeoutMma = 1u << 2,
-    kErrTimeoutEpilogue = 1u << 3,
-    kErrTimeoutDrain = 1u << 4,
-};
-
 // A pipeline wait that has not completed after this long is treated as a
 // hang: ~2 s, several orders of magnitude above any legitimate stage wait.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -71,6 +56,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+#ifdef UFP4_PIPELINE_KERNELS
+// ---------------------------------------------------------------------------
+// Device error word.  Bounded waits that give up OR a code in here and make
+// their kernel unwind; the host reads it through ufp4_check_device_status().
+// Only the pipelined GEMM translation unit includes this section.
+static __device__ uint32_t g_error_word = 0;
+
+enum : uint32_t {
+    kErrTimeoutProducer = 1u << 0,
+    kErrTimeoutTransform = 1u << 1,
+    kErrTimeoutMma = 1u << 2,
+    kErrTimeoutEpilogue = 1u << 3,
+    kErrTimeoutDrain = 1u << 4,
+};
+
 // Waits for the phase with the given parity to complete.  Gives up after
 // kWaitLimitNs (or at once when *abort is set by another role of the CTA),
 // records `err` in the device error word and returns false.
@@ -89,24 +89,77 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
     }
 }
 
+// Cluster-scope acquire wait, for barriers that a peer CTA arrives at.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint32_t err,
+                                                  volatile uint32_t *abort) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_error_word, err);
+            *abort = 1u;
+            return false;
+        }
+    }
+}
+
+// Arrive on the same-offset barrier of CTA `rank` of this cluster.
+__device__ __forceinline__ void mbar_arrive_remote(uint64_t *bar, uint32_t rank) {
+    asm volatile(
+        "{\n\t.reg .b32 ra;\n\t"
+        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+        "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_addr(bar)),
+        "r"(rank)
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+
 // Warp-uniform form for roles whose lanes must stay converged (they execute
 // __syncwarp and .sync.aligned tcgen05 loads afterwards): lane 0 performs the
 // bounded wait and broadcasts the outcome; on success the other lanes observe
 // the (already completed, and stable until this warp releases its slot) phase
 // themselves, with an iteration cap.
+template <bool kCluster = false>
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, uint32_t err,
                                           volatile uint32_t *abort) {
     const int lane = threadIdx.x & 31;
     bool ok = true;
-    if (lane == 0) ok = mbar_wait(bar, parity, err, abort);
+    if (lane == 0)
+        ok = kCluster ? mbar_wait_cluster(bar, parity, err, abort) : mbar_wait(bar, parity, err, abort);
     ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
     if (ok && lane != 0) {
         for (int i = 0; i < (1 << 20); ++i)
-            if (mbar_try_wait(bar, parity)) break;
+            if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) break;
     }
     __syncwarp();
     return ok;
 }
+
+#endif  // UFP4_PIPELINE_KERNELS
 
 // ---------------------------------------------------------------------------
 // TMA: 2-D tiled bulk tensor load into this CTA's shared memory, completion
@@ -139,6 +192,19 @@ __device__ __forceinline__ void tmem_alloc(uint32_t *smem_result, uint32_t ncols
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *smem_result, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(smem_result)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                  : "memory");
@@ -160,6 +226,88 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// CTA-pair MMA (M = 256 split over the two CTAs of a cluster, B split along
+// N), issued by the even CTA.
+__device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Pair commit: arrive on the same-offset mbarrier of every CTA in `mask`.
+__device__ __forceinline__ void umma_commit_pair_mc(uint64_t *bar, uint16_t mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_addr(bar)),
+        "h"(mask)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_addr(bar))
+        : "memory");
+}
+
+// Block-scaled FP4 MMA: D[tmem] (+)= (A * SFA)[smem] * (B * SFB)[smem]^T with
+// E2M1 operands and UE4M3 scale factors per 16 elements along K (taken from
+// TMEM at sfa / sfb), fp32 accumulate, K = 64 per instruction.
+__device__ __forceinline__ void umma_fp4_bs(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Shared memory -> TMEM copy of a 32 x 128-bit block (one scale-factor atom of
+// 128 rows x 4 scales), replicated to the four 32-lane groups.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+
+// Descriptor of a 512-byte scale-factor atom in shared memory: 32 rows of 16
+// bytes, no swizzle (8-row core matrices, 128 bytes apart).
+__device__ __forceinline__ uint64_t sf_atom_desc(uint32_t smem_byte_addr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(128u >> 4) << 16;
+    d |= static_cast<uint64_t>(128u >> 4) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    return d;
+}
+
+// K-major operand in the 64-byte swizzle layout: rows of 64 bytes, 8-row
+// atoms of 512 bytes (stride byte offset 512), layout type 4 = SWIZZLE_64B.
+__device__ __forceinline__ uint64_t umma_desc_sw64(uint32_t smem_byte_addr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(1u) << 16;
+    d |= static_cast<uint64_t>(512u >> 4) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(4u) << 61;
+    return d;
+}
+
+// Instruction descriptor, kind::mxf4nvf4 block-scaled: A = B = E2M1, UE4M3
+// scale factors, fp32 accumulate, both K-major.
+__host__ __device__ constexpr uint32_t umma_idesc_fp4_bs(int M, int N) {
+    return (1u << 7) | (1u << 10)                      // A, B: E2M1
+           | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+           | (0u << 23)                                // scale format UE4M3
+           | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
 // Arrive on an mbarrier once every prior tcgen05 async op of this thread is done.
@@ -217,8 +365,6 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
 
-#endif  // UFP4_PIPELINE_KERNELS
-
 // ---------------------------------------------------------------------------
 // Philox4x32-10 (Salmon et al., SC'11): 32x32->64 multiplies by 0xD2511F53 /
 // 0xCD9E8D57, key bumped by 0x9E3779B9 / 0xBB67AE85 between ten rounds.
@@ -229,11 +375,40 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
             k.x += 0x9E3779B9u;
             k.y += 0xBB67AE85u;
         }
-        const uint32_t lo0 = 0xD2511F53u * c.x;
-        const uint32_t hi0 = __umulhi(0xD2511F53u, c.x);
-        const uint32_t lo1 = 0xCD9E8D57u * c.z;
-        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z);
-        c = make_uint4(hi1 ^ c.y ^ k.x, lo1, hi0 ^ c.w ^ k.y, lo0);
+        const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c.x;
+        const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c.z;
+        c = make_uint4(static_cast<uint32_t>(p1 >> 32) ^ c.y ^ k.x, static_cast<uint32_t>(p1),
+                       static_cast<uint32_t>(p0 >> 32) ^ c.w ^ k.y, static_cast<uint32_t>(p0));
+    }
+    return c;
+}
+
+// The ten round keys of one Philox key (the key schedule does not depend on
+// the counter, so a thread computes it once).
+struct PhiloxKeys {
+    uint32_t x[10], y[10];
+};
+
+__device__ __forceinline__ PhiloxKeys philox_keys(uint64_t seed) {
+    PhiloxKeys ks;
+    uint32_t a = static_cast<uint32_t>(seed), b = static_cast<uint32_t>(seed >> 32);
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        ks.x[r] = a;
+        ks.y[r] = b;
+        a += 0x9E3779B9u;
+        b += 0xBB67AE85u;
+    }
+    return ks;
+}
+
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, const PhiloxKeys &ks) {
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c.x;
+        const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c.z;
+        c = make_uint4(static_cast<uint32_t>(p1 >> 32) ^ c.y ^ ks.x[r], static_cast<uint32_t>(p1),
+                       static_cast<uint32_t>(p0 >> 32) ^ c.w ^ ks.y[r], static_cast<uint32_t>(p0));
     }
     return c;
 }

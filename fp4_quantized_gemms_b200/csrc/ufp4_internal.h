@@ -52,12 +52,14 @@ struct GemmArgs {
 
 // mode 0: fp32 block scales (per-block partial products, CUDA-core scaling)
 // mode 1: E4M3 x fp32 two-level scales (scales folded into fp16 operands)
+// mode 2: mode 1 on a CTA pair (cta_group::2, 256 x 256 tiles)
 cudaError_t launch_gemm(const GemmArgs &args, int mode, int grid_kind, int num_sms,
                         cudaStream_t stream);
 
 // Driver entry point for tensor-map encoding (resolved once at run time).
 CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
                               uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                              uint32_t box_inner, uint32_t box_outer);
+                              uint32_t box_inner, uint32_t box_outer,
+                              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE);
 
 }  // namespace ufp4

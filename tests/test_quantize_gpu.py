@@ -73,6 +73,7 @@ def test_quantize_exact_ties_and_zero_blocks(axis, grid):
     X[5, :] = 0.0
     X[9, 32:48] = 0.0
     X[11, 64:80] = np.float32(1e-30)
+    X[13, 96:112] = np.float32(3e-39) * rng.integers(-5, 6, 16)   # subnormal block scale
     bits = wl.bf16_bits(X)
     for rounding in (ufp4.ROUND_RTNE, ufp4.ROUND_SR):
         cfg = ufp4.QuantConfig(grid=grid, rounding=rounding, sr_seed=7, hadamard_n=0)
