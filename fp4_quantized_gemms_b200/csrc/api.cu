@@ -8,6 +8,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "ufp4.h"
@@ -98,16 +99,22 @@ ufp4_status_t check_pair(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b, bool 
     return UFP4_OK;
 }
 
+std::atomic<int32_t> g_two_level_path{UFP4_GEMM_PATH_AUTO};
+
 ufp4_status_t encode_operand_maps(const ufp4_qtensor_t *q, int box_rows, int mode,
                                   CUtensorMap *codes, CUtensorMap *scales) {
     const int64_t rows_t = q->rows > 0 ? q->rows : 1;
+    // mode 3 stages 128 K elements (64 code bytes, 64-byte swizzle) per step,
+    // the others 64 (32 bytes, 32-byte swizzle).
+    const bool native = mode == 3;
     CUresult r = encode_tensor_map_2d(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, q->codes,
                                       static_cast<uint64_t>(q->kpad / 2),
                                       static_cast<uint64_t>(rows_t),
-                                      static_cast<uint64_t>(q->kpad / 2), 32,
-                                      static_cast<uint32_t>(box_rows), CU_TENSOR_MAP_SWIZZLE_32B);
+                                      static_cast<uint64_t>(q->kpad / 2), native ? 64 : 32,
+                                      static_cast<uint32_t>(box_rows),
+                                      native ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
     if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
-    const int nblk_stage = 64 / q->cfg.block;
+    const int nblk_stage = (native ? 128 : 64) / q->cfg.block;
     const uint64_t nblk = static_cast<uint64_t>(q->kpad / q->cfg.block);
     if (mode != 0) {
         r = encode_tensor_map_2d(scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, q->scales,
@@ -137,10 +144,18 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
         return UFP4_ERR_ALIGNMENT;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // fp32 block scales: per-block partials (mode 0).  Two-level scales: the
-    // CTA-pair kernel (256 x 256 tiles, mode 2), or one CTA per 128 x 256 tile
-    // (mode 1) when a single problem has at most 128 rows.
+    // native block-scaled FP4 kernel (mode 3) unless the caller picked one of
+    // the fp16-operand kernels (mode 1: one CTA per 128 x 256 tile, mode 2:
+    // CTA pairs on 256 x 256 tiles).
     int mode = 0;
-    if (a->cfg.scale_fmt == UFP4_SCALE_E4M3_X_FP32) mode = (groups_dev != nullptr || m > 128) ? 2 : 1;
+    if (a->cfg.scale_fmt == UFP4_SCALE_E4M3_X_FP32) {
+        switch (g_two_level_path.load()) {
+            case UFP4_GEMM_PATH_FP16: mode = 1; break;
+            case UFP4_GEMM_PATH_FP16_PAIR: mode = 2; break;
+            case UFP4_GEMM_PATH_NATIVE_FP4: mode = 3; break;
+            default: mode = 3; break;
+        }
+    }
     if (groups_dev == nullptr) {
         if (m == 0 || n == 0) return UFP4_OK;
         if (a->kpad == 0) {
@@ -155,7 +170,7 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
 
     GemmArgs args;
     memset(&args, 0, sizeof(args));
-    const int bn = mode == 1 ? 256 : 128;   // B rows staged per CTA
+    const int bn = (mode == 1 || mode == 3) ? 256 : 128;   // B rows staged per CTA
     s = encode_operand_maps(a, 128, mode, &args.tm_a_codes, &args.tm_a_scales);
     if (s != UFP4_OK) return s;
     s = encode_operand_maps(b, bn, mode, &args.tm_b_codes, &args.tm_b_scales);
@@ -330,6 +345,14 @@ ufp4_status_t ufp4_grouped_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b
     if (c_dev == nullptr) return UFP4_ERR_INVALID_ARG;
     return run_gemm(a, b, groups_dev, num_groups, c_dev, ldc, 0, 0, stream);
 }
+
+ufp4_status_t ufp4_set_two_level_gemm_path(int32_t path) {
+    if (path < UFP4_GEMM_PATH_AUTO || path > UFP4_GEMM_PATH_NATIVE_FP4) return UFP4_ERR_INVALID_ARG;
+    g_two_level_path.store(path);
+    return UFP4_OK;
+}
+
+int32_t ufp4_get_two_level_gemm_path(void) { return g_two_level_path.load(); }
 
 ufp4_status_t ufp4_check_device_status(void) {
     uint32_t w = 0;

@@ -875,8 +875,9 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
                         tmem_cp_32x128b_x4(sf0 + 12 + 8 * j,
                                            sf_atom_desc(smem_addr(st + C::o_sf_b + 1024 * j + 512)));
                     }
-                    // a K tail of 64 (k not a multiple of 128) uses only the first half
-                    const int steps = (ks == nks - 1 && (tl.g.k % C::BKE) != 0) ? 1 : 2;
+                    // K steps of 64 in this stage (a tail may use only the first)
+                    const int64_t rem = tl.g.k - static_cast<int64_t>(ks) * C::BKE;
+                    const int steps = rem >= C::BKE ? 2 : 1;
                     const uint32_t a0 = smem_addr(st + C::o_codes_a), b0 = smem_addr(st + C::o_codes_b);
                     for (int j = 0; j < steps; ++j) {
                         const uint32_t sfa = sf0 + 4 * j, sfb = sf0 + 8 + 8 * j;

@@ -53,6 +53,7 @@ struct GemmArgs {
 // mode 0: fp32 block scales (per-block partial products, CUDA-core scaling)
 // mode 1: E4M3 x fp32 two-level scales (scales folded into fp16 operands)
 // mode 2: mode 1 on a CTA pair (cta_group::2, 256 x 256 tiles)
+// mode 3: two-level scales on the native block-scaled FP4 MMA (kind::mxf4nvf4)
 cudaError_t launch_gemm(const GemmArgs &args, int mode, int grid_kind, int num_sms,
                         cudaStream_t stream);
 

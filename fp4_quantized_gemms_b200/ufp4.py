@@ -29,7 +29,8 @@ DEFAULT_SIGN_MASK = 0x09F1FD9D03F0A9B4
 EXPORTED = [
     "ufp4_qtensor_layout", "ufp4_rht_amax", "ufp4_rht_quantize", "ufp4_gemm_fprop",
     "ufp4_gemm_dgrad", "ufp4_gemm_wgrad", "ufp4_grouped_gemm", "ufp4_check_device_status",
-    "ufp4_status_string", "ufp4_version",
+    "ufp4_status_string", "ufp4_version", "ufp4_set_two_level_gemm_path",
+    "ufp4_get_two_level_gemm_path",
 ]
 
 
@@ -91,6 +92,10 @@ def lib() -> ctypes.CDLL:
                                         i32, P, i64, P]
         L.ufp4_check_device_status.restype = st
         L.ufp4_check_device_status.argtypes = []
+        L.ufp4_set_two_level_gemm_path.restype = st
+        L.ufp4_set_two_level_gemm_path.argtypes = [i32]
+        L.ufp4_get_two_level_gemm_path.restype = i32
+        L.ufp4_get_two_level_gemm_path.argtypes = []
         _lib = L
     return _lib
 
@@ -244,6 +249,18 @@ def grouped_gemm(a: QTensor, b: QTensor, groups: torch.Tensor, out: torch.Tensor
                                    ctypes.c_void_p(out.data_ptr()), out.stride(0),
                                    _stream_ptr(out.device)), "ufp4_grouped_gemm")
     return out
+
+
+GEMM_PATH_AUTO, GEMM_PATH_FP16, GEMM_PATH_FP16_PAIR, GEMM_PATH_NATIVE_FP4 = 0, 1, 2, 3
+
+
+def set_two_level_gemm_path(path: int) -> None:
+    """Process-wide kernel family for GEMMs on two-level-scaled operands."""
+    _check(lib().ufp4_set_two_level_gemm_path(path), "ufp4_set_two_level_gemm_path")
+
+
+def get_two_level_gemm_path() -> int:
+    return lib().ufp4_get_two_level_gemm_path()
 
 
 def check_device_status() -> int:

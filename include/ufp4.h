@@ -196,6 +196,29 @@ ufp4_status_t ufp4_grouped_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b
                                 const ufp4_group_t *groups_dev, int32_t num_groups,
                                 float *c_dev, int64_t ldc, void *stream);
 
+/* Kernel family for GEMMs whose operands carry two-level (E4M3 x fp32)
+ * scales.  Every family computes the same contraction (the quantized values
+ * are exact in each operand format and products accumulate in fp32); they
+ * differ in how the tensor core is fed:
+ *   UFP4_GEMM_PATH_FP16       scales folded into exact fp16 operands,
+ *                             kind::f16 MMA, one CTA per 128 x 256 tile;
+ *   UFP4_GEMM_PATH_FP16_PAIR  the same on a CTA pair (256 x 256 tiles);
+ *   UFP4_GEMM_PATH_NATIVE_FP4 block-scaled FP4 MMA (kind::mxf4nvf4, UE4M3
+ *                             factors per 16 elements); E1M2 codes are split
+ *                             exactly into two E2M1 planes (four MMAs);
+ *   UFP4_GEMM_PATH_AUTO       the library's choice (default; currently the
+ *                             native FP4 path).
+ * The setting is process-wide and read at each GEMM call; fp32 block scales
+ * are unaffected.  Errors: INVALID_ARG for an unknown path. */
+typedef enum {
+    UFP4_GEMM_PATH_AUTO = 0,
+    UFP4_GEMM_PATH_FP16 = 1,
+    UFP4_GEMM_PATH_FP16_PAIR = 2,
+    UFP4_GEMM_PATH_NATIVE_FP4 = 3
+} ufp4_gemm_path_t;
+ufp4_status_t ufp4_set_two_level_gemm_path(int32_t path);
+int32_t ufp4_get_two_level_gemm_path(void);
+
 /* Reads and clears the device-side error word that kernels set when a
  * bounded pipeline wait gives up (synchronises the current device).
  * Returns UFP4_OK or UFP4_ERR_DEVICE_TIMEOUT (or UFP4_ERR_CUDA). */

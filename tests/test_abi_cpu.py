@@ -142,3 +142,19 @@ def test_quantize_validation_rejects_before_launch(L):
     assert Q(x, 64, 128, 128, 0, None, ctypes.byref(two), None) == ufp4.ERR_INVALID_ARG   # no amax
     assert L.ufp4_rht_amax(x, 64, 128, 128, 0, 8, 0, ctypes.c_void_p(4096), None) == ufp4.ERR_UNSUPPORTED
     assert L.ufp4_rht_amax(x, 64, 128, 128, 0, 16, 0, None, None) == ufp4.ERR_INVALID_ARG
+
+
+def test_two_level_gemm_path_selector(L):
+    """The path setting is host state: it round-trips and rejects unknown values."""
+    old = ufp4.get_two_level_gemm_path()
+    try:
+        for p in (ufp4.GEMM_PATH_NATIVE_FP4, ufp4.GEMM_PATH_FP16, ufp4.GEMM_PATH_FP16_PAIR,
+                  ufp4.GEMM_PATH_AUTO):
+            ufp4.set_two_level_gemm_path(p)
+            assert ufp4.get_two_level_gemm_path() == p
+        for bad in (-1, 4, 99):
+            with pytest.raises(ufp4.UFP4Error):
+                ufp4.set_two_level_gemm_path(bad)
+        assert ufp4.get_two_level_gemm_path() == ufp4.GEMM_PATH_AUTO
+    finally:
+        ufp4.set_two_level_gemm_path(old)
