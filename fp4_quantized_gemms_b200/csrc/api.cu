@@ -186,6 +186,18 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
     args.single.m = m;
     args.single.n = n;
     args.single.k = a->kpad;
+    if (mode == 3 && aligned16(c) && ldc % 4 == 0) {
+        // Output tensor map for the TMA-store epilogue: the exact m x n window
+        // of a single problem (stores clip at its edges); for a group table
+        // the row count is not known here, so the map spans ldc columns and
+        // 2^30 rows and the kernel stores only chunks inside a group.
+        const uint64_t inner = groups_dev == nullptr ? static_cast<uint64_t>(n) : static_cast<uint64_t>(ldc);
+        const uint64_t outer = groups_dev == nullptr ? static_cast<uint64_t>(m) : (1ull << 30);
+        CUresult r = encode_tensor_map_2d(&args.tm_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c, inner, outer,
+                                          static_cast<uint64_t>(ldc) * 4, 32, 128,
+                                          CU_TENSOR_MAP_SWIZZLE_128B);
+        args.c_tma = r == CUDA_SUCCESS ? 1 : 0;
+    }
     cudaError_t e = launch_gemm(args, mode, a->cfg.grid, sm_count(), st);
     return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
 }

@@ -704,62 +704,87 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
 //
 // kind::mxf4nvf4 multiplies E2M1 operands scaled per 16 elements by UE4M3
 // factors, which is exactly an E2M1 operand under the two-level scales (the
-// block scale e_b is a positive E4M3 byte).  E2M1 codes go from TMA straight
-// to the tensor core.  An E1M2 code k splits exactly into two E2M1 values,
-// k = hi + lo with hi in {0,1,2,3,4,4,6,6}[k] and lo = 1 for k in {5,7}, so
-// sum_k k_a k_b e_a e_b = sum over the four plane products, each one native
-// FP4 MMA with the same scale factors.  The split is a per-byte bit
-// operation done in place in shared memory (hi overwrites the code bytes).
+// block scale e_b is a non-negative E4M3 byte).  E2M1 codes go from TMA
+// straight to the tensor core.  An E1M2 code with magnitude k (value k/4 of
+// the step) splits exactly into two E2M1 operands: the code bits read as an
+// E2M1 number e(k) = {0, .5, 1, 1.5, 2, 3, 4, 6}[k], plus a correction plane
+// d(k) = k - e(k) = {0, .5, 1, 1.5, 2, 2, 2, 1}[k], which is E2M1 as well.
+// Then sum k_a k_b = sum (e_a + d_a)(e_b + d_b): four native MMAs with the
+// same scale factors, the raw code tiles used as they arrived and only the
+// correction planes written by the transform warps (a per-byte bit function).
 //
-// Tile 128 x 256, 128 K elements (64 bytes of codes per row, 64-byte TMA
-// swizzle) per stage.  A transform group permutes the block-major E4M3 bytes
-// into the 128-row x 4-scale atoms that tcgen05.cp moves to TMEM.
+// Tile 128 x 256, 128 K elements (64 code bytes per row, 64-byte TMA
+// swizzle) per stage.  The transform warps permute the block-major E4M3
+// bytes into the 32-row x 16-byte atoms that tcgen05.cp moves to TMEM (a 4x4
+// byte transpose per 4 rows), and build the E1M2 correction planes into a
+// two-slot ring.  The epilogue stages 128 x 32 fp32 chunks in shared memory
+// (128-byte swizzle) and writes them with TMA stores.
 template <int GRID>
 struct Fp4Cfg {
     static constexpr int BN = 256;
-    static constexpr int BKE = 128;            // K elements per stage
-    static constexpr int kRow = 64;            // code bytes per row per stage
-    static constexpr int NSTAGE = GRID == 0 ? 3 : 5;
-    static constexpr int NT = 4;               // transform warps
-    static constexpr int NE = 4;               // epilogue warps
+    static constexpr int BKE = 128;                 // K elements per stage
+    static constexpr int kRow = 64;                 // code bytes per row per stage
+    static constexpr int NS = GRID == 0 ? 4 : 6;    // TMA ring stages
+    static constexpr int ND = GRID == 0 ? 2 : 0;    // correction-plane slots
+    static constexpr int NT = GRID == 0 ? 8 : 4;    // transform warps
+    static constexpr int NE = 4;                    // epilogue warps
     static constexpr int kCodesA = BM * kRow;
     static constexpr int kCodesB = BN * kRow;
-    static constexpr int kLoA = GRID == 0 ? kCodesA : 0;
-    static constexpr int kLoB = GRID == 0 ? kCodesB : 0;
     static constexpr int kRawA = BM * (BKE / 16);
     static constexpr int kRawB = BN * (BKE / 16);
-    static constexpr int kSfA = 2 * 512;        // 2 K-steps x 1 row tile
-    static constexpr int kSfB = 2 * 2 * 512;    // 2 K-steps x 2 row tiles
+    static constexpr int kSfA = 2 * 512;            // 2 K steps x 1 row atom group
+    static constexpr int kSfB = 2 * 2 * 512;        // 2 K steps x 2 row atom groups
     static constexpr int o_codes_a = 0;
     static constexpr int o_codes_b = o_codes_a + kCodesA;
-    static constexpr int o_lo_a = o_codes_b + kCodesB;
-    static constexpr int o_lo_b = o_lo_a + kLoA;
-    static constexpr int o_raw_a = o_lo_b + kLoB;
+    static constexpr int o_raw_a = o_codes_b + kCodesB;
     static constexpr int o_raw_b = o_raw_a + kRawA;
     static constexpr int o_sf_a = o_raw_b + kRawB;
     static constexpr int o_sf_b = o_sf_a + kSfA;
     static constexpr int kStage = (o_sf_b + kSfB + 1023) / 1024 * 1024;
-    static constexpr int o_bar = NSTAGE * kStage;
-    // barriers: full, ready, empty per stage; acc_full, acc_empty, drain
-    static constexpr int kNumBars = 3 * NSTAGE + 3;
+    static constexpr int kCorr = kCodesA + kCodesB;  // one correction slot
+    static constexpr int o_corr = NS * kStage;
+    static constexpr int kOutChunk = BM * 32 * 4;   // 128 rows x 32 fp32
+    static constexpr int o_out = o_corr + ND * kCorr;
+    static constexpr int o_bar = o_out + 2 * kOutChunk;
+    // full, ready, empty per stage; acc_full, acc_empty, drain; out_full[2], out_free[2]
+    static constexpr int kNumBars = 3 * NS + 3 + 4;
     static constexpr int o_misc = o_bar + kNumBars * 8;
     static constexpr int kAlloc = o_misc + 64 + 1024;
     static constexpr int kThreads = 32 * (2 + NT + NE);
-    static constexpr int kSfColsPerStage = 24;  // SFA 2 x 4, SFB 2 x 8
+    static constexpr int kSfColsPerStage = 24;      // SFA 2 x 4, SFB 2 x 8
     static constexpr int kAccCols = 256;
-    static_assert(kAccCols + NSTAGE * kSfColsPerStage <= 512, "TMEM budget");
+    static_assert(kAccCols + NS * kSfColsPerStage <= 512, "TMEM budget");
     static_assert(kAlloc <= 232448, "shared memory budget");
+    static_assert(o_corr % 1024 == 0 && o_out % 1024 == 0, "swizzle alignment");
 };
 
-// hi / lo E2M1 planes of 8 E1M2 codes (see above); signs copied to both.
-__device__ __forceinline__ void split_e1m2(uint32_t w, uint32_t &hi, uint32_t &lo) {
-    const uint32_t M = 0x11111111u;
-    const uint32_t b0 = w & M, b1 = (w >> 1) & M, b2 = (w >> 2) & M, s = w & 0x88888888u;
-    const uint32_t h2 = b2 | b1;
-    const uint32_t h1 = b2 | (~b1 & b0);
-    const uint32_t h0 = b1 & (b0 | b2);
-    hi = s | (h2 << 2) | (h1 << 1) | h0;
-    lo = s | ((b2 & b0) << 1);
+// Correction plane of 8 E1M2 codes (sign copied, magnitude d(k) as E2M1):
+// d = 4 for k in {4,5,6}, 2 for k in {2,3,7}, and bit 0 = (k in {1,3}).
+__device__ __forceinline__ uint32_t e1m2_correction(uint32_t w) {
+    const uint32_t r1 = w >> 1, r2 = w >> 2, l1 = w << 1, l2 = w << 2;
+    const uint32_t d0 = w & ~r2 & 0x11111111u;       // b0 & ~b2
+    const uint32_t d1 = w & (~r1 | l1);              // at bit 1: b1 & (~b2 | b0)
+    const uint32_t d2 = w & ~(l1 & l2);              // at bit 2: b2 & ~(b1 & b0)
+    const uint32_t y = (d2 & 0x44444444u) | (d1 & ~0x44444444u);
+    const uint32_t z = (w & 0x88888888u) | (y & ~0x88888888u);
+    return (z & ~0x11111111u) | d0;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// 4 x 4 byte transpose: out_i holds byte i of w0, w1, w2, w3 (low to high).
+__device__ __forceinline__ void transpose4x4(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
+                                             uint32_t (&o)[4]) {
+    const uint32_t t0 = prmt(w0, w1, 0x5140u), t1 = prmt(w0, w1, 0x7362u);
+    const uint32_t t2 = prmt(w2, w3, 0x5140u), t3 = prmt(w2, w3, 0x7362u);
+    o[0] = prmt(t0, t2, 0x5410u);
+    o[1] = prmt(t0, t2, 0x7632u);
+    o[2] = prmt(t1, t3, 0x5410u);
+    o[3] = prmt(t1, t3, 0x7632u);
 }
 
 template <int GRID>
@@ -767,15 +792,18 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
     gemm_fp4_kernel(const __grid_constant__ GemmArgs args) {
     using C = Fp4Cfg<GRID>;
     constexpr int BN = C::BN;
+    constexpr int NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::o_bar);
-    uint64_t *ready = full + C::NSTAGE;
-    uint64_t *empty = ready + C::NSTAGE;
-    uint64_t *acc_full = empty + C::NSTAGE;
+    uint64_t *ready = full + NS;
+    uint64_t *empty = ready + NS;
+    uint64_t *acc_full = empty + NS;
     uint64_t *acc_empty = acc_full + 1;
     uint64_t *drain = acc_empty + 1;
+    uint64_t *out_full = drain + 1;     // [2]: chunk staged by all epilogue threads
+    uint64_t *out_free = out_full + 2;  // [2]: the TMA store has read the chunk
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::o_misc);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::o_misc + 4);
     auto stage = [&](int s) { return smem + s * C::kStage; };
@@ -786,7 +814,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
     const int nraw = C::BKE / blk;                    // raw scale rows per stage
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < C::NSTAGE; ++i) {
+        for (int i = 0; i < NS; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&ready[i], C::NT);
             mbar_init(&empty[i], 1);
@@ -794,6 +822,10 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, C::NE);
         mbar_init(drain, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&out_full[i], 32 * C::NE);
+            mbar_init(&out_free[i], 1);
+        }
         *abort_flag = 0u;
         fence_barrier_init();
     }
@@ -802,6 +834,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
         tma_prefetch_desc(&args.tm_b_codes);
         tma_prefetch_desc(&args.tm_a_scales);
         tma_prefetch_desc(&args.tm_b_scales);
+        if (args.c_tma) tma_prefetch_desc(&args.tm_c);
     }
     if (warp == 1) tmem_alloc(tmem_slot, 512);
     tc_fence_before();
@@ -821,9 +854,8 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
                 const int32_t arow = static_cast<int32_t>(tl.g.a_row + tl.m0);
                 const int32_t brow = static_cast<int32_t>(tl.g.b_row + tl.n0);
                 for (int ks = 0; ks < nks; ++ks, ++it) {
-                    const int s = it % C::NSTAGE;
-                    if (!mbar_wait(&empty[s], ((it / C::NSTAGE) & 1) ^ 1, kErrTimeoutProducer,
-                                   abort_flag)) {
+                    const int s = it % NS;
+                    if (!mbar_wait(&empty[s], ((it / NS) & 1) ^ 1, kErrTimeoutProducer, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -837,11 +869,12 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
                     tma_load_2d(st + C::o_raw_b, &args.tm_b_scales, &full[s], brow, bcol / blk);
                 }
             }
-            for (int s = 0; s < C::NSTAGE; ++s) {
+            // Drain: the last copy into each stage has landed before exit.
+            for (int s = 0; s < NS; ++s) {
                 if (it > static_cast<uint32_t>(s)) {
-                    const uint32_t last = (it - 1 - s) / C::NSTAGE * C::NSTAGE + s;
+                    const uint32_t last = (it - 1 - s) / NS * NS + s;
                     uint32_t dummy = 0;
-                    mbar_wait(&full[s], (last / C::NSTAGE) & 1, kErrTimeoutDrain,
+                    mbar_wait(&full[s], (last / NS) & 1, kErrTimeoutDrain,
                               reinterpret_cast<volatile uint32_t *>(&dummy));
                 }
             }
@@ -859,8 +892,8 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
                 tc_fence_after();
                 bool first = true;
                 for (int ks = 0; ks < nks && ok; ++ks, ++it) {
-                    const int s = it % C::NSTAGE;
-                    if (!mbar_wait(&ready[s], (it / C::NSTAGE) & 1, kErrTimeoutMma, abort_flag)) {
+                    const int s = it % NS;
+                    if (!mbar_wait(&ready[s], (it / NS) & 1, kErrTimeoutMma, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -879,24 +912,20 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
                     const int64_t rem = tl.g.k - static_cast<int64_t>(ks) * C::BKE;
                     const int steps = rem >= C::BKE ? 2 : 1;
                     const uint32_t a0 = smem_addr(st + C::o_codes_a), b0 = smem_addr(st + C::o_codes_b);
+                    const uint32_t ac = smem_addr(smem + C::o_corr + (it & 1) * C::kCorr);
+                    const uint32_t bc = ac + C::kCodesA;
                     for (int j = 0; j < steps; ++j) {
                         const uint32_t sfa = sf0 + 4 * j, sfb = sf0 + 8 + 8 * j;
-                        if (GRID == 1) {
-                            umma_fp4_bs(tmem_base, umma_desc_sw64(a0 + 32 * j), umma_desc_sw64(b0 + 32 * j),
-                                        idesc, sfa, sfb, first ? 0u : 1u);
-                            first = false;
-                        } else {
-                            const uint32_t al = smem_addr(st + C::o_lo_a), bl = smem_addr(st + C::o_lo_b);
-                            const uint32_t as[2] = {a0, al}, bs[2] = {b0, bl};
-#pragma unroll
-                            for (int pa = 0; pa < 2; ++pa)
-#pragma unroll
-                                for (int pb = 0; pb < 2; ++pb) {
-                                    umma_fp4_bs(tmem_base, umma_desc_sw64(as[pa] + 32 * j),
-                                                umma_desc_sw64(bs[pb] + 32 * j), idesc, sfa, sfb,
-                                                first ? 0u : 1u);
-                                    first = false;
-                                }
+                        umma_fp4_bs(tmem_base, umma_desc_sw64(a0 + 32 * j), umma_desc_sw64(b0 + 32 * j),
+                                    idesc, sfa, sfb, first ? 0u : 1u);
+                        first = false;
+                        if (GRID == 0) {
+                            umma_fp4_bs(tmem_base, umma_desc_sw64(a0 + 32 * j), umma_desc_sw64(bc + 32 * j),
+                                        idesc, sfa, sfb, 1u);
+                            umma_fp4_bs(tmem_base, umma_desc_sw64(ac + 32 * j), umma_desc_sw64(b0 + 32 * j),
+                                        idesc, sfa, sfb, 1u);
+                            umma_fp4_bs(tmem_base, umma_desc_sw64(ac + 32 * j), umma_desc_sw64(bc + 32 * j),
+                                        idesc, sfa, sfb, 1u);
                         }
                     }
                     umma_commit(&empty[s]);
@@ -911,52 +940,71 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
         // ------------------------------------------------------------ transform
         const int tt = threadIdx.x - 64;
         constexpr int kThr = C::NT * 32;
+        constexpr int kUnits = (BM + BN) / 4 * 2;   // (4 rows, K step) scale units
         uint32_t it = 0;
         bool ok = true;
         for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
             const Tile tl = get_tile<BM, BN>(args, t);
             const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
             for (int ks = 0; ks < nks; ++ks, ++it) {
-                const int s = it % C::NSTAGE;
-                if (!warp_wait(&full[s], (it / C::NSTAGE) & 1, kErrTimeoutTransform, abort_flag)) {
+                const int s = it % NS;
+                if (!warp_wait(&full[s], (it / NS) & 1, kErrTimeoutTransform, abort_flag)) {
                     ok = false;
                     break;
                 }
-                uint8_t *st = stage(s);
-                // scale atoms: unit = (row, K-step j): 4 scales of 16 elements
-                for (int u = tt; u < 2 * (BM + BN); u += kThr) {
-                    const int j = u & 1;
-                    const int row = u >> 1;
-                    const bool isA = row < BM;
-                    const int r = isA ? row : row - BM;
-                    const uint8_t *raw = st + (isA ? C::o_raw_a : C::o_raw_b);
-                    const int rows = isA ? BM : BN;
-                    uint32_t word = 0;
-#pragma unroll
-                    for (int kb = 0; kb < 4; ++kb) {
-                        const int b16 = 4 * j + kb;                  // 16-element block in the stage
-                        const int braw = blk == 16 ? b16 : (b16 >> 1);
-                        word |= static_cast<uint32_t>(raw[braw * rows + r]) << (8 * kb);
+                // The correction slot of this stage was last read by the MMAs
+                // of iteration it - 2.
+                if (GRID == 0 && it >= 2) {
+                    const uint32_t p = it - 2;
+                    if (!warp_wait(&empty[p % NS], (p / NS) & 1, kErrTimeoutTransform, abort_flag)) {
+                        ok = false;
+                        break;
                     }
-                    uint8_t *atom = st + (isA ? C::o_sf_a + 512 * j
-                                              : C::o_sf_b + 1024 * j + 512 * (r >> 7));
-                    const int rr = r & 127;
-                    *reinterpret_cast<uint32_t *>(atom + 16 * (rr & 31) + 4 * (rr >> 5)) = word;
+                }
+                uint8_t *st = stage(s);
+                // Scale atoms: byte 16 (r % 32) + 4 ((r / 32) % 4) + kb of the
+                // atom of 128-row group r / 128 and K step j holds the factor
+                // of 16-element block 4 j + kb of row r.
+                for (int u = tt; u < kUnits; u += kThr) {
+                    const int j = u & 1;
+                    const int q4 = u >> 1;
+                    const bool isA = q4 < BM / 4;
+                    const int r0 = 4 * (isA ? q4 : q4 - BM / 4);
+                    const int rows = isA ? BM : BN;
+                    const uint8_t *raw = st + (isA ? C::o_raw_a : C::o_raw_b) + r0;
+                    uint32_t w[4];
+                    if (blk == 16) {
+#pragma unroll
+                        for (int kb = 0; kb < 4; ++kb)
+                            w[kb] = *reinterpret_cast<const uint32_t *>(raw + (4 * j + kb) * rows);
+                    } else {
+                        w[0] = w[1] = *reinterpret_cast<const uint32_t *>(raw + (2 * j) * rows);
+                        w[2] = w[3] = *reinterpret_cast<const uint32_t *>(raw + (2 * j + 1) * rows);
+                    }
+                    uint32_t o[4];
+                    transpose4x4(w[0], w[1], w[2], w[3], o);
+                    uint8_t *atom = st + (isA ? C::o_sf_a + 512 * j : C::o_sf_b + 1024 * j + 512 * (r0 >> 7));
+                    const int rr = r0 & 127;
+                    uint8_t *dst = atom + 16 * (rr & 31) + 4 * (rr >> 5);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) *reinterpret_cast<uint32_t *>(dst + 16 * i) = o[i];
                 }
                 if (GRID == 0) {
-                    // E1M2 planes: 16-byte chunks of the code tiles, in place.
-                    for (int c = tt; c < (C::kCodesA + C::kCodesB) / 16; c += kThr) {
-                        const int off = c * 16;
-                        uint8_t *src = st + off;   // codes A then codes B are contiguous
-                        uint8_t *lo_dst = st + C::o_lo_a + off;
-                        uint4 w = *reinterpret_cast<const uint4 *>(src);
-                        uint4 h, l;
-                        split_e1m2(w.x, h.x, l.x);
-                        split_e1m2(w.y, h.y, l.y);
-                        split_e1m2(w.z, h.z, l.z);
-                        split_e1m2(w.w, h.w, l.w);
-                        *reinterpret_cast<uint4 *>(src) = h;
-                        *reinterpret_cast<uint4 *>(lo_dst) = l;
+                    // Correction planes of both code tiles (same swizzled
+                    // offsets; the function is per byte).
+                    constexpr int kChunks = C::kCorr / 16;
+                    static_assert(kChunks % kThr == 0, "whole chunks per thread");
+                    constexpr int kPer = kChunks / kThr;
+                    uint8_t *corr = smem + C::o_corr + (it & 1) * C::kCorr;
+                    uint4 w[kPer];
+#pragma unroll
+                    for (int i = 0; i < kPer; ++i)
+                        w[i] = *reinterpret_cast<const uint4 *>(st + 16 * (tt + i * kThr));
+#pragma unroll
+                    for (int i = 0; i < kPer; ++i) {
+                        const uint4 d = make_uint4(e1m2_correction(w[i].x), e1m2_correction(w[i].y),
+                                                   e1m2_correction(w[i].z), e1m2_correction(w[i].w));
+                        *reinterpret_cast<uint4 *>(corr + 16 * (tt + i * kThr)) = d;
                     }
                 }
                 fence_proxy_async_smem();
@@ -969,17 +1017,24 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
         const int q = warp & 3;
         const int row_in_tile = 32 * q + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-        // E1M2 planes carry k = 4 * level on both sides: 1/16 (exact).
+        const bool elected = threadIdx.x == 32 * (2 + C::NT);
+        // E1M2 operands carry k = 4 * level on both sides: 1/16 (exact).
         const float mult = __fmul_rn(__fmul_rn(*args.a_S, *args.b_S),
                                      args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f));
-        uint32_t tcount = 0;
-        for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
+        uint32_t tcount = 0, ecount = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
             const Tile tl = get_tile<BM, BN>(args, t);
             if (!warp_wait(acc_full, tcount & 1, kErrTimeoutEpilogue, abort_flag)) break;
             tc_fence_after();
             const int64_t row = tl.m0 + row_in_tile;
             const bool row_ok = row < tl.g.m;
             float *crow = args.c + (tl.g.c_row + row) * args.ldc + tl.g.c_col + tl.n0;
+            // TMA stores clip at the output's edges; a group's window has no
+            // tensor map of its own, so there only whole chunks go that way.
+            const bool grouped = args.groups != nullptr;
+            const bool tma_tile =
+                args.c_tma && (!grouped || (tl.m0 + BM <= tl.g.m && (tl.g.c_col & 3) == 0));
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
@@ -990,24 +1045,53 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(acc_empty);
                 }
-                if (!row_ok) continue;
                 const int64_t col0 = tl.n0 + 32 * c;
+                if (col0 >= tl.g.n) continue;
                 float v[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     v[i] = tl.g.k > 0 ? __fmul_rn(__uint_as_float(r[i]), mult) : 0.0f;
-                float *dst = crow + 32 * c;
-                const bool vec = (col0 + 32 <= tl.g.n) && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
-                if (vec) {
+                if (tma_tile && (!grouped || col0 + 32 <= tl.g.n)) {
+                    const int b = ecount & 1;
+                    const uint32_t use = ecount >> 1;
+                    if (use > 0 &&
+                        !warp_wait(&out_free[b], (use - 1) & 1, kErrTimeoutEpilogue, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *rowp = smem + C::o_out + b * C::kOutChunk + row_in_tile * 128;
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4)
-                        *reinterpret_cast<float4 *>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-                } else {
-                    for (int i = 0; i < 32; ++i)
-                        if (col0 + i < tl.g.n) dst[i] = v[i];
+                    for (int ch = 0; ch < 8; ++ch)
+                        *reinterpret_cast<float4 *>(rowp + ((ch ^ (row_in_tile & 7)) << 4)) =
+                            make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
+                    fence_proxy_async_smem();
+                    mbar_arrive(&out_full[b]);
+                    if (elected) {
+                        if (mbar_wait(&out_full[b], use & 1, kErrTimeoutEpilogue, abort_flag)) {
+                            tma_store_2d(&args.tm_c, smem + C::o_out + b * C::kOutChunk,
+                                         static_cast<int32_t>(tl.g.c_col + col0),
+                                         static_cast<int32_t>(tl.g.c_row + tl.m0));
+                            bulk_commit_group();
+                            bulk_wait_group_read<1>();
+                            if (ecount > 0) mbar_arrive(&out_free[(ecount - 1) & 1]);
+                        }
+                    }
+                    ++ecount;
+                } else if (row_ok) {
+                    float *dst = crow + 32 * c;
+                    const bool vec = (col0 + 32 <= tl.g.n) && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
+                    if (vec) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4)
+                            *reinterpret_cast<float4 *>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                    } else {
+                        for (int i = 0; i < 32; ++i)
+                            if (col0 + i < tl.g.n) dst[i] = v[i];
+                    }
                 }
             }
         }
+        if (elected) bulk_wait_group<0>();
     }
 
     tc_fence_before();

@@ -48,6 +48,8 @@ struct GemmArgs {
     const GemmGroup *groups;              // device table or nullptr
     int num_groups;
     GemmGroup single;                     // used when groups == nullptr
+    CUtensorMap tm_c;                     // fp32 output, box 32 x 128 (mode 3)
+    int c_tma;                            // tm_c usable (aligned output)
 };
 
 // mode 0: fp32 block scales (per-block partial products, CUDA-core scaling)
