@@ -101,31 +101,36 @@ ufp4_status_t check_pair(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b, bool 
 
 std::atomic<int32_t> g_two_level_path{UFP4_GEMM_PATH_AUTO};
 
-ufp4_status_t encode_operand_maps(const ufp4_qtensor_t *q, int box_rows, int mode,
+ufp4_status_t encode_operand_maps(const ufp4_qtensor_t *q, int code_rows, int scale_rows, int mode,
                                   CUtensorMap *codes, CUtensorMap *scales) {
     const int64_t rows_t = q->rows > 0 ? q->rows : 1;
-    // mode 3 stages 128 K elements (64 code bytes, 64-byte swizzle) per step,
-    // the others 64 (32 bytes, 32-byte swizzle).
-    const bool native = mode == 3;
+    // The native kernels (modes 3, 4) stage 128 (E1M2) or 256 (E2M1) K
+    // elements per step: 64- or 128-byte code rows with the matching swizzle.
+    // The fp16-operand kernels stage 64 (32-byte rows, 32-byte swizzle).
+    const bool native = mode >= 3;
+    const int k_stage = native ? (q->cfg.grid == UFP4_GRID_E1M2 ? 128 : 256) : 64;
+    const uint32_t row_bytes = static_cast<uint32_t>(k_stage / 2);
+    const CUtensorMapSwizzle swz = row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                   : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                     : CU_TENSOR_MAP_SWIZZLE_32B;
     CUresult r = encode_tensor_map_2d(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, q->codes,
                                       static_cast<uint64_t>(q->kpad / 2),
                                       static_cast<uint64_t>(rows_t),
-                                      static_cast<uint64_t>(q->kpad / 2), native ? 64 : 32,
-                                      static_cast<uint32_t>(box_rows),
-                                      native ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+                                      static_cast<uint64_t>(q->kpad / 2), row_bytes,
+                                      static_cast<uint32_t>(code_rows), swz);
     if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
-    const int nblk_stage = (native ? 128 : 64) / q->cfg.block;
+    const int nblk_stage = k_stage / q->cfg.block;
     const uint64_t nblk = static_cast<uint64_t>(q->kpad / q->cfg.block);
     if (mode != 0) {
         r = encode_tensor_map_2d(scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, q->scales,
                                  static_cast<uint64_t>(q->scale_ld), nblk,
-                                 static_cast<uint64_t>(q->scale_ld), static_cast<uint32_t>(box_rows),
+                                 static_cast<uint64_t>(q->scale_ld), static_cast<uint32_t>(scale_rows),
                                  static_cast<uint32_t>(nblk_stage));
     } else {
         r = encode_tensor_map_2d(scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, q->scales,
                                  static_cast<uint64_t>(q->scale_ld), nblk,
                                  static_cast<uint64_t>(q->scale_ld) * 4,
-                                 static_cast<uint32_t>(box_rows), static_cast<uint32_t>(nblk_stage));
+                                 static_cast<uint32_t>(scale_rows), static_cast<uint32_t>(nblk_stage));
     }
     return r == CUDA_SUCCESS ? UFP4_OK : UFP4_ERR_CUDA;
 }
@@ -144,15 +149,17 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
         return UFP4_ERR_ALIGNMENT;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // fp32 block scales: per-block partials (mode 0).  Two-level scales: the
-    // native block-scaled FP4 kernel (mode 3) unless the caller picked one of
-    // the fp16-operand kernels (mode 1: one CTA per 128 x 256 tile, mode 2:
-    // CTA pairs on 256 x 256 tiles).
+    // native block-scaled FP4 kernel with one CTA per 128 x 256 tile (mode 3),
+    // or what the caller picked: the same on CTA pairs with 256 x 256 tiles
+    // (mode 4), the fp16-operand kernels (mode 1: one CTA per 128 x 256 tile,
+    // mode 2: CTA pairs).
     int mode = 0;
     if (a->cfg.scale_fmt == UFP4_SCALE_E4M3_X_FP32) {
         switch (g_two_level_path.load()) {
             case UFP4_GEMM_PATH_FP16: mode = 1; break;
             case UFP4_GEMM_PATH_FP16_PAIR: mode = 2; break;
             case UFP4_GEMM_PATH_NATIVE_FP4: mode = 3; break;
+            case UFP4_GEMM_PATH_NATIVE_FP4_PAIR: mode = 4; break;
             default: mode = 3; break;
         }
     }
@@ -170,10 +177,12 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
 
     GemmArgs args;
     memset(&args, 0, sizeof(args));
-    const int bn = (mode == 1 || mode == 3) ? 256 : 128;   // B rows staged per CTA
-    s = encode_operand_maps(a, 128, mode, &args.tm_a_codes, &args.tm_a_scales);
+    // B code rows staged per CTA; the native kernels stage the scales of all
+    // 256 B rows of a tile in each CTA.
+    const int bn = (mode == 1 || mode == 3) ? 256 : 128;
+    s = encode_operand_maps(a, 128, 128, mode, &args.tm_a_codes, &args.tm_a_scales);
     if (s != UFP4_OK) return s;
-    s = encode_operand_maps(b, bn, mode, &args.tm_b_codes, &args.tm_b_scales);
+    s = encode_operand_maps(b, bn, mode >= 3 ? 256 : bn, mode, &args.tm_b_codes, &args.tm_b_scales);
     if (s != UFP4_OK) return s;
     args.a_S = a->tensor_scale;
     args.b_S = b->tensor_scale;
@@ -186,7 +195,7 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
     args.single.m = m;
     args.single.n = n;
     args.single.k = a->kpad;
-    if (mode == 3 && aligned16(c) && ldc % 4 == 0) {
+    if (mode >= 3 && aligned16(c) && ldc % 4 == 0) {
         // Output tensor map for the TMA-store epilogue: the exact m x n window
         // of a single problem (stores clip at its edges); for a group table
         // the row count is not known here, so the map spans ldc columns and
@@ -359,7 +368,7 @@ ufp4_status_t ufp4_grouped_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b
 }
 
 ufp4_status_t ufp4_set_two_level_gemm_path(int32_t path) {
-    if (path < UFP4_GEMM_PATH_AUTO || path > UFP4_GEMM_PATH_NATIVE_FP4) return UFP4_ERR_INVALID_ARG;
+    if (path < UFP4_GEMM_PATH_AUTO || path > UFP4_GEMM_PATH_NATIVE_FP4_PAIR) return UFP4_ERR_INVALID_ARG;
     g_two_level_path.store(path);
     return UFP4_OK;
 }

@@ -700,7 +700,7 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Native block-scaled FP4 path for two-level scales (mode 3).
+// Native block-scaled FP4 path for two-level scales (modes 3 and 4).
 //
 // kind::mxf4nvf4 multiplies E2M1 operands scaled per 16 elements by UE4M3
 // factors, which is exactly an E2M1 operand under the two-level scales (the
@@ -713,27 +713,33 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
 // same scale factors, the raw code tiles used as they arrived and only the
 // correction planes written by the transform warps (a per-byte bit function).
 //
-// Tile 128 x 256, 128 K elements (64 code bytes per row, 64-byte TMA
-// swizzle) per stage.  The transform warps permute the block-major E4M3
-// bytes into the 32-row x 16-byte atoms that tcgen05.cp moves to TMEM (a 4x4
-// byte transpose per 4 rows), and build the E1M2 correction planes into a
-// two-slot ring.  The epilogue stages 128 x 32 fp32 chunks in shared memory
-// (128-byte swizzle) and writes them with TMA stores.
-template <int GRID>
+// Tiles: 128 x 256 on one CTA (mode 3) or 256 x 256 on a CTA pair with
+// cta_group::2 MMAs (mode 4): rank r of the pair stages A rows [128 r, +128)
+// and B rows [128 r, +128) of the tile, holds accumulator rows [128 r, +128),
+// and both ranks hold the scale factors of all 256 B rows.  A stage covers
+// 128 K elements for E1M2 (64-byte code rows, 64-byte TMA swizzle) and 256
+// for E2M1 (128-byte rows and swizzle).  The transform warps permute the
+// block-major E4M3 bytes into the 32-row x 16-byte atoms that tcgen05.cp
+// moves to TMEM (a 4x4 byte transpose per 4 rows) and build the E1M2
+// correction planes into a two-slot ring.  The epilogue stages 128 x 32 fp32
+// chunks in shared memory (128-byte swizzle) and writes them by TMA store.
+template <int GRID, int CG>
 struct Fp4Cfg {
-    static constexpr int BN = 256;
-    static constexpr int BKE = 128;                 // K elements per stage
-    static constexpr int kRow = 64;                 // code bytes per row per stage
-    static constexpr int NS = GRID == 0 ? 4 : 6;    // TMA ring stages
-    static constexpr int ND = GRID == 0 ? 2 : 0;    // correction-plane slots
+    static constexpr int BN = 256;                  // tile columns (B rows)
+    static constexpr int BNh = BN / CG;             // B code rows staged per CTA
+    static constexpr int TM = BM * CG;              // tile rows
+    static constexpr int BKE = GRID == 0 ? 128 : 256;   // K elements per stage
+    static constexpr int kRow = BKE / 2;            // code bytes per row per stage
+    static constexpr int KST = BKE / 64;            // MMA K steps per stage
     static constexpr int NT = GRID == 0 ? 8 : 4;    // transform warps
     static constexpr int NE = 4;                    // epilogue warps
+    static constexpr int ND = GRID == 0 ? 2 : 0;    // correction-plane slots
     static constexpr int kCodesA = BM * kRow;
-    static constexpr int kCodesB = BN * kRow;
+    static constexpr int kCodesB = BNh * kRow;
     static constexpr int kRawA = BM * (BKE / 16);
     static constexpr int kRawB = BN * (BKE / 16);
-    static constexpr int kSfA = 2 * 512;            // 2 K steps x 1 row atom group
-    static constexpr int kSfB = 2 * 2 * 512;        // 2 K steps x 2 row atom groups
+    static constexpr int kSfA = KST * 512;          // one 128-row atom group per K step
+    static constexpr int kSfB = KST * 1024;         // two per K step
     static constexpr int o_codes_a = 0;
     static constexpr int o_codes_b = o_codes_a + kCodesA;
     static constexpr int o_raw_a = o_codes_b + kCodesB;
@@ -741,18 +747,24 @@ struct Fp4Cfg {
     static constexpr int o_sf_a = o_raw_b + kRawB;
     static constexpr int o_sf_b = o_sf_a + kSfA;
     static constexpr int kStage = (o_sf_b + kSfB + 1023) / 1024 * 1024;
-    static constexpr int kCorr = kCodesA + kCodesB;  // one correction slot
-    static constexpr int o_corr = NS * kStage;
+    static constexpr int kCorr = kCodesA + kCodesB; // one correction slot
     static constexpr int kOutChunk = BM * 32 * 4;   // 128 rows x 32 fp32
+    static constexpr int kSfColsPerStage = KST * 12;  // SFA 4 + SFB 8 per K step
+    static constexpr int kAccCols = 256;
+    static constexpr int kBudget = 232448 - 2048;   // barriers, alignment slack
+    static constexpr int kNsSmem = (kBudget - ND * kCorr - 2 * kOutChunk) / kStage;
+    static constexpr int kNsTmem = (512 - kAccCols) / kSfColsPerStage;
+    static constexpr int NS = kNsSmem < kNsTmem ? kNsSmem : kNsTmem;   // TMA ring stages
+    static constexpr int o_corr = NS * kStage;
     static constexpr int o_out = o_corr + ND * kCorr;
     static constexpr int o_bar = o_out + 2 * kOutChunk;
-    // full, ready, empty per stage; acc_full, acc_empty, drain; out_full[2], out_free[2]
-    static constexpr int kNumBars = 3 * NS + 3 + 4;
+    // full, ready, empty, tdone per stage; acc_full, acc_empty, edone, drain;
+    // out_full[2], out_free[2]
+    static constexpr int kNumBars = 4 * NS + 4 + 4;
     static constexpr int o_misc = o_bar + kNumBars * 8;
     static constexpr int kAlloc = o_misc + 64 + 1024;
     static constexpr int kThreads = 32 * (2 + NT + NE);
-    static constexpr int kSfColsPerStage = 24;      // SFA 2 x 4, SFB 2 x 8
-    static constexpr int kAccCols = 256;
+    static_assert(NS >= 2, "pipeline depth");
     static_assert(kAccCols + NS * kSfColsPerStage <= 512, "TMEM budget");
     static_assert(kAlloc <= 232448, "shared memory budget");
     static_assert(o_corr % 1024 == 0 && o_out % 1024 == 0, "swizzle alignment");
@@ -787,21 +799,61 @@ __device__ __forceinline__ void transpose4x4(uint32_t w0, uint32_t w1, uint32_t 
     o[3] = prmt(t1, t3, 0x7632u);
 }
 
-template <int GRID>
-__global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
+// K-major operand descriptor for the code tiles: 64- or 128-byte rows.
+template <int kRowBytes>
+__device__ __forceinline__ uint64_t code_desc(uint32_t addr) {
+    if constexpr (kRowBytes == 64) return umma_desc_sw64(addr);
+    else return umma_desc_sw128(addr);
+}
+
+// Arrive on the barrier at the same offset in CTA 0 of the cluster (plain
+// local arrive when this CTA is CTA 0 or there is no cluster).
+template <int CG>
+__device__ __forceinline__ void arrive_leader(uint64_t *bar, uint32_t rank) {
+    if (CG == 1 || rank == 0) mbar_arrive(bar);
+    else mbar_arrive_remote(bar, 0);
+}
+
+template <int CG>
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+    if constexpr (CG == 1) tmem_cp_32x128b_x4(taddr, sdesc);
+    else tmem_cp_32x128b_x4_pair(taddr, sdesc);
+}
+
+template <int CG>
+__device__ __forceinline__ void umma_fp4_bs_cg(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc,
+                                               uint32_t sfa, uint32_t sfb, uint32_t acc) {
+    if constexpr (CG == 1) umma_fp4_bs(d, ad, bd, idesc, sfa, sfb, acc);
+    else umma_fp4_bs_pair(d, ad, bd, idesc, sfa, sfb, acc);
+}
+
+// Completion of this thread's MMAs arrives on the barrier in every CTA of
+// the pair (or in this CTA).
+template <int CG>
+__device__ __forceinline__ void umma_commit_cg(uint64_t *bar) {
+    if constexpr (CG == 1) umma_commit(bar);
+    else umma_commit_pair_mc(bar, 0x3);
+}
+
+template <int GRID, int CG>
+__global__ void __launch_bounds__(Fp4Cfg<GRID, CG>::kThreads, 1)
     gemm_fp4_kernel(const __grid_constant__ GemmArgs args) {
-    using C = Fp4Cfg<GRID>;
+    using C = Fp4Cfg<GRID, CG>;
     constexpr int BN = C::BN;
+    constexpr int TM = C::TM;
     constexpr int NS = C::NS;
+    constexpr bool kPair = CG == 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::o_bar);
-    uint64_t *ready = full + NS;
-    uint64_t *empty = ready + NS;
-    uint64_t *acc_full = empty + NS;
-    uint64_t *acc_empty = acc_full + 1;
-    uint64_t *drain = acc_empty + 1;
+    uint64_t *ready = full + NS;        // in CTA 0: stage transformed (all CTAs)
+    uint64_t *empty = ready + NS;       // MMAs done with the stage (multicast commit)
+    uint64_t *tdone = empty + NS;       // this CTA's transform warps done (pairs)
+    uint64_t *acc_full = tdone + NS;
+    uint64_t *acc_empty = acc_full + 1; // in CTA 0: accumulators drained (all CTAs)
+    uint64_t *edone = acc_empty + 1;    // this CTA's epilogue warps drained (pairs)
+    uint64_t *drain = edone + 1;
     uint64_t *out_full = drain + 1;     // [2]: chunk staged by all epilogue threads
     uint64_t *out_free = out_full + 2;  // [2]: the TMA store has read the chunk
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::o_misc);
@@ -812,15 +864,20 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
     const int lane = threadIdx.x & 31;
     const int blk = args.block;                       // 16 or 32
     const int nraw = C::BKE / blk;                    // raw scale rows per stage
+    const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+    const int64_t unit = kPair ? (blockIdx.x >> 1) : blockIdx.x;
+    const int64_t nunits = kPair ? (gridDim.x >> 1) : gridDim.x;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&ready[i], C::NT);
+            mbar_init(&ready[i], kPair ? CG : C::NT);
             mbar_init(&empty[i], 1);
+            mbar_init(&tdone[i], C::NT);
         }
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, C::NE);
+        mbar_init(acc_empty, kPair ? CG : C::NE);
+        mbar_init(edone, C::NE);
         mbar_init(drain, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&out_full[i], 32 * C::NE);
@@ -836,22 +893,26 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
         tma_prefetch_desc(&args.tm_b_scales);
         if (args.c_tma) tma_prefetch_desc(&args.tm_c);
     }
-    if (warp == 1) tmem_alloc(tmem_slot, 512);
+    if (warp == 1) {
+        if constexpr (kPair) tmem_alloc_pair(tmem_slot, 512);
+        else tmem_alloc(tmem_slot, 512);
+    }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (kPair) cluster_sync();
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int64_t ntiles = total_tiles<BM, BN>(args);
+    const int64_t ntiles = total_tiles<TM, BN>(args);
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-                const Tile tl = get_tile<BM, BN>(args, t);
+            for (int64_t t = unit; t < ntiles && ok; t += nunits) {
+                const Tile tl = get_tile<TM, BN>(args, t);
                 const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
-                const int32_t arow = static_cast<int32_t>(tl.g.a_row + tl.m0);
+                const int32_t arow = static_cast<int32_t>(tl.g.a_row + tl.m0 + BM * rank);
                 const int32_t brow = static_cast<int32_t>(tl.g.b_row + tl.n0);
                 for (int ks = 0; ks < nks; ++ks, ++it) {
                     const int s = it % NS;
@@ -864,7 +925,8 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
                     uint8_t *st = stage(s);
                     mbar_arrive_expect_tx(&full[s], C::kCodesA + C::kCodesB + (BM + BN) * nraw);
                     tma_load_2d(st + C::o_codes_a, &args.tm_a_codes, &full[s], acol / 2, arow);
-                    tma_load_2d(st + C::o_codes_b, &args.tm_b_codes, &full[s], bcol / 2, brow);
+                    tma_load_2d(st + C::o_codes_b, &args.tm_b_codes, &full[s], bcol / 2,
+                                brow + C::BNh * static_cast<int32_t>(rank));
                     tma_load_2d(st + C::o_raw_a, &args.tm_a_scales, &full[s], arow, acol / blk);
                     tma_load_2d(st + C::o_raw_b, &args.tm_b_scales, &full[s], brow, bcol / blk);
                 }
@@ -880,20 +942,24 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ UMMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = umma_idesc_fp4_bs(BM, BN);
+        // ------------------------------------------------------------ UMMA issuer (CTA 0)
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = umma_idesc_fp4_bs(TM, BN);
+            auto wait_any = [&](uint64_t *bar, uint32_t parity) {
+                return kPair ? mbar_wait_cluster(bar, parity, kErrTimeoutMma, abort_flag)
+                             : mbar_wait(bar, parity, kErrTimeoutMma, abort_flag);
+            };
             uint32_t it = 0, tcount = 0;
             bool ok = true;
-            for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
-                const Tile tl = get_tile<BM, BN>(args, t);
+            for (int64_t t = unit; t < ntiles && ok; t += nunits, ++tcount) {
+                const Tile tl = get_tile<TM, BN>(args, t);
                 const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
-                if (!mbar_wait(acc_empty, (tcount & 1) ^ 1, kErrTimeoutMma, abort_flag)) break;
+                if (!wait_any(acc_empty, (tcount & 1) ^ 1)) break;
                 tc_fence_after();
                 bool first = true;
                 for (int ks = 0; ks < nks && ok; ++ks, ++it) {
                     const int s = it % NS;
-                    if (!mbar_wait(&ready[s], (it / NS) & 1, kErrTimeoutMma, abort_flag)) {
+                    if (!wait_any(&ready[s], (it / NS) & 1)) {
                         ok = false;
                         break;
                     }
@@ -901,38 +967,42 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
                     uint8_t *st = stage(s);
                     const uint32_t sf0 = tmem_base + C::kAccCols + s * C::kSfColsPerStage;
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        tmem_cp_32x128b_x4(sf0 + 4 * j, sf_atom_desc(smem_addr(st + C::o_sf_a + 512 * j)));
-                        tmem_cp_32x128b_x4(sf0 + 8 + 8 * j,
-                                           sf_atom_desc(smem_addr(st + C::o_sf_b + 1024 * j)));
-                        tmem_cp_32x128b_x4(sf0 + 12 + 8 * j,
-                                           sf_atom_desc(smem_addr(st + C::o_sf_b + 1024 * j + 512)));
+                    for (int j = 0; j < C::KST; ++j) {
+                        const uint32_t col = sf0 + 12 * j;
+                        const uint32_t sa = smem_addr(st + C::o_sf_a + 512 * j);
+                        const uint32_t sb = smem_addr(st + C::o_sf_b + 1024 * j);
+                        tmem_cp_sf<CG>(col, sf_atom_desc(sa));
+                        tmem_cp_sf<CG>(col + 4, sf_atom_desc(sb));
+                        tmem_cp_sf<CG>(col + 8, sf_atom_desc(sb + 512));
                     }
-                    // K steps of 64 in this stage (a tail may use only the first)
+                    // K steps of 64 in this stage (a tail uses only its own)
                     const int64_t rem = tl.g.k - static_cast<int64_t>(ks) * C::BKE;
-                    const int steps = rem >= C::BKE ? 2 : 1;
+                    const int steps = rem >= C::BKE ? C::KST : static_cast<int>((rem + 63) / 64);
                     const uint32_t a0 = smem_addr(st + C::o_codes_a), b0 = smem_addr(st + C::o_codes_b);
                     const uint32_t ac = smem_addr(smem + C::o_corr + (it & 1) * C::kCorr);
                     const uint32_t bc = ac + C::kCodesA;
                     for (int j = 0; j < steps; ++j) {
-                        const uint32_t sfa = sf0 + 4 * j, sfb = sf0 + 8 + 8 * j;
-                        umma_fp4_bs(tmem_base, umma_desc_sw64(a0 + 32 * j), umma_desc_sw64(b0 + 32 * j),
-                                    idesc, sfa, sfb, first ? 0u : 1u);
+                        const uint32_t sfa = sf0 + 12 * j, sfb = sfa + 4;
+                        const uint32_t dk = 32 * j;
+                        umma_fp4_bs_cg<CG>(tmem_base, code_desc<C::kRow>(a0 + dk), code_desc<C::kRow>(b0 + dk),
+                                           idesc, sfa, sfb, first ? 0u : 1u);
                         first = false;
                         if (GRID == 0) {
-                            umma_fp4_bs(tmem_base, umma_desc_sw64(a0 + 32 * j), umma_desc_sw64(bc + 32 * j),
-                                        idesc, sfa, sfb, 1u);
-                            umma_fp4_bs(tmem_base, umma_desc_sw64(ac + 32 * j), umma_desc_sw64(b0 + 32 * j),
-                                        idesc, sfa, sfb, 1u);
-                            umma_fp4_bs(tmem_base, umma_desc_sw64(ac + 32 * j), umma_desc_sw64(bc + 32 * j),
-                                        idesc, sfa, sfb, 1u);
+                            umma_fp4_bs_cg<CG>(tmem_base, code_desc<C::kRow>(a0 + dk),
+                                               code_desc<C::kRow>(bc + dk), idesc, sfa, sfb, 1u);
+                            umma_fp4_bs_cg<CG>(tmem_base, code_desc<C::kRow>(ac + dk),
+                                               code_desc<C::kRow>(b0 + dk), idesc, sfa, sfb, 1u);
+                            umma_fp4_bs_cg<CG>(tmem_base, code_desc<C::kRow>(ac + dk),
+                                               code_desc<C::kRow>(bc + dk), idesc, sfa, sfb, 1u);
                         }
                     }
-                    umma_commit(&empty[s]);
+                    umma_commit_cg<CG>(&empty[s]);
                 }
-                if (ok) umma_commit(acc_full);
+                if (ok) umma_commit_cg<CG>(acc_full);
             }
-            umma_commit(drain);
+            // Drain: every MMA issued here completes before TMEM is freed.
+            if constexpr (kPair) umma_commit_pair(drain);
+            else umma_commit(drain);
             uint32_t dummy = 0;
             mbar_wait(drain, 0, kErrTimeoutDrain, reinterpret_cast<volatile uint32_t *>(&dummy));
         }
@@ -940,11 +1010,11 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
         // ------------------------------------------------------------ transform
         const int tt = threadIdx.x - 64;
         constexpr int kThr = C::NT * 32;
-        constexpr int kUnits = (BM + BN) / 4 * 2;   // (4 rows, K step) scale units
+        constexpr int kUnits = (BM + BN) / 4 * C::KST;   // (4 rows, K step) scale units
         uint32_t it = 0;
         bool ok = true;
-        for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const Tile tl = get_tile<BM, BN>(args, t);
+        for (int64_t t = unit; t < ntiles && ok; t += nunits) {
+            const Tile tl = get_tile<TM, BN>(args, t);
             const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
             for (int ks = 0; ks < nks; ++ks, ++it) {
                 const int s = it % NS;
@@ -966,8 +1036,8 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
                 // atom of 128-row group r / 128 and K step j holds the factor
                 // of 16-element block 4 j + kb of row r.
                 for (int u = tt; u < kUnits; u += kThr) {
-                    const int j = u & 1;
-                    const int q4 = u >> 1;
+                    const int j = u % C::KST;
+                    const int q4 = u / C::KST;
                     const bool isA = q4 < BM / 4;
                     const int r0 = 4 * (isA ? q4 : q4 - BM / 4);
                     const int rows = isA ? BM : BN;
@@ -1007,9 +1077,25 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
                         *reinterpret_cast<uint4 *>(corr + 16 * (tt + i * kThr)) = d;
                     }
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ready[s]);
+                if constexpr (kPair) {
+                    // The MMAs of CTA 0 read this CTA's tiles: one relay
+                    // arrive per CTA after all of its transform warps.
+                    fence_proxy_async_cluster();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tdone[s]);
+                    if (tt == 0) {
+                        if (!mbar_wait(&tdone[s], (it / NS) & 1, kErrTimeoutTransform, abort_flag)) {
+                            ok = false;
+                        } else {
+                            arrive_leader<CG>(&ready[s], rank);
+                        }
+                    }
+                    __syncwarp();
+                } else {
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ready[s]);
+                }
             }
         }
     } else {
@@ -1023,18 +1109,19 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
                                      args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f));
         uint32_t tcount = 0, ecount = 0;
         bool ok = true;
-        for (int64_t t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
-            const Tile tl = get_tile<BM, BN>(args, t);
+        for (int64_t t = unit; t < ntiles && ok; t += nunits, ++tcount) {
+            const Tile tl = get_tile<TM, BN>(args, t);
             if (!warp_wait(acc_full, tcount & 1, kErrTimeoutEpilogue, abort_flag)) break;
             tc_fence_after();
-            const int64_t row = tl.m0 + row_in_tile;
+            const int64_t m0 = tl.m0 + BM * rank;     // this CTA's accumulator rows
+            const int64_t row = m0 + row_in_tile;
             const bool row_ok = row < tl.g.m;
             float *crow = args.c + (tl.g.c_row + row) * args.ldc + tl.g.c_col + tl.n0;
             // TMA stores clip at the output's edges; a group's window has no
             // tensor map of its own, so there only whole chunks go that way.
             const bool grouped = args.groups != nullptr;
             const bool tma_tile =
-                args.c_tma && (!grouped || (tl.m0 + BM <= tl.g.m && (tl.g.c_col & 3) == 0));
+                args.c_tma && (!grouped || (m0 + BM <= tl.g.m && (tl.g.c_col & 3) == 0));
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
@@ -1043,7 +1130,16 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
                 if (c == BN / 32 - 1) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(acc_empty);
+                    if constexpr (kPair) {
+                        if (lane == 0) mbar_arrive(edone);
+                        if (elected) {
+                            if (mbar_wait(edone, tcount & 1, kErrTimeoutEpilogue, abort_flag))
+                                arrive_leader<CG>(acc_empty, rank);
+                        }
+                        __syncwarp();
+                    } else {
+                        if (lane == 0) mbar_arrive(acc_empty);
+                    }
                 }
                 const int64_t col0 = tl.n0 + 32 * c;
                 if (col0 >= tl.g.n) continue;
@@ -1070,7 +1166,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
                         if (mbar_wait(&out_full[b], use & 1, kErrTimeoutEpilogue, abort_flag)) {
                             tma_store_2d(&args.tm_c, smem + C::o_out + b * C::kOutChunk,
                                          static_cast<int32_t>(tl.g.c_col + col0),
-                                         static_cast<int32_t>(tl.g.c_row + tl.m0));
+                                         static_cast<int32_t>(tl.g.c_row + m0));
                             bulk_commit_group();
                             bulk_wait_group_read<1>();
                             if (ecount > 0) mbar_arrive(&out_free[(ecount - 1) & 1]);
@@ -1095,32 +1191,45 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID>::kThreads, 1)
     }
 
     tc_fence_before();
-    __syncthreads();
+    if constexpr (kPair) cluster_sync();
+    else __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, 512);
+        if constexpr (kPair) tmem_dealloc_pair(tmem_base, 512);
+        else tmem_dealloc(tmem_base, 512);
     }
 }
 
-template <int GRID>
+template <int GRID, int CG>
 cudaError_t launch_fp4(const GemmArgs &args, int num_sms, cudaStream_t stream) {
-    using C = Fp4Cfg<GRID>;
+    using C = Fp4Cfg<GRID, CG>;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_fp4_kernel<GRID>,
+        cudaError_t e = cudaFuncSetAttribute(gemm_fp4_kernel<GRID, CG>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc);
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    int units = num_sms;
+    int units = num_sms / CG;
     if (args.groups == nullptr) {
         const GemmGroup &g = args.single;
-        const int64_t tiles = ((g.m + BM - 1) / BM) * ((g.n + C::BN - 1) / C::BN);
+        const int64_t tiles = ((g.m + C::TM - 1) / C::TM) * ((g.n + C::BN - 1) / C::BN);
         if (tiles < units) units = static_cast<int>(tiles);
     }
     if (units <= 0) return cudaSuccess;
-    gemm_fp4_kernel<GRID><<<units, C::kThreads, C::kAlloc, stream>>>(args);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(units * CG, 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_fp4_kernel<GRID, CG>, args);
 }
 
 template <int MODE, int GRID>
@@ -1170,9 +1279,12 @@ cudaError_t launch_gemm(const GemmArgs &args, int mode, int grid_kind, int num_s
         case 2:
             return grid_kind == 0 ? launch_impl<2, 0>(args, num_sms, stream)
                                   : launch_impl<2, 1>(args, num_sms, stream);
+        case 3:
+            return grid_kind == 0 ? launch_fp4<0, 1>(args, num_sms, stream)
+                                  : launch_fp4<1, 1>(args, num_sms, stream);
         default:
-            return grid_kind == 0 ? launch_fp4<0>(args, num_sms, stream)
-                                  : launch_fp4<1>(args, num_sms, stream);
+            return grid_kind == 0 ? launch_fp4<0, 2>(args, num_sms, stream)
+                                  : launch_fp4<1, 2>(args, num_sms, stream);
     }
 }
 

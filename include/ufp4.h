@@ -205,16 +205,20 @@ ufp4_status_t ufp4_grouped_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b
  *   UFP4_GEMM_PATH_FP16_PAIR  the same on a CTA pair (256 x 256 tiles);
  *   UFP4_GEMM_PATH_NATIVE_FP4 block-scaled FP4 MMA (kind::mxf4nvf4, UE4M3
  *                             factors per 16 elements); E1M2 codes are split
- *                             exactly into two E2M1 planes (four MMAs);
+ *                             exactly into two E2M1 planes (four MMAs); one
+ *                             CTA per 128 x 256 tile;
+ *   UFP4_GEMM_PATH_NATIVE_FP4_PAIR  the same on CTA pairs (cta_group::2,
+ *                             256 x 256 tiles);
  *   UFP4_GEMM_PATH_AUTO       the library's choice (default; currently the
- *                             native FP4 path).
+ *                             one-CTA native FP4 path).
  * The setting is process-wide and read at each GEMM call; fp32 block scales
  * are unaffected.  Errors: INVALID_ARG for an unknown path. */
 typedef enum {
     UFP4_GEMM_PATH_AUTO = 0,
     UFP4_GEMM_PATH_FP16 = 1,
     UFP4_GEMM_PATH_FP16_PAIR = 2,
-    UFP4_GEMM_PATH_NATIVE_FP4 = 3
+    UFP4_GEMM_PATH_NATIVE_FP4 = 3,
+    UFP4_GEMM_PATH_NATIVE_FP4_PAIR = 4
 } ufp4_gemm_path_t;
 ufp4_status_t ufp4_set_two_level_gemm_path(int32_t path);
 int32_t ufp4_get_two_level_gemm_path(void);
