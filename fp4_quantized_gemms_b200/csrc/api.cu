@@ -78,6 +78,10 @@ ufp4_status_t check_qtensor(const ufp4_qtensor_t *q) {
     }
     if (q->cfg.scale_fmt == UFP4_SCALE_E4M3_X_FP32 && q->tensor_scale == nullptr)
         return UFP4_ERR_INVALID_ARG;
+    if (q->corr != nullptr) {   // E1M2 correction plane: same layout as codes
+        if (q->cfg.grid != UFP4_GRID_E1M2) return UFP4_ERR_INVALID_ARG;
+        if (!aligned16(q->corr)) return UFP4_ERR_ALIGNMENT;
+    }
     if (q->rows > (int64_t(1) << 31) || q->kpad > (int64_t(1) << 31)) return UFP4_ERR_UNSUPPORTED;
     return UFP4_OK;
 }
@@ -104,11 +108,11 @@ std::atomic<int32_t> g_two_level_path{UFP4_GEMM_PATH_AUTO};
 ufp4_status_t encode_operand_maps(const ufp4_qtensor_t *q, int code_rows, int scale_rows, int mode,
                                   CUtensorMap *codes, CUtensorMap *scales) {
     const int64_t rows_t = q->rows > 0 ? q->rows : 1;
-    // The native kernels (modes 3, 4) stage 128 (E1M2) or 256 (E2M1) K
-    // elements per step: 64- or 128-byte code rows with the matching swizzle.
-    // The fp16-operand kernels stage 64 (32-byte rows, 32-byte swizzle).
+    // The native kernels (modes 3, 4) stage 128 K elements per step (64-byte
+    // code rows, 64-byte swizzle), the fp16-operand kernels 64 (32-byte rows,
+    // 32-byte swizzle).
     const bool native = mode >= 3;
-    const int k_stage = native ? (q->cfg.grid == UFP4_GRID_E1M2 ? 128 : 256) : 64;
+    const int k_stage = native ? 128 : 64;
     const uint32_t row_bytes = static_cast<uint32_t>(k_stage / 2);
     const CUtensorMapSwizzle swz = row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                    : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -149,8 +153,8 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
         return UFP4_ERR_ALIGNMENT;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // fp32 block scales: per-block partials (mode 0).  Two-level scales: the
-    // native block-scaled FP4 kernel with one CTA per 128 x 256 tile (mode 3),
-    // or what the caller picked: the same on CTA pairs with 256 x 256 tiles
+    // native block-scaled FP4 kernel with one CTA per 128 x 224 tile (mode 3),
+    // or what the caller picked: the same on CTA pairs with 256 x 224 tiles
     // (mode 4), the fp16-operand kernels (mode 1: one CTA per 128 x 256 tile,
     // mode 2: CTA pairs).
     int mode = 0;
@@ -177,12 +181,19 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
 
     GemmArgs args;
     memset(&args, 0, sizeof(args));
-    // B code rows staged per CTA; the native kernels stage the scales of all
-    // 256 B rows of a tile in each CTA.
-    const int bn = (mode == 1 || mode == 3) ? 256 : 128;
+    // B code rows staged per CTA: fp32-scale kernel 128, fp16 kernels 256
+    // (one CTA) or 128 (pairs), native kernels 224 or 112, with the scales of
+    // all 224 B rows of a tile in each CTA.
+    int bn = 128;
+    switch (mode) {
+        case 1: bn = 256; break;
+        case 3: bn = 224; break;
+        case 4: bn = 112; break;
+        default: bn = 128; break;
+    }
     s = encode_operand_maps(a, 128, 128, mode, &args.tm_a_codes, &args.tm_a_scales);
     if (s != UFP4_OK) return s;
-    s = encode_operand_maps(b, bn, mode >= 3 ? 256 : bn, mode, &args.tm_b_codes, &args.tm_b_scales);
+    s = encode_operand_maps(b, bn, mode >= 3 ? 224 : bn, mode, &args.tm_b_codes, &args.tm_b_scales);
     if (s != UFP4_OK) return s;
     args.a_S = a->tensor_scale;
     args.b_S = b->tensor_scale;
@@ -195,18 +206,21 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
     args.single.m = m;
     args.single.n = n;
     args.single.k = a->kpad;
-    if (mode >= 3 && aligned16(c) && ldc % 4 == 0) {
-        // Output tensor map for the TMA-store epilogue: the exact m x n window
-        // of a single problem (stores clip at its edges); for a group table
-        // the row count is not known here, so the map spans ldc columns and
-        // 2^30 rows and the kernel stores only chunks inside a group.
-        const uint64_t inner = groups_dev == nullptr ? static_cast<uint64_t>(n) : static_cast<uint64_t>(ldc);
-        const uint64_t outer = groups_dev == nullptr ? static_cast<uint64_t>(m) : (1ull << 30);
-        CUresult r = encode_tensor_map_2d(&args.tm_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c, inner, outer,
-                                          static_cast<uint64_t>(ldc) * 4, 32, 128,
-                                          CU_TENSOR_MAP_SWIZZLE_128B);
-        args.c_tma = r == CUDA_SUCCESS ? 1 : 0;
+    // E1M2 operands that carry correction planes: the native kernels load
+    // them with the codes (same box, same swizzle).
+    if (mode >= 3 && a->cfg.grid == UFP4_GRID_E1M2 && a->corr != nullptr && b->corr != nullptr) {
+        ufp4_qtensor_t ac = *a, bc = *b;
+        ac.codes = a->corr;
+        bc.codes = b->corr;
+        CUtensorMap scratch;
+        s = encode_operand_maps(&ac, 128, 128, mode, &args.tm_a_corr, &scratch);
+        if (s != UFP4_OK) return s;
+        s = encode_operand_maps(&bc, bn, 224, mode, &args.tm_b_corr, &scratch);
+        if (s != UFP4_OK) return s;
+        args.corr_in = 1;
     }
+    // Native kernels store 16-byte pieces when the output allows it.
+    args.c_vec = (aligned16(c) && ldc % 4 == 0) ? 1 : 0;
     cudaError_t e = launch_gemm(args, mode, a->cfg.grid, sm_count(), st);
     return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
 }
@@ -326,6 +340,7 @@ ufp4_status_t ufp4_rht_quantize(const void *x_dev, int64_t rows, int64_t cols, i
     a.kpad = out->kpad;
     a.scale_ld = out->scale_ld;
     a.codes = static_cast<uint8_t *>(out->codes);
+    a.corr = static_cast<uint8_t *>(out->corr);
     a.scales = out->scales;
     a.S_out = two_level ? out->tensor_scale : nullptr;
     a.amax_t = two_level ? tensor_amax_dev : nullptr;

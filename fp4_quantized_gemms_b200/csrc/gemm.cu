@@ -713,74 +713,78 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
 // same scale factors, the raw code tiles used as they arrived and only the
 // correction planes written by the transform warps (a per-byte bit function).
 //
-// Tiles: 128 x 256 on one CTA (mode 3) or 256 x 256 on a CTA pair with
+// Tiles: 128 x 224 on one CTA (mode 3) or 256 x 224 on a CTA pair with
 // cta_group::2 MMAs (mode 4): rank r of the pair stages A rows [128 r, +128)
-// and B rows [128 r, +128) of the tile, holds accumulator rows [128 r, +128),
-// and both ranks hold the scale factors of all 256 B rows.  A stage covers
-// 128 K elements for E1M2 (64-byte code rows, 64-byte TMA swizzle) and 256
-// for E2M1 (128-byte rows and swizzle).  The transform warps permute the
-// block-major E4M3 bytes into the 32-row x 16-byte atoms that tcgen05.cp
-// moves to TMEM (a 4x4 byte transpose per 4 rows) and build the E1M2
-// correction planes into a two-slot ring.  The epilogue stages 128 x 32 fp32
-// chunks in shared memory (128-byte swizzle) and writes them by TMA store.
-template <int GRID, int CG>
+// and B rows [112 r, +112) of the tile, holds accumulator rows [128 r, +128),
+// and both ranks hold the scale factors of all 224 B rows.  224 columns let
+// two accumulators share TMEM with the scale factors, so the epilogue of one
+// tile overlaps the MMAs of the next.  A stage covers 128 K elements
+// (64-byte code rows, 64-byte TMA swizzle).
+//
+// The transform warps write the scale factors into TMEM themselves
+// (tcgen05.st), so the tensor pipe runs MMAs only: a warp turns the
+// block-major E4M3 bytes of a 128-row group into a 32-row x 16-byte atom
+// (a 4x4 byte transpose per 4 rows) in its scratch and stores it into its
+// 32-lane quarter of the atom's 4 columns (the layout the MMA reads, the same
+// in all four quarters).  They also build the E1M2 correction planes.  Scale
+// factors and correction planes use two-slot rings, refilled once the MMAs
+// two stages back have completed.  The epilogue stages 128 x 32 fp32 chunks
+// in shared memory (128-byte swizzle) and writes them with coalesced 16-byte
+// stores.
+template <int GRID, int CG, bool CIN>
 struct Fp4Cfg {
-    static constexpr int BN = 256;                  // tile columns (B rows)
+    static constexpr int BN = 224;                  // tile columns (B rows)
     static constexpr int BNh = BN / CG;             // B code rows staged per CTA
     static constexpr int TM = BM * CG;              // tile rows
-    static constexpr int BKE = GRID == 0 ? 128 : 256;   // K elements per stage
+    static constexpr int BKE = 128;                 // K elements per stage
     static constexpr int kRow = BKE / 2;            // code bytes per row per stage
     static constexpr int KST = BKE / 64;            // MMA K steps per stage
-    static constexpr int NT = GRID == 0 ? 8 : 4;    // transform warps
+    static constexpr int NT = 8;                    // transform warps
     static constexpr int NE = 4;                    // epilogue warps
-    static constexpr int ND = GRID == 0 ? 2 : 0;    // correction-plane slots
+    // E1M2 correction planes: loaded with the codes (CIN) or built by the
+    // transform warps into a two-slot ring
+    static constexpr int ND = (GRID == 0 && !CIN) ? 2 : 0;
     static constexpr int kCodesA = BM * kRow;
     static constexpr int kCodesB = BNh * kRow;
     static constexpr int kRawA = BM * (BKE / 16);
     static constexpr int kRawB = BN * (BKE / 16);
-    static constexpr int kSfA = KST * 512;          // one 128-row atom group per K step
-    static constexpr int kSfB = KST * 1024;         // two per K step
+    static constexpr int kIn = CIN ? 2 : 1;         // code planes loaded per stage
     static constexpr int o_codes_a = 0;
     static constexpr int o_codes_b = o_codes_a + kCodesA;
-    static constexpr int o_raw_a = o_codes_b + kCodesB;
+    static constexpr int o_cin_a = o_codes_b + kCodesB;         // CIN only
+    static constexpr int o_cin_b = o_cin_a + kCodesA;
+    static constexpr int o_raw_a = o_codes_a + kIn * (kCodesA + kCodesB);
     static constexpr int o_raw_b = o_raw_a + kRawA;
-    static constexpr int o_sf_a = o_raw_b + kRawB;
-    static constexpr int o_sf_b = o_sf_a + kSfA;
-    static constexpr int kStage = (o_sf_b + kSfB + 1023) / 1024 * 1024;
-    static constexpr int kCorr = kCodesA + kCodesB; // one correction slot
+    static constexpr int kStage = (o_raw_b + kRawB + 1023) / 1024 * 1024;
+    static constexpr int kCorr = (kCodesA + kCodesB + 1023) / 1024 * 1024;  // one slot
     static constexpr int kOutChunk = BM * 32 * 4;   // 128 rows x 32 fp32
-    static constexpr int kSfColsPerStage = KST * 12;  // SFA 4 + SFB 8 per K step
-    static constexpr int kAccCols = 256;
+    // scale-factor atoms per stage: K step j, kind 0 = SFA, 1 / 2 = SFB rows
+    // [0, 128) / [128, 224)
+    static constexpr int kAtoms = 3 * KST;
+    static constexpr int kSubs = NT / 4;            // warps per TMEM lane quarter
+    static constexpr int kMine = kAtoms / kSubs;    // atoms one warp stores
+    static constexpr int kScr = NT * kMine * 512;   // per-warp atom scratch
+    static constexpr int kAccCols = 224;            // one accumulator
+    static constexpr int kSfCols = KST * 12;        // one scale-factor slot
+    static constexpr int kSfBase = 2 * kAccCols;
     static constexpr int kBudget = 232448 - 2048;   // barriers, alignment slack
-    static constexpr int kNsSmem = (kBudget - ND * kCorr - 2 * kOutChunk) / kStage;
-    static constexpr int kNsTmem = (512 - kAccCols) / kSfColsPerStage;
-    static constexpr int NS = kNsSmem < kNsTmem ? kNsSmem : kNsTmem;   // TMA ring stages
+    static constexpr int NS = (kBudget - ND * kCorr - 2 * kOutChunk - kScr) / kStage;
     static constexpr int o_corr = NS * kStage;
     static constexpr int o_out = o_corr + ND * kCorr;
-    static constexpr int o_bar = o_out + 2 * kOutChunk;
-    // full, ready, empty, tdone per stage; acc_full, acc_empty, edone, drain;
-    // out_full[2], out_free[2]
-    static constexpr int kNumBars = 4 * NS + 4 + 4;
+    static constexpr int o_scr = o_out + 2 * kOutChunk;
+    static constexpr int o_bar = o_scr + kScr;
+    // full, ready, empty, tdone per stage; acc_full[2], acc_empty[2], edone, drain
+    static constexpr int kNumBars = 4 * NS + 6;
     static constexpr int o_misc = o_bar + kNumBars * 8;
     static constexpr int kAlloc = o_misc + 64 + 1024;
     static constexpr int kThreads = 32 * (2 + NT + NE);
-    static_assert(NS >= 2, "pipeline depth");
-    static_assert(kAccCols + NS * kSfColsPerStage <= 512, "TMEM budget");
+    static_assert(kAtoms % kSubs == 0, "atoms per warp");
+    static_assert(NS >= 3, "pipeline depth");
+    static_assert(kSfBase + 2 * kSfCols <= 512, "TMEM budget");
     static_assert(kAlloc <= 232448, "shared memory budget");
     static_assert(o_corr % 1024 == 0 && o_out % 1024 == 0, "swizzle alignment");
+    static_assert(BN % 32 == 0 && BN > 128 && BN <= 256, "two SFB row groups, 32-column chunks");
 };
-
-// Correction plane of 8 E1M2 codes (sign copied, magnitude d(k) as E2M1):
-// d = 4 for k in {4,5,6}, 2 for k in {2,3,7}, and bit 0 = (k in {1,3}).
-__device__ __forceinline__ uint32_t e1m2_correction(uint32_t w) {
-    const uint32_t r1 = w >> 1, r2 = w >> 2, l1 = w << 1, l2 = w << 2;
-    const uint32_t d0 = w & ~r2 & 0x11111111u;       // b0 & ~b2
-    const uint32_t d1 = w & (~r1 | l1);              // at bit 1: b1 & (~b2 | b0)
-    const uint32_t d2 = w & ~(l1 & l2);              // at bit 2: b2 & ~(b1 & b0)
-    const uint32_t y = (d2 & 0x44444444u) | (d1 & ~0x44444444u);
-    const uint32_t z = (w & 0x88888888u) | (y & ~0x88888888u);
-    return (z & ~0x11111111u) | d0;
-}
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t d;
@@ -799,25 +803,12 @@ __device__ __forceinline__ void transpose4x4(uint32_t w0, uint32_t w1, uint32_t 
     o[3] = prmt(t1, t3, 0x7632u);
 }
 
-// K-major operand descriptor for the code tiles: 64- or 128-byte rows.
-template <int kRowBytes>
-__device__ __forceinline__ uint64_t code_desc(uint32_t addr) {
-    if constexpr (kRowBytes == 64) return umma_desc_sw64(addr);
-    else return umma_desc_sw128(addr);
-}
-
 // Arrive on the barrier at the same offset in CTA 0 of the cluster (plain
 // local arrive when this CTA is CTA 0 or there is no cluster).
 template <int CG>
 __device__ __forceinline__ void arrive_leader(uint64_t *bar, uint32_t rank) {
     if (CG == 1 || rank == 0) mbar_arrive(bar);
     else mbar_arrive_remote(bar, 0);
-}
-
-template <int CG>
-__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
-    if constexpr (CG == 1) tmem_cp_32x128b_x4(taddr, sdesc);
-    else tmem_cp_32x128b_x4_pair(taddr, sdesc);
 }
 
 template <int CG>
@@ -835,10 +826,10 @@ __device__ __forceinline__ void umma_commit_cg(uint64_t *bar) {
     else umma_commit_pair_mc(bar, 0x3);
 }
 
-template <int GRID, int CG>
-__global__ void __launch_bounds__(Fp4Cfg<GRID, CG>::kThreads, 1)
+template <int GRID, int CG, bool CIN>
+__global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
     gemm_fp4_kernel(const __grid_constant__ GemmArgs args) {
-    using C = Fp4Cfg<GRID, CG>;
+    using C = Fp4Cfg<GRID, CG, CIN>;
     constexpr int BN = C::BN;
     constexpr int TM = C::TM;
     constexpr int NS = C::NS;
@@ -850,12 +841,10 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG>::kThreads, 1)
     uint64_t *ready = full + NS;        // in CTA 0: stage transformed (all CTAs)
     uint64_t *empty = ready + NS;       // MMAs done with the stage (multicast commit)
     uint64_t *tdone = empty + NS;       // this CTA's transform warps done (pairs)
-    uint64_t *acc_full = tdone + NS;
-    uint64_t *acc_empty = acc_full + 1; // in CTA 0: accumulators drained (all CTAs)
-    uint64_t *edone = acc_empty + 1;    // this CTA's epilogue warps drained (pairs)
+    uint64_t *acc_full = tdone + NS;    // [2]
+    uint64_t *acc_empty = acc_full + 2; // [2], in CTA 0: accumulator drained (all CTAs)
+    uint64_t *edone = acc_empty + 2;    // this CTA's epilogue warps drained (pairs)
     uint64_t *drain = edone + 1;
-    uint64_t *out_full = drain + 1;     // [2]: chunk staged by all epilogue threads
-    uint64_t *out_free = out_full + 2;  // [2]: the TMA store has read the chunk
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::o_misc);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::o_misc + 4);
     auto stage = [&](int s) { return smem + s * C::kStage; };
@@ -875,14 +864,12 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG>::kThreads, 1)
             mbar_init(&empty[i], 1);
             mbar_init(&tdone[i], C::NT);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, kPair ? CG : C::NE);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], kPair ? CG : C::NE);
+        }
         mbar_init(edone, C::NE);
         mbar_init(drain, 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&out_full[i], 32 * C::NE);
-            mbar_init(&out_free[i], 1);
-        }
         *abort_flag = 0u;
         fence_barrier_init();
     }
@@ -891,7 +878,10 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG>::kThreads, 1)
         tma_prefetch_desc(&args.tm_b_codes);
         tma_prefetch_desc(&args.tm_a_scales);
         tma_prefetch_desc(&args.tm_b_scales);
-        if (args.c_tma) tma_prefetch_desc(&args.tm_c);
+        if (CIN) {
+            tma_prefetch_desc(&args.tm_a_corr);
+            tma_prefetch_desc(&args.tm_b_corr);
+        }
     }
     if (warp == 1) {
         if constexpr (kPair) tmem_alloc_pair(tmem_slot, 512);
@@ -923,10 +913,15 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG>::kThreads, 1)
                     const int32_t acol = static_cast<int32_t>(tl.g.a_col + ks * C::BKE);
                     const int32_t bcol = static_cast<int32_t>(tl.g.b_col + ks * C::BKE);
                     uint8_t *st = stage(s);
-                    mbar_arrive_expect_tx(&full[s], C::kCodesA + C::kCodesB + (BM + BN) * nraw);
+                    mbar_arrive_expect_tx(&full[s],
+                                          C::kIn * (C::kCodesA + C::kCodesB) + (BM + BN) * nraw);
+                    const int32_t brow_h = brow + C::BNh * static_cast<int32_t>(rank);
                     tma_load_2d(st + C::o_codes_a, &args.tm_a_codes, &full[s], acol / 2, arow);
-                    tma_load_2d(st + C::o_codes_b, &args.tm_b_codes, &full[s], bcol / 2,
-                                brow + C::BNh * static_cast<int32_t>(rank));
+                    tma_load_2d(st + C::o_codes_b, &args.tm_b_codes, &full[s], bcol / 2, brow_h);
+                    if (CIN) {
+                        tma_load_2d(st + C::o_cin_a, &args.tm_a_corr, &full[s], acol / 2, arow);
+                        tma_load_2d(st + C::o_cin_b, &args.tm_b_corr, &full[s], bcol / 2, brow_h);
+                    }
                     tma_load_2d(st + C::o_raw_a, &args.tm_a_scales, &full[s], arow, acol / blk);
                     tma_load_2d(st + C::o_raw_b, &args.tm_b_scales, &full[s], brow, bcol / blk);
                 }
@@ -954,8 +949,10 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG>::kThreads, 1)
             for (int64_t t = unit; t < ntiles && ok; t += nunits, ++tcount) {
                 const Tile tl = get_tile<TM, BN>(args, t);
                 const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
-                if (!wait_any(acc_empty, (tcount & 1) ^ 1)) break;
+                const int ab = tcount & 1;
+                if (!wait_any(&acc_empty[ab], ((tcount >> 1) & 1) ^ 1)) break;
                 tc_fence_after();
+                const uint32_t d_tmem = tmem_base + ab * C::kAccCols;
                 bool first = true;
                 for (int ks = 0; ks < nks && ok; ++ks, ++it) {
                     const int s = it % NS;
@@ -965,40 +962,35 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG>::kThreads, 1)
                     }
                     tc_fence_after();
                     uint8_t *st = stage(s);
-                    const uint32_t sf0 = tmem_base + C::kAccCols + s * C::kSfColsPerStage;
-#pragma unroll
-                    for (int j = 0; j < C::KST; ++j) {
-                        const uint32_t col = sf0 + 12 * j;
-                        const uint32_t sa = smem_addr(st + C::o_sf_a + 512 * j);
-                        const uint32_t sb = smem_addr(st + C::o_sf_b + 1024 * j);
-                        tmem_cp_sf<CG>(col, sf_atom_desc(sa));
-                        tmem_cp_sf<CG>(col + 4, sf_atom_desc(sb));
-                        tmem_cp_sf<CG>(col + 8, sf_atom_desc(sb + 512));
-                    }
+                    // scale factors of K step j: SFA at 12 j, SFB rows 0-127
+                    // at 12 j + 4, rows 128-223 at 12 j + 8 of slot it & 1
+                    // (written by the transform warps of each CTA)
+                    const uint32_t sf0 = tmem_base + C::kSfBase + (it & 1) * C::kSfCols;
                     // K steps of 64 in this stage (a tail uses only its own)
                     const int64_t rem = tl.g.k - static_cast<int64_t>(ks) * C::BKE;
                     const int steps = rem >= C::BKE ? C::KST : static_cast<int>((rem + 63) / 64);
                     const uint32_t a0 = smem_addr(st + C::o_codes_a), b0 = smem_addr(st + C::o_codes_b);
-                    const uint32_t ac = smem_addr(smem + C::o_corr + (it & 1) * C::kCorr);
+                    const uint32_t ac = CIN ? smem_addr(st + C::o_cin_a)
+                                            : smem_addr(smem + C::o_corr + (it & 1) * C::kCorr);
                     const uint32_t bc = ac + C::kCodesA;
                     for (int j = 0; j < steps; ++j) {
                         const uint32_t sfa = sf0 + 12 * j, sfb = sfa + 4;
                         const uint32_t dk = 32 * j;
-                        umma_fp4_bs_cg<CG>(tmem_base, code_desc<C::kRow>(a0 + dk), code_desc<C::kRow>(b0 + dk),
-                                           idesc, sfa, sfb, first ? 0u : 1u);
+                        umma_fp4_bs_cg<CG>(d_tmem, umma_desc_sw64(a0 + dk), umma_desc_sw64(b0 + dk), idesc,
+                                           sfa, sfb, first ? 0u : 1u);
                         first = false;
                         if (GRID == 0) {
-                            umma_fp4_bs_cg<CG>(tmem_base, code_desc<C::kRow>(a0 + dk),
-                                               code_desc<C::kRow>(bc + dk), idesc, sfa, sfb, 1u);
-                            umma_fp4_bs_cg<CG>(tmem_base, code_desc<C::kRow>(ac + dk),
-                                               code_desc<C::kRow>(b0 + dk), idesc, sfa, sfb, 1u);
-                            umma_fp4_bs_cg<CG>(tmem_base, code_desc<C::kRow>(ac + dk),
-                                               code_desc<C::kRow>(bc + dk), idesc, sfa, sfb, 1u);
+                            umma_fp4_bs_cg<CG>(d_tmem, umma_desc_sw64(a0 + dk), umma_desc_sw64(bc + dk),
+                                               idesc, sfa, sfb, 1u);
+                            umma_fp4_bs_cg<CG>(d_tmem, umma_desc_sw64(ac + dk), umma_desc_sw64(b0 + dk),
+                                               idesc, sfa, sfb, 1u);
+                            umma_fp4_bs_cg<CG>(d_tmem, umma_desc_sw64(ac + dk), umma_desc_sw64(bc + dk),
+                                               idesc, sfa, sfb, 1u);
                         }
                     }
                     umma_commit_cg<CG>(&empty[s]);
                 }
-                if (ok) umma_commit_cg<CG>(acc_full);
+                if (ok) umma_commit_cg<CG>(&acc_full[ab]);
             }
             // Drain: every MMA issued here completes before TMEM is freed.
             if constexpr (kPair) umma_commit_pair(drain);
@@ -1010,7 +1002,12 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG>::kThreads, 1)
         // ------------------------------------------------------------ transform
         const int tt = threadIdx.x - 64;
         constexpr int kThr = C::NT * 32;
-        constexpr int kUnits = (BM + BN) / 4 * C::KST;   // (4 rows, K step) scale units
+        constexpr int kChunks = (C::kCodesA + C::kCodesB) / 16;   // correction pieces
+        constexpr int kPer = (kChunks + kThr - 1) / kThr;
+        const int tw = warp - 2;
+        const int sub = tw >> 2;             // which of the warps of this lane quarter
+        uint8_t *scr = smem + C::o_scr + tw * (C::kMine * 512);
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
         uint32_t it = 0;
         bool ok = true;
         for (int64_t t = unit; t < ntiles && ok; t += nunits) {
@@ -1022,61 +1019,85 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG>::kThreads, 1)
                     ok = false;
                     break;
                 }
-                // The correction slot of this stage was last read by the MMAs
-                // of iteration it - 2.
-                if (GRID == 0 && it >= 2) {
+                // Slot it & 1 of the scale-factor and correction rings was
+                // last read by the MMAs of iteration it - 2.
+                if (it >= 2) {
                     const uint32_t p = it - 2;
                     if (!warp_wait(&empty[p % NS], (p / NS) & 1, kErrTimeoutTransform, abort_flag)) {
                         ok = false;
                         break;
                     }
                 }
-                uint8_t *st = stage(s);
-                // Scale atoms: byte 16 (r % 32) + 4 ((r / 32) % 4) + kb of the
-                // atom of 128-row group r / 128 and K step j holds the factor
-                // of 16-element block 4 j + kb of row r.
-                for (int u = tt; u < kUnits; u += kThr) {
-                    const int j = u % C::KST;
-                    const int q4 = u / C::KST;
-                    const bool isA = q4 < BM / 4;
-                    const int r0 = 4 * (isA ? q4 : q4 - BM / 4);
-                    const int rows = isA ? BM : BN;
-                    const uint8_t *raw = st + (isA ? C::o_raw_a : C::o_raw_b) + r0;
-                    uint32_t w[4];
-                    if (blk == 16) {
+                const uint8_t *st = stage(s);
+                // Loads first: raw scale words of this warp's atoms (lane
+                // builds rows 4 lane .. 4 lane + 3 of a 128-row group) and the
+                // code pieces this thread corrects.
+                uint32_t w[C::kMine][4];
 #pragma unroll
-                        for (int kb = 0; kb < 4; ++kb)
-                            w[kb] = *reinterpret_cast<const uint32_t *>(raw + (4 * j + kb) * rows);
+                for (int x = 0; x < C::kMine; ++x) {
+                    const int a = sub + C::kSubs * x;
+                    const int jk = a / 3, kind = a % 3;
+                    const int rows = kind == 0 ? BM : BN;
+                    const int r = 4 * lane + (kind == 2 ? 128 : 0);
+                    const uint8_t *raw = st + (kind == 0 ? C::o_raw_a : C::o_raw_b) + r;
+                    if (r < rows) {
+                        if (blk == 16) {
+#pragma unroll
+                            for (int kb = 0; kb < 4; ++kb)
+                                w[x][kb] = *reinterpret_cast<const uint32_t *>(raw + (4 * jk + kb) * rows);
+                        } else {
+                            w[x][0] = w[x][1] = *reinterpret_cast<const uint32_t *>(raw + (2 * jk) * rows);
+                            w[x][2] = w[x][3] =
+                                *reinterpret_cast<const uint32_t *>(raw + (2 * jk + 1) * rows);
+                        }
                     } else {
-                        w[0] = w[1] = *reinterpret_cast<const uint32_t *>(raw + (2 * j) * rows);
-                        w[2] = w[3] = *reinterpret_cast<const uint32_t *>(raw + (2 * j + 1) * rows);
+                        w[x][0] = w[x][1] = w[x][2] = w[x][3] = 0u;
                     }
-                    uint32_t o[4];
-                    transpose4x4(w[0], w[1], w[2], w[3], o);
-                    uint8_t *atom = st + (isA ? C::o_sf_a + 512 * j : C::o_sf_b + 1024 * j + 512 * (r0 >> 7));
-                    const int rr = r0 & 127;
-                    uint8_t *dst = atom + 16 * (rr & 31) + 4 * (rr >> 5);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) *reinterpret_cast<uint32_t *>(dst + 16 * i) = o[i];
                 }
-                if (GRID == 0) {
-                    // Correction planes of both code tiles (same swizzled
-                    // offsets; the function is per byte).
-                    constexpr int kChunks = C::kCorr / 16;
-                    static_assert(kChunks % kThr == 0, "whole chunks per thread");
-                    constexpr int kPer = kChunks / kThr;
-                    uint8_t *corr = smem + C::o_corr + (it & 1) * C::kCorr;
-                    uint4 w[kPer];
-#pragma unroll
-                    for (int i = 0; i < kPer; ++i)
-                        w[i] = *reinterpret_cast<const uint4 *>(st + 16 * (tt + i * kThr));
+                constexpr bool kBuild = GRID == 0 && !CIN;   // correction planes here
+                uint4 cw[kBuild ? kPer : 1];
+                if constexpr (kBuild) {
 #pragma unroll
                     for (int i = 0; i < kPer; ++i) {
-                        const uint4 d = make_uint4(e1m2_correction(w[i].x), e1m2_correction(w[i].y),
-                                                   e1m2_correction(w[i].z), e1m2_correction(w[i].w));
-                        *reinterpret_cast<uint4 *>(corr + 16 * (tt + i * kThr)) = d;
+                        const int idx = tt + i * kThr;
+                        if (idx < kChunks) cw[i] = *reinterpret_cast<const uint4 *>(st + 16 * idx);
                     }
                 }
+                // Scale atoms: byte 16 (r % 32) + 4 (r / 32) + kb holds the
+                // factor of 16-element block 4 jk + kb of row r.
+#pragma unroll
+                for (int x = 0; x < C::kMine; ++x) {
+                    uint32_t o[4];
+                    transpose4x4(w[x][0], w[x][1], w[x][2], w[x][3], o);
+                    uint8_t *dst = scr + x * 512 + 16 * ((4 * lane) & 31) + 4 * ((4 * lane) >> 5);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) *reinterpret_cast<uint32_t *>(dst + 16 * q4) = o[q4];
+                }
+                if constexpr (kBuild) {
+                    // Correction planes of both code tiles (same swizzled
+                    // offsets; the function is per byte).
+                    uint8_t *corr = smem + C::o_corr + (it & 1) * C::kCorr;
+#pragma unroll
+                    for (int i = 0; i < kPer; ++i) {
+                        const int idx = tt + i * kThr;
+                        if (idx < kChunks) {
+                            const uint4 d = make_uint4(e1m2_correction(cw[i].x), e1m2_correction(cw[i].y),
+                                                       e1m2_correction(cw[i].z), e1m2_correction(cw[i].w));
+                            *reinterpret_cast<uint4 *>(corr + 16 * idx) = d;
+                        }
+                    }
+                }
+                __syncwarp();
+                const uint32_t sfw = lane_base + C::kSfBase + (it & 1) * C::kSfCols;
+#pragma unroll
+                for (int x = 0; x < C::kMine; ++x) {
+                    const int a = sub + C::kSubs * x;
+                    const uint4 row = *reinterpret_cast<const uint4 *>(scr + x * 512 + 16 * lane);
+                    tmem_st_32x32b_x4(sfw + 12 * (a / 3) + 4 * (a % 3), row.x, row.y, row.z, row.w);
+                }
+                tmem_wait_st();
+                __syncwarp();
+                tc_fence_before();
                 if constexpr (kPair) {
                     // The MMAs of CTA 0 read this CTA's tiles: one relay
                     // arrive per CTA after all of its transform warps.
@@ -1101,93 +1122,92 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG>::kThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;
+        const int et = threadIdx.x - 32 * (2 + C::NT);   // 0 .. 127
         const int row_in_tile = 32 * q + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-        const bool elected = threadIdx.x == 32 * (2 + C::NT);
+        const bool elected = et == 0;
+        constexpr uint32_t kEpiThreads = 32 * C::NE;
         // E1M2 operands carry k = 4 * level on both sides: 1/16 (exact).
         const float mult = __fmul_rn(__fmul_rn(*args.a_S, *args.b_S),
                                      args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f));
         uint32_t tcount = 0, ecount = 0;
-        bool ok = true;
-        for (int64_t t = unit; t < ntiles && ok; t += nunits, ++tcount) {
+        for (int64_t t = unit; t < ntiles; t += nunits, ++tcount) {
             const Tile tl = get_tile<TM, BN>(args, t);
-            if (!warp_wait(acc_full, tcount & 1, kErrTimeoutEpilogue, abort_flag)) break;
+            const int ab = tcount & 1;
+            const bool ok = warp_wait(&acc_full[ab], (tcount >> 1) & 1, kErrTimeoutEpilogue, abort_flag);
+            // one decision for the four epilogue warps (they share barrier 1)
+            if (named_bar_or(1, kEpiThreads, !ok)) break;
             tc_fence_after();
             const int64_t m0 = tl.m0 + BM * rank;     // this CTA's accumulator rows
             const int64_t row = m0 + row_in_tile;
             const bool row_ok = row < tl.g.m;
             float *crow = args.c + (tl.g.c_row + row) * args.ldc + tl.g.c_col + tl.n0;
-            // TMA stores clip at the output's edges; a group's window has no
-            // tensor map of its own, so there only whole chunks go that way.
-            const bool grouped = args.groups != nullptr;
-            const bool tma_tile =
-                args.c_tma && (!grouped || (m0 + BM <= tl.g.m && (tl.g.c_col & 3) == 0));
+            const bool vec_tile = args.c_vec && (tl.g.c_col & 3) == 0;
+            const uint32_t acc = tmem_base + ab * C::kAccCols + lane_addr;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem_base + 32 * c + lane_addr, r);
+                tmem_ld_32x32b_x32(acc + 32 * c, r);
                 tmem_wait_ld();
                 if (c == BN / 32 - 1) {
+                    // accumulator drained: the MMAs of tile t + 2 may start
                     tc_fence_before();
                     __syncwarp();
                     if constexpr (kPair) {
                         if (lane == 0) mbar_arrive(edone);
                         if (elected) {
                             if (mbar_wait(edone, tcount & 1, kErrTimeoutEpilogue, abort_flag))
-                                arrive_leader<CG>(acc_empty, rank);
+                                arrive_leader<CG>(&acc_empty[ab], rank);
                         }
                         __syncwarp();
                     } else {
-                        if (lane == 0) mbar_arrive(acc_empty);
+                        if (lane == 0) mbar_arrive(&acc_empty[ab]);
                     }
                 }
                 const int64_t col0 = tl.n0 + 32 * c;
-                if (col0 >= tl.g.n) continue;
+                if (col0 >= tl.g.n) continue;             // the same for all threads
                 float v[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     v[i] = tl.g.k > 0 ? __fmul_rn(__uint_as_float(r[i]), mult) : 0.0f;
-                if (tma_tile && (!grouped || col0 + 32 <= tl.g.n)) {
-                    const int b = ecount & 1;
-                    const uint32_t use = ecount >> 1;
-                    if (use > 0 &&
-                        !warp_wait(&out_free[b], (use - 1) & 1, kErrTimeoutEpilogue, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t *rowp = smem + C::o_out + b * C::kOutChunk + row_in_tile * 128;
+                if (vec_tile) {
+                    // Stage the 128 x 32 chunk (128-byte rows, 16-byte pieces
+                    // XOR-swizzled by row), then write 4 whole rows per warp
+                    // instruction.  Two buffers: the barrier of chunk c + 1
+                    // orders every read of chunk c before chunk c + 2's writes.
+                    uint8_t *buf = smem + C::o_out + (ecount & 1) * C::kOutChunk;
+                    uint8_t *rowp = buf + row_in_tile * 128;
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch)
                         *reinterpret_cast<float4 *>(rowp + ((ch ^ (row_in_tile & 7)) << 4)) =
                             make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
-                    fence_proxy_async_smem();
-                    mbar_arrive(&out_full[b]);
-                    if (elected) {
-                        if (mbar_wait(&out_full[b], use & 1, kErrTimeoutEpilogue, abort_flag)) {
-                            tma_store_2d(&args.tm_c, smem + C::o_out + b * C::kOutChunk,
-                                         static_cast<int32_t>(tl.g.c_col + col0),
-                                         static_cast<int32_t>(tl.g.c_row + m0));
-                            bulk_commit_group();
-                            bulk_wait_group_read<1>();
-                            if (ecount > 0) mbar_arrive(&out_free[(ecount - 1) & 1]);
+                    named_bar_sync(1, kEpiThreads);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int p = et + 128 * k;
+                        const int rr = p >> 3, c16 = p & 7;
+                        const float4 val =
+                            *reinterpret_cast<const float4 *>(buf + rr * 128 + ((c16 ^ (rr & 7)) << 4));
+                        const int64_t grow = m0 + rr;
+                        const int64_t gcol = col0 + 4 * c16;
+                        if (grow < tl.g.m && gcol < tl.g.n) {
+                            float *dst = args.c + (tl.g.c_row + grow) * args.ldc + tl.g.c_col + gcol;
+                            if (gcol + 4 <= tl.g.n) {
+                                *reinterpret_cast<float4 *>(dst) = val;
+                            } else {
+                                const float e4[4] = {val.x, val.y, val.z, val.w};
+                                for (int e = 0; e < 4 && gcol + e < tl.g.n; ++e) dst[e] = e4[e];
+                            }
                         }
                     }
                     ++ecount;
                 } else if (row_ok) {
                     float *dst = crow + 32 * c;
-                    const bool vec = (col0 + 32 <= tl.g.n) && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
-                    if (vec) {
-#pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            *reinterpret_cast<float4 *>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-                    } else {
-                        for (int i = 0; i < 32; ++i)
-                            if (col0 + i < tl.g.n) dst[i] = v[i];
-                    }
+                    for (int i = 0; i < 32; ++i)
+                        if (col0 + i < tl.g.n) dst[i] = v[i];
                 }
             }
         }
-        if (elected) bulk_wait_group<0>();
     }
 
     tc_fence_before();
@@ -1200,12 +1220,12 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG>::kThreads, 1)
     }
 }
 
-template <int GRID, int CG>
+template <int GRID, int CG, bool CIN>
 cudaError_t launch_fp4(const GemmArgs &args, int num_sms, cudaStream_t stream) {
-    using C = Fp4Cfg<GRID, CG>;
+    using C = Fp4Cfg<GRID, CG, CIN>;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_fp4_kernel<GRID, CG>,
+        cudaError_t e = cudaFuncSetAttribute(gemm_fp4_kernel<GRID, CG, CIN>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc);
         if (e != cudaSuccess) return e;
         configured = true;
@@ -1229,7 +1249,7 @@ cudaError_t launch_fp4(const GemmArgs &args, int num_sms, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_fp4_kernel<GRID, CG>, args);
+    return cudaLaunchKernelEx(&cfg, gemm_fp4_kernel<GRID, CG, CIN>, args);
 }
 
 template <int MODE, int GRID>
@@ -1280,11 +1300,13 @@ cudaError_t launch_gemm(const GemmArgs &args, int mode, int grid_kind, int num_s
             return grid_kind == 0 ? launch_impl<2, 0>(args, num_sms, stream)
                                   : launch_impl<2, 1>(args, num_sms, stream);
         case 3:
-            return grid_kind == 0 ? launch_fp4<0, 1>(args, num_sms, stream)
-                                  : launch_fp4<1, 1>(args, num_sms, stream);
+            if (grid_kind == 1) return launch_fp4<1, 1, false>(args, num_sms, stream);
+            return args.corr_in ? launch_fp4<0, 1, true>(args, num_sms, stream)
+                                : launch_fp4<0, 1, false>(args, num_sms, stream);
         default:
-            return grid_kind == 0 ? launch_fp4<0, 2>(args, num_sms, stream)
-                                  : launch_fp4<1, 2>(args, num_sms, stream);
+            if (grid_kind == 1) return launch_fp4<1, 2, false>(args, num_sms, stream);
+            return args.corr_in ? launch_fp4<0, 2, true>(args, num_sms, stream)
+                                : launch_fp4<0, 2, false>(args, num_sms, stream);
     }
 }
 

@@ -528,6 +528,14 @@ __global__ void __launch_bounds__(kThreads) rht_quantize_kernel(const __grid_con
             uint4 *dst = reinterpret_cast<uint4 *>(a.codes + orow * (a.kpad / 2) + k0 / 2);
             dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
             dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+            if (GRID == 0 && a.corr != nullptr) {
+                // E1M2 correction plane for the block-scaled FP4 GEMM
+                uint4 *cdst = reinterpret_cast<uint4 *>(a.corr + orow * (a.kpad / 2) + k0 / 2);
+                cdst[0] = make_uint4(e1m2_correction(codes[0]), e1m2_correction(codes[1]),
+                                     e1m2_correction(codes[2]), e1m2_correction(codes[3]));
+                cdst[1] = make_uint4(e1m2_correction(codes[4]), e1m2_correction(codes[5]),
+                                     e1m2_correction(codes[6]), e1m2_correction(codes[7]));
+            }
             constexpr int kBlocks = 64 / BLK;
 #pragma unroll
             for (int b = 0; b < kBlocks; ++b) {

@@ -56,6 +56,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// E1M2 correction plane of 8 codes: an E1M2 magnitude k equals e(k) + d(k)
+// with e(k) the code's bits read as an E2M1 value {0,.5,1,1.5,2,3,4,6}[k]
+// and d(k) = {0,.5,1,1.5,2,2,2,1}[k], itself E2M1 (codes {0,1,2,3,4,4,4,2}).
+// Per nibble, sign copied: d = 4 for k in {4,5,6}, 2 for k in {2,3,7}, and
+// bit 0 = (k in {1,3}).
+__device__ __forceinline__ uint32_t e1m2_correction(uint32_t w) {
+    const uint32_t r1 = w >> 1, r2 = w >> 2, l1 = w << 1, l2 = w << 2;
+    const uint32_t d0 = w & ~r2 & 0x11111111u;       // b0 & ~b2
+    const uint32_t d1 = w & (~r1 | l1);              // at bit 1: b1 & (~b2 | b0)
+    const uint32_t d2 = w & ~(l1 & l2);              // at bit 2: b2 & ~(b1 & b0)
+    const uint32_t y = (d2 & 0x44444444u) | (d1 & ~0x44444444u);
+    const uint32_t z = (w & 0x88888888u) | (y & ~0x88888888u);
+    return (z & ~0x11111111u) | d0;
+}
+
 #ifdef UFP4_PIPELINE_KERNELS
 // ---------------------------------------------------------------------------
 // Device error word.  Bounded waits that give up OR a code in here and make
@@ -372,6 +387,37 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
 
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Register -> TMEM store: thread t writes 4 consecutive 32-bit columns of
+// lane (base + t).  Asynchronous; tmem_wait_st orders it before later reads.
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c,
+                                                  uint32_t d) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a),
+                 "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Named barrier over `count` threads that also ORs a predicate across them.
+__device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t count, bool pred) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(out)
+        : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
+        : "memory");
+    return out != 0;
+}
+
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+    asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // 32 lanes x 32 consecutive 32-bit columns; thread t receives lane (base+t).

@@ -14,6 +14,7 @@ struct QuantArgs {
     int64_t out_rows;    // rows of the K-major output
     int64_t K, kpad, scale_ld;
     uint8_t *codes;      // [out_rows][kpad/2]
+    uint8_t *corr;       // E1M2 correction plane, same layout, or nullptr
     void *scales;        // block-major [kpad/B][scale_ld], fp32 or E4M3
     float *S_out;        // two-level: receives S
     const float *amax_t; // two-level: rotated tensor amax
@@ -48,8 +49,9 @@ struct GemmArgs {
     const GemmGroup *groups;              // device table or nullptr
     int num_groups;
     GemmGroup single;                     // used when groups == nullptr
-    CUtensorMap tm_c;                     // fp32 output, box 32 x 128 (mode 3)
-    int c_tma;                            // tm_c usable (aligned output)
+    int c_vec;                            // c 16-byte aligned and ldc % 4 == 0
+    CUtensorMap tm_a_corr, tm_b_corr;     // E1M2 correction planes (corr_in)
+    int corr_in;                          // both operands carry correction planes
 };
 
 // mode 0: fp32 block scales (per-block partial products, CUDA-core scaling)

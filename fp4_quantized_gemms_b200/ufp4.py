@@ -51,7 +51,7 @@ class QTensorC(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("tensor_scale", ctypes.c_void_p), ("rows", ctypes.c_int64),
                 ("k", ctypes.c_int64), ("kpad", ctypes.c_int64), ("scale_ld", ctypes.c_int64),
-                ("cfg", QuantCfgC)]
+                ("cfg", QuantCfgC), ("corr", ctypes.c_void_p)]
 
 
 class GroupC(ctypes.Structure):
@@ -160,14 +160,22 @@ class QTensor:
     kpad: int
     scale_ld: int
     cfg: QuantConfig
+    corr: torch.Tensor | None = None    # uint8 [rows, kpad/2]: E1M2 correction plane
 
     def c(self) -> QTensorC:
         return QTensorC(self.codes.data_ptr(), self.scales.data_ptr(),
                         self.tensor_scale.data_ptr() if self.tensor_scale is not None else None,
-                        self.rows, self.k, self.kpad, self.scale_ld, self.cfg.c())
+                        self.rows, self.k, self.kpad, self.scale_ld, self.cfg.c(),
+                        self.corr.data_ptr() if self.corr is not None else None)
 
 
-def empty_qtensor(rows: int, k: int, cfg: QuantConfig, device="cuda") -> QTensor:
+def wants_corr(cfg: QuantConfig) -> bool:
+    """Operands the native block-scaled GEMM reads as two E2M1 planes."""
+    return cfg.grid == GRID_E1M2 and cfg.scale_fmt == SCALE_E4M3_X_FP32
+
+
+def empty_qtensor(rows: int, k: int, cfg: QuantConfig, device="cuda",
+                  with_corr: bool | None = None) -> QTensor:
     kpad, sld, _, _ = layout(rows, k, cfg)
     nblk = kpad // cfg.block
     codes = torch.empty((rows, kpad // 2), dtype=torch.uint8, device=device)
@@ -177,7 +185,10 @@ def empty_qtensor(rows: int, k: int, cfg: QuantConfig, device="cuda") -> QTensor
     else:
         scales = torch.empty((nblk, sld), dtype=torch.uint8, device=device)
         ts = torch.empty(1, dtype=torch.float32, device=device)
-    return QTensor(codes, scales, ts, rows, k, kpad, sld, cfg)
+    if with_corr is None:
+        with_corr = wants_corr(cfg)
+    corr = torch.empty_like(codes) if with_corr else None
+    return QTensor(codes, scales, ts, rows, k, kpad, sld, cfg, corr)
 
 
 # ---------------------------------------------------------------- entry points
@@ -196,14 +207,17 @@ def rht_amax(x: torch.Tensor, axis: int, hadamard_n: int,
 
 
 def rht_quantize(x: torch.Tensor, axis: int, cfg: QuantConfig,
-                 tensor_amax: torch.Tensor | None = None, out: QTensor | None = None) -> QTensor:
-    """Fused RHT + block scale + 4-bit rounding + packing of a bf16 operand."""
+                 tensor_amax: torch.Tensor | None = None, out: QTensor | None = None,
+                 with_corr: bool | None = None) -> QTensor:
+    """Fused RHT + block scale + 4-bit rounding + packing of a bf16 operand
+    (plus the E1M2 correction plane when with_corr, by default for E1M2
+    operands with two-level scales)."""
     _require_cuda(x, tensor_amax)
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     rows, cols = x.shape
     orows, k = (rows, cols) if axis == ALONG_COLS else (cols, rows)
     if out is None:
-        out = empty_qtensor(orows, k, cfg, device=x.device)
+        out = empty_qtensor(orows, k, cfg, device=x.device, with_corr=with_corr)
     if cfg.scale_fmt == SCALE_E4M3_X_FP32 and tensor_amax is None:
         tensor_amax = rht_amax(x, axis, cfg.hadamard_n, cfg.rht_sign_mask)
     qc = out.c()

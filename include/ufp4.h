@@ -44,6 +44,14 @@
  *                                      is e_b * S with S = *tensor_scale.
  *   The dequantized (rotated) value of element (r, t) is s * lvl(code); the
  *   Hadamard normalisation 1/n is applied once in the GEMM (n = 0: none).
+ *   corr      optional, E1M2 only: the same layout as codes, each nibble the
+ *             E2M1 code of d(k) = k - e(k), where e(k) is the code's bits read
+ *             as an E2M1 number (d = {0,.5,1,1.5,2,2,2,1}[k] as E2M1 codes
+ *             {0,1,2,3,4,4,4,2}, sign bit copied).  k = e(k) + d(k) exactly,
+ *             so the block-scaled FP4 GEMM multiplies E1M2 operands as two
+ *             E2M1 planes.  ufp4_rht_quantize writes it when non-NULL; the
+ *             GEMMs read it when both operands carry one (else they derive it
+ *             on the fly).  Must be NULL for E2M1 operands.
  */
 #ifndef UFP4_H
 #define UFP4_H
@@ -103,6 +111,7 @@ typedef struct {
     int64_t kpad;           /* k rounded up to 64                            */
     int64_t scale_ld;       /* rows rounded up to 64                         */
     ufp4_quant_cfg_t cfg;   /* how it was quantized                          */
+    void *corr;             /* device u8 [rows][kpad/2] or NULL, see below   */
 } ufp4_qtensor_t;
 
 /* One sub-problem of ufp4_grouped_gemm:
@@ -206,9 +215,9 @@ ufp4_status_t ufp4_grouped_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b
  *   UFP4_GEMM_PATH_NATIVE_FP4 block-scaled FP4 MMA (kind::mxf4nvf4, UE4M3
  *                             factors per 16 elements); E1M2 codes are split
  *                             exactly into two E2M1 planes (four MMAs); one
- *                             CTA per 128 x 256 tile;
+ *                             CTA per 128 x 224 tile;
  *   UFP4_GEMM_PATH_NATIVE_FP4_PAIR  the same on CTA pairs (cta_group::2,
- *                             256 x 256 tiles);
+ *                             256 x 224 tiles);
  *   UFP4_GEMM_PATH_AUTO       the library's choice (default; currently the
  *                             one-CTA native FP4 path).
  * The setting is process-wide and read at each GEMM call; fp32 block scales

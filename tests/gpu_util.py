@@ -46,7 +46,40 @@ def tensor_scale(q: ufp4.QTensor) -> float:
     return float(q.tensor_scale.cpu().numpy()[0]) if q.tensor_scale is not None else 1.0
 
 
+E2M1_VALUES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def expected_corr(codes: np.ndarray) -> np.ndarray:
+    """E1M2 correction-plane nibbles from E1M2 code nibbles: magnitude k =
+    e(k) + d(k) with e(k) the E2M1 value of the same bits, d(k) an E2M1 value
+    (its code returned here), sign copied."""
+    lut = np.zeros(16, dtype=np.int8)
+    for nib in range(16):
+        k, sign = nib & 7, nib & 8
+        d = k - E2M1_VALUES[k]
+        assert d in E2M1_VALUES, (k, d)
+        lut[nib] = sign | E2M1_VALUES.index(d)
+    return lut[codes.astype(np.int64) & 15]
+
+
+def unpack_plane(t: torch.Tensor, rows=None) -> np.ndarray:
+    c = t if rows is None else t[torch.as_tensor(rows, device=t.device)]
+    b = c.cpu().numpy()
+    out = np.empty((b.shape[0], b.shape[1] * 2), dtype=np.int8)
+    out[:, 0::2] = b & 0x0F
+    out[:, 1::2] = b >> 4
+    return out
+
+
 def assert_quant_equal(q: ufp4.QTensor, ref: oracle.QTensor, rows=None):
+    if q.corr is not None:
+        got_c = unpack_plane(q.corr, rows)
+        want_c = expected_corr(ref.codes)
+        if not np.array_equal(got_c, want_c):
+            bad = np.argwhere(got_c != want_c)
+            r, c = bad[0]
+            raise AssertionError(f"{len(bad)} correction nibbles differ; first at ({r},{c}): gpu "
+                                 f"{got_c[r, c]} expected {want_c[r, c]} (code {ref.codes[r, c]})")
     got = unpack_codes(q, rows)
     if not np.array_equal(got, ref.codes):
         bad = np.argwhere(got != ref.codes)

@@ -48,8 +48,9 @@ def test_struct_layouts_match_header(tmp_path):
 int main(void) {
   printf("%zu %zu %zu %zu %zu\\n", sizeof(ufp4_quant_cfg_t), offsetof(ufp4_quant_cfg_t, sr_seed),
          offsetof(ufp4_quant_cfg_t, rht_sign_mask), offsetof(ufp4_quant_cfg_t, scale_fmt), 0);
-  printf("%zu %zu %zu %zu\\n", sizeof(ufp4_qtensor_t), offsetof(ufp4_qtensor_t, rows),
-         offsetof(ufp4_qtensor_t, scale_ld), offsetof(ufp4_qtensor_t, cfg));
+  printf("%zu %zu %zu %zu %zu\\n", sizeof(ufp4_qtensor_t), offsetof(ufp4_qtensor_t, rows),
+         offsetof(ufp4_qtensor_t, scale_ld), offsetof(ufp4_qtensor_t, cfg),
+         offsetof(ufp4_qtensor_t, corr));
   printf("%zu %zu\\n", sizeof(ufp4_group_t), offsetof(ufp4_group_t, c_col));
   return 0;
 }
@@ -62,7 +63,7 @@ int main(void) {
     c3 = list(map(int, out[2].split()))
     Q, T, G = ufp4.QuantCfgC, ufp4.QTensorC, ufp4.GroupC
     assert c1[:4] == [ctypes.sizeof(Q), Q.sr_seed.offset, Q.rht_sign_mask.offset, Q.scale_fmt.offset]
-    assert c2 == [ctypes.sizeof(T), T.rows.offset, T.scale_ld.offset, T.cfg.offset]
+    assert c2 == [ctypes.sizeof(T), T.rows.offset, T.scale_ld.offset, T.cfg.offset, T.corr.offset]
     assert c3 == [ctypes.sizeof(G), G.c_col.offset]
 
 

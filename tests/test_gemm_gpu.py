@@ -155,3 +155,32 @@ def test_layer_config_sampled(gemm, fmt):
 def test_large_config_sampled(gemm, fmt, grid):
     """M=16384, K=8192, N=28672 (1% outlier channels x50): the largest layer."""
     _sampled(wl.LARGE, fmt, grid, gemm, n_rows=64, n_cols=64)
+
+
+@pytest.mark.parametrize("path", [ufp4.GEMM_PATH_NATIVE_FP4, ufp4.GEMM_PATH_NATIVE_FP4_PAIR,
+                                  ufp4.GEMM_PATH_FP16])
+@pytest.mark.parametrize("corr", [True, False])
+@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1])
+def test_two_level_kernel_families(path, corr, grid):
+    """Every kernel family for two-level scales gives the oracle's result, with
+    the E1M2 correction planes stored by the quantizer or derived in the GEMM;
+    shapes with partial tiles in M, N (224-wide tiles) and a K tail."""
+    if grid == ufp4.GRID_E2M1 and corr:
+        pytest.skip("correction planes exist for E1M2 only")
+    old = ufp4.get_two_level_gemm_path()
+    ufp4.set_two_level_gemm_path(path)
+    try:
+        for (M, N, K) in [(520, 700, 448), (130, 230, 200)]:
+            X = wl.normal_with_outlier_channels(M, K, 1.0, 2, 20.0)
+            W = wl.normal(N, K, 0.02, 2)
+            cfg = _cfg(grid=grid, fmt=ufp4.SCALE_E4M3_X_FP32)
+            x, w = to_dev(X), to_dev(W)
+            qx = ufp4.rht_quantize(x, C, cfg, with_corr=corr)
+            qw = ufp4.rht_quantize(w, C, cfg, with_corr=corr)
+            oc = oracle_cfg(cfg)
+            rx = oracle.quantize(X, C, oc, tensor_amax=oracle.rht_amax(X, C, 16, cfg.rht_sign_mask))
+            rw = oracle.quantize(W, C, oc, tensor_amax=oracle.rht_amax(W, C, 16, cfg.rht_sign_mask))
+            assert (qx.corr is not None) == corr
+            _check_full(qx, rx, qw, rw, ufp4.gemm_fprop)
+    finally:
+        ufp4.set_two_level_gemm_path(old)
