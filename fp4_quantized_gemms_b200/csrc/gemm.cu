@@ -722,15 +722,16 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
 // (64-byte code rows, 64-byte TMA swizzle).
 //
 // The transform warps write the scale factors into TMEM themselves
-// (tcgen05.st), so the tensor pipe runs MMAs only: a warp turns the
-// block-major E4M3 bytes of a 128-row group into a 32-row x 16-byte atom
-// (a 4x4 byte transpose per 4 rows) in its scratch and stores it into its
-// 32-lane quarter of the atom's 4 columns (the layout the MMA reads, the same
-// in all four quarters).  They also build the E1M2 correction planes.  Scale
-// factors and correction planes use two-slot rings, refilled once the MMAs
-// two stages back have completed.  The epilogue stages 128 x 32 fp32 chunks
-// in shared memory (128-byte swizzle) and writes them with coalesced 16-byte
-// stores.
+// (tcgen05.st), so the tensor pipe runs MMAs only: for each 128-row group and
+// K step, lane i of every 32-lane quarter holds, in 4 consecutive columns,
+// the 4 block factors of rows i, 32 + i, 64 + i and 96 + i (the layout the
+// MMA reads, the same in all four quarters); a warp builds an atom with a
+// 4x4 byte transpose per 4 rows in its scratch.  E1M2 correction planes are
+// loaded with the codes
+// when the quantizer stored them, else the transform builds them.  Scale
+// factors and built planes use two-slot rings, refilled once the MMAs two
+// stages back have completed.  The epilogue stages 128 x 32 fp32 chunks in
+// shared memory and writes them with coalesced 16-byte stores.
 template <int GRID, int CG, bool CIN>
 struct Fp4Cfg {
     static constexpr int BN = 224;                  // tile columns (B rows)
@@ -757,7 +758,6 @@ struct Fp4Cfg {
     static constexpr int o_raw_b = o_raw_a + kRawA;
     static constexpr int kStage = (o_raw_b + kRawB + 1023) / 1024 * 1024;
     static constexpr int kCorr = (kCodesA + kCodesB + 1023) / 1024 * 1024;  // one slot
-    static constexpr int kOutChunk = BM * 32 * 4;   // 128 rows x 32 fp32
     // scale-factor atoms per stage: K step j, kind 0 = SFA, 1 / 2 = SFB rows
     // [0, 128) / [128, 224)
     static constexpr int kAtoms = 3 * KST;
@@ -768,10 +768,11 @@ struct Fp4Cfg {
     static constexpr int kSfCols = KST * 12;        // one scale-factor slot
     static constexpr int kSfBase = 2 * kAccCols;
     static constexpr int kBudget = 232448 - 2048;   // barriers, alignment slack
-    static constexpr int NS = (kBudget - ND * kCorr - 2 * kOutChunk - kScr) / kStage;
+    static constexpr int kOutChunk = BM * 32 * 4;   // epilogue staging: 128 rows x 32 fp32
+    static constexpr int NS = (kBudget - ND * kCorr - kOutChunk - kScr) / kStage;
     static constexpr int o_corr = NS * kStage;
     static constexpr int o_out = o_corr + ND * kCorr;
-    static constexpr int o_scr = o_out + 2 * kOutChunk;
+    static constexpr int o_scr = o_out + kOutChunk;
     static constexpr int o_bar = o_scr + kScr;
     // full, ready, empty, tdone per stage; acc_full[2], acc_empty[2], edone, drain
     static constexpr int kNumBars = 4 * NS + 6;
@@ -779,7 +780,7 @@ struct Fp4Cfg {
     static constexpr int kAlloc = o_misc + 64 + 1024;
     static constexpr int kThreads = 32 * (2 + NT + NE);
     static_assert(kAtoms % kSubs == 0, "atoms per warp");
-    static_assert(NS >= 3, "pipeline depth");
+    static_assert(NS >= 4, "pipeline depth");
     static_assert(kSfBase + 2 * kSfCols <= 512, "TMEM budget");
     static_assert(kAlloc <= 232448, "shared memory budget");
     static_assert(o_corr % 1024 == 0 && o_out % 1024 == 0, "swizzle alignment");
@@ -1121,16 +1122,22 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // Thread = accumulator row.  Each 128 x 32 fp32 chunk is staged in
+        // shared memory (128-byte rows, 16-byte pieces XOR-swizzled by row)
+        // and written 4 whole rows per warp instruction, keeping the load /
+        // store unit free for the transform warps.  The double-buffered
+        // accumulator lets these stores overlap the next tile.
         const int q = warp & 3;
         const int et = threadIdx.x - 32 * (2 + C::NT);   // 0 .. 127
         const int row_in_tile = 32 * q + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
         const bool elected = et == 0;
         constexpr uint32_t kEpiThreads = 32 * C::NE;
+        uint8_t *buf = smem + C::o_out;
         // E1M2 operands carry k = 4 * level on both sides: 1/16 (exact).
         const float mult = __fmul_rn(__fmul_rn(*args.a_S, *args.b_S),
                                      args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f));
-        uint32_t tcount = 0, ecount = 0;
+        uint32_t tcount = 0;
         for (int64_t t = unit; t < ntiles; t += nunits, ++tcount) {
             const Tile tl = get_tile<TM, BN>(args, t);
             const int ab = tcount & 1;
@@ -1171,17 +1178,12 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                 for (int i = 0; i < 32; ++i)
                     v[i] = tl.g.k > 0 ? __fmul_rn(__uint_as_float(r[i]), mult) : 0.0f;
                 if (vec_tile) {
-                    // Stage the 128 x 32 chunk (128-byte rows, 16-byte pieces
-                    // XOR-swizzled by row), then write 4 whole rows per warp
-                    // instruction.  Two buffers: the barrier of chunk c + 1
-                    // orders every read of chunk c before chunk c + 2's writes.
-                    uint8_t *buf = smem + C::o_out + (ecount & 1) * C::kOutChunk;
                     uint8_t *rowp = buf + row_in_tile * 128;
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch)
                         *reinterpret_cast<float4 *>(rowp + ((ch ^ (row_in_tile & 7)) << 4)) =
                             make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
-                    named_bar_sync(1, kEpiThreads);
+                    named_bar_sync(1, kEpiThreads);          // chunk staged
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const int p = et + 128 * k;
@@ -1200,7 +1202,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                             }
                         }
                     }
-                    ++ecount;
+                    named_bar_sync(1, kEpiThreads);          // chunk read out
                 } else if (row_ok) {
                     float *dst = crow + 32 * c;
                     for (int i = 0; i < 32; ++i)
