@@ -16,7 +16,8 @@
 
 namespace ufp4 {
 
-cudaError_t read_and_clear_error_word(uint32_t *out);   // gemm.cu
+cudaError_t read_and_clear_error_word(uint32_t *out);            // gemm.cu
+cudaError_t quantize_read_and_clear_error_word(uint32_t *out);   // quantize.cu
 
 namespace {
 
@@ -393,6 +394,9 @@ int32_t ufp4_get_two_level_gemm_path(void) { return g_two_level_path.load(); }
 ufp4_status_t ufp4_check_device_status(void) {
     uint32_t w = 0;
     if (read_and_clear_error_word(&w) != cudaSuccess) return UFP4_ERR_CUDA;
+    uint32_t wq = 0;
+    if (quantize_read_and_clear_error_word(&wq) != cudaSuccess) return UFP4_ERR_CUDA;
+    w |= wq;
     return w == 0 ? UFP4_OK : UFP4_ERR_DEVICE_TIMEOUT;
 }
 

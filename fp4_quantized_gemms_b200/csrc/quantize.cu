@@ -25,6 +25,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#define UFP4_PIPELINE_KERNELS 1
 #include "ufp4_device.cuh"
 #include "ufp4_internal.h"
 
@@ -232,10 +233,21 @@ __device__ __forceinline__ uint32_t cvt_e2m1x4(float a0, float a1, float a2, flo
     return out;
 }
 
+// The 16 values and 8 random words of a chunk, passed by value so that the
+// out-of-line exact path below keeps them in registers.
+struct Chunk16 {
+    float4 v0, v1, v2, v3;
+};
+struct Rand8 {
+    uint4 r0, r1;
+};
+
 // Exact path: every element decided by the fma boundary tests.
 template <int GRID, int RND>
-__device__ __noinline__ uint2 round_pack_exact(const float (&v)[16], const ScaleOut &sc,
-                                               const uint32_t (&rnd)[8]) {
+__device__ __noinline__ uint2 round_pack_exact(const Chunk16 c, const ScaleOut sc, const Rand8 rr) {
+    const float v[16] = {c.v0.x, c.v0.y, c.v0.z, c.v0.w, c.v1.x, c.v1.y, c.v1.z, c.v1.w,
+                         c.v2.x, c.v2.y, c.v2.z, c.v2.w, c.v3.x, c.v3.y, c.v3.z, c.v3.w};
+    const uint32_t rnd[8] = {rr.r0.x, rr.r0.y, rr.r0.z, rr.r0.w, rr.r1.x, rr.r1.y, rr.r1.z, rr.r1.w};
     uint32_t w0 = 0, w1 = 0;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -331,7 +343,12 @@ __device__ __forceinline__ uint2 round_pack(const float (&v)[16], const ScaleOut
     } else {
         risky = true;   // E2M1 SR: exact path only
     }
-    if (risky) return round_pack_exact<GRID, RND>(v, sc, rnd);
+    if (risky) {
+        const Chunk16 c{make_float4(v[0], v[1], v[2], v[3]), make_float4(v[4], v[5], v[6], v[7]),
+                        make_float4(v[8], v[9], v[10], v[11]), make_float4(v[12], v[13], v[14], v[15])};
+        const Rand8 rr{make_uint4(rnd[0], rnd[1], rnd[2], rnd[3]), make_uint4(rnd[4], rnd[5], rnd[6], rnd[7])};
+        return round_pack_exact<GRID, RND>(c, sc, rr);
+    }
     return make_uint2(canonical_zero(w[0]), canonical_zero(w[1]));
 }
 
@@ -350,18 +367,24 @@ __device__ __forceinline__ uint2 round_pack(const float (&v)[16], const ScaleOut
 // consecutive rows of each block) go straight to global memory.
 constexpr int kUnitRows = 256;
 constexpr int kStageBytes = kUnitRows * 64 * 2;   // 32 KB of bf16
-constexpr int kQuantSmem = 2 * kStageBytes + 1024 + 64;
+constexpr int kStages = 2;
+constexpr int kComputeWarps = kThreads / 32;
+constexpr int kCtaThreads = kThreads + 32;        // + one producer warp
+constexpr int kQuantSmem = kStages * kStageBytes + 1024 + 64;
 
 template <int AXIS, int NH, int BLK, int GRID, int RND, bool AMAX_ONLY>
-__global__ void __launch_bounds__(kThreads) rht_quantize_kernel(const __grid_constant__ QuantArgs a,
-                                                               const __grid_constant__ CUtensorMap tmap) {
+__global__ void __launch_bounds__(kCtaThreads, 3) rht_quantize_kernel(const __grid_constant__ QuantArgs a,
+                                                                  const __grid_constant__ CUtensorMap tmap) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + 2 * kStageBytes);
-    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + 2 * kStageBytes + 16);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
+    uint64_t *empty = full + kStages;
+    volatile uint32_t *abort_flag =
+        reinterpret_cast<volatile uint32_t *>(smem + kStages * kStageBytes + 16 * kStages);
     const int t = threadIdx.x;
     const int lane = t & 31;
+    const int warp = t >> 5;
     const int64_t nseg = a.kpad / 64;
     const int64_t nrb = (a.out_rows + kUnitRows - 1) / kUnitRows;
     const int64_t nunits = nseg * nrb;
@@ -393,16 +416,35 @@ __global__ void __launch_bounds__(kThreads) rht_quantize_kernel(const __grid_con
     };
 
     if (t == 0) {
-        mbar_init(&full[0], 1);
-        mbar_init(&full[1], 1);
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kComputeWarps);
+        }
         *abort_flag = 0u;
         fence_barrier_init();
     }
     __syncthreads();
-    int64_t u0 = blockIdx.x;
-    if (t == 0) {
-        if (u0 < nunits) issue(u0, 0);
-        if (u0 + gridDim.x < nunits) issue(u0 + gridDim.x, 1);
+    const int64_t u0 = blockIdx.x;
+    if (warp == kComputeWarps) {
+        // Producer warp: refills a stage once every compute warp released it.
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int64_t u = u0; u < nunits; u += gridDim.x, ++it) {
+                const int s = it % kStages;
+                if (it >= kStages &&
+                    !mbar_wait(&empty[s], ((it / kStages) - 1) & 1, kErrTimeoutProducer, abort_flag))
+                    break;
+                issue(u, s);
+            }
+            // Drain: the last copies have landed before the CTA exits.
+            for (uint32_t d = 0; d < kStages && d < it; ++d) {
+                const uint32_t idx = it - 1 - d;
+                uint32_t dummy = 0;
+                mbar_wait(&full[idx % kStages], (idx / kStages) & 1, kErrTimeoutDrain,
+                          reinterpret_cast<volatile uint32_t *>(&dummy));
+            }
+        }
+        return;
     }
 
     float S = 1.0f, G = 0.0f;
@@ -424,24 +466,20 @@ __global__ void __launch_bounds__(kThreads) rht_quantize_kernel(const __grid_con
     if (RND == 1) keys = philox_keys(a.seed);
     float amax_acc = 0.0f;
 
+    // Column-wise: byte offset of column cc (= t & 63) within K row r of a
+    // 64-column box for r % 8 (the 128-byte swizzle XORs the 16-byte chunk
+    // index with the row mod 8).
+    uint32_t col_off[8];
+    {
+        const int cc = t & 63;
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+            col_off[r] = static_cast<uint32_t>((t >> 6) * 8192 + ((((cc >> 3) ^ r) & 7) << 4) + (cc & 7) * 2);
+    }
     uint32_t it = 0;
     for (int64_t u = u0; u < nunits; u += gridDim.x, ++it) {
-        const int s = it & 1;
-        const uint32_t parity = (it >> 1) & 1;
-        // every thread observes the phase itself (bounded)
-        bool ok = mbar_try_wait(&full[s], parity);
-        if (!ok) {
-            const uint64_t t0 = globaltimer_ns();
-            while (!(ok = mbar_try_wait(&full[s], parity))) {
-                if (*abort_flag) break;
-                if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                    *abort_flag = 1u;
-                    break;
-                }
-            }
-        }
-        // one decision for the whole CTA (its barriers must stay matched)
-        if (!__syncthreads_and(ok ? 1 : 0)) break;
+        const int s = it % kStages;
+        if (!warp_wait(&full[s], (it / kStages) & 1, kErrTimeoutTransform, abort_flag)) break;
         int64_t rb, seg;
         unit_coords(u, rb, seg);
         const int64_t orow = rb * kUnitRows + t;
@@ -470,13 +508,11 @@ __global__ void __launch_bounds__(kThreads) rht_quantize_kernel(const __grid_con
                     }
                 }
             } else {
-                const int cc = t & 63;
-                const uint8_t *colp = tile + (t >> 6) * 8192 + (cc & 7) * 2;
 #pragma unroll
                 for (int i = 0; i < GS; ++i) {
                     const int kr = g0 + i;
-                    const uint16_t b = *reinterpret_cast<const uint16_t *>(
-                        colp + kr * 128 + ((((cc >> 3) ^ kr) & 7) << 4));
+                    const uint16_t b =
+                        *reinterpret_cast<const uint16_t *>(tile + col_off[kr & 7] + kr * 128);
                     v[i] = __uint_as_float(static_cast<uint32_t>(b) << 16);
                 }
             }
@@ -547,22 +583,8 @@ __global__ void __launch_bounds__(kThreads) rht_quantize_kernel(const __grid_con
                         static_cast<uint8_t>(stored[b]);
             }
         }
-        __syncthreads();   // stage s fully consumed
-        if (t == 0 && u + 2 * static_cast<int64_t>(gridDim.x) < nunits)
-            issue(u + 2 * gridDim.x, s);
-    }
-    // Drain in-flight copies before the CTA exits (time-bounded).
-    if (t == 0) {
-        for (uint32_t k = 0; k < 2; ++k) {
-            // the copies issued for iterations it and it+1 (if any)
-            const int64_t u = u0 + static_cast<int64_t>(it + k) * gridDim.x;
-            if (u >= nunits) break;
-            const int s = (it + k) & 1;
-            const uint32_t parity = ((it + k) >> 1) & 1;
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(&full[s], parity))
-                if (globaltimer_ns() - t0 > kWaitLimitNs) break;
-        }
+        __syncwarp();      // this warp is done with stage s
+        if (lane == 0) mbar_arrive(&empty[s]);
     }
     if (AMAX_ONLY) {
 #pragma unroll
@@ -587,7 +609,7 @@ cudaError_t launch_one(const QuantArgs &a, const CUtensorMap &tmap, int num_sms,
     const int64_t cap = static_cast<int64_t>(num_sms) * 3;
     const int grid = static_cast<int>(nunits < cap ? nunits : cap);
     if (grid <= 0) return cudaSuccess;
-    rht_quantize_kernel<AXIS, NH, BLK, GRID, RND, AMAX_ONLY><<<grid, kThreads, kQuantSmem, stream>>>(a, tmap);
+    rht_quantize_kernel<AXIS, NH, BLK, GRID, RND, AMAX_ONLY><<<grid, kCtaThreads, kQuantSmem, stream>>>(a, tmap);
     return cudaGetLastError();
 }
 
@@ -652,6 +674,15 @@ cudaError_t launch_rht_amax(QuantArgs a, int hadamard_n, int num_sms, cudaStream
     if (e != cudaSuccess) return e;
     if (a.axis == 0) return dispatch_nh_blk<0, true>(a, m, hadamard_n, 16, 0, 0, num_sms, stream);
     return dispatch_nh_blk<1, true>(a, m, hadamard_n, 16, 0, 0, num_sms, stream);
+}
+
+cudaError_t quantize_read_and_clear_error_word(uint32_t *out) {
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(out, g_error_word, sizeof(uint32_t));
+    if (e != cudaSuccess) return e;
+    const uint32_t zero = 0;
+    return cudaMemcpyToSymbol(g_error_word, &zero, sizeof(uint32_t));
 }
 
 }  // namespace ufp4
