@@ -1,0 +1,78 @@
+"""Small single-kernel cases for ncu captures (inputs larger than L2, a few
+hundred MB on the device at most), so that a full-metric capture of one
+launch ends quickly.  Each case runs its kernel twice: a warm-up launch and
+the launch to capture.
+
+    python -m fp4_quantized_gemms_b200.profile_cases gemm --m 4096 --n 4096 --k 2048 --grid e1m2
+    python -m fp4_quantized_gemms_b200.profile_cases quantize --rows 8192 --cols 8192 --axis rows --sr
+"""
+from __future__ import annotations
+
+import argparse
+
+import numpy as np
+import torch
+
+from fp4_quantized_gemms_b200 import ufp4
+from fp4_quantized_gemms_b200 import workloads as wl
+
+
+def _dev(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def gemm_case(m: int, n: int, k: int, grid: int, path: int) -> None:
+    """Quantize X [m, k] and W [n, k] (two-level scales, RHT16, block 16),
+    then run the FPROP GEMM twice."""
+    cfg = ufp4.QuantConfig(grid=grid, hadamard_n=16, block=16, scale_fmt=ufp4.SCALE_E4M3_X_FP32)
+    qx = ufp4.rht_quantize(_dev(wl.normal(m, k, 1.0, 1)), ufp4.ALONG_COLS, cfg)
+    qw = ufp4.rht_quantize(_dev(wl.normal(n, k, 0.02, 2)), ufp4.ALONG_COLS, cfg)
+    ufp4.set_two_level_gemm_path(path)
+    out = torch.empty((m, n), dtype=torch.float32, device="cuda")
+    for _ in range(2):
+        ufp4.gemm_fprop(qx, qw, out)
+    torch.cuda.synchronize()
+    if ufp4.check_device_status() != ufp4.OK:
+        raise RuntimeError("device error word set")
+
+
+def quantize_case(rows: int, cols: int, axis: int, sr: bool, two_level: bool) -> None:
+    """Rotated amax + quantize of one bf16 operand, twice."""
+    fmt = ufp4.SCALE_E4M3_X_FP32 if two_level else ufp4.SCALE_FP32
+    cfg = ufp4.QuantConfig(grid=ufp4.GRID_E1M2, rounding=ufp4.ROUND_SR if sr else ufp4.ROUND_RTNE,
+                           sr_seed=1234, hadamard_n=16, block=16, scale_fmt=fmt)
+    x = _dev(wl.normal(rows, cols, 1e-3, 3))
+    q = None
+    for _ in range(2):
+        q = ufp4.rht_quantize(x, axis, cfg, out=q)
+    torch.cuda.synchronize()
+    if ufp4.check_device_status() != ufp4.OK:
+        raise RuntimeError("device error word set")
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    sub = ap.add_subparsers(dest="case", required=True)
+    g = sub.add_parser("gemm")
+    g.add_argument("--m", type=int, default=4096)
+    g.add_argument("--n", type=int, default=4096)
+    g.add_argument("--k", type=int, default=2048)
+    g.add_argument("--grid", choices=["e1m2", "e2m1"], default="e1m2")
+    g.add_argument("--path", type=int, default=ufp4.GEMM_PATH_AUTO)
+    q = sub.add_parser("quantize")
+    q.add_argument("--rows", type=int, default=8192)
+    q.add_argument("--cols", type=int, default=8192)
+    q.add_argument("--axis", choices=["cols", "rows"], default="cols")
+    q.add_argument("--sr", action="store_true")
+    q.add_argument("--fp32-scales", action="store_true")
+    a = ap.parse_args()
+    if a.case == "gemm":
+        gemm_case(a.m, a.n, a.k, ufp4.GRID_E1M2 if a.grid == "e1m2" else ufp4.GRID_E2M1, a.path)
+    else:
+        quantize_case(a.rows, a.cols, ufp4.ALONG_COLS if a.axis == "cols" else ufp4.ALONG_ROWS,
+                      a.sr, not a.fp32_scales)
+    print("ok")
+
+
+if __name__ == "__main__":
+    main()
