@@ -154,8 +154,8 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
         return UFP4_ERR_ALIGNMENT;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // fp32 block scales: per-block partials (mode 0).  Two-level scales: the
-    // native block-scaled FP4 kernel with one CTA per 128 x 224 tile (mode 3),
-    // or what the caller picked: the same on CTA pairs with 256 x 224 tiles
+    // native block-scaled FP4 kernel with one CTA per 128 x 192 tile (mode 3),
+    // or what the caller picked: the same on CTA pairs with 256 x 192 tiles
     // (mode 4), the fp16-operand kernels (mode 1: one CTA per 128 x 256 tile,
     // mode 2: CTA pairs).
     int mode = 0;
@@ -183,18 +183,18 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
     GemmArgs args;
     memset(&args, 0, sizeof(args));
     // B code rows staged per CTA: fp32-scale kernel 128, fp16 kernels 256
-    // (one CTA) or 128 (pairs), native kernels 224 or 112, with the scales of
-    // all 224 B rows of a tile in each CTA.
+    // (one CTA) or 128 (pairs), native kernels 192 or 96, with the scales of
+    // all 192 B rows of a tile in each CTA.
     int bn = 128;
     switch (mode) {
         case 1: bn = 256; break;
-        case 3: bn = 224; break;
-        case 4: bn = 112; break;
+        case 3: bn = kNativeTileN; break;
+        case 4: bn = kNativeTileN / 2; break;
         default: bn = 128; break;
     }
     s = encode_operand_maps(a, 128, 128, mode, &args.tm_a_codes, &args.tm_a_scales);
     if (s != UFP4_OK) return s;
-    s = encode_operand_maps(b, bn, mode >= 3 ? 224 : bn, mode, &args.tm_b_codes, &args.tm_b_scales);
+    s = encode_operand_maps(b, bn, mode >= 3 ? kNativeTileN : bn, mode, &args.tm_b_codes, &args.tm_b_scales);
     if (s != UFP4_OK) return s;
     args.a_S = a->tensor_scale;
     args.b_S = b->tensor_scale;
@@ -216,7 +216,7 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
         CUtensorMap scratch;
         s = encode_operand_maps(&ac, 128, 128, mode, &args.tm_a_corr, &scratch);
         if (s != UFP4_OK) return s;
-        s = encode_operand_maps(&bc, bn, 224, mode, &args.tm_b_corr, &scratch);
+        s = encode_operand_maps(&bc, bn, kNativeTileN, mode, &args.tm_b_corr, &scratch);
         if (s != UFP4_OK) return s;
         args.corr_in = 1;
     }

@@ -713,12 +713,13 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
 // same scale factors, the raw code tiles used as they arrived and only the
 // correction planes written by the transform warps (a per-byte bit function).
 //
-// Tiles: 128 x 224 on one CTA (mode 3) or 256 x 224 on a CTA pair with
+// Tiles: 128 x 192 on one CTA (mode 3) or 256 x 192 on a CTA pair with
 // cta_group::2 MMAs (mode 4): rank r of the pair stages A rows [128 r, +128)
-// and B rows [112 r, +112) of the tile, holds accumulator rows [128 r, +128),
-// and both ranks hold the scale factors of all 224 B rows.  224 columns let
-// two accumulators share TMEM with the scale factors, so the epilogue of one
-// tile overlaps the MMAs of the next.  A stage covers 128 K elements
+// and B rows [96 r, +96) of the tile, holds accumulator rows [128 r, +128),
+// and both ranks hold the scale factors of all 192 B rows.  192 columns let
+// two accumulators share TMEM with one scale-factor slot per TMA stage, so the
+// epilogue of one tile overlaps the MMAs of the next and the transform runs
+// ahead of the MMAs as far as the TMA ring allows.  A stage covers 128 K elements
 // (64-byte code rows, 64-byte TMA swizzle).
 //
 // The transform warps write the scale factors into TMEM themselves
@@ -726,15 +727,16 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
 // K step, lane i of every 32-lane quarter holds, in 4 consecutive columns,
 // the 4 block factors of rows i, 32 + i, 64 + i and 96 + i (the layout the
 // MMA reads, the same in all four quarters); a warp builds an atom with a
-// 4x4 byte transpose per 4 rows in its scratch.  E1M2 correction planes are
-// loaded with the codes
+// 4x4 byte transpose per 4 rows in its scratch, and two groups of transform
+// warps take alternate stages.  E1M2 correction planes are loaded with the
+// codes
 // when the quantizer stored them, else the transform builds them.  Scale
 // factors and built planes use two-slot rings, refilled once the MMAs two
 // stages back have completed.  The epilogue stages 128 x 32 fp32 chunks in
 // shared memory and writes them with coalesced 16-byte stores.
 template <int GRID, int CG, bool CIN>
 struct Fp4Cfg {
-    static constexpr int BN = 224;                  // tile columns (B rows)
+    static constexpr int BN = kNativeTileN;         // tile columns (B rows)
     static constexpr int BNh = BN / CG;             // B code rows staged per CTA
     static constexpr int TM = BM * CG;              // tile rows
     static constexpr int BKE = 128;                 // K elements per stage
@@ -759,17 +761,18 @@ struct Fp4Cfg {
     static constexpr int kStage = (o_raw_b + kRawB + 1023) / 1024 * 1024;
     static constexpr int kCorr = (kCodesA + kCodesB + 1023) / 1024 * 1024;  // one slot
     // scale-factor atoms per stage: K step j, kind 0 = SFA, 1 / 2 = SFB rows
-    // [0, 128) / [128, 224)
+    // [0, 128) / [128, BN)
     static constexpr int kAtoms = 3 * KST;
-    static constexpr int kSubs = NT / 4;            // warps per TMEM lane quarter
-    static constexpr int kMine = kAtoms / kSubs;    // atoms one warp stores
-    static constexpr int kScr = NT * kMine * 512;   // per-warp atom scratch
-    static constexpr int kAccCols = 224;            // one accumulator
-    static constexpr int kSfCols = KST * 12;        // one scale-factor slot
+    static constexpr int kGroupWarps = NT / 2;      // transform warps per stage
+    static constexpr int kScr = NT * kAtoms * 512;  // per-warp atom scratch
+    static constexpr int kAccCols = BN;             // one accumulator
+    static constexpr int kSfCols = KST * 12;        // scale factors of one stage
     static constexpr int kSfBase = 2 * kAccCols;
     static constexpr int kBudget = 232448 - 2048;   // barriers, alignment slack
     static constexpr int kOutChunk = BM * 32 * 4;   // epilogue staging: 128 rows x 32 fp32
-    static constexpr int NS = (kBudget - ND * kCorr - kOutChunk - kScr) / kStage;
+    static constexpr int kNsSmem = (kBudget - ND * kCorr - kOutChunk - kScr) / kStage;
+    static constexpr int kNsTmem = (512 - kSfBase) / kSfCols;   // one scale-factor slot per stage
+    static constexpr int NS = kNsSmem < kNsTmem ? kNsSmem : kNsTmem;
     static constexpr int o_corr = NS * kStage;
     static constexpr int o_out = o_corr + ND * kCorr;
     static constexpr int o_scr = o_out + kOutChunk;
@@ -779,12 +782,13 @@ struct Fp4Cfg {
     static constexpr int o_misc = o_bar + kNumBars * 8;
     static constexpr int kAlloc = o_misc + 64 + 1024;
     static constexpr int kThreads = 32 * (2 + NT + NE);
-    static_assert(kAtoms % kSubs == 0, "atoms per warp");
+    static_assert(kGroupWarps == 4, "one warp per TMEM lane quarter in each transform group");
     static_assert(NS >= 4, "pipeline depth");
-    static_assert(kSfBase + 2 * kSfCols <= 512, "TMEM budget");
+    static_assert(kSfBase + NS * kSfCols <= 512, "TMEM budget");
     static_assert(kAlloc <= 232448, "shared memory budget");
     static_assert(o_corr % 1024 == 0 && o_out % 1024 == 0, "swizzle alignment");
     static_assert(BN % 32 == 0 && BN > 128 && BN <= 256, "two SFB row groups, 32-column chunks");
+    static_assert((BN / CG) % 8 == 0, "B rows per CTA");
 };
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -861,9 +865,9 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&ready[i], kPair ? CG : C::NT);
+            mbar_init(&ready[i], kPair ? CG : C::kGroupWarps);
             mbar_init(&empty[i], 1);
-            mbar_init(&tdone[i], C::NT);
+            mbar_init(&tdone[i], C::kGroupWarps);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
@@ -964,9 +968,9 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                     tc_fence_after();
                     uint8_t *st = stage(s);
                     // scale factors of K step j: SFA at 12 j, SFB rows 0-127
-                    // at 12 j + 4, rows 128-223 at 12 j + 8 of slot it & 1
+                    // at 12 j + 4, rows 128+ at 12 j + 8 of the stage's slot
                     // (written by the transform warps of each CTA)
-                    const uint32_t sf0 = tmem_base + C::kSfBase + (it & 1) * C::kSfCols;
+                    const uint32_t sf0 = tmem_base + C::kSfBase + s * C::kSfCols;
                     // K steps of 64 in this stage (a tail uses only its own)
                     const int64_t rem = tl.g.k - static_cast<int64_t>(ks) * C::BKE;
                     const int steps = rem >= C::BKE ? C::KST : static_cast<int>((rem + 63) / 64);
@@ -1001,13 +1005,18 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
         }
     } else if (warp < 2 + C::NT) {
         // ------------------------------------------------------------ transform
-        const int tt = threadIdx.x - 64;
-        constexpr int kThr = C::NT * 32;
-        constexpr int kChunks = (C::kCodesA + C::kCodesB) / 16;   // correction pieces
-        constexpr int kPer = (kChunks + kThr - 1) / kThr;
+        // Two groups of four warps (one per TMEM lane quarter) take alternate
+        // stages.  Each warp builds every scale-factor atom of its stage for
+        // its lane quarter (a 4x4 byte transpose per 4 rows into its scratch)
+        // and stores it with tcgen05.st into the stage's slot; that slot was
+        // last read by the MMAs that released this stage's TMA buffer.
         const int tw = warp - 2;
-        const int sub = tw >> 2;             // which of the warps of this lane quarter
-        uint8_t *scr = smem + C::o_scr + tw * (C::kMine * 512);
+        const int grp = tw >> 2;
+        const int gt = (tw & 3) * 32 + lane;            // thread index within the group
+        constexpr int kGrpThr = 32 * C::kGroupWarps;
+        constexpr int kChunks = (C::kCodesA + C::kCodesB) / 16;   // correction pieces
+        constexpr int kPer = (kChunks + kGrpThr - 1) / kGrpThr;
+        uint8_t *scr = smem + C::o_scr + tw * (C::kAtoms * 512);
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
         uint32_t it = 0;
         bool ok = true;
@@ -1015,14 +1024,15 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
             const Tile tl = get_tile<TM, BN>(args, t);
             const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
             for (int ks = 0; ks < nks; ++ks, ++it) {
+                if (static_cast<int>(it & 1) != grp) continue;
                 const int s = it % NS;
                 if (!warp_wait(&full[s], (it / NS) & 1, kErrTimeoutTransform, abort_flag)) {
                     ok = false;
                     break;
                 }
-                // Slot it & 1 of the scale-factor and correction rings was
-                // last read by the MMAs of iteration it - 2.
-                if (it >= 2) {
+                constexpr bool kBuild = GRID == 0 && !CIN;   // correction planes here
+                // Correction slot it & 1 was last read by the MMAs of it - 2.
+                if (kBuild && it >= 2) {
                     const uint32_t p = it - 2;
                     if (!warp_wait(&empty[p % NS], (p / NS) & 1, kErrTimeoutTransform, abort_flag)) {
                         ok = false;
@@ -1030,13 +1040,11 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                     }
                 }
                 const uint8_t *st = stage(s);
-                // Loads first: raw scale words of this warp's atoms (lane
-                // builds rows 4 lane .. 4 lane + 3 of a 128-row group) and the
-                // code pieces this thread corrects.
-                uint32_t w[C::kMine][4];
+                // Loads first: raw scale words (lane builds rows 4 lane ..
+                // 4 lane + 3 of a 128-row group) and the code pieces to correct.
+                uint32_t w[C::kAtoms][4];
 #pragma unroll
-                for (int x = 0; x < C::kMine; ++x) {
-                    const int a = sub + C::kSubs * x;
+                for (int a = 0; a < C::kAtoms; ++a) {
                     const int jk = a / 3, kind = a % 3;
                     const int rows = kind == 0 ? BM : BN;
                     const int r = 4 * lane + (kind == 2 ? 128 : 0);
@@ -1045,32 +1053,31 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                         if (blk == 16) {
 #pragma unroll
                             for (int kb = 0; kb < 4; ++kb)
-                                w[x][kb] = *reinterpret_cast<const uint32_t *>(raw + (4 * jk + kb) * rows);
+                                w[a][kb] = *reinterpret_cast<const uint32_t *>(raw + (4 * jk + kb) * rows);
                         } else {
-                            w[x][0] = w[x][1] = *reinterpret_cast<const uint32_t *>(raw + (2 * jk) * rows);
-                            w[x][2] = w[x][3] =
+                            w[a][0] = w[a][1] = *reinterpret_cast<const uint32_t *>(raw + (2 * jk) * rows);
+                            w[a][2] = w[a][3] =
                                 *reinterpret_cast<const uint32_t *>(raw + (2 * jk + 1) * rows);
                         }
                     } else {
-                        w[x][0] = w[x][1] = w[x][2] = w[x][3] = 0u;
+                        w[a][0] = w[a][1] = w[a][2] = w[a][3] = 0u;
                     }
                 }
-                constexpr bool kBuild = GRID == 0 && !CIN;   // correction planes here
                 uint4 cw[kBuild ? kPer : 1];
                 if constexpr (kBuild) {
 #pragma unroll
                     for (int i = 0; i < kPer; ++i) {
-                        const int idx = tt + i * kThr;
+                        const int idx = gt + i * kGrpThr;
                         if (idx < kChunks) cw[i] = *reinterpret_cast<const uint4 *>(st + 16 * idx);
                     }
                 }
-                // Scale atoms: byte 16 (r % 32) + 4 (r / 32) + kb holds the
-                // factor of 16-element block 4 jk + kb of row r.
+                // Atom byte 16 (r % 32) + 4 (r / 32) + kb holds the factor of
+                // 16-element block 4 jk + kb of row r of the group.
 #pragma unroll
-                for (int x = 0; x < C::kMine; ++x) {
+                for (int a = 0; a < C::kAtoms; ++a) {
                     uint32_t o[4];
-                    transpose4x4(w[x][0], w[x][1], w[x][2], w[x][3], o);
-                    uint8_t *dst = scr + x * 512 + 16 * ((4 * lane) & 31) + 4 * ((4 * lane) >> 5);
+                    transpose4x4(w[a][0], w[a][1], w[a][2], w[a][3], o);
+                    uint8_t *dst = scr + a * 512 + 16 * ((4 * lane) & 31) + 4 * ((4 * lane) >> 5);
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) *reinterpret_cast<uint32_t *>(dst + 16 * q4) = o[q4];
                 }
@@ -1080,7 +1087,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                     uint8_t *corr = smem + C::o_corr + (it & 1) * C::kCorr;
 #pragma unroll
                     for (int i = 0; i < kPer; ++i) {
-                        const int idx = tt + i * kThr;
+                        const int idx = gt + i * kGrpThr;
                         if (idx < kChunks) {
                             const uint4 d = make_uint4(e1m2_correction(cw[i].x), e1m2_correction(cw[i].y),
                                                        e1m2_correction(cw[i].z), e1m2_correction(cw[i].w));
@@ -1089,11 +1096,10 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                     }
                 }
                 __syncwarp();
-                const uint32_t sfw = lane_base + C::kSfBase + (it & 1) * C::kSfCols;
+                const uint32_t sfw = lane_base + C::kSfBase + s * C::kSfCols;
 #pragma unroll
-                for (int x = 0; x < C::kMine; ++x) {
-                    const int a = sub + C::kSubs * x;
-                    const uint4 row = *reinterpret_cast<const uint4 *>(scr + x * 512 + 16 * lane);
+                for (int a = 0; a < C::kAtoms; ++a) {
+                    const uint4 row = *reinterpret_cast<const uint4 *>(scr + a * 512 + 16 * lane);
                     tmem_st_32x32b_x4(sfw + 12 * (a / 3) + 4 * (a % 3), row.x, row.y, row.z, row.w);
                 }
                 tmem_wait_st();
@@ -1101,11 +1107,11 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                 tc_fence_before();
                 if constexpr (kPair) {
                     // The MMAs of CTA 0 read this CTA's tiles: one relay
-                    // arrive per CTA after all of its transform warps.
+                    // arrive per CTA after all warps of the group.
                     fence_proxy_async_cluster();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&tdone[s]);
-                    if (tt == 0) {
+                    if (gt == 0) {
                         if (!mbar_wait(&tdone[s], (it / NS) & 1, kErrTimeoutTransform, abort_flag)) {
                             ok = false;
                         } else {

@@ -54,6 +54,9 @@ struct GemmArgs {
     int corr_in;                          // both operands carry correction planes
 };
 
+// Tile columns (B rows) of the native block-scaled FP4 kernels (modes 3, 4).
+constexpr int kNativeTileN = 192;
+
 // mode 0: fp32 block scales (per-block partial products, CUDA-core scaling)
 // mode 1: E4M3 x fp32 two-level scales (scales folded into fp16 operands)
 // mode 2: mode 1 on a CTA pair (cta_group::2, 256 x 256 tiles)

@@ -215,9 +215,9 @@ ufp4_status_t ufp4_grouped_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b
  *   UFP4_GEMM_PATH_NATIVE_FP4 block-scaled FP4 MMA (kind::mxf4nvf4, UE4M3
  *                             factors per 16 elements); E1M2 codes are split
  *                             exactly into two E2M1 planes (four MMAs); one
- *                             CTA per 128 x 224 tile;
+ *                             CTA per 128 x 192 tile;
  *   UFP4_GEMM_PATH_NATIVE_FP4_PAIR  the same on CTA pairs (cta_group::2,
- *                             256 x 224 tiles);
+ *                             256 x 192 tiles);
  *   UFP4_GEMM_PATH_AUTO       the library's choice (default; currently the
  *                             one-CTA native FP4 path).
  * The setting is process-wide and read at each GEMM call; fp32 block scales
