@@ -172,6 +172,16 @@ __device__ __forceinline__ uint32_t lane_sign_bits(uint64_t mask, int j) {
     return static_cast<uint32_t>(mask >> off) & 0xFFFFu;
 }
 
+// Reciprocal for the fp32 estimate only (every decision it feeds is either
+// certified by the 2^-16 margin or re-decided exactly): rcp.approx has at
+// most 1 ulp error; a subnormal argument flushes to zero and gives +inf,
+// which sends the block to the exact path.
+__device__ __forceinline__ float approx_rcp(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 struct ScaleOut {
     float m1;    // factor folded into the threshold (1 or e_b)
     float b;     // fp32 scale multiplied inside the fma (s or S)
@@ -188,7 +198,7 @@ __device__ __forceinline__ ScaleOut block_scale(float amax, int scale_fmt, float
         o.m1 = 1.0f;
         o.b = s;
         o.zero = !(s > 0.0f);
-        o.inv = o.zero ? 0.0f : __frcp_rn(s);
+        o.inv = o.zero ? 0.0f : approx_rcp(s);
         o.stored = __float_as_uint(s);
     } else {
         const float q = __fdiv_rn(amax, G);
@@ -197,7 +207,7 @@ __device__ __forceinline__ ScaleOut block_scale(float amax, int scale_fmt, float
         o.m1 = e;
         o.b = S;
         o.zero = !(e > 0.0f);
-        o.inv = o.zero ? 0.0f : __frcp_rn(e * S);
+        o.inv = o.zero ? 0.0f : approx_rcp(e * S);
         o.stored = e8;
     }
     return o;
@@ -238,16 +248,30 @@ __device__ __forceinline__ uint32_t cvt_e2m1x4(float a0, float a1, float a2, flo
 struct Chunk16 {
     float4 v0, v1, v2, v3;
 };
-struct Rand8 {
-    uint4 r0, r1;
+// Where a chunk's SR words come from: Philox key (seed) and counter base.
+struct RandSrc {
+    uint64_t seed;
+    uint64_t L0;
+    uint32_t stream;
 };
 
 // Exact path: every element decided by the fma boundary tests.
 template <int GRID, int RND>
-__device__ __noinline__ uint2 round_pack_exact(const Chunk16 c, const ScaleOut sc, const Rand8 rr) {
+__device__ __noinline__ uint2 round_pack_exact(const Chunk16 c, const ScaleOut sc, const RandSrc src) {
     const float v[16] = {c.v0.x, c.v0.y, c.v0.z, c.v0.w, c.v1.x, c.v1.y, c.v1.z, c.v1.w,
                          c.v2.x, c.v2.y, c.v2.z, c.v2.w, c.v3.x, c.v3.y, c.v3.z, c.v3.w};
-    const uint32_t rnd[8] = {rr.r0.x, rr.r0.y, rr.r0.z, rr.r0.w, rr.r1.x, rr.r1.y, rr.r1.z, rr.r1.w};
+    // the chunk's SR words again (this path is rare)
+    uint32_t rnd[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (RND == 1) {
+        const PhiloxKeys keys = philox_keys(src.seed);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint64_t g = (src.L0 >> 3) + h;
+            const uint4 r = philox4x32_10(
+                make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), src.stream, 0u), keys);
+            rnd[4 * h] = r.x, rnd[4 * h + 1] = r.y, rnd[4 * h + 2] = r.z, rnd[4 * h + 3] = r.w;
+        }
+    }
     uint32_t w0 = 0, w1 = 0;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -275,7 +299,8 @@ __device__ __noinline__ uint2 round_pack_exact(const Chunk16 c, const ScaleOut s
 // result always equals the exact-quotient rule.
 template <int GRID, int RND>
 __device__ __forceinline__ uint2 round_pack(const float (&v)[16], const ScaleOut &sc,
-                                            const PhiloxKeys &keys, uint32_t stream, uint64_t L0) {
+                                            const PhiloxKeys &keys, uint32_t stream, uint64_t L0,
+                                            uint64_t seed) {
     uint32_t rnd[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (RND == 1) {
         const uint64_t g0 = L0 >> 3;
@@ -346,10 +371,95 @@ __device__ __forceinline__ uint2 round_pack(const float (&v)[16], const ScaleOut
     if (risky) {
         const Chunk16 c{make_float4(v[0], v[1], v[2], v[3]), make_float4(v[4], v[5], v[6], v[7]),
                         make_float4(v[8], v[9], v[10], v[11]), make_float4(v[12], v[13], v[14], v[15])};
-        const Rand8 rr{make_uint4(rnd[0], rnd[1], rnd[2], rnd[3]), make_uint4(rnd[4], rnd[5], rnd[6], rnd[7])};
-        return round_pack_exact<GRID, RND>(c, sc, rr);
+        return round_pack_exact<GRID, RND>(c, sc, RandSrc{seed, L0, stream});
     }
     return make_uint2(canonical_zero(w[0]), canonical_zero(w[1]));
+}
+
+// ---------------------------------------------------------------------------
+// Two chunks at once in packed fp32x2 arithmetic (lane x = chunk a, lane y =
+// chunk b): the same IEEE operations per lane as the scalar code.
+
+// Butterfly on two lanes: (x0 + x1, x0 - x1); fma(x1, -1, x0) rounds x0 - x1
+// exactly like a subtraction.
+__device__ __forceinline__ void bfly2(float2 &x0, float2 &x1) {
+    const float2 s = __fadd2_rn(x0, x1);
+    const float2 d = __ffma2_rn(x1, make_float2(-1.0f, -1.0f), x0);
+    x0 = s;
+    x1 = d;
+}
+
+// 0x4B000000 | (16 bits of w): the float 2^23 + r16 (lo or hi half).
+__device__ __forceinline__ float r16_magic(uint32_t w, bool hi) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(w), "r"(0x4B000000u), "r"(hi ? 0x7432u : 0x7410u));
+    return __uint_as_float(d);
+}
+
+// E1M2, RTNE or SR, for two chunks with their own block scales: the fast
+// paths of round_pack (same decisions, same certification) with the fp32
+// adds / fmas done two lanes at a time.
+template <int RND>
+__device__ __forceinline__ void round_pack2_e1m2(const float (&va)[16], const float (&vb)[16],
+                                                 const ScaleOut &sa, const ScaleOut &sb,
+                                                 const PhiloxKeys &keys, uint32_t stream, uint64_t seed,
+                                                 uint64_t L0a, uint64_t L0b, uint2 &outa, uint2 &outb) {
+    const float inv4a = sa.inv * 4.0f, inv4b = sb.inv * 4.0f;
+    float deva = 0.0f, devb = 0.0f;      // largest distance from a rint half-way point
+    uint32_t wa[2] = {0u, 0u}, wb[2] = {0u, 0u};
+    const float2 kR = make_float2(kRound, kRound);
+    const float2 kRn = make_float2(-kRound, -kRound);
+    const float2 m1 = make_float2(-1.0f, -1.0f);
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        // SR words of elements 8 hf .. 8 hf + 7 of each chunk (one Philox call each)
+        uint4 ra = make_uint4(0, 0, 0, 0), rb = make_uint4(0, 0, 0, 0);
+        if (RND == 1) {
+            const uint64_t ga = (L0a >> 3) + hf, gb = (L0b >> 3) + hf;
+            ra = philox4x32_10(make_uint4(static_cast<uint32_t>(ga), static_cast<uint32_t>(ga >> 32), stream, 0u),
+                               keys);
+            rb = philox4x32_10(make_uint4(static_cast<uint32_t>(gb), static_cast<uint32_t>(gb >> 32), stream, 0u),
+                               keys);
+        }
+        const uint32_t rwa[4] = {ra.x, ra.y, ra.z, ra.w}, rwb[4] = {rb.x, rb.y, rb.z, rb.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int i = 8 * hf + e;
+            const float ya = fminf(fabsf(va[i]) * inv4a, 7.0f);
+            const float yb = fminf(fabsf(vb[i]) * inv4b, 7.0f);
+            float2 h = make_float2(ya, yb);
+            if (RND == 1) {
+                // h = y - r16 * 2^-16 + 1/2 (k = ceil(q - r) = rint(h) off the
+                // integers, which the margin test sends to the exact path)
+                const float2 rf = __fadd2_rn(make_float2(r16_magic(rwa[e >> 1], e & 1), r16_magic(rwb[e >> 1], e & 1)),
+                                             make_float2(-8421376.0f, -8421376.0f));   // r16 - 2^15
+                h = __ffma2_rn(rf, make_float2(-1.0f / 65536.0f, -1.0f / 65536.0f), h);
+            }
+            const float2 f = __fadd2_rn(h, kR);
+            const float2 g = __fadd2_rn(f, kRn);
+            const float2 d = __ffma2_rn(g, m1, h);       // h - rint(h), in [-1/2, 1/2]
+            deva = fmaxf(deva, fabsf(d.x));
+            devb = fmaxf(devb, fabsf(d.y));
+            const uint32_t ca = (__float_as_uint(f.x) & 7u) | ((__float_as_uint(va[i]) >> 28) & 8u);
+            const uint32_t cb = (__float_as_uint(f.y) & 7u) | ((__float_as_uint(vb[i]) >> 28) & 8u);
+            wa[hf] |= ca << (4 * e);
+            wb[hf] |= cb << (4 * e);
+        }
+    }
+    const bool riska = !(inv4a < INFINITY) || deva > 0.5f - kMargin;
+    const bool riskb = !(inv4b < INFINITY) || devb > 0.5f - kMargin;
+    outa = sa.zero ? make_uint2(0u, 0u) : make_uint2(canonical_zero(wa[0]), canonical_zero(wa[1]));
+    outb = sb.zero ? make_uint2(0u, 0u) : make_uint2(canonical_zero(wb[0]), canonical_zero(wb[1]));
+    if (riska && !sa.zero) {
+        const Chunk16 c{make_float4(va[0], va[1], va[2], va[3]), make_float4(va[4], va[5], va[6], va[7]),
+                        make_float4(va[8], va[9], va[10], va[11]), make_float4(va[12], va[13], va[14], va[15])};
+        outa = round_pack_exact<0, RND>(c, sa, RandSrc{seed, L0a, stream});
+    }
+    if (riskb && !sb.zero) {
+        const Chunk16 c{make_float4(vb[0], vb[1], vb[2], vb[3]), make_float4(vb[4], vb[5], vb[6], vb[7]),
+                        make_float4(vb[8], vb[9], vb[10], vb[11]), make_float4(vb[12], vb[13], vb[14], vb[15])};
+        outb = round_pack_exact<0, RND>(c, sb, RandSrc{seed, L0b, stream});
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -462,6 +572,11 @@ __global__ void __launch_bounds__(kCtaThreads, 3) rht_quantize_kernel(const __gr
         for (int off = 0; off < 64; off += (NH > 0 ? NH : 64)) pat |= m << off;
     }
     const uint32_t pat_lo = static_cast<uint32_t>(pat), pat_hi = static_cast<uint32_t>(pat >> 32);
+    // Sign of D at position i mod 16 as an fp32 sign bit (NH <= 16); adding
+    // it to a widened bf16 flips the sign bit like an xor.
+    uint32_t smask[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) smask[i] = NH > 0 ? ((pat_lo >> i) & 1u) << 31 : 0u;
     PhiloxKeys keys;
     if (RND == 1) keys = philox_keys(a.seed);
     float amax_acc = 0.0f;
@@ -491,6 +606,88 @@ __global__ void __launch_bounds__(kCtaThreads, 3) rht_quantize_kernel(const __gr
         constexpr int GS = (NH > BLK ? NH : BLK) > 16 ? (NH > BLK ? NH : BLK) : 16;
         uint32_t codes[8];
         uint32_t stored[4];
+        if constexpr (GS == 16) {
+            // Groups g and g + 16 side by side as the two lanes of fp32x2
+            // values: same positions mod 16, so the same signs of D; the
+            // butterflies and the rounding arithmetic run two lanes at a time.
+            // Not unrolled: one copy of the body keeps the kernel small.
+#pragma unroll 1
+            for (int gp = 0; gp < 64; gp += 32) {
+                float va[16], vb[16];
+                if (AXIS == 0) {
+                    const uint8_t *rowp = tile + t * 128;
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const uint4 qa = *reinterpret_cast<const uint4 *>(rowp + (((gp / 8 + c) ^ (t & 7)) << 4));
+                        const uint4 qb = *reinterpret_cast<const uint4 *>(rowp + (((gp / 8 + 2 + c) ^ (t & 7)) << 4));
+                        const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w}, wb[4] = {qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int i0 = 8 * c + 2 * e;
+                            va[i0] = __uint_as_float((wa[e] << 16) + smask[i0]);
+                            va[i0 + 1] = __uint_as_float((wa[e] & 0xFFFF0000u) ^ smask[i0 + 1]);
+                            vb[i0] = __uint_as_float((wb[e] << 16) + smask[i0]);
+                            vb[i0 + 1] = __uint_as_float((wb[e] & 0xFFFF0000u) ^ smask[i0 + 1]);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int ka = gp + i, kb = gp + 16 + i;
+                        const uint32_t ba = *reinterpret_cast<const uint16_t *>(tile + col_off[ka & 7] + ka * 128);
+                        const uint32_t bb = *reinterpret_cast<const uint16_t *>(tile + col_off[kb & 7] + kb * 128);
+                        va[i] = __uint_as_float((ba << 16) + smask[i]);
+                        vb[i] = __uint_as_float((bb << 16) + smask[i]);
+                    }
+                }
+                if (NH == 16) {
+                    float2 pr[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) pr[i] = make_float2(va[i], vb[i]);
+#pragma unroll
+                    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (!(i & h)) bfly2(pr[i], pr[i + h]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        va[i] = pr[i].x;
+                        vb[i] = pr[i].y;
+                    }
+                }
+                if (AMAX_ONLY) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        amax_acc = fmaxf(amax_acc, fmaxf(fabsf(va[i]), fabsf(vb[i])));
+                    continue;
+                }
+                float ama = 0.0f, amb = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    ama = fmaxf(ama, fabsf(va[i]));
+                    amb = fmaxf(amb, fabsf(vb[i]));
+                }
+                const ScaleOut sa = block_scale<GRID>(ama, a.scale_fmt, S, G);
+                const ScaleOut sb = block_scale<GRID>(amb, a.scale_fmt, S, G);
+                const uint64_t L0a = static_cast<uint64_t>(orow) * static_cast<uint64_t>(a.kpad) +
+                                     static_cast<uint64_t>(k0 + gp);
+                uint2 pa, pb;
+                if (GRID == 0) {
+                    round_pack2_e1m2<RND>(va, vb, sa, sb, keys, a.stream, a.seed, L0a, L0a + 16, pa, pb);
+                } else {
+                    pa = round_pack<GRID, RND>(va, sa, keys, a.stream, L0a, a.seed);
+                    pb = round_pack<GRID, RND>(vb, sb, keys, a.stream, L0a + 16, a.seed);
+                }
+                if (gp == 0) {
+                    codes[0] = pa.x, codes[1] = pa.y, codes[2] = pb.x, codes[3] = pb.y;
+                    stored[0] = sa.stored, stored[1] = sb.stored;
+                } else {
+                    codes[4] = pa.x, codes[5] = pa.y, codes[6] = pb.x, codes[7] = pb.y;
+                    stored[2] = sa.stored, stored[3] = sb.stored;
+                }
+            }
+        } else
 #pragma unroll
         for (int g0 = 0; g0 < 64; g0 += GS) {
             float v[GS];
@@ -554,7 +751,7 @@ __global__ void __launch_bounds__(kCtaThreads, 3) rht_quantize_kernel(const __gr
                     const int kc = g0 + b0 + c0;
                     const uint64_t L0 = static_cast<uint64_t>(orow) * static_cast<uint64_t>(a.kpad) +
                                         static_cast<uint64_t>(k0 + kc);
-                    const uint2 pk = round_pack<GRID, RND>(chunk, sc, keys, a.stream, L0);
+                    const uint2 pk = round_pack<GRID, RND>(chunk, sc, keys, a.stream, L0, a.seed);
                     codes[kc / 8] = pk.x;
                     codes[kc / 8 + 1] = pk.y;
                 }
