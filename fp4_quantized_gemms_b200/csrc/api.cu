@@ -210,14 +210,35 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
     // E1M2 operands that carry correction planes: the native kernels load
     // them with the codes (same box, same swizzle).
     if (mode >= 3 && a->cfg.grid == UFP4_GRID_E1M2 && a->corr != nullptr && b->corr != nullptr) {
-        ufp4_qtensor_t ac = *a, bc = *b;
-        ac.codes = a->corr;
-        bc.codes = b->corr;
-        CUtensorMap scratch;
-        s = encode_operand_maps(&ac, 128, 128, mode, &args.tm_a_corr, &scratch);
-        if (s != UFP4_OK) return s;
-        s = encode_operand_maps(&bc, bn, kNativeTileN, mode, &args.tm_b_corr, &scratch);
-        if (s != UFP4_OK) return s;
+        // When each operand's plane follows its codes in one allocation
+        // ([2][rows][kpad/2]), one 3-D box per operand fetches both.
+        auto adjacent = [](const ufp4_qtensor_t *q) {
+            const uint64_t plane = static_cast<uint64_t>(q->rows) * static_cast<uint64_t>(q->kpad / 2);
+            return q->rows > 0 && reinterpret_cast<uintptr_t>(q->corr) ==
+                                      reinterpret_cast<uintptr_t>(q->codes) + plane;
+        };
+        if (adjacent(a) && adjacent(b)) {
+            const uint64_t pa = static_cast<uint64_t>(a->rows) * static_cast<uint64_t>(a->kpad / 2);
+            const uint64_t pb = static_cast<uint64_t>(b->rows) * static_cast<uint64_t>(b->kpad / 2);
+            CUresult r = encode_tensor_map_planes(&args.tm_a_corr, a->codes, static_cast<uint64_t>(a->kpad / 2),
+                                                  static_cast<uint64_t>(a->rows), 2, pa, 64, 128,
+                                                  CU_TENSOR_MAP_SWIZZLE_64B);
+            if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
+            r = encode_tensor_map_planes(&args.tm_b_corr, b->codes, static_cast<uint64_t>(b->kpad / 2),
+                                         static_cast<uint64_t>(b->rows), 2, pb, 64, static_cast<uint32_t>(bn),
+                                         CU_TENSOR_MAP_SWIZZLE_64B);
+            if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
+            args.planes3d = 1;
+        } else {
+            ufp4_qtensor_t ac = *a, bc = *b;
+            ac.codes = a->corr;
+            bc.codes = b->corr;
+            CUtensorMap scratch;
+            s = encode_operand_maps(&ac, 128, 128, mode, &args.tm_a_corr, &scratch);
+            if (s != UFP4_OK) return s;
+            s = encode_operand_maps(&bc, bn, kNativeTileN, mode, &args.tm_b_corr, &scratch);
+            if (s != UFP4_OK) return s;
+        }
         args.corr_in = 1;
     }
     // Native kernels store 16-byte pieces when the output allows it.
@@ -251,6 +272,20 @@ CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, const
     return fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estride,
               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+CUresult encode_tensor_map_planes(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                                  uint64_t planes, uint64_t plane_bytes, uint32_t box_inner,
+                                  uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (fn == nullptr) return CUDA_ERROR_NOT_INITIALIZED;
+    const cuuint64_t dims[3] = {inner, outer, planes};
+    const cuuint64_t strides[2] = {inner, plane_bytes};
+    const cuuint32_t box[3] = {box_inner, box_outer, static_cast<cuuint32_t>(planes)};
+    const cuuint32_t estride[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estride,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
 }  // namespace ufp4

@@ -752,10 +752,12 @@ struct Fp4Cfg {
     static constexpr int kRawA = BM * (BKE / 16);
     static constexpr int kRawB = BN * (BKE / 16);
     static constexpr int kIn = CIN ? 2 : 1;         // code planes loaded per stage
+    // [codes A | planes A | codes B | planes B | raw scales A | raw scales B]
+    // (the planes only with CIN): a 3-D box fills an operand's two tiles.
     static constexpr int o_codes_a = 0;
-    static constexpr int o_codes_b = o_codes_a + kCodesA;
-    static constexpr int o_cin_a = o_codes_b + kCodesB;         // CIN only
-    static constexpr int o_cin_b = o_cin_a + kCodesA;
+    static constexpr int o_cin_a = o_codes_a + kCodesA;         // CIN only
+    static constexpr int o_codes_b = o_codes_a + kIn * kCodesA;
+    static constexpr int o_cin_b = o_codes_b + kCodesB;         // CIN only
     static constexpr int o_raw_a = o_codes_a + kIn * (kCodesA + kCodesB);
     static constexpr int o_raw_b = o_raw_a + kRawA;
     static constexpr int kStage = (o_raw_b + kRawB + 1023) / 1024 * 1024;
@@ -921,11 +923,16 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                     mbar_arrive_expect_tx(&full[s],
                                           C::kIn * (C::kCodesA + C::kCodesB) + (BM + BN) * nraw);
                     const int32_t brow_h = brow + C::BNh * static_cast<int32_t>(rank);
-                    tma_load_2d(st + C::o_codes_a, &args.tm_a_codes, &full[s], acol / 2, arow);
-                    tma_load_2d(st + C::o_codes_b, &args.tm_b_codes, &full[s], bcol / 2, brow_h);
-                    if (CIN) {
-                        tma_load_2d(st + C::o_cin_a, &args.tm_a_corr, &full[s], acol / 2, arow);
-                        tma_load_2d(st + C::o_cin_b, &args.tm_b_corr, &full[s], bcol / 2, brow_h);
+                    if (CIN && args.planes3d) {
+                        tma_load_3d(st + C::o_codes_a, &args.tm_a_corr, &full[s], acol / 2, arow, 0);
+                        tma_load_3d(st + C::o_codes_b, &args.tm_b_corr, &full[s], bcol / 2, brow_h, 0);
+                    } else {
+                        tma_load_2d(st + C::o_codes_a, &args.tm_a_codes, &full[s], acol / 2, arow);
+                        tma_load_2d(st + C::o_codes_b, &args.tm_b_codes, &full[s], bcol / 2, brow_h);
+                        if (CIN) {
+                            tma_load_2d(st + C::o_cin_a, &args.tm_a_corr, &full[s], acol / 2, arow);
+                            tma_load_2d(st + C::o_cin_b, &args.tm_b_corr, &full[s], bcol / 2, brow_h);
+                        }
                     }
                     tma_load_2d(st + C::o_raw_a, &args.tm_a_scales, &full[s], arow, acol / blk);
                     tma_load_2d(st + C::o_raw_b, &args.tm_b_scales, &full[s], brow, bcol / blk);
@@ -977,7 +984,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                     const uint32_t a0 = smem_addr(st + C::o_codes_a), b0 = smem_addr(st + C::o_codes_b);
                     const uint32_t ac = CIN ? smem_addr(st + C::o_cin_a)
                                             : smem_addr(smem + C::o_corr + (it & 1) * C::kCorr);
-                    const uint32_t bc = ac + C::kCodesA;
+                    const uint32_t bc = CIN ? smem_addr(st + C::o_cin_b) : ac + C::kCodesA;
                     for (int j = 0; j < steps; ++j) {
                         const uint32_t sfa = sf0 + 12 * j, sfb = sfa + 4;
                         const uint32_t dk = 32 * j;

@@ -405,6 +405,10 @@ __device__ __forceinline__ void round_pack2_e1m2(const float (&va)[16], const fl
                                                  const PhiloxKeys &keys, uint32_t stream, uint64_t seed,
                                                  uint64_t L0a, uint64_t L0b, uint2 &outa, uint2 &outb) {
     const float inv4a = sa.inv * 4.0f, inv4b = sb.inv * 4.0f;
+    // min(|u| * inv4, 7) as 7 * sat(|u| * inv4 / 7): a saturating multiply on
+    // the fma pipe instead of a min (the estimate moves by a few ulp, far
+    // inside the 2^-16 margin; at and above 7 both give exactly 7).
+    const float c7a = inv4a * (1.0f / 7.0f), c7b = inv4b * (1.0f / 7.0f);
     float deva = 0.0f, devb = 0.0f;      // largest distance from a rint half-way point
     uint32_t wa[2] = {0u, 0u}, wb[2] = {0u, 0u};
     const float2 kR = make_float2(kRound, kRound);
@@ -425,15 +429,17 @@ __device__ __forceinline__ void round_pack2_e1m2(const float (&va)[16], const fl
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const int i = 8 * hf + e;
-            const float ya = fminf(fabsf(va[i]) * inv4a, 7.0f);
-            const float yb = fminf(fabsf(vb[i]) * inv4b, 7.0f);
-            float2 h = make_float2(ya, yb);
+            const float2 y7 = make_float2(__saturatef(fabsf(va[i]) * c7a), __saturatef(fabsf(vb[i]) * c7b));
+            float2 h;
             if (RND == 1) {
                 // h = y - r16 * 2^-16 + 1/2 (k = ceil(q - r) = rint(h) off the
                 // integers, which the margin test sends to the exact path)
                 const float2 rf = __fadd2_rn(make_float2(r16_magic(rwa[e >> 1], e & 1), r16_magic(rwb[e >> 1], e & 1)),
                                              make_float2(-8421376.0f, -8421376.0f));   // r16 - 2^15
-                h = __ffma2_rn(rf, make_float2(-1.0f / 65536.0f, -1.0f / 65536.0f), h);
+                const float2 rt = __fmul2_rn(rf, make_float2(-1.0f / 65536.0f, -1.0f / 65536.0f));   // exact
+                h = __ffma2_rn(y7, make_float2(7.0f, 7.0f), rt);
+            } else {
+                h = __fmul2_rn(y7, make_float2(7.0f, 7.0f));
             }
             const float2 f = __fadd2_rn(h, kR);
             const float2 g = __fadd2_rn(f, kRn);
@@ -442,8 +448,9 @@ __device__ __forceinline__ void round_pack2_e1m2(const float (&va)[16], const fl
             devb = fmaxf(devb, fabsf(d.y));
             const uint32_t ca = (__float_as_uint(f.x) & 7u) | ((__float_as_uint(va[i]) >> 28) & 8u);
             const uint32_t cb = (__float_as_uint(f.y) & 7u) | ((__float_as_uint(vb[i]) >> 28) & 8u);
-            wa[hf] |= ca << (4 * e);
-            wb[hf] |= cb << (4 * e);
+            // nibbles do not overlap: a multiply-add places them
+            wa[hf] = ca * (1u << (4 * e)) + wa[hf];
+            wb[hf] = cb * (1u << (4 * e)) + wb[hf];
         }
     }
     const bool riska = !(inv4a < INFINITY) || deva > 0.5f - kMargin;

@@ -50,8 +50,10 @@ struct GemmArgs {
     int num_groups;
     GemmGroup single;                     // used when groups == nullptr
     int c_vec;                            // c 16-byte aligned and ldc % 4 == 0
-    CUtensorMap tm_a_corr, tm_b_corr;     // E1M2 correction planes (corr_in)
+    CUtensorMap tm_a_corr, tm_b_corr;     // E1M2 correction planes (corr_in); with
+                                          // planes3d: 3-D maps over {codes, corr}
     int corr_in;                          // both operands carry correction planes
+    int planes3d;                         // corr = codes + rows * kpad / 2 for both
 };
 
 // Tile columns (B rows) of the native block-scaled FP4 kernels (modes 3, 4).
@@ -69,5 +71,9 @@ CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, const
                               uint64_t inner, uint64_t outer, uint64_t row_bytes,
                               uint32_t box_inner, uint32_t box_outer,
                               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE);
+// u8 planes [planes][outer][inner] (plane_bytes apart), boxes of every plane.
+CUresult encode_tensor_map_planes(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                                  uint64_t planes, uint64_t plane_bytes, uint32_t box_inner,
+                                  uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
 }  // namespace ufp4

@@ -178,16 +178,19 @@ def empty_qtensor(rows: int, k: int, cfg: QuantConfig, device="cuda",
                   with_corr: bool | None = None) -> QTensor:
     kpad, sld, _, _ = layout(rows, k, cfg)
     nblk = kpad // cfg.block
-    codes = torch.empty((rows, kpad // 2), dtype=torch.uint8, device=device)
+    if with_corr is None:
+        with_corr = wants_corr(cfg)
+    # codes and the correction plane in one allocation ([2][rows][kpad/2]):
+    # the GEMM then fetches both planes of a tile with one copy
+    planes = torch.empty((2 if with_corr else 1, rows, kpad // 2), dtype=torch.uint8, device=device)
+    codes = planes[0]
     if cfg.scale_fmt == SCALE_FP32:
         scales = torch.empty((nblk, sld), dtype=torch.float32, device=device)
         ts = None
     else:
         scales = torch.empty((nblk, sld), dtype=torch.uint8, device=device)
         ts = torch.empty(1, dtype=torch.float32, device=device)
-    if with_corr is None:
-        with_corr = wants_corr(cfg)
-    corr = torch.empty_like(codes) if with_corr else None
+    corr = planes[1] if with_corr else None
     return QTensor(codes, scales, ts, rows, k, kpad, sld, cfg, corr)
 
 

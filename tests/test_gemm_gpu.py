@@ -184,3 +184,27 @@ def test_two_level_kernel_families(path, corr, grid):
             _check_full(qx, rx, qw, rw, ufp4.gemm_fprop)
     finally:
         ufp4.set_two_level_gemm_path(old)
+
+
+@pytest.mark.parametrize("fmt", [ufp4.SCALE_FP32, ufp4.SCALE_E4M3_X_FP32])
+def test_e2m1_reference_recipe_layer(fmt):
+    """The comparison recipe of the pages (E2M1 grid, RHT on the WGRAD
+    operands only, SR on dY, RTNE elsewhere): all three GEMMs of a small
+    layer against the oracle."""
+    M, K, N = 384, 320, 264
+    X = wl.normal_with_outlier_channels(M, K, 1.0, 3, 30.0)
+    W = wl.normal(N, K, 0.02, 2)
+    dY = wl.normal(M, N, 1e-3, 3)
+    plain = _cfg(grid=ufp4.GRID_E2M1, fmt=fmt, n=0)
+    sr_plain = _cfg(grid=ufp4.GRID_E2M1, fmt=fmt, n=0, rounding=1, stream=0)
+    rot = _cfg(grid=ufp4.GRID_E2M1, fmt=fmt, n=16)
+    sr_rot = _cfg(grid=ufp4.GRID_E2M1, fmt=fmt, n=16, rounding=1, stream=1)
+    qx, rx = _quant_both(X, C, plain)
+    qw, rw = _quant_both(W, C, plain)
+    _check_full(qx, rx, qw, rw, ufp4.gemm_fprop)
+    qdy, rdy = _quant_both(dY, C, sr_plain)
+    qwt, rwt = _quant_both(W, R, plain)
+    _check_full(qdy, rdy, qwt, rwt, ufp4.gemm_dgrad)
+    qdyt, rdyt = _quant_both(dY, R, sr_rot)
+    qxt, rxt = _quant_both(X, R, rot)
+    _check_full(qdyt, rdyt, qxt, rxt, ufp4.gemm_wgrad)
