@@ -198,6 +198,71 @@ def quant_bytes(step: LayerStep) -> float:
     return total
 
 
+def run_moe(device, two_level: bool, reps: int = 10):
+    """The grouped (mixture-of-experts) GEMMs of one expert FFN: 16384 tokens,
+    top-6 of 64 experts (Zipf(1.2) counts, segments padded to 64 rows), hidden
+    2048, FFN 1408.  Operands are quantized once (untimed); the three grouped
+    GEMMs are timed with CUDA events over `reps` launches each."""
+    from fp4_quantized_gemms_b200 import ufp4
+    shp = wl.MOE
+    counts = wl.moe_expert_counts(shp)
+    starts, padded, total = wl.padded_offsets(counts, 64)
+    E, Hd, F = shp.experts, shp.hidden, shp.ffn
+    rng_rows = np.zeros(total, dtype=bool)
+    for s0, c in zip(starts, counts):
+        rng_rows[s0:s0 + c] = True
+
+    def routed(cols, std, seed):
+        a = wl.normal(total, cols, std, seed)
+        a[~rng_rows] = 0
+        return to_dev(a, device)
+
+    fmt = ufp4.SCALE_E4M3_X_FP32 if two_level else ufp4.SCALE_FP32
+    rt = ufp4.QuantConfig(grid=ufp4.GRID_E1M2, hadamard_n=16, block=16, scale_fmt=fmt)
+    sr0 = rt.with_(rounding=ufp4.ROUND_SR, sr_seed=SR_SEED, sr_stream=0)
+    sr1 = rt.with_(rounding=ufp4.ROUND_SR, sr_seed=SR_SEED, sr_stream=1)
+    C, R = ufp4.ALONG_COLS, ufp4.ALONG_ROWS
+    X = routed(Hd, 1.0, 1)
+    dY = routed(Hd, 1e-3, 3)
+    H = routed(F, 1.0, 5)
+    Wgu = to_dev(wl.normal(E * 2 * F, Hd, 0.02, 2), device)
+    Wd = to_dev(wl.normal(E * Hd, F, 0.02, 4), device)
+    q = ufp4.rht_quantize
+    jobs = {
+        "fprop_gate_up": (q(X, C, rt), q(Wgu, C, rt),
+                          [(counts[e], 2 * F, Hd, starts[e], 0, e * 2 * F, 0, starts[e], 0) for e in range(E)],
+                          (total, 2 * F)),
+        "dgrad_down": (q(dY, C, sr0), q(Wd, R, rt),
+                       [(counts[e], F, Hd, starts[e], 0, 0, e * Hd, starts[e], 0) for e in range(E)],
+                       (total, F)),
+        "wgrad_down": (q(dY, R, sr1), q(H, R, rt),
+                       [(Hd, F, padded[e], 0, starts[e], 0, starts[e], e * Hd, 0) for e in range(E)],
+                       (E * Hd, F)),
+    }
+    out = {}
+    for name, (qa, qb, groups, oshape) in jobs.items():
+        g = torch.tensor(np.array(groups, dtype=np.int64), device=device)
+        c = torch.empty(oshape, dtype=torch.float32, device=device)
+        flops = sum(2 * m * n * k for (m, n, k, *_r) in groups)
+        for _ in range(3):
+            ufp4.grouped_gemm(qa, qb, g, c)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(device)
+        e0.record()
+        for _ in range(reps):
+            ufp4.grouped_gemm(qa, qb, g, c)
+        e1.record()
+        torch.cuda.synchronize(device)
+        ms = e0.elapsed_time(e1) / reps
+        out[name] = {"ms": round(ms, 4), "TFLOPs": round(flops / (ms * 1e-3) / 1e12, 1),
+                     "GFLOP": round(flops / 1e9, 1)}
+    if ufp4.check_device_status() != ufp4.OK:
+        raise RuntimeError("device error word set in the MoE measurement")
+    out["workload"] = ("16384 tokens, top-6 of 64 experts (Zipf 1.2 counts, 64-row padded segments), "
+                       "hidden 2048, FFN 1408; grouped GEMMs over a device group table")
+    return out
+
+
 def run_device(args, rank, world, device):
     from fp4_quantized_gemms_b200 import ufp4
     peaks, peak_kind = load_peaks()
@@ -240,6 +305,9 @@ def run_device(args, rank, world, device):
 
     # ---- end to end through the public API with host buffers (rank-local)
     e2e = run_e2e(step, args, device)
+
+    # ---- grouped (MoE) GEMMs of the mixture-of-experts config (reported, not in `value`)
+    moe = run_moe(device, step.two)
 
     value = world * flops / (ms_per_step * 1e-3) / 1e12
     gemm_tf = [2 * s.M * s.N * s.K / (g * 1e-3) / 1e12 for g in g_ms]
@@ -298,6 +366,7 @@ def run_device(args, rank, world, device):
             "traffic": None,
         },
         "e2e": e2e,
+        "moe_grouped": moe,
         "device_status": ufp4.status_string(status),
     }
     result["clocks"] = clk.summary()
