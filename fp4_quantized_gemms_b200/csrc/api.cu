@@ -29,7 +29,8 @@ int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool cfg_valid(const ufp4_quant_cfg_t &c) {
-    if (c.grid != UFP4_GRID_E1M2 && c.grid != UFP4_GRID_E2M1) return false;
+    if (c.grid != UFP4_GRID_E1M2 && c.grid != UFP4_GRID_E2M1 && c.grid != UFP4_GRID_E2M1_MAX2)
+        return false;
     if (c.rounding != UFP4_ROUND_RTNE && c.rounding != UFP4_ROUND_SR) return false;
     if (!(c.hadamard_n == 0 || c.hadamard_n == 16 || c.hadamard_n == 32 || c.hadamard_n == 64))
         return false;
@@ -243,7 +244,9 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
     }
     // Native kernels store 16-byte pieces when the output allows it.
     args.c_vec = (aligned16(c) && ldc % 4 == 0) ? 1 : 0;
-    cudaError_t e = launch_gemm(args, mode, a->cfg.grid, sm_count(), st);
+    // The restricted E2M1 grid stores E2M1 codes (0..4): the E2M1 kernels.
+    const int grid_kind = a->cfg.grid == UFP4_GRID_E1M2 ? 0 : 1;
+    cudaError_t e = launch_gemm(args, mode, grid_kind, sm_count(), st);
     return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
 }
 

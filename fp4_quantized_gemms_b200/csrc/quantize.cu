@@ -36,29 +36,37 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
+// Grids: 0 = E1M2 (levels k/4, k <= 7), 1 = E2M1 (OCP FP4 magnitudes),
+// 2 = E2M1 restricted to max_fpx = 2.0 (the E2M1 codes 0..4, levels k/2).
+// Grids 0 and 2 are uniform: level k = k / kUnit.
+template <int GRID>
+constexpr int top_of() { return GRID == 2 ? 4 : 7; }
+template <int GRID>
+constexpr float unit_of() { return GRID == 0 ? 4.0f : 2.0f; }
+
 template <int GRID>
 __device__ __forceinline__ float level_of(int k) {
-    if (GRID == 0) return static_cast<float>(k) * 0.25f;
+    if (GRID != 1) return static_cast<float>(k) * (1.0f / unit_of<GRID>());
     return k <= 4 ? static_cast<float>(k) * 0.5f : (k == 5 ? 3.0f : (k == 6 ? 4.0f : 6.0f));
 }
 
-// Midpoint between level j and level j+1 (j in 0..6), exact in fp32.
+// Midpoint between level j and level j+1 (j < top), exact in fp32.
 template <int GRID>
 __device__ __forceinline__ float mid_of(int j) {
-    if (GRID == 0) return static_cast<float>(2 * j + 1) * 0.125f;
+    if (GRID != 1) return static_cast<float>(2 * j + 1) * (0.5f / unit_of<GRID>());
     return j <= 3 ? static_cast<float>(2 * j + 1) * 0.25f
                   : (j == 4 ? 2.5f : (j == 5 ? 3.5f : 5.0f));
 }
 
 template <int GRID>
 __device__ __forceinline__ float gmax_of() {
-    return GRID == 0 ? 1.75f : 6.0f;
+    return GRID == 0 ? 1.75f : (GRID == 1 ? 6.0f : 2.0f);
 }
 
 // Nearest level index of an approximate quotient y (within one of the truth).
 template <int GRID>
 __device__ __forceinline__ int estimate_nearest(float y) {
-    if (GRID == 0) return min(max(__float2int_rn(y * 4.0f), 0), 7);
+    if (GRID != 1) return min(max(__float2int_rn(y * unit_of<GRID>()), 0), top_of<GRID>());
     return (y > 0.25f) + (y > 0.75f) + (y > 1.25f) + (y > 1.75f) + (y > 2.5f) + (y > 3.5f) +
            (y > 5.0f);
 }
@@ -66,7 +74,7 @@ __device__ __forceinline__ int estimate_nearest(float y) {
 // Largest level index whose level is <= y (approximate, within one).
 template <int GRID>
 __device__ __forceinline__ int estimate_floor(float y) {
-    if (GRID == 0) return min(max(__float2int_rd(y * 4.0f), 0), 7);
+    if (GRID != 1) return min(max(__float2int_rd(y * unit_of<GRID>()), 0), top_of<GRID>());
     return (y >= 0.5f) + (y >= 1.0f) + (y >= 1.5f) + (y >= 2.0f) + (y >= 3.0f) + (y >= 4.0f) +
            (y >= 6.0f);
 }
@@ -84,7 +92,7 @@ __device__ __forceinline__ int round_rtne(float au, float m1, float b, float inv
         // Subnormal step: no usable reciprocal, count the boundaries passed.
         int k = 0;
 #pragma unroll
-        for (int j = 0; j < 7; ++j) {
+        for (int j = 0; j < top_of<GRID>(); ++j) {
             const float d = exact_diff(au, mid_of<GRID>(j), m1, b);
             if (d > 0.0f || (d == 0.0f && (j & 1))) k = j + 1;
         }
@@ -95,7 +103,7 @@ __device__ __forceinline__ int round_rtne(float au, float m1, float b, float inv
         const float d = exact_diff(au, mid_of<GRID>(k - 1), m1, b);
         if (d < 0.0f || (d == 0.0f && (k & 1))) --k;
     }
-    if (k < 7) {
+    if (k < top_of<GRID>()) {
         const float d = exact_diff(au, mid_of<GRID>(k), m1, b);
         if (d > 0.0f || (d == 0.0f && (k & 1))) ++k;
     }
@@ -110,17 +118,17 @@ __device__ __forceinline__ int round_sr(float au, float m1, float b, float inv, 
     if (!(fabsf(inv) < INFINITY)) {
         lo = 0;
 #pragma unroll
-        for (int j = 1; j < 8; ++j)
+        for (int j = 1; j <= top_of<GRID>(); ++j)
             if (exact_diff(au, level_of<GRID>(j), m1, b) >= 0.0f) lo = j;
     } else {
         lo = estimate_floor<GRID>(au * inv);
         if (lo > 0 && exact_diff(au, level_of<GRID>(lo), m1, b) < 0.0f) {
             --lo;
-        } else if (lo < 7 && exact_diff(au, level_of<GRID>(lo + 1), m1, b) >= 0.0f) {
+        } else if (lo < top_of<GRID>() && exact_diff(au, level_of<GRID>(lo + 1), m1, b) >= 0.0f) {
             ++lo;
         }
     }
-    if (lo >= 7) return 7;
+    if (lo >= top_of<GRID>()) return top_of<GRID>();
     const float l0 = level_of<GRID>(lo);
     const float step = level_of<GRID>(lo + 1) - l0;
     const float c = __fmaf_rn(static_cast<float>(r16), step * (1.0f / 65536.0f), l0);
@@ -318,29 +326,31 @@ __device__ __forceinline__ uint2 round_pack(const float (&v)[16], const ScaleOut
     if (sc.zero) return make_uint2(0u, 0u);
     uint32_t w[2] = {0u, 0u};
     bool risky = !(sc.inv * 4.0f < INFINITY);   // tiny (subnormal) step: exact path
-    if (GRID == 0 && RND == 0) {
-        // E1M2 RTNE: k = rint(min(|u| * 4/s, 7)).
-        const float inv4 = sc.inv * 4.0f;
+    constexpr float kTop = static_cast<float>(top_of<GRID>());
+    if (GRID != 1 && RND == 0) {
+        // Uniform grid RTNE: k = rint(min(|u| * unit/s, top)).
+        const float inv4 = sc.inv * unit_of<GRID>();
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const float u = v[i];
-            const float y = fminf(fabsf(u) * inv4, 7.0f);
+            const float y = fminf(fabsf(u) * inv4, kTop);
             const float f = y + kRound;
             risky |= fabsf(y - (f - kRound)) > 0.5f - kMargin;
             const uint32_t code = (__float_as_uint(f) & 7u) | ((__float_as_uint(u) >> 28) & 8u);
             w[i >> 3] |= code << (4 * (i & 7));
         }
-    } else if (GRID == 0 && RND == 1) {
-        // E1M2 SR.  With q = |u|/(s/4) and r = r16 * 2^-16, "lo = floor(q), up
-        // iff q > lo + r" is exactly k = ceil(q - r): for q = lo + f the value
-        // q - r lies in (lo, lo+1) when f > r and in (lo-1, lo] otherwise.
-        // q >= 7 gives 7 (clamp first).  ceil(t) = rint(t + 1/2) except when t
-        // is (near) an integer, which the margin test sends to the exact path.
-        const float inv4 = sc.inv * 4.0f;
+    } else if (GRID != 1 && RND == 1) {
+        // Uniform grid SR.  With q = |u|/(s/unit) and r = r16 * 2^-16, "lo =
+        // floor(q), up iff q > lo + r" is exactly k = ceil(q - r): for q =
+        // lo + f the value q - r lies in (lo, lo+1) when f > r and in
+        // (lo-1, lo] otherwise.  q >= top gives top (clamp first).  ceil(t) =
+        // rint(t + 1/2) except when t is (near) an integer, which the margin
+        // test sends to the exact path.
+        const float inv4 = sc.inv * unit_of<GRID>();
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const float u = v[i];
-            const float y = fminf(fabsf(u) * inv4, 7.0f);
+            const float y = fminf(fabsf(u) * inv4, kTop);
             const uint32_t word = rnd[i >> 1];
             const uint32_t r16 = (i & 1) ? (word >> 16) : (word & 0xFFFFu);
             const float rf = __uint_as_float(0x4B000000u | r16) - 8388608.0f;   // r16 exactly
@@ -396,19 +406,20 @@ __device__ __forceinline__ float r16_magic(uint32_t w, bool hi) {
     return __uint_as_float(d);
 }
 
-// E1M2, RTNE or SR, for two chunks with their own block scales: the fast
-// paths of round_pack (same decisions, same certification) with the fp32
-// adds / fmas done two lanes at a time.
-template <int RND>
-__device__ __forceinline__ void round_pack2_e1m2(const float (&va)[16], const float (&vb)[16],
+// A uniform grid (E1M2 or restricted E2M1), RTNE or SR, for two chunks with
+// their own block scales: the fast paths of round_pack (same decisions, same
+// certification) with the fp32 adds / fmas done two lanes at a time.
+template <int GRID, int RND>
+__device__ __forceinline__ void round_pack2_uniform(const float (&va)[16], const float (&vb)[16],
                                                  const ScaleOut &sa, const ScaleOut &sb,
                                                  const PhiloxKeys &keys, uint32_t stream, uint64_t seed,
                                                  uint64_t L0a, uint64_t L0b, uint2 &outa, uint2 &outb) {
-    const float inv4a = sa.inv * 4.0f, inv4b = sb.inv * 4.0f;
-    // min(|u| * inv4, 7) as 7 * sat(|u| * inv4 / 7): a saturating multiply on
-    // the fma pipe instead of a min (the estimate moves by a few ulp, far
-    // inside the 2^-16 margin; at and above 7 both give exactly 7).
-    const float c7a = inv4a * (1.0f / 7.0f), c7b = inv4b * (1.0f / 7.0f);
+    constexpr float kTop = static_cast<float>(top_of<GRID>());
+    const float inv4a = sa.inv * unit_of<GRID>(), inv4b = sb.inv * unit_of<GRID>();
+    // min(|u| * inv4, top) as top * sat(|u| * inv4 / top): a saturating
+    // multiply on the fma pipe instead of a min (the estimate moves by a few
+    // ulp, far inside the 2^-16 margin; at and above top both give top).
+    const float c7a = inv4a * (1.0f / kTop), c7b = inv4b * (1.0f / kTop);
     float deva = 0.0f, devb = 0.0f;      // largest distance from a rint half-way point
     uint32_t wa[2] = {0u, 0u}, wb[2] = {0u, 0u};
     const float2 kR = make_float2(kRound, kRound);
@@ -437,9 +448,9 @@ __device__ __forceinline__ void round_pack2_e1m2(const float (&va)[16], const fl
                 const float2 rf = __fadd2_rn(make_float2(r16_magic(rwa[e >> 1], e & 1), r16_magic(rwb[e >> 1], e & 1)),
                                              make_float2(-8421376.0f, -8421376.0f));   // r16 - 2^15
                 const float2 rt = __fmul2_rn(rf, make_float2(-1.0f / 65536.0f, -1.0f / 65536.0f));   // exact
-                h = __ffma2_rn(y7, make_float2(7.0f, 7.0f), rt);
+                h = __ffma2_rn(y7, make_float2(kTop, kTop), rt);
             } else {
-                h = __fmul2_rn(y7, make_float2(7.0f, 7.0f));
+                h = __fmul2_rn(y7, make_float2(kTop, kTop));
             }
             const float2 f = __fadd2_rn(h, kR);
             const float2 g = __fadd2_rn(f, kRn);
@@ -460,12 +471,12 @@ __device__ __forceinline__ void round_pack2_e1m2(const float (&va)[16], const fl
     if (riska && !sa.zero) {
         const Chunk16 c{make_float4(va[0], va[1], va[2], va[3]), make_float4(va[4], va[5], va[6], va[7]),
                         make_float4(va[8], va[9], va[10], va[11]), make_float4(va[12], va[13], va[14], va[15])};
-        outa = round_pack_exact<0, RND>(c, sa, RandSrc{seed, L0a, stream});
+        outa = round_pack_exact<GRID, RND>(c, sa, RandSrc{seed, L0a, stream});
     }
     if (riskb && !sb.zero) {
         const Chunk16 c{make_float4(vb[0], vb[1], vb[2], vb[3]), make_float4(vb[4], vb[5], vb[6], vb[7]),
                         make_float4(vb[8], vb[9], vb[10], vb[11]), make_float4(vb[12], vb[13], vb[14], vb[15])};
-        outb = round_pack_exact<0, RND>(c, sb, RandSrc{seed, L0b, stream});
+        outb = round_pack_exact<GRID, RND>(c, sb, RandSrc{seed, L0b, stream});
     }
 }
 
@@ -680,8 +691,9 @@ __global__ void __launch_bounds__(kCtaThreads, 3) rht_quantize_kernel(const __gr
                 const uint64_t L0a = static_cast<uint64_t>(orow) * static_cast<uint64_t>(a.kpad) +
                                      static_cast<uint64_t>(k0 + gp);
                 uint2 pa, pb;
-                if (GRID == 0) {
-                    round_pack2_e1m2<RND>(va, vb, sa, sb, keys, a.stream, a.seed, L0a, L0a + 16, pa, pb);
+                if (GRID != 1) {
+                    round_pack2_uniform<GRID, RND>(va, vb, sa, sb, keys, a.stream, a.seed, L0a, L0a + 16,
+                                                   pa, pb);
                 } else {
                     pa = round_pack<GRID, RND>(va, sa, keys, a.stream, L0a, a.seed);
                     pb = round_pack<GRID, RND>(vb, sb, keys, a.stream, L0a + 16, a.seed);
@@ -824,6 +836,10 @@ cudaError_t dispatch_grid_round(const QuantArgs &a, const CUtensorMap &m, int gr
     if (grid_kind == 0) {
         return rnd == 0 ? launch_one<AXIS, NH, BLK, 0, 0, false>(a, m, num_sms, stream)
                         : launch_one<AXIS, NH, BLK, 0, 1, false>(a, m, num_sms, stream);
+    }
+    if (grid_kind == 2) {
+        return rnd == 0 ? launch_one<AXIS, NH, BLK, 2, 0, false>(a, m, num_sms, stream)
+                        : launch_one<AXIS, NH, BLK, 2, 1, false>(a, m, num_sms, stream);
     }
     return rnd == 0 ? launch_one<AXIS, NH, BLK, 1, 0, false>(a, m, num_sms, stream)
                     : launch_one<AXIS, NH, BLK, 1, 1, false>(a, m, num_sms, stream);

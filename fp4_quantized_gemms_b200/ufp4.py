@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libufp4.so")
 # enums (include/ufp4.h)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_OPERAND_MISMATCH, ERR_CUDA, \
     ERR_DEVICE_TIMEOUT = range(7)
-GRID_E1M2, GRID_E2M1 = 0, 1
+GRID_E1M2, GRID_E2M1, GRID_E2M1_MAX2 = 0, 1, 2
 ROUND_RTNE, ROUND_SR = 0, 1
 SCALE_FP32, SCALE_E4M3_X_FP32 = 0, 1
 ALONG_COLS, ALONG_ROWS = 0, 1

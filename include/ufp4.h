@@ -35,7 +35,8 @@
  *   codes     u8 [rows][kpad/2], row-major.  Byte j of a row holds element 2j
  *             in its low nibble and element 2j+1 in its high nibble.  A nibble
  *             is sign-magnitude: bit 3 = sign, bits 0..2 = magnitude index k
- *             of the grid (E1M2: k/4; E2M1: {0,.5,1,1.5,2,3,4,6}[k]).  Zero is
+ *             of the grid (E1M2: k/4; E2M1: {0,.5,1,1.5,2,3,4,6}[k]; the
+ *             restricted E2M1 grid uses k <= 4 of the E2M1 list).  Zero is
  *             always 0x0, never 0x8.
  *   scales    block-major: entry (row r, block b) at scales[b*scale_ld + r],
  *             scale_ld = rows rounded up to a multiple of 64.
@@ -74,8 +75,17 @@ typedef enum {
 } ufp4_status_t;
 
 /* 4-bit grids, [PL] §2 "FP4 formats" and §4.  INT4 is the E1M2 grid (same
- * codes under absmax scaling). */
-typedef enum { UFP4_GRID_E1M2 = 0, UFP4_GRID_E2M1 = 1 } ufp4_grid_t;
+ * codes under absmax scaling).  UFP4_GRID_E2M1_MAX2 is the range-restricted
+ * E2M1 variant of [PL] §5 "Q4: Recipe ablations" (max_fpx = 2.0): block
+ * scales map the block maximum to 2.0 and only the E2M1 magnitudes
+ * {0, 0.5, 1, 1.5, 2} (codes 0..4) are used; its codes are E2M1 codes, so its
+ * operands run on the E2M1 GEMM kernels.  Operands of one GEMM must share a
+ * grid (else UFP4_ERR_OPERAND_MISMATCH). */
+typedef enum {
+    UFP4_GRID_E1M2 = 0,
+    UFP4_GRID_E2M1 = 1,
+    UFP4_GRID_E2M1_MAX2 = 2
+} ufp4_grid_t;
 /* Rounding rules, [PL] §2 "Rounding rules": RTNE for X and W, SR on dY. */
 typedef enum { UFP4_ROUND_RTNE = 0, UFP4_ROUND_SR = 1 } ufp4_round_t;
 /* Block scale formats: plain fp32 per block, or the two-level hierarchy of

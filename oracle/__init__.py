@@ -28,7 +28,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "ufp4_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "libufp4_oracle.so")
 
-GRID_E1M2, GRID_E2M1 = 0, 1
+GRID_E1M2, GRID_E2M1, GRID_E2M1_MAX2 = 0, 1, 2
 ROUND_RTNE, ROUND_SR = 0, 1
 SCALE_FP32, SCALE_E4M3_X_FP32 = 0, 1
 ALONG_COLS, ALONG_ROWS = 0, 1
@@ -69,6 +69,8 @@ def lib():
         L.uo_level.argtypes = [i32, i32]
         L.uo_gmax.restype = ctypes.c_double
         L.uo_gmax.argtypes = [i32]
+        L.uo_top_code.restype = i32
+        L.uo_top_code.argtypes = [i32]
         L.uo_fwht_f32.argtypes = [P, i32]
         L.uo_fwht_f64.argtypes = [P, i32]
         L.uo_e4m3_rne_satfinite.restype = ctypes.c_uint8
@@ -115,8 +117,14 @@ def level(grid: int, k: int) -> float:
     return lib().uo_level(grid, k)
 
 
+def top_code(grid: int) -> int:
+    """Largest magnitude code the grid uses (7; 4 for E2M1 with max 2.0)."""
+    return int(lib().uo_top_code(grid))
+
+
 def levels(grid: int) -> np.ndarray:
-    return np.array([level(grid, k) for k in range(8)])
+    """Magnitudes of codes 0 .. top_code(grid), indexed by code."""
+    return np.array([level(grid, k) for k in range(top_code(grid) + 1)])
 
 
 def gmax(grid: int) -> float:

@@ -29,11 +29,18 @@ static const double kE2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
 double uo_level(int grid, int k)
 {
     if (k < 0 || k > 7) return 0.0;
-    if (grid == UO_GRID_E2M1) return kE2M1[k];
+    if (grid == UO_GRID_E2M1 || grid == UO_GRID_E2M1_MAX2) return kE2M1[k];
     return (double)k / 4.0;
 }
 
-double uo_gmax(int grid) { return uo_level(grid, 7); }
+/* The largest magnitude code a grid uses.  The range-restricted E2M1 variant
+ * ([PL] §5 Q4, max_fpx = 2.0) keeps the E2M1 code points but stops at code 4
+ * (magnitude 2.0): block scales map the block maximum to 2.0 and larger
+ * quotients saturate there.  Reading: "max_fpx" is the grid maximum that the
+ * scale targets, the level set being the printed {0, 0.5, 1, 1.5, 2}. */
+int uo_top_code(int grid) { return grid == UO_GRID_E2M1_MAX2 ? 4 : 7; }
+
+double uo_gmax(int grid) { return uo_level(grid, uo_top_code(grid)); }
 
 float uo_bf16_to_f32(uint16_t b)
 {
@@ -178,13 +185,14 @@ uint32_t uo_sr_u16(uint64_t seed, uint32_t stream, uint64_t L)
  * Magnitudes beyond gmax saturate to gmax ("no clipping", [PL] limitations). */
 int uo_round_rtne(int grid, double au, double s)
 {
-    for (int j = 0; j < 7; j++) {
+    const int top = uo_top_code(grid);
+    for (int j = 0; j < top; j++) {
         double mid = (uo_level(grid, j) + uo_level(grid, j + 1)) / 2.0;
         double t = mid * s;
         if (au < t) return j;
         if (au == t) return (j % 2 == 0) ? j : j + 1;
     }
-    return 7;
+    return top;
 }
 
 /* SR: between the adjacent levels lo <= |u|/s < hi, round up iff
@@ -192,9 +200,10 @@ int uo_round_rtne(int grid, double au, double s)
  * position within the bin (to 2^-16) and values on a level never move. */
 int uo_round_sr(int grid, double au, double s, uint32_t r16)
 {
-    int lo = 7;
+    const int top = uo_top_code(grid);
+    int lo = top;
     while (lo > 0 && uo_level(grid, lo) * s > au) lo--;
-    if (lo == 7) return 7;
+    if (lo == top) return top;
     double L0 = uo_level(grid, lo), L1 = uo_level(grid, lo + 1);
     double c = L0 + (L1 - L0) * ((double)r16 / 65536.0);
     return (au > c * s) ? lo + 1 : lo;

@@ -27,7 +27,7 @@
 extern "C" {
 #endif
 
-enum { UO_GRID_E1M2 = 0, UO_GRID_E2M1 = 1 };
+enum { UO_GRID_E1M2 = 0, UO_GRID_E2M1 = 1, UO_GRID_E2M1_MAX2 = 2 };
 enum { UO_ROUND_RTNE = 0, UO_ROUND_SR = 1 };
 enum { UO_SCALE_FP32 = 0, UO_SCALE_E4M3_X_FP32 = 1 };
 enum { UO_ALONG_COLS = 0, UO_ALONG_ROWS = 1 };
@@ -46,6 +46,7 @@ typedef struct {
 /* grids */
 double uo_level(int grid, int k);
 double uo_gmax(int grid);
+int uo_top_code(int grid);   /* largest magnitude code the grid uses */
 
 /* bf16 bit pattern -> float (exact) */
 float uo_bf16_to_f32(uint16_t b);

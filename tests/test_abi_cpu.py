@@ -100,6 +100,8 @@ def _gemm(L, a, b, c_ptr=64 * 1024, ldc=128):
 def test_gemm_validation_rejects_before_launch(L):
     """Every rejection below happens on the host: no CUDA call is made."""
     assert _gemm(L, _q(grid=0), _q(grid=1)) == ufp4.ERR_OPERAND_MISMATCH
+    assert _gemm(L, _q(grid=1), _q(grid=2)) == ufp4.ERR_OPERAND_MISMATCH
+    assert _gemm(L, _q(grid=3), _q(grid=3)) == ufp4.ERR_INVALID_ARG
     assert _gemm(L, _q(block=16), _q(block=32)) == ufp4.ERR_OPERAND_MISMATCH
     assert _gemm(L, _q(hadamard_n=16), _q(hadamard_n=32)) == ufp4.ERR_OPERAND_MISMATCH
     assert _gemm(L, _q(rht_sign_mask=1), _q(rht_sign_mask=2)) == ufp4.ERR_OPERAND_MISMATCH

@@ -61,7 +61,7 @@ def _cfg(grid=0, fmt=0, n=16, block=16, rounding=0, stream=0):
                             hadamard_n=n, block=block, scale_fmt=fmt)
 
 
-@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1])
+@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1, ufp4.GRID_E2M1_MAX2])
 @pytest.mark.parametrize("fmt", [ufp4.SCALE_FP32, ufp4.SCALE_E4M3_X_FP32])
 def test_fprop_tiny_config(grid, fmt):
     """X 256x512 with 4 outlier columns x20, W 512x512 ~ N(0, 0.02), RHT16, block 16."""
@@ -88,10 +88,11 @@ def test_fprop_ragged_shapes(M, N, K, fmt, grid, n, block):
 
 
 @pytest.mark.parametrize("fmt", [ufp4.SCALE_FP32, ufp4.SCALE_E4M3_X_FP32])
-@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1])
+@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1, ufp4.GRID_E2M1_MAX2])
 def test_layer_dgrad_wgrad_small(fmt, grid):
     """The full recipe on a small layer: RHT on every operand along its GEMM's
-    K, RTNE for X / W, SR on dY (stream 0 for DGRAD, 1 for WGRAD)."""
+    K, RTNE for X / W, SR on dY (stream 0 for DGRAD, 1 for WGRAD).  With the
+    restricted E2M1 grid this is the full-RHT max_fpx = 2.0 ablation."""
     M, K, N = 384, 320, 264
     X = wl.normal_with_outlier_channels(M, K, 1.0, 3, 30.0)
     W = wl.normal(N, K, 0.02, 2)
@@ -160,12 +161,12 @@ def test_large_config_sampled(gemm, fmt, grid):
 @pytest.mark.parametrize("path", [ufp4.GEMM_PATH_NATIVE_FP4, ufp4.GEMM_PATH_NATIVE_FP4_PAIR,
                                   ufp4.GEMM_PATH_FP16])
 @pytest.mark.parametrize("corr", [True, False])
-@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1])
+@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1, ufp4.GRID_E2M1_MAX2])
 def test_two_level_kernel_families(path, corr, grid):
     """Every kernel family for two-level scales gives the oracle's result, with
     the E1M2 correction planes stored by the quantizer or derived in the GEMM;
     shapes with partial tiles in M, N (224-wide tiles) and a K tail."""
-    if grid == ufp4.GRID_E2M1 and corr:
+    if grid != ufp4.GRID_E1M2 and corr:
         pytest.skip("correction planes exist for E1M2 only")
     old = ufp4.get_two_level_gemm_path()
     ufp4.set_two_level_gemm_path(path)

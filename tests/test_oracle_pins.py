@@ -15,7 +15,8 @@ import oracle
 from fp4_quantized_gemms_b200 import workloads as wl
 from tests.conftest import read_golden
 
-E1M2, E2M1 = oracle.GRID_E1M2, oracle.GRID_E2M1
+E1M2, E2M1, MAX2 = oracle.GRID_E1M2, oracle.GRID_E2M1, oracle.GRID_E2M1_MAX2
+ALL_GRIDS = [E1M2, E2M1, MAX2]
 
 
 # ------------------------------------------------------------------ RHT (C1)
@@ -92,6 +93,17 @@ def test_e2m1_range_restricted_prefix_matches_pages():
     lv = oracle.levels(E2M1)
     assert list(lv[lv <= float(g["max_fpx"])]) == printed
     assert oracle.gmax(E2M1) == 6.0
+    # the restricted grid itself: exactly the printed set, topped at max_fpx,
+    # with the E2M1 code points (code k means the same magnitude in both)
+    assert list(oracle.levels(MAX2)) == printed
+    assert oracle.gmax(MAX2) == float(g["max_fpx"]) and oracle.top_code(MAX2) == 4
+    assert list(oracle.levels(MAX2)) == list(lv[:5])
+
+
+def test_e2m1_range_restricted_grid_is_uniform():
+    """The restricted set is uniform (step 0.5): no geometric asymmetry, so no
+    conditional RTNE bias at its interior levels (checked by Monte Carlo below)."""
+    assert np.all(np.diff(oracle.levels(MAX2)) == 0.5)
 
 
 def _half_widths(grid, i):
@@ -114,6 +126,7 @@ def test_shrinkage_bias_worked_example_matches_pages():
     (E2M1, 3.0, 0.0), (E2M1, 4.0, -0.25),
     (E1M2, 0.25, 0.0), (E1M2, 0.5, 0.0), (E1M2, 0.75, 0.0), (E1M2, 1.0, 0.0),
     (E1M2, 1.25, 0.0), (E1M2, 1.5, 0.0),
+    (MAX2, 0.5, 0.0), (MAX2, 1.0, 0.0), (MAX2, 1.5, 0.0),
 ])
 def test_rtne_conditional_bias_monte_carlo(grid, level, expect):
     """P6: uniform draws inside the RTNE bin of a level, rounded by the oracle,
@@ -140,7 +153,7 @@ def _brute_rtne(grid, u, s):
     uf, sf = Fraction(u), Fraction(s)
     lv = [Fraction(v) for v in oracle.levels(grid)]
     best = None
-    for k in range(8):
+    for k in range(len(lv)):
         for sign in (1, -1):
             if k == 0 and sign == -1:
                 continue
@@ -151,7 +164,7 @@ def _brute_rtne(grid, u, s):
     return best[1]
 
 
-@pytest.mark.parametrize("grid", [E1M2, E2M1])
+@pytest.mark.parametrize("grid", ALL_GRIDS)
 def test_rtne_matches_brute_force_sweep(grid):
     """P9: dense sweep of |u|/s across every bin, exact ties and both edges."""
     lv = oracle.levels(grid)
@@ -168,7 +181,7 @@ def test_rtne_matches_brute_force_sweep(grid):
     assert list(got) == want
 
 
-@pytest.mark.parametrize("grid", [E1M2, E2M1])
+@pytest.mark.parametrize("grid", ALL_GRIDS)
 def test_rtne_matches_brute_force_random_blocks(grid):
     """P9 on random 16-blocks with non-power-of-two fp32 scales."""
     rng = np.random.default_rng(5)
@@ -180,17 +193,17 @@ def test_rtne_matches_brute_force_random_blocks(grid):
         want = [_brute_rtne(grid, float(abs(v)), float(s)) for v in u]
         assert list(got) == want
         # P8: the block maximum maps to gmax (no clipping)
-        assert got.max() == 7
+        assert got.max() == len(oracle.levels(grid)) - 1
 
 
-@pytest.mark.parametrize("grid", [E1M2, E2M1])
+@pytest.mark.parametrize("grid", ALL_GRIDS)
 def test_sr_is_unbiased_over_seeds(grid):
     """P10: the mean of SR-dequantized values over 2^20 seeds equals x within
     Delta*2^-16 + 4 sigma; P11: every result is one of the two adjacent levels."""
     lv = oracle.levels(grid)
     rng = np.random.default_rng(17 + grid)
     seeds = np.arange(1 << 20, dtype=np.uint64)
-    for lo in [0, 2, 4, 5]:
+    for lo in [0, 2, 4, 5] if grid != MAX2 else [0, 1, 2, 3]:
         x = rng.uniform(lv[lo], lv[lo + 1])
         delta = lv[lo + 1] - lv[lo]
         r16 = oracle.sr_u16_over_seeds(seeds, 0, 12345)
@@ -201,12 +214,12 @@ def test_sr_is_unbiased_over_seeds(grid):
         assert abs(q.mean() - x) <= delta * 2.0 ** -16 + 4 * sigma
 
 
-@pytest.mark.parametrize("grid", [E1M2, E2M1])
+@pytest.mark.parametrize("grid", ALL_GRIDS)
 def test_sr_never_moves_values_on_a_level(grid):
     """P12: a value exactly on a level stays there for every uniform draw."""
     lv = oracle.levels(grid)
     r16 = np.arange(65536, dtype=np.uint32)
-    for k in range(8):
+    for k in range(len(lv)):
         got = oracle.round_sr(grid, np.full(r16.size, lv[k] * 0.375), 0.375, r16)
         assert np.all(got == k)
 
@@ -260,7 +273,7 @@ def _cfg(**kw):
     return oracle.QuantCfg(**kw)
 
 
-@pytest.mark.parametrize("grid", [E1M2, E2M1])
+@pytest.mark.parametrize("grid", ALL_GRIDS)
 @pytest.mark.parametrize("axis", [oracle.ALONG_COLS, oracle.ALONG_ROWS])
 def test_quantize_structure(grid, axis):
     """Canonical zero, |k| <= 7, fp32 scale = RN(amax/gmax) of the rotated block,
@@ -270,14 +283,15 @@ def test_quantize_structure(grid, axis):
     q, u = oracle.quantize(X, axis, cfg, want_u=True)
     K = 72 if axis == oracle.ALONG_COLS else 40
     assert q.kpad == (128 if K == 72 else 64) and q.k == K
+    top = len(oracle.levels(grid)) - 1
     assert not np.any(q.codes == 8)
-    assert np.all((q.codes & 7) <= 7)
+    assert np.all((q.codes & 7) <= top)
     nb = q.kpad // 16
     amax = np.abs(u.reshape(u.shape[0], nb, 16)).max(axis=2)
     want = (amax / np.float32(oracle.gmax(grid))).astype(np.float32)
     assert np.array_equal(q.scales, want)
     mags = (q.codes & 7).reshape(q.codes.shape[0], nb, 16).max(axis=2)
-    assert np.all(mags[amax > 0] == 7)
+    assert np.all(mags[amax > 0] == top)
     assert np.all(u[:, ((K + 15) // 16) * 16:] == 0)
 
 
@@ -323,7 +337,7 @@ def test_gemm_oracle_exact_on_grid_values():
     assert all(Fraction(float(C[i, j])) == exact[i, j] for i in range(M) for j in range(N))
 
 
-@pytest.mark.parametrize("grid", [E1M2, E2M1])
+@pytest.mark.parametrize("grid", ALL_GRIDS)
 @pytest.mark.parametrize("scale_fmt", [oracle.SCALE_FP32, oracle.SCALE_E4M3_X_FP32])
 def test_quantized_gemm_tracks_bf16_gemm(grid, scale_fmt):
     """End to end: the oracle's quantized FPROP approximates the fp64 X W^T of
@@ -362,3 +376,55 @@ def test_two_level_scales_follow_hierarchy():
     assert np.all(np.abs(deq[sat]) == top_level[sat])
     step = e * q.S * 0.25
     assert np.all(np.abs(deq - u)[~sat] <= step[~sat] / 2 * (1 + 1e-6))
+
+
+# ------------------------------------------------------------------ restricted E2M1
+def test_restricted_e2m1_rounding_is_scaled_e1m2_rounding_capped():
+    """The restricted levels are 2x the E1M2 levels of codes 0..4, so rounding
+    |u| at scale s onto them must pick the E1M2 code of |u| at scale 2s, capped
+    at 4 (both rules are exact-quotient; both break ties to even codes).  A
+    wrong top code, a stale loop bound or a missed saturation fails this."""
+    rng = np.random.default_rng(33)
+    s = 0.375
+    au = np.concatenate([rng.uniform(0, 3.0 * s, 200_000),
+                         s * np.arange(0, 2.5, 0.25)])           # levels and midpoints
+    want = np.minimum(oracle.round_rtne(E1M2, au, 2 * s), 4)
+    assert np.array_equal(oracle.round_rtne(MAX2, au, s), want)
+    r16 = rng.integers(0, 65536, au.size).astype(np.uint32)
+    got = oracle.round_sr(MAX2, au, s, r16)
+    inside = au <= 2.0 * s
+    assert np.array_equal(got[inside], oracle.round_sr(E1M2, au[inside], 2 * s, r16[inside]))
+    assert np.all(got[~inside] == 4)
+
+
+def test_restricted_e2m1_block_maximum_is_exact():
+    """P8 with max_fpx = 2.0: the fp32 scale is amax/2 (exact), so the element
+    that sets the block maximum dequantizes to itself, code 4."""
+    X = wl.normal_with_outlier_channels(16, 64, 1.0, 2, 20.0)
+    cfg = _cfg(grid=MAX2, hadamard_n=16, sign_mask=0x9A3C, block=16)
+    q, u = oracle.quantize(X, oracle.ALONG_COLS, cfg, want_u=True)
+    deq = q.dequantize()
+    blocks = np.abs(u).reshape(u.shape[0], -1, 16)
+    arg = blocks.argmax(axis=2)
+    r = np.arange(u.shape[0])[:, None]
+    c = np.arange(blocks.shape[1])[None, :] * 16 + arg
+    assert np.array_equal(np.abs(deq[r, c]), blocks.max(axis=2).astype(np.float64))
+    assert np.all((q.codes[r, c] & 7) == 4)
+
+
+def test_restricted_e2m1_two_level_tensor_scale():
+    """Two-level scales with max_fpx = 2.0: S maps the rotated tensor amax to
+    2.0 x 448; blocks whose E4M3 factor rounds down saturate at code 4."""
+    X = wl.student_t(32, 256)
+    cfg = _cfg(grid=MAX2, hadamard_n=16, sign_mask=0x5EED, block=16,
+               scale_fmt=oracle.SCALE_E4M3_X_FP32)
+    amax = oracle.rht_amax(X, oracle.ALONG_COLS, 16, 0x5EED)
+    q, u = oracle.quantize(X, oracle.ALONG_COLS, cfg, tensor_amax=amax, want_u=True)
+    assert q.S == np.float32(amax / np.float32(896.0))
+    assert np.all((q.codes & 7) <= 4)
+    e = np.array([[oracle.e4m3_value(b) for b in row] for row in q.escales]).repeat(16, axis=1)
+    top_level = 2.0 * e * q.S
+    deq = q.dequantize()
+    sat = np.abs(u) > top_level
+    assert np.all(np.abs(deq[sat]) == top_level[sat])
+    assert np.all(np.abs(deq - u)[~sat] <= (0.25 * e * q.S)[~sat] * (1 + 1e-6))

@@ -42,7 +42,7 @@ def _run(x_bits, axis, cfg, rows=None):
     return q
 
 
-GRID_ROUND_FMT = list(itertools.product([ufp4.GRID_E1M2, ufp4.GRID_E2M1],
+GRID_ROUND_FMT = list(itertools.product([ufp4.GRID_E1M2, ufp4.GRID_E2M1, ufp4.GRID_E2M1_MAX2],
                                         [ufp4.ROUND_RTNE, ufp4.ROUND_SR],
                                         [ufp4.SCALE_FP32, ufp4.SCALE_E4M3_X_FP32]))
 
@@ -60,7 +60,7 @@ def test_quantize_matches_oracle_small(axis, n, block, grid, rounding, fmt):
 
 
 @pytest.mark.parametrize("axis", AXES)
-@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1])
+@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1, ufp4.GRID_E2M1_MAX2])
 def test_quantize_exact_ties_and_zero_blocks(axis, grid):
     """n = 0 with values on grid midpoints (exact RTNE ties), level values (SR
     must not move them), all-zero blocks and a block whose max is tiny."""
@@ -83,7 +83,7 @@ def test_quantize_exact_ties_and_zero_blocks(axis, grid):
 @pytest.mark.parametrize("axis", AXES)
 def test_quantize_medium_with_outliers(axis):
     X = wl.normal_with_outlier_channels(1000, 1000, 1.0, 5, 30.0)
-    for grid, rnd in [(0, 0), (0, 1), (1, 0)]:
+    for grid, rnd in [(0, 0), (0, 1), (1, 0), (2, 0), (2, 1)]:
         cfg = ufp4.QuantConfig(grid=grid, rounding=rnd, sr_seed=1234, hadamard_n=16, block=16)
         _run(X, axis, cfg)
 
