@@ -88,6 +88,12 @@ ufp4_status_t check_qtensor(const ufp4_qtensor_t *q) {
     return UFP4_OK;
 }
 
+// D agrees on its n positions (mask bits beyond n are unused).
+bool same_signs(uint64_t x, uint64_t y, int n) {
+    const uint64_t m = n == 64 ? ~uint64_t(0) : ((uint64_t(1) << n) - 1);
+    return (x & m) == (y & m);
+}
+
 ufp4_status_t check_pair(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b, bool same_k) {
     ufp4_status_t s = check_qtensor(a);
     if (s != UFP4_OK) return s;
@@ -97,10 +103,8 @@ ufp4_status_t check_pair(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b, bool 
     if (x.grid != y.grid || x.block != y.block || x.scale_fmt != y.scale_fmt ||
         x.hadamard_n != y.hadamard_n)
         return UFP4_ERR_OPERAND_MISMATCH;
-    if (x.hadamard_n > 0) {
-        const uint64_t m = x.hadamard_n == 64 ? ~uint64_t(0) : ((uint64_t(1) << x.hadamard_n) - 1);
-        if ((x.rht_sign_mask & m) != (y.rht_sign_mask & m)) return UFP4_ERR_OPERAND_MISMATCH;
-    }
+    if (x.hadamard_n > 0 && !same_signs(x.rht_sign_mask, y.rht_sign_mask, x.hadamard_n))
+        return UFP4_ERR_OPERAND_MISMATCH;
     if (same_k && (a->k != b->k || a->kpad != b->kpad)) return UFP4_ERR_OPERAND_MISMATCH;
     return UFP4_OK;
 }
@@ -261,6 +265,39 @@ ufp4_status_t check_input(const void *x, int64_t rows, int64_t cols, int64_t ld,
     return UFP4_OK;
 }
 
+// Validates `out` against the input shape and fills the kernel arguments of
+// one quantization (x along `axis`).
+ufp4_status_t fill_quant_args(const void *x_dev, int64_t rows, int64_t cols, int64_t ld, int32_t axis,
+                              const float *tensor_amax_dev, const ufp4_qtensor_t *out, QuantArgs *a) {
+    ufp4_status_t s = check_qtensor(out);
+    if (s != UFP4_OK) return s;
+    const int64_t out_rows = axis == UFP4_ALONG_COLS ? rows : cols;
+    const int64_t K = axis == UFP4_ALONG_COLS ? cols : rows;
+    if (out->rows != out_rows || out->k != K) return UFP4_ERR_INVALID_ARG;
+    const bool two_level = out->cfg.scale_fmt == UFP4_SCALE_E4M3_X_FP32;
+    if (two_level && tensor_amax_dev == nullptr) return UFP4_ERR_INVALID_ARG;
+    memset(a, 0, sizeof(*a));
+    a->x = static_cast<const uint16_t *>(x_dev);
+    a->rows = rows;
+    a->cols = cols;
+    a->ld = ld;
+    a->axis = axis;
+    a->out_rows = out_rows;
+    a->K = K;
+    a->kpad = out->kpad;
+    a->scale_ld = out->scale_ld;
+    a->codes = static_cast<uint8_t *>(out->codes);
+    a->corr = static_cast<uint8_t *>(out->corr);
+    a->scales = out->scales;
+    a->S_out = two_level ? out->tensor_scale : nullptr;
+    a->amax_t = two_level ? tensor_amax_dev : nullptr;
+    a->seed = out->cfg.sr_seed;
+    a->stream = out->cfg.sr_stream;
+    a->sign_mask = out->cfg.rht_sign_mask;
+    a->scale_fmt = out->cfg.scale_fmt;
+    return UFP4_OK;
+}
+
 }  // namespace
 
 CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
@@ -359,37 +396,74 @@ ufp4_status_t ufp4_rht_quantize(const void *x_dev, int64_t rows, int64_t cols, i
                                 void *stream) {
     ufp4_status_t s = check_input(x_dev, rows, cols, ld, axis);
     if (s != UFP4_OK) return s;
-    s = check_qtensor(out);
-    if (s != UFP4_OK) return s;
-    const int64_t out_rows = axis == UFP4_ALONG_COLS ? rows : cols;
-    const int64_t K = axis == UFP4_ALONG_COLS ? cols : rows;
-    if (out->rows != out_rows || out->k != K) return UFP4_ERR_INVALID_ARG;
-    const bool two_level = out->cfg.scale_fmt == UFP4_SCALE_E4M3_X_FP32;
-    if (two_level && tensor_amax_dev == nullptr) return UFP4_ERR_INVALID_ARG;
-    if (out_rows == 0 || out->kpad == 0) return UFP4_OK;
     QuantArgs a;
-    memset(&a, 0, sizeof(a));
-    a.x = static_cast<const uint16_t *>(x_dev);
-    a.rows = rows;
-    a.cols = cols;
-    a.ld = ld;
-    a.axis = axis;
-    a.out_rows = out_rows;
-    a.K = K;
-    a.kpad = out->kpad;
-    a.scale_ld = out->scale_ld;
-    a.codes = static_cast<uint8_t *>(out->codes);
-    a.corr = static_cast<uint8_t *>(out->corr);
-    a.scales = out->scales;
-    a.S_out = two_level ? out->tensor_scale : nullptr;
-    a.amax_t = two_level ? tensor_amax_dev : nullptr;
-    a.seed = out->cfg.sr_seed;
-    a.stream = out->cfg.sr_stream;
-    a.sign_mask = out->cfg.rht_sign_mask;
-    a.scale_fmt = out->cfg.scale_fmt;
+    s = fill_quant_args(x_dev, rows, cols, ld, axis, tensor_amax_dev, out, &a);
+    if (s != UFP4_OK) return s;
+    if (a.out_rows == 0 || a.kpad == 0) return UFP4_OK;
     cudaError_t e = launch_rht_quantize(a, out->cfg.hadamard_n, out->cfg.block, out->cfg.grid,
                                         out->cfg.rounding, sm_count(),
                                         static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
+}
+
+ufp4_status_t ufp4_rht_amax_dual(const void *x_dev, int64_t rows, int64_t cols, int64_t ld,
+                                 int32_t hadamard_n, uint64_t rht_sign_mask, float *amax_cols_dev,
+                                 float *amax_rows_dev, void *stream) {
+    ufp4_status_t s = check_input(x_dev, rows, cols, ld, UFP4_ALONG_COLS);
+    if (s != UFP4_OK) return s;
+    if (amax_cols_dev == nullptr || amax_rows_dev == nullptr) return UFP4_ERR_INVALID_ARG;
+    if (!(hadamard_n == 0 || hadamard_n == 16 || hadamard_n == 32 || hadamard_n == 64))
+        return UFP4_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (rows == 0 || cols == 0) {
+        if (cudaMemsetAsync(amax_cols_dev, 0, sizeof(float), st) != cudaSuccess ||
+            cudaMemsetAsync(amax_rows_dev, 0, sizeof(float), st) != cudaSuccess)
+            return UFP4_ERR_CUDA;
+        return UFP4_OK;
+    }
+    QuantArgs ar, ac;
+    memset(&ar, 0, sizeof(ar));
+    ar.x = static_cast<const uint16_t *>(x_dev);
+    ar.rows = rows;
+    ar.cols = cols;
+    ar.ld = ld;
+    ar.sign_mask = rht_sign_mask;
+    ac = ar;
+    ar.axis = UFP4_ALONG_ROWS;
+    ar.out_rows = cols;
+    ar.K = rows;
+    ar.kpad = round_up(rows, kKAlign);
+    ar.amax_out = amax_rows_dev;
+    ac.axis = UFP4_ALONG_COLS;
+    ac.out_rows = rows;
+    ac.K = cols;
+    ac.kpad = round_up(cols, kKAlign);
+    ac.amax_out = amax_cols_dev;
+    cudaError_t e = launch_rht_amax_dual(ar, ac, hadamard_n, sm_count(), st);
+    return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
+}
+
+ufp4_status_t ufp4_rht_quantize_dual(const void *x_dev, int64_t rows, int64_t cols, int64_t ld,
+                                     const float *tensor_amax_cols_dev,
+                                     const float *tensor_amax_rows_dev, ufp4_qtensor_t *out_cols,
+                                     ufp4_qtensor_t *out_rows, void *stream) {
+    ufp4_status_t s = check_input(x_dev, rows, cols, ld, UFP4_ALONG_COLS);
+    if (s != UFP4_OK) return s;
+    QuantArgs ac, ar;
+    s = fill_quant_args(x_dev, rows, cols, ld, UFP4_ALONG_COLS, tensor_amax_cols_dev, out_cols, &ac);
+    if (s != UFP4_OK) return s;
+    s = fill_quant_args(x_dev, rows, cols, ld, UFP4_ALONG_ROWS, tensor_amax_rows_dev, out_rows, &ar);
+    if (s != UFP4_OK) return s;
+    // One kernel computes both: the same recipe on both sides, except the
+    // SR stream (DGRAD and WGRAD draw independent bits from one tensor).
+    const ufp4_quant_cfg_t &c = out_cols->cfg, &r = out_rows->cfg;
+    if (c.grid != r.grid || c.rounding != r.rounding || c.hadamard_n != r.hadamard_n ||
+        c.block != r.block || c.scale_fmt != r.scale_fmt || c.sr_seed != r.sr_seed ||
+        (c.hadamard_n > 0 && !same_signs(c.rht_sign_mask, r.rht_sign_mask, c.hadamard_n)))
+        return UFP4_ERR_UNSUPPORTED;
+    if (rows == 0 || cols == 0) return UFP4_OK;
+    cudaError_t e = launch_rht_quantize_dual(ar, ac, c.hadamard_n, c.block, c.grid, c.rounding, sm_count(),
+                                             static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
 }
 

@@ -481,16 +481,22 @@ __device__ __forceinline__ void round_pack2_uniform(const float (&va)[16], const
 }
 
 // ---------------------------------------------------------------------------
-// Kernel.  A CTA of 256 threads owns a unit of 256 output rows x 64 elements
-// of K; thread t owns output row r0 + t of the unit (all 64 K elements, so any
-// Hadamard size up to 64 and either block size stays inside the thread).  The
-// unit's bf16 tile is staged in shared memory by TMA with the 128-byte
-// swizzle, double-buffered across the CTA's units:
-//   row-wise    one 64 (K) x 256 (rows) box; thread t reads row t, eight
-//               16-byte chunks (chunk c of row t sits at chunk c ^ (t & 7)).
-//   column-wise four 64 (columns) x 64 (K rows) boxes side by side; thread t
-//               reads column t, one bf16 per K row; a warp reads 32
-//               consecutive columns of one K row (no bank conflicts).
+// Kernel.  A CTA of 256 compute threads plus one producer warp takes units of
+// 256 x 64 bf16 elements, staged in shared memory by TMA with the 128-byte
+// swizzle and double-buffered across the CTA's units.  Every compute thread
+// quantizes 64 consecutive K elements of one output row, so any Hadamard size
+// up to 64 and either block size stays inside the thread:
+//   AXIS 0 (row-wise)    one 64 (K) x 256 (rows) box; thread t reads row t,
+//                        eight 16-byte chunks (chunk c of row t sits at chunk
+//                        c ^ (t & 7)).
+//   AXIS 1 (column-wise) four 64 (columns) x 64 (K rows) boxes side by side;
+//                        thread t reads column t, one bf16 per K row; a warp
+//                        reads 32 consecutive columns of one K row.
+//   AXIS 2 (both)        the AXIS 1 tile quantized twice: column-wise into
+//                        `a` exactly as AXIS 1, then row-wise into `a2`, where
+//                        thread t takes row t & 63 of box t >> 6 (64 columns
+//                        of one input row).  One read of the tensor serves
+//                        both of its GEMM operands.
 // Codes (32 bytes per thread) and block-major scales (a warp writes 32
 // consecutive rows of each block) go straight to global memory.
 constexpr int kUnitRows = 256;
@@ -500,222 +506,123 @@ constexpr int kComputeWarps = kThreads / 32;
 constexpr int kCtaThreads = kThreads + 32;        // + one producer warp
 constexpr int kQuantSmem = kStages * kStageBytes + 1024 + 64;
 
-template <int AXIS, int NH, int BLK, int GRID, int RND, bool AMAX_ONLY>
-__global__ void __launch_bounds__(kCtaThreads, 3) rht_quantize_kernel(const __grid_constant__ QuantArgs a,
-                                                                  const __grid_constant__ CUtensorMap tmap) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
-    uint64_t *empty = full + kStages;
-    volatile uint32_t *abort_flag =
-        reinterpret_cast<volatile uint32_t *>(smem + kStages * kStageBytes + 16 * kStages);
-    const int t = threadIdx.x;
-    const int lane = t & 31;
-    const int warp = t >> 5;
-    const int64_t nseg = a.kpad / 64;
-    const int64_t nrb = (a.out_rows + kUnitRows - 1) / kUnitRows;
-    const int64_t nunits = nseg * nrb;
+// Two-level tensor scale of one output: S maps the rotated tensor amax to
+// gmax * 448 (the top of E4M3), G = gmax * S is the block-scale divisor.
+template <int GRID>
+__device__ __forceinline__ void tensor_scale(const QuantArgs &q, float &S, float &G) {
+    const float amax_t = *q.amax_t;
+    S = amax_t > 0.0f ? __fdiv_rn(amax_t, gmax_of<GRID>() * 448.0f) : 1.0f;
+    G = __fmul_rn(gmax_of<GRID>(), S);
+    if (blockIdx.x == 0 && threadIdx.x == 0 && q.S_out) *q.S_out = S;
+}
 
-    auto unit_coords = [&](int64_t u, int64_t &rb, int64_t &seg) {
-        if (AXIS == 0) {
-            rb = u / nseg;
-            seg = u % nseg;
-        } else {
-            seg = u / nrb;
-            rb = u % nrb;
-        }
-    };
-    auto issue = [&](int64_t u, int s) {
-        int64_t rb, seg;
-        unit_coords(u, rb, seg);
-        uint8_t *dst = smem + s * kStageBytes;
-        mbar_arrive_expect_tx(&full[s], kStageBytes);
-        if (AXIS == 0) {
-            tma_load_2d(dst, &tmap, &full[s], static_cast<int32_t>(seg * 64),
-                              static_cast<int32_t>(rb * kUnitRows));
-        } else {
-#pragma unroll
-            for (int b = 0; b < 4; ++b)
-                tma_load_2d(dst + b * 8192, &tmap, &full[s],
-                                  static_cast<int32_t>(rb * kUnitRows + 64 * b),
-                                  static_cast<int32_t>(seg * 64));
-        }
-    };
-
-    if (t == 0) {
-        for (int i = 0; i < kStages; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], kComputeWarps);
-        }
-        *abort_flag = 0u;
-        fence_barrier_init();
-    }
-    __syncthreads();
-    const int64_t u0 = blockIdx.x;
-    if (warp == kComputeWarps) {
-        // Producer warp: refills a stage once every compute warp released it.
-        if (lane == 0) {
-            uint32_t it = 0;
-            for (int64_t u = u0; u < nunits; u += gridDim.x, ++it) {
-                const int s = it % kStages;
-                if (it >= kStages &&
-                    !mbar_wait(&empty[s], ((it / kStages) - 1) & 1, kErrTimeoutProducer, abort_flag))
-                    break;
-                issue(u, s);
-            }
-            // Drain: the last copies have landed before the CTA exits.
-            for (uint32_t d = 0; d < kStages && d < it; ++d) {
-                const uint32_t idx = it - 1 - d;
-                uint32_t dummy = 0;
-                mbar_wait(&full[idx % kStages], (idx / kStages) & 1, kErrTimeoutDrain,
-                          reinterpret_cast<volatile uint32_t *>(&dummy));
-            }
-        }
-        return;
-    }
-
-    float S = 1.0f, G = 0.0f;
-    if (!AMAX_ONLY && a.scale_fmt == 1) {
-        const float amax_t = *a.amax_t;
-        S = amax_t > 0.0f ? __fdiv_rn(amax_t, gmax_of<GRID>() * 448.0f) : 1.0f;
-        G = __fmul_rn(gmax_of<GRID>(), S);
-        if (blockIdx.x == 0 && t == 0 && a.S_out) *a.S_out = S;
-    }
-    // D for the 64 positions of a segment (K offsets are multiples of 64).
-    uint64_t pat = 0;
-    if (NH > 0) {
-        const uint64_t m = NH == 64 ? a.sign_mask : (a.sign_mask & ((1ull << NH) - 1));
-#pragma unroll
-        for (int off = 0; off < 64; off += (NH > 0 ? NH : 64)) pat |= m << off;
-    }
-    const uint32_t pat_lo = static_cast<uint32_t>(pat), pat_hi = static_cast<uint32_t>(pat >> 32);
-    // Sign of D at position i mod 16 as an fp32 sign bit (NH <= 16); adding
-    // it to a widened bf16 flips the sign bit like an xor.
-    uint32_t smask[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) smask[i] = NH > 0 ? ((pat_lo >> i) & 1u) << 31 : 0u;
-    PhiloxKeys keys;
-    if (RND == 1) keys = philox_keys(a.seed);
-    float amax_acc = 0.0f;
-
-    // Column-wise: byte offset of column cc (= t & 63) within K row r of a
-    // 64-column box for r % 8 (the 128-byte swizzle XORs the 16-byte chunk
-    // index with the row mod 8).
-    uint32_t col_off[8];
-    {
-        const int cc = t & 63;
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-            col_off[r] = static_cast<uint32_t>((t >> 6) * 8192 + ((((cc >> 3) ^ r) & 7) << 4) + (cc & 7) * 2);
-    }
-    uint32_t it = 0;
-    for (int64_t u = u0; u < nunits; u += gridDim.x, ++it) {
-        const int s = it % kStages;
-        if (!warp_wait(&full[s], (it / kStages) & 1, kErrTimeoutTransform, abort_flag)) break;
-        int64_t rb, seg;
-        unit_coords(u, rb, seg);
-        const int64_t orow = rb * kUnitRows + t;
-        const int64_t k0 = seg * 64;
-        const uint8_t *tile = smem + s * kStageBytes;
-
-        // ---- per group of GS elements (the Hadamard block and the scale block
-        // both lie inside one group): load, D, H, block scales, round, pack.
-        constexpr int GS = (NH > BLK ? NH : BLK) > 16 ? (NH > BLK ? NH : BLK) : 16;
-        uint32_t codes[8];
-        uint32_t stored[4];
-        if constexpr (GS == 16) {
-            // Groups g and g + 16 side by side as the two lanes of fp32x2
-            // values: same positions mod 16, so the same signs of D; the
-            // butterflies and the rounding arithmetic run two lanes at a time.
-            // Not unrolled: one copy of the body keeps the kernel small.
+// Quantizes K elements [k0, k0 + 64) of output row orow of `a`:
+//   RD 0: they are one swizzled 128-byte row at src (chunk c at (c ^ swz) << 4);
+//   RD 1: they are one column of the four-box tile at src, K row kr at
+//         src + col_off[kr & 7] + kr * 128.
+// The rotated values' amax goes to amax_acc (AMAX_ONLY) or the codes and
+// scales to `a` (rows beyond a.out_rows are computed but not stored).
+template <int RD, int NH, int BLK, int GRID, int RND, bool AMAX_ONLY>
+__device__ __forceinline__ void quantize64(const QuantArgs &a, const uint8_t *src, int swz,
+                                           const uint32_t (&col_off)[8], int64_t orow, int64_t k0,
+                                           float S, float G, const PhiloxKeys &keys,
+                                           const uint32_t (&smask)[16], uint32_t pat_lo,
+                                           uint32_t pat_hi, float &amax_acc) {
+    // Per group of GS elements (the Hadamard block and the scale block both
+    // lie inside one group): load, D, H, block scales, round, pack.
+    constexpr int GS = (NH > BLK ? NH : BLK) > 16 ? (NH > BLK ? NH : BLK) : 16;
+    uint32_t codes[8];
+    uint32_t stored[4];
+    if constexpr (GS == 16) {
+        // Groups g and g + 16 side by side as the two lanes of fp32x2
+        // values: same positions mod 16, so the same signs of D; the
+        // butterflies and the rounding arithmetic run two lanes at a time.
+        // Not unrolled: one copy of the body keeps the kernel small.
 #pragma unroll 1
-            for (int gp = 0; gp < 64; gp += 32) {
-                float va[16], vb[16];
-                if (AXIS == 0) {
-                    const uint8_t *rowp = tile + t * 128;
+        for (int gp = 0; gp < 64; gp += 32) {
+            float va[16], vb[16];
+            if (RD == 0) {
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const uint4 qa = *reinterpret_cast<const uint4 *>(rowp + (((gp / 8 + c) ^ (t & 7)) << 4));
-                        const uint4 qb = *reinterpret_cast<const uint4 *>(rowp + (((gp / 8 + 2 + c) ^ (t & 7)) << 4));
-                        const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w}, wb[4] = {qb.x, qb.y, qb.z, qb.w};
+                for (int c = 0; c < 2; ++c) {
+                    const uint4 qa = *reinterpret_cast<const uint4 *>(src + (((gp / 8 + c) ^ swz) << 4));
+                    const uint4 qb = *reinterpret_cast<const uint4 *>(src + (((gp / 8 + 2 + c) ^ swz) << 4));
+                    const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w}, wb[4] = {qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i0 = 8 * c + 2 * e;
-                            va[i0] = __uint_as_float((wa[e] << 16) + smask[i0]);
-                            va[i0 + 1] = __uint_as_float((wa[e] & 0xFFFF0000u) ^ smask[i0 + 1]);
-                            vb[i0] = __uint_as_float((wb[e] << 16) + smask[i0]);
-                            vb[i0 + 1] = __uint_as_float((wb[e] & 0xFFFF0000u) ^ smask[i0 + 1]);
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int ka = gp + i, kb = gp + 16 + i;
-                        const uint32_t ba = *reinterpret_cast<const uint16_t *>(tile + col_off[ka & 7] + ka * 128);
-                        const uint32_t bb = *reinterpret_cast<const uint16_t *>(tile + col_off[kb & 7] + kb * 128);
-                        va[i] = __uint_as_float((ba << 16) + smask[i]);
-                        vb[i] = __uint_as_float((bb << 16) + smask[i]);
+                    for (int e = 0; e < 4; ++e) {
+                        const int i0 = 8 * c + 2 * e;
+                        va[i0] = __uint_as_float((wa[e] << 16) + smask[i0]);
+                        va[i0 + 1] = __uint_as_float((wa[e] & 0xFFFF0000u) ^ smask[i0 + 1]);
+                        vb[i0] = __uint_as_float((wb[e] << 16) + smask[i0]);
+                        vb[i0 + 1] = __uint_as_float((wb[e] & 0xFFFF0000u) ^ smask[i0 + 1]);
                     }
                 }
-                if (NH == 16) {
-                    float2 pr[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) pr[i] = make_float2(va[i], vb[i]);
-#pragma unroll
-                    for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            if (!(i & h)) bfly2(pr[i], pr[i + h]);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        va[i] = pr[i].x;
-                        vb[i] = pr[i].y;
-                    }
-                }
-                if (AMAX_ONLY) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        amax_acc = fmaxf(amax_acc, fmaxf(fabsf(va[i]), fabsf(vb[i])));
-                    continue;
-                }
-                float ama = 0.0f, amb = 0.0f;
+            } else {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    ama = fmaxf(ama, fabsf(va[i]));
-                    amb = fmaxf(amb, fabsf(vb[i]));
-                }
-                const ScaleOut sa = block_scale<GRID>(ama, a.scale_fmt, S, G);
-                const ScaleOut sb = block_scale<GRID>(amb, a.scale_fmt, S, G);
-                const uint64_t L0a = static_cast<uint64_t>(orow) * static_cast<uint64_t>(a.kpad) +
-                                     static_cast<uint64_t>(k0 + gp);
-                uint2 pa, pb;
-                if (GRID != 1) {
-                    round_pack2_uniform<GRID, RND>(va, vb, sa, sb, keys, a.stream, a.seed, L0a, L0a + 16,
-                                                   pa, pb);
-                } else {
-                    pa = round_pack<GRID, RND>(va, sa, keys, a.stream, L0a, a.seed);
-                    pb = round_pack<GRID, RND>(vb, sb, keys, a.stream, L0a + 16, a.seed);
-                }
-                if (gp == 0) {
-                    codes[0] = pa.x, codes[1] = pa.y, codes[2] = pb.x, codes[3] = pb.y;
-                    stored[0] = sa.stored, stored[1] = sb.stored;
-                } else {
-                    codes[4] = pa.x, codes[5] = pa.y, codes[6] = pb.x, codes[7] = pb.y;
-                    stored[2] = sa.stored, stored[3] = sb.stored;
+                    const int ka = gp + i, kb = gp + 16 + i;
+                    const uint32_t ba = *reinterpret_cast<const uint16_t *>(src + col_off[ka & 7] + ka * 128);
+                    const uint32_t bb = *reinterpret_cast<const uint16_t *>(src + col_off[kb & 7] + kb * 128);
+                    va[i] = __uint_as_float((ba << 16) + smask[i]);
+                    vb[i] = __uint_as_float((bb << 16) + smask[i]);
                 }
             }
-        } else
+            if (NH == 16) {
+                float2 pr[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pr[i] = make_float2(va[i], vb[i]);
+#pragma unroll
+                for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (!(i & h)) bfly2(pr[i], pr[i + h]);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    va[i] = pr[i].x;
+                    vb[i] = pr[i].y;
+                }
+            }
+            if (AMAX_ONLY) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    amax_acc = fmaxf(amax_acc, fmaxf(fabsf(va[i]), fabsf(vb[i])));
+                continue;
+            }
+            float ama = 0.0f, amb = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                ama = fmaxf(ama, fabsf(va[i]));
+                amb = fmaxf(amb, fabsf(vb[i]));
+            }
+            const ScaleOut sa = block_scale<GRID>(ama, a.scale_fmt, S, G);
+            const ScaleOut sb = block_scale<GRID>(amb, a.scale_fmt, S, G);
+            const uint64_t L0a = static_cast<uint64_t>(orow) * static_cast<uint64_t>(a.kpad) +
+                                 static_cast<uint64_t>(k0 + gp);
+            uint2 pa, pb;
+            if (GRID != 1) {
+                round_pack2_uniform<GRID, RND>(va, vb, sa, sb, keys, a.stream, a.seed, L0a, L0a + 16,
+                                               pa, pb);
+            } else {
+                pa = round_pack<GRID, RND>(va, sa, keys, a.stream, L0a, a.seed);
+                pb = round_pack<GRID, RND>(vb, sb, keys, a.stream, L0a + 16, a.seed);
+            }
+            if (gp == 0) {
+                codes[0] = pa.x, codes[1] = pa.y, codes[2] = pb.x, codes[3] = pb.y;
+                stored[0] = sa.stored, stored[1] = sb.stored;
+            } else {
+                codes[4] = pa.x, codes[5] = pa.y, codes[6] = pb.x, codes[7] = pb.y;
+                stored[2] = sa.stored, stored[3] = sb.stored;
+            }
+        }
+    } else {
 #pragma unroll
         for (int g0 = 0; g0 < 64; g0 += GS) {
             float v[GS];
-            if (AXIS == 0) {
-                const uint8_t *rowp = tile + t * 128;
+            if (RD == 0) {
 #pragma unroll
                 for (int c = 0; c < GS / 8; ++c) {
                     const int cg = g0 / 8 + c;
-                    const uint4 q = *reinterpret_cast<const uint4 *>(rowp + ((cg ^ (t & 7)) << 4));
+                    const uint4 q = *reinterpret_cast<const uint4 *>(src + ((cg ^ swz) << 4));
                     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -727,8 +634,7 @@ __global__ void __launch_bounds__(kCtaThreads, 3) rht_quantize_kernel(const __gr
 #pragma unroll
                 for (int i = 0; i < GS; ++i) {
                     const int kr = g0 + i;
-                    const uint16_t b =
-                        *reinterpret_cast<const uint16_t *>(tile + col_off[kr & 7] + kr * 128);
+                    const uint16_t b = *reinterpret_cast<const uint16_t *>(src + col_off[kr & 7] + kr * 128);
                     v[i] = __uint_as_float(static_cast<uint32_t>(b) << 16);
                 }
             }
@@ -776,27 +682,161 @@ __global__ void __launch_bounds__(kCtaThreads, 3) rht_quantize_kernel(const __gr
                 }
             }
         }
-        if (!AMAX_ONLY && orow < a.out_rows) {
-            uint4 *dst = reinterpret_cast<uint4 *>(a.codes + orow * (a.kpad / 2) + k0 / 2);
-            dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-            dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-            if (GRID == 0 && a.corr != nullptr) {
-                // E1M2 correction plane for the block-scaled FP4 GEMM
-                uint4 *cdst = reinterpret_cast<uint4 *>(a.corr + orow * (a.kpad / 2) + k0 / 2);
-                cdst[0] = make_uint4(e1m2_correction(codes[0]), e1m2_correction(codes[1]),
-                                     e1m2_correction(codes[2]), e1m2_correction(codes[3]));
-                cdst[1] = make_uint4(e1m2_correction(codes[4]), e1m2_correction(codes[5]),
-                                     e1m2_correction(codes[6]), e1m2_correction(codes[7]));
-            }
-            constexpr int kBlocks = 64 / BLK;
+    }
+    if (!AMAX_ONLY && orow < a.out_rows) {
+        uint4 *dst = reinterpret_cast<uint4 *>(a.codes + orow * (a.kpad / 2) + k0 / 2);
+        dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+        dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+        if (GRID == 0 && a.corr != nullptr) {
+            // E1M2 correction plane for the block-scaled FP4 GEMM
+            uint4 *cdst = reinterpret_cast<uint4 *>(a.corr + orow * (a.kpad / 2) + k0 / 2);
+            cdst[0] = make_uint4(e1m2_correction(codes[0]), e1m2_correction(codes[1]),
+                                 e1m2_correction(codes[2]), e1m2_correction(codes[3]));
+            cdst[1] = make_uint4(e1m2_correction(codes[4]), e1m2_correction(codes[5]),
+                                 e1m2_correction(codes[6]), e1m2_correction(codes[7]));
+        }
+        constexpr int kBlocks = 64 / BLK;
 #pragma unroll
-            for (int b = 0; b < kBlocks; ++b) {
-                const int64_t blk = k0 / BLK + b;
-                if (a.scale_fmt == 0)
-                    reinterpret_cast<uint32_t *>(a.scales)[blk * a.scale_ld + orow] = stored[b];
-                else
-                    reinterpret_cast<uint8_t *>(a.scales)[blk * a.scale_ld + orow] =
-                        static_cast<uint8_t>(stored[b]);
+        for (int b = 0; b < kBlocks; ++b) {
+            const int64_t blk = k0 / BLK + b;
+            if (a.scale_fmt == 0)
+                reinterpret_cast<uint32_t *>(a.scales)[blk * a.scale_ld + orow] = stored[b];
+            else
+                reinterpret_cast<uint8_t *>(a.scales)[blk * a.scale_ld + orow] = static_cast<uint8_t>(stored[b]);
+        }
+    }
+}
+
+// `a` drives the units (AXIS 0: row-wise output; AXIS 1 and 2: column-wise
+// output); `a2` is the row-wise output of AXIS 2 and unused otherwise.
+template <int AXIS, int NH, int BLK, int GRID, int RND, bool AMAX_ONLY>
+__global__ void __launch_bounds__(kCtaThreads, 3) rht_quantize_kernel(const __grid_constant__ QuantArgs a,
+                                                                  const __grid_constant__ QuantArgs a2,
+                                                                  const __grid_constant__ CUtensorMap tmap) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
+    uint64_t *empty = full + kStages;
+    volatile uint32_t *abort_flag =
+        reinterpret_cast<volatile uint32_t *>(smem + kStages * kStageBytes + 16 * kStages);
+    const int t = threadIdx.x;
+    const int lane = t & 31;
+    const int warp = t >> 5;
+    const int64_t nseg = a.kpad / 64;
+    const int64_t nrb = (a.out_rows + kUnitRows - 1) / kUnitRows;
+    const int64_t nunits = nseg * nrb;
+
+    auto unit_coords = [&](int64_t u, int64_t &rb, int64_t &seg) {
+        if (AXIS == 0) {
+            rb = u / nseg;
+            seg = u % nseg;
+        } else {
+            seg = u / nrb;
+            rb = u % nrb;
+        }
+    };
+    auto issue = [&](int64_t u, int s) {
+        int64_t rb, seg;
+        unit_coords(u, rb, seg);
+        uint8_t *dst = smem + s * kStageBytes;
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        if (AXIS == 0) {
+            tma_load_2d(dst, &tmap, &full[s], static_cast<int32_t>(seg * 64),
+                        static_cast<int32_t>(rb * kUnitRows));
+        } else {
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                tma_load_2d(dst + b * 8192, &tmap, &full[s], static_cast<int32_t>(rb * kUnitRows + 64 * b),
+                            static_cast<int32_t>(seg * 64));
+        }
+    };
+
+    if (t == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kComputeWarps);
+        }
+        *abort_flag = 0u;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    const int64_t u0 = blockIdx.x;
+    if (warp == kComputeWarps) {
+        // Producer warp: refills a stage once every compute warp released it.
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int64_t u = u0; u < nunits; u += gridDim.x, ++it) {
+                const int s = it % kStages;
+                if (it >= kStages &&
+                    !mbar_wait(&empty[s], ((it / kStages) - 1) & 1, kErrTimeoutProducer, abort_flag))
+                    break;
+                issue(u, s);
+            }
+            // Drain: the last copies have landed before the CTA exits.
+            for (uint32_t d = 0; d < kStages && d < it; ++d) {
+                const uint32_t idx = it - 1 - d;
+                uint32_t dummy = 0;
+                mbar_wait(&full[idx % kStages], (idx / kStages) & 1, kErrTimeoutDrain,
+                          reinterpret_cast<volatile uint32_t *>(&dummy));
+            }
+        }
+        return;
+    }
+
+    float S = 1.0f, G = 0.0f, S2 = 1.0f, G2 = 0.0f;
+    if (!AMAX_ONLY && a.scale_fmt == 1) tensor_scale<GRID>(a, S, G);
+    if (AXIS == 2 && !AMAX_ONLY && a2.scale_fmt == 1) tensor_scale<GRID>(a2, S2, G2);
+    // D for the 64 positions of a segment (K offsets are multiples of 64).
+    uint64_t pat = 0;
+    if (NH > 0) {
+        const uint64_t m = NH == 64 ? a.sign_mask : (a.sign_mask & ((1ull << NH) - 1));
+#pragma unroll
+        for (int off = 0; off < 64; off += (NH > 0 ? NH : 64)) pat |= m << off;
+    }
+    const uint32_t pat_lo = static_cast<uint32_t>(pat), pat_hi = static_cast<uint32_t>(pat >> 32);
+    // Sign of D at position i mod 16 as an fp32 sign bit (NH <= 16); adding
+    // it to a widened bf16 flips the sign bit like an xor.
+    uint32_t smask[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) smask[i] = NH > 0 ? ((pat_lo >> i) & 1u) << 31 : 0u;
+    PhiloxKeys keys;
+    if (RND == 1) keys = philox_keys(a.seed);
+    float amax_acc = 0.0f, amax_acc2 = 0.0f;
+
+    // Column-wise: byte offset of column cc (= t & 63) within K row r of a
+    // 64-column box for r % 8 (the 128-byte swizzle XORs the 16-byte chunk
+    // index with the row mod 8).
+    uint32_t col_off[8];
+    {
+        const int cc = t & 63;
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+            col_off[r] = static_cast<uint32_t>((t >> 6) * 8192 + ((((cc >> 3) ^ r) & 7) << 4) + (cc & 7) * 2);
+    }
+    uint32_t it = 0;
+    for (int64_t u = u0; u < nunits; u += gridDim.x, ++it) {
+        const int s = it % kStages;
+        if (!warp_wait(&full[s], (it / kStages) & 1, kErrTimeoutTransform, abort_flag)) break;
+        int64_t rb, seg;
+        unit_coords(u, rb, seg);
+        const uint8_t *tile = smem + s * kStageBytes;
+        if (AXIS == 0) {
+            quantize64<0, NH, BLK, GRID, RND, AMAX_ONLY>(a, tile + t * 128, t & 7, col_off, rb * kUnitRows + t,
+                                                         seg * 64, S, G, keys, smask, pat_lo, pat_hi,
+                                                         amax_acc);
+        } else {
+            quantize64<1, NH, BLK, GRID, RND, AMAX_ONLY>(a, tile, 0, col_off, rb * kUnitRows + t, seg * 64, S,
+                                                         G, keys, smask, pat_lo, pat_hi, amax_acc);
+            if (AXIS == 2) {
+                // Row-wise output: input row 64 seg + (t & 63), K columns from
+                // 256 rb + 64 (t >> 6).  Boxes past the padded K (the last
+                // column block of a ragged width) are skipped, per warp.
+                const int64_t k0 = rb * kUnitRows + 64 * (t >> 6);
+                if (k0 < a2.kpad)
+                    quantize64<0, NH, BLK, GRID, RND, AMAX_ONLY>(a2, tile + (t >> 6) * 8192 + (t & 63) * 128, t & 7,
+                                                                 col_off, seg * 64 + (t & 63), k0, S2, G2, keys,
+                                                                 smask, pat_lo, pat_hi, amax_acc2);
             }
         }
         __syncwarp();      // this warp is done with stage s
@@ -804,15 +844,19 @@ __global__ void __launch_bounds__(kCtaThreads, 3) rht_quantize_kernel(const __gr
     }
     if (AMAX_ONLY) {
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
+        for (int off = 16; off > 0; off >>= 1) {
             amax_acc = fmaxf(amax_acc, __shfl_xor_sync(0xFFFFFFFFu, amax_acc, off));
+            if (AXIS == 2) amax_acc2 = fmaxf(amax_acc2, __shfl_xor_sync(0xFFFFFFFFu, amax_acc2, off));
+        }
         if (lane == 0 && amax_acc > 0.0f)
             atomicMax(reinterpret_cast<unsigned int *>(a.amax_out), __float_as_uint(amax_acc));
+        if (AXIS == 2 && lane == 0 && amax_acc2 > 0.0f)
+            atomicMax(reinterpret_cast<unsigned int *>(a2.amax_out), __float_as_uint(amax_acc2));
     }
 }
 
 template <int AXIS, int NH, int BLK, int GRID, int RND, bool AMAX_ONLY>
-cudaError_t launch_one(const QuantArgs &a, const CUtensorMap &tmap, int num_sms,
+cudaError_t launch_one(const QuantArgs &a, const QuantArgs &a2, const CUtensorMap &tmap, int num_sms,
                        cudaStream_t stream) {
     static bool configured = false;
     if (!configured) {
@@ -825,32 +869,32 @@ cudaError_t launch_one(const QuantArgs &a, const CUtensorMap &tmap, int num_sms,
     const int64_t cap = static_cast<int64_t>(num_sms) * 3;
     const int grid = static_cast<int>(nunits < cap ? nunits : cap);
     if (grid <= 0) return cudaSuccess;
-    rht_quantize_kernel<AXIS, NH, BLK, GRID, RND, AMAX_ONLY><<<grid, kCtaThreads, kQuantSmem, stream>>>(a, tmap);
+    rht_quantize_kernel<AXIS, NH, BLK, GRID, RND, AMAX_ONLY><<<grid, kCtaThreads, kQuantSmem, stream>>>(a, a2, tmap);
     return cudaGetLastError();
 }
 
 template <int AXIS, int NH, int BLK, bool AMAX_ONLY>
-cudaError_t dispatch_grid_round(const QuantArgs &a, const CUtensorMap &m, int grid_kind, int rnd,
-                                int num_sms, cudaStream_t stream) {
-    if (AMAX_ONLY) return launch_one<AXIS, NH, BLK, 0, 0, true>(a, m, num_sms, stream);
+cudaError_t dispatch_grid_round(const QuantArgs &a, const QuantArgs &a2, const CUtensorMap &m, int grid_kind,
+                                int rnd, int num_sms, cudaStream_t stream) {
+    if (AMAX_ONLY) return launch_one<AXIS, NH, BLK, 0, 0, true>(a, a2, m, num_sms, stream);
     if (grid_kind == 0) {
-        return rnd == 0 ? launch_one<AXIS, NH, BLK, 0, 0, false>(a, m, num_sms, stream)
-                        : launch_one<AXIS, NH, BLK, 0, 1, false>(a, m, num_sms, stream);
+        return rnd == 0 ? launch_one<AXIS, NH, BLK, 0, 0, false>(a, a2, m, num_sms, stream)
+                        : launch_one<AXIS, NH, BLK, 0, 1, false>(a, a2, m, num_sms, stream);
     }
     if (grid_kind == 2) {
-        return rnd == 0 ? launch_one<AXIS, NH, BLK, 2, 0, false>(a, m, num_sms, stream)
-                        : launch_one<AXIS, NH, BLK, 2, 1, false>(a, m, num_sms, stream);
+        return rnd == 0 ? launch_one<AXIS, NH, BLK, 2, 0, false>(a, a2, m, num_sms, stream)
+                        : launch_one<AXIS, NH, BLK, 2, 1, false>(a, a2, m, num_sms, stream);
     }
-    return rnd == 0 ? launch_one<AXIS, NH, BLK, 1, 0, false>(a, m, num_sms, stream)
-                    : launch_one<AXIS, NH, BLK, 1, 1, false>(a, m, num_sms, stream);
+    return rnd == 0 ? launch_one<AXIS, NH, BLK, 1, 0, false>(a, a2, m, num_sms, stream)
+                    : launch_one<AXIS, NH, BLK, 1, 1, false>(a, a2, m, num_sms, stream);
 }
 
 template <int AXIS, bool AMAX_ONLY>
-cudaError_t dispatch_nh_blk(const QuantArgs &a, const CUtensorMap &m, int nh, int blk,
+cudaError_t dispatch_nh_blk(const QuantArgs &a, const QuantArgs &a2, const CUtensorMap &m, int nh, int blk,
                             int grid_kind, int rnd, int num_sms, cudaStream_t stream) {
 #define UFP4_CASE(N, B)                                                                          \
     if (nh == N && blk == B)                                                                     \
-        return dispatch_grid_round<AXIS, N, B, AMAX_ONLY>(a, m, grid_kind, rnd, num_sms, stream);
+        return dispatch_grid_round<AXIS, N, B, AMAX_ONLY>(a, a2, m, grid_kind, rnd, num_sms, stream);
     UFP4_CASE(0, 16)
     UFP4_CASE(0, 32)
     UFP4_CASE(16, 16)
@@ -864,7 +908,8 @@ cudaError_t dispatch_nh_blk(const QuantArgs &a, const CUtensorMap &m, int nh, in
 }
 
 // bf16 input as a 2-D tensor map: rows x cols, row pitch ld; 128-byte swizzle,
-// box 64 x 256 (row-wise: K x rows) or 64 x 64 (column-wise: columns x K).
+// box 64 x 256 (row-wise: K x rows) or 64 x 64 (column-wise and dual:
+// columns x K).
 cudaError_t make_input_map(const QuantArgs &a, CUtensorMap *m) {
     const uint32_t box_outer = a.axis == 0 ? kUnitRows : 64;
     CUresult r = encode_tensor_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x,
@@ -882,8 +927,17 @@ cudaError_t launch_rht_quantize(QuantArgs a, int hadamard_n, int block, int grid
     cudaError_t e = make_input_map(a, &m);
     if (e != cudaSuccess) return e;
     if (a.axis == 0)
-        return dispatch_nh_blk<0, false>(a, m, hadamard_n, block, grid_kind, rounding, num_sms, stream);
-    return dispatch_nh_blk<1, false>(a, m, hadamard_n, block, grid_kind, rounding, num_sms, stream);
+        return dispatch_nh_blk<0, false>(a, a, m, hadamard_n, block, grid_kind, rounding, num_sms, stream);
+    return dispatch_nh_blk<1, false>(a, a, m, hadamard_n, block, grid_kind, rounding, num_sms, stream);
+}
+
+cudaError_t launch_rht_quantize_dual(QuantArgs a_rows, QuantArgs a_cols, int hadamard_n, int block,
+                                     int grid_kind, int rounding, int num_sms, cudaStream_t stream) {
+    CUtensorMap m;
+    cudaError_t e = make_input_map(a_rows, &m);
+    if (e != cudaSuccess) return e;
+    return dispatch_nh_blk<2, false>(a_rows, a_cols, m, hadamard_n, block, grid_kind, rounding, num_sms,
+                                     stream);
 }
 
 cudaError_t launch_rht_amax(QuantArgs a, int hadamard_n, int num_sms, cudaStream_t stream) {
@@ -892,8 +946,19 @@ cudaError_t launch_rht_amax(QuantArgs a, int hadamard_n, int num_sms, cudaStream
     CUtensorMap m;
     e = make_input_map(a, &m);
     if (e != cudaSuccess) return e;
-    if (a.axis == 0) return dispatch_nh_blk<0, true>(a, m, hadamard_n, 16, 0, 0, num_sms, stream);
-    return dispatch_nh_blk<1, true>(a, m, hadamard_n, 16, 0, 0, num_sms, stream);
+    if (a.axis == 0) return dispatch_nh_blk<0, true>(a, a, m, hadamard_n, 16, 0, 0, num_sms, stream);
+    return dispatch_nh_blk<1, true>(a, a, m, hadamard_n, 16, 0, 0, num_sms, stream);
+}
+
+cudaError_t launch_rht_amax_dual(QuantArgs a_rows, QuantArgs a_cols, int hadamard_n, int num_sms,
+                                 cudaStream_t stream) {
+    cudaError_t e = cudaMemsetAsync(a_rows.amax_out, 0, sizeof(float), stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(a_cols.amax_out, 0, sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+    CUtensorMap m;
+    e = make_input_map(a_rows, &m);
+    if (e != cudaSuccess) return e;
+    return dispatch_nh_blk<2, true>(a_rows, a_cols, m, hadamard_n, 16, 0, 0, num_sms, stream);
 }
 
 cudaError_t quantize_read_and_clear_error_word(uint32_t *out) {

@@ -29,6 +29,12 @@ struct QuantArgs {
 cudaError_t launch_rht_quantize(QuantArgs a, int hadamard_n, int block, int grid_kind,
                                 int rounding, int num_sms, cudaStream_t stream);
 cudaError_t launch_rht_amax(QuantArgs a, int hadamard_n, int num_sms, cudaStream_t stream);
+// One read of the input, both outputs: a_rows (axis 1, drives the units) and
+// a_cols (axis 0); same grid / rounding / RHT / block for both.
+cudaError_t launch_rht_quantize_dual(QuantArgs a_rows, QuantArgs a_cols, int hadamard_n, int block,
+                                     int grid_kind, int rounding, int num_sms, cudaStream_t stream);
+cudaError_t launch_rht_amax_dual(QuantArgs a_rows, QuantArgs a_cols, int hadamard_n, int num_sms,
+                                 cudaStream_t stream);
 
 // One contraction problem (a group of the grouped GEMM, or the whole GEMM).
 struct GemmGroup {

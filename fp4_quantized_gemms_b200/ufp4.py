@@ -30,7 +30,7 @@ EXPORTED = [
     "ufp4_qtensor_layout", "ufp4_rht_amax", "ufp4_rht_quantize", "ufp4_gemm_fprop",
     "ufp4_gemm_dgrad", "ufp4_gemm_wgrad", "ufp4_grouped_gemm", "ufp4_check_device_status",
     "ufp4_status_string", "ufp4_version", "ufp4_set_two_level_gemm_path",
-    "ufp4_get_two_level_gemm_path",
+    "ufp4_get_two_level_gemm_path", "ufp4_rht_quantize_dual", "ufp4_rht_amax_dual",
 ]
 
 
@@ -83,6 +83,11 @@ def lib() -> ctypes.CDLL:
         L.ufp4_rht_amax.argtypes = [P, i64, i64, i64, i32, i32, u64, P, P]
         L.ufp4_rht_quantize.restype = st
         L.ufp4_rht_quantize.argtypes = [P, i64, i64, i64, i32, P, ctypes.POINTER(QTensorC), P]
+        L.ufp4_rht_amax_dual.restype = st
+        L.ufp4_rht_amax_dual.argtypes = [P, i64, i64, i64, i32, u64, P, P, P]
+        L.ufp4_rht_quantize_dual.restype = st
+        L.ufp4_rht_quantize_dual.argtypes = [P, i64, i64, i64, P, P, ctypes.POINTER(QTensorC),
+                                             ctypes.POINTER(QTensorC), P]
         for name in ("ufp4_gemm_fprop", "ufp4_gemm_dgrad", "ufp4_gemm_wgrad"):
             f = getattr(L, name)
             f.restype = st
@@ -227,6 +232,48 @@ def rht_quantize(x: torch.Tensor, axis: int, cfg: QuantConfig,
     _check(lib().ufp4_rht_quantize(ctypes.c_void_p(x.data_ptr()), rows, cols, x.stride(0), axis,
                                    ctypes.c_void_p(tensor_amax.data_ptr()) if tensor_amax is not None else None,
                                    ctypes.byref(qc), _stream_ptr(x.device)), "ufp4_rht_quantize")
+    return out
+
+
+def rht_amax_dual(x: torch.Tensor, hadamard_n: int, sign_mask: int = DEFAULT_SIGN_MASK,
+                  out: torch.Tensor | None = None) -> torch.Tensor:
+    """Both rotated amaxes from one read -> float32 [2] on device:
+    [ALONG_COLS, ALONG_ROWS]."""
+    _require_cuda(x)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2
+    if out is None:
+        out = torch.empty(2, dtype=torch.float32, device=x.device)
+    rows, cols = x.shape
+    _check(lib().ufp4_rht_amax_dual(ctypes.c_void_p(x.data_ptr()), rows, cols, x.stride(0), hadamard_n,
+                                    sign_mask, ctypes.c_void_p(out[0:1].data_ptr()),
+                                    ctypes.c_void_p(out[1:2].data_ptr()), _stream_ptr(x.device)),
+           "ufp4_rht_amax_dual")
+    return out
+
+
+def rht_quantize_dual(x: torch.Tensor, cfg_cols: QuantConfig, cfg_rows: QuantConfig | None = None,
+                      tensor_amax: torch.Tensor | None = None,
+                      out: tuple[QTensor, QTensor] | None = None,
+                      with_corr: bool | None = None) -> tuple[QTensor, QTensor]:
+    """Both quantizations of x from one read: (ALONG_COLS result, ALONG_ROWS
+    result).  cfg_rows defaults to cfg_cols; the two may differ in sr_stream
+    only.  tensor_amax: float32 [2] device tensor from rht_amax_dual (two-level
+    scales; computed here when None)."""
+    _require_cuda(x, tensor_amax)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    cfg_rows = cfg_cols if cfg_rows is None else cfg_rows
+    rows, cols = x.shape
+    if out is None:
+        out = (empty_qtensor(rows, cols, cfg_cols, device=x.device, with_corr=with_corr),
+               empty_qtensor(cols, rows, cfg_rows, device=x.device, with_corr=with_corr))
+    if cfg_cols.scale_fmt == SCALE_E4M3_X_FP32 and tensor_amax is None:
+        tensor_amax = rht_amax_dual(x, cfg_cols.hadamard_n, cfg_cols.rht_sign_mask)
+    qc, qr = out[0].c(), out[1].c()
+    am_c = ctypes.c_void_p(tensor_amax[0:1].data_ptr()) if tensor_amax is not None else None
+    am_r = ctypes.c_void_p(tensor_amax[1:2].data_ptr()) if tensor_amax is not None else None
+    _check(lib().ufp4_rht_quantize_dual(ctypes.c_void_p(x.data_ptr()), rows, cols, x.stride(0), am_c, am_r,
+                                        ctypes.byref(qc), ctypes.byref(qr), _stream_ptr(x.device)),
+           "ufp4_rht_quantize_dual")
     return out
 
 

@@ -174,6 +174,38 @@ ufp4_status_t ufp4_rht_quantize(const void *x_dev, int64_t rows, int64_t cols, i
                                 int32_t axis, const float *tensor_amax_dev,
                                 ufp4_qtensor_t *out, void *stream);
 
+/* Dual-output quantizer: both quantizations of one tensor from a single read
+ * of it.  Every operand of the recipe feeds two GEMMs along different axes
+ * (X: FPROP along cols, WGRAD along rows; W: FPROP along cols, DGRAD along
+ * rows; dY: DGRAD along cols, WGRAD along rows), so reading the bf16 tile
+ * once and writing both results extends the fusion of RHT into the quantizer
+ * that [GS] "Efficiëntie" (kernel fusion) describes.  No counterpart call on
+ * the pages: the results are bit-identical to
+ *   ufp4_rht_quantize(x, ..., UFP4_ALONG_COLS, tensor_amax_cols_dev, out_cols)
+ *   ufp4_rht_quantize(x, ..., UFP4_ALONG_ROWS, tensor_amax_rows_dev, out_rows)
+ * (SR draws included: they depend on seed, stream, output row and column only).
+ *   x_dev       bf16 [rows][ld], the constraints of ufp4_rht_quantize.
+ *   out_cols    the ALONG_COLS result (rows = rows, k = cols).
+ *   out_rows    the ALONG_ROWS result (rows = cols, k = rows).
+ *   tensor_amax_cols_dev / tensor_amax_rows_dev  rotated amaxes along each
+ *               axis (two-level scale only, from ufp4_rht_amax_dual), else NULL.
+ * The two cfgs must agree on everything but sr_stream (grid, rounding,
+ * sr_seed, hadamard_n and the first hadamard_n sign bits, block, scale_fmt),
+ * else UFP4_ERR_UNSUPPORTED: call ufp4_rht_quantize twice instead.
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED, CUDA. */
+ufp4_status_t ufp4_rht_quantize_dual(const void *x_dev, int64_t rows, int64_t cols, int64_t ld,
+                                     const float *tensor_amax_cols_dev,
+                                     const float *tensor_amax_rows_dev, ufp4_qtensor_t *out_cols,
+                                     ufp4_qtensor_t *out_rows, void *stream);
+
+/* Both rotated amaxes of one tensor from a single read: amax_cols_dev
+ * receives ufp4_rht_amax(..., UFP4_ALONG_COLS, ...) and amax_rows_dev
+ * ufp4_rht_amax(..., UFP4_ALONG_ROWS, ...) (bit-identical).  Input
+ * constraints and errors as ufp4_rht_amax. */
+ufp4_status_t ufp4_rht_amax_dual(const void *x_dev, int64_t rows, int64_t cols, int64_t ld,
+                                 int32_t hadamard_n, uint64_t rht_sign_mask, float *amax_cols_dev,
+                                 float *amax_rows_dev, void *stream);
+
 /* FPROP, fwd_y:  Y[M][N] = X W^T.  xq: X quantized ALONG_COLS ([M][K]);
  * wq: W quantized ALONG_COLS ([N][K]).  y_dev fp32 [M][ldy], ldy >= N,
  * 4-byte aligned (rows that are 16-byte aligned get vector stores).

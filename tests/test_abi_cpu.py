@@ -147,6 +147,33 @@ def test_quantize_validation_rejects_before_launch(L):
     assert L.ufp4_rht_amax(x, 64, 128, 128, 0, 16, 0, None, None) == ufp4.ERR_INVALID_ARG
 
 
+def test_dual_quantize_validation_rejects_before_launch(L):
+    """The dual quantizer checks both descriptors and that their recipes agree
+    (all but sr_stream) before any CUDA call."""
+    x = ctypes.c_void_p(4096)
+    D = L.ufp4_rht_quantize_dual
+
+    def call(oc, orr, rows=64, cols=128, ld=128, am=None):
+        return D(x, rows, cols, ld, am, am, ctypes.byref(oc), ctypes.byref(orr), None)
+
+    assert call(_q(rows=64, k=128), _q(rows=128, k=128)) == ufp4.ERR_INVALID_ARG   # rows-out shape
+    assert call(_q(rows=128, k=64), _q(rows=128, k=64)) == ufp4.ERR_INVALID_ARG    # cols-out shape
+    for kw in ({"grid": 1}, {"rounding": 1}, {"hadamard_n": 32}, {"block": 32}, {"sr_seed": 5},
+               {"hadamard_n": 16, "rht_sign_mask": 0x1}):
+        base = {"hadamard_n": 16, "rht_sign_mask": 0x2} if "rht_sign_mask" in kw else {}
+        assert call(_q(rows=64, k=128, **base), _q(rows=128, k=64, **kw)) == ufp4.ERR_UNSUPPORTED, kw
+    two_c, two_r = _q(rows=64, k=128, scale_fmt=1), _q(rows=128, k=64, scale_fmt=1)
+    assert call(two_c, two_r) == ufp4.ERR_INVALID_ARG                              # no amax
+    assert D(None, 64, 128, 128, None, None, ctypes.byref(_q(rows=64, k=128)),
+             ctypes.byref(_q(rows=128, k=64)), None) == ufp4.ERR_INVALID_ARG
+    # empty input: validated, nothing to launch
+    assert call(_q(rows=0, k=128), _q(rows=128, k=0), rows=0) == ufp4.OK
+    A = L.ufp4_rht_amax_dual
+    assert A(x, 64, 128, 128, 8, 0, x, x, None) == ufp4.ERR_UNSUPPORTED
+    assert A(x, 64, 128, 128, 16, 0, None, x, None) == ufp4.ERR_INVALID_ARG
+    assert A(x, 64, 120, 124, 16, 0, x, x, None) == ufp4.ERR_ALIGNMENT
+
+
 def test_two_level_gemm_path_selector(L):
     """The path setting is host state: it round-trips and rejects unknown values."""
     old = ufp4.get_two_level_gemm_path()

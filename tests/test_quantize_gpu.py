@@ -115,3 +115,81 @@ def test_quantize_sweep_sizes_sampled(shape, axis):
         _run(X, axis, cfg, rows=sample)
     cfg = ufp4.QuantConfig(hadamard_n=16, block=16, scale_fmt=ufp4.SCALE_E4M3_X_FP32)
     _run(X, axis, cfg, rows=sample)
+
+
+# ------------------------------------------------------------------ dual output
+def _oracle_ref(x_bits, axis, cfg, amax, rows=None):
+    oc = oracle_cfg(cfg)
+    if rows is None:
+        return oracle.quantize(x_bits, axis, oc, tensor_amax=amax)
+    refs = [oracle.quantize(x_bits, axis, oc, tensor_amax=amax, r0=int(r), nr=1) for r in rows]
+    ref = refs[0]
+    ref.codes = np.concatenate([r.codes for r in refs])
+    if ref.scales is not None:
+        ref.scales = np.concatenate([r.scales for r in refs])
+    else:
+        ref.escales = np.concatenate([r.escales for r in refs])
+    return ref
+
+
+def _run_dual(x_bits, cfg_c, cfg_r, rows_c=None, rows_r=None, with_corr=None):
+    """One dual call against the oracle on both outputs (and both amaxes)."""
+    x = to_dev(x_bits)
+    am_c = am_r = 0.0
+    am_d = None
+    if cfg_c.scale_fmt == ufp4.SCALE_E4M3_X_FP32:
+        am_c = oracle.rht_amax(x_bits, ufp4.ALONG_COLS, cfg_c.hadamard_n, cfg_c.rht_sign_mask)
+        am_r = oracle.rht_amax(x_bits, ufp4.ALONG_ROWS, cfg_c.hadamard_n, cfg_c.rht_sign_mask)
+        am_d = ufp4.rht_amax_dual(x, cfg_c.hadamard_n, cfg_c.rht_sign_mask)
+        got = am_d.cpu().numpy()
+        assert got[0] == np.float32(am_c) and got[1] == np.float32(am_r)
+    qc, qr = ufp4.rht_quantize_dual(x, cfg_c, cfg_r, tensor_amax=am_d, with_corr=with_corr)
+    torch.cuda.synchronize()
+    assert ufp4.check_device_status() == ufp4.OK
+    assert_quant_equal(qc, _oracle_ref(x_bits, ufp4.ALONG_COLS, cfg_c, am_c, rows_c), rows_c)
+    assert_quant_equal(qr, _oracle_ref(x_bits, ufp4.ALONG_ROWS, cfg_r, am_r, rows_r), rows_r)
+    return qc, qr
+
+
+@pytest.mark.parametrize("n,block", [(0, 16), (16, 16), (16, 32), (32, 16), (64, 32)])
+@pytest.mark.parametrize("grid,rounding,fmt", GRID_ROUND_FMT)
+def test_dual_quantize_matches_oracle_small(n, block, grid, rounding, fmt):
+    """300 x 600: five 64-row K segments for the row-wise output (ragged last)
+    and three 256-column blocks (the last with only two of its four 64-column
+    K segments inside the padded width)."""
+    X = wl.student_t(300, 600, seed=13)
+    cfg = ufp4.QuantConfig(grid=grid, rounding=rounding, sr_seed=1234, sr_stream=0,
+                           hadamard_n=n, block=block, scale_fmt=fmt)
+    _run_dual(X, cfg, cfg.with_(sr_stream=1))
+
+
+def test_dual_quantize_equals_two_single_calls():
+    """The dual call writes exactly what two single calls write (layer recipe:
+    dY with SR, streams 0 and 1, two-level scales, correction planes)."""
+    dY = wl.normal(520, 712, 1e-3, 3)
+    x = to_dev(dY)
+    cfg = ufp4.QuantConfig(rounding=ufp4.ROUND_SR, sr_seed=77, hadamard_n=16, block=16,
+                           scale_fmt=ufp4.SCALE_E4M3_X_FP32)
+    qc, qr = ufp4.rht_quantize_dual(x, cfg, cfg.with_(sr_stream=1))
+    sc = ufp4.rht_quantize(x, ufp4.ALONG_COLS, cfg)
+    sr = ufp4.rht_quantize(x, ufp4.ALONG_ROWS, cfg.with_(sr_stream=1))
+    torch.cuda.synchronize()
+    for d, s in ((qc, sc), (qr, sr)):
+        assert torch.equal(d.codes, s.codes) and torch.equal(d.scales, s.scales)
+        assert torch.equal(d.corr, s.corr) and torch.equal(d.tensor_scale, s.tensor_scale)
+
+
+@pytest.mark.parametrize("shape", [wl.QUANT_SWEEP_SHAPES[0], wl.QUANT_SWEEP_SHAPES[-1]])
+def test_dual_quantize_full_size_sampled(shape):
+    """Quantizer-sweep sizes through the dual kernel, 40 sampled output rows of
+    each result (plus the first and last) against the oracle."""
+    rows, cols = shape
+    X = wl.student_t(rows, cols)
+    rng = np.random.default_rng(rows + cols)
+    rc = np.unique(np.concatenate([[0, rows - 1], rng.choice(rows, 40, replace=False)]))
+    rr = np.unique(np.concatenate([[0, cols - 1], rng.choice(cols, 40, replace=False)]))
+    cfg = ufp4.QuantConfig(rounding=ufp4.ROUND_SR, sr_seed=1234, hadamard_n=16, block=16,
+                           scale_fmt=ufp4.SCALE_E4M3_X_FP32)
+    _run_dual(X, cfg, cfg.with_(sr_stream=1), rows_c=rc, rows_r=rr)
+    cfg = ufp4.QuantConfig(hadamard_n=16, block=16)
+    _run_dual(X, cfg, cfg, rows_c=rc, rows_r=rr)
