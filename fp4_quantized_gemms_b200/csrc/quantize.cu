@@ -34,7 +34,6 @@ namespace ufp4 {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
 
 // Grids: 0 = E1M2 (levels k/4, k <= 7), 1 = E2M1 (OCP FP4 magnitudes),
 // 2 = E2M1 restricted to max_fpx = 2.0 (the E2M1 codes 0..4, levels k/2).
@@ -135,50 +134,6 @@ __device__ __forceinline__ int round_sr(float au, float m1, float b, float inv, 
     return exact_diff(au, c, m1, b) > 0.0f ? lo + 1 : lo;
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// In-place unnormalised Walsh-Hadamard transform of one 16-chunk plus the
-// cross-lane stages of a 32 / 64 block.  Stage order h = 1, 2, ..., NH/2.
-template <int NH>
-__device__ __forceinline__ void fwht_chunk(float (&v)[16], int j) {
-    if constexpr (NH > 0) {
-#pragma unroll
-        for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                if (i & h) continue;
-                const float a = v[i], b = v[i + h];
-                v[i] = __fadd_rn(a, b);
-                v[i + h] = __fsub_rn(a, b);
-            }
-        }
-    }
-    if constexpr (NH >= 32) {
-        const bool upper = (j & 1) != 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float p = __shfl_xor_sync(0xFFFFFFFFu, v[i], 1);
-            v[i] = upper ? __fsub_rn(p, v[i]) : __fadd_rn(v[i], p);
-        }
-    }
-    if constexpr (NH >= 64) {
-        const bool upper = (j & 2) != 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float p = __shfl_xor_sync(0xFFFFFFFFu, v[i], 2);
-            v[i] = upper ? __fsub_rn(p, v[i]) : __fadd_rn(v[i], p);
-        }
-    }
-}
-
-// Signs of D for this lane's 16 positions (bit i: position i of the chunk).
-template <int NH>
-__device__ __forceinline__ uint32_t lane_sign_bits(uint64_t mask, int j) {
-    if (NH == 0) return 0u;
-    const int off = 16 * (j & (NH / 16 - 1));
-    return static_cast<uint32_t>(mask >> off) & 0xFFFFu;
-}
 
 // Reciprocal for the fp32 estimate only (every decision it feeds is either
 // certified by the 2^-16 margin or re-decided exactly): rcp.approx has at
@@ -505,6 +460,10 @@ constexpr int kStages = 2;
 constexpr int kComputeWarps = kThreads / 32;
 constexpr int kCtaThreads = kThreads + 32;        // + one producer warp
 constexpr int kQuantSmem = kStages * kStageBytes + 1024 + 64;
+// Resident CTAs per SM: three for one output (72 registers a thread); the
+// dual kernel does twice the work per staged tile and keeps more state, two.
+template <int AXIS>
+constexpr int ctas_per_sm() { return AXIS == 2 ? 2 : 3; }
 
 // Two-level tensor scale of one output: S maps the rotated tensor amax to
 // gmax * 448 (the top of E4M3), G = gmax * S is the block-scale divisor.
@@ -656,11 +615,10 @@ __device__ __forceinline__ void quantize64(const QuantArgs &a, const uint8_t *sr
                     }
                 }
             }
-            if (AMAX_ONLY) {
+            if constexpr (AMAX_ONLY) {
 #pragma unroll
                 for (int i = 0; i < GS; ++i) amax_acc = fmaxf(amax_acc, fabsf(v[i]));
-                continue;
-            }
+            } else {
 #pragma unroll
             for (int b0 = 0; b0 < GS; b0 += BLK) {
                 float am = 0.0f;
@@ -681,9 +639,11 @@ __device__ __forceinline__ void quantize64(const QuantArgs &a, const uint8_t *sr
                     codes[kc / 8 + 1] = pk.y;
                 }
             }
+            }
         }
     }
-    if (!AMAX_ONLY && orow < a.out_rows) {
+    if constexpr (!AMAX_ONLY) {
+        if (orow >= a.out_rows) return;
         uint4 *dst = reinterpret_cast<uint4 *>(a.codes + orow * (a.kpad / 2) + k0 / 2);
         dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
         dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
@@ -710,7 +670,7 @@ __device__ __forceinline__ void quantize64(const QuantArgs &a, const uint8_t *sr
 // `a` drives the units (AXIS 0: row-wise output; AXIS 1 and 2: column-wise
 // output); `a2` is the row-wise output of AXIS 2 and unused otherwise.
 template <int AXIS, int NH, int BLK, int GRID, int RND, bool AMAX_ONLY>
-__global__ void __launch_bounds__(kCtaThreads, 3) rht_quantize_kernel(const __grid_constant__ QuantArgs a,
+__global__ void __launch_bounds__(kCtaThreads, ctas_per_sm<AXIS>()) rht_quantize_kernel(const __grid_constant__ QuantArgs a,
                                                                   const __grid_constant__ QuantArgs a2,
                                                                   const __grid_constant__ CUtensorMap tmap) {
     extern __shared__ uint8_t smem_raw[];
@@ -795,13 +755,11 @@ __global__ void __launch_bounds__(kCtaThreads, 3) rht_quantize_kernel(const __gr
         for (int off = 0; off < 64; off += (NH > 0 ? NH : 64)) pat |= m << off;
     }
     const uint32_t pat_lo = static_cast<uint32_t>(pat), pat_hi = static_cast<uint32_t>(pat >> 32);
-    // Sign of D at position i mod 16 as an fp32 sign bit (NH <= 16); adding
-    // it to a widened bf16 flips the sign bit like an xor.
-    uint32_t smask[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) smask[i] = NH > 0 ? ((pat_lo >> i) & 1u) << 31 : 0u;
-    PhiloxKeys keys;
-    if (RND == 1) keys = philox_keys(a.seed);
+    // Sign of D at position i mod 16 as an fp32 sign bit (NH <= 16; adding it
+    // to a widened bf16 flips the sign bit like an xor) and the Philox round
+    // keys: both from the parameter bank, no registers held.
+    const uint32_t (&smask)[16] = a.smask;
+    const PhiloxKeys &keys = a.keys;
     float amax_acc = 0.0f, amax_acc2 = 0.0f;
 
     // Column-wise: byte offset of column cc (= t & 63) within K row r of a
@@ -855,6 +813,20 @@ __global__ void __launch_bounds__(kCtaThreads, 3) rht_quantize_kernel(const __gr
     }
 }
 
+// Host side of the per-call constants: Philox round keys of the seed and the
+// D sign bits of positions 0..15 (used by the kernels with NH <= 16).
+void fill_call_constants(QuantArgs &a, int hadamard_n) {
+    uint32_t kx = static_cast<uint32_t>(a.seed), ky = static_cast<uint32_t>(a.seed >> 32);
+    for (int r = 0; r < 10; ++r) {
+        a.keys.x[r] = kx;
+        a.keys.y[r] = ky;
+        kx += 0x9E3779B9u;
+        ky += 0xBB67AE85u;
+    }
+    for (int i = 0; i < 16; ++i)
+        a.smask[i] = hadamard_n > 0 ? static_cast<uint32_t>((a.sign_mask >> i) & 1u) << 31 : 0u;
+}
+
 template <int AXIS, int NH, int BLK, int GRID, int RND, bool AMAX_ONLY>
 cudaError_t launch_one(const QuantArgs &a, const QuantArgs &a2, const CUtensorMap &tmap, int num_sms,
                        cudaStream_t stream) {
@@ -866,7 +838,7 @@ cudaError_t launch_one(const QuantArgs &a, const QuantArgs &a2, const CUtensorMa
         configured = true;
     }
     const int64_t nunits = (a.kpad / 64) * ((a.out_rows + kUnitRows - 1) / kUnitRows);
-    const int64_t cap = static_cast<int64_t>(num_sms) * 3;
+    const int64_t cap = static_cast<int64_t>(num_sms) * ctas_per_sm<AXIS>();
     const int grid = static_cast<int>(nunits < cap ? nunits : cap);
     if (grid <= 0) return cudaSuccess;
     rht_quantize_kernel<AXIS, NH, BLK, GRID, RND, AMAX_ONLY><<<grid, kCtaThreads, kQuantSmem, stream>>>(a, a2, tmap);
@@ -923,6 +895,7 @@ cudaError_t make_input_map(const QuantArgs &a, CUtensorMap *m) {
 
 cudaError_t launch_rht_quantize(QuantArgs a, int hadamard_n, int block, int grid_kind,
                                 int rounding, int num_sms, cudaStream_t stream) {
+    fill_call_constants(a, hadamard_n);
     CUtensorMap m;
     cudaError_t e = make_input_map(a, &m);
     if (e != cudaSuccess) return e;
@@ -933,6 +906,8 @@ cudaError_t launch_rht_quantize(QuantArgs a, int hadamard_n, int block, int grid
 
 cudaError_t launch_rht_quantize_dual(QuantArgs a_rows, QuantArgs a_cols, int hadamard_n, int block,
                                      int grid_kind, int rounding, int num_sms, cudaStream_t stream) {
+    fill_call_constants(a_rows, hadamard_n);
+    fill_call_constants(a_cols, hadamard_n);
     CUtensorMap m;
     cudaError_t e = make_input_map(a_rows, &m);
     if (e != cudaSuccess) return e;
@@ -941,6 +916,7 @@ cudaError_t launch_rht_quantize_dual(QuantArgs a_rows, QuantArgs a_cols, int had
 }
 
 cudaError_t launch_rht_amax(QuantArgs a, int hadamard_n, int num_sms, cudaStream_t stream) {
+    fill_call_constants(a, hadamard_n);
     cudaError_t e = cudaMemsetAsync(a.amax_out, 0, sizeof(float), stream);
     if (e != cudaSuccess) return e;
     CUtensorMap m;
@@ -952,6 +928,8 @@ cudaError_t launch_rht_amax(QuantArgs a, int hadamard_n, int num_sms, cudaStream
 
 cudaError_t launch_rht_amax_dual(QuantArgs a_rows, QuantArgs a_cols, int hadamard_n, int num_sms,
                                  cudaStream_t stream) {
+    fill_call_constants(a_rows, hadamard_n);
+    fill_call_constants(a_cols, hadamard_n);
     cudaError_t e = cudaMemsetAsync(a_rows.amax_out, 0, sizeof(float), stream);
     if (e == cudaSuccess) e = cudaMemsetAsync(a_cols.amax_out, 0, sizeof(float), stream);
     if (e != cudaSuccess) return e;

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
+#include "ufp4_internal.h"
 
 namespace ufp4 {
 
@@ -491,12 +492,8 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
     return c;
 }
 
-// The ten round keys of one Philox key (the key schedule does not depend on
-// the counter, so a thread computes it once).
-struct PhiloxKeys {
-    uint32_t x[10], y[10];
-};
-
+// The ten round keys of one Philox key (PhiloxKeys, ufp4_internal.h): the
+// key schedule does not depend on the counter.
 __device__ __forceinline__ PhiloxKeys philox_keys(uint64_t seed) {
     PhiloxKeys ks;
     uint32_t a = static_cast<uint32_t>(seed), b = static_cast<uint32_t>(seed >> 32);

@@ -7,6 +7,12 @@
 
 namespace ufp4 {
 
+// The ten round keys of a Philox4x32-10 key: (x, y)_r = key + r * (the two
+// Weyl constants), the schedule of Salmon et al. (SC'11).
+struct PhiloxKeys {
+    uint32_t x[10], y[10];
+};
+
 struct QuantArgs {
     const uint16_t *x;   // bf16 input [rows][ld]
     int64_t rows, cols, ld;
@@ -24,6 +30,10 @@ struct QuantArgs {
     uint64_t sign_mask;
     int scale_fmt;
     int64_t num_units;   // filled by the launcher
+    // Per-call constants the kernels read from the parameter bank instead of
+    // holding in registers (filled by the launcher from seed / sign_mask):
+    PhiloxKeys keys;     // round keys of `seed`
+    uint32_t smask[16];  // D sign of position i mod 16, as an fp32 sign bit
 };
 
 cudaError_t launch_rht_quantize(QuantArgs a, int hadamard_n, int block, int grid_kind,
