@@ -148,22 +148,31 @@ class LayerStep:
         self.qwt = E(s.K, s.N, self.c_rtne, device)       # DGRAD B
         self.qdyt = E(s.N, s.M, self.c_sr1, device)       # WGRAD A
         self.qxt = E(s.K, s.M, self.c_rtne, device)       # WGRAD B
-        self.jobs = [(self.X, C, self.qx), (self.W, C, self.qw), (self.dY, C, self.qdy),
-                     (self.W, R, self.qwt), (self.dY, R, self.qdyt), (self.X, R, self.qxt)]
-        self.amax = torch.zeros(len(self.jobs), dtype=torch.float32, device=device)
+        # Each tensor feeds two GEMMs, one along each axis.  X and W (RTNE)
+        # go through the dual-output quantizer (one read, both results); dY
+        # (SR) through two single calls, which are faster for the ALU-bound
+        # SR path.  The rotated amaxes come from one dual pass per tensor.
+        self.dual = [(self.X, self.qx, self.qxt), (self.W, self.qw, self.qwt)]
+        self.single = [(self.dY, C, self.qdy), (self.dY, R, self.qdyt)]
+        self.amax = torch.zeros(6, dtype=torch.float32, device=device)   # [cols, rows] per tensor
         self.Y = torch.empty((s.M, s.N), dtype=torch.float32, device=device)
         self.dX = torch.empty((s.M, s.K), dtype=torch.float32, device=device)
         self.dW = torch.empty((s.N, s.K), dtype=torch.float32, device=device)
-        self.launches = len(self.jobs) * (2 if two else 1) + 3
-        self.quant_elems = sum(j[0].numel() for j in self.jobs)
+        self.launches = (3 if two else 0) + len(self.dual) + len(self.single) + 3
+        self.tensor_elems = self.X.numel() + self.W.numel() + self.dY.numel()
+        self.quant_elems = 2 * self.tensor_elems         # elements quantized per step
 
     def quantize_all(self):
         u = self.u
-        for i, (x, axis, q) in enumerate(self.jobs):
-            am = None
-            if self.two:
-                am = self.amax[i:i + 1]
-                u.rht_amax(x, axis, 16, q.cfg.rht_sign_mask, out=am)
+        sm = self.c_rtne.rht_sign_mask
+        if self.two:
+            for i, x in enumerate((self.X, self.W, self.dY)):
+                u.rht_amax_dual(x, 16, sm, out=self.amax[2 * i:2 * i + 2])
+        for i, (x, qc, qr) in enumerate(self.dual):
+            am = self.amax[2 * i:2 * i + 2] if self.two else None
+            u.rht_quantize_dual(x, qc.cfg, qr.cfg, tensor_amax=am, out=(qc, qr))
+        for j, (x, axis, q) in enumerate(self.single):
+            am = self.amax[4 + j:5 + j] if self.two else None
             u.rht_quantize(x, axis, q.cfg, tensor_amax=am, out=q)
 
     def gemms(self, events=None):
@@ -188,13 +197,16 @@ class LayerStep:
 
 
 def quant_bytes(step: LayerStep) -> float:
-    """Algorithmic bytes of the six quantize calls: bf16 in, packed codes,
-    block scales (fp32, or E4M3 + the amax pass re-reading the input)."""
-    n = step.quant_elems
-    per = 2 + 0.5 + (4 / 16 if not step.two else 1 / 16)
-    total = n * per
+    """Algorithmic bytes of the step's quantization: each quantized element
+    writes its code and its share of a block scale (fp32, or E4M3); bf16 inputs
+    are read once per dual call and once per single call; with two-level
+    scales the dual amax pass reads each tensor once more."""
+    out_per = 0.5 + (4 / 16 if not step.two else 1 / 16)
+    total = step.quant_elems * out_per
+    total += sum(x.numel() for x, _, _ in step.dual) * 2
+    total += sum(x.numel() for x, _, _ in step.single) * 2
     if step.two:
-        total += n * 2   # rotated-amax pass reads the input once more
+        total += step.tensor_elems * 2
     return total
 
 
