@@ -15,7 +15,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libufp4.so")
 BUILD_DIR = os.path.join(PKG, "_build")
-SOURCES = ["api.cu", "quantize.cu", "gemm.cu"]
+SOURCES = ["api.cu", "quantize.cu", "gemm.cu", "diag.cu"]
 NVCC = os.environ.get("NVCC", "nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",

@@ -9,6 +9,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <cmath>
 #include <mutex>
 
 #include "ufp4.h"
@@ -464,6 +465,70 @@ ufp4_status_t ufp4_rht_quantize_dual(const void *x_dev, int64_t rows, int64_t co
     if (rows == 0 || cols == 0) return UFP4_OK;
     cudaError_t e = launch_rht_quantize_dual(ar, ac, c.hadamard_n, c.block, c.grid, c.rounding, sm_count(),
                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
+}
+
+ufp4_status_t ufp4_quant_stats(const void *x_dev, int64_t rows, int64_t cols, int64_t ld,
+                               int32_t axis, const ufp4_qtensor_t *q, ufp4_qstats_t *stats_dev,
+                               void *stream) {
+    ufp4_status_t s = check_input(x_dev, rows, cols, ld, axis);
+    if (s != UFP4_OK) return s;
+    s = check_qtensor(q);
+    if (s != UFP4_OK) return s;
+    if (stats_dev == nullptr) return UFP4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(stats_dev) & 7u) != 0) return UFP4_ERR_ALIGNMENT;
+    const int64_t out_rows = axis == UFP4_ALONG_COLS ? rows : cols;
+    const int64_t K = axis == UFP4_ALONG_COLS ? cols : rows;
+    if (q->rows != out_rows || q->k != K) return UFP4_ERR_INVALID_ARG;
+    DiagArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x = static_cast<const uint16_t *>(x_dev);
+    a.rows = rows;
+    a.cols = cols;
+    a.ld = ld;
+    a.axis = axis;
+    a.out_rows = out_rows;
+    a.K = K;
+    a.kpad = q->kpad;
+    a.scale_ld = q->scale_ld;
+    a.codes = static_cast<const uint8_t *>(q->codes);
+    a.scales = q->scales;
+    a.S = q->tensor_scale;
+    a.scale_fmt = q->cfg.scale_fmt;
+    a.grid = q->cfg.grid == UFP4_GRID_E1M2 ? 0 : 1;   // level table: E1M2 or E2M1 codes
+    a.block = q->cfg.block;
+    a.sign_mask = q->cfg.rht_sign_mask;
+    a.out = stats_dev;
+    cudaError_t e = launch_quant_stats(a, q->cfg.hadamard_n, sm_count(), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
+}
+
+ufp4_status_t ufp4_qstats_summarize(const ufp4_qstats_t *st, int32_t grid, ufp4_qstats_summary_t *out) {
+    if (st == nullptr || out == nullptr) return UFP4_ERR_INVALID_ARG;
+    if (grid != UFP4_GRID_E1M2 && grid != UFP4_GRID_E2M1 && grid != UFP4_GRID_E2M1_MAX2)
+        return UFP4_ERR_INVALID_ARG;
+    out->sqnr_db = st->noise > 0.0 ? 10.0 * log10(st->signal / st->noise) : HUGE_VAL;
+    uint64_t total = 0;
+    for (int c = 0; c < 16; ++c) total += st->code_count[c];
+    int occupied = 0;
+    for (int c = 0; c < 16; ++c)
+        if (total > 0 && st->code_count[c] * 240.0 > static_cast<double>(total)) ++occupied;
+    const int grid_codes = grid == UFP4_GRID_E2M1_MAX2 ? 9 : 15;
+    out->bucket_ratio = static_cast<double>(occupied) / grid_codes;
+    out->underflow_ratio = st->nonzero ? static_cast<double>(st->underflow) / st->nonzero : 0.0;
+    for (int k = 0; k < 8; ++k)
+        out->level_mean_err[k] = st->level_n[k] ? st->level_err[k] / st->level_n[k] : NAN;
+    return UFP4_OK;
+}
+
+ufp4_status_t ufp4_sqnr_sums(const float *ref_dev, int64_t ld_ref, const float *test_dev,
+                             int64_t ld_test, int64_t rows, int64_t cols, double *sums_dev,
+                             void *stream) {
+    if (rows < 0 || cols < 0 || sums_dev == nullptr) return UFP4_ERR_INVALID_ARG;
+    if (rows > 0 && cols > 0 && (ref_dev == nullptr || test_dev == nullptr || ld_ref < cols || ld_test < cols))
+        return UFP4_ERR_INVALID_ARG;
+    cudaError_t e = launch_sqnr_sums(ref_dev, ld_ref, test_dev, ld_test, rows, cols, sums_dev, sm_count(),
+                                     static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
 }
 

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "ufp4.h"
+
 namespace ufp4 {
 
 // The ten round keys of a Philox4x32-10 key: (x, y)_r = key + r * (the two
@@ -45,6 +47,24 @@ cudaError_t launch_rht_quantize_dual(QuantArgs a_rows, QuantArgs a_cols, int had
                                      int grid_kind, int rounding, int num_sms, cudaStream_t stream);
 cudaError_t launch_rht_amax_dual(QuantArgs a_rows, QuantArgs a_cols, int hadamard_n, int num_sms,
                                  cudaStream_t stream);
+
+// Statistics of one quantized operand (diag.cu).
+struct DiagArgs {
+    const uint16_t *x;      // bf16 input [rows][ld]
+    int64_t rows, cols, ld;
+    int axis;
+    int64_t out_rows, K, kpad, scale_ld;
+    const uint8_t *codes;   // [out_rows][kpad/2]
+    const void *scales;     // block-major, fp32 or E4M3
+    const float *S;         // two-level tensor scale (device)
+    int scale_fmt, grid, block;
+    uint64_t sign_mask;
+    ufp4_qstats_t *out;     // device
+};
+
+cudaError_t launch_quant_stats(const DiagArgs &a, int hadamard_n, int num_sms, cudaStream_t stream);
+cudaError_t launch_sqnr_sums(const float *ref, int64_t ld_ref, const float *test, int64_t ld_test,
+                             int64_t rows, int64_t cols, double *sums, int num_sms, cudaStream_t stream);
 
 // One contraction problem (a group of the grouped GEMM, or the whole GEMM).
 struct GemmGroup {

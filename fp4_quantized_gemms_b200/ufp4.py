@@ -31,6 +31,7 @@ EXPORTED = [
     "ufp4_gemm_dgrad", "ufp4_gemm_wgrad", "ufp4_grouped_gemm", "ufp4_check_device_status",
     "ufp4_status_string", "ufp4_version", "ufp4_set_two_level_gemm_path",
     "ufp4_get_two_level_gemm_path", "ufp4_rht_quantize_dual", "ufp4_rht_amax_dual",
+    "ufp4_quant_stats", "ufp4_qstats_summarize", "ufp4_sqnr_sums",
 ]
 
 
@@ -59,6 +60,18 @@ class GroupC(ctypes.Structure):
                 ("m", "n", "k", "a_row", "a_col", "b_row", "b_col", "c_row", "c_col")]
 
 
+class QStatsC(ctypes.Structure):
+    _fields_ = [("signal", ctypes.c_double), ("noise", ctypes.c_double),
+                ("level_err", ctypes.c_double * 8), ("level_n", ctypes.c_uint64 * 8),
+                ("code_count", ctypes.c_uint64 * 16), ("nonzero", ctypes.c_uint64),
+                ("underflow", ctypes.c_uint64)]
+
+
+class QStatsSummaryC(ctypes.Structure):
+    _fields_ = [("sqnr_db", ctypes.c_double), ("bucket_ratio", ctypes.c_double),
+                ("underflow_ratio", ctypes.c_double), ("level_mean_err", ctypes.c_double * 8)]
+
+
 _lib = None
 
 
@@ -83,6 +96,12 @@ def lib() -> ctypes.CDLL:
         L.ufp4_rht_amax.argtypes = [P, i64, i64, i64, i32, i32, u64, P, P]
         L.ufp4_rht_quantize.restype = st
         L.ufp4_rht_quantize.argtypes = [P, i64, i64, i64, i32, P, ctypes.POINTER(QTensorC), P]
+        L.ufp4_quant_stats.restype = st
+        L.ufp4_quant_stats.argtypes = [P, i64, i64, i64, i32, ctypes.POINTER(QTensorC), P, P]
+        L.ufp4_qstats_summarize.restype = st
+        L.ufp4_qstats_summarize.argtypes = [ctypes.POINTER(QStatsC), i32, ctypes.POINTER(QStatsSummaryC)]
+        L.ufp4_sqnr_sums.restype = st
+        L.ufp4_sqnr_sums.argtypes = [P, i64, P, i64, i64, i64, P, P]
         L.ufp4_rht_amax_dual.restype = st
         L.ufp4_rht_amax_dual.argtypes = [P, i64, i64, i64, i32, u64, P, P, P]
         L.ufp4_rht_quantize_dual.restype = st
@@ -274,6 +293,45 @@ def rht_quantize_dual(x: torch.Tensor, cfg_cols: QuantConfig, cfg_rows: QuantCon
     _check(lib().ufp4_rht_quantize_dual(ctypes.c_void_p(x.data_ptr()), rows, cols, x.stride(0), am_c, am_r,
                                         ctypes.byref(qc), ctypes.byref(qr), _stream_ptr(x.device)),
            "ufp4_rht_quantize_dual")
+    return out
+
+
+def quant_stats(x: torch.Tensor, axis: int, q: QTensor, out: torch.Tensor | None = None) -> dict:
+    """Diagnostics sums of operand q quantized from x along axis (a host copy
+    of ufp4_qstats_t as a dict, plus its ufp4_qstats_summarize figures)."""
+    _require_cuda(x, q.codes)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    if out is None:
+        out = torch.zeros(ctypes.sizeof(QStatsC) // 8, dtype=torch.float64, device=x.device)
+    rows, cols = x.shape
+    qc = q.c()
+    _check(lib().ufp4_quant_stats(ctypes.c_void_p(x.data_ptr()), rows, cols, x.stride(0), axis,
+                                  ctypes.byref(qc), ctypes.c_void_p(out.data_ptr()), _stream_ptr(x.device)),
+           "ufp4_quant_stats")
+    host = QStatsC.from_buffer_copy(out.cpu().numpy().tobytes())
+    sm = QStatsSummaryC()
+    _check(lib().ufp4_qstats_summarize(ctypes.byref(host), q.cfg.grid, ctypes.byref(sm)),
+           "ufp4_qstats_summarize")
+    return {
+        "signal": host.signal, "noise": host.noise, "level_err": list(host.level_err),
+        "level_n": list(host.level_n), "code_count": list(host.code_count),
+        "nonzero": host.nonzero, "underflow": host.underflow,
+        "sqnr_db": sm.sqnr_db, "bucket_ratio": sm.bucket_ratio, "underflow_ratio": sm.underflow_ratio,
+        "level_mean_err": list(sm.level_mean_err),
+    }
+
+
+def sqnr_sums(ref: torch.Tensor, test: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """[sum ref^2, sum (test - ref)^2] (float64 [2] on device) of two fp32 matrices."""
+    _require_cuda(ref, test)
+    assert ref.dtype == torch.float32 and test.dtype == torch.float32 and ref.shape == test.shape
+    assert ref.stride(1) == 1 and test.stride(1) == 1
+    if out is None:
+        out = torch.empty(2, dtype=torch.float64, device=ref.device)
+    rows, cols = ref.shape
+    _check(lib().ufp4_sqnr_sums(ctypes.c_void_p(ref.data_ptr()), ref.stride(0),
+                                ctypes.c_void_p(test.data_ptr()), test.stride(0), rows, cols,
+                                ctypes.c_void_p(out.data_ptr()), _stream_ptr(ref.device)), "ufp4_sqnr_sums")
     return out
 
 

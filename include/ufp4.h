@@ -274,6 +274,68 @@ typedef enum {
 ufp4_status_t ufp4_set_two_level_gemm_path(int32_t path);
 int32_t ufp4_get_two_level_gemm_path(void);
 
+/* ---------------------------------------------------------------------------
+ * Quantization diagnostics ([PL] §5 "Q1: Grid geometry and RHT" and Appendix A
+ * "RHT-Induced SQNR Changes in Tensors and GEMM Outputs"; [GS] "Kwantisatie en
+ * GEMM Diagnostiek": tensor and GEMM-output SQNR, their change under the RHT,
+ * bucket use, and the signed level error of §3.1 "Shrinkage Bias").  The
+ * pages print no formulas; the definitions below are this library's.
+ *
+ * Sums and counts over the logical columns [0, k) of every output row of a
+ * quantized operand, u the rotated value the quantizer rounded (recomputed
+ * from x with the operand's cfg) and sigma its block step (s, or e_b * S):
+ *   signal          sum u^2
+ *   noise           sum (u - deq)^2, deq = +-lvl(code) * sigma
+ *   level_err[k]    sum over elements of magnitude code k in blocks with
+ *                   sigma > 0 of lvl(k) - |u| / sigma (grid units; < 0 means
+ *                   the level sits below the values it stands for)
+ *   level_n[k]      the number of those elements
+ *   code_count[c]   elements per 4-bit code c (0x8 never occurs)
+ *   nonzero         elements with u != 0;  underflow: of those, coded 0
+ * The floating-point sums are accumulated in fp32 over each 64-element
+ * segment of a row and in fp64 across segments (relative error well below
+ * 1e-5); the order of the fp64 additions is not fixed (atomics). */
+typedef struct {
+    double signal;
+    double noise;
+    double level_err[8];
+    uint64_t level_n[8];
+    uint64_t code_count[16];
+    uint64_t nonzero;
+    uint64_t underflow;
+} ufp4_qstats_t;
+
+/* Fills *stats_dev (device memory, zeroed by the call) for the operand q
+ * quantized from x_dev along axis (the arguments of the ufp4_rht_quantize
+ * call that produced q).  Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED, CUDA. */
+ufp4_status_t ufp4_quant_stats(const void *x_dev, int64_t rows, int64_t cols, int64_t ld,
+                               int32_t axis, const ufp4_qtensor_t *q, ufp4_qstats_t *stats_dev,
+                               void *stream);
+
+/* Derived figures of a host copy of the sums (plain host arithmetic):
+ *   sqnr_db          10 log10(signal / noise) (+inf when noise = 0)
+ *   bucket_ratio     share of the grid's codes (15; 9 for the restricted
+ *                    E2M1 grid) holding more than 1/(15*16) of the elements
+ *   underflow_ratio  underflow / nonzero (0 when nonzero = 0)
+ *   level_mean_err   level_err[k] / level_n[k] (NaN when level_n[k] = 0)
+ * Errors: INVALID_ARG (NULL pointer, unknown grid). */
+typedef struct {
+    double sqnr_db;
+    double bucket_ratio;
+    double underflow_ratio;
+    double level_mean_err[8];
+} ufp4_qstats_summary_t;
+ufp4_status_t ufp4_qstats_summarize(const ufp4_qstats_t *stats_host, int32_t grid,
+                                    ufp4_qstats_summary_t *out);
+
+/* GEMM-output SQNR sums: sums_dev[0] = sum ref^2, sums_dev[1] = sum (test -
+ * ref)^2 over a rows x cols fp32 region (row pitches ld_ref, ld_test >= cols),
+ * accumulated in fp64 (device memory, zeroed by the call).  SQNR =
+ * 10 log10(sums[0] / sums[1]).  Errors: INVALID_ARG, CUDA. */
+ufp4_status_t ufp4_sqnr_sums(const float *ref_dev, int64_t ld_ref, const float *test_dev,
+                             int64_t ld_test, int64_t rows, int64_t cols, double *sums_dev,
+                             void *stream);
+
 /* Reads and clears the device-side error word that kernels set when a
  * bounded pipeline wait gives up (synchronises the current device).
  * Returns UFP4_OK or UFP4_ERR_DEVICE_TIMEOUT (or UFP4_ERR_CUDA). */

@@ -2,6 +2,7 @@
 function ``include/ufp4.h`` declares, the ctypes mirrors match the C struct
 layouts, and host-side validation rejects bad arguments before any launch."""
 import ctypes
+import math
 import os
 import re
 import subprocess
@@ -52,6 +53,9 @@ int main(void) {
          offsetof(ufp4_qtensor_t, scale_ld), offsetof(ufp4_qtensor_t, cfg),
          offsetof(ufp4_qtensor_t, corr));
   printf("%zu %zu\\n", sizeof(ufp4_group_t), offsetof(ufp4_group_t, c_col));
+  printf("%zu %zu %zu %zu %zu\\n", sizeof(ufp4_qstats_t), offsetof(ufp4_qstats_t, level_n),
+         offsetof(ufp4_qstats_t, code_count), offsetof(ufp4_qstats_t, underflow),
+         sizeof(ufp4_qstats_summary_t));
   return 0;
 }
 """)
@@ -61,7 +65,11 @@ int main(void) {
     c1 = list(map(int, out[0].split()))
     c2 = list(map(int, out[1].split()))
     c3 = list(map(int, out[2].split()))
+    c4 = list(map(int, out[3].split()))
     Q, T, G = ufp4.QuantCfgC, ufp4.QTensorC, ufp4.GroupC
+    St, Sm = ufp4.QStatsC, ufp4.QStatsSummaryC
+    assert c4 == [ctypes.sizeof(St), St.level_n.offset, St.code_count.offset, St.underflow.offset,
+                  ctypes.sizeof(Sm)]
     assert c1[:4] == [ctypes.sizeof(Q), Q.sr_seed.offset, Q.rht_sign_mask.offset, Q.scale_fmt.offset]
     assert c2 == [ctypes.sizeof(T), T.rows.offset, T.scale_ld.offset, T.cfg.offset, T.corr.offset]
     assert c3 == [ctypes.sizeof(G), G.c_col.offset]
@@ -188,3 +196,44 @@ def test_two_level_gemm_path_selector(L):
         assert ufp4.get_two_level_gemm_path() == ufp4.GEMM_PATH_AUTO
     finally:
         ufp4.set_two_level_gemm_path(old)
+
+
+def test_qstats_summarize_host_arithmetic(L):
+    """The summary is plain host arithmetic: closed-form values of a made-up
+    set of sums, and the argument checks."""
+    st = ufp4.QStatsC()
+    st.signal, st.noise = 1000.0, 10.0                  # 20 dB
+    for c, n in {0: 500, 1: 300, 9: 150, 7: 40, 15: 9, 3: 1}.items():
+        st.code_count[c] = n                            # 1000 elements; threshold 1000/240
+    st.level_err[1], st.level_n[1] = -4.5, 450
+    st.nonzero, st.underflow = 800, 300
+    sm = ufp4.QStatsSummaryC()
+    assert L.ufp4_qstats_summarize(ctypes.byref(st), 0, ctypes.byref(sm)) == ufp4.OK
+    assert sm.sqnr_db == 20.0
+    assert sm.bucket_ratio == 5 / 15                     # codes 0, 1, 9, 7, 15 (9 > 4.17)
+    assert sm.underflow_ratio == 300 / 800
+    assert sm.level_mean_err[1] == -0.01 and math.isnan(sm.level_mean_err[2])
+    assert L.ufp4_qstats_summarize(ctypes.byref(st), 2, ctypes.byref(sm)) == ufp4.OK
+    assert sm.bucket_ratio == 5 / 9
+    st.noise = 0.0
+    assert L.ufp4_qstats_summarize(ctypes.byref(st), 1, ctypes.byref(sm)) == ufp4.OK
+    assert math.isinf(sm.sqnr_db)
+    assert L.ufp4_qstats_summarize(ctypes.byref(st), 3, ctypes.byref(sm)) == ufp4.ERR_INVALID_ARG
+    assert L.ufp4_qstats_summarize(None, 0, ctypes.byref(sm)) == ufp4.ERR_INVALID_ARG
+
+
+def test_diagnostics_validation_rejects_before_launch(L):
+    x = ctypes.c_void_p(4096)
+    q = _q(rows=64, k=128)
+    st = ctypes.c_void_p(8192)
+    S = L.ufp4_quant_stats
+    assert S(x, 64, 128, 128, 0, ctypes.byref(q), None, None) == ufp4.ERR_INVALID_ARG
+    assert S(x, 64, 128, 128, 0, ctypes.byref(q), ctypes.c_void_p(8196), None) == ufp4.ERR_ALIGNMENT
+    assert S(x, 64, 128, 128, 1, ctypes.byref(q), st, None) == ufp4.ERR_INVALID_ARG   # shape
+    assert S(x, 64, 128, 100, 0, ctypes.byref(q), st, None) == ufp4.ERR_INVALID_ARG   # ld < cols
+    assert S(None, 64, 128, 128, 0, ctypes.byref(q), st, None) == ufp4.ERR_INVALID_ARG
+    Q = L.ufp4_sqnr_sums
+    assert Q(x, 128, x, 128, 4, 128, None, None) == ufp4.ERR_INVALID_ARG
+    assert Q(x, 100, x, 128, 4, 128, st, None) == ufp4.ERR_INVALID_ARG
+    assert Q(None, 128, x, 128, 4, 128, st, None) == ufp4.ERR_INVALID_ARG
+    assert Q(x, 128, x, 128, -1, 128, st, None) == ufp4.ERR_INVALID_ARG
