@@ -320,6 +320,7 @@ def run_device(args, rank, world, device):
 
     # ---- grouped (MoE) GEMMs of the mixture-of-experts config (reported, not in `value`)
     moe = run_moe(device, step.two)
+    diag = run_diag(step)
 
     value = world * flops / (ms_per_step * 1e-3) / 1e12
     gemm_tf = [2 * s.M * s.N * s.K / (g * 1e-3) / 1e12 for g in g_ms]
@@ -379,10 +380,55 @@ def run_device(args, rank, world, device):
         },
         "e2e": e2e,
         "moe_grouped": moe,
+        "diagnostics": diag,
         "device_status": ufp4.status_string(status),
     }
     result["clocks"] = clk.summary()
     return result
+
+
+def run_diag(step: LayerStep, reps: int = 10) -> dict:
+    """Diagnostics of the step's six operands (SQNR, bucket ratio, underflow
+    ratio from ufp4_quant_stats) and the time of the two diagnostics kernels
+    on the largest tensors: quant_stats of dY^T (8192 x 8192) and the
+    GEMM-output SQNR sums of the 8192 x 8192 fp32 output Y against a copy of
+    it held in a separate buffer (both read from HBM)."""
+    u = step.u
+    C, R = u.ALONG_COLS, u.ALONG_ROWS
+    out = {}
+    for name, x, axis, q in (("X", step.X, C, step.qx), ("W", step.W, C, step.qw),
+                             ("dY", step.dY, C, step.qdy), ("dY^T", step.dY, R, step.qdyt),
+                             ("W^T", step.W, R, step.qwt), ("X^T", step.X, R, step.qxt)):
+        st = u.quant_stats(x, axis, q)
+        out[name] = {"sqnr_db": round(st["sqnr_db"], 3), "bucket_ratio": round(st["bucket_ratio"], 4),
+                     "underflow_ratio": round(st["underflow_ratio"], 5)}
+    buf = torch.zeros(64, dtype=torch.float64, device=step.dev)
+    sums = torch.zeros(2, dtype=torch.float64, device=step.dev)
+    ref = step.Y
+    test = step.Y.clone()
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize(step.dev)
+        return a.elapsed_time(b) / reps
+
+    t_stats = timed(lambda: u.quant_stats_launch(step.dY, R, step.qdyt, out=buf))
+    t_sqnr = timed(lambda: u.sqnr_sums(ref, test, out=sums))
+    n = step.dY.numel()
+    per = 2 + 0.5 + (1 / 16 if step.two else 4 / 16)
+    out["quant_stats_dYT"] = {"ms": round(t_stats, 4), "GBps": round(n * per / (t_stats * 1e-3) / 1e9, 1),
+                              "bytes_per_element": per}
+    m = ref.numel()
+    out["sqnr_sums_8192x8192"] = {"ms": round(t_sqnr, 4), "GBps": round(m * 8 / (t_sqnr * 1e-3) / 1e9, 1)}
+    del test
+    return out
 
 
 def run_e2e(step: LayerStep, args, device):

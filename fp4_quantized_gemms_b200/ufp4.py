@@ -296,9 +296,9 @@ def rht_quantize_dual(x: torch.Tensor, cfg_cols: QuantConfig, cfg_rows: QuantCon
     return out
 
 
-def quant_stats(x: torch.Tensor, axis: int, q: QTensor, out: torch.Tensor | None = None) -> dict:
-    """Diagnostics sums of operand q quantized from x along axis (a host copy
-    of ufp4_qstats_t as a dict, plus its ufp4_qstats_summarize figures)."""
+def quant_stats_launch(x: torch.Tensor, axis: int, q: QTensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Enqueue ufp4_quant_stats; returns the device buffer holding the
+    ufp4_qstats_t (float64 words)."""
     _require_cuda(x, q.codes)
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     if out is None:
@@ -308,6 +308,13 @@ def quant_stats(x: torch.Tensor, axis: int, q: QTensor, out: torch.Tensor | None
     _check(lib().ufp4_quant_stats(ctypes.c_void_p(x.data_ptr()), rows, cols, x.stride(0), axis,
                                   ctypes.byref(qc), ctypes.c_void_p(out.data_ptr()), _stream_ptr(x.device)),
            "ufp4_quant_stats")
+    return out
+
+
+def quant_stats(x: torch.Tensor, axis: int, q: QTensor, out: torch.Tensor | None = None) -> dict:
+    """Diagnostics sums of operand q quantized from x along axis (a host copy
+    of ufp4_qstats_t as a dict, plus its ufp4_qstats_summarize figures)."""
+    out = quant_stats_launch(x, axis, q, out)
     host = QStatsC.from_buffer_copy(out.cpu().numpy().tobytes())
     sm = QStatsSummaryC()
     _check(lib().ufp4_qstats_summarize(ctypes.byref(host), q.cfg.grid, ctypes.byref(sm)),
