@@ -752,16 +752,19 @@ struct Fp4Cfg {
     static constexpr int kRawA = BM * (BKE / 16);
     static constexpr int kRawB = BN * (BKE / 16);
     static constexpr int kIn = CIN ? 2 : 1;         // code planes loaded per stage
-    // [codes A | planes A | codes B | planes B | raw scales A | raw scales B]
-    // (the planes only with CIN): a 3-D box fills an operand's two tiles.
+    // Code stage: [codes A | planes A | codes B | planes B] (the planes only
+    // with CIN: a 3-D box fills an operand's two tiles).
     static constexpr int o_codes_a = 0;
     static constexpr int o_cin_a = o_codes_a + kCodesA;         // CIN only
     static constexpr int o_codes_b = o_codes_a + kIn * kCodesA;
     static constexpr int o_cin_b = o_codes_b + kCodesB;         // CIN only
-    static constexpr int o_raw_a = o_codes_a + kIn * (kCodesA + kCodesB);
-    static constexpr int o_raw_b = o_raw_a + kRawA;
-    static constexpr int kStage = (o_raw_b + kRawB + 1023) / 1024 * 1024;
+    static constexpr int kStage = (kIn * (kCodesA + kCodesB) + 1023) / 1024 * 1024;
     static constexpr int kCorr = (kCodesA + kCodesB + 1023) / 1024 * 1024;  // one slot
+    // Scale factors run in their own ring, one TMEM slot per raw-scale smem
+    // slot ([raw scales A | raw scales B]), ahead of the code stages.
+    static constexpr int o_raw_a = 0;                           // within a raw slot
+    static constexpr int o_raw_b = kRawA;
+    static constexpr int kRawSlot = (kRawA + kRawB + 127) / 128 * 128;
     // scale-factor atoms per stage: K step j, kind 0 = SFA, 1 / 2 = SFB rows
     // [0, 128) / [128, BN)
     static constexpr int kAtoms = 3 * KST;
@@ -772,21 +775,31 @@ struct Fp4Cfg {
     static constexpr int kSfBase = 2 * kAccCols;
     static constexpr int kBudget = 232448 - 2048;   // barriers, alignment slack
     static constexpr int kOutChunk = BM * 32 * 4;   // epilogue staging: 128 rows x 32 fp32
-    static constexpr int kNsSmem = (kBudget - ND * kCorr - kOutChunk - kScr) / kStage;
-    static constexpr int kNsTmem = (512 - kSfBase) / kSfCols;   // one scale-factor slot per stage
+    // Code stages, capped by the TMEM scale-factor slots: slot s serves code
+    // stage s, so the stage's release (empty) also frees its factors.
+    static constexpr int kNsTmem = (512 - kSfBase) / kSfCols;
+    static constexpr int kNsSmem = (kBudget - ND * kCorr - kOutChunk - kScr - kNsTmem * kRawSlot) / kStage;
     static constexpr int NS = kNsSmem < kNsTmem ? kNsSmem : kNsTmem;
+    static constexpr int NSF = NS;                              // raw-scale slots
+    // E1M2 (eight MMAs a stage): a scale producer warp streams the raw scales
+    // ahead of the code tiles.  E2M1 (two MMAs a stage): the code producer
+    // issues them just before each stage's codes (fewer TMA streams).
+    static constexpr bool kAheadScales = GRID == 0;
     static constexpr int o_corr = NS * kStage;
     static constexpr int o_out = o_corr + ND * kCorr;
     static constexpr int o_scr = o_out + kOutChunk;
-    static constexpr int o_bar = o_scr + kScr;
-    // full, ready, empty, tdone per stage; acc_full[2], acc_empty[2], edone, drain
-    static constexpr int kNumBars = 4 * NS + 6;
+    static constexpr int o_raw = o_scr + kScr;
+    static constexpr int o_bar = o_raw + NSF * kRawSlot;
+    // code ring: full, empty, cfull; scale-factor ring: sfull, sraw_free,
+    // sf_ready, tdone; acc_full[2], acc_empty[2], edone, drain
+    static constexpr int kNumBars = 3 * NS + 4 * NSF + 6;
     static constexpr int o_misc = o_bar + kNumBars * 8;
     static constexpr int kAlloc = o_misc + 64 + 1024;
-    static constexpr int kThreads = 32 * (2 + NT + NE);
+    // producer, MMA issuer, transform warps, epilogue warps, scale producer
+    static constexpr int kThreads = 32 * (3 + NT + NE);
     static_assert(kGroupWarps == 4, "one warp per TMEM lane quarter in each transform group");
-    static_assert(NS >= 4, "pipeline depth");
-    static_assert(kSfBase + NS * kSfCols <= 512, "TMEM budget");
+    static_assert(NS >= 4 && NSF >= 4, "pipeline depth");
+    static_assert(kSfBase + NSF * kSfCols <= 512, "TMEM budget");
     static_assert(kAlloc <= 232448, "shared memory budget");
     static_assert(o_corr % 1024 == 0 && o_out % 1024 == 0, "swizzle alignment");
     static_assert(BN % 32 == 0 && BN > 128 && BN <= 256, "two SFB row groups, 32-column chunks");
@@ -840,21 +853,28 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
     constexpr int BN = C::BN;
     constexpr int TM = C::TM;
     constexpr int NS = C::NS;
+    constexpr int NSF = C::NSF;
     constexpr bool kPair = CG == 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::o_bar);
-    uint64_t *ready = full + NS;        // in CTA 0: stage transformed (all CTAs)
-    uint64_t *empty = ready + NS;       // MMAs done with the stage (multicast commit)
-    uint64_t *tdone = empty + NS;       // this CTA's transform warps done (pairs)
-    uint64_t *acc_full = tdone + NS;    // [2]
-    uint64_t *acc_empty = acc_full + 2; // [2], in CTA 0: accumulator drained (all CTAs)
-    uint64_t *edone = acc_empty + 2;    // this CTA's epilogue warps drained (pairs)
+    // code ring (index s = it % NS)
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::o_bar);   // code tiles landed
+    uint64_t *empty = full + NS;          // MMAs done with the stage (multicast commit)
+    uint64_t *cfull = empty + NS;         // pairs, in CTA 0: CTA 1's code tiles landed
+    // scale-factor ring (index j = it % NSF)
+    uint64_t *sfull = cfull + NS;         // raw scale factors landed
+    uint64_t *sraw_free = sfull + NSF;    // transform read the raw slot
+    uint64_t *sf_ready = sraw_free + NSF; // in CTA 0: factors in TMEM (all CTAs)
+    uint64_t *tdone = sf_ready + NSF;     // this CTA's transform warps done (pairs)
+    uint64_t *acc_full = tdone + NSF;     // [2]
+    uint64_t *acc_empty = acc_full + 2;   // [2], in CTA 0: accumulator drained (all CTAs)
+    uint64_t *edone = acc_empty + 2;      // this CTA's epilogue warps drained (pairs)
     uint64_t *drain = edone + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::o_misc);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::o_misc + 4);
     auto stage = [&](int s) { return smem + s * C::kStage; };
+    auto raw_slot = [&](int j) { return smem + C::o_raw + j * C::kRawSlot; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -867,8 +887,13 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&ready[i], kPair ? CG : C::kGroupWarps);
             mbar_init(&empty[i], 1);
+            mbar_init(&cfull[i], 1);
+        }
+        for (int i = 0; i < NSF; ++i) {
+            mbar_init(&sfull[i], 1);
+            mbar_init(&sraw_free[i], C::kGroupWarps);
+            mbar_init(&sf_ready[i], kPair ? CG : C::kGroupWarps);
             mbar_init(&tdone[i], C::kGroupWarps);
         }
         for (int i = 0; i < 2; ++i) {
@@ -904,6 +929,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
+            const uint64_t pol = l2_policy_evict_last();
             uint32_t it = 0;
             bool ok = true;
             for (int64_t t = unit; t < ntiles && ok; t += nunits) {
@@ -920,22 +946,27 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                     const int32_t acol = static_cast<int32_t>(tl.g.a_col + ks * C::BKE);
                     const int32_t bcol = static_cast<int32_t>(tl.g.b_col + ks * C::BKE);
                     uint8_t *st = stage(s);
-                    mbar_arrive_expect_tx(&full[s],
-                                          C::kIn * (C::kCodesA + C::kCodesB) + (BM + BN) * nraw);
+                    if constexpr (!C::kAheadScales) {
+                        uint8_t *rs = raw_slot(s);
+                        mbar_arrive_expect_tx(&sfull[s], (BM + BN) * nraw);
+                        tma_load_2d_hint(rs + C::o_raw_a, &args.tm_a_scales, &sfull[s], arow, acol / blk, pol);
+                        tma_load_2d_hint(rs + C::o_raw_b, &args.tm_b_scales, &sfull[s], brow, bcol / blk, pol);
+                    }
+                    mbar_arrive_expect_tx(&full[s], C::kIn * (C::kCodesA + C::kCodesB));
                     const int32_t brow_h = brow + C::BNh * static_cast<int32_t>(rank);
+                    // Operand tiles are read by many CTAs: keep them in L2
+                    // ahead of the streamed output.
                     if (CIN && args.planes3d) {
-                        tma_load_3d(st + C::o_codes_a, &args.tm_a_corr, &full[s], acol / 2, arow, 0);
-                        tma_load_3d(st + C::o_codes_b, &args.tm_b_corr, &full[s], bcol / 2, brow_h, 0);
+                        tma_load_3d_hint(st + C::o_codes_a, &args.tm_a_corr, &full[s], acol / 2, arow, 0, pol);
+                        tma_load_3d_hint(st + C::o_codes_b, &args.tm_b_corr, &full[s], bcol / 2, brow_h, 0, pol);
                     } else {
-                        tma_load_2d(st + C::o_codes_a, &args.tm_a_codes, &full[s], acol / 2, arow);
-                        tma_load_2d(st + C::o_codes_b, &args.tm_b_codes, &full[s], bcol / 2, brow_h);
+                        tma_load_2d_hint(st + C::o_codes_a, &args.tm_a_codes, &full[s], acol / 2, arow, pol);
+                        tma_load_2d_hint(st + C::o_codes_b, &args.tm_b_codes, &full[s], bcol / 2, brow_h, pol);
                         if (CIN) {
-                            tma_load_2d(st + C::o_cin_a, &args.tm_a_corr, &full[s], acol / 2, arow);
-                            tma_load_2d(st + C::o_cin_b, &args.tm_b_corr, &full[s], bcol / 2, brow_h);
+                            tma_load_2d_hint(st + C::o_cin_a, &args.tm_a_corr, &full[s], acol / 2, arow, pol);
+                            tma_load_2d_hint(st + C::o_cin_b, &args.tm_b_corr, &full[s], bcol / 2, brow_h, pol);
                         }
                     }
-                    tma_load_2d(st + C::o_raw_a, &args.tm_a_scales, &full[s], arow, acol / blk);
-                    tma_load_2d(st + C::o_raw_b, &args.tm_b_scales, &full[s], brow, bcol / blk);
                 }
             }
             // Drain: the last copy into each stage has landed before exit.
@@ -945,11 +976,34 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                     uint32_t dummy = 0;
                     mbar_wait(&full[s], (last / NS) & 1, kErrTimeoutDrain,
                               reinterpret_cast<volatile uint32_t *>(&dummy));
+                    if constexpr (!C::kAheadScales)
+                        mbar_wait(&sfull[s], (last / NS) & 1, kErrTimeoutDrain,
+                                  reinterpret_cast<volatile uint32_t *>(&dummy));
                 }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ UMMA issuer (CTA 0)
+        if constexpr (kPair) {
+            // CTA 1: relay each stage's landed code tiles to CTA 0's MMAs.
+            if (lane == 0 && rank == 1) {
+                uint32_t it = 0;
+                bool ok = true;
+                for (int64_t t = unit; t < ntiles && ok; t += nunits) {
+                    const Tile tl = get_tile<TM, BN>(args, t);
+                    const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
+                    for (int ks = 0; ks < nks; ++ks, ++it) {
+                        const int s = it % NS;
+                        if (!mbar_wait(&full[s], (it / NS) & 1, kErrTimeoutMma, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        fence_proxy_async_cluster();
+                        mbar_arrive_remote(&cfull[s], 0);
+                    }
+                }
+            }
+        }
         if (lane == 0 && rank == 0) {
             constexpr uint32_t idesc = umma_idesc_fp4_bs(TM, BN);
             auto wait_any = [&](uint64_t *bar, uint32_t parity) {
@@ -968,7 +1022,12 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                 bool first = true;
                 for (int ks = 0; ks < nks && ok; ++ks, ++it) {
                     const int s = it % NS;
-                    if (!wait_any(&ready[s], (it / NS) & 1)) {
+                    const int j = it % NSF;
+                    // factors in TMEM (with pairs: both CTAs'), then the code
+                    // tiles (with pairs: CTA 1's relayed by its idle MMA warp)
+                    if (!wait_any(&sf_ready[j], (it / NSF) & 1) ||
+                        !mbar_wait(&full[s], (it / NS) & 1, kErrTimeoutMma, abort_flag) ||
+                        (kPair && !wait_any(&cfull[s], (it / NS) & 1))) {
                         ok = false;
                         break;
                     }
@@ -977,7 +1036,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                     // scale factors of K step j: SFA at 12 j, SFB rows 0-127
                     // at 12 j + 4, rows 128+ at 12 j + 8 of the stage's slot
                     // (written by the transform warps of each CTA)
-                    const uint32_t sf0 = tmem_base + C::kSfBase + s * C::kSfCols;
+                    const uint32_t sf0 = tmem_base + C::kSfBase + j * C::kSfCols;
                     // K steps of 64 in this stage (a tail uses only its own)
                     const int64_t rem = tl.g.k - static_cast<int64_t>(ks) * C::BKE;
                     const int steps = rem >= C::BKE ? C::KST : static_cast<int>((rem + 63) / 64);
@@ -1013,10 +1072,12 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
     } else if (warp < 2 + C::NT) {
         // ------------------------------------------------------------ transform
         // Two groups of four warps (one per TMEM lane quarter) take alternate
-        // stages.  Each warp builds every scale-factor atom of its stage for
-        // its lane quarter (a 4x4 byte transpose per 4 rows into its scratch)
-        // and stores it with tcgen05.st into the stage's slot; that slot was
-        // last read by the MMAs that released this stage's TMA buffer.
+        // iterations.  Each warp builds every scale-factor atom of its
+        // iteration for its lane quarter (a 4x4 byte transpose per 4 rows into
+        // its scratch) and stores it with tcgen05.st into TMEM slot it % NS,
+        // once the MMAs that last read that slot (and released the code stage
+        // of the same index) are done.  The raw scales arrive in their own
+        // ring, ahead of the code tiles.
         const int tw = warp - 2;
         const int grp = tw >> 2;
         const int gt = (tw & 3) * 32 + lane;            // thread index within the group
@@ -1033,11 +1094,17 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
             for (int ks = 0; ks < nks; ++ks, ++it) {
                 if (static_cast<int>(it & 1) != grp) continue;
                 const int s = it % NS;
-                if (!warp_wait(&full[s], (it / NS) & 1, kErrTimeoutTransform, abort_flag)) {
+                const int j = it % NSF;
+                const uint32_t jph = (it / NSF) & 1;
+                constexpr bool kBuild = GRID == 0 && !CIN;   // correction planes here
+                // The factors need the raw scales and a free TMEM slot;
+                // building correction planes needs the codes.
+                if (!warp_wait(&sfull[j], jph, kErrTimeoutTransform, abort_flag) ||
+                    !warp_wait(&empty[j], jph ^ 1, kErrTimeoutTransform, abort_flag) ||
+                    (kBuild && !warp_wait(&full[s], (it / NS) & 1, kErrTimeoutTransform, abort_flag))) {
                     ok = false;
                     break;
                 }
-                constexpr bool kBuild = GRID == 0 && !CIN;   // correction planes here
                 // Correction slot it & 1 was last read by the MMAs of it - 2.
                 if (kBuild && it >= 2) {
                     const uint32_t p = it - 2;
@@ -1055,7 +1122,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                     const int jk = a / 3, kind = a % 3;
                     const int rows = kind == 0 ? BM : BN;
                     const int r = 4 * lane + (kind == 2 ? 128 : 0);
-                    const uint8_t *raw = st + (kind == 0 ? C::o_raw_a : C::o_raw_b) + r;
+                    const uint8_t *raw = raw_slot(j) + (kind == 0 ? C::o_raw_a : C::o_raw_b) + r;
                     if (r < rows) {
                         if (blk == 16) {
 #pragma unroll
@@ -1070,6 +1137,9 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                         w[a][0] = w[a][1] = w[a][2] = w[a][3] = 0u;
                     }
                 }
+                // raw slot j read: the scale producer may refill it
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sraw_free[j]);
                 uint4 cw[kBuild ? kPer : 1];
                 if constexpr (kBuild) {
 #pragma unroll
@@ -1103,7 +1173,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                     }
                 }
                 __syncwarp();
-                const uint32_t sfw = lane_base + C::kSfBase + s * C::kSfCols;
+                const uint32_t sfw = lane_base + C::kSfBase + j * C::kSfCols;
 #pragma unroll
                 for (int a = 0; a < C::kAtoms; ++a) {
                     const uint4 row = *reinterpret_cast<const uint4 *>(scr + a * 512 + 16 * lane);
@@ -1117,23 +1187,23 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                     // arrive per CTA after all warps of the group.
                     fence_proxy_async_cluster();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&tdone[s]);
+                    if (lane == 0) mbar_arrive(&tdone[j]);
                     if (gt == 0) {
-                        if (!mbar_wait(&tdone[s], (it / NS) & 1, kErrTimeoutTransform, abort_flag)) {
+                        if (!mbar_wait(&tdone[j], jph, kErrTimeoutTransform, abort_flag)) {
                             ok = false;
                         } else {
-                            arrive_leader<CG>(&ready[s], rank);
+                            arrive_leader<CG>(&sf_ready[j], rank);
                         }
                     }
                     __syncwarp();
                 } else {
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&ready[s]);
+                    if (lane == 0) mbar_arrive(&sf_ready[j]);
                 }
             }
         }
-    } else {
+    } else if (warp < 2 + C::NT + C::NE) {
         // ------------------------------------------------------------ epilogue
         // Thread = accumulator row.  Each 128 x 32 fp32 chunk is staged in
         // shared memory (128-byte rows, 16-byte pieces XOR-swizzled by row)
@@ -1208,7 +1278,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                         if (grow < tl.g.m && gcol < tl.g.n) {
                             float *dst = args.c + (tl.g.c_row + grow) * args.ldc + tl.g.c_col + gcol;
                             if (gcol + 4 <= tl.g.n) {
-                                *reinterpret_cast<float4 *>(dst) = val;
+                                __stcs(reinterpret_cast<float4 *>(dst), val);   // streamed: evict first
                             } else {
                                 const float e4[4] = {val.x, val.y, val.z, val.w};
                                 for (int e = 0; e < 4 && gcol + e < tl.g.n; ++e) dst[e] = e4[e];
@@ -1220,6 +1290,44 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                     float *dst = crow + 32 * c;
                     for (int i = 0; i < 32; ++i)
                         if (col0 + i < tl.g.n) dst[i] = v[i];
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ scale producer
+        // Streams each iteration's raw scale factors (A rows of this CTA, all
+        // BN B rows) into raw slot it % NSF once the transform has read the
+        // slot's previous contents.
+        if (C::kAheadScales && lane == 0) {
+            const uint64_t pol = l2_policy_evict_last();
+            uint32_t it = 0;
+            bool ok = true;
+            for (int64_t t = unit; t < ntiles && ok; t += nunits) {
+                const Tile tl = get_tile<TM, BN>(args, t);
+                const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
+                const int32_t arow = static_cast<int32_t>(tl.g.a_row + tl.m0 + BM * rank);
+                const int32_t brow = static_cast<int32_t>(tl.g.b_row + tl.n0);
+                for (int ks = 0; ks < nks; ++ks, ++it) {
+                    const int j = it % NSF;
+                    if (!mbar_wait(&sraw_free[j], ((it / NSF) & 1) ^ 1, kErrTimeoutProducer, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const int32_t acol = static_cast<int32_t>(tl.g.a_col + ks * C::BKE);
+                    const int32_t bcol = static_cast<int32_t>(tl.g.b_col + ks * C::BKE);
+                    uint8_t *rs = raw_slot(j);
+                    mbar_arrive_expect_tx(&sfull[j], (BM + BN) * nraw);
+                    tma_load_2d_hint(rs + C::o_raw_a, &args.tm_a_scales, &sfull[j], arow, acol / blk, pol);
+                    tma_load_2d_hint(rs + C::o_raw_b, &args.tm_b_scales, &sfull[j], brow, bcol / blk, pol);
+                }
+            }
+            // Drain: the last copy into each slot has landed before exit.
+            for (int j = 0; j < NSF; ++j) {
+                if (it > static_cast<uint32_t>(j)) {
+                    const uint32_t last = (it - 1 - j) / NSF * NSF + j;
+                    uint32_t dummy = 0;
+                    mbar_wait(&sfull[j], (last / NSF) & 1, kErrTimeoutDrain,
+                              reinterpret_cast<volatile uint32_t *>(&dummy));
                 }
             }
         }

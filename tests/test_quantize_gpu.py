@@ -175,7 +175,10 @@ def test_dual_quantize_equals_two_single_calls():
     sr = ufp4.rht_quantize(x, ufp4.ALONG_ROWS, cfg.with_(sr_stream=1))
     torch.cuda.synchronize()
     for d, s in ((qc, sc), (qr, sr)):
-        assert torch.equal(d.codes, s.codes) and torch.equal(d.scales, s.scales)
+        # scale columns past the operand's rows (up to scale_ld) are padding
+        # that neither call writes
+        assert torch.equal(d.codes, s.codes)
+        assert torch.equal(d.scales[:, :d.rows], s.scales[:, :s.rows])
         assert torch.equal(d.corr, s.corr) and torch.equal(d.tensor_scale, s.tensor_scale)
 
 
