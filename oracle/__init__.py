@@ -30,7 +30,7 @@ _LIB_PATH = os.path.join(_HERE, "libufp4_oracle.so")
 
 GRID_E1M2, GRID_E2M1, GRID_E2M1_MAX2 = 0, 1, 2
 ROUND_RTNE, ROUND_SR = 0, 1
-SCALE_FP32, SCALE_E4M3_X_FP32 = 0, 1
+SCALE_FP32, SCALE_E4M3_X_FP32, SCALE_UE8M0 = 0, 1, 2
 ALONG_COLS, ALONG_ROWS = 0, 1
 
 
@@ -68,6 +68,10 @@ def lib():
         L.uo_level.restype = ctypes.c_double
         L.uo_level.argtypes = [i32, i32]
         L.uo_gmax.restype = ctypes.c_double
+        L.uo_ue8m0_scale.restype = ctypes.c_uint8
+        L.uo_ue8m0_scale.argtypes = [i32, ctypes.c_float]
+        L.uo_ue8m0_value.restype = ctypes.c_double
+        L.uo_ue8m0_value.argtypes = [ctypes.c_uint8]
         L.uo_gmax.argtypes = [i32]
         L.uo_top_code.restype = i32
         L.uo_top_code.argtypes = [i32]
@@ -129,6 +133,15 @@ def levels(grid: int) -> np.ndarray:
 
 def gmax(grid: int) -> float:
     return lib().uo_gmax(grid)
+
+
+def ue8m0_scale(grid: int, amax: float) -> int:
+    """MX block-scale byte (biased exponent) of a block maximum."""
+    return int(lib().uo_ue8m0_scale(grid, float(np.float32(amax))))
+
+
+def ue8m0_value(e: int) -> float:
+    return lib().uo_ue8m0_value(e)
 
 
 def kpad(k: int) -> int:
@@ -288,7 +301,9 @@ def quantize(x, axis: int, cfg: QuantCfg, tensor_amax: float = 0.0,
     if rc != 0:
         raise ValueError(f"oracle quantize rejected the configuration (code {rc})")
     two = cfg.scale_fmt == SCALE_E4M3_X_FP32
-    q = QTensor(codes=codes, scales=None if two else scales, escales=escales if two else None,
+    byte_scales = cfg.scale_fmt != SCALE_FP32      # E4M3 bytes, or UE8M0 exponent bytes
+    q = QTensor(codes=codes, scales=None if byte_scales else scales,
+                escales=escales if byte_scales else None,
                 S=float(S[0]) if two else 1.0, cfg=cfg, k=K, kpad=kp, row0=r0)
     return (q, u) if want_u else q
 

@@ -32,10 +32,12 @@ import oracle
 
 
 def _steps(q: oracle.QTensor) -> np.ndarray:
-    """Per-element block step sigma (float64): s, or e_b * S (exact in fp64)."""
+    """Per-element block step sigma (float64): s, e_b * S, or 2^(E - 127) (exact in fp64)."""
     B = q.cfg.block
     if q.scales is not None:
         per_block = q.scales.astype(np.float64)
+    elif q.cfg.scale_fmt == oracle.SCALE_UE8M0:
+        per_block = np.ldexp(1.0, q.escales.astype(np.int64) - 127)
     else:
         table = np.array([oracle.e4m3_value(b) for b in range(256)], dtype=np.float64)
         per_block = table[q.escales] * float(np.float32(q.S))

@@ -229,6 +229,24 @@ float uo_block_decode_base(int grid, float S)
     return gm * S;
 }
 
+/* MX-style block scale.  [PL] §6 places the study in the lineage of MXFP4,
+ * whose block scaling is coarser than NVFP4's: OCP MX formats give a block of
+ * 32 elements one shared scale that is a power of two, stored as an 8-bit
+ * biased exponent (UE8M0).  Reading: the scale 2^X is the smallest power of
+ * two that keeps the block maximum on the grid (amax <= gmax * 2^X, the "no
+ * clipping" rule of the other formats), X clamped to the byte's range
+ * [-127, 127]; an all-zero block stores 0.  Found by plain search over X. */
+uint8_t uo_ue8m0_scale(int grid, float amax)
+{
+    if (!(amax > 0.0f)) return 0;
+    const double gm = uo_gmax(grid);
+    int X = -127;
+    while (X < 127 && ldexp(gm, X) < (double)amax) X++;
+    return (uint8_t)(X + 127);
+}
+
+double uo_ue8m0_value(uint8_t e) { return ldexp(1.0, (int)e - 127); }
+
 /* ------------------------------------------------------------------------ */
 /* Load logical row r of the K-major view, zero padded to kpad, apply D then
  * H_n per n-block.  [PL] §2: for the three training GEMMs the rotation acts
@@ -292,6 +310,7 @@ int uo_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int a
     const int n = cfg->hadamard_n, B = cfg->block, grid = cfg->grid;
     if (!(n == 0 || n == 16 || n == 32 || n == 64)) return 1;
     if (!(B == 16 || B == 32)) return 2;
+    if (cfg->scale_fmt == UO_SCALE_UE8M0 && B != 32) return 3;   /* MX blocks are 32 long */
     const int64_t K = (axis == UO_ALONG_COLS) ? cols : rows;
     const int64_t kpad = uo_kpad(K);
     const int64_t nb = kpad / B;
@@ -322,6 +341,10 @@ int uo_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, int a
                     float sf = amax / (float)gmax;
                     scales[i * nb + b] = sf;
                     s = (double)sf;
+                } else if (cfg->scale_fmt == UO_SCALE_UE8M0) {
+                    uint8_t e = uo_ue8m0_scale(grid, amax);
+                    escales[i * nb + b] = e;
+                    s = uo_ue8m0_value(e);
                 } else {
                     float q = amax / G;
                     uint8_t e = uo_e4m3_rne_satfinite(q);
@@ -364,9 +387,9 @@ void uo_dequantize(const int8_t *codes, const float *scales, const uint8_t *esca
             double lv = uo_level(grid, c & 7);
             if (c & 8) lv = -lv;
             int64_t b = t / block;
-            double s = (scale_fmt == UO_SCALE_FP32)
-                           ? (double)scales[i * nb + b]
-                           : uo_e4m3_value(escales[i * nb + b]) * (double)S;
+            double s = (scale_fmt == UO_SCALE_FP32)    ? (double)scales[i * nb + b]
+                       : (scale_fmt == UO_SCALE_UE8M0) ? uo_ue8m0_value(escales[i * nb + b])
+                                                       : uo_e4m3_value(escales[i * nb + b]) * (double)S;
             out[i * kpad + t] = s * lv;
         }
     }

@@ -29,7 +29,7 @@ extern "C" {
 
 enum { UO_GRID_E1M2 = 0, UO_GRID_E2M1 = 1, UO_GRID_E2M1_MAX2 = 2 };
 enum { UO_ROUND_RTNE = 0, UO_ROUND_SR = 1 };
-enum { UO_SCALE_FP32 = 0, UO_SCALE_E4M3_X_FP32 = 1 };
+enum { UO_SCALE_FP32 = 0, UO_SCALE_E4M3_X_FP32 = 1, UO_SCALE_UE8M0 = 2 };
 enum { UO_ALONG_COLS = 0, UO_ALONG_ROWS = 1 };
 
 typedef struct {
@@ -46,6 +46,10 @@ typedef struct {
 /* grids */
 double uo_level(int grid, int k);
 double uo_gmax(int grid);
+/* MX-style power-of-two block scale: byte X + 127 of the smallest X with
+ * amax <= gmax * 2^X (clamped to [-127, 127]; 0 when amax = 0), and its value */
+uint8_t uo_ue8m0_scale(int grid, float amax);
+double uo_ue8m0_value(uint8_t e);
 int uo_top_code(int grid);   /* largest magnitude code the grid uses */
 
 /* bf16 bit pattern -> float (exact) */
