@@ -36,7 +36,10 @@ bool cfg_valid(const ufp4_quant_cfg_t &c) {
     if (!(c.hadamard_n == 0 || c.hadamard_n == 16 || c.hadamard_n == 32 || c.hadamard_n == 64))
         return false;
     if (c.block != 16 && c.block != 32) return false;
-    if (c.scale_fmt != UFP4_SCALE_FP32 && c.scale_fmt != UFP4_SCALE_E4M3_X_FP32) return false;
+    if (c.scale_fmt != UFP4_SCALE_FP32 && c.scale_fmt != UFP4_SCALE_E4M3_X_FP32 &&
+        c.scale_fmt != UFP4_SCALE_UE8M0)
+        return false;
+    if (c.scale_fmt == UFP4_SCALE_UE8M0 && c.block != 32) return false;   // MX blocks are 32 long
     return true;
 }
 
@@ -132,7 +135,7 @@ ufp4_status_t encode_operand_maps(const ufp4_qtensor_t *q, int code_rows, int sc
     if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
     const int nblk_stage = k_stage / q->cfg.block;
     const uint64_t nblk = static_cast<uint64_t>(q->kpad / q->cfg.block);
-    if (mode != 0) {
+    if (mode != 0 || q->cfg.scale_fmt == UFP4_SCALE_UE8M0) {   // byte scales
         r = encode_tensor_map_2d(scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, q->scales,
                                  static_cast<uint64_t>(q->scale_ld), nblk,
                                  static_cast<uint64_t>(q->scale_ld), static_cast<uint32_t>(scale_rows),
@@ -159,7 +162,7 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
     if (groups_dev != nullptr && (reinterpret_cast<uintptr_t>(groups_dev) & 7u))
         return UFP4_ERR_ALIGNMENT;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // fp32 block scales: per-block partials (mode 0).  Two-level scales: the
+    // fp32 or UE8M0 block scales: per-block partials (mode 0).  Two-level scales: the
     // native block-scaled FP4 kernel with one CTA per 128 x 192 tile (mode 3),
     // or what the caller picked: the same on CTA pairs with 256 x 192 tiles
     // (mode 4), the fp16-operand kernels (mode 1: one CTA per 128 x 256 tile,
@@ -188,6 +191,7 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
 
     GemmArgs args;
     memset(&args, 0, sizeof(args));
+    args.scale_ue8m0 = a->cfg.scale_fmt == UFP4_SCALE_UE8M0 ? 1 : 0;
     // B code rows staged per CTA: fp32-scale kernel 128, fp16 kernels 256
     // (one CTA) or 128 (pairs), native kernels 192 or 96, with the scales of
     // all 192 B rows of a tile in each CTA.

@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(kDiagThreads) quant_stats_kernel(const __grid_
 #pragma unroll
     for (int j = 0; j < 8; ++j) lerr[j] = 0.0;
     uint32_t nonzero = 0, underflow = 0;
-    const float S = a.scale_fmt == 1 ? *a.S : 1.0f;
+    const float S = a.scale_fmt == 1 ? *a.S : 1.0f;   // two-level only
     const int64_t nseg = a.kpad / 64;
     const int64_t units = nseg * a.out_rows;
     for (int64_t u = static_cast<int64_t>(blockIdx.x) * kDiagThreads + t; u < units;
@@ -120,6 +120,9 @@ __global__ void __launch_bounds__(kDiagThreads) quant_stats_kernel(const __grid_
             if (a.scale_fmt == 0) {
                 sm[j] = 1.0f;
                 sb[j] = reinterpret_cast<const float *>(a.scales)[b * a.scale_ld + r];
+            } else if (a.scale_fmt == 2) {           // UE8M0: 2^(E - 127), exact
+                sm[j] = 1.0f;
+                sb[j] = ldexpf(1.0f, static_cast<int>(reinterpret_cast<const uint8_t *>(a.scales)[b * a.scale_ld + r]) - 127);
             } else {
                 sm[j] = e4m3_to_f32(reinterpret_cast<const uint8_t *>(a.scales)[b * a.scale_ld + r]);
                 sb[j] = S;

@@ -393,7 +393,8 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
                             ++it;   // the code copies of this stage were issued
                             break;
                         }
-                        mbar_arrive_expect_tx(&sc_full[ss], (BM + BN) * nblk_stage * 4);
+                        mbar_arrive_expect_tx(&sc_full[ss],
+                                              (BM + BN) * nblk_stage * (args.scale_ue8m0 ? 1 : 4));
                         tma_load_2d(sc_a(ss), &args.tm_a_scales, &sc_full[ss], arow, acol / args.block);
                         tma_load_2d(sc_b(ss), &args.tm_b_scales, &sc_full[ss], brow, bcol / args.block);
                         ++sit;
@@ -632,6 +633,10 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
                     }
                     const float *sa_tile = reinterpret_cast<const float *>(sc_a(ss));
                     const float *sb_tile = reinterpret_cast<const float *>(sc_b(ss));
+                    // UE8M0 scales: exponent bytes in the same slots, 2^(E - 127)
+                    const uint8_t *sa_u8 = sc_a(ss);
+                    const uint8_t *sb_u8 = sc_b(ss);
+                    const bool ue8 = args.scale_ue8m0 != 0;
                     for (int bi = 0; bi < nblk_stage; ++bi, ++pq) {
                         const int p = pq % C::NP;
                         if (!warp_wait(&p_full[p], (pq / C::NP) & 1, kErrTimeoutEpilogue, abort_flag)) {
@@ -639,8 +644,10 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
                             break;
                         }
                         tc_fence_after();
-                        const float sa = sa_tile[bi * BM + row_in_tile];
+                        const float sa = ue8 ? ldexpf(1.0f, static_cast<int>(sa_u8[bi * BM + row_in_tile]) - 127)
+                                             : sa_tile[bi * BM + row_in_tile];
                         const float4 *sb4 = reinterpret_cast<const float4 *>(sb_tile + bi * BN + h * 64);
+                        const uchar4 *sb4u = reinterpret_cast<const uchar4 *>(sb_u8 + bi * BN + h * 64);
                         const uint32_t ta = tmem_base + p * BN + h * 64 + lane_addr;
 #pragma unroll
                         for (int half = 0; half < 2; ++half) {
@@ -654,7 +661,16 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
                             }
 #pragma unroll
                             for (int c4 = 0; c4 < 8; ++c4) {
-                                const float4 sb = sb4[8 * half + c4];
+                                float4 sb;
+                                if (ue8) {
+                                    const uchar4 e = sb4u[8 * half + c4];
+                                    sb = make_float4(ldexpf(1.0f, static_cast<int>(e.x) - 127),
+                                                     ldexpf(1.0f, static_cast<int>(e.y) - 127),
+                                                     ldexpf(1.0f, static_cast<int>(e.z) - 127),
+                                                     ldexpf(1.0f, static_cast<int>(e.w) - 127));
+                                } else {
+                                    sb = sb4[8 * half + c4];
+                                }
                                 float *ac = acc + 32 * half + 4 * c4;
                                 ac[0] = __fmaf_rn(__fmul_rn(sa, sb.x), __uint_as_float(r[4 * c4 + 0]), ac[0]);
                                 ac[1] = __fmaf_rn(__fmul_rn(sa, sb.y), __uint_as_float(r[4 * c4 + 1]), ac[1]);

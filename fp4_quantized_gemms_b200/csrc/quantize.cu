@@ -153,9 +153,34 @@ struct ScaleOut {
     uint32_t stored;  // fp32 bits of s, or the E4M3 byte
 };
 
+// MX block-scale exponent: the smallest X with amax <= gmax * 2^X, clamped to
+// [-127, 127] (-127 for amax = 0).  With amax = ma 2^ea and gmax = mg 2^eg
+// (mantissas in [1, 2)) it is ea - eg, plus one when ma > mg; the comparison
+// is exact on the scaled-down mantissas.
+template <int GRID>
+__device__ __forceinline__ int ue8m0_exponent(float amax) {
+    if (!(amax > 0.0f)) return -127;
+    const int ea = ilogbf(amax);
+    const int eg = GRID == 0 ? 0 : (GRID == 1 ? 2 : 1);     // 1.75, 6 = 1.5 * 4, 2 = 1 * 2
+    const float mg = GRID == 0 ? 1.75f : (GRID == 1 ? 1.5f : 1.0f);
+    const float ma = ldexpf(amax, -ea);                      // exact, in [1, 2)
+    const int X = ea - eg + (ma > mg ? 1 : 0);
+    return X < -127 ? -127 : (X > 127 ? 127 : X);
+}
+
 template <int GRID>
 __device__ __forceinline__ ScaleOut block_scale(float amax, int scale_fmt, float S, float G) {
     ScaleOut o;
+    if (scale_fmt == 2) {
+        // power-of-two step: every quotient |u| / 2^X is exact
+        const int X = ue8m0_exponent<GRID>(amax);
+        o.m1 = 1.0f;
+        o.b = ldexpf(1.0f, X);
+        o.zero = !(amax > 0.0f);
+        o.inv = ldexpf(1.0f, -X);
+        o.stored = static_cast<uint32_t>(X + 127);
+        return o;
+    }
     if (scale_fmt == 0) {
         const float s = __fdiv_rn(amax, gmax_of<GRID>());
         o.m1 = 1.0f;

@@ -89,6 +89,7 @@ struct GemmArgs {
     CUtensorMap tm_a_corr, tm_b_corr;     // E1M2 correction planes (corr_in); with
                                           // planes3d: 3-D maps over {codes, corr}
     int corr_in;                          // both operands carry correction planes
+    int scale_ue8m0;                      // mode 0: scales are UE8M0 exponent bytes
     int planes3d;                         // corr = codes + rows * kpad / 2 for both
 };
 

@@ -22,7 +22,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_OPERAND_MISMATCH, ERR_C
     ERR_DEVICE_TIMEOUT = range(7)
 GRID_E1M2, GRID_E2M1, GRID_E2M1_MAX2 = 0, 1, 2
 ROUND_RTNE, ROUND_SR = 0, 1
-SCALE_FP32, SCALE_E4M3_X_FP32 = 0, 1
+SCALE_FP32, SCALE_E4M3_X_FP32, SCALE_UE8M0 = 0, 1, 2
 ALONG_COLS, ALONG_ROWS = 0, 1
 DEFAULT_SIGN_MASK = 0x09F1FD9D03F0A9B4
 
@@ -213,7 +213,7 @@ def empty_qtensor(rows: int, k: int, cfg: QuantConfig, device="cuda",
         ts = None
     else:
         scales = torch.empty((nblk, sld), dtype=torch.uint8, device=device)
-        ts = torch.empty(1, dtype=torch.float32, device=device)
+        ts = torch.empty(1, dtype=torch.float32, device=device) if cfg.scale_fmt == SCALE_E4M3_X_FP32 else None
     corr = planes[1] if with_corr else None
     return QTensor(codes, scales, ts, rows, k, kpad, sld, cfg, corr)
 

@@ -43,6 +43,9 @@
  *             UFP4_SCALE_FP32:         fp32, s = RN(amax_b / gmax).
  *             UFP4_SCALE_E4M3_X_FP32:  u8 OCP E4M3 e_b; the step of the block
  *                                      is e_b * S with S = *tensor_scale.
+ *             UFP4_SCALE_UE8M0:        u8 biased exponent E; the step of the
+ *                                      block is 2^(E - 127) (tensor_scale
+ *                                      unused); GEMMs run the fp32-scale kernel.
  *   The dequantized (rotated) value of element (r, t) is s * lvl(code); the
  *   Hadamard normalisation 1/n is applied once in the GEMM (n = 0: none).
  *   corr      optional, E1M2 only: the same layout as codes, each nibble the
@@ -90,8 +93,16 @@ typedef enum {
 typedef enum { UFP4_ROUND_RTNE = 0, UFP4_ROUND_SR = 1 } ufp4_round_t;
 /* Block scale formats: plain fp32 per block, or the two-level hierarchy of
  * NVFP4 ([PL] §6 "FP4 formats, block scaling, and scale hierarchy") that UFP4
- * inherits ([DW]: the NVFP4 recipe with the grid swapped). */
-typedef enum { UFP4_SCALE_FP32 = 0, UFP4_SCALE_E4M3_X_FP32 = 1 } ufp4_scale_fmt_t;
+ * inherits ([DW]: the NVFP4 recipe with the grid swapped), or the MX-style
+ * power-of-two scale of the MXFP4 lineage that [PL] §6 also names: per block of
+ * 32 (block must be 32) the smallest 2^X with amax <= gmax * 2^X, X clamped to
+ * [-127, 127], stored as the biased exponent byte X + 127 (UE8M0; 0 for an
+ * all-zero block), no tensor scale. */
+typedef enum {
+    UFP4_SCALE_FP32 = 0,
+    UFP4_SCALE_E4M3_X_FP32 = 1,
+    UFP4_SCALE_UE8M0 = 2
+} ufp4_scale_fmt_t;
 /* Which input dimension is the GEMM's reduction dimension ([PL] §2: input
  * channels for fwd_y, output channels for bwd_dx, tokens for bwd_dw).
  * ALONG_COLS: the contiguous dimension; output row r = input row r.

@@ -86,6 +86,7 @@ def test_status_strings_and_version(L):
     (500, 16, ufp4.SCALE_FP32, 512, 256 * 256, 32 * 256 * 4),
     (2048, 32, ufp4.SCALE_E4M3_X_FP32, 2048, 256 * 1024, 64 * 256),
     (0, 16, ufp4.SCALE_FP32, 0, 0, 0),
+    (1000, 32, ufp4.SCALE_UE8M0, 1024, 256 * 512, 32 * 256),
 ])
 def test_layout(L, k, block, fmt, kpad, codes, scales):
     cfg = ufp4.QuantConfig(block=block, scale_fmt=fmt)
@@ -118,6 +119,8 @@ def test_gemm_validation_rejects_before_launch(L):
     assert _gemm(L, a, b, c_ptr=64 * 1024 + 2) == ufp4.ERR_ALIGNMENT
     assert _gemm(L, _q(k=256), _q(k=192)) == ufp4.ERR_OPERAND_MISMATCH
     assert _gemm(L, _q(scale_fmt=0), _q(scale_fmt=1)) == ufp4.ERR_OPERAND_MISMATCH
+    assert _gemm(L, _q(scale_fmt=2, block=32), _q(scale_fmt=0, block=32)) == ufp4.ERR_OPERAND_MISMATCH
+    assert _gemm(L, _q(scale_fmt=2, block=16), _q(scale_fmt=2, block=16)) == ufp4.ERR_INVALID_ARG  # MX: 32
     bad = _q()
     bad.kpad = 100
     assert _gemm(L, bad, _q()) == ufp4.ERR_INVALID_ARG

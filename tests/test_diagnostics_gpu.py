@@ -130,3 +130,12 @@ def test_sqnr_sums_match_oracle(rows, cols):
     want = dg.gemm_sqnr_sums(ref, test)
     assert got[0] == pytest.approx(want[0], rel=1e-12)
     assert got[1] == pytest.approx(want[1], rel=1e-12)
+
+
+@pytest.mark.parametrize("axis", AXES)
+@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1, ufp4.GRID_E2M1_MAX2])
+def test_quant_stats_ue8m0(axis, grid):
+    """Diagnostics of MX (UE8M0, block 32) operands against the oracle."""
+    X = wl.normal_with_outlier_channels(200, 136, 1.0, 3, 30.0)
+    cfg = ufp4.QuantConfig(grid=grid, hadamard_n=16, block=32, scale_fmt=ufp4.SCALE_UE8M0)
+    _run(X, axis, cfg)

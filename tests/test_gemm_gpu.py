@@ -209,3 +209,30 @@ def test_e2m1_reference_recipe_layer(fmt):
     qdyt, rdyt = _quant_both(dY, R, sr_rot)
     qxt, rxt = _quant_both(X, R, rot)
     _check_full(qdyt, rdyt, qxt, rxt, ufp4.gemm_wgrad)
+
+
+# ------------------------------------------------------------------ MX block scales
+@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1, ufp4.GRID_E2M1_MAX2])
+def test_ue8m0_gemms(grid):
+    """UE8M0 (MX, block 32) operands through the fp32-scale kernel: FPROP on
+    ragged shapes, and DGRAD / WGRAD of a small layer with SR on dY."""
+    for (M, N, K) in [(300, 200, 200), (129, 257, 136), (1, 1, 8)]:
+        X = wl.normal_with_outlier_channels(M, K, 1.0, 2, 20.0)
+        W = wl.normal(N, K, 0.02, 2)
+        cfg = _cfg(grid=grid, fmt=ufp4.SCALE_UE8M0, block=32)
+        qx, rx = _quant_both(X, C, cfg)
+        qw, rw = _quant_both(W, C, cfg)
+        _check_full(qx, rx, qw, rw, ufp4.gemm_fprop)
+    M, K, N = 384, 320, 264
+    X = wl.normal_with_outlier_channels(M, K, 1.0, 3, 30.0)
+    W = wl.normal(N, K, 0.02, 2)
+    dY = wl.normal(M, N, 1e-3, 3)
+    rt = _cfg(grid=grid, fmt=ufp4.SCALE_UE8M0, block=32)
+    sr0 = _cfg(grid=grid, fmt=ufp4.SCALE_UE8M0, block=32, rounding=1, stream=0)
+    sr1 = _cfg(grid=grid, fmt=ufp4.SCALE_UE8M0, block=32, rounding=1, stream=1)
+    qdy, rdy = _quant_both(dY, C, sr0)
+    qwt, rwt = _quant_both(W, R, rt)
+    _check_full(qdy, rdy, qwt, rwt, ufp4.gemm_dgrad)
+    qdyt, rdyt = _quant_both(dY, R, sr1)
+    qxt, rxt = _quant_both(X, R, rt)
+    _check_full(qdyt, rdyt, qxt, rxt, ufp4.gemm_wgrad)

@@ -196,3 +196,43 @@ def test_dual_quantize_full_size_sampled(shape):
     _run_dual(X, cfg, cfg.with_(sr_stream=1), rows_c=rc, rows_r=rr)
     cfg = ufp4.QuantConfig(hadamard_n=16, block=16)
     _run_dual(X, cfg, cfg, rows_c=rc, rows_r=rr)
+
+
+# ------------------------------------------------------------------ MX block scales
+@pytest.mark.parametrize("axis", AXES)
+@pytest.mark.parametrize("n", [0, 16, 64])
+@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1, ufp4.GRID_E2M1_MAX2])
+@pytest.mark.parametrize("rounding", [ufp4.ROUND_RTNE, ufp4.ROUND_SR])
+def test_quantize_ue8m0_matches_oracle(axis, n, grid, rounding):
+    """UE8M0 (MX) block scales, block 32: exponent bytes and codes bit-exact on
+    a 200 x 136 outlier tensor, ragged in rows and K."""
+    X = wl.normal_with_outlier_channels(200, 136, 1.0, 3, 30.0)
+    cfg = ufp4.QuantConfig(grid=grid, rounding=rounding, sr_seed=321, sr_stream=axis, hadamard_n=n,
+                           block=32, scale_fmt=ufp4.SCALE_UE8M0)
+    _run(X, axis, cfg)
+
+
+@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1, ufp4.GRID_E2M1_MAX2])
+def test_quantize_ue8m0_exponent_edges(grid):
+    """Block maxima exactly at gmax * 2^k, one ulp either side, tiny (clamped
+    at 2^-127), huge, and zero blocks, without RHT (n = 0) so the maxima are
+    the inputs themselves."""
+    gm = oracle.gmax(grid)
+    rng = np.random.default_rng(7)
+    rows = []
+    for k in range(-120, 120, 9):
+        tb = int(wl.bf16_bits(np.array([gm * 2.0 ** k], np.float32))[0])
+        for bb in (tb - 1, tb, tb + 1):             # the bf16 neighbours of gmax * 2^k
+            v = np.float32(wl.bf16_to_f32(np.array([bb], np.uint16))[0])
+            r = rng.uniform(-1, 1, 64).astype(np.float32) * v
+            r[5] = v
+            r[40] = -v
+            rows.append(r)
+    rows.append(np.full(64, 1e-40, np.float32))
+    rows.append(np.zeros(64, np.float32))
+    rows.append(np.full(64, 3.0e38, np.float32))
+    X = wl.bf16_bits(np.stack(rows))
+    for rounding in (ufp4.ROUND_RTNE, ufp4.ROUND_SR):
+        cfg = ufp4.QuantConfig(grid=grid, rounding=rounding, sr_seed=3, hadamard_n=0, block=32,
+                               scale_fmt=ufp4.SCALE_UE8M0)
+        _run(X, ufp4.ALONG_COLS, cfg)
