@@ -210,6 +210,38 @@ def quant_bytes(step: LayerStep) -> float:
     return total
 
 
+def run_mx(step: LayerStep, reps: int = 5) -> dict:
+    """The layer's FPROP with MX block scales (UE8M0, block 32): quantize X and
+    W (dual calls) and the GEMM through the fp32-block-scale kernel, timed
+    with CUDA events (reported, not in `value`)."""
+    u = step.u
+    cfg = u.QuantConfig(grid=u.GRID_E1M2, hadamard_n=16, block=32, scale_fmt=u.SCALE_UE8M0)
+    s = SHAPE
+    qx, qxt = u.rht_quantize_dual(step.X, cfg)
+    qw, qwt = u.rht_quantize_dual(step.W, cfg)
+    out = torch.empty((s.M, s.N), dtype=torch.float32, device=step.dev)
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize(step.dev)
+        return a.elapsed_time(b) / reps
+
+    t_q = timed(lambda: (u.rht_quantize_dual(step.X, cfg, out=(qx, qxt)),
+                         u.rht_quantize_dual(step.W, cfg, out=(qw, qwt))))
+    t_g = timed(lambda: u.gemm_fprop(qx, qw, out))
+    del out
+    return {"quantize_XW_dual_ms": round(t_q, 4), "fprop_ms": round(t_g, 4),
+            "fprop_TFLOPs": round(2 * s.M * s.N * s.K / (t_g * 1e-3) / 1e12, 1),
+            "kernel": "gemm_tn_kernel<0> (kind::f16 per-block partials, exponent-byte scales)"}
+
+
 def run_moe(device, two_level: bool, reps: int = 10):
     """The grouped (mixture-of-experts) GEMMs of one expert FFN: 16384 tokens,
     top-6 of 64 experts (Zipf(1.2) counts, segments padded to 64 rows), hidden
@@ -321,6 +353,7 @@ def run_device(args, rank, world, device):
     # ---- grouped (MoE) GEMMs of the mixture-of-experts config (reported, not in `value`)
     moe = run_moe(device, step.two)
     diag = run_diag(step)
+    mx = run_mx(step)
 
     value = world * flops / (ms_per_step * 1e-3) / 1e12
     gemm_tf = [2 * s.M * s.N * s.K / (g * 1e-3) / 1e12 for g in g_ms]
@@ -381,6 +414,7 @@ def run_device(args, rank, world, device):
         "e2e": e2e,
         "moe_grouped": moe,
         "diagnostics": diag,
+        "mx_block32": mx,
         "device_status": ufp4.status_string(status),
     }
     result["clocks"] = clk.summary()

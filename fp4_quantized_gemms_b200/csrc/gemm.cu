@@ -274,6 +274,12 @@ __device__ __forceinline__ __half2 e4m3_pair(uint32_t byte) {
 }
 
 // ---------------------------------------------------------------------------
+// 2^(E - 127) of a UE8M0 byte E <= 254: the byte is the fp32 exponent field
+// (E = 0 is the subnormal 2^-127).
+__device__ __forceinline__ float ue8m0_to_f32(uint32_t e) {
+    return __uint_as_float(e ? (e << 23) : 0x00400000u);
+}
+
 template <int MODE, int GRID>
 __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
     gemm_tn_kernel(const __grid_constant__ GemmArgs args) {
@@ -644,7 +650,7 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
                             break;
                         }
                         tc_fence_after();
-                        const float sa = ue8 ? ldexpf(1.0f, static_cast<int>(sa_u8[bi * BM + row_in_tile]) - 127)
+                        const float sa = ue8 ? ue8m0_to_f32(sa_u8[bi * BM + row_in_tile])
                                              : sa_tile[bi * BM + row_in_tile];
                         const float4 *sb4 = reinterpret_cast<const float4 *>(sb_tile + bi * BN + h * 64);
                         const uchar4 *sb4u = reinterpret_cast<const uchar4 *>(sb_u8 + bi * BN + h * 64);
@@ -664,10 +670,8 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
                                 float4 sb;
                                 if (ue8) {
                                     const uchar4 e = sb4u[8 * half + c4];
-                                    sb = make_float4(ldexpf(1.0f, static_cast<int>(e.x) - 127),
-                                                     ldexpf(1.0f, static_cast<int>(e.y) - 127),
-                                                     ldexpf(1.0f, static_cast<int>(e.z) - 127),
-                                                     ldexpf(1.0f, static_cast<int>(e.w) - 127));
+                                    sb = make_float4(ue8m0_to_f32(e.x), ue8m0_to_f32(e.y), ue8m0_to_f32(e.z),
+                                                     ue8m0_to_f32(e.w));
                                 } else {
                                     sb = sb4[8 * half + c4];
                                 }
