@@ -41,6 +41,22 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 L2_BYTES = 126 * 1024 * 1024
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of the ranks' values; every rank takes part (NCCL on the
+    GPU machine, any backend the process group was created with)."""
+    if world <= 1:
+        return x
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_per_step: float, ms_per_step: float) -> float:
+    """Whole-job throughput of `world` replicas each doing `flops_per_step` per
+    step, the step time being the slowest rank's."""
+    return world * flops_per_step / (ms_per_step * 1e-3) / 1e12
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -336,11 +352,7 @@ def run_device(args, rank, world, device):
         torch.cuda.synchronize(device)
     if world > 1:
         torch.distributed.barrier()
-    total_ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(start.elapsed_time(end), world, device)
     ms_per_step = total_ms / args.steps
     q_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps))
     g_ms = [statistics.mean(ev[i][1 + j].elapsed_time(ev[i][2 + j]) for i in range(args.steps))
@@ -355,7 +367,7 @@ def run_device(args, rank, world, device):
     diag = run_diag(step)
     mx = run_mx(step)
 
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    value = job_tflops(world, flops, ms_per_step)
     gemm_tf = [2 * s.M * s.N * s.K / (g * 1e-3) / 1e12 for g in g_ms]
     bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     if step.two:

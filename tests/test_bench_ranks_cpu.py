@@ -1,0 +1,61 @@
+"""Host-side logic of the multi-GPU bench on CPU: two `gloo` ranks take the
+max over ranks of their step times and report whole-job throughput; the
+reference arm runs on rank 0 only."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        local_ms = [12.5, 17.25][rank]            # the slower rank sets the step time
+        ms = bench.max_over_ranks(local_ms, world, torch.device("cpu"))
+        out[rank] = (ms, bench.job_tflops(world, 1e12, ms / 10))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_job_throughput_with_two_gloo_ranks():
+    world = 2
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True,
+                           start_method="spawn")
+        res = dict(out)
+    assert res[0][0] == res[1][0] == 17.25
+    # 2 replicas x 1e12 flop per step, 1.725 ms per step
+    assert res[0][1] == pytest.approx(2 * 1e12 / 1.725e-3 / 1e12)
+
+
+def test_single_rank_needs_no_process_group():
+    assert bench.max_over_ranks(3.0, 1, torch.device("cpu")) == 3.0
+    assert bench.job_tflops(1, 2e12, 2.0) == pytest.approx(1000.0)
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    """Under torchrun, a rank other than 0 of `--impl reference` exits 0
+    without work or output."""
+    import subprocess
+    import sys
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(os.path.dirname(bench.__file__), "bench.py"),
+                        "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == ""
