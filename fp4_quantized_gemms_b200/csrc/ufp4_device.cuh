@@ -217,42 +217,6 @@ __device__ __forceinline__ void tma_load_3d_hint(void *smem_dst, const CUtensorM
         : "memory");
 }
 
-// The same for a 3-D tensor map (x innermost).
-__device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *map,
-                                            uint64_t *bar, int32_t x, int32_t y, int32_t z) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_addr(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z)
-        : "memory");
-}
-
-// TMA 2-D tiled store from this CTA's shared memory (bulk async-group
-// completion); elements outside the tensor map are not written.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *smem_src, int32_t x,
-                                             int32_t y) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(smem_addr(smem_src)), "r"(x), "r"(y)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit_group() {
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Wait until at most N committed bulk groups still read their shared memory.
-template <int N>
-__device__ __forceinline__ void bulk_wait_group_read() {
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-
-// Wait until at most N committed bulk groups are incomplete (writes done).
-template <int N>
-__device__ __forceinline__ void bulk_wait_group() {
-    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
-}
-
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -370,31 +334,6 @@ __device__ __forceinline__ void umma_fp4_bs_pair(uint32_t d_tmem, uint64_t adesc
         : "memory");
 }
 
-// Shared memory -> TMEM copy of a 32 x 128-bit block (one scale-factor atom of
-// 128 rows x 4 scales), replicated to the four 32-lane groups.
-__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-                 : "memory");
-}
-
-// The same copy issued by CTA 0 of a CTA pair: each CTA copies the block at
-// this shared-memory offset into its own TMEM.
-__device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-                 : "memory");
-}
-
-// Descriptor of a 512-byte scale-factor atom in shared memory: 32 rows of 16
-// bytes, no swizzle (8-row core matrices, 128 bytes apart).
-__device__ __forceinline__ uint64_t sf_atom_desc(uint32_t smem_byte_addr) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>(128u >> 4) << 16;
-    d |= static_cast<uint64_t>(128u >> 4) << 32;
-    d |= static_cast<uint64_t>(1u) << 46;
-    return d;
-}
-
 // K-major operand in the 64-byte swizzle layout: rows of 64 bytes, 8-row
 // atoms of 512 bytes (stride byte offset 512), layout type 4 = SWIZZLE_64B.
 __device__ __forceinline__ uint64_t umma_desc_sw64(uint32_t smem_byte_addr) {
@@ -494,12 +433,6 @@ __host__ __device__ constexpr uint32_t umma_idesc_f16_f32(int M, int N) {
            | (0u << 7) | (0u << 10)                   // A, B: f16
            | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
            | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
-}
-
-// Byte offset of the 16-byte chunk `chunk` (0..7) of row `row` inside a tile
-// stored with the 128-byte swizzle (tile base 1024-byte aligned).
-__device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
-    return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
 
 // ---------------------------------------------------------------------------
