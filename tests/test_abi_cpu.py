@@ -240,3 +240,22 @@ def test_diagnostics_validation_rejects_before_launch(L):
     assert Q(x, 100, x, 128, 4, 128, st, None) == ufp4.ERR_INVALID_ARG
     assert Q(None, 128, x, 128, 4, 128, st, None) == ufp4.ERR_INVALID_ARG
     assert Q(x, 128, x, 128, -1, 128, st, None) == ufp4.ERR_INVALID_ARG
+
+
+def test_product_path_fails_loudly_without_the_library_or_cuda(tmp_path):
+    """No CPU fallback: a missing library raises on first use, and CPU tensors
+    are refused before any call."""
+    import sys
+    code = ("import sys; sys.path.insert(0, %r)\n"
+            "from fp4_quantized_gemms_b200 import ufp4\n"
+            "ufp4.LIB_PATH = %r\n"
+            "try:\n    ufp4.lib()\nexcept RuntimeError as e:\n    print('raised', 'missing' in str(e))\n"
+            % (ROOT, str(tmp_path / "absent.so")))
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120)
+    assert r.stdout.strip() == "raised True", r.stderr
+    import torch
+    x = torch.zeros((16, 64), dtype=torch.bfloat16)
+    with pytest.raises(RuntimeError, match="CUDA"):
+        ufp4.rht_quantize(x, ufp4.ALONG_COLS, ufp4.QuantConfig())
+    with pytest.raises(RuntimeError, match="CUDA"):
+        ufp4.rht_quantize_dual(x, ufp4.QuantConfig())
