@@ -259,3 +259,24 @@ def test_product_path_fails_loudly_without_the_library_or_cuda(tmp_path):
         ufp4.rht_quantize(x, ufp4.ALONG_COLS, ufp4.QuantConfig())
     with pytest.raises(RuntimeError, match="CUDA"):
         ufp4.rht_quantize_dual(x, ufp4.QuantConfig())
+
+
+@pytest.mark.parametrize("grid,fmt,block", [
+    (ufp4.GRID_E1M2, ufp4.SCALE_FP32, 16), (ufp4.GRID_E1M2, ufp4.SCALE_E4M3_X_FP32, 16),
+    (ufp4.GRID_E2M1, ufp4.SCALE_E4M3_X_FP32, 32), (ufp4.GRID_E2M1_MAX2, ufp4.SCALE_UE8M0, 32),
+    (ufp4.GRID_E1M2, ufp4.SCALE_UE8M0, 32),
+])
+def test_binding_allocates_what_the_layout_call_sizes(grid, fmt, block):
+    """empty_qtensor (host tensors here) matches ufp4_qtensor_layout: codes,
+    block-major scales of the format's element size, the E1M2 correction plane
+    for two-level operands only, a tensor scale for two-level only."""
+    cfg = ufp4.QuantConfig(grid=grid, block=block, scale_fmt=fmt)
+    kpad, sld, cbytes, sbytes = ufp4.layout(300, 200, cfg)
+    q = ufp4.empty_qtensor(300, 200, cfg, device="cpu")
+    assert q.codes.numel() == cbytes and q.scales.numel() * q.scales.element_size() == sbytes
+    assert q.scales.shape == (kpad // block, sld) and sld % 64 == 0 and sld >= 300
+    assert (q.corr is not None) == (grid == ufp4.GRID_E1M2 and fmt == ufp4.SCALE_E4M3_X_FP32)
+    assert (q.tensor_scale is not None) == (fmt == ufp4.SCALE_E4M3_X_FP32)
+    c = q.c()
+    assert c.rows == 300 and c.k == 200 and c.kpad == kpad and c.scale_ld == sld
+    assert c.cfg.scale_fmt == fmt and c.cfg.block == block and c.cfg.grid == grid
