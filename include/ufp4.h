@@ -18,6 +18,11 @@
  *      over the dequantized operands, fp32 accumulation, fp32 output.
  *   3. ufp4_grouped_gemm: the same contraction for a table of independent
  *      sub-problems (mixture-of-experts layers).
+ *   4. ufp4_rht_quantize_dual / ufp4_rht_amax_dual: both quantizations (both
+ *      rotated amaxes) of one tensor from a single read of it.
+ *   5. ufp4_quant_stats / ufp4_qstats_summarize / ufp4_sqnr_sums: the
+ *      quantization diagnostics of [PL] §5 and Appendix A (SQNR, level error,
+ *      code occupancy, underflow).
  *
  * Conventions shared by every call:
  *   - All pointers named *_dev, and every pointer inside ufp4_qtensor_t, are
