@@ -5,6 +5,8 @@ the launch to capture.
 
     python -m fp4_quantized_gemms_b200.profile_cases gemm --m 4096 --n 4096 --k 2048 --grid e1m2
     python -m fp4_quantized_gemms_b200.profile_cases quantize --rows 8192 --cols 8192 --axis rows --sr
+    python -m fp4_quantized_gemms_b200.profile_cases quantize --rows 8192 --cols 2048 --dual
+    python -m fp4_quantized_gemms_b200.profile_cases stats --rows 8192 --cols 8192 --axis rows
 """
 from __future__ import annotations
 
@@ -36,15 +38,33 @@ def gemm_case(m: int, n: int, k: int, grid: int, path: int) -> None:
         raise RuntimeError("device error word set")
 
 
-def quantize_case(rows: int, cols: int, axis: int, sr: bool, two_level: bool) -> None:
-    """Rotated amax + quantize of one bf16 operand, twice."""
+def quantize_case(rows: int, cols: int, axis: int, sr: bool, two_level: bool, dual: bool = False) -> None:
+    """Rotated amax + quantize of one bf16 operand, twice (with `dual`: both
+    layouts from one read, through the dual-output kernel)."""
     fmt = ufp4.SCALE_E4M3_X_FP32 if two_level else ufp4.SCALE_FP32
     cfg = ufp4.QuantConfig(grid=ufp4.GRID_E1M2, rounding=ufp4.ROUND_SR if sr else ufp4.ROUND_RTNE,
                            sr_seed=1234, hadamard_n=16, block=16, scale_fmt=fmt)
     x = _dev(wl.normal(rows, cols, 1e-3, 3))
     q = None
     for _ in range(2):
-        q = ufp4.rht_quantize(x, axis, cfg, out=q)
+        if dual:
+            q = ufp4.rht_quantize_dual(x, cfg, cfg.with_(sr_stream=1), out=q)
+        else:
+            q = ufp4.rht_quantize(x, axis, cfg, out=q)
+    torch.cuda.synchronize()
+    if ufp4.check_device_status() != ufp4.OK:
+        raise RuntimeError("device error word set")
+
+
+def stats_case(rows: int, cols: int, axis: int) -> None:
+    """Quantize once, then the diagnostics kernel on the operand, twice."""
+    cfg = ufp4.QuantConfig(grid=ufp4.GRID_E1M2, hadamard_n=16, block=16,
+                           scale_fmt=ufp4.SCALE_E4M3_X_FP32)
+    x = _dev(wl.normal(rows, cols, 1e-3, 3))
+    q = ufp4.rht_quantize(x, axis, cfg)
+    buf = None
+    for _ in range(2):
+        buf = ufp4.quant_stats_launch(x, axis, q, out=buf)
     torch.cuda.synchronize()
     if ufp4.check_device_status() != ufp4.OK:
         raise RuntimeError("device error word set")
@@ -65,12 +85,19 @@ def main() -> None:
     q.add_argument("--axis", choices=["cols", "rows"], default="cols")
     q.add_argument("--sr", action="store_true")
     q.add_argument("--fp32-scales", action="store_true")
+    q.add_argument("--dual", action="store_true")
+    t = sub.add_parser("stats")
+    t.add_argument("--rows", type=int, default=8192)
+    t.add_argument("--cols", type=int, default=8192)
+    t.add_argument("--axis", choices=["cols", "rows"], default="rows")
     a = ap.parse_args()
     if a.case == "gemm":
         gemm_case(a.m, a.n, a.k, ufp4.GRID_E1M2 if a.grid == "e1m2" else ufp4.GRID_E2M1, a.path)
+    elif a.case == "stats":
+        stats_case(a.rows, a.cols, ufp4.ALONG_COLS if a.axis == "cols" else ufp4.ALONG_ROWS)
     else:
         quantize_case(a.rows, a.cols, ufp4.ALONG_COLS if a.axis == "cols" else ufp4.ALONG_ROWS,
-                      a.sr, not a.fp32_scales)
+                      a.sr, not a.fp32_scales, a.dual)
     print("ok")
 
 
