@@ -520,67 +520,86 @@ def run_e2e(step: LayerStep, args, device):
 
 
 # ------------------------------------------------------------------ oracle arm
-def oracle_sample_step(rng, n_rows=8, n_cols=8):
-    """A bounded sample of one step on the host cores: the oracle quantizes
-    n_rows / n_cols output rows of every operand (full reduction length) and
-    contracts the n_rows x n_cols sampled block of each GEMM.  Returns
-    (effective GEMM flops of the sampled entries, seconds)."""
-    import oracle
-    s = SHAPE
-    X, W, dY = wl.layer_inputs(s)
-    rt = oracle.QuantCfg(grid=0, hadamard_n=16, block=16, sign_mask=0x09F1FD9D03F0A9B4)
-    sr0 = oracle.QuantCfg(grid=0, rounding=1, sr_seed=SR_SEED, sr_stream=0, hadamard_n=16,
-                          block=16, sign_mask=0x09F1FD9D03F0A9B4)
-    sr1 = oracle.QuantCfg(grid=0, rounding=1, sr_seed=SR_SEED, sr_stream=1, hadamard_n=16,
-                          block=16, sign_mask=0x09F1FD9D03F0A9B4)
-    gemms = [((X, 0, rt, s.M), (W, 0, rt, s.N), s.K),
-             ((dY, 0, sr0, s.M), (W, 1, rt, s.K), s.N),
-             ((dY, 1, sr1, s.N), (X, 1, rt, s.K), s.M)]
-    flops = 0.0
-    t0 = time.perf_counter()
-    for (a_bits, a_ax, a_cfg, a_rows), (b_bits, b_ax, b_cfg, b_rows), K in gemms:
-        ia = rng.choice(a_rows, n_rows, replace=False)
-        jb = rng.choice(b_rows, n_cols, replace=False)
-        qa = [oracle.quantize(a_bits, a_ax, a_cfg, r0=int(r), nr=1) for r in ia]
-        qb = [oracle.quantize(b_bits, b_ax, b_cfg, r0=int(r), nr=1) for r in jb]
-        A = np.concatenate([q.dequantize() for q in qa])
-        B = np.concatenate([q.dequantize() for q in qb])
-        out = np.empty(n_rows * n_cols)
-        ii = np.repeat(np.arange(n_rows), n_cols)
-        jj = np.tile(np.arange(n_cols), n_rows)
-        qa[0].codes = np.concatenate([q.codes for q in qa])
-        qa[0].scales = np.concatenate([q.scales for q in qa])
-        qb[0].codes = np.concatenate([q.codes for q in qb])
-        qb[0].scales = np.concatenate([q.scales for q in qb])
-        out = oracle.gemm_tn_entries(qa[0], qb[0], ii, jj)
-        flops += 2.0 * K * out.size
-        del A, B
-    return flops, time.perf_counter() - t0
+class OracleSample:
+    """Bounded samples of one step on the host cores, in the configuration the
+    GPU arm runs (`scale`): the oracle quantizes sampled output rows of every
+    operand (full reduction length) and contracts the sampled block of each
+    GEMM.  Inputs and, with two-level scales, the six rotated tensor amaxes
+    are prepared once, outside any timed region."""
+
+    MASK = 0x09F1FD9D03F0A9B4       # the binding's default D sign mask
+
+    def __init__(self, scale: str):
+        import oracle
+        self.oracle = oracle
+        oracle.build()
+        self.X, self.W, self.dY = wl.layer_inputs(SHAPE)
+        self.two = scale == "two-level"
+        fmt = oracle.SCALE_E4M3_X_FP32 if self.two else oracle.SCALE_FP32
+        base = dict(grid=0, hadamard_n=16, block=16, sign_mask=self.MASK, scale_fmt=fmt)
+        self.rt = oracle.QuantCfg(**base)
+        self.sr0 = oracle.QuantCfg(rounding=1, sr_seed=SR_SEED, sr_stream=0, **base)
+        self.sr1 = oracle.QuantCfg(rounding=1, sr_seed=SR_SEED, sr_stream=1, **base)
+        self.amax = {}
+        for name, bits in (("X", self.X), ("W", self.W), ("dY", self.dY)):
+            for ax in (0, 1):
+                self.amax[name, ax] = oracle.rht_amax(bits, ax, 16, self.MASK) if self.two else 0.0
+
+    def step(self, rng, n_rows=8, n_cols=8):
+        """One sampled step; returns (GEMM flops of the sampled entries, seconds)."""
+        oracle = self.oracle
+        s = SHAPE
+        gemms = [(("X", 0, self.rt, s.M), ("W", 0, self.rt, s.N), s.K),
+                 (("dY", 0, self.sr0, s.M), ("W", 1, self.rt, s.K), s.N),
+                 (("dY", 1, self.sr1, s.N), ("X", 1, self.rt, s.K), s.M)]
+        bits = {"X": self.X, "W": self.W, "dY": self.dY}
+
+        def rows_q(name, ax, cfg, picks):
+            parts = [oracle.quantize(bits[name], ax, cfg, tensor_amax=self.amax[name, ax], r0=int(r), nr=1)
+                     for r in picks]
+            q = parts[0]
+            q.codes = np.concatenate([p.codes for p in parts])
+            if q.scales is not None:
+                q.scales = np.concatenate([p.scales for p in parts])
+            else:
+                q.escales = np.concatenate([p.escales for p in parts])
+            return q
+
+        flops = 0.0
+        t0 = time.perf_counter()
+        for (an, aax, acfg, arows), (bn, bax, bcfg, brows), K in gemms:
+            qa = rows_q(an, aax, acfg, rng.choice(arows, n_rows, replace=False))
+            qb = rows_q(bn, bax, bcfg, rng.choice(brows, n_cols, replace=False))
+            ii = np.repeat(np.arange(n_rows), n_cols)
+            jj = np.tile(np.arange(n_cols), n_rows)
+            out = oracle.gemm_tn_entries(qa, qb, ii, jj)
+            flops += 2.0 * K * out.size
+        return flops, time.perf_counter() - t0
 
 
 def run_reference(args, world):
-    import oracle
-    oracle.build()
+    smp = OracleSample(args.scale)       # inputs and tensor amaxes outside the timed region
     rng = np.random.default_rng(0)
-    wl.layer_inputs(SHAPE)   # generate inputs outside the timed region
     for _ in range(args.warmup):
-        oracle_sample_step(rng)
+        smp.step(rng)
     times, flops = [], 0.0
     for _ in range(args.steps):
-        f, t = oracle_sample_step(rng)
+        f, t = smp.step(rng)
         times.append(t)
         flops += f
     total = sum(times)
     value = flops / total / 1e12
-    cores = oracle.num_threads()
+    cores = smp.oracle.num_threads()
     sample = ("per step: 8 sampled output rows of each of the 6 quantized operands "
-              "(full reduction length) and the 8x8 sampled block of each GEMM")
+              "(full reduction length) and the 8x8 sampled block of each GEMM"
+              + ("; the rotated tensor amaxes are computed once before the timed steps"
+                 if smp.two else ""))
     res = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64 oracle (fp32 RHT, exact rounding decisions)", "data": "synthetic",
-        "config": {**workload_desc("fp32"), "parallelism": "host cores"},
+        "config": {**workload_desc(args.scale), "parallelism": "host cores"},
         "impl": "reference",
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
@@ -590,23 +609,24 @@ def run_reference(args, world):
     return res
 
 
-def cpu_baseline_quick():
-    """The oracle as it stands, on a bounded sample of the workload (rank 0)."""
-    import oracle
-    oracle.build()
+def cpu_baseline_quick(scale: str = "two-level"):
+    """The oracle as it stands, on a bounded sample of the workload (rank 0),
+    in the GPU arm's scale configuration."""
+    smp = OracleSample(scale)
     rng = np.random.default_rng(1)
-    oracle_sample_step(rng, 4, 4)       # warm caches / page in
+    smp.step(rng, 4, 4)                 # warm caches / page in
     flops, secs = 0.0, 0.0
     n = 0
     while secs < 10.0 and n < 200:
-        f, t = oracle_sample_step(rng, 32, 32)
+        f, t = smp.step(rng, 32, 32)
         flops += f
         secs += t
         n += 1
-    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": smp.oracle.num_threads(),
             "kind": "oracle",
             "sample": (f"{n} sampled steps: 32 output rows of each of the 6 quantized operands "
-                       f"(full K) and a 32x32 block of each GEMM, {secs:.1f} s of CPU work")}
+                       f"(full K) and a 32x32 block of each GEMM, {secs:.1f} s of CPU work"
+                       + ("; tensor amaxes computed before timing" if smp.two else ""))}
 
 
 def main():
@@ -640,7 +660,7 @@ def main():
     res = run_device(args, rank, world, device)
     if rank == 0:
         if not args.no_cpu_baseline:
-            res["cpu_baseline"] = cpu_baseline_quick()
+            res["cpu_baseline"] = cpu_baseline_quick(args.scale)
         print(json.dumps(res), flush=True)
     if world > 1:
         torch.distributed.barrier()
