@@ -278,8 +278,8 @@ ufp4_status_t ufp4_grouped_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b
  *                             256 x 192 tiles);
  *   UFP4_GEMM_PATH_AUTO       the library's choice (default; currently the
  *                             one-CTA native FP4 path).
- * The setting is process-wide and read at each GEMM call; fp32 block scales
- * are unaffected.  Errors: INVALID_ARG for an unknown path. */
+ * The setting is process-wide and read at each GEMM call; fp32 and UE8M0
+ * block scales are unaffected (they always run the fp32-scale kernel).  Errors: INVALID_ARG for an unknown path. */
 typedef enum {
     UFP4_GEMM_PATH_AUTO = 0,
     UFP4_GEMM_PATH_FP16 = 1,
