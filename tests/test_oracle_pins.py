@@ -489,3 +489,125 @@ def test_ue8m0_quantize_structure(grid, rounding):
         assert np.all(np.abs(deq - u) <= half * step * (1 + 1e-12))
     with pytest.raises(ValueError):
         oracle.quantize(X, oracle.ALONG_COLS, _cfg(grid=grid, block=16, scale_fmt=oracle.SCALE_UE8M0))
+
+
+# ------------------------------------------------------------------ rotated amax and the row-wise view
+def _rotated_f64(X_bits: np.ndarray, axis: int, n: int, mask: int) -> np.ndarray:
+    """u = H_n D x of every row of the operand's K-major view, computed
+    independently of the oracle: scipy's Sylvester matrix times the sign-
+    flipped block, in fp64, with K zero-padded to a multiple of 64."""
+    x = wl.bf16_to_f32(X_bits).astype(np.float64)
+    if axis == oracle.ALONG_ROWS:
+        x = x.T
+    rows, K = x.shape
+    kp = (K + 63) // 64 * 64
+    v = np.zeros((rows, kp))
+    v[:, :K] = x
+    if n == 0:
+        return v
+    d = np.array([-1.0 if (mask >> i) & 1 else 1.0 for i in range(n)])
+    H = scipy.linalg.hadamard(n).astype(np.float64)
+    blocks = v.reshape(rows, kp // n, n) * d
+    return (blocks @ H.T).reshape(rows, kp)
+
+
+@pytest.mark.parametrize("n", [0, 16, 32, 64])
+@pytest.mark.parametrize("axis", [oracle.ALONG_COLS, oracle.ALONG_ROWS])
+def test_rht_amax_matches_independent_hadamard(n, axis):
+    """The oracle's rotated tensor amax equals max |H_n D x| from scipy's
+    Hadamard matrix in fp64, to the fp32 butterflies' error bound, on a
+    non-square tensor with outlier channels (there the rotated amax differs
+    from the raw amax and from the other axis's, so an amax taken before the
+    rotation, along the wrong axis or over part of the blocks fails)."""
+    mask = 0x09F1FD9D03F0A9B4
+    X = wl.normal_with_outlier_channels(72, 136, 1.0, 3, 30.0)
+    got = oracle.rht_amax(X, axis, n, mask)
+    u = _rotated_f64(X, axis, n, mask)
+    want = np.abs(u).max()
+    x = wl.bf16_to_f32(X).astype(np.float64)
+    xa = np.abs(x.T if axis == oracle.ALONG_ROWS else x)
+    # |fp32 butterflies - exact| <= n 2^-24 sum|x| over the block (see the
+    # fp32 FWHT pin above); the largest block sum bounds every block
+    kp = u.shape[1]
+    pad = np.zeros((xa.shape[0], kp))
+    pad[:, :xa.shape[1]] = xa
+    bsum = pad.reshape(pad.shape[0], -1, max(n, 1)).sum(axis=2).max() if n else 0.0
+    assert abs(got - want) <= n * 2.0 ** -24 * bsum
+    if n == 0:
+        assert got == np.float32(np.abs(x).max())
+    else:
+        raw = np.abs(x).max()
+        other = np.abs(_rotated_f64(X, 1 - axis, n, mask)).max()
+        margin = n * 2.0 ** -24 * bsum
+        assert abs(want - raw) > 10 * margin and abs(want - other) > 10 * margin
+
+
+@pytest.mark.parametrize("grid", ALL_GRIDS)
+@pytest.mark.parametrize("rounding", [oracle.ROUND_RTNE, oracle.ROUND_SR])
+@pytest.mark.parametrize("scale_fmt", [oracle.SCALE_FP32, oracle.SCALE_E4M3_X_FP32, oracle.SCALE_UE8M0])
+def test_quantize_along_rows_is_transpose_of_along_cols(grid, rounding, scale_fmt):
+    """Quantizing X along its rows (the strided dimension, output transposed)
+    gives exactly what quantizing the explicit transpose along its columns
+    gives: codes, scales, tensor scale and the SR draws (both index the draws
+    by output row and column).  With a non-square X whose row count is not a
+    multiple of 64, a mix-up of row pitch and row count, a missing transpose or
+    a draw index taken from the input layout fails this."""
+    X = wl.normal_with_outlier_channels(100, 72, 1.0, 3, 25.0)
+    XT = np.ascontiguousarray(X.T)
+    block = 32 if scale_fmt == oracle.SCALE_UE8M0 else 16
+    cfg = _cfg(grid=grid, rounding=rounding, sr_seed=1234, sr_stream=1, hadamard_n=16,
+               sign_mask=0x09F1FD9D03F0A9B4, block=block, scale_fmt=scale_fmt)
+    am_r = oracle.rht_amax(X, oracle.ALONG_ROWS, 16, cfg.sign_mask)
+    am_c = oracle.rht_amax(XT, oracle.ALONG_COLS, 16, cfg.sign_mask)
+    assert am_r == am_c
+    a, ua = oracle.quantize(X, oracle.ALONG_ROWS, cfg, tensor_amax=am_r, want_u=True)
+    b, ub = oracle.quantize(XT, oracle.ALONG_COLS, cfg, tensor_amax=am_c, want_u=True)
+    assert a.k == b.k == 100 and a.kpad == b.kpad == 128 and a.codes.shape == (72, 128)
+    assert np.array_equal(ua, ub)
+    assert np.array_equal(a.codes, b.codes)
+    if scale_fmt == oracle.SCALE_FP32:
+        assert np.array_equal(a.scales, b.scales)
+    else:
+        assert np.array_equal(a.escales, b.escales)
+    assert a.S == b.S
+    # the transposed view really is the other axis: quantizing X along its
+    # columns gives a different operand
+    c = oracle.quantize(X, oracle.ALONG_COLS, cfg,
+                        tensor_amax=oracle.rht_amax(X, oracle.ALONG_COLS, 16, cfg.sign_mask))
+    assert c.codes.shape == (100, 128)
+
+
+@pytest.mark.parametrize("grid", ALL_GRIDS)
+@pytest.mark.parametrize("scale_fmt", [oracle.SCALE_FP32, oracle.SCALE_E4M3_X_FP32])
+def test_quantized_backward_gemms_track_bf16_gemms(grid, scale_fmt):
+    """End to end for the two backward GEMMs, with the recipe's operands:
+    DGRAD dX = dY W from dY along its columns (SR, stream 0) and W along its
+    rows; WGRAD dW = dY^T X from dY (SR, stream 1) and X both along their rows.
+    Each approximates the fp64 product of the bf16 inputs to 4-bit accuracy; a
+    transposed operand, a row-wise read along the wrong axis or a missing 1/n
+    is off by orders of magnitude."""
+    M, K, N = 128, 96, 80
+    X = wl.normal_with_outlier_channels(M, K, 1.0, 3, 20.0)
+    W = wl.normal(N, K, 0.02, 2)
+    dY = wl.normal(M, N, 1e-3, 3)
+    mask = 0x5EED
+    base = dict(grid=grid, hadamard_n=16, sign_mask=mask, block=16, scale_fmt=scale_fmt)
+    rt = _cfg(**base)
+    sr0 = _cfg(rounding=oracle.ROUND_SR, sr_seed=1234, sr_stream=0, **base)
+    sr1 = _cfg(rounding=oracle.ROUND_SR, sr_seed=1234, sr_stream=1, **base)
+    C, R = oracle.ALONG_COLS, oracle.ALONG_ROWS
+
+    def q(bits, axis, cfg):
+        return oracle.quantize(bits, axis, cfg, tensor_amax=oracle.rht_amax(bits, axis, 16, mask))
+
+    f = lambda b: wl.bf16_to_f32(b).astype(np.float64)  # noqa: E731
+    dX = oracle.gemm_tn(q(dY, C, sr0), q(W, R, rt))
+    dW = oracle.gemm_tn(q(dY, R, sr1), q(X, R, rt))
+    ref_dX = f(dY) @ f(W)
+    ref_dW = f(dY).T @ f(X)
+    assert dX.shape == ref_dX.shape == (M, K) and dW.shape == ref_dW.shape == (N, K)
+    # measured 0.14-0.17 (E1M2, E2M1) and 0.25-0.26 for the 5-level restricted grid
+    bound = 0.35 if grid == MAX2 else 0.22
+    for got, ref in ((dX, ref_dX), (dW, ref_dW)):
+        rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+        assert rel < bound, rel

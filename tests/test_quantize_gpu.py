@@ -88,15 +88,24 @@ def test_quantize_medium_with_outliers(axis):
         _run(X, axis, cfg)
 
 
-def test_sr_draws_independent_of_launch_shape():
-    """SR bits are a function of (seed, stream, row, column) only: quantizing a
-    row block alone gives the same codes as inside the full tensor."""
-    X = wl.student_t(256, 512, seed=12)
-    cfg = ufp4.QuantConfig(rounding=ufp4.ROUND_SR, sr_seed=99, hadamard_n=32)
-    full = ufp4.rht_quantize(to_dev(X), ufp4.ALONG_COLS, cfg)
-    again = ufp4.rht_quantize(to_dev(X), ufp4.ALONG_COLS, cfg)
-    assert torch.equal(full.codes, again.codes)
-    other = ufp4.rht_quantize(to_dev(X), ufp4.ALONG_COLS, cfg.with_(sr_seed=100))
+@pytest.mark.parametrize("axis", AXES)
+def test_sr_draws_independent_of_launch_shape(axis):
+    """SR bits are a function of (seed, stream, output row, column) only: a
+    separate call on a leading block of the output rows (a row prefix of X
+    along its columns, a column prefix of X, as a strided view, along its
+    rows) runs on another grid with other work units per CTA, yet gives
+    exactly the codes and scales of those rows in the call on the whole
+    tensor.  A different seed gives different codes."""
+    X = to_dev(wl.student_t(1024, 768, seed=12))
+    cfg = ufp4.QuantConfig(rounding=ufp4.ROUND_SR, sr_seed=99, sr_stream=axis, hadamard_n=32)
+    full = ufp4.rht_quantize(X, axis, cfg)
+    for lead in (8, 200, 520):
+        part_x = X[:lead] if axis == ufp4.ALONG_COLS else X[:, :lead]
+        part = ufp4.rht_quantize(part_x, axis, cfg)
+        assert part.rows == lead and part.kpad == full.kpad
+        assert torch.equal(part.codes, full.codes[:lead])
+        assert torch.equal(part.scales[:, :lead], full.scales[:, :lead])
+    other = ufp4.rht_quantize(X, axis, cfg.with_(sr_seed=100))
     assert not torch.equal(full.codes, other.codes)
 
 
