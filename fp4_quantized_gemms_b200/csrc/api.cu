@@ -396,6 +396,32 @@ ufp4_status_t ufp4_rht_amax(const void *x_dev, int64_t rows, int64_t cols, int64
     return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
 }
 
+ufp4_status_t ufp4_rht_bf16(const void *x_dev, int64_t rows, int64_t cols, int64_t ld, int32_t hadamard_n,
+                            uint64_t rht_sign_mask, void *y_dev, int64_t ldy, void *stream) {
+    ufp4_status_t s = check_input(x_dev, rows, cols, ld, UFP4_ALONG_COLS);
+    if (s != UFP4_OK) return s;
+    if (!(hadamard_n == 0 || hadamard_n == 16 || hadamard_n == 32 || hadamard_n == 64))
+        return UFP4_ERR_UNSUPPORTED;
+    if (cols % 64 != 0) return UFP4_ERR_UNSUPPORTED;
+    if (rows > 0 && cols > 0) {
+        if (y_dev == nullptr) return UFP4_ERR_INVALID_ARG;
+        if (ldy < cols) return UFP4_ERR_INVALID_ARG;
+        if (!aligned16(y_dev) || ldy % 8 != 0) return UFP4_ERR_ALIGNMENT;
+        if ((ld % 8) != 0) return UFP4_ERR_ALIGNMENT;
+    }
+    if (rows == 0 || cols == 0) return UFP4_OK;
+    QuantArgs a;
+    memset(&a, 0, sizeof(a));
+    a.x = static_cast<const uint16_t *>(x_dev);
+    a.rows = rows;
+    a.cols = cols;
+    a.ld = ld;
+    a.sign_mask = rht_sign_mask;
+    cudaError_t e = launch_rht_bf16(a, hadamard_n, static_cast<uint16_t *>(y_dev), ldy, sm_count(),
+                                    static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
+}
+
 ufp4_status_t ufp4_rht_quantize(const void *x_dev, int64_t rows, int64_t cols, int64_t ld,
                                 int32_t axis, const float *tensor_amax_dev, ufp4_qtensor_t *out,
                                 void *stream) {

@@ -5,22 +5,28 @@
 // transforms", "Blockwise quantization", "Rounding rules"; §4 UFP4 recipe;
 // gist.science "Efficiëntie" (RHT fused with the quantizer).
 //
-// Work decomposition.  A warp owns a 64-long segment of the reduction
-// dimension K for 8 output rows (row-wise, K contiguous) or for 64 output rows
-// (column-wise, K strided: the operand is transposed on the fly).  Inside a
-// warp, lane = 4*g + j: j picks the 16-element chunk [16j, 16j+16) of the
-// segment, so a 32- or 64-point Hadamard block spans lanes j^1 / j^2 and is
-// finished with shuffles.  Every lane holds whole 16-element chunks in
-// registers: loads are 16-byte vectors, coalesced along K (row-wise) or along
-// the contiguous input columns (column-wise), the "transpose" is free because
-// each bf16 is widened to fp32 individually anyway.
+// Work decomposition.  A persistent CTA (8 compute warps + one TMA producer
+// warp) takes units of 256 output rows x 64 K elements whose bf16 tile a TMA
+// copy stages in shared memory (128-byte swizzle, 3-stage ring).  Every
+// compute thread quantizes 64 elements of a unit as 32 "entries", each a pair
+// of fp32 values held as the two lanes of an fp32x2 register: lane x and lane
+// y are two 32-long runs along K that share their D signs position by
+// position, so the butterflies, the rounding estimate and the packing run two
+// elements per instruction:
+//   row map   (K contiguous)  one output row, K [0, 32) in x, [32, 64) in y;
+//   col2 map  (K strided, n <= 32)  two adjacent output rows (input columns
+//             c, c + 1: one 32-bit shared load gives both), 32 K each;
+//   col1 map  (K strided, n = 64)  one output row, K [0, 32) in x, [32, 64) in y.
 //
 // Exactness.  The butterflies are the same fp32 adds in the same stage order
-// as the definition; every rounding decision compares |u| with
-// (threshold * m1) * b by one fma, whose sign is exact (threshold * m1 is an
-// exact fp32 value, b the fp32 scale), so codes match the exact-quotient rule
-// bit for bit.  An fp32 estimate picks the candidate; the fma tests fix it.
+// as the definition.  Codes come from an fp32 estimate of u / s that is
+// certified: every decision whose estimate lies within 2^-16 grid steps of a
+// boundary (and every block whose step is subnormal or could saturate) sends
+// the thread's 64 elements to the exact path, which decides each element by
+// fma sign tests against exact thresholds, so codes always equal the
+// exact-quotient rule bit for bit.
 
+#include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -33,7 +39,6 @@ namespace ufp4 {
 
 namespace {
 
-constexpr int kThreads = 256;
 
 // Grids: 0 = E1M2 (levels k/4, k <= 7), 1 = E2M1 (OCP FP4 magnitudes),
 // 2 = E2M1 restricted to max_fpx = 2.0 (the E2M1 codes 0..4, levels k/2).
@@ -213,8 +218,10 @@ __device__ __forceinline__ uint32_t canonical_zero(uint32_t w) {
 constexpr float kRound = 12582912.0f;
 // A candidate closer than this (in units of the grid step) to a decision
 // boundary is re-decided by the exact path.  The estimate's error is below
-// 2^-20 steps (two roundings of a quotient below 8).
-constexpr float kMargin = 1.0f / 65536.0f;
+// 2^-19 steps: a quotient below 8 with a relative error under 2^-22 (the
+// reciprocal's ulp, the product's rounding, and for two-level scales the
+// rounding of e_b * S).
+constexpr float kMargin = 1.0f / 262144.0f;
 
 // E2M1 RTNE of (b, a) -> one byte, low nibble = a (OCP FP4 encoding, sign kept).
 __device__ __forceinline__ uint32_t cvt_e2m1x4(float a0, float a1, float a2, float a3, float a4,
@@ -231,152 +238,21 @@ __device__ __forceinline__ uint32_t cvt_e2m1x4(float a0, float a1, float a2, flo
     return out;
 }
 
-// The 16 values and 8 random words of a chunk, passed by value so that the
-// out-of-line exact path below keeps them in registers.
-struct Chunk16 {
-    float4 v0, v1, v2, v3;
-};
-// Where a chunk's SR words come from: Philox key (seed) and counter base.
-struct RandSrc {
-    uint64_t seed;
-    uint64_t L0;
-    uint32_t stream;
-};
-
-// Exact path: every element decided by the fma boundary tests.
-template <int GRID, int RND>
-__device__ __noinline__ uint2 round_pack_exact(const Chunk16 c, const ScaleOut sc, const RandSrc src) {
-    const float v[16] = {c.v0.x, c.v0.y, c.v0.z, c.v0.w, c.v1.x, c.v1.y, c.v1.z, c.v1.w,
-                         c.v2.x, c.v2.y, c.v2.z, c.v2.w, c.v3.x, c.v3.y, c.v3.z, c.v3.w};
-    // the chunk's SR words again (this path is rare)
-    uint32_t rnd[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (RND == 1) {
-        const PhiloxKeys keys = philox_keys(src.seed);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const uint64_t g = (src.L0 >> 3) + h;
-            const uint4 r = philox4x32_10(
-                make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), src.stream, 0u), keys);
-            rnd[4 * h] = r.x, rnd[4 * h + 1] = r.y, rnd[4 * h + 2] = r.z, rnd[4 * h + 3] = r.w;
-        }
-    }
-    uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float u = v[i];
-        const float au = fabsf(u);
-        int k;
-        if (RND == 0) {
-            k = round_rtne<GRID>(au, sc.m1, sc.b, sc.inv);
-        } else {
-            const uint32_t word = rnd[i >> 1];
-            const uint32_t r16 = (i & 1) ? (word >> 16) : (word & 0xFFFFu);
-            k = round_sr<GRID>(au, sc.m1, sc.b, sc.inv, r16);
-        }
-        const uint32_t code = static_cast<uint32_t>(k) | ((__float_as_uint(u) >> 28) & 8u);
-        if (i < 8) w0 |= code << (4 * i);
-        else w1 |= code << (4 * (i - 8));
-    }
-    return make_uint2(canonical_zero(w0), canonical_zero(w1));
-}
-
-// Round the 16 rotated values of one chunk and pack them (2 codes / byte,
-// low nibble = lower K index).  A certified fast path decides each element
-// from an fp32 estimate of |u|/s; when any element of the chunk lies within
-// kMargin of a decision boundary the chunk is re-decided exactly, so the
-// result always equals the exact-quotient rule.
-template <int GRID, int RND>
-__device__ __forceinline__ uint2 round_pack(const float (&v)[16], const ScaleOut &sc,
-                                            const PhiloxKeys &keys, uint32_t stream, uint64_t L0,
-                                            uint64_t seed) {
-    uint32_t rnd[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (RND == 1) {
-        const uint64_t g0 = L0 >> 3;
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const uint64_t g = g0 + c;
-            const uint4 r = philox4x32_10(
-                make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), stream, 0u), keys);
-            rnd[4 * c + 0] = r.x;
-            rnd[4 * c + 1] = r.y;
-            rnd[4 * c + 2] = r.z;
-            rnd[4 * c + 3] = r.w;
-        }
-    }
-    if (sc.zero) return make_uint2(0u, 0u);
-    uint32_t w[2] = {0u, 0u};
-    bool risky = !(sc.inv * 4.0f < INFINITY);   // tiny (subnormal) step: exact path
-    constexpr float kTop = static_cast<float>(top_of<GRID>());
-    if (GRID != 1 && RND == 0) {
-        // Uniform grid RTNE: k = rint(min(|u| * unit/s, top)).
-        const float inv4 = sc.inv * unit_of<GRID>();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float u = v[i];
-            const float y = fminf(fabsf(u) * inv4, kTop);
-            const float f = y + kRound;
-            risky |= fabsf(y - (f - kRound)) > 0.5f - kMargin;
-            const uint32_t code = (__float_as_uint(f) & 7u) | ((__float_as_uint(u) >> 28) & 8u);
-            w[i >> 3] |= code << (4 * (i & 7));
-        }
-    } else if (GRID != 1 && RND == 1) {
-        // Uniform grid SR.  With q = |u|/(s/unit) and r = r16 * 2^-16, "lo =
-        // floor(q), up iff q > lo + r" is exactly k = ceil(q - r): for q =
-        // lo + f the value q - r lies in (lo, lo+1) when f > r and in
-        // (lo-1, lo] otherwise.  q >= top gives top (clamp first).  ceil(t) =
-        // rint(t + 1/2) except when t is (near) an integer, which the margin
-        // test sends to the exact path.
-        const float inv4 = sc.inv * unit_of<GRID>();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float u = v[i];
-            const float y = fminf(fabsf(u) * inv4, kTop);
-            const uint32_t word = rnd[i >> 1];
-            const uint32_t r16 = (i & 1) ? (word >> 16) : (word & 0xFFFFu);
-            const float rf = __uint_as_float(0x4B000000u | r16) - 8388608.0f;   // r16 exactly
-            const float th = __fmaf_rn(rf, -1.0f / 65536.0f, y) + 0.5f;          // q - r + 1/2
-            const float f = th + kRound;
-            risky |= fabsf(th - (f - kRound)) > 0.5f - kMargin;
-            const uint32_t code = (__float_as_uint(f) & 7u) | ((__float_as_uint(u) >> 28) & 8u);
-            w[i >> 3] |= code << (4 * (i & 7));
-        }
-    } else if (GRID == 1 && RND == 0) {
-        // E2M1 RTNE: the hardware E2M1 conversion of u/s (ties to even); the
-        // distance to the nearest midpoint is measured in a scale where the
-        // midpoints are half-integers (x2 below 2, x1 below 4, x0.5 above).
-        float y[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            y[i] = v[i] * sc.inv;
-            const float ay = fminf(fabsf(y[i]), 6.0f);
-            const float scl = ay < 2.0f ? 2.0f : (ay < 4.0f ? 1.0f : 0.5f);
-            const float m = __fmaf_rn(ay, scl, -0.5f);
-            risky |= fabsf(m - ((m + kRound) - kRound)) < kMargin;
-        }
-        w[0] = cvt_e2m1x4(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
-        w[1] = cvt_e2m1x4(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
-    } else {
-        risky = true;   // E2M1 SR: exact path only
-    }
-    if (risky) {
-        const Chunk16 c{make_float4(v[0], v[1], v[2], v[3]), make_float4(v[4], v[5], v[6], v[7]),
-                        make_float4(v[8], v[9], v[10], v[11]), make_float4(v[12], v[13], v[14], v[15])};
-        return round_pack_exact<GRID, RND>(c, sc, RandSrc{seed, L0, stream});
-    }
-    return make_uint2(canonical_zero(w[0]), canonical_zero(w[1]));
-}
-
 // ---------------------------------------------------------------------------
-// Two chunks at once in packed fp32x2 arithmetic (lane x = chunk a, lane y =
-// chunk b): the same IEEE operations per lane as the scalar code.
-
-// Butterfly on two lanes: (x0 + x1, x0 - x1); fma(x1, -1, x0) rounds x0 - x1
-// exactly like a subtraction.
+// Packed fp32x2 arithmetic: the same IEEE operation per lane as the scalar
+// code.  The butterfly's difference is fma(x1, -1, x0), rounded exactly like
+// x0 - x1.
 __device__ __forceinline__ void bfly2(float2 &x0, float2 &x1) {
     const float2 s = __fadd2_rn(x0, x1);
     const float2 d = __ffma2_rn(x1, make_float2(-1.0f, -1.0f), x0);
     x0 = s;
     x1 = d;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
 }
 
 // 0x4B000000 | (16 bits of w): the float 2^23 + r16 (lo or hi half).
@@ -386,318 +262,526 @@ __device__ __forceinline__ float r16_magic(uint32_t w, bool hi) {
     return __uint_as_float(d);
 }
 
-// A uniform grid (E1M2 or restricted E2M1), RTNE or SR, for two chunks with
-// their own block scales: the fast paths of round_pack (same decisions, same
-// certification) with the fp32 adds / fmas done two lanes at a time.
-template <int GRID, int RND>
-__device__ __forceinline__ void round_pack2_uniform(const float (&va)[16], const float (&vb)[16],
-                                                 const ScaleOut &sa, const ScaleOut &sb,
-                                                 const PhiloxKeys &keys, uint32_t stream, uint64_t seed,
-                                                 uint64_t L0a, uint64_t L0b, uint2 &outa, uint2 &outb) {
-    constexpr float kTop = static_cast<float>(top_of<GRID>());
-    const float inv4a = sa.inv * unit_of<GRID>(), inv4b = sb.inv * unit_of<GRID>();
-    // min(|u| * inv4, top) as top * sat(|u| * inv4 / top): a saturating
-    // multiply on the fma pipe instead of a min (the estimate moves by a few
-    // ulp, far inside the 2^-16 margin; at and above top both give top).
-    const float c7a = inv4a * (1.0f / kTop), c7b = inv4b * (1.0f / kTop);
-    float deva = 0.0f, devb = 0.0f;      // largest distance from a rint half-way point
-    uint32_t wa[2] = {0u, 0u}, wb[2] = {0u, 0u};
-    const float2 kR = make_float2(kRound, kRound);
-    const float2 kRn = make_float2(-kRound, -kRound);
-    const float2 m1 = make_float2(-1.0f, -1.0f);
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-        // SR words of elements 8 hf .. 8 hf + 7 of each chunk (one Philox call each)
-        uint4 ra = make_uint4(0, 0, 0, 0), rb = make_uint4(0, 0, 0, 0);
-        if (RND == 1) {
-            const uint64_t ga = (L0a >> 3) + hf, gb = (L0b >> 3) + hf;
-            ra = philox4x32_10(make_uint4(static_cast<uint32_t>(ga), static_cast<uint32_t>(ga >> 32), stream, 0u),
-                               keys);
-            rb = philox4x32_10(make_uint4(static_cast<uint32_t>(gb), static_cast<uint32_t>(gb >> 32), stream, 0u),
-                               keys);
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Offset-binary nibbles o = g + 8 (g in [-7, 7]) -> sign-magnitude codes:
+// g >= 0 gives o ^ 8 = g; g < 0 (o < 8) gives (o ^ 15) + 1 = 8 + |g|.  Eight
+// nibbles at once, no carries between them; g = 0 gives 0 (canonical zero).
+__device__ __forceinline__ uint32_t offset_to_sign_magnitude(uint32_t o) {
+    const uint32_t neg = (~o & 0x88888888u) >> 3;     // 1 in each negative nibble
+    return (o ^ (neg * 15u | 0x88888888u)) + neg;
+}
+
+// bf16 -> fp32 with the D sign s (0 or 0x80000000) applied: adding s flips
+// the sign bit like an xor.
+__device__ __forceinline__ float lo_f(uint32_t w, uint32_t s) { return __uint_as_float((w << 16) + s); }
+__device__ __forceinline__ float hi_f(uint32_t w, uint32_t s) {
+    return __uint_as_float((w & 0xFFFF0000u) ^ s);
+}
+
+// Grid constants of the runtime-selected grid (the two uniform grids share
+// one kernel): gmax, grid units per step (u / s * unit is the level index),
+// the top index, and frexp-style (mantissa in [1, 2), exponent) of gmax.
+struct GridK {
+    float gmax, unit, top, mg;
+    int eg;
+};
+
+__device__ __forceinline__ GridK grid_constants(int grid) {
+    if (grid == 0) return GridK{1.75f, 4.0f, 7.0f, 1.75f, 0};   // E1M2: k / 4
+    if (grid == 1) return GridK{6.0f, 1.0f, 7.0f, 1.5f, 2};     // E2M1 (unit unused)
+    return GridK{2.0f, 2.0f, 4.0f, 1.0f, 1};                    // E2M1, max_fpx 2: k / 2
+}
+
+// block_scale with the grid taken at run time: the same operations as the
+// templated version, so the stored scales and steps are identical.
+__device__ __forceinline__ ScaleOut block_scale_rt(float amax, int scale_fmt, float S, float G, const GridK &gk) {
+    ScaleOut o;
+    if (scale_fmt == 2) {
+        int X = -127;
+        if (amax > 0.0f) {
+            const int ea = ilogbf(amax);
+            const float ma = ldexpf(amax, -ea);
+            X = ea - gk.eg + (ma > gk.mg ? 1 : 0);
+            X = X < -127 ? -127 : (X > 127 ? 127 : X);
         }
-        const uint32_t rwa[4] = {ra.x, ra.y, ra.z, ra.w}, rwb[4] = {rb.x, rb.y, rb.z, rb.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int i = 8 * hf + e;
-            const float2 y7 = make_float2(__saturatef(fabsf(va[i]) * c7a), __saturatef(fabsf(vb[i]) * c7b));
-            float2 h;
-            if (RND == 1) {
-                // h = y - r16 * 2^-16 + 1/2 (k = ceil(q - r) = rint(h) off the
-                // integers, which the margin test sends to the exact path)
-                const float2 rf = __fadd2_rn(make_float2(r16_magic(rwa[e >> 1], e & 1), r16_magic(rwb[e >> 1], e & 1)),
-                                             make_float2(-8421376.0f, -8421376.0f));   // r16 - 2^15
-                const float2 rt = __fmul2_rn(rf, make_float2(-1.0f / 65536.0f, -1.0f / 65536.0f));   // exact
-                h = __ffma2_rn(y7, make_float2(kTop, kTop), rt);
-            } else {
-                h = __fmul2_rn(y7, make_float2(kTop, kTop));
-            }
-            const float2 f = __fadd2_rn(h, kR);
-            const float2 g = __fadd2_rn(f, kRn);
-            const float2 d = __ffma2_rn(g, m1, h);       // h - rint(h), in [-1/2, 1/2]
-            deva = fmaxf(deva, fabsf(d.x));
-            devb = fmaxf(devb, fabsf(d.y));
-            const uint32_t ca = (__float_as_uint(f.x) & 7u) | ((__float_as_uint(va[i]) >> 28) & 8u);
-            const uint32_t cb = (__float_as_uint(f.y) & 7u) | ((__float_as_uint(vb[i]) >> 28) & 8u);
-            // nibbles do not overlap: a multiply-add places them
-            wa[hf] = ca * (1u << (4 * e)) + wa[hf];
-            wb[hf] = cb * (1u << (4 * e)) + wb[hf];
-        }
+        o.m1 = 1.0f;
+        o.b = ldexpf(1.0f, X);
+        o.zero = !(amax > 0.0f);
+        o.inv = ldexpf(1.0f, -X);
+        o.stored = static_cast<uint32_t>(X + 127);
+        return o;
     }
-    const bool riska = !(inv4a < INFINITY) || deva > 0.5f - kMargin;
-    const bool riskb = !(inv4b < INFINITY) || devb > 0.5f - kMargin;
-    outa = sa.zero ? make_uint2(0u, 0u) : make_uint2(canonical_zero(wa[0]), canonical_zero(wa[1]));
-    outb = sb.zero ? make_uint2(0u, 0u) : make_uint2(canonical_zero(wb[0]), canonical_zero(wb[1]));
-    if (riska && !sa.zero) {
-        const Chunk16 c{make_float4(va[0], va[1], va[2], va[3]), make_float4(va[4], va[5], va[6], va[7]),
-                        make_float4(va[8], va[9], va[10], va[11]), make_float4(va[12], va[13], va[14], va[15])};
-        outa = round_pack_exact<GRID, RND>(c, sa, RandSrc{seed, L0a, stream});
+    if (scale_fmt == 0) {
+        const float s = __fdiv_rn(amax, gk.gmax);
+        o.m1 = 1.0f;
+        o.b = s;
+        o.zero = !(s > 0.0f);
+        o.inv = o.zero ? 0.0f : approx_rcp(s);
+        o.stored = __float_as_uint(s);
+    } else {
+        const float q = __fdiv_rn(amax, G);
+        const __nv_fp8_storage_t e8 = __nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3);
+        const float e = e4m3_to_f32(e8);
+        o.m1 = e;
+        o.b = S;
+        o.zero = !(e > 0.0f);
+        o.inv = o.zero ? 0.0f : approx_rcp(e * S);
+        o.stored = e8;
     }
-    if (riskb && !sb.zero) {
-        const Chunk16 c{make_float4(vb[0], vb[1], vb[2], vb[3]), make_float4(vb[4], vb[5], vb[6], vb[7]),
-                        make_float4(vb[8], vb[9], vb[10], vb[11]), make_float4(vb[12], vb[13], vb[14], vb[15])};
-        outb = round_pack_exact<GRID, RND>(c, sb, RandSrc{seed, L0b, stream});
-    }
+    return o;
 }
 
 // ---------------------------------------------------------------------------
-// Kernel.  A CTA of 256 compute threads plus one producer warp takes units of
-// 256 x 64 bf16 elements, staged in shared memory by TMA with the 128-byte
-// swizzle and double-buffered across the CTA's units.  Every compute thread
-// quantizes 64 consecutive K elements of one output row, so any Hadamard size
-// up to 64 and either block size stays inside the thread:
-//   AXIS 0 (row-wise)    one 64 (K) x 256 (rows) box; thread t reads row t,
-//                        eight 16-byte chunks (chunk c of row t sits at chunk
-//                        c ^ (t & 7)).
-//   AXIS 1 (column-wise) four 64 (columns) x 64 (K rows) boxes side by side;
-//                        thread t reads column t, one bf16 per K row; a warp
-//                        reads 32 consecutive columns of one K row.
-//   AXIS 2 (both)        the AXIS 1 tile quantized twice: column-wise into
-//                        `a` exactly as AXIS 1, then row-wise into `a2`, where
-//                        thread t takes row t & 63 of box t >> 6 (64 columns
-//                        of one input row).  One read of the tensor serves
-//                        both of its GEMM operands.
-// Codes (32 bytes per thread) and block-major scales (a warp writes 32
-// consecutive rows of each block) go straight to global memory.
+// Work unit and thread maps.
+constexpr int kComputeWarps = 8;
+constexpr int kThreads = kComputeWarps * 32;
+constexpr int kCtaThreads = kThreads + 32;        // + one producer warp
 constexpr int kUnitRows = 256;
 constexpr int kStageBytes = kUnitRows * 64 * 2;   // 32 KB of bf16
-constexpr int kStages = 2;
-constexpr int kComputeWarps = kThreads / 32;
-constexpr int kCtaThreads = kThreads + 32;        // + one producer warp
-constexpr int kQuantSmem = kStages * kStageBytes + 1024 + 64;
-// Resident CTAs per SM: three for one output (72 registers a thread); the
-// dual kernel does twice the work per staged tile and keeps more state, two.
-template <int AXIS>
-constexpr int ctas_per_sm() { return AXIS == 2 ? 2 : 3; }
+constexpr int kStages = 3;
+constexpr int kCtasPerSm = 2;
+constexpr int kQuantSmem = kStages * kStageBytes + 1024 + 128;
 
-// Two-level tensor scale of one output: S maps the rotated tensor amax to
-// gmax * 448 (the top of E4M3), G = gmax * S is the block-scale divisor.
-template <int GRID>
-__device__ __forceinline__ void tensor_scale(const QuantArgs &q, float &S, float &G) {
-    const float amax_t = *q.amax_t;
-    S = amax_t > 0.0f ? __fdiv_rn(amax_t, gmax_of<GRID>() * 448.0f) : 1.0f;
-    G = __fmul_rn(gmax_of<GRID>(), S);
-    if (blockIdx.x == 0 && threadIdx.x == 0 && q.S_out) *q.S_out = S;
+enum { MAP_ROW = 0, MAP_COL2 = 1, MAP_COL1 = 2 };
+
+// Where a thread reads its 64 bf16 values in the staged tile.
+//   row:  p = the thread's 128-byte tile row, off8[0] = its swizzle (row & 7);
+//   col2: p = the box's first K row of this half, off8[j] = byte offset of the
+//         thread's column pair in a K row r with r % 8 == j (without the
+//         swizzle every off8[j] is off8[0]);
+//   col1: p = the box, off8[j] = the same for the thread's single column.
+struct Src {
+    const uint8_t *p;
+    uint32_t off8[8];
+};
+
+// Output rows and first output column of the lane-x and lane-y runs
+// (callers validate rows and kpad below 2^31).
+struct Site {
+    int32_t row_x, row_y, k_x, k_y;
+};
+
+// D sign bit of lane-run position p (p < 64; the launcher stores the mask
+// pattern repeated with period n), 0 without a rotation.
+template <int NH>
+__device__ __forceinline__ uint32_t dsign(const QuantArgs &a, int p) {
+    return NH == 0 ? 0u : a.smask[p];
 }
 
-// Quantizes K elements [k0, k0 + 64) of output row orow of `a`:
-//   RD 0: they are one swizzled 128-byte row at src (chunk c at (c ^ swz) << 4);
-//   RD 1: they are one column of the four-box tile at src, K row kr at
-//         src + col_off[kr & 7] + kr * 128.
-// The rotated values' amax goes to amax_acc (AMAX_ONLY) or the codes and
-// scales to `a` (rows beyond a.out_rows are computed but not stored).
-template <int RD, int NH, int BLK, int GRID, int RND, bool AMAX_ONLY>
-__device__ __forceinline__ void quantize64(const QuantArgs &a, const uint8_t *src, int swz,
-                                           const uint32_t (&col_off)[8], int64_t orow, int64_t k0,
-                                           float S, float G, const PhiloxKeys &keys,
-                                           const uint32_t (&smask)[16], uint32_t pat_lo,
-                                           uint32_t pat_hi, float &amax_acc) {
-    // Per group of GS elements (the Hadamard block and the scale block both
-    // lie inside one group): load, D, H, block scales, round, pack.
-    constexpr int GS = (NH > BLK ? NH : BLK) > 16 ? (NH > BLK ? NH : BLK) : 16;
-    uint32_t codes[8];
-    uint32_t stored[4];
-    if constexpr (GS == 16) {
-        // Groups g and g + 16 side by side as the two lanes of fp32x2
-        // values: same positions mod 16, so the same signs of D; the
-        // butterflies and the rounding arithmetic run two lanes at a time.
-        // Not unrolled: one copy of the body keeps the kernel small.
-#pragma unroll 1
-        for (int gp = 0; gp < 64; gp += 32) {
-            float va[16], vb[16];
-            if (RD == 0) {
+// Entries processed together: 16 when both the Hadamard block and the scale
+// block fit in 16 positions, else the whole run of 32.
+template <int NH, int BLK>
+constexpr int ent_of() { return (NH <= 16 && BLK == 16) ? 16 : 32; }
+
+// Entries [E0, E0 + ENT) of the thread's run pair.
+template <int MAP, bool SWZ, int NH, int E0, int ENT>
+__device__ __forceinline__ void load_entries(const QuantArgs &a, const Src &src, float2 (&v)[ENT]) {
+    if constexpr (MAP == MAP_ROW) {
+        const uint32_t swz = src.off8[0];
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const uint4 qa = *reinterpret_cast<const uint4 *>(src + (((gp / 8 + c) ^ swz) << 4));
-                    const uint4 qb = *reinterpret_cast<const uint4 *>(src + (((gp / 8 + 2 + c) ^ swz) << 4));
-                    const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w}, wb[4] = {qb.x, qb.y, qb.z, qb.w};
+        for (int c = E0 / 8; c < (E0 + ENT) / 8; ++c) {
+            const uint4 qx = *reinterpret_cast<const uint4 *>(src.p + ((c ^ swz) << 4));
+            const uint4 qy = *reinterpret_cast<const uint4 *>(src.p + (((c + 4) ^ swz) << 4));
+            const uint32_t wx[4] = {qx.x, qx.y, qx.z, qx.w}, wy[4] = {qy.x, qy.y, qy.z, qy.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i0 = 8 * c + 2 * e;
-                        va[i0] = __uint_as_float((wa[e] << 16) + smask[i0]);
-                        va[i0 + 1] = __uint_as_float((wa[e] & 0xFFFF0000u) ^ smask[i0 + 1]);
-                        vb[i0] = __uint_as_float((wb[e] << 16) + smask[i0]);
-                        vb[i0 + 1] = __uint_as_float((wb[e] & 0xFFFF0000u) ^ smask[i0 + 1]);
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int ka = gp + i, kb = gp + 16 + i;
-                    const uint32_t ba = *reinterpret_cast<const uint16_t *>(src + col_off[ka & 7] + ka * 128);
-                    const uint32_t bb = *reinterpret_cast<const uint16_t *>(src + col_off[kb & 7] + kb * 128);
-                    va[i] = __uint_as_float((ba << 16) + smask[i]);
-                    vb[i] = __uint_as_float((bb << 16) + smask[i]);
-                }
+            for (int e = 0; e < 4; ++e) {
+                const int i = 8 * c + 2 * e;
+                v[i - E0] = make_float2(lo_f(wx[e], dsign<NH>(a, i)), lo_f(wy[e], dsign<NH>(a, i + 32)));
+                v[i + 1 - E0] =
+                    make_float2(hi_f(wx[e], dsign<NH>(a, i + 1)), hi_f(wy[e], dsign<NH>(a, i + 33)));
             }
-            if (NH == 16) {
-                float2 pr[16];
+        }
+    } else if constexpr (MAP == MAP_COL2) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) pr[i] = make_float2(va[i], vb[i]);
-#pragma unroll
-                for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (!(i & h)) bfly2(pr[i], pr[i + h]);
-                }
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    va[i] = pr[i].x;
-                    vb[i] = pr[i].y;
-                }
-            }
-            if (AMAX_ONLY) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    amax_acc = fmaxf(amax_acc, fmaxf(fabsf(va[i]), fabsf(vb[i])));
-                continue;
-            }
-            float ama = 0.0f, amb = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                ama = fmaxf(ama, fabsf(va[i]));
-                amb = fmaxf(amb, fabsf(vb[i]));
-            }
-            const ScaleOut sa = block_scale<GRID>(ama, a.scale_fmt, S, G);
-            const ScaleOut sb = block_scale<GRID>(amb, a.scale_fmt, S, G);
-            const uint64_t L0a = static_cast<uint64_t>(orow) * static_cast<uint64_t>(a.kpad) +
-                                 static_cast<uint64_t>(k0 + gp);
-            uint2 pa, pb;
-            if (GRID != 1) {
-                round_pack2_uniform<GRID, RND>(va, vb, sa, sb, keys, a.stream, a.seed, L0a, L0a + 16,
-                                               pa, pb);
-            } else {
-                pa = round_pack<GRID, RND>(va, sa, keys, a.stream, L0a, a.seed);
-                pb = round_pack<GRID, RND>(vb, sb, keys, a.stream, L0a + 16, a.seed);
-            }
-            if (gp == 0) {
-                codes[0] = pa.x, codes[1] = pa.y, codes[2] = pb.x, codes[3] = pb.y;
-                stored[0] = sa.stored, stored[1] = sb.stored;
-            } else {
-                codes[4] = pa.x, codes[5] = pa.y, codes[6] = pb.x, codes[7] = pb.y;
-                stored[2] = sa.stored, stored[3] = sb.stored;
-            }
+        for (int i = E0; i < E0 + ENT; ++i) {
+            const uint32_t off = SWZ ? src.off8[i & 7] : src.off8[0];
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(src.p + i * 128 + off);
+            v[i - E0] = make_float2(lo_f(w, dsign<NH>(a, i)), hi_f(w, dsign<NH>(a, i)));
         }
     } else {
 #pragma unroll
-        for (int g0 = 0; g0 < 64; g0 += GS) {
-            float v[GS];
-            if (RD == 0) {
+        for (int i = E0; i < E0 + ENT; ++i) {
+            const uint32_t off = SWZ ? src.off8[i & 7] : src.off8[0];
+            const uint32_t bx = *reinterpret_cast<const uint16_t *>(src.p + i * 128 + off);
+            const uint32_t by = *reinterpret_cast<const uint16_t *>(src.p + (i + 32) * 128 + off);
+            v[i - E0] = make_float2(lo_f(bx, dsign<NH>(a, i)), lo_f(by, dsign<NH>(a, i + 32)));
+        }
+    }
+}
+
+// u = H_n (D x) per n-block along each lane's run (stages h = 1, 2, ..., n/2;
+// for n = 64 the last stage pairs lane x with lane y, positions i and i + 32).
+template <int NH, int ENT>
+__device__ __forceinline__ void rht_entries(float2 (&v)[ENT]) {
+    constexpr int HI = NH > 32 ? 32 : NH;
 #pragma unroll
-                for (int c = 0; c < GS / 8; ++c) {
-                    const int cg = g0 / 8 + c;
-                    const uint4 q = *reinterpret_cast<const uint4 *>(src + ((cg ^ swz) << 4));
-                    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    for (int h = 1; h < HI; h <<= 1) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        v[8 * c + 2 * e] = __uint_as_float(w[e] << 16);
-                        v[8 * c + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-                    }
-                }
-            } else {
+        for (int i = 0; i < ENT; ++i)
+            if (!(i & h)) bfly2(v[i], v[i + h]);
+    }
+    if constexpr (NH == 64) {
 #pragma unroll
-                for (int i = 0; i < GS; ++i) {
-                    const int kr = g0 + i;
-                    const uint16_t b = *reinterpret_cast<const uint16_t *>(src + col_off[kr & 7] + kr * 128);
-                    v[i] = __uint_as_float(static_cast<uint32_t>(b) << 16);
+        for (int i = 0; i < ENT; ++i) {
+            const float x0 = v[i].x, x1 = v[i].y;
+            v[i] = make_float2(__fadd_rn(x0, x1), __fsub_rn(x0, x1));
+        }
+    }
+}
+
+// Block amaxes of both lanes: am[b] lane x, am[NB + b] lane y.
+template <int BLK, int ENT>
+__device__ __forceinline__ void block_amax(const float2 (&v)[ENT], float (&am)[2 * ENT / BLK]) {
+    constexpr int NB = ENT / BLK;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        float mx = 0.0f, my = 0.0f;
+#pragma unroll
+        for (int i = b * BLK; i < (b + 1) * BLK; i += 2) {
+            mx = max3(mx, fabsf(v[i].x), fabsf(v[i + 1].x));
+            my = max3(my, fabsf(v[i].y), fabsf(v[i + 1].y));
+        }
+        am[b] = mx;
+        am[NB + b] = my;
+    }
+}
+
+// Stores the 16 code bytes (and the E1M2 correction plane) and the block
+// scales of one lane run.
+template <int BLK>
+__device__ __forceinline__ void store_run(const QuantArgs &a, int32_t row, int32_t k0, const uint32_t *w,
+                                          const uint32_t *st) {
+    if (row >= a.out_rows) return;
+    const int64_t off = static_cast<int64_t>(row) * (a.kpad / 2) + k0 / 2;
+    *reinterpret_cast<uint4 *>(a.codes + off) = make_uint4(w[0], w[1], w[2], w[3]);
+    if (a.corr != nullptr)
+        *reinterpret_cast<uint4 *>(a.corr + off) = make_uint4(e1m2_correction(w[0]), e1m2_correction(w[1]),
+                                                              e1m2_correction(w[2]), e1m2_correction(w[3]));
+#pragma unroll
+    for (int b = 0; b < 32 / BLK; ++b) {
+        const int64_t at = static_cast<int64_t>(k0 / BLK + b) * a.scale_ld + row;
+        if (a.scale_fmt == 0)
+            reinterpret_cast<uint32_t *>(a.scales)[at] = st[b];
+        else
+            reinterpret_cast<uint8_t *>(a.scales)[at] = static_cast<uint8_t>(st[b]);
+    }
+}
+
+// Exact path, cooperative: the warp re-derives the 64 elements of each of
+// its threads whose fast decision was not certified ("owners"), from the
+// staged tile that is still in place.  Lane l holds run position l of the
+// owner (its lane-x and lane-y elements as one fp32x2 value), so the
+// butterflies become shuffles (the lower partner forms a + b, the upper one
+// a - b: the same IEEE operations), block maxima are shuffle reductions, and
+// every lane decides its two codes by the fma boundary tests.  Few registers,
+// no call: the fast path keeps its registers.
+template <int MAP, bool SWZ, int NH>
+__device__ __forceinline__ float2 load_entry(const QuantArgs &a, const uint8_t *p, const uint32_t (&off8)[8], int l) {
+    const uint32_t off = SWZ ? off8[l & 7] : off8[0];
+    if constexpr (MAP == MAP_ROW) {
+        const uint32_t swz = off8[0], c = static_cast<uint32_t>(l >> 3), e = static_cast<uint32_t>(l & 7);
+        const uint32_t bx = *reinterpret_cast<const uint16_t *>(p + ((c ^ swz) << 4) + 2 * e);
+        const uint32_t by = *reinterpret_cast<const uint16_t *>(p + (((c + 4) ^ swz) << 4) + 2 * e);
+        return make_float2(lo_f(bx, dsign<NH>(a, l)), lo_f(by, dsign<NH>(a, l + 32)));
+    } else if constexpr (MAP == MAP_COL2) {
+        const uint32_t w = *reinterpret_cast<const uint32_t *>(p + l * 128 + off);
+        return make_float2(lo_f(w, dsign<NH>(a, l)), hi_f(w, dsign<NH>(a, l)));
+    } else {
+        const uint32_t bx = *reinterpret_cast<const uint16_t *>(p + l * 128 + off);
+        const uint32_t by = *reinterpret_cast<const uint16_t *>(p + (l + 32) * 128 + off);
+        return make_float2(lo_f(bx, dsign<NH>(a, l)), lo_f(by, dsign<NH>(a, l + 32)));
+    }
+}
+
+template <int MAP, bool SWZ, int NH, int BLK, int GRID, int RND>
+__device__ __forceinline__ void coop_exact(const QuantArgs &a, const uint8_t *tile, uint32_t pofs,
+                                        const uint32_t (&off8)[8], Site site, float S, float G,
+                                        uint32_t owners) {
+    const int lane = threadIdx.x & 31;
+    while (owners != 0u) {
+        const int o = __ffs(owners) - 1;
+        owners &= owners - 1u;
+        uint32_t off[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) off[j] = __shfl_sync(0xFFFFFFFFu, off8[j], o);
+        const uint8_t *p = tile + __shfl_sync(0xFFFFFFFFu, pofs, o);
+        Site so;
+        so.row_x = __shfl_sync(0xFFFFFFFFu, site.row_x, o);
+        so.row_y = __shfl_sync(0xFFFFFFFFu, site.row_y, o);
+        so.k_x = __shfl_sync(0xFFFFFFFFu, site.k_x, o);
+        so.k_y = __shfl_sync(0xFFFFFFFFu, site.k_y, o);
+        float2 v = load_entry<MAP, SWZ, NH>(a, p, off, lane);
+        constexpr int HI = NH > 32 ? 32 : NH;
+#pragma unroll
+        for (int h = 1; h < HI; h <<= 1) {
+            const float px = __shfl_xor_sync(0xFFFFFFFFu, v.x, h), py = __shfl_xor_sync(0xFFFFFFFFu, v.y, h);
+            if (lane & h) v = make_float2(__fsub_rn(px, v.x), __fsub_rn(py, v.y));
+            else v = make_float2(__fadd_rn(v.x, px), __fadd_rn(v.y, py));
+        }
+        if (NH == 64) v = make_float2(__fadd_rn(v.x, v.y), __fsub_rn(v.x, v.y));
+        float mx = fabsf(v.x), my = fabsf(v.y);
+#pragma unroll
+        for (int m = 1; m < BLK; m <<= 1) {
+            mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, m));
+            my = fmaxf(my, __shfl_xor_sync(0xFFFFFFFFu, my, m));
+        }
+        uint32_t nib[2];
+        uint32_t stv[2];
+#pragma unroll
+        for (int ln = 0; ln < 2; ++ln) {
+            const float u = ln ? v.y : v.x;
+            const ScaleOut sc = block_scale<GRID>(ln ? my : mx, a.scale_fmt, S, G);
+            stv[ln] = sc.stored;
+            int k = 0;
+            if (!sc.zero) {
+                if (RND == 0) {
+                    k = round_rtne<GRID>(fabsf(u), sc.m1, sc.b, sc.inv);
+                } else {
+                    const int64_t row = ln ? so.row_y : so.row_x, k0 = ln ? so.k_y : so.k_x;
+                    const uint64_t g = ((static_cast<uint64_t>(row) * static_cast<uint64_t>(a.kpad) +
+                                         static_cast<uint64_t>(k0)) >> 3) + (lane >> 3);
+                    const uint4 r = philox4x32_10(make_uint4(static_cast<uint32_t>(g),
+                                                             static_cast<uint32_t>(g >> 32), a.stream, 0u),
+                                                  a.keys);
+                    const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+                    const uint32_t word = rw[(lane >> 1) & 3];
+                    const uint32_t r16 = (lane & 1) ? (word >> 16) : (word & 0xFFFFu);
+                    k = round_sr<GRID>(fabsf(u), sc.m1, sc.b, sc.inv, r16);
                 }
             }
-            if (NH > 0) {
+            nib[ln] = k == 0 ? 0u : (static_cast<uint32_t>(k) | ((__float_as_uint(u) >> 28) & 8u));
+        }
+        // 8 lanes' nibbles -> one code word; lane 8j stores word j of each run
+        uint32_t wx = nib[0] << (4 * (lane & 7)), wy = nib[1] << (4 * (lane & 7));
 #pragma unroll
-                for (int i = 0; i < GS; ++i) {
-                    const int p = g0 + i;
-                    const uint32_t bit = p < 32 ? (pat_lo >> p) & 1u : (pat_hi >> (p - 32)) & 1u;
-                    v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (bit << 31));
-                }
+        for (int m = 1; m < 8; m <<= 1) {
+            wx |= __shfl_xor_sync(0xFFFFFFFFu, wx, m);
+            wy |= __shfl_xor_sync(0xFFFFFFFFu, wy, m);
+        }
 #pragma unroll
-                for (int h = 1; h < NH; h <<= 1) {
-#pragma unroll
-                    for (int i = 0; i < GS; ++i) {
-                        if (i & h) continue;
-                        const float x0 = v[i], x1 = v[i + h];
-                        v[i] = __fadd_rn(x0, x1);
-                        v[i + h] = __fsub_rn(x0, x1);
-                    }
-                }
+        for (int ln = 0; ln < 2; ++ln) {
+            const int32_t row = ln ? so.row_y : so.row_x, k0 = ln ? so.k_y : so.k_x;
+            if (row >= a.out_rows) continue;
+            const uint32_t w = ln ? wy : wx;
+            if ((lane & 7) == 0) {
+                const int64_t at = static_cast<int64_t>(row) * (a.kpad / 2) + k0 / 2 + 4 * (lane >> 3);
+                *reinterpret_cast<uint32_t *>(a.codes + at) = w;
+                if (a.corr != nullptr) *reinterpret_cast<uint32_t *>(a.corr + at) = e1m2_correction(w);
             }
-            if constexpr (AMAX_ONLY) {
-#pragma unroll
-                for (int i = 0; i < GS; ++i) amax_acc = fmaxf(amax_acc, fabsf(v[i]));
-            } else {
-#pragma unroll
-            for (int b0 = 0; b0 < GS; b0 += BLK) {
-                float am = 0.0f;
-#pragma unroll
-                for (int i = 0; i < BLK; ++i) am = fmaxf(am, fabsf(v[b0 + i]));
-                const ScaleOut sc = block_scale<GRID>(am, a.scale_fmt, S, G);
-                stored[(g0 + b0) / BLK] = sc.stored;
-#pragma unroll
-                for (int c0 = 0; c0 < BLK; c0 += 16) {
-                    float chunk[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) chunk[i] = v[b0 + c0 + i];
-                    const int kc = g0 + b0 + c0;
-                    const uint64_t L0 = static_cast<uint64_t>(orow) * static_cast<uint64_t>(a.kpad) +
-                                        static_cast<uint64_t>(k0 + kc);
-                    const uint2 pk = round_pack<GRID, RND>(chunk, sc, keys, a.stream, L0, a.seed);
-                    codes[kc / 8] = pk.x;
-                    codes[kc / 8 + 1] = pk.y;
-                }
-            }
+            if (lane % BLK == 0) {
+                const int64_t at = static_cast<int64_t>(k0 / BLK + lane / BLK) * a.scale_ld + row;
+                if (a.scale_fmt == 0) reinterpret_cast<uint32_t *>(a.scales)[at] = stv[ln];
+                else reinterpret_cast<uint8_t *>(a.scales)[at] = static_cast<uint8_t>(stv[ln]);
             }
         }
     }
-    if constexpr (!AMAX_ONLY) {
-        if (orow >= a.out_rows) return;
-        uint4 *dst = reinterpret_cast<uint4 *>(a.codes + orow * (a.kpad / 2) + k0 / 2);
-        dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-        dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-        if (GRID == 0 && a.corr != nullptr) {
-            // E1M2 correction plane for the block-scaled FP4 GEMM
-            uint4 *cdst = reinterpret_cast<uint4 *>(a.corr + orow * (a.kpad / 2) + k0 / 2);
-            cdst[0] = make_uint4(e1m2_correction(codes[0]), e1m2_correction(codes[1]),
-                                 e1m2_correction(codes[2]), e1m2_correction(codes[3]));
-            cdst[1] = make_uint4(e1m2_correction(codes[4]), e1m2_correction(codes[5]),
-                                 e1m2_correction(codes[6]), e1m2_correction(codes[7]));
-        }
-        constexpr int kBlocks = 64 / BLK;
+}
+
+// Perturbation of the E2M1 estimate (relative): far above its error (a few
+// ulp) and far below the distance that separates grid decisions.
+constexpr float kE2m1Eps = 1.0f / 1048576.0f;
+// Start value of a code accumulator: 2^23 + 0x8888 (offset 8 per nibble).
+constexpr float kPackBase = 8423560.0f;
+
+// One thread's 64 elements: load, rotate, block scales, certified fast
+// rounding, packing, stores (or the exact path).  GRID 0 = the uniform grids
+// (E1M2, restricted E2M1; a.grid picks the constants), GRID 1 = E2M1.
+template <int MAP, bool SWZ, int NH, int BLK, int GRID, int RND>
+__device__ __forceinline__ bool quant_thread(const QuantArgs &a, const Src &src, const Site &site, float S,
+                                             float G, const GridK &gk) {
+    constexpr int ENT = ent_of<NH, BLK>();
+    constexpr int NBP = ENT / BLK;          // blocks per lane in a pass
+    constexpr int NB = 32 / BLK;            // blocks per lane run
+    uint32_t cw[8];                         // codes: lane x words 0..3, lane y words 4..7
+    uint32_t st[2 * NB];                    // stored scales: lane x, then lane y
+    bool risky = (GRID == 1 && RND == 1);   // E2M1 SR: exact path
+    uint64_t gx = 0, gy = 0;
+    if (RND == 1 && GRID == 0) {
+        gx = (static_cast<uint64_t>(site.row_x) * static_cast<uint64_t>(a.kpad) +
+              static_cast<uint64_t>(site.k_x)) >> 3;
+        gy = (static_cast<uint64_t>(site.row_y) * static_cast<uint64_t>(a.kpad) +
+              static_cast<uint64_t>(site.k_y)) >> 3;
+    }
 #pragma unroll
-        for (int b = 0; b < kBlocks; ++b) {
-            const int64_t blk = k0 / BLK + b;
-            if (a.scale_fmt == 0)
-                reinterpret_cast<uint32_t *>(a.scales)[blk * a.scale_ld + orow] = stored[b];
-            else
-                reinterpret_cast<uint8_t *>(a.scales)[blk * a.scale_ld + orow] = static_cast<uint8_t>(stored[b]);
+    for (int p = 0; p < 32 / ENT; ++p) {
+        float2 v[ENT];
+        if (p == 0) load_entries<MAP, SWZ, NH, 0, ENT>(a, src, v);
+        else load_entries<MAP, SWZ, NH, (32 / ENT > 1 ? ENT : 0), ENT>(a, src, v);
+        rht_entries<NH, ENT>(v);
+        float am[2 * NBP];
+        block_amax<BLK, ENT>(v, am);
+        float inv[2 * NBP];
+#pragma unroll
+        for (int j = 0; j < 2 * NBP; ++j) {
+            const ScaleOut sc = block_scale_rt(am[j], a.scale_fmt, S, G, gk);
+            st[(j / NBP) * NB + p * NBP + (j % NBP)] = sc.stored;
+            const float iv = sc.zero ? 0.0f : (GRID == 1 ? sc.inv : sc.inv * gk.unit);
+            inv[j] = iv;
+            risky |= !(iv < INFINITY);              // subnormal step: no usable reciprocal
+            // RTNE without a clamp: the block maximum must stay below top + 1/2
+            if (RND == 0 && GRID == 0) risky |= am[j] * iv >= gk.top + 0.4921875f;
+        }
+        if constexpr (GRID == 1) {
+            // E2M1 RTNE: the hardware E2M1 conversion (ties to even,
+            // saturating at 6) of the estimate scaled up and down by
+            // kE2m1Eps; equal codes certify every quotient in between.
+#pragma unroll
+            for (int j = 0; j < ENT / 8; ++j) {
+                float y1[2][8], y2[2][8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int i = 8 * j + e;
+                    const int b = i / BLK;
+                    const float2 p1 = __fmul2_rn(v[i], make_float2(inv[b] * (1.0f + kE2m1Eps),
+                                                                  inv[NBP + b] * (1.0f + kE2m1Eps)));
+                    const float2 p2 = __fmul2_rn(v[i], make_float2(inv[b] * (1.0f - kE2m1Eps),
+                                                                  inv[NBP + b] * (1.0f - kE2m1Eps)));
+                    y1[0][e] = p1.x, y1[1][e] = p1.y, y2[0][e] = p2.x, y2[1][e] = p2.y;
+                }
+#pragma unroll
+                for (int ln = 0; ln < 2; ++ln) {
+                    const uint32_t c1 = cvt_e2m1x4(y1[ln][0], y1[ln][1], y1[ln][2], y1[ln][3], y1[ln][4],
+                                                   y1[ln][5], y1[ln][6], y1[ln][7]);
+                    const uint32_t c2 = cvt_e2m1x4(y2[ln][0], y2[ln][1], y2[ln][2], y2[ln][3], y2[ln][4],
+                                                   y2[ln][5], y2[ln][6], y2[ln][7]);
+                    risky |= c1 != c2;
+                    cw[4 * ln + p * (ENT / 8) + j] = canonical_zero(c1);
+                }
+            }
+        } else {
+            // Uniform grids: g = rint(t) with t = u/s in grid units (RTNE) or
+            // t = sign(u) (min(|u|/s, top) + 1/2 - r) (SR: ceil(|q| - r) off
+            // the integers), by the 1.5 * 2^23 rint; d = t - g certifies it.
+            // The signed g are packed four per fp32 accumulator as
+            // offset-binary nibbles (exact integer fmas), then turned into
+            // sign-magnitude codes.
+            const float2 kR2 = make_float2(kRound, kRound), kRn2 = make_float2(-kRound, -kRound);
+            const float2 m1 = make_float2(-1.0f, -1.0f);
+            float2 acc[ENT / 4];
+#pragma unroll
+            for (int j = 0; j < ENT / 4; ++j) acc[j] = make_float2(kPackBase, kPackBase);
+            float dev = 0.0f;
+#pragma unroll
+            for (int j = 0; j < ENT / 8; ++j) {
+                uint4 rx = make_uint4(0u, 0u, 0u, 0u), ry = rx;
+                if (RND == 1) {
+                    const uint64_t cx = gx + p * (ENT / 8) + j, cy = gy + p * (ENT / 8) + j;
+                    rx = philox4x32_10(make_uint4(static_cast<uint32_t>(cx), static_cast<uint32_t>(cx >> 32),
+                                                  a.stream, 0u), a.keys);
+                    ry = philox4x32_10(make_uint4(static_cast<uint32_t>(cy), static_cast<uint32_t>(cy >> 32),
+                                                  a.stream, 0u), a.keys);
+                }
+                const uint32_t wx[4] = {rx.x, rx.y, rx.z, rx.w}, wy[4] = {ry.x, ry.y, ry.z, ry.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int i = 8 * j + e;
+                    const int b = i / BLK;
+                    const float2 y = __fmul2_rn(v[i], make_float2(inv[b], inv[NBP + b]));
+                    float2 t;
+                    if (RND == 1) {
+                        const float2 ya = make_float2(fminf(fabsf(y.x), gk.top), fminf(fabsf(y.y), gk.top));
+                        const float2 rf =
+                            make_float2(r16_magic(wx[e >> 1], e & 1), r16_magic(wy[e >> 1], e & 1));
+                        // 1/2 - r16 2^-16, exact: (2^23 + r16) 2^-16 = 128 + r16 2^-16
+                        const float2 c = __ffma2_rn(rf, make_float2(-1.0f / 65536.0f, -1.0f / 65536.0f),
+                                                    make_float2(128.5f, 128.5f));
+                        const float2 ta = __fadd2_rn(ya, c);
+                        t = make_float2(
+                            __uint_as_float(__float_as_uint(ta.x) ^ (__float_as_uint(v[i].x) & 0x80000000u)),
+                            __uint_as_float(__float_as_uint(ta.y) ^ (__float_as_uint(v[i].y) & 0x80000000u)));
+                    } else {
+                        t = y;
+                    }
+                    const float2 f = __fadd2_rn(t, kR2);
+                    const float2 g = __fadd2_rn(f, kRn2);
+                    const float2 d = __ffma2_rn(g, m1, t);
+                    dev = max3(dev, fabsf(d.x), fabsf(d.y));
+                    const float wgt = static_cast<float>(1 << (4 * (i & 3)));
+                    acc[i >> 2] = __ffma2_rn(g, make_float2(wgt, wgt), acc[i >> 2]);
+                }
+            }
+            risky |= dev > 0.5f - kMargin;
+#pragma unroll
+            for (int j = 0; j < ENT / 8; ++j) {
+                cw[p * (ENT / 8) + j] = offset_to_sign_magnitude(
+                    prmt(__float_as_uint(acc[2 * j].x), __float_as_uint(acc[2 * j + 1].x), 0x5410u));
+                cw[4 + p * (ENT / 8) + j] = offset_to_sign_magnitude(
+                    prmt(__float_as_uint(acc[2 * j].y), __float_as_uint(acc[2 * j + 1].y), 0x5410u));
+            }
+        }
+    }
+    if (risky) return true;        // decided again by the warp (coop_exact)
+    store_run<BLK>(a, site.row_x, site.k_x, cw, st);
+    store_run<BLK>(a, site.row_y, site.k_y, cw + 4, st + NB);
+    return false;
+}
+
+template <int MAP, bool SWZ, int NH>
+__device__ __forceinline__ float amax_thread(const QuantArgs &a, const Src &src) {
+    constexpr int ENT = NH <= 16 ? 16 : 32;
+    float m = 0.0f;
+#pragma unroll
+    for (int p = 0; p < 32 / ENT; ++p) {
+        float2 v[ENT];
+        if (p == 0) load_entries<MAP, SWZ, NH, 0, ENT>(a, src, v);
+        else load_entries<MAP, SWZ, NH, (32 / ENT > 1 ? ENT : 0), ENT>(a, src, v);
+        rht_entries<NH, ENT>(v);
+#pragma unroll
+        for (int i = 0; i < ENT; ++i) m = max3(m, fabsf(v[i].x), fabsf(v[i].y));
+    }
+    return m;
+}
+
+// Two-level tensor scale of one output: S maps the rotated tensor amax to
+// gmax * 448 (the top of E4M3), G = gmax * S is the block-scale divisor.
+__device__ __forceinline__ void tensor_scale(const QuantArgs &q, const GridK &gk, float &S, float &G) {
+    const float amax_t = *q.amax_t;
+    S = amax_t > 0.0f ? __fdiv_rn(amax_t, gk.gmax * 448.0f) : 1.0f;
+    G = __fmul_rn(gk.gmax, S);
+    if (blockIdx.x == 0 && threadIdx.x == 0 && q.S_out) *q.S_out = S;
+}
+
+// One thread's part of a unit over the staged tile; `q` is the output it
+// fills.  Warp-uniform call: threads whose fast decision was not certified
+// are decided again by the whole warp.
+template <int MAP, bool SWZ, int NH, int BLK, int GRID, int RND, bool AMAX_ONLY>
+__device__ __forceinline__ void unit_part(const QuantArgs &q, const uint8_t *tile, const Src &src, const Site &site,
+                                          float S, float G, const GridK &gk, float &amax_acc) {
+    if constexpr (AMAX_ONLY) {
+        amax_acc = fmaxf(amax_acc, amax_thread<MAP, SWZ, NH>(q, src));
+    } else {
+        const bool risky = quant_thread<MAP, SWZ, NH, BLK, GRID, RND>(q, src, site, S, G, gk);
+        const uint32_t owners = __ballot_sync(0xFFFFFFFFu, risky);
+        if (owners != 0u) {
+            const uint32_t pofs = static_cast<uint32_t>(src.p - tile);
+            if (GRID == 1) coop_exact<MAP, SWZ, NH, BLK, 1, RND>(q, tile, pofs, src.off8, site, S, G, owners);
+            else if (q.grid == 0) coop_exact<MAP, SWZ, NH, BLK, 0, RND>(q, tile, pofs, src.off8, site, S, G, owners);
+            else coop_exact<MAP, SWZ, NH, BLK, 2, RND>(q, tile, pofs, src.off8, site, S, G, owners);
         }
     }
 }
 
 // `a` drives the units (AXIS 0: row-wise output; AXIS 1 and 2: column-wise
 // output); `a2` is the row-wise output of AXIS 2 and unused otherwise.
+//   AXIS 0  one 64 (K) x 256 (rows) box, 128-byte swizzle: thread t takes
+//           tile row t (row map);
+//   AXIS 1  four 64 (columns) x 64 (K rows) boxes, no swizzle (a warp's
+//           32-bit loads of one K row are 128 consecutive bytes): warp w
+//           takes box w & 3, K half w >> 2, lane l columns 2l, 2l + 1 (col2),
+//           or for n = 64 thread t takes column t & 63 of box t >> 6 (col1);
+//   AXIS 2  the AXIS 1 tile with the 128-byte swizzle quantized twice:
+//           column-wise into `a` as AXIS 1, then row-wise into `a2` (thread t
+//           takes row t & 63 of box t >> 6: 64 columns of one input row).
+//           One read of the tensor serves both of its GEMM operands.
 template <int AXIS, int NH, int BLK, int GRID, int RND, bool AMAX_ONLY>
-__global__ void __launch_bounds__(kCtaThreads, ctas_per_sm<AXIS>()) rht_quantize_kernel(const __grid_constant__ QuantArgs a,
-                                                                  const __grid_constant__ QuantArgs a2,
-                                                                  const __grid_constant__ CUtensorMap tmap) {
+__global__ void __launch_bounds__(kCtaThreads, kCtasPerSm)
+    rht_quantize_kernel(const __grid_constant__ QuantArgs a, const __grid_constant__ QuantArgs a2,
+                        const __grid_constant__ CUtensorMap tmap) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -711,6 +795,7 @@ __global__ void __launch_bounds__(kCtaThreads, ctas_per_sm<AXIS>()) rht_quantize
     const int64_t nseg = a.kpad / 64;
     const int64_t nrb = (a.out_rows + kUnitRows - 1) / kUnitRows;
     const int64_t nunits = nseg * nrb;
+    constexpr bool kSwz = AXIS != 1;
 
     auto unit_coords = [&](int64_t u, int64_t &rb, int64_t &seg) {
         if (AXIS == 0) {
@@ -769,33 +854,24 @@ __global__ void __launch_bounds__(kCtaThreads, ctas_per_sm<AXIS>()) rht_quantize
         return;
     }
 
+    const GridK gk = grid_constants(a.grid);
     float S = 1.0f, G = 0.0f, S2 = 1.0f, G2 = 0.0f;
-    if (!AMAX_ONLY && a.scale_fmt == 1) tensor_scale<GRID>(a, S, G);
-    if (AXIS == 2 && !AMAX_ONLY && a2.scale_fmt == 1) tensor_scale<GRID>(a2, S2, G2);
-    // D for the 64 positions of a segment (K offsets are multiples of 64).
-    uint64_t pat = 0;
-    if (NH > 0) {
-        const uint64_t m = NH == 64 ? a.sign_mask : (a.sign_mask & ((1ull << NH) - 1));
-#pragma unroll
-        for (int off = 0; off < 64; off += (NH > 0 ? NH : 64)) pat |= m << off;
-    }
-    const uint32_t pat_lo = static_cast<uint32_t>(pat), pat_hi = static_cast<uint32_t>(pat >> 32);
-    // Sign of D at position i mod 16 as an fp32 sign bit (NH <= 16; adding it
-    // to a widened bf16 flips the sign bit like an xor) and the Philox round
-    // keys: both from the parameter bank, no registers held.
-    const uint32_t (&smask)[16] = a.smask;
-    const PhiloxKeys &keys = a.keys;
+    if (!AMAX_ONLY && a.scale_fmt == 1) tensor_scale(a, gk, S, G);
+    if (AXIS == 2 && !AMAX_ONLY && a2.scale_fmt == 1) tensor_scale(a2, gk, S2, G2);
     float amax_acc = 0.0f, amax_acc2 = 0.0f;
 
-    // Column-wise: byte offset of column cc (= t & 63) within K row r of a
-    // 64-column box for r % 8 (the 128-byte swizzle XORs the 16-byte chunk
-    // index with the row mod 8).
-    uint32_t col_off[8];
-    {
-        const int cc = t & 63;
+    // Column maps: byte offsets of the thread's column(s) within a K row r
+    // of a 64-column box, for r % 8 = j (the 128-byte swizzle XORs the
+    // 16-byte chunk index with the row mod 8).
+    constexpr int CMAP = NH == 64 ? MAP_COL1 : MAP_COL2;
+    Src csrc;
+    csrc.p = nullptr;
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
-            col_off[r] = static_cast<uint32_t>((t >> 6) * 8192 + ((((cc >> 3) ^ r) & 7) << 4) + (cc & 7) * 2);
+    for (int j = 0; j < 8; ++j) {
+        const int jj = kSwz ? j : 0;
+        csrc.off8[j] = CMAP == MAP_COL2
+                           ? static_cast<uint32_t>((((lane >> 2) ^ jj) << 4) + 4 * (lane & 3))
+                           : static_cast<uint32_t>(((((t & 63) >> 3) ^ jj) << 4) + 2 * (t & 7));
     }
     uint32_t it = 0;
     for (int64_t u = u0; u < nunits; u += gridDim.x, ++it) {
@@ -805,21 +881,43 @@ __global__ void __launch_bounds__(kCtaThreads, ctas_per_sm<AXIS>()) rht_quantize
         unit_coords(u, rb, seg);
         const uint8_t *tile = smem + s * kStageBytes;
         if (AXIS == 0) {
-            quantize64<0, NH, BLK, GRID, RND, AMAX_ONLY>(a, tile + t * 128, t & 7, col_off, rb * kUnitRows + t,
-                                                         seg * 64, S, G, keys, smask, pat_lo, pat_hi,
-                                                         amax_acc);
+            Src src;
+            src.p = tile + t * 128;
+            src.off8[0] = static_cast<uint32_t>(t & 7);
+            const int32_t row = static_cast<int32_t>(rb * kUnitRows + t);
+            const int32_t k0 = static_cast<int32_t>(seg * 64);
+            const Site site{row, row, k0, k0 + 32};
+            unit_part<MAP_ROW, true, NH, BLK, GRID, RND, AMAX_ONLY>(a, tile, src, site, S, G, gk, amax_acc);
         } else {
-            quantize64<1, NH, BLK, GRID, RND, AMAX_ONLY>(a, tile, 0, col_off, rb * kUnitRows + t, seg * 64, S,
-                                                         G, keys, smask, pat_lo, pat_hi, amax_acc);
+            Src src = csrc;
+            Site site;
+            if (CMAP == MAP_COL2) {
+                const int box = warp & 3, half = warp >> 2;
+                src.p = tile + box * 8192 + half * 32 * 128;
+                const int32_t row = static_cast<int32_t>(rb * kUnitRows + 64 * box + 2 * lane);
+                const int32_t k0 = static_cast<int32_t>(seg * 64 + 32 * half);
+                site = Site{row, row + 1, k0, k0};
+            } else {
+                src.p = tile + (t >> 6) * 8192;
+                const int32_t row = static_cast<int32_t>(rb * kUnitRows + t);
+                const int32_t k0 = static_cast<int32_t>(seg * 64);
+                site = Site{row, row, k0, k0 + 32};
+            }
+            unit_part<CMAP, kSwz, NH, BLK, GRID, RND, AMAX_ONLY>(a, tile, src, site, S, G, gk, amax_acc);
             if (AXIS == 2) {
                 // Row-wise output: input row 64 seg + (t & 63), K columns from
                 // 256 rb + 64 (t >> 6).  Boxes past the padded K (the last
                 // column block of a ragged width) are skipped, per warp.
                 const int64_t k0 = rb * kUnitRows + 64 * (t >> 6);
-                if (k0 < a2.kpad)
-                    quantize64<0, NH, BLK, GRID, RND, AMAX_ONLY>(a2, tile + (t >> 6) * 8192 + (t & 63) * 128, t & 7,
-                                                                 col_off, seg * 64 + (t & 63), k0, S2, G2, keys,
-                                                                 smask, pat_lo, pat_hi, amax_acc2);
+                if (k0 < a2.kpad) {
+                    Src rs;
+                    rs.p = tile + (t >> 6) * 8192 + (t & 63) * 128;
+                    rs.off8[0] = static_cast<uint32_t>(t & 7);
+                    const int32_t row = static_cast<int32_t>(seg * 64 + (t & 63));
+                    const Site rsite{row, row, static_cast<int32_t>(k0), static_cast<int32_t>(k0 + 32)};
+                    unit_part<MAP_ROW, true, NH, BLK, GRID, RND, AMAX_ONLY>(a2, tile, rs, rsite, S2, G2, gk,
+                                                                             amax_acc2);
+                }
             }
         }
         __syncwarp();      // this warp is done with stage s
@@ -838,8 +936,60 @@ __global__ void __launch_bounds__(kCtaThreads, ctas_per_sm<AXIS>()) rht_quantize
     }
 }
 
+
+// ---------------------------------------------------------------------------
+// Unfused RHT (the baseline the fused kernel is compared with, [GS]
+// "Efficiëntie"): y = bf16_RN(H_n D x) along the contiguous dimension, the
+// same fp32 butterflies as the quantizer, one 64-element row segment per
+// thread (global loads and stores of 128 contiguous bytes), grid-stride.
+template <int NH>
+__global__ void __launch_bounds__(256) rht_bf16_kernel(const __grid_constant__ QuantArgs a, uint16_t *y,
+                                                        int64_t ldy) {
+    const int64_t nseg = a.cols / 64;
+    const int64_t total = a.rows * nseg;
+    for (int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; w < total;
+         w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = w / nseg, seg = w % nseg;
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.x + r * a.ld + seg * 64);
+        float v[64];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 q = src[c];
+            const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = 8 * c + 2 * e;
+                v[i] = lo_f(wd[e], NH ? a.smask[i] : 0u);
+                v[i + 1] = hi_f(wd[e], NH ? a.smask[i + 1] : 0u);
+            }
+        }
+#pragma unroll
+        for (int h = 1; h < NH; h <<= 1) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                if (i & h) continue;
+                const float x0 = v[i], x1 = v[i + h];
+                v[i] = __fadd_rn(x0, x1);
+                v[i + h] = __fsub_rn(x0, x1);
+            }
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(y + r * ldy + seg * 64);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const __nv_bfloat162 b = __floats2bfloat162_rn(v[8 * c + 2 * e], v[8 * c + 2 * e + 1]);
+                o[e] = *reinterpret_cast<const uint32_t *>(&b);
+            }
+            dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
 // Host side of the per-call constants: Philox round keys of the seed and the
-// D sign bits of positions 0..15 (used by the kernels with NH <= 16).
+// D sign bit of every position 0..63 of a lane run (the n-bit mask repeated
+// with period n).
 void fill_call_constants(QuantArgs &a, int hadamard_n) {
     uint32_t kx = static_cast<uint32_t>(a.seed), ky = static_cast<uint32_t>(a.seed >> 32);
     for (int r = 0; r < 10; ++r) {
@@ -848,8 +998,8 @@ void fill_call_constants(QuantArgs &a, int hadamard_n) {
         kx += 0x9E3779B9u;
         ky += 0xBB67AE85u;
     }
-    for (int i = 0; i < 16; ++i)
-        a.smask[i] = hadamard_n > 0 ? static_cast<uint32_t>((a.sign_mask >> i) & 1u) << 31 : 0u;
+    for (int p = 0; p < 64; ++p)
+        a.smask[p] = hadamard_n > 0 ? static_cast<uint32_t>((a.sign_mask >> (p % hadamard_n)) & 1u) << 31 : 0u;
 }
 
 template <int AXIS, int NH, int BLK, int GRID, int RND, bool AMAX_ONLY>
@@ -863,24 +1013,21 @@ cudaError_t launch_one(const QuantArgs &a, const QuantArgs &a2, const CUtensorMa
         configured = true;
     }
     const int64_t nunits = (a.kpad / 64) * ((a.out_rows + kUnitRows - 1) / kUnitRows);
-    const int64_t cap = static_cast<int64_t>(num_sms) * ctas_per_sm<AXIS>();
+    const int64_t cap = static_cast<int64_t>(num_sms) * kCtasPerSm;
     const int grid = static_cast<int>(nunits < cap ? nunits : cap);
     if (grid <= 0) return cudaSuccess;
     rht_quantize_kernel<AXIS, NH, BLK, GRID, RND, AMAX_ONLY><<<grid, kCtaThreads, kQuantSmem, stream>>>(a, a2, tmap);
     return cudaGetLastError();
 }
 
+// grid_kind: 0 E1M2, 1 E2M1, 2 restricted E2M1 (the uniform grids share GRID 0).
 template <int AXIS, int NH, int BLK, bool AMAX_ONLY>
 cudaError_t dispatch_grid_round(const QuantArgs &a, const QuantArgs &a2, const CUtensorMap &m, int grid_kind,
                                 int rnd, int num_sms, cudaStream_t stream) {
     if (AMAX_ONLY) return launch_one<AXIS, NH, BLK, 0, 0, true>(a, a2, m, num_sms, stream);
-    if (grid_kind == 0) {
+    if (grid_kind != 1) {
         return rnd == 0 ? launch_one<AXIS, NH, BLK, 0, 0, false>(a, a2, m, num_sms, stream)
                         : launch_one<AXIS, NH, BLK, 0, 1, false>(a, a2, m, num_sms, stream);
-    }
-    if (grid_kind == 2) {
-        return rnd == 0 ? launch_one<AXIS, NH, BLK, 2, 0, false>(a, a2, m, num_sms, stream)
-                        : launch_one<AXIS, NH, BLK, 2, 1, false>(a, a2, m, num_sms, stream);
     }
     return rnd == 0 ? launch_one<AXIS, NH, BLK, 1, 0, false>(a, a2, m, num_sms, stream)
                     : launch_one<AXIS, NH, BLK, 1, 1, false>(a, a2, m, num_sms, stream);
@@ -889,6 +1036,8 @@ cudaError_t dispatch_grid_round(const QuantArgs &a, const QuantArgs &a2, const C
 template <int AXIS, bool AMAX_ONLY>
 cudaError_t dispatch_nh_blk(const QuantArgs &a, const QuantArgs &a2, const CUtensorMap &m, int nh, int blk,
                             int grid_kind, int rnd, int num_sms, cudaStream_t stream) {
+    // The amax pass has no blocks: one instantiation per Hadamard size.
+    if (AMAX_ONLY) blk = 16;
 #define UFP4_CASE(N, B)                                                                          \
     if (nh == N && blk == B)                                                                     \
         return dispatch_grid_round<AXIS, N, B, AMAX_ONLY>(a, a2, m, grid_kind, rnd, num_sms, stream);
@@ -904,15 +1053,16 @@ cudaError_t dispatch_nh_blk(const QuantArgs &a, const QuantArgs &a2, const CUten
     return cudaErrorInvalidValue;
 }
 
-// bf16 input as a 2-D tensor map: rows x cols, row pitch ld; 128-byte swizzle,
-// box 64 x 256 (row-wise: K x rows) or 64 x 64 (column-wise and dual:
-// columns x K).
-cudaError_t make_input_map(const QuantArgs &a, CUtensorMap *m) {
+// bf16 input as a 2-D tensor map: rows x cols, row pitch ld; box 64 x 256
+// (row-wise: K x rows, 128-byte swizzle) or 64 x 64 (column-wise: columns x
+// K, no swizzle; dual: 128-byte swizzle).
+cudaError_t make_input_map(const QuantArgs &a, CUtensorMap *m, bool dual) {
     const uint32_t box_outer = a.axis == 0 ? kUnitRows : 64;
+    const CUtensorMapSwizzle swz =
+        (a.axis == 0 || dual) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
     CUresult r = encode_tensor_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x,
                                       static_cast<uint64_t>(a.cols), static_cast<uint64_t>(a.rows),
-                                      static_cast<uint64_t>(a.ld) * 2, 64, box_outer,
-                                      CU_TENSOR_MAP_SWIZZLE_128B);
+                                      static_cast<uint64_t>(a.ld) * 2, 64, box_outer, swz);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
@@ -921,8 +1071,9 @@ cudaError_t make_input_map(const QuantArgs &a, CUtensorMap *m) {
 cudaError_t launch_rht_quantize(QuantArgs a, int hadamard_n, int block, int grid_kind,
                                 int rounding, int num_sms, cudaStream_t stream) {
     fill_call_constants(a, hadamard_n);
+    a.grid = grid_kind;
     CUtensorMap m;
-    cudaError_t e = make_input_map(a, &m);
+    cudaError_t e = make_input_map(a, &m, false);
     if (e != cudaSuccess) return e;
     if (a.axis == 0)
         return dispatch_nh_blk<0, false>(a, a, m, hadamard_n, block, grid_kind, rounding, num_sms, stream);
@@ -933,8 +1084,9 @@ cudaError_t launch_rht_quantize_dual(QuantArgs a_rows, QuantArgs a_cols, int had
                                      int grid_kind, int rounding, int num_sms, cudaStream_t stream) {
     fill_call_constants(a_rows, hadamard_n);
     fill_call_constants(a_cols, hadamard_n);
+    a_rows.grid = a_cols.grid = grid_kind;
     CUtensorMap m;
-    cudaError_t e = make_input_map(a_rows, &m);
+    cudaError_t e = make_input_map(a_rows, &m, true);
     if (e != cudaSuccess) return e;
     return dispatch_nh_blk<2, false>(a_rows, a_cols, m, hadamard_n, block, grid_kind, rounding, num_sms,
                                      stream);
@@ -942,10 +1094,11 @@ cudaError_t launch_rht_quantize_dual(QuantArgs a_rows, QuantArgs a_cols, int had
 
 cudaError_t launch_rht_amax(QuantArgs a, int hadamard_n, int num_sms, cudaStream_t stream) {
     fill_call_constants(a, hadamard_n);
+    a.grid = 0;
     cudaError_t e = cudaMemsetAsync(a.amax_out, 0, sizeof(float), stream);
     if (e != cudaSuccess) return e;
     CUtensorMap m;
-    e = make_input_map(a, &m);
+    e = make_input_map(a, &m, false);
     if (e != cudaSuccess) return e;
     if (a.axis == 0) return dispatch_nh_blk<0, true>(a, a, m, hadamard_n, 16, 0, 0, num_sms, stream);
     return dispatch_nh_blk<1, true>(a, a, m, hadamard_n, 16, 0, 0, num_sms, stream);
@@ -955,13 +1108,32 @@ cudaError_t launch_rht_amax_dual(QuantArgs a_rows, QuantArgs a_cols, int hadamar
                                  cudaStream_t stream) {
     fill_call_constants(a_rows, hadamard_n);
     fill_call_constants(a_cols, hadamard_n);
+    a_rows.grid = a_cols.grid = 0;
     cudaError_t e = cudaMemsetAsync(a_rows.amax_out, 0, sizeof(float), stream);
     if (e == cudaSuccess) e = cudaMemsetAsync(a_cols.amax_out, 0, sizeof(float), stream);
     if (e != cudaSuccess) return e;
     CUtensorMap m;
-    e = make_input_map(a_rows, &m);
+    e = make_input_map(a_rows, &m, true);
     if (e != cudaSuccess) return e;
     return dispatch_nh_blk<2, true>(a_rows, a_cols, m, hadamard_n, 16, 0, 0, num_sms, stream);
+}
+
+cudaError_t launch_rht_bf16(QuantArgs a, int hadamard_n, uint16_t *y, int64_t ldy, int num_sms,
+                            cudaStream_t stream) {
+    fill_call_constants(a, hadamard_n);
+    const int64_t total = a.rows * (a.cols / 64);
+    if (total == 0) return cudaSuccess;
+    const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+    const int64_t need = (total + 255) / 256;
+    const int grid = static_cast<int>(need < cap ? need : cap);
+    switch (hadamard_n) {
+        case 0: rht_bf16_kernel<0><<<grid, 256, 0, stream>>>(a, y, ldy); break;
+        case 16: rht_bf16_kernel<16><<<grid, 256, 0, stream>>>(a, y, ldy); break;
+        case 32: rht_bf16_kernel<32><<<grid, 256, 0, stream>>>(a, y, ldy); break;
+        case 64: rht_bf16_kernel<64><<<grid, 256, 0, stream>>>(a, y, ldy); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
 }
 
 cudaError_t quantize_read_and_clear_error_word(uint32_t *out) {

@@ -31,16 +31,20 @@ struct QuantArgs {
     uint32_t stream;
     uint64_t sign_mask;
     int scale_fmt;
+    int grid;            // ufp4_grid_t (filled by the launcher)
     int64_t num_units;   // filled by the launcher
     // Per-call constants the kernels read from the parameter bank instead of
     // holding in registers (filled by the launcher from seed / sign_mask):
     PhiloxKeys keys;     // round keys of `seed`
-    uint32_t smask[16];  // D sign of position i mod 16, as an fp32 sign bit
+    uint32_t smask[64];  // D sign of lane-run position p (period n), fp32 sign bit
 };
 
 cudaError_t launch_rht_quantize(QuantArgs a, int hadamard_n, int block, int grid_kind,
                                 int rounding, int num_sms, cudaStream_t stream);
 cudaError_t launch_rht_amax(QuantArgs a, int hadamard_n, int num_sms, cudaStream_t stream);
+// Unfused RHT: y = bf16(H_n D x) along cols (cols % 64 == 0).
+cudaError_t launch_rht_bf16(QuantArgs a, int hadamard_n, uint16_t *y, int64_t ldy, int num_sms,
+                            cudaStream_t stream);
 // One read of the input, both outputs: a_rows (axis 1, drives the units) and
 // a_cols (axis 0); same grid / rounding / RHT / block for both.
 cudaError_t launch_rht_quantize_dual(QuantArgs a_rows, QuantArgs a_cols, int hadamard_n, int block,

@@ -31,7 +31,7 @@ EXPORTED = [
     "ufp4_gemm_dgrad", "ufp4_gemm_wgrad", "ufp4_grouped_gemm", "ufp4_check_device_status",
     "ufp4_status_string", "ufp4_version", "ufp4_set_two_level_gemm_path",
     "ufp4_get_two_level_gemm_path", "ufp4_rht_quantize_dual", "ufp4_rht_amax_dual",
-    "ufp4_quant_stats", "ufp4_qstats_summarize", "ufp4_sqnr_sums",
+    "ufp4_quant_stats", "ufp4_qstats_summarize", "ufp4_sqnr_sums", "ufp4_rht_bf16",
 ]
 
 
@@ -94,6 +94,8 @@ def lib() -> ctypes.CDLL:
                                           ctypes.POINTER(ctypes.c_size_t)]
         L.ufp4_rht_amax.restype = st
         L.ufp4_rht_amax.argtypes = [P, i64, i64, i64, i32, i32, u64, P, P]
+        L.ufp4_rht_bf16.restype = st
+        L.ufp4_rht_bf16.argtypes = [P, i64, i64, i64, i32, u64, P, i64, P]
         L.ufp4_rht_quantize.restype = st
         L.ufp4_rht_quantize.argtypes = [P, i64, i64, i64, i32, P, ctypes.POINTER(QTensorC), P]
         L.ufp4_quant_stats.restype = st
@@ -230,6 +232,21 @@ def rht_amax(x: torch.Tensor, axis: int, hadamard_n: int,
     _check(lib().ufp4_rht_amax(ctypes.c_void_p(x.data_ptr()), rows, cols, x.stride(0), axis,
                                hadamard_n, sign_mask, ctypes.c_void_p(out.data_ptr()),
                                _stream_ptr(x.device)), "ufp4_rht_amax")
+    return out
+
+
+def rht_bf16(x: torch.Tensor, hadamard_n: int, sign_mask: int = DEFAULT_SIGN_MASK,
+             out: torch.Tensor | None = None) -> torch.Tensor:
+    """Unfused RHT along the columns: bf16(H_n D x) of every n-block of every
+    row (the separate pass the fused quantizer is compared with)."""
+    _require_cuda(x)
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    if out is None:
+        out = torch.empty_like(x, memory_format=torch.contiguous_format)
+    rows, cols = x.shape
+    _check(lib().ufp4_rht_bf16(ctypes.c_void_p(x.data_ptr()), rows, cols, x.stride(0), hadamard_n,
+                               sign_mask, ctypes.c_void_p(out.data_ptr()), out.stride(0),
+                               _stream_ptr(x.device)), "ufp4_rht_bf16")
     return out
 
 

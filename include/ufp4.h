@@ -171,6 +171,22 @@ ufp4_status_t ufp4_rht_amax(const void *x_dev, int64_t rows, int64_t cols, int64
                             int32_t axis, int32_t hadamard_n, uint64_t rht_sign_mask,
                             float *amax_dev, void *stream);
 
+/* Unfused RHT, the baseline of [GS] "Efficiëntie" (kernel fusion: the
+ * pages time RHT fused into the FP4 quantizer against a separate RHT pass
+ * followed by quantization).  y = bf16_RN(H_n D x) along the contiguous
+ * dimension, per n-block of each row, with the quantizer's fp32 butterflies
+ * (stages h = 1 .. n/2) and sign mask convention; n = 0 copies x.
+ *   x_dev  bf16 [rows][ld], 16-byte aligned, ld % 8 == 0, cols % 64 == 0.
+ *   y_dev  bf16 [rows][ldy] (caller-owned, 16-byte aligned, ldy % 8 == 0,
+ *          ldy >= cols); may not overlap x.
+ * Quantizing y with hadamard_n = 0 approximates ufp4_rht_quantize(x, n): the
+ * rotated values pass through bf16 in between, so codes may differ where that
+ * rounding moves a value across a decision boundary.
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (n not in {0,16,32,64}, cols
+ * not a multiple of 64), CUDA. */
+ufp4_status_t ufp4_rht_bf16(const void *x_dev, int64_t rows, int64_t cols, int64_t ld, int32_t hadamard_n,
+                            uint64_t rht_sign_mask, void *y_dev, int64_t ldy, void *stream);
+
 /* Fused RHT + block absmax + scale + 4-bit rounding + packing ([PL] §2
  * "Blockwise quantization", "Rounding rules", "Random Hadamard transforms";
  * [PL] §5 and [GS] "Efficiëntie": RHT fused into the quantizer).

@@ -156,6 +156,14 @@ def test_quantize_validation_rejects_before_launch(L):
     assert Q(x, 64, 128, 128, 0, None, ctypes.byref(two), None) == ufp4.ERR_INVALID_ARG   # no amax
     assert L.ufp4_rht_amax(x, 64, 128, 128, 0, 8, 0, ctypes.c_void_p(4096), None) == ufp4.ERR_UNSUPPORTED
     assert L.ufp4_rht_amax(x, 64, 128, 128, 0, 16, 0, None, None) == ufp4.ERR_INVALID_ARG
+    R = L.ufp4_rht_bf16
+    y = ctypes.c_void_p(8192)
+    assert R(x, 64, 128, 128, 8, 0, y, 128, None) == ufp4.ERR_UNSUPPORTED       # n
+    assert R(x, 64, 136, 136, 16, 0, y, 136, None) == ufp4.ERR_UNSUPPORTED     # cols % 64
+    assert R(x, 64, 128, 128, 16, 0, None, 128, None) == ufp4.ERR_INVALID_ARG   # no output
+    assert R(x, 64, 128, 128, 16, 0, y, 64, None) == ufp4.ERR_INVALID_ARG       # ldy < cols
+    assert R(x, 64, 128, 128, 16, 0, ctypes.c_void_p(8200), 128, None) == ufp4.ERR_ALIGNMENT
+    assert R(x, 0, 128, 128, 16, 0, None, 0, None) == ufp4.OK                   # empty: no launch
 
 
 def test_dual_quantize_validation_rejects_before_launch(L):

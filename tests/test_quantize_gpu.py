@@ -245,3 +245,23 @@ def test_quantize_ue8m0_exponent_edges(grid):
         cfg = ufp4.QuantConfig(grid=grid, rounding=rounding, sr_seed=3, hadamard_n=0, block=32,
                                scale_fmt=ufp4.SCALE_UE8M0)
         _run(X, ufp4.ALONG_COLS, cfg)
+
+
+# ------------------------------------------------------------------ unfused RHT
+@pytest.mark.parametrize("n", [0, 16, 32, 64])
+def test_rht_bf16_matches_oracle_rotation(n):
+    """The unfused RHT pass equals the oracle's rotated values (the same fp32
+    butterflies) rounded to bf16 with round-to-nearest-even, bit for bit, on a
+    ragged row count with outlier channels and a strided input view."""
+    X = wl.normal_with_outlier_channels(200, 320, 1.0, 4, 30.0)
+    cfg = ufp4.QuantConfig(hadamard_n=n)
+    x_full = to_dev(np.concatenate([X, np.zeros((200, 64), np.uint16)], axis=1))
+    x = x_full[:, :320]                       # ld = 384, cols = 320
+    y = ufp4.rht_bf16(x, n, cfg.rht_sign_mask)
+    torch.cuda.synchronize()
+    _, u = oracle.quantize(X, oracle.ALONG_COLS, oracle_cfg(cfg), want_u=True)
+    want = wl.bf16_bits(u[:, :320])
+    got = y.cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, want)
+    with pytest.raises(ufp4.UFP4Error):
+        ufp4.rht_bf16(to_dev(X[:, :136]), n)          # cols not a multiple of 64
