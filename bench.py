@@ -1,25 +1,30 @@
 """Benchmark of the UFP4 hot path on B200.
 
-One step = the whole data-parallel hot path of one linear layer of LLM
+One step = the whole data-parallel hot path of one large linear layer of LLM
 pretraining under the UFP4 recipe: RHT + block-scale + 4-bit quantize of every
 GEMM operand along its reduction dimension (X and W: RTNE; dY: stochastic
 rounding, Philox seed 1234) and the three training GEMMs
     FPROP Y = X W^T,  DGRAD dX = dY W,  WGRAD dW = dY^T X
-on X [8192, 2048] ~ N(0,1) with 10 outlier channels x30, W [8192, 2048]
-~ N(0, 0.02), dY [8192, 8192] ~ N(0, 1e-3); RHT16, scale block 16, E1M2 grid.
+on X [16384, 8192] ~ N(0,1) with 82 (1%) outlier channels x50, W [28672, 8192]
+~ N(0, 0.01), dY [16384, 28672] ~ N(0, 1e-4); RHT16, scale block 16, E1M2 grid
+with two-level (E4M3 block x fp32 tensor) scales.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--scale two-level|fp32]
+                    [--scale two-level|fp32] [--workload large|layer] [--quick]
 
 Prints one JSON line (rank 0).  `value` is the effective UFP4 GEMM throughput of
-the whole step: 3 * 2*M*N*K / step time (quantization included).  Multi-GPU
-runs are independent replicas (the path has no exchange step): weak scaling,
-time = max over ranks.
+the whole step: 3 * 2*M*N*K / step time (quantization included).  The line also
+carries the E2M1-RTNE baseline of the same layer, the quantizer sweep over the
+three sweep tensors, the fused-vs-unfused RHT ratio, the grouped MoE GEMMs, the
+quantization diagnostics, the MX block-32 FPROP, the end-to-end figure through
+host buffers and the CPU oracle baseline.  Multi-GPU runs are independent
+replicas (the path has no exchange step): weak scaling, time = max over ranks.
 """
 from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -35,10 +40,12 @@ import torch  # noqa: E402
 from fp4_quantized_gemms_b200 import workloads as wl  # noqa: E402
 
 METRIC = "UFP4 GEMM TFLOPS & % tensor peak; RHT-quantize HBM GB/s & % of 8 TB/s"
-SHAPE = wl.LAYER
+SHAPES = {"large": wl.LARGE, "layer": wl.LAYER}
 SR_SEED = 1234
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+HBM_SPEC_GBS = 8000.0
 L2_BYTES = 126 * 1024 * 1024
+FP4_OVER_BF16 = 4.0          # nominal dense fp4 / bf16 tensor rates (9 / 2.25 PFLOP/s)
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
@@ -66,17 +73,19 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def workload_desc(scale: str) -> dict:
-    s = SHAPE
+def workload_desc(shape, scale: str) -> dict:
+    s = shape
+    n_out = int(round(s.x_outlier_frac * s.K))
+    name = "large dense layer" if s is wl.LARGE else "one linear layer"
     return {
-        "workload": (f"one linear layer, all three GEMMs: X bf16 {s.M}x{s.K} ~N(0,1) with 0.5% "
-                     f"outlier channels x30, W bf16 {s.N}x{s.K} ~N(0,0.02), dY bf16 {s.M}x{s.N} "
-                     f"~N(0,1e-3); RHT16 on every operand along its K, block 16, E1M2; "
-                     f"RTNE X/W, SR (Philox seed {SR_SEED}) dY"),
+        "workload": (f"{name}, all three GEMMs: X bf16 {s.M}x{s.K} ~N(0,1) with {n_out} "
+                     f"({s.x_outlier_frac:.1%}) outlier channels x{s.x_outlier_factor:g}, W bf16 "
+                     f"{s.N}x{s.K} ~N(0,{s.w_std:g}), dY bf16 {s.M}x{s.N} ~N(0,{s.dy_std:g}); RHT16 on "
+                     f"every operand along its K, block 16, E1M2; RTNE X/W, SR (Philox seed {SR_SEED}) dY"),
         "scales": "E4M3 block x fp32 tensor (two-level)" if scale == "two-level" else "fp32 per block",
         "M": s.M, "K": s.K, "N": s.N,
         "gemm_flops_per_step": 3 * 2 * s.M * s.N * s.K,
-        "l2": "inputs larger than L2: one step reads and writes ~0.9 GB (outputs 0.4 GB)",
+        "l2": "inputs larger than L2: every operand and output of a step is larger than the 126 MB L2",
     }
 
 
@@ -140,22 +149,28 @@ def to_dev(bits: np.ndarray, device) -> torch.Tensor:
 
 
 class LayerStep:
-    """Preallocated buffers and one call sequence of the hot path."""
+    """Preallocated buffers and one call sequence of the hot path of a layer:
+    grid E1M2 (the recipe: RTNE on X and W, SR on dY) or E2M1 (the baseline
+    grid, RTNE on every operand)."""
 
-    def __init__(self, device, scale: str):
+    def __init__(self, device, scale: str, shape, inputs, grid: int | None = None):
         from fp4_quantized_gemms_b200 import ufp4
         self.u = ufp4
         self.dev = device
+        self.shape = shape
+        self.grid = ufp4.GRID_E1M2 if grid is None else grid
         two = scale == "two-level"
         fmt = ufp4.SCALE_E4M3_X_FP32 if two else ufp4.SCALE_FP32
-        base = ufp4.QuantConfig(grid=ufp4.GRID_E1M2, hadamard_n=16, block=16, scale_fmt=fmt)
+        base = ufp4.QuantConfig(grid=self.grid, hadamard_n=16, block=16, scale_fmt=fmt)
         self.two = two
         self.c_rtne = base
-        self.c_sr0 = base.with_(rounding=ufp4.ROUND_SR, sr_seed=SR_SEED, sr_stream=0)
-        self.c_sr1 = base.with_(rounding=ufp4.ROUND_SR, sr_seed=SR_SEED, sr_stream=1)
-        s = SHAPE
-        X, W, dY = wl.layer_inputs(s)
-        self.X, self.W, self.dY = to_dev(X, device), to_dev(W, device), to_dev(dY, device)
+        if self.grid == ufp4.GRID_E1M2:
+            self.c_sr0 = base.with_(rounding=ufp4.ROUND_SR, sr_seed=SR_SEED, sr_stream=0)
+            self.c_sr1 = base.with_(rounding=ufp4.ROUND_SR, sr_seed=SR_SEED, sr_stream=1)
+        else:
+            self.c_sr0 = self.c_sr1 = base
+        s = shape
+        self.X, self.W, self.dY = inputs
         C, R = ufp4.ALONG_COLS, ufp4.ALONG_ROWS
         E = ufp4.empty_qtensor
         self.qx = E(s.M, s.K, self.c_rtne, device)        # FPROP A
@@ -164,10 +179,10 @@ class LayerStep:
         self.qwt = E(s.K, s.N, self.c_rtne, device)       # DGRAD B
         self.qdyt = E(s.N, s.M, self.c_sr1, device)       # WGRAD A
         self.qxt = E(s.K, s.M, self.c_rtne, device)       # WGRAD B
-        # Each tensor feeds two GEMMs, one along each axis.  X and W (RTNE)
-        # go through the dual-output quantizer (one read, both results); dY
-        # (SR) through two single calls, which are faster for the ALU-bound
-        # SR path.  The rotated amaxes come from one dual pass per tensor.
+        # Each tensor feeds two GEMMs, one along each axis.  X and W go
+        # through the dual-output quantizer (one read, both results); dY
+        # through one call per axis.  The rotated amaxes of all six operands
+        # come from one dual pass per tensor.
         self.dual = [(self.X, self.qx, self.qxt), (self.W, self.qw, self.qwt)]
         self.single = [(self.dY, C, self.qdy), (self.dY, R, self.qdyt)]
         self.amax = torch.zeros(6, dtype=torch.float32, device=device)   # [cols, rows] per tensor
@@ -211,12 +226,17 @@ class LayerStep:
         self.quantize_all()
         self.gemms(events[1:] if events else None)
 
+    def free(self):
+        for name in ("qx", "qw", "qdy", "qwt", "qdyt", "qxt", "Y", "dX", "dW", "amax"):
+            setattr(self, name, None)
+
 
 def quant_bytes(step: LayerStep) -> float:
     """Algorithmic bytes of the step's quantization: each quantized element
     writes its code and its share of a block scale (fp32, or E4M3); bf16 inputs
     are read once per dual call and once per single call; with two-level
-    scales the dual amax pass reads each tensor once more."""
+    scales the dual amax pass reads each tensor once more.  The E1M2
+    correction planes the GEMM reads are not counted."""
     out_per = 0.5 + (4 / 16 if not step.two else 1 / 16)
     total = step.quant_elems * out_per
     total += sum(x.numel() for x, _, _ in step.dual) * 2
@@ -226,34 +246,187 @@ def quant_bytes(step: LayerStep) -> float:
     return total
 
 
-def run_mx(step: LayerStep, reps: int = 5) -> dict:
+def time_steps(step: LayerStep, steps: int, warmup: int, world: int, device, clocks: bool):
+    """Device-timed steps: CUDA events on the launching stream, bracketed by a
+    barrier and a synchronize on both sides; per-phase event splits."""
+    stream = torch.cuda.current_stream(device)
+    for _ in range(warmup):
+        step.step()
+    torch.cuda.synchronize(device)
+    if step.u.check_device_status() != step.u.OK:
+        raise RuntimeError("device error word set during warm-up")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    clk = ClockSampler(device.index if device.index is not None else 0) if clocks else None
+    if clk:
+        clk.__enter__()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        step.step(ev[i])
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    if clk:
+        clk.__exit__()
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = max_over_ranks(start.elapsed_time(end), world, device)
+    q_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(steps))
+    g_ms = [statistics.mean(ev[i][1 + j].elapsed_time(ev[i][2 + j]) for i in range(steps)) for j in range(3)]
+    return total_ms / steps, q_ms, g_ms, (clk.summary() if clk else None)
+
+
+# ------------------------------------------------------------------ quantizer sweep
+def _timed(fn, flush, reps: int = 5, warm: int = 2) -> float:
+    """Median of `reps` CUDA-event timings of fn, L2 flushed (256 MB write)
+    before each."""
+    for _ in range(warm):
+        fn()
+    ts = []
+    for _ in range(reps):
+        flush.add_(1.0)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    ts.sort()
+    return ts[len(ts) // 2]
+
+
+def sweep_input(rows: int, cols: int, device) -> torch.Tensor:
+    """0.1 * Student-t(nu = 4) bf16 tensor of the sweep, drawn on the device
+    from a seeded generator (the parity tests draw the same distribution with
+    the host generator of `workloads.student_t`)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(wl.SEED_STUDENT)
+    z = torch.randn((rows, cols), generator=g, device=device, dtype=torch.float32)
+    chi2 = torch.empty((rows, cols), device=device, dtype=torch.float32)
+    # chi-square with 4 degrees of freedom as -2 log(u1 u2) (two exponentials)
+    u1 = torch.rand((rows, cols), generator=g, device=device, dtype=torch.float32).clamp_(min=1e-30)
+    u2 = torch.rand((rows, cols), generator=g, device=device, dtype=torch.float32).clamp_(min=1e-30)
+    torch.mul(u1, u2, out=chi2).log_().mul_(-2.0)
+    del u1, u2
+    z.mul_(torch.rsqrt(chi2.div_(4.0))).mul_(0.1)
+    del chi2
+    return z.to(torch.bfloat16)
+
+
+def run_sweep(device, peaks, quick: bool = False) -> dict:
+    """The quantizer sweep: bf16 4096x4096, 16384x8192, 32768x16384 ~0.1 t(4);
+    Hadamard 16/32/64, block 16/32; E1M2 RTNE, E1M2 SR, E2M1 RTNE; fp32
+    scales; both axes (plus the dual-output call at n = 16, block 16).  GB/s
+    of algorithmic bytes: 2 (bf16 in) + 0.5 (codes) + 4/B (fp32 scales) per
+    element of each output (dual: 2 + 2 (0.5 + 4/B))."""
+    from fp4_quantized_gemms_b200 import ufp4 as u
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    rows_out = []
+    shapes = wl.QUANT_SWEEP_SHAPES[-1:] if quick else wl.QUANT_SWEEP_SHAPES
+    modes = [("e1m2_rtne", u.GRID_E1M2, u.ROUND_RTNE), ("e1m2_sr", u.GRID_E1M2, u.ROUND_SR),
+             ("e2m1_rtne", u.GRID_E2M1, u.ROUND_RTNE)]
+    ratio = None
+    for (R, C) in shapes:
+        x = sweep_input(R, C, device)
+        for n in (16, 32, 64):
+            for blk in (16, 32):
+                for mode, grid, rnd in modes:
+                    cfg = u.QuantConfig(grid=grid, rounding=rnd, sr_seed=SR_SEED, hadamard_n=n, block=blk,
+                                        scale_fmt=u.SCALE_FP32)
+                    for axis in (u.ALONG_COLS, u.ALONG_ROWS):
+                        q = u.rht_quantize(x, axis, cfg)
+                        ms = _timed(lambda: u.rht_quantize(x, axis, cfg, out=q), flush)
+                        gbs = R * C * (2.5 + 4 / blk) / (ms * 1e-3) / 1e9
+                        rows_out.append({"shape": [R, C], "n": n, "block": blk, "mode": mode,
+                                         "axis": ("cols", "rows")[axis], "ms": round(ms, 4),
+                                         "GBps": round(gbs, 1)})
+                        del q
+                    if n == 16 and blk == 16:
+                        qq = u.rht_quantize_dual(x, cfg)
+                        ms = _timed(lambda: u.rht_quantize_dual(x, cfg, out=qq), flush)
+                        gbs = R * C * (2 + 2 * (0.5 + 4 / blk)) / (ms * 1e-3) / 1e9
+                        rows_out.append({"shape": [R, C], "n": n, "block": blk, "mode": mode,
+                                         "axis": "dual", "ms": round(ms, 4), "GBps": round(gbs, 1)})
+                        del qq
+        if (R, C) == wl.QUANT_SWEEP_SHAPES[-1]:
+            ratio = fused_vs_unfused(x, flush)
+        del x
+        torch.cuda.empty_cache()
+    big = [r for r in rows_out if r["shape"] == list(wl.QUANT_SWEEP_SHAPES[-1])]
+
+    def best(pred):
+        sel = [r for r in big if pred(r)]
+        return max(sel, key=lambda r: r["GBps"]) if sel else None
+
+    def worst(pred):
+        sel = [r for r in big if pred(r)]
+        return min(sel, key=lambda r: r["GBps"]) if sel else None
+
+    rec = [r for r in big if r["n"] == 16 and r["block"] == 16 and r["mode"] == "e1m2_rtne"
+           and r["axis"] in ("cols", "rows")]
+    rec_gbs = min(r["GBps"] for r in rec) if rec else None
+    summary = {
+        "largest_tensor": list(wl.QUANT_SWEEP_SHAPES[-1]),
+        "recipe_e1m2_rtne_n16_b16_GBps": rec_gbs,
+        "recipe_frac_of_8TBps": round(rec_gbs / HBM_SPEC_GBS, 4) if rec_gbs else None,
+        "recipe_frac_of_measured_hbm": round(rec_gbs / hbm, 4) if rec_gbs else None,
+        "best": best(lambda r: r["axis"] != "dual"),
+        "worst": worst(lambda r: r["axis"] != "dual"),
+        "e1m2_sr_worst": worst(lambda r: r["mode"] == "e1m2_sr" and r["axis"] != "dual"),
+    }
+    return {"workload": ("quantizer sweep: bf16 4096x4096, 16384x8192, 32768x16384 ~0.1 Student-t(4) "
+                         "(device generator, seed 5); RHT 16/32/64, block 16/32; E1M2 RTNE, E1M2 SR "
+                         "(seed 1234), E2M1 RTNE; fp32 scales; both axes; L2 flushed between runs"),
+            "bytes_per_element": "2 + 0.5 + 4/B (dual: 2 + 2 (0.5 + 4/B))",
+            "hbm_peak_GBps": hbm, "summary": summary, "fused_vs_unfused": ratio, "rows": rows_out}
+
+
+def fused_vs_unfused(x: torch.Tensor, flush) -> dict:
+    """The pages' kernel-fusion comparison on the largest sweep tensor, row-wise,
+    E1M2 RTNE, block 16, fp32 scales: quantization alone (n = 0), the fused
+    RHT16 + quantization, and the unfused pair (a separate RHT pass writing
+    bf16, then quantization with n = 0)."""
+    from fp4_quantized_gemms_b200 import ufp4 as u
+    cfg16 = u.QuantConfig(hadamard_n=16, block=16)
+    cfg0 = cfg16.with_(hadamard_n=0)
+    q = u.rht_quantize(x, u.ALONG_COLS, cfg16)
+    y = torch.empty_like(x)
+    t_fused = _timed(lambda: u.rht_quantize(x, u.ALONG_COLS, cfg16, out=q), flush)
+    t_plain = _timed(lambda: u.rht_quantize(x, u.ALONG_COLS, cfg0, out=q), flush)
+    t_rht = _timed(lambda: u.rht_bf16(x, 16, out=y), flush)
+    u.rht_bf16(x, 16, out=y)
+    t_q_rot = _timed(lambda: u.rht_quantize(y, u.ALONG_COLS, cfg0, out=q), flush)
+    t_unfused = t_rht + t_q_rot
+    del y, q
+    return {"tensor": list(x.shape), "quantize_only_ms": round(t_plain, 4), "fused_rht16_ms": round(t_fused, 4),
+            "rht_pass_ms": round(t_rht, 4), "quantize_of_rotated_ms": round(t_q_rot, 4),
+            "unfused_ms": round(t_unfused, 4),
+            "fused_over_quantize_only": round(t_fused / t_plain, 3),
+            "unfused_over_quantize_only": round(t_unfused / t_plain, 3),
+            "pages": "fused ~1.06-1.07x, unfused ~1.4-1.6x of standalone quantization (SM90/SM100, "
+                     "shapes not stated; context only)"}
+
+
+# ------------------------------------------------------------------ side measurements
+def run_mx(step: LayerStep, reps: int = 3) -> dict:
     """The layer's FPROP with MX block scales (UE8M0, block 32): quantize X and
     W (dual calls) and the GEMM through the fp32-block-scale kernel, timed
     with CUDA events (reported, not in `value`)."""
     u = step.u
     cfg = u.QuantConfig(grid=u.GRID_E1M2, hadamard_n=16, block=32, scale_fmt=u.SCALE_UE8M0)
-    s = SHAPE
-    qx, qxt = u.rht_quantize_dual(step.X, cfg)
-    qw, qwt = u.rht_quantize_dual(step.W, cfg)
+    s = step.shape
+    qx, _ = u.rht_quantize_dual(step.X, cfg)
+    qw, _ = u.rht_quantize_dual(step.W, cfg)
     out = torch.empty((s.M, s.N), dtype=torch.float32, device=step.dev)
-
-    def timed(fn):
-        for _ in range(2):
-            fn()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(reps):
-            fn()
-        b.record()
-        torch.cuda.synchronize(step.dev)
-        return a.elapsed_time(b) / reps
-
-    t_q = timed(lambda: (u.rht_quantize_dual(step.X, cfg, out=(qx, qxt)),
-                         u.rht_quantize_dual(step.W, cfg, out=(qw, qwt))))
-    t_g = timed(lambda: u.gemm_fprop(qx, qw, out))
-    del out
-    return {"quantize_XW_dual_ms": round(t_q, 4), "fprop_ms": round(t_g, 4),
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=step.dev)
+    t_g = _timed(lambda: u.gemm_fprop(qx, qw, out), flush, reps=reps, warm=1)
+    del out, qx, qw, flush
+    return {"fprop_ms": round(t_g, 4),
             "fprop_TFLOPs": round(2 * s.M * s.N * s.K / (t_g * 1e-3) / 1e12, 1),
             "kernel": "gemm_tn_kernel<0> (kind::f16 per-block partials, exponent-byte scales)"}
 
@@ -323,122 +496,21 @@ def run_moe(device, two_level: bool, reps: int = 10):
     return out
 
 
-def run_device(args, rank, world, device):
-    from fp4_quantized_gemms_b200 import ufp4
-    peaks, peak_kind = load_peaks()
-    s = SHAPE
-    flops = 3 * 2 * s.M * s.N * s.K
-    step = LayerStep(device, args.scale)
-    stream = torch.cuda.current_stream(device)
-
-    for _ in range(args.warmup):
-        step.step()
-    torch.cuda.synchronize(device)
-    if ufp4.check_device_status() != ufp4.OK:
-        raise RuntimeError("device error word set during warm-up")
-
-    nev = 5
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(device)
-    with ClockSampler(device.index if device.index is not None else 0) as clk:
-        start = torch.cuda.Event(enable_timing=True)
-        end = torch.cuda.Event(enable_timing=True)
-        start.record(stream)
-        for i in range(args.steps):
-            step.step(ev[i])
-        end.record(stream)
-        torch.cuda.synchronize(device)
-    if world > 1:
-        torch.distributed.barrier()
-    total_ms = max_over_ranks(start.elapsed_time(end), world, device)
-    ms_per_step = total_ms / args.steps
-    q_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps))
-    g_ms = [statistics.mean(ev[i][1 + j].elapsed_time(ev[i][2 + j]) for i in range(args.steps))
-            for j in range(3)]
-    status = ufp4.check_device_status()
-
-    # ---- end to end through the public API with host buffers (rank-local)
-    e2e = run_e2e(step, args, device)
-
-    # ---- grouped (MoE) GEMMs of the mixture-of-experts config (reported, not in `value`)
-    moe = run_moe(device, step.two)
-    diag = run_diag(step)
-    mx = run_mx(step)
-
-    value = job_tflops(world, flops, ms_per_step)
-    gemm_tf = [2 * s.M * s.N * s.K / (g * 1e-3) / 1e12 for g in g_ms]
-    bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    if step.two:
-        # Native block-scaled FP4 GEMM (kind::mxf4nvf4): the kind's peak is the
-        # measured bf16 peak times the nominal fp4 / bf16 ratio (9 / 2.25); an
-        # E1M2 operand pair takes four FP4 MMAs per K step (two E2M1 planes
-        # each), so the tensor pipe executes 4x the useful FLOPs.
-        peak_tf = bf16_peak * 4.0
-        issue_factor = 4.0
-        kern = "gemm_fp4_kernel, kind::mxf4nvf4.block16 tcgen05 (E1M2 as 2 E2M1 planes)"
-        peak_src = f"{peak_kind} bf16 dense x 4 (nominal fp4 / bf16 dense ratio), burst"
-    else:
-        peak_tf = bf16_peak
-        issue_factor = 1.0
-        kern = "gemm_tn_kernel<0>, kind::f16 tcgen05 (fp16 operands, fp32 block-scale epilogue)"
-        peak_src = f"{peak_kind} bf16 dense (fp16 runs at the bf16 rate), burst"
-    qbytes = quant_bytes(step)
-    q_gbs = qbytes / (q_ms * 1e-3) / 1e9
-    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    dom = int(np.argmax(g_ms))
-    result = {
-        "metric": METRIC,
-        "value": round(value, 2),
-        "unit": "TFLOP/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": round(ms_per_step, 4),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": ("e1m2 codes as two e2m1 planes (ue4m3 block-16 factors), fp32 accumulate"
-                  if step.two else "e1m2 codes, fp16 tensor-core operands, fp32 accumulate"),
-        "data": "synthetic (seeded PCG64 inputs of the workload's shapes and distributions)",
-        "config": {**workload_desc(args.scale), "parallelism": f"replicas x{world}"},
-        "gpu_launches": step.launches * args.steps,
-        "kernels": {
-            "quantize_all_ms": round(q_ms, 4),
-            "quantize_GBps": round(q_gbs, 1),
-            "quantize_frac_of_8TBps": round(q_gbs / 8000.0, 4),
-            "quantize_frac_of_measured_hbm": round(q_gbs / hbm, 4),
-            "gemm_ms": {k: round(v, 4) for k, v in zip(("fprop", "dgrad", "wgrad"), g_ms)},
-            "gemm_TFLOPs": {k: round(v, 1) for k, v in zip(("fprop", "dgrad", "wgrad"), gemm_tf)},
-        },
-        "roofline": {
-            "kernel": f"{kern} ({('fprop', 'dgrad', 'wgrad')[dom]})",
-            "bound": "tensor",
-            "achieved": round(gemm_tf[dom] * issue_factor, 1),
-            "achieved_useful": round(gemm_tf[dom], 1),
-            "peak": round(peak_tf, 1),
-            "peak_source": peak_src,
-            "unit": "TFLOP/s",
-            "frac": round(gemm_tf[dom] * issue_factor / peak_tf, 4),
-            "traffic": None,
-        },
-        "e2e": e2e,
-        "moe_grouped": moe,
-        "diagnostics": diag,
-        "mx_block32": mx,
-        "device_status": ufp4.status_string(status),
-    }
-    result["clocks"] = clk.summary()
-    return result
+def _occupancy(code_count, grid: int) -> dict:
+    """Code-occupancy histogram (share of elements per magnitude code, both
+    signs) and its entropy in bits, beside the bucket ratio."""
+    mags = [code_count[k] + (code_count[8 + k] if k else 0) for k in range(8)]
+    tot = float(sum(mags)) or 1.0
+    p = [m / tot for m in mags]
+    ent = -sum(q * math.log2(q) for q in p if q > 0)
+    return {"magnitude_share": [round(q, 5) for q in p], "entropy_bits": round(ent, 4)}
 
 
-def run_diag(step: LayerStep, reps: int = 10) -> dict:
-    """Diagnostics of the step's six operands (SQNR, bucket ratio, underflow
-    ratio from ufp4_quant_stats) and the time of the two diagnostics kernels
-    on the largest tensors: quant_stats of dY^T (8192 x 8192) and the
-    GEMM-output SQNR sums of the 8192 x 8192 fp32 output Y against a copy of
-    it held in a separate buffer (both read from HBM)."""
+def run_diag(step: LayerStep, reps: int = 5) -> dict:
+    """Diagnostics of the step's six operands (SQNR, bucket ratio, code
+    occupancy, underflow ratio from ufp4_quant_stats) and the time of the two
+    diagnostics kernels on the largest tensors: quant_stats of dY^T and the
+    GEMM-output SQNR sums of Y against a copy of it (both read from HBM)."""
     u = step.u
     C, R = u.ALONG_COLS, u.ALONG_ROWS
     out = {}
@@ -447,42 +519,31 @@ def run_diag(step: LayerStep, reps: int = 10) -> dict:
                              ("W^T", step.W, R, step.qwt), ("X^T", step.X, R, step.qxt)):
         st = u.quant_stats(x, axis, q)
         out[name] = {"sqnr_db": round(st["sqnr_db"], 3), "bucket_ratio": round(st["bucket_ratio"], 4),
-                     "underflow_ratio": round(st["underflow_ratio"], 5)}
+                     "underflow_ratio": round(st["underflow_ratio"], 5),
+                     **_occupancy(st["code_count"], q.cfg.grid)}
     buf = torch.zeros(64, dtype=torch.float64, device=step.dev)
     sums = torch.zeros(2, dtype=torch.float64, device=step.dev)
     ref = step.Y
     test = step.Y.clone()
-
-    def timed(fn):
-        for _ in range(3):
-            fn()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(reps):
-            fn()
-        b.record()
-        torch.cuda.synchronize(step.dev)
-        return a.elapsed_time(b) / reps
-
-    t_stats = timed(lambda: u.quant_stats_launch(step.dY, R, step.qdyt, out=buf))
-    t_sqnr = timed(lambda: u.sqnr_sums(ref, test, out=sums))
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=step.dev)
+    t_stats = _timed(lambda: u.quant_stats_launch(step.dY, R, step.qdyt, out=buf), flush, reps=reps)
+    t_sqnr = _timed(lambda: u.sqnr_sums(ref, test, out=sums), flush, reps=reps)
     n = step.dY.numel()
     per = 2 + 0.5 + (1 / 16 if step.two else 4 / 16)
     out["quant_stats_dYT"] = {"ms": round(t_stats, 4), "GBps": round(n * per / (t_stats * 1e-3) / 1e9, 1),
                               "bytes_per_element": per}
     m = ref.numel()
-    out["sqnr_sums_8192x8192"] = {"ms": round(t_sqnr, 4), "GBps": round(m * 8 / (t_sqnr * 1e-3) / 1e9, 1)}
-    del test
+    out["sqnr_sums_Y"] = {"ms": round(t_sqnr, 4), "GBps": round(m * 8 / (t_sqnr * 1e-3) / 1e9, 1)}
+    del test, flush
     return out
 
 
-def run_e2e(step: LayerStep, args, device):
+def run_e2e(step: LayerStep, host_inputs, args, device):
     """Same step through the public API with HOST inputs and outputs: pinned
     H2D copies of X, W, dY, the hot path, D2H copies of Y, dX, dW, all inside
     the timed region."""
-    s = SHAPE
-    X, W, dY = wl.layer_inputs(s)
+    s = step.shape
+    X, W, dY = host_inputs
     hX = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).pin_memory()
     hW = torch.from_numpy(W.view(np.int16)).view(torch.bfloat16).pin_memory()
     hdY = torch.from_numpy(dY.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -504,7 +565,7 @@ def run_e2e(step: LayerStep, args, device):
     for _ in range(max(1, min(args.warmup, 3))):
         one()
     torch.cuda.synchronize(device)
-    n = max(1, min(args.steps, 10))
+    n = max(1, min(args.steps, 5))
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record()
@@ -519,21 +580,128 @@ def run_e2e(step: LayerStep, args, device):
             "steps": n}
 
 
+def gemm_roofline(g_ms, shape, peaks, peak_kind, two: bool, grid: int) -> dict:
+    """Roofline of the dominant (slowest) GEMM of a step: useful flops 2MNK
+    over its CUDA-event time, against the peak of the MMA kind it runs on."""
+    s = shape
+    tf = [2 * s.M * s.N * s.K / (g * 1e-3) / 1e12 for g in g_ms]
+    dom = int(np.argmax(g_ms))
+    bf16 = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    if two:
+        peak = bf16 * FP4_OVER_BF16
+        kern = ("gemm_fp4_kernel, tcgen05.mma kind::mxf4nvf4.block_scale.block16"
+                + (" (E1M2 as two E2M1 planes: four MMAs per K step)" if grid == 0 else ""))
+        src = f"{peak_kind} bf16 dense x 4 (nominal fp4 / bf16 dense ratio), burst"
+    else:
+        peak = bf16
+        kern = "gemm_tn_kernel<0>, tcgen05.mma kind::f16 (fp16 operands, fp32 block-scale epilogue)"
+        src = f"{peak_kind} bf16 dense (fp16 runs at the bf16 rate), burst"
+    r = {"kernel": f"{kern} ({('fprop', 'dgrad', 'wgrad')[dom]})", "bound": "tensor",
+         "achieved": round(tf[dom], 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+         "frac": round(tf[dom] / peak, 4), "traffic": None, "peak_source": src,
+         "achieved_is": "useful flops 2MNK / CUDA-event time of the dominant GEMM"}
+    if two and grid == 0:
+        r["frac_of_bf16_rate_ceiling"] = round(tf[dom] / bf16, 4)
+        r["ceiling_note"] = ("an exact E1M2 product needs four FP4 MMAs per K step (no native uniform-grid "
+                             "kind), so its ceiling is the FP4 rate / 4 = the bf16 rate")
+        r["issued_fp4_TFLOPs"] = round(4 * tf[dom], 1)
+    r["traffic_note"] = ("null: a full-size launch is outside the ncu capture-size rule and its DRAM "
+                         "bytes do not scale from a small capture (operands are re-read from L2)")
+    return r
+
+
+def run_device(args, rank, world, device):
+    from fp4_quantized_gemms_b200 import ufp4
+    peaks, peak_kind = load_peaks()
+    shape = SHAPES[args.workload]
+    s = shape
+    flops = 3 * 2 * s.M * s.N * s.K
+    host = wl.layer_inputs(shape)
+    dev_inputs = tuple(to_dev(b, device) for b in host)
+    step = LayerStep(device, args.scale, shape, dev_inputs)
+    ms_per_step, q_ms, g_ms, clk = time_steps(step, args.steps, args.warmup, world, device, clocks=True)
+    status = ufp4.check_device_status()
+    value = job_tflops(world, flops, ms_per_step)
+    qbytes = quant_bytes(step)
+    q_gbs = qbytes / (q_ms * 1e-3) / 1e9
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    gemm_tf = [2 * s.M * s.N * s.K / (g * 1e-3) / 1e12 for g in g_ms]
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": ("e1m2 codes as two e2m1 planes (ue4m3 block-16 factors), fp32 accumulate"
+                  if step.two else "e1m2 codes, fp16 tensor-core operands, fp32 accumulate"),
+        "data": "synthetic (seeded PCG64 inputs of the workload's shapes and distributions)",
+        "config": {**workload_desc(shape, args.scale), "parallelism": f"replicas x{world}"},
+        "gpu_launches": step.launches * args.steps,
+        "kernels": {
+            "quantize_all_ms": round(q_ms, 4),
+            "quantize_GBps": round(q_gbs, 1),
+            "quantize_frac_of_8TBps": round(q_gbs / HBM_SPEC_GBS, 4),
+            "quantize_frac_of_measured_hbm": round(q_gbs / hbm, 4),
+            "gemm_ms": {k: round(v, 4) for k, v in zip(("fprop", "dgrad", "wgrad"), g_ms)},
+            "gemm_TFLOPs": {k: round(v, 1) for k, v in zip(("fprop", "dgrad", "wgrad"), gemm_tf)},
+        },
+        "roofline": gemm_roofline(g_ms, shape, peaks, peak_kind, step.two, step.grid),
+        "device_status": ufp4.status_string(status),
+        "clocks": clk,
+    }
+    if rank == 0 and not args.quick:
+        result["diagnostics"] = run_diag(step)
+        result["mx_block32"] = run_mx(step)
+    result["e2e"] = run_e2e(step, host, args, device)
+    step.free()
+    del step
+    torch.cuda.empty_cache()
+    if not args.quick:
+        # the E2M1 baseline grid of the same layer, RTNE on every operand
+        b = LayerStep(device, args.scale, shape, dev_inputs, grid=ufp4.GRID_E2M1)
+        ms_b, q_b, g_b, _ = time_steps(b, max(3, args.steps // 4), 3, 1, device, clocks=False)
+        result["e2m1_baseline"] = {
+            "recipe": "E2M1 grid, RTNE on X, W and dY, RHT16, block 16, two-level scales",
+            "ms_per_step": round(ms_b, 4), "value": round(flops / (ms_b * 1e-3) / 1e12, 2),
+            "quantize_all_ms": round(q_b, 4),
+            "gemm_TFLOPs": {k: round(2 * s.M * s.N * s.K / (g * 1e-3) / 1e12, 1)
+                            for k, g in zip(("fprop", "dgrad", "wgrad"), g_b)},
+            "roofline": gemm_roofline(g_b, shape, peaks, peak_kind, b.two, b.grid),
+        }
+        b.free()
+        del b
+        torch.cuda.empty_cache()
+    del dev_inputs
+    torch.cuda.empty_cache()
+    if rank == 0 and not args.quick:
+        result["moe_grouped"] = run_moe(device, args.scale == "two-level")
+        result["quantize_sweep"] = run_sweep(device, peaks)
+    if ufp4.check_device_status() != ufp4.OK:
+        raise RuntimeError("device error word set")
+    return result
+
+
 # ------------------------------------------------------------------ oracle arm
 class OracleSample:
-    """Bounded samples of one step on the host cores, in the configuration the
-    GPU arm runs (`scale`): the oracle quantizes sampled output rows of every
-    operand (full reduction length) and contracts the sampled block of each
-    GEMM.  Inputs and, with two-level scales, the six rotated tensor amaxes
-    are prepared once, outside any timed region."""
+    """The oracle as it stands, on the host cores, in the GPU arm's
+    configuration (`scale`): it quantizes sampled output rows of every operand
+    (full reduction length) and contracts a sampled block of each GEMM.  The
+    inputs and, with two-level scales, the six rotated tensor amaxes are
+    prepared once, outside any timed region."""
 
     MASK = 0x09F1FD9D03F0A9B4       # the binding's default D sign mask
 
-    def __init__(self, scale: str):
+    def __init__(self, scale: str, shape):
         import oracle
         self.oracle = oracle
         oracle.build()
-        self.X, self.W, self.dY = wl.layer_inputs(SHAPE)
+        self.shape = shape
+        self.X, self.W, self.dY = wl.layer_inputs(shape)
         self.two = scale == "two-level"
         fmt = oracle.SCALE_E4M3_X_FP32 if self.two else oracle.SCALE_FP32
         base = dict(grid=0, hadamard_n=16, block=16, sign_mask=self.MASK, scale_fmt=fmt)
@@ -545,10 +713,11 @@ class OracleSample:
             for ax in (0, 1):
                 self.amax[name, ax] = oracle.rht_amax(bits, ax, 16, self.MASK) if self.two else 0.0
 
-    def step(self, rng, n_rows=8, n_cols=8):
-        """One sampled step; returns (GEMM flops of the sampled entries, seconds)."""
+    def step(self, rng, n_rows: int, n_cols: int):
+        """One sampled step: returns (elements quantized, quantize seconds,
+        GEMM flops of the sampled entries, GEMM seconds)."""
         oracle = self.oracle
-        s = SHAPE
+        s = self.shape
         gemms = [(("X", 0, self.rt, s.M), ("W", 0, self.rt, s.N), s.K),
                  (("dY", 0, self.sr0, s.M), ("W", 1, self.rt, s.K), s.N),
                  (("dY", 1, self.sr1, s.N), ("X", 1, self.rt, s.K), s.M)]
@@ -565,68 +734,121 @@ class OracleSample:
                 q.escales = np.concatenate([p.escales for p in parts])
             return q
 
-        flops = 0.0
-        t0 = time.perf_counter()
+        elems = flops = 0.0
+        tq = tg = 0.0
         for (an, aax, acfg, arows), (bn, bax, bcfg, brows), K in gemms:
+            t0 = time.perf_counter()
             qa = rows_q(an, aax, acfg, rng.choice(arows, n_rows, replace=False))
             qb = rows_q(bn, bax, bcfg, rng.choice(brows, n_cols, replace=False))
+            t1 = time.perf_counter()
             ii = np.repeat(np.arange(n_rows), n_cols)
             jj = np.tile(np.arange(n_cols), n_rows)
             out = oracle.gemm_tn_entries(qa, qb, ii, jj)
+            t2 = time.perf_counter()
+            elems += (n_rows + n_cols) * K
             flops += 2.0 * K * out.size
-        return flops, time.perf_counter() - t0
+            tq += t1 - t0
+            tg += t2 - t1
+        return elems, tq, flops, tg
+
+
+def oracle_rates(smp: OracleSample, rng, budget_s: float, n_rows: int, n_cols: int, max_steps: int):
+    """Runs sampled steps until `budget_s` of CPU work; returns the oracle's
+    quantize rate (elements/s), GEMM rate (flop/s), the steps run and the
+    seconds spent."""
+    E = Q = F = G = 0.0
+    n = 0
+    while (Q + G) < budget_s and n < max_steps:
+        e, q, f, g = smp.step(rng, n_rows, n_cols)
+        E, Q, F, G = E + e, Q + q, F + f, G + g
+        n += 1
+    return E / Q, F / G, n, Q + G
+
+
+def oracle_step_figures(shape, two: bool, q_rate: float, g_rate: float) -> dict:
+    """The oracle's whole-step throughput in the GPU arm's unit, from its
+    measured rates: a step quantizes every operand in full (2 (MK + NK + MN)
+    elements) and contracts the three GEMMs (3 * 2MNK flops)."""
+    s = shape
+    elems = 2 * (s.M * s.K + s.N * s.K + s.M * s.N)
+    flops = 3 * 2 * s.M * s.N * s.K
+    t = elems / q_rate + flops / g_rate
+    per = 2.5 + (1 / 16 if two else 4 / 16)
+    return {"step_s": t, "value": flops / t / 1e12,
+            "quantize_GBps": q_rate * per / 1e9, "gemm_GFLOPs": g_rate / 1e9}
 
 
 def run_reference(args, world):
-    smp = OracleSample(args.scale)       # inputs and tensor amaxes outside the timed region
+    shape = SHAPES[args.workload]
+    smp = OracleSample(args.scale, shape)       # inputs and tensor amaxes outside the timed region
     rng = np.random.default_rng(0)
     for _ in range(args.warmup):
-        smp.step(rng)
-    times, flops = [], 0.0
-    for _ in range(args.steps):
-        f, t = smp.step(rng)
-        times.append(t)
-        flops += f
-    total = sum(times)
-    value = flops / total / 1e12
+        smp.step(rng, 2, 2)
     cores = smp.oracle.num_threads()
-    sample = ("per step: 8 sampled output rows of each of the 6 quantized operands "
-              "(full reduction length) and the 8x8 sampled block of each GEMM"
-              + ("; the rotated tensor amaxes are computed once before the timed steps"
-                 if smp.two else ""))
+    n_rows = max(2, min(16, cores))
+    times = []
+    Eq = Tq = Fg = Tg = 0.0
+    for _ in range(args.steps):
+        e, q, f, g = smp.step(rng, n_rows, n_rows)
+        Eq, Tq, Fg, Tg = Eq + e, Tq + q, Fg + f, Tg + g
+        times.append(q + g)
+    fig = oracle_step_figures(shape, smp.two, Eq / Tq, Fg / Tg)
+    sample = (f"per step: {n_rows} sampled output rows of each of the 6 quantized operands "
+              f"(full reduction length) and the {n_rows}x{n_rows} sampled block of each GEMM; "
+              "value = full-step flops / (elements of a step / measured quantize rate + flops of a step / "
+              "measured GEMM rate)" + ("; the rotated tensor amaxes are computed once before the timed steps"
+                                       if smp.two else ""))
+    value = fig["value"]
     res = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": fig["step_s"] * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64 oracle (fp32 RHT, exact rounding decisions)", "data": "synthetic",
-        "config": {**workload_desc(args.scale), "parallelism": "host cores"},
+        "config": {**workload_desc(shape, args.scale), "parallelism": f"replicas x{world}"},
         "impl": "reference",
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
-        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
-                "d2h_bytes_per_step": 0},
+                         "sample": sample, "quantize_GBps": round(fig["quantize_GBps"], 4),
+                         "gemm_GFLOPs": round(fig["gemm_GFLOPs"], 3),
+                         "sampled_wall_s": round(sum(times), 3)},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     return res
 
 
-def cpu_baseline_quick(scale: str = "two-level"):
-    """The oracle as it stands, on a bounded sample of the workload (rank 0),
-    in the GPU arm's scale configuration."""
-    smp = OracleSample(scale)
+def cpu_baseline(scale: str, shape, budget_s: float = 10.0) -> dict:
+    """The oracle as it stands on the host cores (rank 0), in the GPU arm's
+    configuration: quantize GB/s on sampled full-K rows of the large layer's
+    six operands, GEMM GFLOP/s on the sampled entries of its three GEMMs, the
+    full tiny FPROP as a second GEMM figure, and the modeled whole-step
+    throughput in the GPU arm's unit."""
+    import oracle
+    smp = OracleSample(scale, shape)
+    cores = smp.oracle.num_threads()
     rng = np.random.default_rng(1)
-    smp.step(rng, 4, 4)                 # warm caches / page in
-    flops, secs = 0.0, 0.0
-    n = 0
-    while secs < 10.0 and n < 200:
-        f, t = smp.step(rng, 32, 32)
-        flops += f
-        secs += t
-        n += 1
-    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": smp.oracle.num_threads(),
-            "kind": "oracle",
-            "sample": (f"{n} sampled steps: 32 output rows of each of the 6 quantized operands "
-                       f"(full K) and a 32x32 block of each GEMM, {secs:.1f} s of CPU work"
-                       + ("; tensor amaxes computed before timing" if smp.two else ""))}
+    smp.step(rng, 2, 2)                     # warm caches / page in
+    n_rows = max(8, 2 * cores)
+    q_rate, g_rate, n, secs = oracle_rates(smp, rng, budget_s, n_rows, n_rows, 50)
+    fig = oracle_step_figures(shape, smp.two, q_rate, g_rate)
+    # the tiny FPROP in full (256 x 512 x 512)
+    t = wl.TINY
+    X, W, _ = wl.layer_inputs(t, want_dy=False, cache=False)
+    cfg = oracle.QuantCfg(grid=0, hadamard_n=16, block=16, sign_mask=OracleSample.MASK)
+    t0 = time.perf_counter()
+    qa = oracle.quantize(X, 0, cfg)
+    qb = oracle.quantize(W, 0, cfg)
+    t1 = time.perf_counter()
+    oracle.gemm_tn(qa, qb)
+    t2 = time.perf_counter()
+    tiny_gflops = 2 * t.M * t.N * t.K / (t2 - t1) / 1e9
+    return {"value": fig["value"], "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": (f"{n} sampled steps of the large layer ({secs:.1f} s of CPU work): {n_rows} output rows "
+                       f"of each of the 6 quantized operands (full K) and a {n_rows}x{n_rows} block of each "
+                       "GEMM; value = full-step flops / (step elements / quantize rate + step flops / GEMM rate)"
+                       + ("; tensor amaxes computed before timing" if smp.two else "")),
+            "quantize_GBps": round(fig["quantize_GBps"], 4),
+            "gemm_GFLOPs": round(fig["gemm_GFLOPs"], 3),
+            "tiny_fprop_full": {"shape": [t.M, t.K, t.N], "gemm_GFLOPs": round(tiny_gflops, 3),
+                                "quantize_ms": round((t1 - t0) * 1e3, 2)}}
 
 
 def main():
@@ -636,6 +858,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ufp4", choices=["ufp4", "reference"])
     ap.add_argument("--scale", default="two-level", choices=["two-level", "fp32"])
+    ap.add_argument("--workload", default="large", choices=sorted(SHAPES))
+    ap.add_argument("--quick", action="store_true", help="the timed step and e2e only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -660,7 +884,7 @@ def main():
     res = run_device(args, rank, world, device)
     if rank == 0:
         if not args.no_cpu_baseline:
-            res["cpu_baseline"] = cpu_baseline_quick(args.scale)
+            res["cpu_baseline"] = cpu_baseline(args.scale, SHAPES[args.workload])
         print(json.dumps(res), flush=True)
     if world > 1:
         torch.distributed.barrier()

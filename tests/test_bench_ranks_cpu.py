@@ -69,7 +69,7 @@ def test_reference_arm_json_line():
     import sys
     env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
     r = subprocess.run([sys.executable, os.path.join(os.path.dirname(bench.__file__), "bench.py"),
-                        "--impl", "reference", "--steps", "1", "--warmup", "3"],
+                        "--impl", "reference", "--steps", "1", "--warmup", "3", "--workload", "layer"],
                        env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     line = json.loads(r.stdout.strip().splitlines()[-1])
@@ -80,3 +80,20 @@ def test_reference_arm_json_line():
     assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "TFLOP/s"
     assert line["config"]["scales"].startswith("E4M3")          # the GPU arm's default scales
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["cpu_baseline"]["quantize_GBps"] > 0 and line["cpu_baseline"]["gemm_GFLOPs"] > 0
+    assert line["config"]["M"] == 8192 and line["config"]["N"] == 8192
+
+
+def test_oracle_step_model_units():
+    """The oracle's whole-step figure: elements / rate + flops / rate, in the
+    GPU arm's unit; a doubled GEMM rate can at most halve the step time."""
+    from fp4_quantized_gemms_b200 import workloads as wl
+    s = wl.LARGE
+    a = bench.oracle_step_figures(s, True, 1e8, 1e10)
+    elems = 2 * (s.M * s.K + s.N * s.K + s.M * s.N)
+    flops = 6 * s.M * s.N * s.K
+    assert a["step_s"] == pytest.approx(elems / 1e8 + flops / 1e10)
+    assert a["value"] == pytest.approx(flops / a["step_s"] / 1e12)
+    assert a["quantize_GBps"] == pytest.approx(1e8 * (2.5 + 1 / 16) / 1e9)
+    b = bench.oracle_step_figures(s, True, 1e8, 2e10)
+    assert a["step_s"] / 2 < b["step_s"] < a["step_s"]
