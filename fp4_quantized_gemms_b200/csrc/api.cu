@@ -169,12 +169,21 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
     // mode 2: CTA pairs).
     int mode = 0;
     if (a->cfg.scale_fmt == UFP4_SCALE_E4M3_X_FP32) {
+        // The CTA-pair kernel (mode 5) takes E1M2 operands whose correction
+        // planes follow their codes in one allocation, and E2M1 operands.
+        auto adjacent_planes = [](const ufp4_qtensor_t *q) {
+            const uint64_t plane = static_cast<uint64_t>(q->rows) * static_cast<uint64_t>(q->kpad / 2);
+            return q->rows > 0 && q->corr != nullptr &&
+                   reinterpret_cast<uintptr_t>(q->corr) == reinterpret_cast<uintptr_t>(q->codes) + plane;
+        };
+        const bool pair_ok = a->cfg.grid != UFP4_GRID_E1M2 || (adjacent_planes(a) && adjacent_planes(b));
         switch (g_two_level_path.load()) {
             case UFP4_GEMM_PATH_FP16: mode = 1; break;
             case UFP4_GEMM_PATH_FP16_PAIR: mode = 2; break;
             case UFP4_GEMM_PATH_NATIVE_FP4: mode = 3; break;
             case UFP4_GEMM_PATH_NATIVE_FP4_PAIR: mode = 4; break;
-            default: mode = 3; break;
+            case UFP4_GEMM_PATH_NATIVE_FP4_PAIR256: mode = pair_ok ? 5 : 3; break;
+            default: mode = pair_ok ? 5 : 3; break;
         }
     }
     if (groups_dev == nullptr) {
@@ -195,16 +204,17 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
     // B code rows staged per CTA: fp32-scale kernel 128, fp16 kernels 256
     // (one CTA) or 128 (pairs), native kernels 192 or 96, with the scales of
     // all 192 B rows of a tile in each CTA.
-    int bn = 128;
+    int bn = 128, bscale = 128;
     switch (mode) {
-        case 1: bn = 256; break;
-        case 3: bn = kNativeTileN; break;
-        case 4: bn = kNativeTileN / 2; break;
-        default: bn = 128; break;
+        case 1: bn = bscale = 256; break;
+        case 3: bn = bscale = kNativeTileN; break;
+        case 4: bn = kNativeTileN / 2; bscale = kNativeTileN; break;
+        case 5: bn = 128; bscale = 256; break;
+        default: bn = bscale = 128; break;
     }
     s = encode_operand_maps(a, 128, 128, mode, &args.tm_a_codes, &args.tm_a_scales);
     if (s != UFP4_OK) return s;
-    s = encode_operand_maps(b, bn, mode >= 3 ? kNativeTileN : bn, mode, &args.tm_b_codes, &args.tm_b_scales);
+    s = encode_operand_maps(b, bn, bscale, mode, &args.tm_b_codes, &args.tm_b_scales);
     if (s != UFP4_OK) return s;
     args.a_S = a->tensor_scale;
     args.b_S = b->tensor_scale;
@@ -246,13 +256,22 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
             CUtensorMap scratch;
             s = encode_operand_maps(&ac, 128, 128, mode, &args.tm_a_corr, &scratch);
             if (s != UFP4_OK) return s;
-            s = encode_operand_maps(&bc, bn, kNativeTileN, mode, &args.tm_b_corr, &scratch);
+            s = encode_operand_maps(&bc, bn, bscale, mode, &args.tm_b_corr, &scratch);
             if (s != UFP4_OK) return s;
         }
         args.corr_in = 1;
     }
     // Native kernels store 16-byte pieces when the output allows it.
     args.c_vec = (aligned16(c) && ldc % 4 == 0) ? 1 : 0;
+    // The CTA-pair kernel writes whole 128 x 32 output pieces with TMA bulk
+    // stores (clipped at m and n) when the output is a single dense problem.
+    if (mode == 5 && groups_dev == nullptr && args.c_vec) {
+        CUresult r = encode_tensor_map_2d(&args.tm_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c, static_cast<uint64_t>(n),
+                                          static_cast<uint64_t>(m), static_cast<uint64_t>(ldc) * 4, 32, 128,
+                                          CU_TENSOR_MAP_SWIZZLE_128B);
+        if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
+        args.c_tma = 1;
+    }
     // The restricted E2M1 grid stores E2M1 codes (0..4): the E2M1 kernels.
     const int grid_kind = a->cfg.grid == UFP4_GRID_E1M2 ? 0 : 1;
     cudaError_t e = launch_gemm(args, mode, grid_kind, sm_count(), st);
@@ -591,7 +610,7 @@ ufp4_status_t ufp4_grouped_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b
 }
 
 ufp4_status_t ufp4_set_two_level_gemm_path(int32_t path) {
-    if (path < UFP4_GEMM_PATH_AUTO || path > UFP4_GEMM_PATH_NATIVE_FP4_PAIR) return UFP4_ERR_INVALID_ARG;
+    if (path < UFP4_GEMM_PATH_AUTO || path > UFP4_GEMM_PATH_NATIVE_FP4_PAIR256) return UFP4_ERR_INVALID_ARG;
     g_two_level_path.store(path);
     return UFP4_OK;
 }

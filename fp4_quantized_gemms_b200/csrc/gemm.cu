@@ -1363,6 +1363,477 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// CTA-pair native kernel for two-level scales (mode 5): 256 x 256 output
+// tiles on a CTA pair with cta_group::2 MMAs of M = 256, N = 256, K = 64.
+// Rank r of the pair stages A rows [128 r, +128) and B rows [128 r, +128) of
+// the tile (E1M2: codes and correction planes, one 3-D box per operand) and
+// holds accumulator rows [128 r, +128) x 256 fp32 columns of TMEM.  Per SM
+// that is half the operand bytes per flop of a one-CTA 128 x 256 tile.  The
+// other 256 TMEM columns hold the scale factors of up to ten stages in
+// flight (slot s of stage s, freed by the same MMA commit that frees the
+// stage's shared memory).
+//   warp 0     producer: each stage's code tiles (completion counted on the
+//              leader CTA's barrier, which expects both CTAs' bytes) and
+//              this CTA's raw block-major factors (A rows, all 256 B rows);
+//   warp 1     TMEM owner; in the leader, the single-thread MMA issuer;
+//   warps 4-7  factor writers, one per TMEM lane quarter: build the stage's
+//              atoms (lane i of a quarter holds the 4 block factors of rows
+//              i, 32 + i, 64 + i, 96 + i of a 128-row group) by 4 x 4 byte
+//              transposes and store them with tcgen05.st;
+//   warps 8-11 epilogue: TMEM -> registers -> x S_a S_b / (16 n) -> staged
+//              in shared memory -> coalesced 16-byte stores.
+// One accumulator per CTA: the epilogue of a tile (about 2% of a K = 8192
+// main loop) runs before the next tile's MMAs start.
+template <int GRID>
+struct PairCfg {
+    static constexpr int TM = 256;
+    static constexpr int BN = 256;
+    static constexpr int BKE = 128;                 // K elements per stage
+    static constexpr int KST = BKE / 64;            // MMA K steps per stage
+    static constexpr int kRow = BKE / 2;            // code bytes per row per stage
+    static constexpr int kPlanes = GRID == 0 ? 2 : 1;
+    static constexpr int kTile = 128 * kRow;        // one plane of a 128-row tile
+    static constexpr int o_a = 0;                   // [codes | corr] of A
+    static constexpr int o_b = kPlanes * kTile;     // [codes | corr] of this CTA's B half
+    static constexpr int kCodeBytes = 2 * kPlanes * kTile;   // per CTA per stage
+    static constexpr int o_raw_a = kCodeBytes;      // raw factors: [blocks][128 rows]
+    static constexpr int kRawA = 128 * (BKE / 16);
+    static constexpr int o_raw_b = o_raw_a + kRawA; // [blocks][256 rows]
+    static constexpr int kRawB = 256 * (BKE / 16);
+    static constexpr int kStage = (kCodeBytes + kRawA + kRawB + 1023) / 1024 * 1024;
+    static constexpr int kAtoms = 3 * KST;          // SFA, SFB rows 0-127, SFB rows 128-255 per K step
+    static constexpr int kScr = 4 * kAtoms * 512;   // one atom scratch per factor warp
+    static constexpr int kOutChunk = 128 * 32 * 4;  // epilogue staging: 128 rows x 32 fp32
+    static constexpr int kOutBufs = 2;              // staging buffers (bulk stores in flight)
+    static constexpr int kSfBase = 256;             // TMEM column of the first factor slot
+    static constexpr int kSfCols = 12 * KST;        // TMEM columns of one stage's factors
+    static constexpr int kNsTmem = (512 - kSfBase) / kSfCols;
+    static constexpr int kBudget = 232448 - 2048;
+    static constexpr int kNsSmem = (kBudget - kScr - kOutBufs * kOutChunk) / kStage;
+    static constexpr int NS = kNsSmem < kNsTmem ? kNsSmem : kNsTmem;
+    static constexpr int o_out = NS * kStage;
+    static constexpr int o_scr = o_out + kOutBufs * kOutChunk;
+    static constexpr int o_bar = o_scr + kScr;
+    // full[NS], empty[NS], sfull[NS], sfready[NS], sflocal[NS], acc_full,
+    // acc_empty, drain
+    static constexpr int kNumBars = 5 * NS + 3;
+    static constexpr int o_misc = o_bar + kNumBars * 8;
+    static constexpr int kAlloc = o_misc + 64 + 1024;
+    static constexpr int kThreads = 32 * 12;
+    static_assert(NS >= 4, "pipeline depth");
+    static_assert(kAlloc <= 232448, "shared memory budget");
+    static_assert(kSfBase + NS * kSfCols <= 512, "TMEM budget");
+};
+
+// TMA tile loads whose completion is counted on a barrier of the leader CTA
+// of the pair (`bar_cluster`: a shared::cluster address from mapa).  The
+// destination is this CTA's shared memory.  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const CUtensorMap *map, uint32_t bar_cluster,
+                                                 int32_t x, int32_t y, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_addr(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d_pair(void *smem_dst, const CUtensorMap *map, uint32_t bar_cluster,
+                                                 int32_t x, int32_t y, int32_t z, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_addr(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y), "r"(z), "l"(policy)
+        : "memory");
+}
+
+// shared::cluster address of the same-offset object in CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+    return r;
+}
+
+template <int GRID>
+__global__ void __launch_bounds__(PairCfg<GRID>::kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ GemmArgs args) {
+    using C = PairCfg<GRID>;
+    constexpr int TM = C::TM, BN = C::BN, NS = C::NS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::o_bar);   // leader: both CTAs' code tiles landed
+    uint64_t *empty = full + NS;          // MMAs done with stage s (commit to both CTAs)
+    uint64_t *sfull = empty + NS;         // this CTA's raw factors of stage s landed
+    uint64_t *sfready = sfull + NS;       // leader: factors of stage s in both CTAs' TMEM
+    uint64_t *sflocal = sfready + NS;     // peer: its four factor warps wrote stage s
+    uint64_t *acc_full = sflocal + NS;    // accumulator complete (commit to both CTAs)
+    uint64_t *acc_empty = acc_full + 1;   // leader: both CTAs' epilogues drained TMEM (8 warps)
+    uint64_t *drain = acc_empty + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::o_misc);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::o_misc + 4);
+    auto stage = [&](int s) { return smem + s * C::kStage; };
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int blk = args.block;                       // 16 or 32
+    const int nraw = C::BKE / blk;                    // raw factor rows per stage
+    const uint32_t rank = cluster_ctarank();
+    const int64_t unit = blockIdx.x >> 1;
+    const int64_t nunits = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+            mbar_init(&sfull[i], 1);
+            mbar_init(&sfready[i], 5);     // the leader's four factor warps + the peer's relay
+            mbar_init(&sflocal[i], 4);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 8);
+        mbar_init(drain, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(GRID == 0 ? &args.tm_a_corr : &args.tm_a_codes);
+        tma_prefetch_desc(GRID == 0 ? &args.tm_b_corr : &args.tm_b_codes);
+        tma_prefetch_desc(&args.tm_a_scales);
+        tma_prefetch_desc(&args.tm_b_scales);
+    }
+    if (warp == 1) tmem_alloc_pair(tmem_slot, 512);
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int64_t ntiles = total_tiles<TM, BN>(args);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint64_t pol = l2_policy_evict_last();
+            uint32_t it = 0;
+            bool ok = true;
+            for (int64_t t = unit; t < ntiles && ok; t += nunits) {
+                const Tile tl = get_tile<TM, BN>(args, t);
+                const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
+                const int32_t arow = static_cast<int32_t>(tl.g.a_row + tl.m0 + 128 * rank);
+                const int32_t brow = static_cast<int32_t>(tl.g.b_row + tl.n0);
+                const int32_t brow_h = brow + 128 * static_cast<int32_t>(rank);
+                for (int ks = 0; ks < nks; ++ks, ++it) {
+                    const int s = it % NS;
+                    if (it >= static_cast<uint32_t>(NS) &&
+                        !mbar_wait(&empty[s], ((it / NS) - 1) & 1, kErrTimeoutProducer, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const int32_t acol = static_cast<int32_t>(tl.g.a_col + ks * C::BKE);
+                    const int32_t bcol = static_cast<int32_t>(tl.g.b_col + ks * C::BKE);
+                    uint8_t *st = stage(s);
+                    // this CTA's raw factors
+                    mbar_arrive_expect_tx(&sfull[s], (128 + 256) * nraw);
+                    tma_load_2d_hint(st + C::o_raw_a, &args.tm_a_scales, &sfull[s], arow, acol / blk, pol);
+                    tma_load_2d_hint(st + C::o_raw_b, &args.tm_b_scales, &sfull[s], brow, bcol / blk, pol);
+                    // code tiles of both CTAs complete on the leader's barrier
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::kCodeBytes);
+                    const uint32_t fb = cluster_addr(&full[s], 0);
+                    if (GRID == 0) {
+                        tma_load_3d_pair(st + C::o_a, &args.tm_a_corr, fb, acol / 2, arow, 0, pol);
+                        tma_load_3d_pair(st + C::o_b, &args.tm_b_corr, fb, bcol / 2, brow_h, 0, pol);
+                    } else {
+                        tma_load_2d_pair(st + C::o_a, &args.tm_a_codes, fb, acol / 2, arow, pol);
+                        tma_load_2d_pair(st + C::o_b, &args.tm_b_codes, fb, bcol / 2, brow_h, pol);
+                    }
+                }
+            }
+            // Drain: this CTA's factor copies have landed before it exits
+            // (the leader's MMAs consumed every code stage it issued).
+            for (uint32_t d = 0; d < static_cast<uint32_t>(NS) && d < it; ++d) {
+                const uint32_t idx = it - 1 - d;
+                uint32_t dummy = 0;
+                mbar_wait(&sfull[idx % NS], (idx / NS) & 1, kErrTimeoutDrain,
+                          reinterpret_cast<volatile uint32_t *>(&dummy));
+                if (rank == 0)
+                    mbar_wait_cluster(&full[idx % NS], (idx / NS) & 1, kErrTimeoutDrain,
+                                      reinterpret_cast<volatile uint32_t *>(&dummy));
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader)
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc = umma_idesc_fp4_bs(TM, BN);
+            uint32_t it = 0, tcount = 0;
+            bool ok = true;
+            for (int64_t t = unit; t < ntiles && ok; t += nunits, ++tcount) {
+                const Tile tl = get_tile<TM, BN>(args, t);
+                const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
+                if (!mbar_wait_cluster(acc_empty, (tcount & 1) ^ 1, kErrTimeoutMma, abort_flag)) break;
+                tc_fence_after();
+                bool first = true;
+                for (int ks = 0; ks < nks; ++ks, ++it) {
+                    const int s = it % NS;
+                    if (!mbar_wait(&full[s], (it / NS) & 1, kErrTimeoutMma, abort_flag) ||
+                        !mbar_wait_cluster(&sfready[s], (it / NS) & 1, kErrTimeoutMma, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    uint8_t *st = stage(s);
+                    const uint32_t sf0 = tmem_base + C::kSfBase + s * C::kSfCols;
+                    const int64_t rem = tl.g.k - static_cast<int64_t>(ks) * C::BKE;
+                    const int steps = rem >= C::BKE ? C::KST : static_cast<int>((rem + 63) / 64);
+                    const uint32_t a0 = smem_addr(st + C::o_a), b0 = smem_addr(st + C::o_b);
+                    const uint32_t ac = a0 + C::kTile, bc = b0 + C::kTile;
+                    for (int j = 0; j < steps; ++j) {
+                        const uint32_t sfa = sf0 + 12 * j, sfb = sfa + 4;
+                        const uint32_t dk = 32 * j;
+                        umma_fp4_bs_pair(tmem_base, umma_desc_sw64(a0 + dk), umma_desc_sw64(b0 + dk), idesc, sfa,
+                                         sfb, first ? 0u : 1u);
+                        first = false;
+                        if (GRID == 0) {
+                            umma_fp4_bs_pair(tmem_base, umma_desc_sw64(a0 + dk), umma_desc_sw64(bc + dk), idesc,
+                                             sfa, sfb, 1u);
+                            umma_fp4_bs_pair(tmem_base, umma_desc_sw64(ac + dk), umma_desc_sw64(b0 + dk), idesc,
+                                             sfa, sfb, 1u);
+                            umma_fp4_bs_pair(tmem_base, umma_desc_sw64(ac + dk), umma_desc_sw64(bc + dk), idesc,
+                                             sfa, sfb, 1u);
+                        }
+                    }
+                    umma_commit_pair_mc(&empty[s], 0x3);
+                }
+                if (ok) umma_commit_pair_mc(acc_full, 0x3);
+            }
+            // Drain: every MMA issued here completes before TMEM is freed.
+            umma_commit_pair(drain);
+            uint32_t dummy = 0;
+            mbar_wait(drain, 0, kErrTimeoutDrain, reinterpret_cast<volatile uint32_t *>(&dummy));
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ factor relay (peer)
+        // One cluster-scope arrive per stage on the leader's barrier once the
+        // peer's four factor warps are done (their arrives stay CTA-local).
+        if (lane == 0 && rank == 1) {
+            const uint32_t ready = cluster_addr(&sfready[0], 0);
+            uint32_t it = 0;
+            bool ok = true;
+            for (int64_t t = unit; t < ntiles && ok; t += nunits) {
+                const Tile tl = get_tile<TM, BN>(args, t);
+                const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
+                for (int ks = 0; ks < nks; ++ks, ++it) {
+                    const int s = it % NS;
+                    if (!mbar_wait(&sflocal[s], (it / NS) & 1, kErrTimeoutTransform, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                                     ready + static_cast<uint32_t>(s) * 8u)
+                                 : "memory");
+                }
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ factor writers
+        uint8_t *scr = smem + C::o_scr + (warp - 4) * (C::kAtoms * 512);
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+        uint32_t it = 0;
+        bool ok = true;
+        for (int64_t t = unit; t < ntiles && ok; t += nunits) {
+            const Tile tl = get_tile<TM, BN>(args, t);
+            const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
+            for (int ks = 0; ks < nks; ++ks, ++it) {
+                const int s = it % NS;
+                // the raw factors landed, and the MMAs that last read TMEM slot s are done
+                if (!warp_wait(&sfull[s], (it / NS) & 1, kErrTimeoutTransform, abort_flag) ||
+                    (it >= static_cast<uint32_t>(NS) &&
+                     !warp_wait(&empty[s], ((it / NS) - 1) & 1, kErrTimeoutTransform, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t *st = stage(s);
+                uint32_t w[C::kAtoms][4];
+#pragma unroll
+                for (int a = 0; a < C::kAtoms; ++a) {
+                    const int jk = a / 3, kind = a % 3;
+                    const int rows = kind == 0 ? 128 : 256;
+                    const int r = 4 * lane + (kind == 2 ? 128 : 0);
+                    const uint8_t *raw = st + (kind == 0 ? C::o_raw_a : C::o_raw_b) + r;
+                    if (blk == 16) {
+#pragma unroll
+                        for (int kb = 0; kb < 4; ++kb)
+                            w[a][kb] = *reinterpret_cast<const uint32_t *>(raw + (4 * jk + kb) * rows);
+                    } else {
+                        w[a][0] = w[a][1] = *reinterpret_cast<const uint32_t *>(raw + (2 * jk) * rows);
+                        w[a][2] = w[a][3] = *reinterpret_cast<const uint32_t *>(raw + (2 * jk + 1) * rows);
+                    }
+                }
+                // Atom byte 16 (r % 32) + 4 (r / 32) + kb holds the factor of
+                // 16-element block 4 jk + kb of row r of the group.
+#pragma unroll
+                for (int a = 0; a < C::kAtoms; ++a) {
+                    uint32_t o[4];
+                    transpose4x4(w[a][0], w[a][1], w[a][2], w[a][3], o);
+                    uint8_t *dst = scr + a * 512 + 16 * ((4 * lane) & 31) + 4 * ((4 * lane) >> 5);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) *reinterpret_cast<uint32_t *>(dst + 16 * q4) = o[q4];
+                }
+                __syncwarp();
+                const uint32_t sfw = lane_base + C::kSfBase + s * C::kSfCols;
+#pragma unroll
+                for (int a = 0; a < C::kAtoms; ++a) {
+                    const uint4 row = *reinterpret_cast<const uint4 *>(scr + a * 512 + 16 * lane);
+                    tmem_st_32x32b_x4(sfw + 12 * (a / 3) + 4 * (a % 3), row.x, row.y, row.z, row.w);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                // the leader's warps arrive on its barrier directly; the
+                // peer's on a local one that its relay forwards
+                if (lane == 0) mbar_arrive(rank == 0 ? &sfready[s] : &sflocal[s]);
+            }
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------ epilogue
+        // Thread = accumulator row.  Each 128 x 32 fp32 piece is staged in
+        // shared memory in the 128-byte-swizzled layout (16-byte units XORed
+        // with the row mod 8) and, for a single dense output, written by one
+        // TMA bulk store while the warps move on (two staging buffers); TMEM
+        // is released right after the last piece is read.  Grouped outputs
+        // (windows of a larger matrix) use coalesced 16-byte stores.
+        const int q = warp & 3;
+        const int et = threadIdx.x - 32 * 8;            // 0 .. 127
+        const int row_in_tile = 32 * q + lane;
+        const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+        constexpr uint32_t kEpiThreads = 128;
+        const bool elected = et == 0;
+        const uint32_t empty_acc = cluster_addr(acc_empty, 0);
+        // E1M2 operands carry k = 4 * level on both sides: 1/16 (exact).
+        const float mult = __fmul_rn(__fmul_rn(*args.a_S, *args.b_S),
+                                     args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f));
+        uint32_t tcount = 0, piece = 0;
+        for (int64_t t = unit; t < ntiles; t += nunits, ++tcount) {
+            const Tile tl = get_tile<TM, BN>(args, t);
+            const bool ok = warp_wait(acc_full, tcount & 1, kErrTimeoutEpilogue, abort_flag);
+            if (named_bar_or(1, kEpiThreads, !ok)) break;
+            tc_fence_after();
+            const int64_t m0 = tl.m0 + 128 * rank;       // this CTA's accumulator rows
+            const int64_t row = m0 + row_in_tile;
+            const bool row_ok = row < tl.g.m;
+            float *crow = args.c + (tl.g.c_row + row) * args.ldc + tl.g.c_col + tl.n0;
+            const bool tma_tile = args.c_tma != 0;
+            const bool vec_tile = args.c_vec && (tl.g.c_col & 3) == 0;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c, ++piece) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + lane_addr + 32 * c, r);
+                tmem_wait_ld();
+                if (c == BN / 32 - 1) {
+                    // accumulator drained: the next tile's MMAs may start
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(empty_acc)
+                                     : "memory");
+                }
+                const int64_t col0 = tl.n0 + 32 * c;
+                if (col0 >= tl.g.n) continue;             // the same for all threads
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    v[i] = tl.g.k > 0 ? __fmul_rn(__uint_as_float(r[i]), mult) : 0.0f;
+                if (tma_tile || vec_tile) {
+                    uint8_t *buf = smem + C::o_out + (piece & 1) * C::kOutChunk;
+                    // the bulk store issued from this buffer two pieces ago has read it
+                    if (tma_tile && elected && piece >= 2)
+                        asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                    named_bar_sync(1, kEpiThreads);
+                    uint8_t *rowp = buf + row_in_tile * 128;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch)
+                        *reinterpret_cast<float4 *>(rowp + ((ch ^ (row_in_tile & 7)) << 4)) =
+                            make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
+                    if (tma_tile) fence_proxy_async_smem();
+                    named_bar_sync(1, kEpiThreads);          // piece staged
+                    if (tma_tile) {
+                        if (elected) {
+                            asm volatile(
+                                "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                                    reinterpret_cast<uint64_t>(&args.tm_c)),
+                                "r"(static_cast<int32_t>(col0)), "r"(static_cast<int32_t>(m0)), "r"(smem_addr(buf))
+                                : "memory");
+                            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const int p = et + 128 * k;
+                            const int rr = p >> 3, c16 = p & 7;
+                            const float4 val =
+                                *reinterpret_cast<const float4 *>(buf + rr * 128 + ((c16 ^ (rr & 7)) << 4));
+                            const int64_t grow = m0 + rr;
+                            const int64_t gcol = col0 + 4 * c16;
+                            if (grow < tl.g.m && gcol < tl.g.n) {
+                                float *dst = args.c + (tl.g.c_row + grow) * args.ldc + tl.g.c_col + gcol;
+                                if (gcol + 4 <= tl.g.n) {
+                                    __stcs(reinterpret_cast<float4 *>(dst), val);   // streamed: evict first
+                                } else {
+                                    const float e4[4] = {val.x, val.y, val.z, val.w};
+                                    for (int e = 0; e < 4 && gcol + e < tl.g.n; ++e) dst[e] = e4[e];
+                                }
+                            }
+                        }
+                    }
+                } else if (row_ok) {
+                    float *dst = crow + 32 * c;
+                    for (int i = 0; i < 32; ++i)
+                        if (col0 + i < tl.g.n) dst[i] = v[i];
+                }
+            }
+        }
+        // every bulk store has completed before the CTA exits
+        if (elected) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    }
+
+    tc_fence_before();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, 512);
+    }
+}
+
+template <int GRID>
+cudaError_t launch_pair(const GemmArgs &args, int num_sms, cudaStream_t stream) {
+    using C = PairCfg<GRID>;
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<GRID>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kAlloc);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    int units = num_sms / 2;
+    if (args.groups == nullptr) {
+        const GemmGroup &g = args.single;
+        const int64_t tiles = ((g.m + C::TM - 1) / C::TM) * ((g.n + C::BN - 1) / C::BN);
+        if (tiles < units) units = static_cast<int>(tiles);
+    }
+    if (units <= 0) return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(units * 2, 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<GRID>, args);
+}
+
 template <int GRID, int CG, bool CIN>
 cudaError_t launch_fp4(const GemmArgs &args, int num_sms, cudaStream_t stream) {
     using C = Fp4Cfg<GRID, CG, CIN>;
@@ -1446,6 +1917,8 @@ cudaError_t launch_gemm(const GemmArgs &args, int mode, int grid_kind, int num_s
             if (grid_kind == 1) return launch_fp4<1, 1, false>(args, num_sms, stream);
             return args.corr_in ? launch_fp4<0, 1, true>(args, num_sms, stream)
                                 : launch_fp4<0, 1, false>(args, num_sms, stream);
+        case 5:
+            return grid_kind == 1 ? launch_pair<1>(args, num_sms, stream) : launch_pair<0>(args, num_sms, stream);
         default:
             if (grid_kind == 1) return launch_fp4<1, 2, false>(args, num_sms, stream);
             return args.corr_in ? launch_fp4<0, 2, true>(args, num_sms, stream)

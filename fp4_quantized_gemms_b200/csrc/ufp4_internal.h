@@ -95,6 +95,8 @@ struct GemmArgs {
     int corr_in;                          // both operands carry correction planes
     int scale_ue8m0;                      // mode 0: scales are UE8M0 exponent bytes
     int planes3d;                         // corr = codes + rows * kpad / 2 for both
+    CUtensorMap tm_c;                     // fp32 output [m][n], box 32 x 128, 128-byte swizzle
+    int c_tma;                            // tm_c valid: single problem, c_vec, c_col == 0
 };
 
 // Tile columns (B rows) of the native block-scaled FP4 kernels (modes 3, 4).

@@ -399,6 +399,7 @@ def grouped_gemm(a: QTensor, b: QTensor, groups: torch.Tensor, out: torch.Tensor
 
 GEMM_PATH_AUTO, GEMM_PATH_FP16, GEMM_PATH_FP16_PAIR, GEMM_PATH_NATIVE_FP4 = 0, 1, 2, 3
 GEMM_PATH_NATIVE_FP4_PAIR = 4
+GEMM_PATH_NATIVE_FP4_PAIR256 = 5
 
 
 def set_two_level_gemm_path(path: int) -> None:

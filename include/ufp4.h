@@ -292,8 +292,14 @@ ufp4_status_t ufp4_grouped_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b
  *                             CTA per 128 x 192 tile;
  *   UFP4_GEMM_PATH_NATIVE_FP4_PAIR  the same on CTA pairs (cta_group::2,
  *                             256 x 192 tiles);
+ *   UFP4_GEMM_PATH_NATIVE_FP4_PAIR256  block-scaled FP4 MMA on CTA pairs with
+ *                             256 x 256 tiles (half the operand bytes per
+ *                             flop of one CTA); needs E2M1 operands, or E1M2
+ *                             operands whose correction planes follow their
+ *                             codes in one allocation (else the one-CTA path);
  *   UFP4_GEMM_PATH_AUTO       the library's choice (default; currently the
- *                             one-CTA native FP4 path).
+ *                             256 x 256 CTA-pair path where it applies, else
+ *                             the one-CTA native FP4 path).
  * The setting is process-wide and read at each GEMM call; fp32 and UE8M0
  * block scales are unaffected (they always run the fp32-scale kernel).  Errors: INVALID_ARG for an unknown path. */
 typedef enum {
@@ -301,7 +307,8 @@ typedef enum {
     UFP4_GEMM_PATH_FP16 = 1,
     UFP4_GEMM_PATH_FP16_PAIR = 2,
     UFP4_GEMM_PATH_NATIVE_FP4 = 3,
-    UFP4_GEMM_PATH_NATIVE_FP4_PAIR = 4
+    UFP4_GEMM_PATH_NATIVE_FP4_PAIR = 4,
+    UFP4_GEMM_PATH_NATIVE_FP4_PAIR256 = 5
 } ufp4_gemm_path_t;
 ufp4_status_t ufp4_set_two_level_gemm_path(int32_t path);
 int32_t ufp4_get_two_level_gemm_path(void);

@@ -198,10 +198,10 @@ def test_two_level_gemm_path_selector(L):
     old = ufp4.get_two_level_gemm_path()
     try:
         for p in (ufp4.GEMM_PATH_NATIVE_FP4, ufp4.GEMM_PATH_FP16, ufp4.GEMM_PATH_FP16_PAIR,
-                  ufp4.GEMM_PATH_NATIVE_FP4_PAIR, ufp4.GEMM_PATH_AUTO):
+                  ufp4.GEMM_PATH_NATIVE_FP4_PAIR, ufp4.GEMM_PATH_NATIVE_FP4_PAIR256, ufp4.GEMM_PATH_AUTO):
             ufp4.set_two_level_gemm_path(p)
             assert ufp4.get_two_level_gemm_path() == p
-        for bad in (-1, 5, 99):
+        for bad in (-1, 6, 99):
             with pytest.raises(ufp4.UFP4Error):
                 ufp4.set_two_level_gemm_path(bad)
         assert ufp4.get_two_level_gemm_path() == ufp4.GEMM_PATH_AUTO

@@ -158,7 +158,7 @@ def test_large_config_sampled(gemm, fmt, grid):
     _sampled(wl.LARGE, fmt, grid, gemm, n_rows=64, n_cols=64)
 
 
-@pytest.mark.parametrize("path", [ufp4.GEMM_PATH_NATIVE_FP4, ufp4.GEMM_PATH_NATIVE_FP4_PAIR,
+@pytest.mark.parametrize("path", [ufp4.GEMM_PATH_NATIVE_FP4, ufp4.GEMM_PATH_NATIVE_FP4_PAIR, ufp4.GEMM_PATH_NATIVE_FP4_PAIR256,
                                   ufp4.GEMM_PATH_FP16])
 @pytest.mark.parametrize("corr", [True, False])
 @pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1, ufp4.GRID_E2M1_MAX2])
