@@ -88,6 +88,10 @@ ufp4_status_t check_qtensor(const ufp4_qtensor_t *q) {
         if (q->cfg.grid != UFP4_GRID_E1M2) return UFP4_ERR_INVALID_ARG;
         if (!aligned16(q->corr)) return UFP4_ERR_ALIGNMENT;
     }
+    if (q->elems8 != nullptr) {   // E4M3 element plane of an MX (UE8M0) E1M2 operand
+        if (q->cfg.grid != UFP4_GRID_E1M2 || q->cfg.scale_fmt != UFP4_SCALE_UE8M0) return UFP4_ERR_INVALID_ARG;
+        if (!aligned16(q->elems8)) return UFP4_ERR_ALIGNMENT;
+    }
     if (q->rows > (int64_t(1) << 31) || q->kpad > (int64_t(1) << 31)) return UFP4_ERR_UNSUPPORTED;
     return UFP4_OK;
 }
@@ -186,6 +190,11 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
             default: mode = pair_ok ? 5 : 3; break;
         }
     }
+    // MX operands that carry E4M3 element planes: the block-scaled FP8 MMA
+    // on CTA pairs (mode 6); otherwise the fp32-block-scale kernel.
+    if (a->cfg.scale_fmt == UFP4_SCALE_UE8M0 && a->cfg.grid == UFP4_GRID_E1M2 && a->elems8 != nullptr &&
+        b->elems8 != nullptr)
+        mode = 6;
     if (groups_dev == nullptr) {
         if (m == 0 || n == 0) return UFP4_OK;
         if (a->kpad == 0) {
@@ -209,13 +218,25 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
         case 1: bn = bscale = 256; break;
         case 3: bn = bscale = kNativeTileN; break;
         case 4: bn = kNativeTileN / 2; bscale = kNativeTileN; break;
-        case 5: bn = 128; bscale = 256; break;
+        case 5:
+        case 6: bn = 128; bscale = 256; break;
         default: bn = bscale = 128; break;
     }
     s = encode_operand_maps(a, 128, 128, mode, &args.tm_a_codes, &args.tm_a_scales);
     if (s != UFP4_OK) return s;
     s = encode_operand_maps(b, bn, bscale, mode, &args.tm_b_codes, &args.tm_b_scales);
     if (s != UFP4_OK) return s;
+    if (mode == 6) {   // E4M3 element planes: 128-byte rows (128 K per stage), 128-byte swizzle
+        const int64_t ra = a->rows > 0 ? a->rows : 1, rb = b->rows > 0 ? b->rows : 1;
+        CUresult r = encode_tensor_map_2d(&args.tm_a_e8, CU_TENSOR_MAP_DATA_TYPE_UINT8, a->elems8,
+                                          static_cast<uint64_t>(a->kpad), static_cast<uint64_t>(ra),
+                                          static_cast<uint64_t>(a->kpad), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
+        r = encode_tensor_map_2d(&args.tm_b_e8, CU_TENSOR_MAP_DATA_TYPE_UINT8, b->elems8,
+                                 static_cast<uint64_t>(b->kpad), static_cast<uint64_t>(rb),
+                                 static_cast<uint64_t>(b->kpad), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
+    }
     args.a_S = a->tensor_scale;
     args.b_S = b->tensor_scale;
     args.c = c;
@@ -265,7 +286,7 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
     args.c_vec = (aligned16(c) && ldc % 4 == 0) ? 1 : 0;
     // The CTA-pair kernel writes whole 128 x 32 output pieces with TMA bulk
     // stores (clipped at m and n) when the output is a single dense problem.
-    if (mode == 5 && groups_dev == nullptr && args.c_vec) {
+    if ((mode == 5 || mode == 6) && groups_dev == nullptr && args.c_vec) {
         CUresult r = encode_tensor_map_2d(&args.tm_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c, static_cast<uint64_t>(n),
                                           static_cast<uint64_t>(m), static_cast<uint64_t>(ldc) * 4, 32, 128,
                                           CU_TENSOR_MAP_SWIZZLE_128B);
@@ -312,6 +333,7 @@ ufp4_status_t fill_quant_args(const void *x_dev, int64_t rows, int64_t cols, int
     a->scale_ld = out->scale_ld;
     a->codes = static_cast<uint8_t *>(out->codes);
     a->corr = static_cast<uint8_t *>(out->corr);
+    a->elems8 = static_cast<uint8_t *>(out->elems8);
     a->scales = out->scales;
     a->S_out = two_level ? out->tensor_scale : nullptr;
     a->amax_t = two_level ? tensor_amax_dev : nullptr;

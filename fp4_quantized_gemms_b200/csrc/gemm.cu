@@ -1385,22 +1385,28 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
 //              in shared memory -> coalesced 16-byte stores.
 // One accumulator per CTA: the epilogue of a tile (about 2% of a K = 8192
 // main loop) runs before the next tile's MMAs start.
+// GRID 3 is the MX path: E1M2 operands as their E4M3 element planes (one
+// byte per element, 128-byte rows, 128-byte swizzle), UE8M0 factors per 32
+// elements applied in the MMA (kind::mxf8f6f4, K = 32 per MMA, four MMAs per
+// stage picking byte j of the same factor atom).
 template <int GRID>
 struct PairCfg {
+    static constexpr bool kMx = GRID == 3;
     static constexpr int TM = 256;
     static constexpr int BN = 256;
     static constexpr int BKE = 128;                 // K elements per stage
-    static constexpr int KST = BKE / 64;            // MMA K steps per stage
-    static constexpr int kRow = BKE / 2;            // code bytes per row per stage
+    static constexpr int KST = kMx ? 1 : BKE / 64;  // factor atom groups per stage
+    static constexpr int kRow = kMx ? BKE : BKE / 2;   // operand bytes per row per stage
     static constexpr int kPlanes = GRID == 0 ? 2 : 1;
     static constexpr int kTile = 128 * kRow;        // one plane of a 128-row tile
     static constexpr int o_a = 0;                   // [codes | corr] of A
     static constexpr int o_b = kPlanes * kTile;     // [codes | corr] of this CTA's B half
     static constexpr int kCodeBytes = 2 * kPlanes * kTile;   // per CTA per stage
+    static constexpr int kRawRows = kMx ? BKE / 32 : BKE / 16;   // factor rows per stage (most)
     static constexpr int o_raw_a = kCodeBytes;      // raw factors: [blocks][128 rows]
-    static constexpr int kRawA = 128 * (BKE / 16);
+    static constexpr int kRawA = 128 * kRawRows;
     static constexpr int o_raw_b = o_raw_a + kRawA; // [blocks][256 rows]
-    static constexpr int kRawB = 256 * (BKE / 16);
+    static constexpr int kRawB = 256 * kRawRows;
     static constexpr int kStage = (kCodeBytes + kRawA + kRawB + 1023) / 1024 * 1024;
     static constexpr int kAtoms = 3 * KST;          // SFA, SFB rows 0-127, SFB rows 128-255 per K step
     static constexpr int kScr = 4 * kAtoms * 512;   // one atom scratch per factor warp
@@ -1454,6 +1460,31 @@ __device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
     return r;
 }
 
+// Block-scaled FP8 MMA on a CTA pair: E4M3 operands, UE8M0 factors per 32
+// elements (byte sf_id of each factor word, chosen in the instruction
+// descriptor), fp32 accumulate, K = 32.
+__device__ __forceinline__ void umma_mxf8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Instruction descriptor, kind::mxf8f6f4 block-scaled: A = B = E4M3, UE8M0
+// factors, fp32 accumulate, both K-major; factor byte sf_id of A and B.
+__host__ __device__ constexpr uint32_t umma_idesc_mxf8(int M, int N, uint32_t sf_id) {
+    return (sf_id << 4)                               // B factor byte
+           | (0u << 7) | (0u << 10)                   // A, B: E4M3
+           | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+           | (1u << 23)                               // factor format UE8M0
+           | (static_cast<uint32_t>(M >> 4) << 24)    // M / 16
+           | (sf_id << 29);                           // A factor byte
+}
+
 template <int GRID>
 __global__ void __launch_bounds__(PairCfg<GRID>::kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ GemmArgs args) {
@@ -1497,8 +1528,8 @@ __global__ void __launch_bounds__(PairCfg<GRID>::kThreads, 1)
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(GRID == 0 ? &args.tm_a_corr : &args.tm_a_codes);
-        tma_prefetch_desc(GRID == 0 ? &args.tm_b_corr : &args.tm_b_codes);
+        tma_prefetch_desc(GRID == 0 ? &args.tm_a_corr : (C::kMx ? &args.tm_a_e8 : &args.tm_a_codes));
+        tma_prefetch_desc(GRID == 0 ? &args.tm_b_corr : (C::kMx ? &args.tm_b_e8 : &args.tm_b_codes));
         tma_prefetch_desc(&args.tm_a_scales);
         tma_prefetch_desc(&args.tm_b_scales);
     }
@@ -1541,6 +1572,9 @@ __global__ void __launch_bounds__(PairCfg<GRID>::kThreads, 1)
                     if (GRID == 0) {
                         tma_load_3d_pair(st + C::o_a, &args.tm_a_corr, fb, acol / 2, arow, 0, pol);
                         tma_load_3d_pair(st + C::o_b, &args.tm_b_corr, fb, bcol / 2, brow_h, 0, pol);
+                    } else if (C::kMx) {
+                        tma_load_2d_pair(st + C::o_a, &args.tm_a_e8, fb, acol, arow, pol);
+                        tma_load_2d_pair(st + C::o_b, &args.tm_b_e8, fb, bcol, brow_h, pol);
                     } else {
                         tma_load_2d_pair(st + C::o_a, &args.tm_a_codes, fb, acol / 2, arow, pol);
                         tma_load_2d_pair(st + C::o_b, &args.tm_b_codes, fb, bcol / 2, brow_h, pol);
@@ -1585,6 +1619,19 @@ __global__ void __launch_bounds__(PairCfg<GRID>::kThreads, 1)
                     const int steps = rem >= C::BKE ? C::KST : static_cast<int>((rem + 63) / 64);
                     const uint32_t a0 = smem_addr(st + C::o_a), b0 = smem_addr(st + C::o_b);
                     const uint32_t ac = a0 + C::kTile, bc = b0 + C::kTile;
+                    if constexpr (C::kMx) {
+                        // K = 32 MMAs (32 bytes of the 128-byte rows), factor byte j:
+                        // four per full stage (a K tail of 64 takes two)
+                        const int nk32 = rem >= C::BKE ? C::BKE / 32 : static_cast<int>(rem / 32);
+                        for (int j = 0; j < nk32; ++j) {
+                            umma_mxf8_pair(tmem_base, umma_desc_sw128(a0 + 32 * j), umma_desc_sw128(b0 + 32 * j),
+                                           umma_idesc_mxf8(TM, BN, static_cast<uint32_t>(j)), sf0, sf0 + 4,
+                                           first ? 0u : 1u);
+                            first = false;
+                        }
+                        umma_commit_pair_mc(&empty[s], 0x3);
+                        continue;
+                    }
                     for (int j = 0; j < steps; ++j) {
                         const uint32_t sfa = sf0 + 12 * j, sfb = sfa + 4;
                         const uint32_t dk = 32 * j;
@@ -1658,7 +1705,9 @@ __global__ void __launch_bounds__(PairCfg<GRID>::kThreads, 1)
                     const int rows = kind == 0 ? 128 : 256;
                     const int r = 4 * lane + (kind == 2 ? 128 : 0);
                     const uint8_t *raw = st + (kind == 0 ? C::o_raw_a : C::o_raw_b) + r;
-                    if (blk == 16) {
+                    if (C::kMx || blk == 16) {
+                        // four factor rows per atom: 16-element blocks 4 jk .. 4 jk + 3,
+                        // or (MX) the stage's four 32-element blocks
 #pragma unroll
                         for (int kb = 0; kb < 4; ++kb)
                             w[a][kb] = *reinterpret_cast<const uint32_t *>(raw + (4 * jk + kb) * rows);
@@ -1707,9 +1756,12 @@ __global__ void __launch_bounds__(PairCfg<GRID>::kThreads, 1)
         constexpr uint32_t kEpiThreads = 128;
         const bool elected = et == 0;
         const uint32_t empty_acc = cluster_addr(acc_empty, 0);
-        // E1M2 operands carry k = 4 * level on both sides: 1/16 (exact).
-        const float mult = __fmul_rn(__fmul_rn(*args.a_S, *args.b_S),
-                                     args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f));
+        // E1M2 operands carry k = 4 * level on both sides: 1/16 (exact).  The
+        // MX path's E4M3 elements are the levels and its factors are in the
+        // MMA: only 1/n.
+        const float mult = C::kMx ? args.inv_n
+                                  : __fmul_rn(__fmul_rn(*args.a_S, *args.b_S),
+                                              args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f));
         uint32_t tcount = 0, piece = 0;
         for (int64_t t = unit; t < ntiles; t += nunits, ++tcount) {
             const Tile tl = get_tile<TM, BN>(args, t);
@@ -1919,6 +1971,8 @@ cudaError_t launch_gemm(const GemmArgs &args, int mode, int grid_kind, int num_s
                                 : launch_fp4<0, 1, false>(args, num_sms, stream);
         case 5:
             return grid_kind == 1 ? launch_pair<1>(args, num_sms, stream) : launch_pair<0>(args, num_sms, stream);
+        case 6:
+            return launch_pair<3>(args, num_sms, stream);
         default:
             if (grid_kind == 1) return launch_fp4<1, 2, false>(args, num_sms, stream);
             return args.corr_in ? launch_fp4<0, 2, true>(args, num_sms, stream)

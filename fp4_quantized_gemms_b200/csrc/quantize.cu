@@ -451,8 +451,20 @@ __device__ __forceinline__ void block_amax(const float2 (&v)[ENT], float (&am)[2
     }
 }
 
-// Stores the 16 code bytes (and the E1M2 correction plane) and the block
-// scales of one lane run.
+// E4M3 bytes of 8 E1M2 codes (nibble i -> byte i, the MX element plane): the
+// magnitude k/4 from a byte table (0x00 0x28 0x30 0x34 0x38 0x3A 0x3C 0x3E
+// for k = 0..7), the sign moved from bit 3 of the nibble to bit 7 of the byte.
+// Codes 0..3 of the low 16 bits of w16 (higher bits ignored).
+__device__ __forceinline__ uint32_t e1m2_to_e4m3x4(uint32_t w16) {
+    const uint32_t mag = prmt(0x34302800u, 0x3E3C3A38u, w16 & 0x7777u);
+    uint32_t v = w16 & 0xFFFFu;
+    v = (v | (v << 8)) & 0x00FF00FFu;                   // nibbles n0 n1 | n2 n3 in bytes 0 and 2
+    v = (v | (v << 4)) & 0x0F0F0F0Fu;                   // one nibble per byte
+    return mag | ((v & 0x08080808u) << 4);
+}
+
+// Stores the 16 code bytes (and the E1M2 correction plane, the MX element
+// plane) and the block scales of one lane run.
 template <int BLK>
 __device__ __forceinline__ void store_run(const QuantArgs &a, int32_t row, int32_t k0, const uint32_t *w,
                                           const uint32_t *st) {
@@ -462,6 +474,13 @@ __device__ __forceinline__ void store_run(const QuantArgs &a, int32_t row, int32
     if (a.corr != nullptr)
         *reinterpret_cast<uint4 *>(a.corr + off) = make_uint4(e1m2_correction(w[0]), e1m2_correction(w[1]),
                                                               e1m2_correction(w[2]), e1m2_correction(w[3]));
+    if (a.elems8 != nullptr) {
+        uint4 *e = reinterpret_cast<uint4 *>(a.elems8 + static_cast<int64_t>(row) * a.kpad + k0);
+        e[0] = make_uint4(e1m2_to_e4m3x4(w[0]), e1m2_to_e4m3x4(w[0] >> 16), e1m2_to_e4m3x4(w[1]),
+                          e1m2_to_e4m3x4(w[1] >> 16));
+        e[1] = make_uint4(e1m2_to_e4m3x4(w[2]), e1m2_to_e4m3x4(w[2] >> 16), e1m2_to_e4m3x4(w[3]),
+                          e1m2_to_e4m3x4(w[3] >> 16));
+    }
 #pragma unroll
     for (int b = 0; b < 32 / BLK; ++b) {
         const int64_t at = static_cast<int64_t>(k0 / BLK + b) * a.scale_ld + row;
@@ -572,6 +591,9 @@ __device__ __forceinline__ void coop_exact(const QuantArgs &a, const uint8_t *ti
                 const int64_t at = static_cast<int64_t>(row) * (a.kpad / 2) + k0 / 2 + 4 * (lane >> 3);
                 *reinterpret_cast<uint32_t *>(a.codes + at) = w;
                 if (a.corr != nullptr) *reinterpret_cast<uint32_t *>(a.corr + at) = e1m2_correction(w);
+                if (a.elems8 != nullptr)
+                    *reinterpret_cast<uint2 *>(a.elems8 + static_cast<int64_t>(row) * a.kpad + k0 + 8 * (lane >> 3)) =
+                        make_uint2(e1m2_to_e4m3x4(w), e1m2_to_e4m3x4(w >> 16));
             }
             if (lane % BLK == 0) {
                 const int64_t at = static_cast<int64_t>(k0 / BLK + lane / BLK) * a.scale_ld + row;

@@ -23,6 +23,7 @@ struct QuantArgs {
     int64_t K, kpad, scale_ld;
     uint8_t *codes;      // [out_rows][kpad/2]
     uint8_t *corr;       // E1M2 correction plane, same layout, or nullptr
+    uint8_t *elems8;     // E4M3 element plane [out_rows][kpad] (MX path), or nullptr
     void *scales;        // block-major [kpad/B][scale_ld], fp32 or E4M3
     float *S_out;        // two-level: receives S
     const float *amax_t; // two-level: rotated tensor amax
@@ -96,6 +97,7 @@ struct GemmArgs {
     int scale_ue8m0;                      // mode 0: scales are UE8M0 exponent bytes
     int planes3d;                         // corr = codes + rows * kpad / 2 for both
     CUtensorMap tm_c;                     // fp32 output [m][n], box 32 x 128, 128-byte swizzle
+    CUtensorMap tm_a_e8, tm_b_e8;         // MX path: E4M3 element planes [rows][kpad]
     int c_tma;                            // tm_c valid: single problem, c_vec, c_col == 0
 };
 

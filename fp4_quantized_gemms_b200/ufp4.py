@@ -52,7 +52,7 @@ class QTensorC(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("tensor_scale", ctypes.c_void_p), ("rows", ctypes.c_int64),
                 ("k", ctypes.c_int64), ("kpad", ctypes.c_int64), ("scale_ld", ctypes.c_int64),
-                ("cfg", QuantCfgC), ("corr", ctypes.c_void_p)]
+                ("cfg", QuantCfgC), ("corr", ctypes.c_void_p), ("elems8", ctypes.c_void_p)]
 
 
 class GroupC(ctypes.Structure):
@@ -187,12 +187,14 @@ class QTensor:
     scale_ld: int
     cfg: QuantConfig
     corr: torch.Tensor | None = None    # uint8 [rows, kpad/2]: E1M2 correction plane
+    elems8: torch.Tensor | None = None  # uint8 [rows, kpad]: E4M3 element plane (MX path)
 
     def c(self) -> QTensorC:
         return QTensorC(self.codes.data_ptr(), self.scales.data_ptr(),
                         self.tensor_scale.data_ptr() if self.tensor_scale is not None else None,
                         self.rows, self.k, self.kpad, self.scale_ld, self.cfg.c(),
-                        self.corr.data_ptr() if self.corr is not None else None)
+                        self.corr.data_ptr() if self.corr is not None else None,
+                        self.elems8.data_ptr() if self.elems8 is not None else None)
 
 
 def wants_corr(cfg: QuantConfig) -> bool:
@@ -200,8 +202,13 @@ def wants_corr(cfg: QuantConfig) -> bool:
     return cfg.grid == GRID_E1M2 and cfg.scale_fmt == SCALE_E4M3_X_FP32
 
 
+def wants_elems8(cfg: QuantConfig) -> bool:
+    """Operands the block-scaled FP8 GEMM reads as E4M3 elements (MX path)."""
+    return cfg.grid == GRID_E1M2 and cfg.scale_fmt == SCALE_UE8M0
+
+
 def empty_qtensor(rows: int, k: int, cfg: QuantConfig, device="cuda",
-                  with_corr: bool | None = None) -> QTensor:
+                  with_corr: bool | None = None, with_elems8: bool | None = None) -> QTensor:
     kpad, sld, _, _ = layout(rows, k, cfg)
     nblk = kpad // cfg.block
     if with_corr is None:
@@ -217,7 +224,10 @@ def empty_qtensor(rows: int, k: int, cfg: QuantConfig, device="cuda",
         scales = torch.empty((nblk, sld), dtype=torch.uint8, device=device)
         ts = torch.empty(1, dtype=torch.float32, device=device) if cfg.scale_fmt == SCALE_E4M3_X_FP32 else None
     corr = planes[1] if with_corr else None
-    return QTensor(codes, scales, ts, rows, k, kpad, sld, cfg, corr)
+    if with_elems8 is None:
+        with_elems8 = wants_elems8(cfg)
+    e8 = torch.empty((rows, kpad), dtype=torch.uint8, device=device) if with_elems8 else None
+    return QTensor(codes, scales, ts, rows, k, kpad, sld, cfg, corr, e8)
 
 
 # ---------------------------------------------------------------- entry points
@@ -252,7 +262,7 @@ def rht_bf16(x: torch.Tensor, hadamard_n: int, sign_mask: int = DEFAULT_SIGN_MAS
 
 def rht_quantize(x: torch.Tensor, axis: int, cfg: QuantConfig,
                  tensor_amax: torch.Tensor | None = None, out: QTensor | None = None,
-                 with_corr: bool | None = None) -> QTensor:
+                 with_corr: bool | None = None, with_elems8: bool | None = None) -> QTensor:
     """Fused RHT + block scale + 4-bit rounding + packing of a bf16 operand
     (plus the E1M2 correction plane when with_corr, by default for E1M2
     operands with two-level scales)."""
@@ -261,7 +271,7 @@ def rht_quantize(x: torch.Tensor, axis: int, cfg: QuantConfig,
     rows, cols = x.shape
     orows, k = (rows, cols) if axis == ALONG_COLS else (cols, rows)
     if out is None:
-        out = empty_qtensor(orows, k, cfg, device=x.device, with_corr=with_corr)
+        out = empty_qtensor(orows, k, cfg, device=x.device, with_corr=with_corr, with_elems8=with_elems8)
     if cfg.scale_fmt == SCALE_E4M3_X_FP32 and tensor_amax is None:
         tensor_amax = rht_amax(x, axis, cfg.hadamard_n, cfg.rht_sign_mask)
     qc = out.c()
@@ -290,7 +300,8 @@ def rht_amax_dual(x: torch.Tensor, hadamard_n: int, sign_mask: int = DEFAULT_SIG
 def rht_quantize_dual(x: torch.Tensor, cfg_cols: QuantConfig, cfg_rows: QuantConfig | None = None,
                       tensor_amax: torch.Tensor | None = None,
                       out: tuple[QTensor, QTensor] | None = None,
-                      with_corr: bool | None = None) -> tuple[QTensor, QTensor]:
+                      with_corr: bool | None = None,
+                      with_elems8: bool | None = None) -> tuple[QTensor, QTensor]:
     """Both quantizations of x from one read: (ALONG_COLS result, ALONG_ROWS
     result).  cfg_rows defaults to cfg_cols; the two may differ in sr_stream
     only.  tensor_amax: float32 [2] device tensor from rht_amax_dual (two-level
@@ -300,8 +311,10 @@ def rht_quantize_dual(x: torch.Tensor, cfg_cols: QuantConfig, cfg_rows: QuantCon
     cfg_rows = cfg_cols if cfg_rows is None else cfg_rows
     rows, cols = x.shape
     if out is None:
-        out = (empty_qtensor(rows, cols, cfg_cols, device=x.device, with_corr=with_corr),
-               empty_qtensor(cols, rows, cfg_rows, device=x.device, with_corr=with_corr))
+        out = (empty_qtensor(rows, cols, cfg_cols, device=x.device, with_corr=with_corr,
+                             with_elems8=with_elems8),
+               empty_qtensor(cols, rows, cfg_rows, device=x.device, with_corr=with_corr,
+                             with_elems8=with_elems8))
     if cfg_cols.scale_fmt == SCALE_E4M3_X_FP32 and tensor_amax is None:
         tensor_amax = rht_amax_dual(x, cfg_cols.hadamard_n, cfg_cols.rht_sign_mask)
     qc, qr = out[0].c(), out[1].c()

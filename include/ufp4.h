@@ -50,7 +50,9 @@
  *                                      is e_b * S with S = *tensor_scale.
  *             UFP4_SCALE_UE8M0:        u8 biased exponent E; the step of the
  *                                      block is 2^(E - 127) (tensor_scale
- *                                      unused); GEMMs run the fp32-scale kernel.
+ *                                      unused); GEMMs run the block-scaled
+ *                                      FP8 MMA when both operands carry an
+ *                                      elems8 plane, else the fp32-scale kernel.
  *   The dequantized (rotated) value of element (r, t) is s * lvl(code); the
  *   Hadamard normalisation 1/n is applied once in the GEMM (n = 0: none).
  *   corr      optional, E1M2 only: the same layout as codes, each nibble the
@@ -61,6 +63,14 @@
  *             E2M1 planes.  ufp4_rht_quantize writes it when non-NULL; the
  *             GEMMs read it when both operands carry one (else they derive it
  *             on the fly).  Must be NULL for E2M1 operands.
+ *   elems8    optional, E1M2 with UE8M0 scales only (the MX path): u8
+ *             [rows][kpad], byte t of a row the OCP E4M3 encoding of element
+ *             t's grid value +-k/4 (0x00 for zero; magnitudes 0x28, 0x30,
+ *             0x34, 0x38, 0x3A, 0x3C, 0x3E for k = 1..7; sign in bit 7), an
+ *             exact remap of the code.  ufp4_rht_quantize writes it when
+ *             non-NULL; when both GEMM operands carry one, the GEMM runs on the
+ *             block-scaled FP8 MMA with the UE8M0 factors applied in the MMA
+ *             (else on the fp32-scale kernel).  Must be NULL otherwise.
  */
 #ifndef UFP4_H
 #define UFP4_H
@@ -137,7 +147,8 @@ typedef struct {
     int64_t kpad;           /* k rounded up to 64                            */
     int64_t scale_ld;       /* rows rounded up to 64                         */
     ufp4_quant_cfg_t cfg;   /* how it was quantized                          */
-    void *corr;             /* device u8 [rows][kpad/2] or NULL, see below   */
+    void *corr;             /* device u8 [rows][kpad/2] or NULL, see above   */
+    void *elems8;           /* device u8 [rows][kpad] or NULL, see above     */
 } ufp4_qtensor_t;
 
 /* One sub-problem of ufp4_grouped_gemm:

@@ -71,6 +71,18 @@ def unpack_plane(t: torch.Tensor, rows=None) -> np.ndarray:
     return out
 
 
+E4M3_OF_E1M2 = [0x00, 0x28, 0x30, 0x34, 0x38, 0x3A, 0x3C, 0x3E]   # E4M3 bytes of k/4, k = 0..7
+
+
+def expected_elems8(codes: np.ndarray) -> np.ndarray:
+    """MX element-plane bytes from E1M2 code nibbles: the OCP E4M3 encoding of
+    +-k/4 (magnitude byte from the table, sign in bit 7)."""
+    c = codes.astype(np.int64) & 15
+    lut = np.array([E4M3_OF_E1M2[n & 7] | (0x80 if (n & 8) and (n & 7) else 0) for n in range(16)],
+                   dtype=np.uint8)
+    return lut[c]
+
+
 def assert_quant_equal(q: ufp4.QTensor, ref: oracle.QTensor, rows=None):
     if q.corr is not None:
         got_c = unpack_plane(q.corr, rows)
@@ -80,6 +92,15 @@ def assert_quant_equal(q: ufp4.QTensor, ref: oracle.QTensor, rows=None):
             r, c = bad[0]
             raise AssertionError(f"{len(bad)} correction nibbles differ; first at ({r},{c}): gpu "
                                  f"{got_c[r, c]} expected {want_c[r, c]} (code {ref.codes[r, c]})")
+    if q.elems8 is not None:
+        e = q.elems8 if rows is None else q.elems8[torch.as_tensor(rows, device=q.elems8.device)]
+        got_e = e.cpu().numpy()
+        want_e = expected_elems8(ref.codes)
+        if not np.array_equal(got_e, want_e):
+            bad = np.argwhere(got_e != want_e)
+            r, c = bad[0]
+            raise AssertionError(f"{len(bad)} E4M3 element bytes differ; first at ({r},{c}): gpu "
+                                 f"{got_e[r, c]:#x} expected {want_e[r, c]:#x} (code {ref.codes[r, c]})")
     got = unpack_codes(q, rows)
     if not np.array_equal(got, ref.codes):
         bad = np.argwhere(got != ref.codes)

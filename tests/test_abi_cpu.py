@@ -7,7 +7,9 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
+import torch
 
 from fp4_quantized_gemms_b200 import build as ufp4_build
 from fp4_quantized_gemms_b200 import ufp4
@@ -49,9 +51,9 @@ def test_struct_layouts_match_header(tmp_path):
 int main(void) {
   printf("%zu %zu %zu %zu %zu\\n", sizeof(ufp4_quant_cfg_t), offsetof(ufp4_quant_cfg_t, sr_seed),
          offsetof(ufp4_quant_cfg_t, rht_sign_mask), offsetof(ufp4_quant_cfg_t, scale_fmt), 0);
-  printf("%zu %zu %zu %zu %zu\\n", sizeof(ufp4_qtensor_t), offsetof(ufp4_qtensor_t, rows),
+  printf("%zu %zu %zu %zu %zu %zu\\n", sizeof(ufp4_qtensor_t), offsetof(ufp4_qtensor_t, rows),
          offsetof(ufp4_qtensor_t, scale_ld), offsetof(ufp4_qtensor_t, cfg),
-         offsetof(ufp4_qtensor_t, corr));
+         offsetof(ufp4_qtensor_t, corr), offsetof(ufp4_qtensor_t, elems8));
   printf("%zu %zu\\n", sizeof(ufp4_group_t), offsetof(ufp4_group_t, c_col));
   printf("%zu %zu %zu %zu %zu\\n", sizeof(ufp4_qstats_t), offsetof(ufp4_qstats_t, level_n),
          offsetof(ufp4_qstats_t, code_count), offsetof(ufp4_qstats_t, underflow),
@@ -71,7 +73,8 @@ int main(void) {
     assert c4 == [ctypes.sizeof(St), St.level_n.offset, St.code_count.offset, St.underflow.offset,
                   ctypes.sizeof(Sm)]
     assert c1[:4] == [ctypes.sizeof(Q), Q.sr_seed.offset, Q.rht_sign_mask.offset, Q.scale_fmt.offset]
-    assert c2 == [ctypes.sizeof(T), T.rows.offset, T.scale_ld.offset, T.cfg.offset, T.corr.offset]
+    assert c2 == [ctypes.sizeof(T), T.rows.offset, T.scale_ld.offset, T.cfg.offset, T.corr.offset,
+                  T.elems8.offset]
     assert c3 == [ctypes.sizeof(G), G.c_col.offset]
 
 
@@ -288,3 +291,15 @@ def test_binding_allocates_what_the_layout_call_sizes(grid, fmt, block):
     c = q.c()
     assert c.rows == 300 and c.k == 200 and c.kpad == kpad and c.scale_ld == sld
     assert c.cfg.scale_fmt == fmt and c.cfg.block == block and c.cfg.grid == grid
+
+
+def test_mx_element_table_is_the_e4m3_encoding():
+    """The MX element plane's byte table (E1M2 level k/4 -> E4M3 byte, used by
+    the GPU tests) equals torch's float8_e4m3fn encoding of k/4, and negation
+    sets bit 7 only."""
+    from tests.gpu_util import E4M3_OF_E1M2, expected_elems8
+    vals = torch.tensor([k / 4 for k in range(8)], dtype=torch.float32)
+    assert list(vals.to(torch.float8_e4m3fn).view(torch.uint8).numpy()) == E4M3_OF_E1M2
+    neg = (-vals[1:]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert list(expected_elems8(np.arange(9, 16))) == list(neg)
+    assert list(expected_elems8(np.arange(0, 8))) == E4M3_OF_E1M2

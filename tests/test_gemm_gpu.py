@@ -19,7 +19,7 @@ pytestmark = needs_gpu
 C, R = ufp4.ALONG_COLS, ufp4.ALONG_ROWS
 
 
-def _quant_both(bits, axis, cfg, rows=None):
+def _quant_both(bits, axis, cfg, rows=None, with_elems8=None):
     """GPU and oracle quantization of the same operand (optionally only some
     output rows on the oracle side)."""
     x = to_dev(bits)
@@ -27,7 +27,7 @@ def _quant_both(bits, axis, cfg, rows=None):
     if cfg.scale_fmt == ufp4.SCALE_E4M3_X_FP32:
         amax_d = ufp4.rht_amax(x, axis, cfg.hadamard_n, cfg.rht_sign_mask)
         amax_o = oracle.rht_amax(bits, axis, cfg.hadamard_n, cfg.rht_sign_mask)
-    q = ufp4.rht_quantize(x, axis, cfg, tensor_amax=amax_d)
+    q = ufp4.rht_quantize(x, axis, cfg, tensor_amax=amax_d, with_elems8=with_elems8)
     oc = oracle_cfg(cfg)
     if rows is None:
         ref = oracle.quantize(bits, axis, oc, tensor_amax=amax_o)
@@ -107,22 +107,22 @@ def test_layer_dgrad_wgrad_small(fmt, grid):
     _check_full(qdyt, rdyt, qxt, rxt, ufp4.gemm_wgrad)
 
 
-def _sampled(shape: wl.LayerShape, fmt, grid, gemm, n_rows=96, n_cols=96):
+def _sampled(shape: wl.LayerShape, fmt, grid, gemm, n_rows=96, n_cols=96, block=16):
     """One GEMM of a full-size layer in the production launch; the oracle
     computes a sampled row x column block of the output."""
     X, W, dY = wl.layer_inputs(shape, want_dy=True)
     rng = np.random.default_rng(17)
     if gemm == "fprop":
-        a_bits, a_axis, a_cfg = X, C, _cfg(grid=grid, fmt=fmt)
-        b_bits, b_axis, b_cfg = W, C, _cfg(grid=grid, fmt=fmt)
+        a_bits, a_axis, a_cfg = X, C, _cfg(grid=grid, fmt=fmt, block=block)
+        b_bits, b_axis, b_cfg = W, C, _cfg(grid=grid, fmt=fmt, block=block)
         fn = ufp4.gemm_fprop
     elif gemm == "dgrad":
-        a_bits, a_axis, a_cfg = dY, C, _cfg(grid=grid, fmt=fmt, rounding=1, stream=0)
-        b_bits, b_axis, b_cfg = W, R, _cfg(grid=grid, fmt=fmt)
+        a_bits, a_axis, a_cfg = dY, C, _cfg(grid=grid, fmt=fmt, rounding=1, stream=0, block=block)
+        b_bits, b_axis, b_cfg = W, R, _cfg(grid=grid, fmt=fmt, block=block)
         fn = ufp4.gemm_dgrad
     else:
-        a_bits, a_axis, a_cfg = dY, R, _cfg(grid=grid, fmt=fmt, rounding=1, stream=1)
-        b_bits, b_axis, b_cfg = X, R, _cfg(grid=grid, fmt=fmt)
+        a_bits, a_axis, a_cfg = dY, R, _cfg(grid=grid, fmt=fmt, rounding=1, stream=1, block=block)
+        b_bits, b_axis, b_cfg = X, R, _cfg(grid=grid, fmt=fmt, block=block)
         fn = ufp4.gemm_wgrad
     ma = a_bits.shape[0] if a_axis == C else a_bits.shape[1]
     nb = b_bits.shape[0] if b_axis == C else b_bits.shape[1]
@@ -143,19 +143,22 @@ def _sampled(shape: wl.LayerShape, fmt, grid, gemm, n_rows=96, n_cols=96):
 
 
 @pytest.mark.parametrize("gemm", ["fprop", "dgrad", "wgrad"])
-@pytest.mark.parametrize("fmt", [ufp4.SCALE_FP32, ufp4.SCALE_E4M3_X_FP32])
+@pytest.mark.parametrize("fmt", [ufp4.SCALE_FP32, ufp4.SCALE_E4M3_X_FP32, ufp4.SCALE_UE8M0])
 def test_layer_config_sampled(gemm, fmt):
-    """X 8192x2048 (10 outlier channels x30), W 8192x2048, dY 8192x8192."""
-    _sampled(wl.LAYER, fmt, ufp4.GRID_E1M2, gemm)
+    """X 8192x2048 (10 outlier channels x30), W 8192x2048, dY 8192x8192
+    (MX scales: block 32, the block-scaled FP8 path)."""
+    _sampled(wl.LAYER, fmt, ufp4.GRID_E1M2, gemm, block=32 if fmt == ufp4.SCALE_UE8M0 else 16)
 
 
 @pytest.mark.parametrize("gemm", ["fprop", "dgrad", "wgrad"])
 @pytest.mark.parametrize("fmt,grid", [(ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E1M2),
                                       (ufp4.SCALE_FP32, ufp4.GRID_E1M2),
-                                      (ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E2M1)])
+                                      (ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E2M1),
+                                      (ufp4.SCALE_UE8M0, ufp4.GRID_E1M2)])
 def test_large_config_sampled(gemm, fmt, grid):
     """M=16384, K=8192, N=28672 (1% outlier channels x50): the largest layer."""
-    _sampled(wl.LARGE, fmt, grid, gemm, n_rows=64, n_cols=64)
+    _sampled(wl.LARGE, fmt, grid, gemm, n_rows=64, n_cols=64,
+             block=32 if fmt == ufp4.SCALE_UE8M0 else 16)
 
 
 @pytest.mark.parametrize("path", [ufp4.GEMM_PATH_NATIVE_FP4, ufp4.GEMM_PATH_NATIVE_FP4_PAIR, ufp4.GEMM_PATH_NATIVE_FP4_PAIR256,
@@ -212,16 +215,20 @@ def test_e2m1_reference_recipe_layer(fmt):
 
 
 # ------------------------------------------------------------------ MX block scales
-@pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1, ufp4.GRID_E2M1_MAX2])
-def test_ue8m0_gemms(grid):
-    """UE8M0 (MX, block 32) operands through the fp32-scale kernel: FPROP on
-    ragged shapes, and DGRAD / WGRAD of a small layer with SR on dY."""
-    for (M, N, K) in [(300, 200, 200), (129, 257, 136), (1, 1, 8)]:
+@pytest.mark.parametrize("grid,e8", [(ufp4.GRID_E1M2, True), (ufp4.GRID_E1M2, False),
+                                     (ufp4.GRID_E2M1, False), (ufp4.GRID_E2M1_MAX2, False)])
+def test_ue8m0_gemms(grid, e8):
+    """UE8M0 (MX, block 32) operands: E1M2 with E4M3 element planes on the
+    block-scaled FP8 MMA (factors in the MMA), otherwise through the
+    fp32-scale kernel.  FPROP on ragged shapes (partial 256-wide tiles, K
+    tails of 64), and DGRAD / WGRAD of a small layer with SR on dY."""
+    for (M, N, K) in [(300, 200, 200), (129, 257, 136), (1, 1, 8), (520, 700, 448)]:
         X = wl.normal_with_outlier_channels(M, K, 1.0, 2, 20.0)
         W = wl.normal(N, K, 0.02, 2)
         cfg = _cfg(grid=grid, fmt=ufp4.SCALE_UE8M0, block=32)
-        qx, rx = _quant_both(X, C, cfg)
-        qw, rw = _quant_both(W, C, cfg)
+        qx, rx = _quant_both(X, C, cfg, with_elems8=e8)
+        qw, rw = _quant_both(W, C, cfg, with_elems8=e8)
+        assert (qx.elems8 is not None) == e8
         _check_full(qx, rx, qw, rw, ufp4.gemm_fprop)
     M, K, N = 384, 320, 264
     X = wl.normal_with_outlier_channels(M, K, 1.0, 3, 30.0)
@@ -230,9 +237,9 @@ def test_ue8m0_gemms(grid):
     rt = _cfg(grid=grid, fmt=ufp4.SCALE_UE8M0, block=32)
     sr0 = _cfg(grid=grid, fmt=ufp4.SCALE_UE8M0, block=32, rounding=1, stream=0)
     sr1 = _cfg(grid=grid, fmt=ufp4.SCALE_UE8M0, block=32, rounding=1, stream=1)
-    qdy, rdy = _quant_both(dY, C, sr0)
-    qwt, rwt = _quant_both(W, R, rt)
+    qdy, rdy = _quant_both(dY, C, sr0, with_elems8=e8)
+    qwt, rwt = _quant_both(W, R, rt, with_elems8=e8)
     _check_full(qdy, rdy, qwt, rwt, ufp4.gemm_dgrad)
-    qdyt, rdyt = _quant_both(dY, R, sr1)
-    qxt, rxt = _quant_both(X, R, rt)
+    qdyt, rdyt = _quant_both(dY, R, sr1, with_elems8=e8)
+    qxt, rxt = _quant_both(X, R, rt, with_elems8=e8)
     _check_full(qdyt, rdyt, qxt, rxt, ufp4.gemm_wgrad)
