@@ -414,21 +414,24 @@ def fused_vs_unfused(x: torch.Tensor, flush) -> dict:
 
 # ------------------------------------------------------------------ side measurements
 def run_mx(step: LayerStep, reps: int = 3) -> dict:
-    """The layer's FPROP with MX block scales (UE8M0, block 32): quantize X and
-    W (dual calls) and the GEMM through the fp32-block-scale kernel, timed
-    with CUDA events (reported, not in `value`)."""
+    """The layer's FPROP with MX block scales (UE8M0, block 32): X and W are
+    quantized by the dual calls, which also write the E4M3 element planes, and
+    the GEMM runs the block-scaled FP8 MMA on CTA pairs.  Both timed with CUDA
+    events (reported, not in `value`)."""
     u = step.u
     cfg = u.QuantConfig(grid=u.GRID_E1M2, hadamard_n=16, block=32, scale_fmt=u.SCALE_UE8M0)
     s = step.shape
-    qx, _ = u.rht_quantize_dual(step.X, cfg)
-    qw, _ = u.rht_quantize_dual(step.W, cfg)
+    qx, qxr = u.rht_quantize_dual(step.X, cfg)
+    qw, qwr = u.rht_quantize_dual(step.W, cfg)
     out = torch.empty((s.M, s.N), dtype=torch.float32, device=step.dev)
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=step.dev)
     t_g = _timed(lambda: u.gemm_fprop(qx, qw, out), flush, reps=reps, warm=1)
-    del out, qx, qw, flush
+    t_q = _timed(lambda: u.rht_quantize_dual(step.X, cfg, out=(qx, qxr)), flush, reps=reps, warm=1)
+    del out, qx, qw, qxr, qwr, flush
     return {"fprop_ms": round(t_g, 4),
             "fprop_TFLOPs": round(2 * s.M * s.N * s.K / (t_g * 1e-3) / 1e12, 1),
-            "kernel": "gemm_tn_kernel<0> (kind::f16 per-block partials, exponent-byte scales)"}
+            "quantize_X_dual_ms": round(t_q, 4),
+            "kernel": "gemm_pair_kernel<3> (kind::mxf8f6f4 block32, E4M3 elements, UE8M0 factors)"}
 
 
 def run_moe(device, two_level: bool, reps: int = 10):

@@ -72,6 +72,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // Common checks of one quantized operand descriptor.
+// Factor-atom slot width along K: 16 for E4M3 factors (the block16 MMA
+// granularity), 32 for UE8M0; 0 = fp32 scales (no atoms).
+int atom_slot(const ufp4_quant_cfg_t &c) {
+    return c.scale_fmt == UFP4_SCALE_E4M3_X_FP32 ? 16 : c.scale_fmt == UFP4_SCALE_UE8M0 ? 32 : 0;
+}
+
+int64_t atoms_k_of(int64_t kpad, const ufp4_quant_cfg_t &c) {
+    const int64_t w = 4 * atom_slot(c);
+    return (kpad + w - 1) / w;
+}
+
 ufp4_status_t check_qtensor(const ufp4_qtensor_t *q) {
     if (q == nullptr) return UFP4_ERR_INVALID_ARG;
     if (!cfg_valid(q->cfg)) return UFP4_ERR_INVALID_ARG;
@@ -91,6 +102,10 @@ ufp4_status_t check_qtensor(const ufp4_qtensor_t *q) {
     if (q->elems8 != nullptr) {   // E4M3 element plane of an MX (UE8M0) E1M2 operand
         if (q->cfg.grid != UFP4_GRID_E1M2 || q->cfg.scale_fmt != UFP4_SCALE_UE8M0) return UFP4_ERR_INVALID_ARG;
         if (!aligned16(q->elems8)) return UFP4_ERR_ALIGNMENT;
+    }
+    if (q->sf_atoms != nullptr) {   // factor atoms: byte block scales only
+        if (atom_slot(q->cfg) == 0) return UFP4_ERR_INVALID_ARG;
+        if (!aligned16(q->sf_atoms)) return UFP4_ERR_ALIGNMENT;
     }
     if (q->rows > (int64_t(1) << 31) || q->kpad > (int64_t(1) << 31)) return UFP4_ERR_UNSUPPORTED;
     return UFP4_OK;
@@ -282,6 +297,24 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
         }
         args.corr_in = 1;
     }
+    // Dense problems on the CTA-pair kernels whose operands both carry factor
+    // atoms: each stage's atoms come with its code tiles (one u64 box of
+    // 128 K elements per 128-row group: two atoms of E4M3 factors, one of
+    // UE8M0) and the MMA issuer copies them into tensor memory.
+    if ((mode == 5 || mode == 6) && groups_dev == nullptr && a->sf_atoms != nullptr && b->sf_atoms != nullptr &&
+        a->rows > 0 && b->rows > 0) {
+        const int64_t ak = atoms_k_of(a->kpad, a->cfg);
+        const uint32_t box_k = static_cast<uint32_t>(64 * (128 / (4 * atom_slot(a->cfg))));
+        CUresult r = encode_tensor_map_2d(&args.tm_a_atoms, CU_TENSOR_MAP_DATA_TYPE_UINT64, a->sf_atoms,
+                                          static_cast<uint64_t>(64 * ak), static_cast<uint64_t>((a->rows + 127) / 128),
+                                          static_cast<uint64_t>(ak) * 512, box_k, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
+        r = encode_tensor_map_2d(&args.tm_b_atoms, CU_TENSOR_MAP_DATA_TYPE_UINT64, b->sf_atoms,
+                                 static_cast<uint64_t>(64 * ak), static_cast<uint64_t>((b->rows + 127) / 128),
+                                 static_cast<uint64_t>(ak) * 512, box_k, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
+        args.atoms = 1;
+    }
     // Native kernels store 16-byte pieces when the output allows it.
     args.c_vec = (aligned16(c) && ldc % 4 == 0) ? 1 : 0;
     // The CTA-pair kernel writes whole 128 x 32 output pieces with TMA bulk
@@ -334,6 +367,8 @@ ufp4_status_t fill_quant_args(const void *x_dev, int64_t rows, int64_t cols, int
     a->codes = static_cast<uint8_t *>(out->codes);
     a->corr = static_cast<uint8_t *>(out->corr);
     a->elems8 = static_cast<uint8_t *>(out->elems8);
+    a->sf_atoms = static_cast<uint8_t *>(out->sf_atoms);
+    a->atoms_k = out->sf_atoms != nullptr ? atoms_k_of(out->kpad, out->cfg) : 0;
     a->scales = out->scales;
     a->S_out = two_level ? out->tensor_scale : nullptr;
     a->amax_t = two_level ? tensor_amax_dev : nullptr;
@@ -406,6 +441,16 @@ ufp4_status_t ufp4_qtensor_layout(int64_t rows, int64_t k, const ufp4_quant_cfg_
     if (scale_ld) *scale_ld = sl;
     if (codes_bytes) *codes_bytes = static_cast<size_t>(rows * (kp / 2));
     if (scales_bytes) *scales_bytes = static_cast<size_t>((kp / cfg->block) * sl * elt);
+    return UFP4_OK;
+}
+
+ufp4_status_t ufp4_sf_atoms_layout(int64_t rows, int64_t k, const ufp4_quant_cfg_t *cfg, int64_t *atoms_k,
+                                   size_t *bytes) {
+    if (cfg == nullptr || rows < 0 || k < 0 || !cfg_valid(*cfg)) return UFP4_ERR_INVALID_ARG;
+    if (atom_slot(*cfg) == 0) return UFP4_ERR_UNSUPPORTED;
+    const int64_t ak = atoms_k_of(round_up(k, kKAlign), *cfg);
+    if (atoms_k) *atoms_k = ak;
+    if (bytes) *bytes = static_cast<size_t>((rows + 127) / 128 * ak * 512);
     return UFP4_OK;
 }
 

@@ -1389,7 +1389,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
 // byte per element, 128-byte rows, 128-byte swizzle), UE8M0 factors per 32
 // elements applied in the MMA (kind::mxf8f6f4, K = 32 per MMA, four MMAs per
 // stage picking byte j of the same factor atom).
-template <int GRID>
+template <int GRID, bool ATOMS>
 struct PairCfg {
     static constexpr bool kMx = GRID == 3;
     static constexpr int TM = 256;
@@ -1409,7 +1409,8 @@ struct PairCfg {
     static constexpr int kRawB = 256 * kRawRows;
     static constexpr int kStage = (kCodeBytes + kRawA + kRawB + 1023) / 1024 * 1024;
     static constexpr int kAtoms = 3 * KST;          // SFA, SFB rows 0-127, SFB rows 128-255 per K step
-    static constexpr int kScr = 4 * kAtoms * 512;   // one atom scratch per factor warp
+    static constexpr int kAtomX = 64 * KST;         // u64 units of one stage's atoms along K (ATOMS)
+    static constexpr int kScr = ATOMS ? 0 : 4 * kAtoms * 512;   // one atom scratch per factor warp
     static constexpr int kOutChunk = 128 * 32 * 4;  // epilogue staging: 128 rows x 32 fp32
     static constexpr int kOutBufs = 2;              // staging buffers (bulk stores in flight)
     static constexpr int kSfBase = 256;             // TMEM column of the first factor slot
@@ -1431,6 +1432,17 @@ struct PairCfg {
     static_assert(kAlloc <= 232448, "shared memory budget");
     static_assert(kSfBase + NS * kSfCols <= 512, "TMEM budget");
 };
+
+// Copy of one 512-byte factor atom (32 rows of 16 bytes, row i at byte 16 i)
+// from shared memory into TMEM columns [taddr, taddr + 4) of all four lane
+// quarters, in both CTAs of the pair (each from its own shared memory at the
+// same address).  Descriptor: no swizzle, K-major, core matrices of 8 rows x
+// 16 bytes at a stride of 128 bytes (SBO); one core matrix along K (LBO unused).
+__device__ __forceinline__ void tmem_cp_atom_pair(uint32_t taddr, uint32_t smem_byte_addr) {
+    const uint64_t d = static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFFu) |
+                       (static_cast<uint64_t>(128u >> 4) << 32) | (static_cast<uint64_t>(1u) << 46);
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
+}
 
 // TMA tile loads whose completion is counted on a barrier of the leader CTA
 // of the pair (`bar_cluster`: a shared::cluster address from mapa).  The
@@ -1485,10 +1497,10 @@ __host__ __device__ constexpr uint32_t umma_idesc_mxf8(int M, int N, uint32_t sf
            | (sf_id << 29);                           // A factor byte
 }
 
-template <int GRID>
-__global__ void __launch_bounds__(PairCfg<GRID>::kThreads, 1)
+template <int GRID, bool ATOMS>
+__global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ GemmArgs args) {
-    using C = PairCfg<GRID>;
+    using C = PairCfg<GRID, ATOMS>;
     constexpr int TM = C::TM, BN = C::BN, NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -1530,8 +1542,8 @@ __global__ void __launch_bounds__(PairCfg<GRID>::kThreads, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(GRID == 0 ? &args.tm_a_corr : (C::kMx ? &args.tm_a_e8 : &args.tm_a_codes));
         tma_prefetch_desc(GRID == 0 ? &args.tm_b_corr : (C::kMx ? &args.tm_b_e8 : &args.tm_b_codes));
-        tma_prefetch_desc(&args.tm_a_scales);
-        tma_prefetch_desc(&args.tm_b_scales);
+        tma_prefetch_desc(ATOMS ? &args.tm_a_atoms : &args.tm_a_scales);
+        tma_prefetch_desc(ATOMS ? &args.tm_b_atoms : &args.tm_b_scales);
     }
     if (warp == 1) tmem_alloc_pair(tmem_slot, 512);
     tc_fence_before();
@@ -1562,13 +1574,22 @@ __global__ void __launch_bounds__(PairCfg<GRID>::kThreads, 1)
                     const int32_t acol = static_cast<int32_t>(tl.g.a_col + ks * C::BKE);
                     const int32_t bcol = static_cast<int32_t>(tl.g.b_col + ks * C::BKE);
                     uint8_t *st = stage(s);
-                    // this CTA's raw factors
-                    mbar_arrive_expect_tx(&sfull[s], (128 + 256) * nraw);
-                    tma_load_2d_hint(st + C::o_raw_a, &args.tm_a_scales, &sfull[s], arow, acol / blk, pol);
-                    tma_load_2d_hint(st + C::o_raw_b, &args.tm_b_scales, &sfull[s], brow, bcol / blk, pol);
-                    // code tiles of both CTAs complete on the leader's barrier
-                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::kCodeBytes);
                     const uint32_t fb = cluster_addr(&full[s], 0);
+                    if constexpr (ATOMS) {
+                        // factor atoms of this CTA's A rows and of all 256 B rows, with the
+                        // code tiles on the leader's barrier: 128 K elements per box
+                        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (C::kCodeBytes + C::kRawA + C::kRawB));
+                        const int32_t ax = static_cast<int32_t>(C::kAtomX * ks);
+                        tma_load_2d_pair(st + C::o_raw_a, &args.tm_a_atoms, fb, ax, arow / 128, pol);
+                        tma_load_2d_pair(st + C::o_raw_b, &args.tm_b_atoms, fb, ax, brow / 128, pol);
+                    } else {
+                        // this CTA's raw factors
+                        mbar_arrive_expect_tx(&sfull[s], (128 + 256) * nraw);
+                        tma_load_2d_hint(st + C::o_raw_a, &args.tm_a_scales, &sfull[s], arow, acol / blk, pol);
+                        tma_load_2d_hint(st + C::o_raw_b, &args.tm_b_scales, &sfull[s], brow, bcol / blk, pol);
+                        // code tiles of both CTAs complete on the leader's barrier
+                        if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::kCodeBytes);
+                    }
                     if (GRID == 0) {
                         tma_load_3d_pair(st + C::o_a, &args.tm_a_corr, fb, acol / 2, arow, 0, pol);
                         tma_load_3d_pair(st + C::o_b, &args.tm_b_corr, fb, bcol / 2, brow_h, 0, pol);
@@ -1586,8 +1607,9 @@ __global__ void __launch_bounds__(PairCfg<GRID>::kThreads, 1)
             for (uint32_t d = 0; d < static_cast<uint32_t>(NS) && d < it; ++d) {
                 const uint32_t idx = it - 1 - d;
                 uint32_t dummy = 0;
-                mbar_wait(&sfull[idx % NS], (idx / NS) & 1, kErrTimeoutDrain,
-                          reinterpret_cast<volatile uint32_t *>(&dummy));
+                if (!ATOMS)
+                    mbar_wait(&sfull[idx % NS], (idx / NS) & 1, kErrTimeoutDrain,
+                              reinterpret_cast<volatile uint32_t *>(&dummy));
                 if (rank == 0)
                     mbar_wait_cluster(&full[idx % NS], (idx / NS) & 1, kErrTimeoutDrain,
                                       reinterpret_cast<volatile uint32_t *>(&dummy));
@@ -1608,13 +1630,24 @@ __global__ void __launch_bounds__(PairCfg<GRID>::kThreads, 1)
                 for (int ks = 0; ks < nks; ++ks, ++it) {
                     const int s = it % NS;
                     if (!mbar_wait(&full[s], (it / NS) & 1, kErrTimeoutMma, abort_flag) ||
-                        !mbar_wait_cluster(&sfready[s], (it / NS) & 1, kErrTimeoutMma, abort_flag)) {
+                        (!ATOMS && !mbar_wait_cluster(&sfready[s], (it / NS) & 1, kErrTimeoutMma, abort_flag))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     uint8_t *st = stage(s);
                     const uint32_t sf0 = tmem_base + C::kSfBase + s * C::kSfCols;
+                    if constexpr (ATOMS) {
+                        // the stage's factor atoms into TMEM slot s of both CTAs (each from its
+                        // own shared memory; the copies run before the MMAs issued after them,
+                        // and after the MMAs that last read the slot)
+#pragma unroll
+                        for (int j = 0; j < C::KST; ++j) {
+                            tmem_cp_atom_pair(sf0 + 12 * j, smem_addr(st + C::o_raw_a + 512 * j));
+                            tmem_cp_atom_pair(sf0 + 12 * j + 4, smem_addr(st + C::o_raw_b + 512 * j));
+                            tmem_cp_atom_pair(sf0 + 12 * j + 8, smem_addr(st + C::o_raw_b + 512 * (C::KST + j)));
+                        }
+                    }
                     const int64_t rem = tl.g.k - static_cast<int64_t>(ks) * C::BKE;
                     const int steps = rem >= C::BKE ? C::KST : static_cast<int>((rem + 63) / 64);
                     const uint32_t a0 = smem_addr(st + C::o_a), b0 = smem_addr(st + C::o_b);
@@ -1660,7 +1693,7 @@ __global__ void __launch_bounds__(PairCfg<GRID>::kThreads, 1)
         // ------------------------------------------------------------ factor relay (peer)
         // One cluster-scope arrive per stage on the leader's barrier once the
         // peer's four factor warps are done (their arrives stay CTA-local).
-        if (lane == 0 && rank == 1) {
+        if (!ATOMS && lane == 0 && rank == 1) {
             const uint32_t ready = cluster_addr(&sfready[0], 0);
             uint32_t it = 0;
             bool ok = true;
@@ -1679,7 +1712,7 @@ __global__ void __launch_bounds__(PairCfg<GRID>::kThreads, 1)
                 }
             }
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (!ATOMS && warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ factor writers
         uint8_t *scr = smem + C::o_scr + (warp - 4) * (C::kAtoms * 512);
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
@@ -1854,13 +1887,13 @@ __global__ void __launch_bounds__(PairCfg<GRID>::kThreads, 1)
     }
 }
 
-template <int GRID>
+template <int GRID, bool ATOMS>
 cudaError_t launch_pair(const GemmArgs &args, int num_sms, cudaStream_t stream) {
-    using C = PairCfg<GRID>;
+    using C = PairCfg<GRID, ATOMS>;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<GRID>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::kAlloc);
+        cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<GRID, ATOMS>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc);
         if (e != cudaSuccess) return e;
         configured = true;
     }
@@ -1883,7 +1916,7 @@ cudaError_t launch_pair(const GemmArgs &args, int num_sms, cudaStream_t stream) 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<GRID>, args);
+    return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<GRID, ATOMS>, args);
 }
 
 template <int GRID, int CG, bool CIN>
@@ -1970,9 +2003,13 @@ cudaError_t launch_gemm(const GemmArgs &args, int mode, int grid_kind, int num_s
             return args.corr_in ? launch_fp4<0, 1, true>(args, num_sms, stream)
                                 : launch_fp4<0, 1, false>(args, num_sms, stream);
         case 5:
-            return grid_kind == 1 ? launch_pair<1>(args, num_sms, stream) : launch_pair<0>(args, num_sms, stream);
+            if (args.atoms)
+                return grid_kind == 1 ? launch_pair<1, true>(args, num_sms, stream)
+                                      : launch_pair<0, true>(args, num_sms, stream);
+            return grid_kind == 1 ? launch_pair<1, false>(args, num_sms, stream)
+                                  : launch_pair<0, false>(args, num_sms, stream);
         case 6:
-            return launch_pair<3>(args, num_sms, stream);
+            return args.atoms ? launch_pair<3, true>(args, num_sms, stream) : launch_pair<3, false>(args, num_sms, stream);
         default:
             if (grid_kind == 1) return launch_fp4<1, 2, false>(args, num_sms, stream);
             return args.corr_in ? launch_fp4<0, 2, true>(args, num_sms, stream)

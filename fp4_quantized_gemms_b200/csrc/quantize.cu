@@ -463,8 +463,28 @@ __device__ __forceinline__ uint32_t e1m2_to_e4m3x4(uint32_t w16) {
     return mag | ((v & 0x08080808u) << 4);
 }
 
+// Factor atoms: byte 16 (r % 32) + 4 ((r / 32) % 4) + slot % 4 of the
+// 512-byte atom (r / 128, slot / 4) holds the factor of K slot `slot` of row
+// r (slots of 16 elements for E4M3 factors, 32 for UE8M0).
+__device__ __forceinline__ uint8_t *atom_byte(const QuantArgs &a, int32_t row, int32_t slot) {
+    return a.sf_atoms + (static_cast<int64_t>(row >> 7) * a.atoms_k + (slot >> 2)) * 512 + 16 * (row & 31) +
+           4 * ((row >> 5) & 3) + (slot & 3);
+}
+
+// The atom bytes of one block factor (stored value `sv`) of block `blk_idx`:
+// UE8M0 fills one 32-element slot, an E4M3 factor of a 16-block one slot,
+// of a 32-block its two 16-element slots.
+template <int BLK>
+__device__ __forceinline__ void store_atom(const QuantArgs &a, int32_t row, int32_t blk_idx, uint32_t sv) {
+    const uint32_t b = sv & 0xFFu;
+    if (a.scale_fmt == 2 || BLK == 16)
+        *atom_byte(a, row, blk_idx) = static_cast<uint8_t>(b);
+    else
+        *reinterpret_cast<uint16_t *>(atom_byte(a, row, 2 * blk_idx)) = static_cast<uint16_t>(b | (b << 8));
+}
+
 // Stores the 16 code bytes (and the E1M2 correction plane, the MX element
-// plane) and the block scales of one lane run.
+// plane) and the block scales (and factor atoms) of one lane run.
 template <int BLK>
 __device__ __forceinline__ void store_run(const QuantArgs &a, int32_t row, int32_t k0, const uint32_t *w,
                                           const uint32_t *st) {
@@ -488,6 +508,13 @@ __device__ __forceinline__ void store_run(const QuantArgs &a, int32_t row, int32
             reinterpret_cast<uint32_t *>(a.scales)[at] = st[b];
         else
             reinterpret_cast<uint8_t *>(a.scales)[at] = static_cast<uint8_t>(st[b]);
+    }
+    if (a.sf_atoms != nullptr) {
+        if (BLK == 16 && a.scale_fmt != 2)   // two adjacent 16-slots: one 16-bit store
+            *reinterpret_cast<uint16_t *>(atom_byte(a, row, k0 / 16)) =
+                static_cast<uint16_t>((st[0] & 0xFFu) | ((st[1] & 0xFFu) << 8));
+        else
+            store_atom<BLK>(a, row, k0 / BLK, st[0]);
     }
 }
 
@@ -599,6 +626,7 @@ __device__ __forceinline__ void coop_exact(const QuantArgs &a, const uint8_t *ti
                 const int64_t at = static_cast<int64_t>(k0 / BLK + lane / BLK) * a.scale_ld + row;
                 if (a.scale_fmt == 0) reinterpret_cast<uint32_t *>(a.scales)[at] = stv[ln];
                 else reinterpret_cast<uint8_t *>(a.scales)[at] = static_cast<uint8_t>(stv[ln]);
+                if (a.sf_atoms != nullptr) store_atom<BLK>(a, row, k0 / BLK + lane / BLK, stv[ln]);
             }
         }
     }

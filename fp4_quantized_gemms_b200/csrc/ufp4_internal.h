@@ -24,6 +24,8 @@ struct QuantArgs {
     uint8_t *codes;      // [out_rows][kpad/2]
     uint8_t *corr;       // E1M2 correction plane, same layout, or nullptr
     uint8_t *elems8;     // E4M3 element plane [out_rows][kpad] (MX path), or nullptr
+    uint8_t *sf_atoms;   // factor atoms [ceil(out_rows/128)][atoms_k][512], or nullptr
+    int64_t atoms_k;     // atoms along K (kpad / 64 for E4M3 factors, kpad / 128 rounded up for UE8M0)
     void *scales;        // block-major [kpad/B][scale_ld], fp32 or E4M3
     float *S_out;        // two-level: receives S
     const float *amax_t; // two-level: rotated tensor amax
@@ -99,6 +101,8 @@ struct GemmArgs {
     CUtensorMap tm_c;                     // fp32 output [m][n], box 32 x 128, 128-byte swizzle
     CUtensorMap tm_a_e8, tm_b_e8;         // MX path: E4M3 element planes [rows][kpad]
     int c_tma;                            // tm_c valid: single problem, c_vec, c_col == 0
+    CUtensorMap tm_a_atoms, tm_b_atoms;   // factor atoms as u64 [row groups][64 atoms_k]
+    int atoms;                            // both operands carry factor atoms (pair kernels)
 };
 
 // Tile columns (B rows) of the native block-scaled FP4 kernels (modes 3, 4).

@@ -32,6 +32,7 @@ EXPORTED = [
     "ufp4_status_string", "ufp4_version", "ufp4_set_two_level_gemm_path",
     "ufp4_get_two_level_gemm_path", "ufp4_rht_quantize_dual", "ufp4_rht_amax_dual",
     "ufp4_quant_stats", "ufp4_qstats_summarize", "ufp4_sqnr_sums", "ufp4_rht_bf16",
+    "ufp4_sf_atoms_layout",
 ]
 
 
@@ -52,7 +53,8 @@ class QTensorC(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("tensor_scale", ctypes.c_void_p), ("rows", ctypes.c_int64),
                 ("k", ctypes.c_int64), ("kpad", ctypes.c_int64), ("scale_ld", ctypes.c_int64),
-                ("cfg", QuantCfgC), ("corr", ctypes.c_void_p), ("elems8", ctypes.c_void_p)]
+                ("cfg", QuantCfgC), ("corr", ctypes.c_void_p), ("elems8", ctypes.c_void_p),
+                ("sf_atoms", ctypes.c_void_p)]
 
 
 class GroupC(ctypes.Structure):
@@ -188,13 +190,15 @@ class QTensor:
     cfg: QuantConfig
     corr: torch.Tensor | None = None    # uint8 [rows, kpad/2]: E1M2 correction plane
     elems8: torch.Tensor | None = None  # uint8 [rows, kpad]: E4M3 element plane (MX path)
+    sf_atoms: torch.Tensor | None = None  # uint8 [ceil(rows/128), atoms_k, 512]: factor atoms
 
     def c(self) -> QTensorC:
         return QTensorC(self.codes.data_ptr(), self.scales.data_ptr(),
                         self.tensor_scale.data_ptr() if self.tensor_scale is not None else None,
                         self.rows, self.k, self.kpad, self.scale_ld, self.cfg.c(),
                         self.corr.data_ptr() if self.corr is not None else None,
-                        self.elems8.data_ptr() if self.elems8 is not None else None)
+                        self.elems8.data_ptr() if self.elems8 is not None else None,
+                        self.sf_atoms.data_ptr() if self.sf_atoms is not None else None)
 
 
 def wants_corr(cfg: QuantConfig) -> bool:
@@ -207,8 +211,24 @@ def wants_elems8(cfg: QuantConfig) -> bool:
     return cfg.grid == GRID_E1M2 and cfg.scale_fmt == SCALE_UE8M0
 
 
+def wants_atoms(cfg: QuantConfig) -> bool:
+    """Byte block scales: the CTA-pair GEMMs copy factor atoms into tensor
+    memory directly."""
+    return cfg.scale_fmt != SCALE_FP32
+
+
+def sf_atoms_layout(rows: int, k: int, cfg: QuantConfig) -> tuple[int, int]:
+    """(atoms_k, bytes) of the factor-atom plane of a [rows, k] operand."""
+    ak, nb = ctypes.c_int64(), ctypes.c_size_t()
+    c = cfg.c()
+    _check(lib().ufp4_sf_atoms_layout(rows, k, ctypes.byref(c), ctypes.byref(ak), ctypes.byref(nb)),
+           "ufp4_sf_atoms_layout")
+    return ak.value, nb.value
+
+
 def empty_qtensor(rows: int, k: int, cfg: QuantConfig, device="cuda",
-                  with_corr: bool | None = None, with_elems8: bool | None = None) -> QTensor:
+                  with_corr: bool | None = None, with_elems8: bool | None = None,
+                  with_atoms: bool | None = None) -> QTensor:
     kpad, sld, _, _ = layout(rows, k, cfg)
     nblk = kpad // cfg.block
     if with_corr is None:
@@ -227,7 +247,13 @@ def empty_qtensor(rows: int, k: int, cfg: QuantConfig, device="cuda",
     if with_elems8 is None:
         with_elems8 = wants_elems8(cfg)
     e8 = torch.empty((rows, kpad), dtype=torch.uint8, device=device) if with_elems8 else None
-    return QTensor(codes, scales, ts, rows, k, kpad, sld, cfg, corr, e8)
+    if with_atoms is None:
+        with_atoms = wants_atoms(cfg)
+    atoms = None
+    if with_atoms:
+        ak, _ = sf_atoms_layout(rows, k, cfg)
+        atoms = torch.empty(((rows + 127) // 128, ak, 512), dtype=torch.uint8, device=device)
+    return QTensor(codes, scales, ts, rows, k, kpad, sld, cfg, corr, e8, atoms)
 
 
 # ---------------------------------------------------------------- entry points
@@ -262,16 +288,19 @@ def rht_bf16(x: torch.Tensor, hadamard_n: int, sign_mask: int = DEFAULT_SIGN_MAS
 
 def rht_quantize(x: torch.Tensor, axis: int, cfg: QuantConfig,
                  tensor_amax: torch.Tensor | None = None, out: QTensor | None = None,
-                 with_corr: bool | None = None, with_elems8: bool | None = None) -> QTensor:
+                 with_corr: bool | None = None, with_elems8: bool | None = None,
+                 with_atoms: bool | None = None) -> QTensor:
     """Fused RHT + block scale + 4-bit rounding + packing of a bf16 operand
     (plus the E1M2 correction plane when with_corr, by default for E1M2
-    operands with two-level scales)."""
+    operands with two-level scales; the MX element plane; factor atoms, by
+    default for byte block scales)."""
     _require_cuda(x, tensor_amax)
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     rows, cols = x.shape
     orows, k = (rows, cols) if axis == ALONG_COLS else (cols, rows)
     if out is None:
-        out = empty_qtensor(orows, k, cfg, device=x.device, with_corr=with_corr, with_elems8=with_elems8)
+        out = empty_qtensor(orows, k, cfg, device=x.device, with_corr=with_corr, with_elems8=with_elems8,
+                            with_atoms=with_atoms)
     if cfg.scale_fmt == SCALE_E4M3_X_FP32 and tensor_amax is None:
         tensor_amax = rht_amax(x, axis, cfg.hadamard_n, cfg.rht_sign_mask)
     qc = out.c()
@@ -301,7 +330,8 @@ def rht_quantize_dual(x: torch.Tensor, cfg_cols: QuantConfig, cfg_rows: QuantCon
                       tensor_amax: torch.Tensor | None = None,
                       out: tuple[QTensor, QTensor] | None = None,
                       with_corr: bool | None = None,
-                      with_elems8: bool | None = None) -> tuple[QTensor, QTensor]:
+                      with_elems8: bool | None = None,
+                      with_atoms: bool | None = None) -> tuple[QTensor, QTensor]:
     """Both quantizations of x from one read: (ALONG_COLS result, ALONG_ROWS
     result).  cfg_rows defaults to cfg_cols; the two may differ in sr_stream
     only.  tensor_amax: float32 [2] device tensor from rht_amax_dual (two-level
@@ -312,9 +342,9 @@ def rht_quantize_dual(x: torch.Tensor, cfg_cols: QuantConfig, cfg_rows: QuantCon
     rows, cols = x.shape
     if out is None:
         out = (empty_qtensor(rows, cols, cfg_cols, device=x.device, with_corr=with_corr,
-                             with_elems8=with_elems8),
+                             with_elems8=with_elems8, with_atoms=with_atoms),
                empty_qtensor(cols, rows, cfg_rows, device=x.device, with_corr=with_corr,
-                             with_elems8=with_elems8))
+                             with_elems8=with_elems8, with_atoms=with_atoms))
     if cfg_cols.scale_fmt == SCALE_E4M3_X_FP32 and tensor_amax is None:
         tensor_amax = rht_amax_dual(x, cfg_cols.hadamard_n, cfg_cols.rht_sign_mask)
     qc, qr = out[0].c(), out[1].c()

@@ -71,6 +71,22 @@
  *             non-NULL; when both GEMM operands carry one, the GEMM runs on the
  *             block-scaled FP8 MMA with the UE8M0 factors applied in the MMA
  *             (else on the fp32-scale kernel).  Must be NULL otherwise.
+ *   sf_atoms  optional, byte block scales only (E4M3 x fp32 or UE8M0): the
+ *             same factors again, in the layout the block-scaled tensor-core
+ *             MMA reads its scale factors from (a copy per 32-lane quarter of
+ *             tensor memory; a hardware layout, not part of the method).  Factors are
+ *             per "slot" of W elements along K: W = 16 for E4M3 factors
+ *             (a block-32 factor fills both of its slots), W = 32 for UE8M0.
+ *             u8 [ceil(rows/128)][atoms_k][512] with atoms_k =
+ *             ceil(kpad / (4 W)); byte 16 (r % 32) + 4 ((r / 32) % 4) + s % 4
+ *             of atom (r / 128, s / 4) holds the factor of slot s of row r.
+ *             Bytes of rows >= rows and of slots at or beyond kpad / W are
+ *             not written and feed no stored GEMM output.  ufp4_sf_atoms_layout
+ *             gives atoms_k and the size.  ufp4_rht_quantize writes it when
+ *             non-NULL; when both operands of a dense GEMM on a CTA-pair path
+ *             carry one, the MMA issuer copies each stage's factors into
+ *             tensor memory itself (no factor-building warps).  Must be NULL
+ *             for fp32 scales.  16-byte aligned.
  */
 #ifndef UFP4_H
 #define UFP4_H
@@ -149,6 +165,7 @@ typedef struct {
     ufp4_quant_cfg_t cfg;   /* how it was quantized                          */
     void *corr;             /* device u8 [rows][kpad/2] or NULL, see above   */
     void *elems8;           /* device u8 [rows][kpad] or NULL, see above     */
+    void *sf_atoms;         /* device u8 factor atoms or NULL, see above     */
 } ufp4_qtensor_t;
 
 /* One sub-problem of ufp4_grouped_gemm:
@@ -171,6 +188,14 @@ typedef struct {
 ufp4_status_t ufp4_qtensor_layout(int64_t rows, int64_t k, const ufp4_quant_cfg_t *cfg,
                                   int64_t *kpad, int64_t *scale_ld,
                                   size_t *codes_bytes, size_t *scales_bytes);
+
+/* Size of the optional factor-atom plane (sf_atoms) of a quantized operand:
+ * atoms_k = ceil(kpad / (4 W)) atoms along K (W = 16 for E4M3 x fp32 scales,
+ * 32 for UE8M0), bytes = ceil(rows / 128) * atoms_k * 512.  Either output may
+ * be NULL.  Errors: INVALID_ARG (rows < 0, k < 0, bad cfg), UNSUPPORTED (fp32
+ * scales: no atoms). */
+ufp4_status_t ufp4_sf_atoms_layout(int64_t rows, int64_t k, const ufp4_quant_cfg_t *cfg, int64_t *atoms_k,
+                                   size_t *bytes);
 
 /* Absolute maximum of the rotated operand, max |H_n D x| over all elements
  * (the tensor amax that the two-level scale S is derived from; [PL] §2

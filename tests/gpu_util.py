@@ -83,6 +83,20 @@ def expected_elems8(codes: np.ndarray) -> np.ndarray:
     return lut[c]
 
 
+def atoms_logical(q: ufp4.QTensor, rows=None) -> np.ndarray:
+    """Factor atoms [ceil(rows/128), atoms_k, 512] -> [rows, slots]: byte
+    16 (r % 32) + 4 ((r / 32) % 4) + s % 4 of atom (r / 128, s / 4) is the
+    factor of K slot s of row r (slots of 16 elements for E4M3 factors, 32
+    for UE8M0)."""
+    w = 32 if q.cfg.scale_fmt == ufp4.SCALE_UE8M0 else 16
+    slots = q.kpad // w
+    r = np.arange(q.rows) if rows is None else np.asarray(rows)
+    a = q.sf_atoms.cpu().numpy()
+    s = np.arange(slots)
+    byte = (16 * (r % 32) + 4 * ((r // 32) % 4))[:, None] + (s % 4)[None, :]
+    return a[(r // 128)[:, None], (s // 4)[None, :], byte]
+
+
 def assert_quant_equal(q: ufp4.QTensor, ref: oracle.QTensor, rows=None):
     if q.corr is not None:
         got_c = unpack_plane(q.corr, rows)
@@ -107,6 +121,15 @@ def assert_quant_equal(q: ufp4.QTensor, ref: oracle.QTensor, rows=None):
         r, c = bad[0]
         raise AssertionError(f"{len(bad)} codes differ; first at ({r},{c}): gpu {got[r, c]} "
                              f"oracle {ref.codes[r, c]}")
+    if q.sf_atoms is not None:
+        w = 32 if q.cfg.scale_fmt == ufp4.SCALE_UE8M0 else 16
+        want_a = ref.escales[:, (np.arange(q.kpad // w) * w) // q.cfg.block]
+        got_a = atoms_logical(q, rows)
+        if not np.array_equal(got_a, want_a):
+            bad = np.argwhere(got_a != want_a)
+            r, c = bad[0]
+            raise AssertionError(f"{len(bad)} factor-atom bytes differ; first at (row {r}, slot {c}): gpu "
+                                 f"{got_a[r, c]:#x} expected {want_a[r, c]:#x}")
     sc = logical_scales(q, rows)
     if ref.scales is not None:
         assert np.array_equal(sc.view(np.uint32), ref.scales.view(np.uint32)), "fp32 scales differ"

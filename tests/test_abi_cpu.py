@@ -51,9 +51,9 @@ def test_struct_layouts_match_header(tmp_path):
 int main(void) {
   printf("%zu %zu %zu %zu %zu\\n", sizeof(ufp4_quant_cfg_t), offsetof(ufp4_quant_cfg_t, sr_seed),
          offsetof(ufp4_quant_cfg_t, rht_sign_mask), offsetof(ufp4_quant_cfg_t, scale_fmt), 0);
-  printf("%zu %zu %zu %zu %zu %zu\\n", sizeof(ufp4_qtensor_t), offsetof(ufp4_qtensor_t, rows),
+  printf("%zu %zu %zu %zu %zu %zu %zu\\n", sizeof(ufp4_qtensor_t), offsetof(ufp4_qtensor_t, rows),
          offsetof(ufp4_qtensor_t, scale_ld), offsetof(ufp4_qtensor_t, cfg),
-         offsetof(ufp4_qtensor_t, corr), offsetof(ufp4_qtensor_t, elems8));
+         offsetof(ufp4_qtensor_t, corr), offsetof(ufp4_qtensor_t, elems8), offsetof(ufp4_qtensor_t, sf_atoms));
   printf("%zu %zu\\n", sizeof(ufp4_group_t), offsetof(ufp4_group_t, c_col));
   printf("%zu %zu %zu %zu %zu\\n", sizeof(ufp4_qstats_t), offsetof(ufp4_qstats_t, level_n),
          offsetof(ufp4_qstats_t, code_count), offsetof(ufp4_qstats_t, underflow),
@@ -74,7 +74,7 @@ int main(void) {
                   ctypes.sizeof(Sm)]
     assert c1[:4] == [ctypes.sizeof(Q), Q.sr_seed.offset, Q.rht_sign_mask.offset, Q.scale_fmt.offset]
     assert c2 == [ctypes.sizeof(T), T.rows.offset, T.scale_ld.offset, T.cfg.offset, T.corr.offset,
-                  T.elems8.offset]
+                  T.elems8.offset, T.sf_atoms.offset]
     assert c3 == [ctypes.sizeof(G), G.c_col.offset]
 
 
@@ -96,6 +96,26 @@ def test_layout(L, k, block, fmt, kpad, codes, scales):
     kp, sld, cb, sb = ufp4.layout(256, k, cfg)
     assert (kp, sld, cb, sb) == (kpad, 256, codes, scales)
     assert ufp4.layout(300, 64, cfg)[1] == 320
+
+
+@pytest.mark.parametrize("rows,k,block,fmt,atoms_k,nbytes", [
+    (256, 512, 16, ufp4.SCALE_E4M3_X_FP32, 8, 2 * 8 * 512),
+    (300, 200, 32, ufp4.SCALE_E4M3_X_FP32, 4, 3 * 4 * 512),     # kpad 256: 16 slots of 16
+    (129, 1000, 32, ufp4.SCALE_UE8M0, 8, 2 * 8 * 512),          # kpad 1024: 32 slots of 32
+    (1, 136, 32, ufp4.SCALE_UE8M0, 2, 1 * 2 * 512),             # kpad 192: 6 slots, 2 atoms
+    (0, 64, 16, ufp4.SCALE_E4M3_X_FP32, 1, 0),
+])
+def test_sf_atoms_layout(L, rows, k, block, fmt, atoms_k, nbytes):
+    """Factor-atom plane size: ceil(rows/128) row groups x ceil(kpad / 4W)
+    atoms of 512 bytes (W = 16 for E4M3 factors, 32 for UE8M0); none for
+    fp32 scales."""
+    cfg = ufp4.QuantConfig(block=block, scale_fmt=fmt)
+    assert ufp4.sf_atoms_layout(rows, k, cfg) == (atoms_k, nbytes)
+    c = ufp4.QuantConfig(scale_fmt=ufp4.SCALE_FP32).c()
+    assert L.ufp4_sf_atoms_layout(64, 64, ctypes.byref(c), None, None) == ufp4.ERR_UNSUPPORTED
+    c = cfg.c()
+    assert L.ufp4_sf_atoms_layout(-1, 64, ctypes.byref(c), None, None) == ufp4.ERR_INVALID_ARG
+    assert L.ufp4_sf_atoms_layout(64, 64, None, None, None) == ufp4.ERR_INVALID_ARG
 
 
 def _q(rows=128, k=256, **kw):
@@ -157,6 +177,12 @@ def test_quantize_validation_rejects_before_launch(L):
     assert Q(x, 64, 128, 128, 1, None, ctypes.byref(out), None) == ufp4.ERR_INVALID_ARG   # shape
     two = _q(rows=64, k=128, scale_fmt=1)
     assert Q(x, 64, 128, 128, 0, None, ctypes.byref(two), None) == ufp4.ERR_INVALID_ARG   # no amax
+    am = ctypes.c_void_p(8192)
+    fp = _q(rows=64, k=128)
+    fp.sf_atoms = 64 * 1024
+    assert Q(x, 64, 128, 128, 0, None, ctypes.byref(fp), None) == ufp4.ERR_INVALID_ARG    # atoms, fp32 scales
+    two.sf_atoms = 64 * 1024 + 8
+    assert Q(x, 64, 128, 128, 0, am, ctypes.byref(two), None) == ufp4.ERR_ALIGNMENT       # atoms alignment
     assert L.ufp4_rht_amax(x, 64, 128, 128, 0, 8, 0, ctypes.c_void_p(4096), None) == ufp4.ERR_UNSUPPORTED
     assert L.ufp4_rht_amax(x, 64, 128, 128, 0, 16, 0, None, None) == ufp4.ERR_INVALID_ARG
     R = L.ufp4_rht_bf16
@@ -288,6 +314,10 @@ def test_binding_allocates_what_the_layout_call_sizes(grid, fmt, block):
     assert q.scales.shape == (kpad // block, sld) and sld % 64 == 0 and sld >= 300
     assert (q.corr is not None) == (grid == ufp4.GRID_E1M2 and fmt == ufp4.SCALE_E4M3_X_FP32)
     assert (q.tensor_scale is not None) == (fmt == ufp4.SCALE_E4M3_X_FP32)
+    if fmt == ufp4.SCALE_FP32:
+        assert q.sf_atoms is None
+    else:
+        assert q.sf_atoms.numel() == ufp4.sf_atoms_layout(300, 200, cfg)[1]
     c = q.c()
     assert c.rows == 300 and c.k == 200 and c.kpad == kpad and c.scale_ld == sld
     assert c.cfg.scale_fmt == fmt and c.cfg.block == block and c.cfg.grid == grid

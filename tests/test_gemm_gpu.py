@@ -190,6 +190,32 @@ def test_two_level_kernel_families(path, corr, grid):
         ufp4.set_two_level_gemm_path(old)
 
 
+@pytest.mark.parametrize("grid,fmt,block", [
+    (ufp4.GRID_E1M2, ufp4.SCALE_E4M3_X_FP32, 16), (ufp4.GRID_E1M2, ufp4.SCALE_E4M3_X_FP32, 32),
+    (ufp4.GRID_E2M1, ufp4.SCALE_E4M3_X_FP32, 16), (ufp4.GRID_E2M1_MAX2, ufp4.SCALE_E4M3_X_FP32, 32),
+    (ufp4.GRID_E1M2, ufp4.SCALE_UE8M0, 32)])
+def test_factor_atoms_path_equals_factor_warps(grid, fmt, block):
+    """Dense CTA-pair GEMMs whose operands carry factor atoms (the MMA issuer
+    copies them into tensor memory) give bit-for-bit the output of the same
+    kernel building the factors from the block-major scales, and the
+    oracle's result; partial 256-wide tiles, one-row operands, K tails of 64
+    and of 128 + 64."""
+    import dataclasses
+    cfg = _cfg(grid=grid, fmt=fmt, block=block)
+    for (M, N, K) in [(520, 700, 448), (130, 230, 200), (1, 1, 8), (300, 513, 1000)]:
+        X = wl.normal_with_outlier_channels(M, K, 1.0, 2, 20.0)
+        W = wl.normal(N, K, 0.02, 2)
+        qx, rx = _quant_both(X, C, cfg)
+        qw, rw = _quant_both(W, C, cfg)
+        assert qx.sf_atoms is not None and qw.sf_atoms is not None
+        _check_full(qx, rx, qw, rw, ufp4.gemm_fprop)
+        with_atoms = ufp4.gemm_fprop(qx, qw)
+        plain = ufp4.gemm_fprop(dataclasses.replace(qx, sf_atoms=None), dataclasses.replace(qw, sf_atoms=None))
+        torch.cuda.synchronize()
+        assert ufp4.check_device_status() == ufp4.OK
+        assert torch.equal(with_atoms, plain), (M, N, K)
+
+
 @pytest.mark.parametrize("fmt", [ufp4.SCALE_FP32, ufp4.SCALE_E4M3_X_FP32])
 def test_e2m1_reference_recipe_layer(fmt):
     """The comparison recipe of the pages (E2M1 grid, RHT on the WGRAD
