@@ -19,6 +19,7 @@ namespace ufp4 {
 
 cudaError_t read_and_clear_error_word(uint32_t *out);            // gemm.cu
 cudaError_t quantize_read_and_clear_error_word(uint32_t *out);   // quantize.cu
+cudaError_t quantize_set_producer_wait_limit(uint64_t limit_ns);  // quantize.cu
 
 namespace {
 
@@ -137,8 +138,8 @@ std::atomic<int32_t> g_two_level_path{UFP4_GEMM_PATH_AUTO};
 ufp4_status_t encode_operand_maps(const ufp4_qtensor_t *q, int code_rows, int scale_rows, int mode,
                                   CUtensorMap *codes, CUtensorMap *scales) {
     const int64_t rows_t = q->rows > 0 ? q->rows : 1;
-    // The native kernels (modes 3, 4) stage 128 K elements per step (64-byte
-    // code rows, 64-byte swizzle), the fp16-operand kernels 64 (32-byte rows,
+    // The FP4 kernels (modes >= 3) stage 128 K elements per step (64-byte
+    // code rows, 64-byte swizzle), the fp32-scale kernel 64 (32-byte rows,
     // 32-byte swizzle).
     const bool native = mode >= 3;
     const int k_stage = native ? 128 : 64;
@@ -181,11 +182,10 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
     if (groups_dev != nullptr && (reinterpret_cast<uintptr_t>(groups_dev) & 7u))
         return UFP4_ERR_ALIGNMENT;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // fp32 or UE8M0 block scales: per-block partials (mode 0).  Two-level scales: the
-    // native block-scaled FP4 kernel with one CTA per 128 x 192 tile (mode 3),
-    // or what the caller picked: the same on CTA pairs with 256 x 192 tiles
-    // (mode 4), the fp16-operand kernels (mode 1: one CTA per 128 x 256 tile,
-    // mode 2: CTA pairs).
+    // fp32 or UE8M0 block scales: per-block partials (mode 0).  Two-level
+    // scales: the block-scaled FP4 kernel on CTA pairs with 256 x 256 tiles
+    // (mode 5) or with one CTA per 128 x 192 tile (mode 3).  MX operands with
+    // E4M3 element planes: the block-scaled FP8 kernel on CTA pairs (mode 6).
     int mode = 0;
     if (a->cfg.scale_fmt == UFP4_SCALE_E4M3_X_FP32) {
         // The CTA-pair kernel (mode 5) takes E1M2 operands whose correction
@@ -196,14 +196,7 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
                    reinterpret_cast<uintptr_t>(q->corr) == reinterpret_cast<uintptr_t>(q->codes) + plane;
         };
         const bool pair_ok = a->cfg.grid != UFP4_GRID_E1M2 || (adjacent_planes(a) && adjacent_planes(b));
-        switch (g_two_level_path.load()) {
-            case UFP4_GEMM_PATH_FP16: mode = 1; break;
-            case UFP4_GEMM_PATH_FP16_PAIR: mode = 2; break;
-            case UFP4_GEMM_PATH_NATIVE_FP4: mode = 3; break;
-            case UFP4_GEMM_PATH_NATIVE_FP4_PAIR: mode = 4; break;
-            case UFP4_GEMM_PATH_NATIVE_FP4_PAIR256: mode = pair_ok ? 5 : 3; break;
-            default: mode = pair_ok ? 5 : 3; break;
-        }
+        mode = (g_two_level_path.load() == UFP4_GEMM_PATH_NATIVE_FP4 || !pair_ok) ? 3 : 5;
     }
     // MX operands that carry E4M3 element planes: the block-scaled FP8 MMA
     // on CTA pairs (mode 6); otherwise the fp32-block-scale kernel.
@@ -225,14 +218,12 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
     GemmArgs args;
     memset(&args, 0, sizeof(args));
     args.scale_ue8m0 = a->cfg.scale_fmt == UFP4_SCALE_UE8M0 ? 1 : 0;
-    // B code rows staged per CTA: fp32-scale kernel 128, fp16 kernels 256
-    // (one CTA) or 128 (pairs), native kernels 192 or 96, with the scales of
-    // all 192 B rows of a tile in each CTA.
+    // B code rows staged per CTA: fp32-scale kernel 128, one-CTA FP4 kernel
+    // 192, CTA-pair kernels 128 (with the scales of all 256 B rows of a tile
+    // in each CTA).
     int bn = 128, bscale = 128;
     switch (mode) {
-        case 1: bn = bscale = 256; break;
         case 3: bn = bscale = kNativeTileN; break;
-        case 4: bn = kNativeTileN / 2; bscale = kNativeTileN; break;
         case 5:
         case 6: bn = 128; bscale = 256; break;
         default: bn = bscale = 128; break;
@@ -298,20 +289,22 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
         args.corr_in = 1;
     }
     // Dense problems on the CTA-pair kernels whose operands both carry factor
-    // atoms: each stage's atoms come with its code tiles (one u64 box of
-    // 128 K elements per 128-row group: two atoms of E4M3 factors, one of
-    // UE8M0) and the MMA issuer copies them into tensor memory.
+    // atoms: each stage's atoms come with its code tiles (one u64 box of 128 K
+    // elements per 128-row group: two atoms of E4M3 factors, one of UE8M0)
+    // and the MMA issuer copies them into tensor memory.  Grouped problems
+    // keep the factor-building warps (measured faster there: short K per
+    // tile, ragged groups).
     if ((mode == 5 || mode == 6) && groups_dev == nullptr && a->sf_atoms != nullptr && b->sf_atoms != nullptr &&
         a->rows > 0 && b->rows > 0) {
-        const int64_t ak = atoms_k_of(a->kpad, a->cfg);
+        const int64_t ak = atoms_k_of(a->kpad, a->cfg), bk = atoms_k_of(b->kpad, b->cfg);
         const uint32_t box_k = static_cast<uint32_t>(64 * (128 / (4 * atom_slot(a->cfg))));
         CUresult r = encode_tensor_map_2d(&args.tm_a_atoms, CU_TENSOR_MAP_DATA_TYPE_UINT64, a->sf_atoms,
                                           static_cast<uint64_t>(64 * ak), static_cast<uint64_t>((a->rows + 127) / 128),
                                           static_cast<uint64_t>(ak) * 512, box_k, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
         r = encode_tensor_map_2d(&args.tm_b_atoms, CU_TENSOR_MAP_DATA_TYPE_UINT64, b->sf_atoms,
-                                 static_cast<uint64_t>(64 * ak), static_cast<uint64_t>((b->rows + 127) / 128),
-                                 static_cast<uint64_t>(ak) * 512, box_k, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
+                                 static_cast<uint64_t>(64 * bk), static_cast<uint64_t>((b->rows + 127) / 128),
+                                 static_cast<uint64_t>(bk) * 512, box_k, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
         args.atoms = 1;
     }
@@ -677,12 +670,17 @@ ufp4_status_t ufp4_grouped_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b
 }
 
 ufp4_status_t ufp4_set_two_level_gemm_path(int32_t path) {
-    if (path < UFP4_GEMM_PATH_AUTO || path > UFP4_GEMM_PATH_NATIVE_FP4_PAIR256) return UFP4_ERR_INVALID_ARG;
+    if (path != UFP4_GEMM_PATH_AUTO && path != UFP4_GEMM_PATH_NATIVE_FP4 && path != UFP4_GEMM_PATH_NATIVE_FP4_PAIR256)
+        return UFP4_ERR_INVALID_ARG;
     g_two_level_path.store(path);
     return UFP4_OK;
 }
 
 int32_t ufp4_get_two_level_gemm_path(void) { return g_two_level_path.load(); }
+
+ufp4_status_t ufp4_test_set_quantize_wait_limit(uint64_t limit_ns) {
+    return quantize_set_producer_wait_limit(limit_ns) == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
+}
 
 ufp4_status_t ufp4_check_device_status(void) {
     uint32_t w = 0;

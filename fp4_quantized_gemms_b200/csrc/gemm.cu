@@ -4,28 +4,28 @@
 //
 // Both operands arrive K-major as packed sign-magnitude nibbles plus block
 // scales, exactly as ufp4_rht_quantize writes them.  FPROP, DGRAD and WGRAD
-// are this one kernel: the quantizer already laid every operand out along its
+// are the same kernels: the quantizer already laid every operand out along its
 // GEMM's reduction dimension (paperlayer.ai summary §2, "for the three
 // training GEMMs, RHT acts along the shared reduction dimension").
 //
-// No tcgen05 MMA kind consumes a uniform 4-bit grid, and none applies an fp32
-// scale per 16 elements.  Both 4-bit grids are exact in fp16, so the kernel
-// expands codes to fp16 in shared memory and runs kind::f16:
-//   mode 1 (E4M3 x fp32 two-level scales): e_b * lvl has at most 7
-//     significant bits and lies in [2^-11, 2688], so it is exact in fp16; the
-//     scale is folded into the operand and one fp32 accumulation runs over
-//     all of K.  The tensor scales S_a * S_b / n are applied in the epilogue.
-//   mode 0 (fp32 block scales): each 16-block is one K=16 MMA into its own
-//     TMEM buffer (an exact partial: sums of at most 32 products on a 1/16
-//     lattice); epilogue warps add s_a * s_b * partial into fp32 registers.
-//
-// Pipeline (one CTA per SM, persistent over output tiles):
-//   warp 0      TMA producer: packed codes (+ scales) of each 64-wide K stage
-//   warp 1      TMEM owner and single-thread UMMA issuer
-//   transform   codes -> fp16 in the 128-byte-swizzled UMMA layout
-//   epilogue    TMEM -> registers -> (scale) -> global fp32
-// Every wait is bounded (see ufp4_device.cuh); a stuck pipeline sets the
-// device error word and the CTA unwinds, drains its copies, frees TMEM.
+// Kernel families (all persistent over output tiles, warp-specialised, every
+// wait bounded: a stuck pipeline sets the device error word and the CTA
+// unwinds, drains its copies and frees TMEM):
+//   gemm_pair_kernel<0/1>  two-level (E4M3 x fp32) scales, the default: CTA
+//       pairs (cta_group::2) with 256 x 256 tiles on the block-scaled FP4 MMA
+//       (kind::mxf4nvf4, UE4M3 factors per 16 elements).  E1M2 codes split
+//       exactly into two E2M1 planes, four MMAs per K step.  The factors come
+//       as the quantizer's factor atoms and the MMA issuer copies them into
+//       TMEM (tcgen05.cp), or, for grouped problems and operands without
+//       atoms, factor warps build them from the block-major scales.
+//   gemm_pair_kernel<3>    MX operands (UE8M0, block 32): the E4M3 element
+//       planes on the block-scaled FP8 MMA (kind::mxf8f6f4), factors in the MMA.
+//   gemm_fp4_kernel        two-level scales with one CTA per 128 x 192 tile
+//       (E1M2 operands whose correction planes are not stored next to their
+//       codes, or when the caller picks it).
+//   gemm_f32s_kernel       fp32 or UE8M0 block scales without element planes:
+//       codes expanded to fp16, one K = 16 MMA per block into its own TMEM
+//       partial, s_a * s_b * partial accumulated in fp32 registers.
 
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -46,89 +46,48 @@ constexpr int BK = 64;             // K elements per pipeline stage
 constexpr int kCodeRow = BK / 2;   // packed bytes per row per stage
 constexpr int kOpRow = BK * 2;     // fp16 bytes per row per stage (= 128)
 
-template <int MODE>
-struct Cfg;
-
-// mode 1: two-level scales folded into fp16 operands, one CTA per 128 x 256 tile
-template <>
-struct Cfg<1> {
-    static constexpr int BN = 256;  // B rows staged per CTA
-    static constexpr int TM = 128;  // output tile rows
-    static constexpr int TN = 256;  // output tile columns (= accumulator columns)
-    static constexpr int CG = 1;    // CTAs per MMA
-    static constexpr int NT = 12;   // transform warps (one operand row per thread)
-    static constexpr int NE = 4;    // epilogue warps
-    static constexpr int NC = 4;    // code ring slots
-    static constexpr int NO = 3;    // fp16 operand ring slots
-    static constexpr int NS = 0;    // separate scale ring slots
-    static constexpr int NP = 2;    // TMEM accumulators
-    static constexpr int kScaleElt = 1;
-};
-
-// mode 2: mode 1 on a CTA pair (cta_group::2): a 256 x 256 tile, each CTA
-// stages 128 rows of A and 128 rows of B and holds 128 accumulator rows.
-template <>
-struct Cfg<2> {
-    static constexpr int BN = 128;
-    static constexpr int TM = 256;
-    static constexpr int TN = 256;
-    static constexpr int CG = 2;
-    static constexpr int NT = 8;
-    static constexpr int NE = 4;
-    static constexpr int NC = 4;
-    static constexpr int NO = 4;
-    static constexpr int NS = 0;
-    static constexpr int NP = 2;
-    static constexpr int kScaleElt = 1;
-};
-
-// mode 0: fp32 block scales, per-block partial products in TMEM
-template <>
-struct Cfg<0> {
-    static constexpr int BN = 128;
+// fp32 (or UE8M0) block scales: no MMA kind applies an fp32 factor per block,
+// so every 16-element K block is one K = 16 fp16 MMA into its own TMEM partial
+// buffer (an exact partial: a sum of at most 16 products on a 1/16 lattice,
+// E1M2 as k, E2M1 as its level), and the epilogue warps accumulate
+// s_a * s_b * partial in fp32 registers.  The loop is bound by the round trip
+// of a partial buffer (MMA -> commit -> epilogue load -> release -> MMA) over
+// the four buffers TMEM holds, not by either pipe's throughput.
+// One CTA per SM per 128 x 128 output tile, persistent over tiles.
+struct F32sCfg {
+    static constexpr int BN = 128;    // B rows staged per stage (= tile columns)
     static constexpr int TM = 128;
     static constexpr int TN = 128;
-    static constexpr int CG = 1;
-    static constexpr int NT = 2;
-    static constexpr int NE = 8;
-    static constexpr int NC = 4;
-    static constexpr int NO = 3;
-    static constexpr int NS = 4;
-    static constexpr int NP = 4;    // TMEM partial buffers
-    static constexpr int kScaleElt = 4;
-};
-
-template <int MODE>
-struct Layout {
-    using C = Cfg<MODE>;
-    static constexpr int BN = C::BN;
+    static constexpr int NT = 2;      // transform warps: codes -> fp16
+    static constexpr int NE = 8;      // epilogue warps: 2 per TMEM lane quarter, 64 columns each
+    static constexpr int NC = 4;      // code ring slots
+    static constexpr int NO = 3;      // fp16 operand ring slots
+    static constexpr int NS = 4;      // scale ring slots
+    static constexpr int NP = 4;      // TMEM partial buffers (BN columns each)
     static constexpr int kOpA = BM * kOpRow;
     static constexpr int kOpB = BN * kOpRow;
     static constexpr int kCodeA = BM * kCodeRow;
     static constexpr int kCodeB = BN * kCodeRow;
-    // scales per stage for the smallest block (16): BK/16 = 4 blocks
-    static constexpr int kScA = BM * (BK / 16) * C::kScaleElt;
-    static constexpr int kScB = BN * (BK / 16) * C::kScaleElt;
+    // fp32 scales of the smallest block (16): BK / 16 blocks per stage
+    static constexpr int kScA = BM * (BK / 16) * 4;
+    static constexpr int kScB = BN * (BK / 16) * 4;
     // code slots start on 1024-byte boundaries (the 32-byte TMA swizzle)
-    static constexpr int kCodeSlot =
-        ((MODE != 0 ? kCodeA + kCodeB + kScA + kScB : kCodeA + kCodeB) + 1023) / 1024 * 1024;
-    static constexpr int kScSlot = MODE == 0 ? kScA + kScB : 0;
-
+    static constexpr int kCodeSlot = (kCodeA + kCodeB + 1023) / 1024 * 1024;
+    static constexpr int kScSlot = kScA + kScB;
     static constexpr int off_op = 0;
-    static constexpr int off_code = off_op + C::NO * (kOpA + kOpB);
-    static constexpr int off_sc = off_code + C::NC * kCodeSlot;
-    static constexpr int off_bar = (off_sc + C::NS * kScSlot + 127) / 128 * 128;
+    static constexpr int off_code = off_op + NO * (kOpA + kOpB);
+    static constexpr int off_sc = off_code + NC * kCodeSlot;
+    static constexpr int off_bar = (off_sc + NS * kScSlot + 127) / 128 * 128;
     // barriers: code_full, code_empty, op_full, op_empty, sc_full, sc_empty,
     //           p_full, p_empty, drain
-    static constexpr int kNumBars = 2 * C::NC + 2 * C::NO + 2 * C::NS + 2 * C::NP + 1;
+    static constexpr int kNumBars = 2 * NC + 2 * NO + 2 * NS + 2 * NP + 1;
     static constexpr int off_misc = off_bar + kNumBars * 8;
-    static constexpr int kBytes = off_misc + 64;
-    static constexpr int kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
-    static constexpr int kThreads = 32 * (2 + C::NT + C::NE);
+    static constexpr int kAlloc = off_misc + 64 + 1024;   // slack for 1024-byte alignment
+    static constexpr int kThreads = 32 * (2 + NT + NE);
     static constexpr int kTmemCols = 512;
-    static constexpr int kAccCols = MODE == 0 ? BN : C::TN;
-    static_assert(C::NP * kAccCols <= kTmemCols, "TMEM budget");
-    static_assert(BM + BN <= C::NT * 32 * 4, "transform rows");
+    static_assert(NP * BN <= kTmemCols, "TMEM budget");
+    static_assert(kThreads % 128 == 0, "whole warp quads");
+    static_assert(NE == 8, "epilogue: 2 warps per lane quarter, 64 columns each");
     static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
@@ -205,10 +164,7 @@ __device__ Tile get_tile(const GemmArgs &a, int64_t t) {
 // leaves every dot product (and every 16-block) unchanged.
 //
 // E1M2 carries the magnitude index k (the level is k/4; the 1/4 moves to the
-// epilogue); E2M1 carries the level itself.  With a block scale e (an E4M3
-// value, fp16-exact) the pair is multiplied in: e*k <= 7*448 and e*lvl <= 6*448
-// have at most 7 significant bits and stay in fp16's normal range, so every
-// operand value is exact.
+// epilogue); E2M1 carries the level itself.  Both are exact in fp16.
 
 // Sign bits of codes i and i+4 (nibble bit 3) moved to fp16 bits 15 and 31.
 template <int I>
@@ -227,7 +183,7 @@ __device__ __forceinline__ uint32_t eight_plus_k(uint32_t w) {
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
 
-// Unscaled expansion (fp32 block-scale mode): k (E1M2) or lvl (E2M1).
+// Expansion of 8 codes: k (E1M2) or lvl (E2M1).
 template <int GRID>
 __device__ __forceinline__ void expand_unscaled(uint32_t w, uint32_t (&o)[4]) {
     if (GRID == 0) {
@@ -248,31 +204,6 @@ __device__ __forceinline__ void expand_unscaled(uint32_t w, uint32_t (&o)[4]) {
     }
 }
 
-// Scaled expansion (two-level mode): e*k (E1M2) via one fma per pair,
-// (8 + k) * e - 8 * e = k * e (exact), or e*lvl (E2M1).
-template <int GRID>
-__device__ __forceinline__ void expand_scaled(uint32_t w, __half2 e2, __half2 m8e2, uint32_t (&o)[4]) {
-    if (GRID == 0) {
-        o[0] = h2_bits(__hfma2(bits_h2(eight_plus_k<0>(w)), e2, m8e2)) ^ sign_pair<0>(w);
-        o[1] = h2_bits(__hfma2(bits_h2(eight_plus_k<1>(w)), e2, m8e2)) ^ sign_pair<1>(w);
-        o[2] = h2_bits(__hfma2(bits_h2(eight_plus_k<2>(w)), e2, m8e2)) ^ sign_pair<2>(w);
-        o[3] = h2_bits(__hfma2(bits_h2(eight_plus_k<3>(w)), e2, m8e2)) ^ sign_pair<3>(w);
-    } else {
-        uint32_t u[4];
-        expand_unscaled<1>(w, u);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) o[q] = h2_bits(__hmul2(bits_h2(u[q]), e2));
-    }
-}
-
-// E4M3 byte -> fp16 pair (e, e), exact (hardware conversion).
-__device__ __forceinline__ __half2 e4m3_pair(uint32_t byte) {
-    const uint16_t two = static_cast<uint16_t>(byte | (byte << 8));
-    uint32_t out;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(out) : "h"(two));
-    return bits_h2(out);
-}
-
 // ---------------------------------------------------------------------------
 // 2^(E - 127) of a UE8M0 byte E <= 254: the byte is the fp32 exponent field
 // (E = 0 is the subnormal 2^-127).
@@ -280,22 +211,16 @@ __device__ __forceinline__ float ue8m0_to_f32(uint32_t e) {
     return __uint_as_float(e ? (e << 23) : 0x00400000u);
 }
 
-template <int MODE, int GRID>
-__global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
-    gemm_tn_kernel(const __grid_constant__ GemmArgs args) {
-    using C = Cfg<MODE>;
-    using Lay = Layout<MODE>;
-    constexpr int BN = C::BN;
-    constexpr int TM = C::TM;
-    constexpr int TN = C::TN;
-    constexpr bool kPair = C::CG == 2;
-    constexpr bool kFolded = MODE != 0;   // two-level scales folded into the operands
-    constexpr int NSr = C::NS > 0 ? C::NS : 1;   // scale-ring modulus (mode 0 only)
+template <int GRID>
+__global__ void __launch_bounds__(F32sCfg::kThreads, 1)
+    gemm_f32s_kernel(const __grid_constant__ GemmArgs args) {
+    using C = F32sCfg;
+    constexpr int BN = C::BN, TM = C::TM, TN = C::TN;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::off_bar);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::off_bar);
     uint64_t *code_full = bars;
     uint64_t *code_empty = code_full + C::NC;
     uint64_t *op_full = code_empty + C::NC;
@@ -305,27 +230,21 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
     uint64_t *p_full = sc_empty + C::NS;
     uint64_t *p_empty = p_full + C::NP;
     uint64_t *drain = p_empty + C::NP;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::off_misc);
-    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + Lay::off_misc + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::off_misc);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::off_misc + 4);
 
-    auto op_a = [&](int s) { return smem + Lay::off_op + s * (Lay::kOpA + Lay::kOpB); };
-    auto op_b = [&](int s) { return op_a(s) + Lay::kOpA; };
-    auto code_a = [&](int s) { return smem + Lay::off_code + s * Lay::kCodeSlot; };
-    auto code_b = [&](int s) { return code_a(s) + Lay::kCodeA; };
-    // folded modes: scales ride in the code slot; mode 0: separate scale ring
-    auto sc_a = [&](int s) {
-        return kFolded ? code_b(s) + Lay::kCodeB : smem + Lay::off_sc + s * Lay::kScSlot;
-    };
-    auto sc_b = [&](int s) { return sc_a(s) + Lay::kScA; };
+    auto op_a = [&](int s) { return smem + C::off_op + s * (C::kOpA + C::kOpB); };
+    auto op_b = [&](int s) { return op_a(s) + C::kOpA; };
+    auto code_a = [&](int s) { return smem + C::off_code + s * C::kCodeSlot; };
+    auto code_b = [&](int s) { return code_a(s) + C::kCodeA; };
+    auto sc_a = [&](int s) { return smem + C::off_sc + s * C::kScSlot; };
+    auto sc_b = [&](int s) { return sc_a(s) + C::kScA; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int nblk_stage = BK / args.block;
-    // CTA pair: rank 0 issues the MMAs; rank r stages rows [128 r, 128 r + 128)
-    // of both the A tile and the B tile and holds accumulator rows 128 r...
-    const uint32_t rank = kPair ? cluster_ctarank() : 0u;
-    const int64_t unit = kPair ? (blockIdx.x >> 1) : blockIdx.x;
-    const int64_t nunits = kPair ? (gridDim.x >> 1) : gridDim.x;
+    const int64_t unit = blockIdx.x;
+    const int64_t nunits = gridDim.x;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::NC; ++i) {
@@ -333,7 +252,7 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
             mbar_init(&code_empty[i], C::NT);
         }
         for (int i = 0; i < C::NO; ++i) {
-            mbar_init(&op_full[i], C::NT * C::CG);
+            mbar_init(&op_full[i], C::NT);
             mbar_init(&op_empty[i], 1);
         }
         for (int i = 0; i < C::NS; ++i) {
@@ -342,7 +261,7 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
         }
         for (int i = 0; i < C::NP; ++i) {
             mbar_init(&p_full[i], 1);
-            mbar_init(&p_empty[i], C::NE * C::CG);
+            mbar_init(&p_empty[i], C::NE);
         }
         mbar_init(drain, 1);
         *abort_flag = 0u;
@@ -354,13 +273,9 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
         tma_prefetch_desc(&args.tm_a_scales);
         tma_prefetch_desc(&args.tm_b_scales);
     }
-    if (warp == 1) {
-        if constexpr (kPair) tmem_alloc_pair(tmem_slot, Lay::kTmemCols);
-        else tmem_alloc(tmem_slot, Lay::kTmemCols);
-    }
+    if (warp == 1) tmem_alloc(tmem_slot, C::kTmemCols);
     tc_fence_before();
-    if constexpr (kPair) cluster_sync();
-    else __syncthreads();
+    __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int64_t ntiles = total_tiles<TM, TN>(args);
@@ -372,8 +287,8 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
             bool ok = true;
             for (int64_t t = unit; t < ntiles && ok; t += nunits) {
                 const Tile tl = get_tile<TM, TN>(args, t);
-                const int32_t arow = static_cast<int32_t>(tl.g.a_row + tl.m0 + 128 * rank);
-                const int32_t brow = static_cast<int32_t>(tl.g.b_row + tl.n0 + BN * rank);
+                const int32_t arow = static_cast<int32_t>(tl.g.a_row + tl.m0);
+                const int32_t brow = static_cast<int32_t>(tl.g.b_row + tl.n0);
                 for (int ks = 0; ks < tl.nks; ++ks, ++it) {
                     const int s = it % C::NC;
                     const uint32_t use = it / C::NC;
@@ -383,28 +298,20 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
                     }
                     const int32_t acol = static_cast<int32_t>(tl.g.a_col + ks * BK);
                     const int32_t bcol = static_cast<int32_t>(tl.g.b_col + ks * BK);
-                    uint32_t bytes = Lay::kCodeA + Lay::kCodeB;
-                    if (kFolded) bytes += (BM + BN) * nblk_stage;
-                    mbar_arrive_expect_tx(&code_full[s], bytes);
+                    mbar_arrive_expect_tx(&code_full[s], C::kCodeA + C::kCodeB);
                     tma_load_2d(code_a(s), &args.tm_a_codes, &code_full[s], acol / 2, arow);
                     tma_load_2d(code_b(s), &args.tm_b_codes, &code_full[s], bcol / 2, brow);
-                    if (kFolded) {
-                        tma_load_2d(sc_a(s), &args.tm_a_scales, &code_full[s], arow, acol / args.block);
-                        tma_load_2d(sc_b(s), &args.tm_b_scales, &code_full[s], brow, bcol / args.block);
-                    } else {
-                        const int ss = sit % NSr;
-                        const uint32_t suse = sit / NSr;
-                        if (!mbar_wait(&sc_empty[ss], (suse & 1) ^ 1, kErrTimeoutProducer, abort_flag)) {
-                            ok = false;
-                            ++it;   // the code copies of this stage were issued
-                            break;
-                        }
-                        mbar_arrive_expect_tx(&sc_full[ss],
-                                              (BM + BN) * nblk_stage * (args.scale_ue8m0 ? 1 : 4));
-                        tma_load_2d(sc_a(ss), &args.tm_a_scales, &sc_full[ss], arow, acol / args.block);
-                        tma_load_2d(sc_b(ss), &args.tm_b_scales, &sc_full[ss], brow, bcol / args.block);
-                        ++sit;
+                    const int ss = sit % C::NS;
+                    const uint32_t suse = sit / C::NS;
+                    if (!mbar_wait(&sc_empty[ss], (suse & 1) ^ 1, kErrTimeoutProducer, abort_flag)) {
+                        ok = false;
+                        ++it;   // the code copies of this stage were issued
+                        break;
                     }
+                    mbar_arrive_expect_tx(&sc_full[ss], (BM + BN) * nblk_stage * (args.scale_ue8m0 ? 1 : 4));
+                    tma_load_2d(sc_a(ss), &args.tm_a_scales, &sc_full[ss], arow, acol / args.block);
+                    tma_load_2d(sc_b(ss), &args.tm_b_scales, &sc_full[ss], brow, bcol / args.block);
+                    ++sit;
                 }
             }
             // Drain: wait (time-bounded, regardless of abort) until the last
@@ -419,94 +326,61 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
             }
             for (int s = 0; s < C::NS; ++s) {
                 if (sit > static_cast<uint32_t>(s)) {
-                    const uint32_t last = (sit - 1 - s) / NSr * NSr + s;
+                    const uint32_t last = (sit - 1 - s) / C::NS * C::NS + s;
                     uint32_t dummy = 0;
-                    mbar_wait(&sc_full[s], (last / NSr) & 1, kErrTimeoutDrain,
+                    mbar_wait(&sc_full[s], (last / C::NS) & 1, kErrTimeoutDrain,
                               reinterpret_cast<volatile uint32_t *>(&dummy));
                 }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ UMMA issuer
-        if (lane == 0 && rank == 0) {
-            constexpr uint32_t idesc = umma_idesc_f16_f32(kPair ? 256 : BM, Lay::kAccCols);
-            uint32_t it = 0, pq = 0, tcount = 0;
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_f16_f32(BM, BN);
+            uint32_t it = 0, pq = 0;
             bool ok = true;
-            auto wait = [&](uint64_t *bar, uint32_t parity) {
-                return kPair ? mbar_wait_cluster(bar, parity, kErrTimeoutMma, abort_flag)
-                             : mbar_wait(bar, parity, kErrTimeoutMma, abort_flag);
-            };
-            for (int64_t t = unit; t < ntiles && ok; t += nunits, ++tcount) {
+            for (int64_t t = unit; t < ntiles && ok; t += nunits) {
                 const Tile tl = get_tile<TM, TN>(args, t);
-                uint32_t acc_col = 0;
-                if (kFolded) {
-                    const int b = tcount & 1;
-                    if (!wait(&p_empty[b], ((tcount >> 1) & 1) ^ 1)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    acc_col = b * Lay::kAccCols;
-                }
                 for (int ks = 0; ks < tl.nks && ok; ++ks, ++it) {
                     const int s = it % C::NO;
-                    if (!wait(&op_full[s], (it / C::NO) & 1)) {
+                    if (!mbar_wait(&op_full[s], (it / C::NO) & 1, kErrTimeoutMma, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t a0 = smem_addr(op_a(s));
                     const uint32_t b0 = smem_addr(op_b(s));
-                    if (kFolded) {
-#pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk) {
-                            const uint64_t ad = umma_desc_sw128(a0 + kk * 32);
-                            const uint64_t bd = umma_desc_sw128(b0 + kk * 32);
-                            const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
-                            if constexpr (kPair) umma_f16_pair(tmem_base + acc_col, ad, bd, idesc, acc);
-                            else umma_f16(tmem_base + acc_col, ad, bd, idesc, acc);
+                    const int slices = args.block / 16;
+                    for (int bi = 0; bi < nblk_stage; ++bi, ++pq) {
+                        const int p = pq % C::NP;
+                        if (!mbar_wait(&p_empty[p], ((pq / C::NP) & 1) ^ 1, kErrTimeoutMma, abort_flag)) {
+                            ok = false;
+                            break;
                         }
-                        if constexpr (kPair) umma_commit_pair_mc(&op_empty[s], 0x3);
-                        else umma_commit(&op_empty[s]);
-                    } else {
-                        const int slices = args.block / 16;
-                        for (int bi = 0; bi < nblk_stage; ++bi, ++pq) {
-                            const int p = pq % C::NP;
-                            if (!wait(&p_empty[p], ((pq / C::NP) & 1) ^ 1)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            for (int sl = 0; sl < slices; ++sl) {
-                                const int kk = bi * slices + sl;
-                                umma_f16(tmem_base + p * BN, umma_desc_sw128(a0 + kk * 32),
-                                         umma_desc_sw128(b0 + kk * 32), idesc, sl > 0 ? 1u : 0u);
-                            }
-                            umma_commit(&p_full[p]);
+                        tc_fence_after();
+                        for (int sl = 0; sl < slices; ++sl) {
+                            const int kk = bi * slices + sl;
+                            umma_f16(tmem_base + p * BN, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32),
+                                     idesc, sl > 0 ? 1u : 0u);
                         }
-                        umma_commit(&op_empty[s]);
+                        umma_commit(&p_full[p]);
                     }
-                }
-                if (kFolded && ok) {
-                    if constexpr (kPair) umma_commit_pair_mc(&p_full[tcount & 1], 0x3);
-                    else umma_commit(&p_full[tcount & 1]);
+                    umma_commit(&op_empty[s]);
                 }
             }
             // Drain: every MMA issued by this thread completes before TMEM is freed.
-            if constexpr (kPair) umma_commit_pair(drain);
-            else umma_commit(drain);
+            umma_commit(drain);
             uint32_t dummy = 0;
             mbar_wait(drain, 0, kErrTimeoutDrain, reinterpret_cast<volatile uint32_t *>(&dummy));
         }
     } else if (warp < 2 + C::NT) {
         // ------------------------------------------------------------ transform
-        // One operand row (64 codes, 32 bytes) per thread per stage.  The code
+        // One operand row (64 codes, 32 bytes) per thread per pass.  The code
         // tiles arrive with the 32-byte TMA swizzle: the two 16-byte halves of
         // row r are swapped when bit 2 of r is set, so the lanes of a quarter
         // warp read distinct banks.
         const int tt = threadIdx.x - 64;
         constexpr int kRows = BM + BN;
-        const int blk_shift = args.block == 16 ? 4 : 5;
         uint32_t it = 0;
         bool ok = true;
         for (int64_t t = unit; t < ntiles && ok; t += nunits) {
@@ -515,15 +389,12 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
                 const int cs = it % C::NC;
                 const int os = it % C::NO;
                 if (!warp_wait(&code_full[cs], (it / C::NC) & 1, kErrTimeoutTransform, abort_flag) ||
-                    !warp_wait<kPair>(&op_empty[os], ((it / C::NO) & 1) ^ 1, kErrTimeoutTransform,
-                                      abort_flag)) {
+                    !warp_wait(&op_empty[os], ((it / C::NO) & 1) ^ 1, kErrTimeoutTransform, abort_flag)) {
                     ok = false;
                     break;
                 }
                 const uint8_t *ca = code_a(cs);
                 const uint8_t *cb = code_b(cs);
-                const uint8_t *sa = sc_a(cs);
-                const uint8_t *sb = sc_b(cs);
                 uint8_t *oa = op_a(os);
                 uint8_t *ob = op_b(os);
 #pragma unroll 1
@@ -537,23 +408,10 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
                     const uint32_t words[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
                     uint8_t *dst = (isA ? oa : ob) + r * 128;
                     const uint32_t sw = static_cast<uint32_t>(r & 7);
-                    __half2 e2[4], n2[4];
-                    if (kFolded) {
-                        const uint8_t *sc = (isA ? sa : sb) + r;
-                        const int ld = isA ? BM : BN;
-                        const __half2 m8 = __float2half2_rn(-8.0f);
-#pragma unroll
-                        for (int b = 0; b < 4; ++b) {
-                            const int blk = (16 * b) >> blk_shift;
-                            e2[b] = e4m3_pair(sc[blk * ld]);
-                            n2[b] = __hmul2(e2[b], m8);
-                        }
-                    }
 #pragma unroll
                     for (int wi = 0; wi < 8; ++wi) {
                         uint32_t o[4];
-                        if (kFolded) expand_scaled<GRID>(words[wi], e2[wi >> 1], n2[wi >> 1], o);
-                        else expand_unscaled<GRID>(words[wi], o);
+                        expand_unscaled<GRID>(words[wi], o);
                         *reinterpret_cast<uint4 *>(dst + ((static_cast<uint32_t>(wi) ^ sw) << 4)) =
                             make_uint4(o[0], o[1], o[2], o[3]);
                     }
@@ -561,166 +419,113 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    if (kPair && rank != 0) mbar_arrive_remote(&op_full[os], 0);
-                    else mbar_arrive(&op_full[os]);
+                    mbar_arrive(&op_full[os]);
                     mbar_arrive(&code_empty[cs]);
                 }
             }
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // acc += (s_a * s_b) * partial per 16/32-block: thread = accumulator
+        // row (its TMEM lane), 64 columns per warp.
         const int ew = warp - 2 - C::NT;      // 0 .. NE-1
         const int q = warp & 3;               // TMEM lane quarter of this warp
+        const int cs = ew >> 2;               // column half: 64 columns
         const int row_in_tile = 32 * q + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-        if (kFolded) {
-            // E1M2 operands carry k = 4 * level on both sides: 1/16 (exact).
-            const float mult = __fmul_rn(__fmul_rn(*args.a_S, *args.b_S),
-                                         args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f));
-            uint32_t tcount = 0;
-            for (int64_t t = unit; t < ntiles; t += nunits, ++tcount) {
-                const Tile tl = get_tile<TM, TN>(args, t);
-                const int b = tcount & 1;
-                if (!warp_wait<kPair>(&p_full[b], (tcount >> 1) & 1, kErrTimeoutEpilogue, abort_flag))
+        const float mult = args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f);
+        const bool ue8 = args.scale_ue8m0 != 0;
+        uint32_t it = 0, pq = 0;
+        bool ok = true;
+        for (int64_t t = unit; t < ntiles && ok; t += nunits) {
+            const Tile tl = get_tile<TM, TN>(args, t);
+            float acc[64];
+#pragma unroll
+            for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
+            for (int ks = 0; ks < tl.nks && ok; ++ks, ++it) {
+                const int ss = it % C::NS;
+                if (!warp_wait(&sc_full[ss], (it / C::NS) & 1, kErrTimeoutEpilogue, abort_flag)) {
+                    ok = false;
                     break;
-                tc_fence_after();
-                const int64_t row = tl.m0 + 128 * rank + row_in_tile;
-                const bool row_ok = row < tl.g.m;
-                float *crow = args.c + (tl.g.c_row + row) * args.ldc + tl.g.c_col + tl.n0;
-#pragma unroll 1
-                for (int c = 0; c < TN / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(tmem_base + b * Lay::kAccCols + 32 * c + lane_addr, r);
-                    tmem_wait_ld();
-                    if (c == TN / 32 - 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) {
-                            if (kPair && rank != 0) mbar_arrive_remote(&p_empty[b], 0);
-                            else mbar_arrive(&p_empty[b]);
-                        }
-                    }
-                    if (!row_ok) continue;
-                    const int64_t col0 = tl.n0 + 32 * c;
-                    float v[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        v[i] = tl.nks > 0 ? __fmul_rn(__uint_as_float(r[i]), mult) : 0.0f;
-                    float *dst = crow + 32 * c;
-                    const bool vec = (col0 + 32 <= tl.g.n) &&
-                                     ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
-                    if (vec) {
-#pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            *reinterpret_cast<float4 *>(dst + i) =
-                                make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-                    } else {
-                        for (int i = 0; i < 32; ++i)
-                            if (col0 + i < tl.g.n) dst[i] = v[i];
-                    }
                 }
-            }
-        } else {
-            // fp32 block scales: acc += (s_a * s_b) * partial, per 16/32-block.
-            const int h = ew >> 2;            // column half (64 columns)
-            const float mult = args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f);
-            uint32_t it = 0, pq = 0;
-            bool ok = true;
-            for (int64_t t = unit; t < ntiles && ok; t += nunits) {
-                const Tile tl = get_tile<TM, TN>(args, t);
-                float acc[64];
-#pragma unroll
-                for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
-                for (int ks = 0; ks < tl.nks && ok; ++ks, ++it) {
-                    const int ss = it % NSr;
-                    if (!warp_wait(&sc_full[ss], (it / NSr) & 1, kErrTimeoutEpilogue, abort_flag)) {
+                const float *sa_tile = reinterpret_cast<const float *>(sc_a(ss));
+                const float *sb_tile = reinterpret_cast<const float *>(sc_b(ss));
+                // UE8M0 scales: exponent bytes in the same slots, 2^(E - 127)
+                const uint8_t *sa_u8 = sc_a(ss);
+                const uint8_t *sb_u8 = sc_b(ss);
+                for (int bi = 0; bi < nblk_stage; ++bi, ++pq) {
+                    const int p = pq % C::NP;
+                    if (!warp_wait(&p_full[p], (pq / C::NP) & 1, kErrTimeoutEpilogue, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    const float *sa_tile = reinterpret_cast<const float *>(sc_a(ss));
-                    const float *sb_tile = reinterpret_cast<const float *>(sc_b(ss));
-                    // UE8M0 scales: exponent bytes in the same slots, 2^(E - 127)
-                    const uint8_t *sa_u8 = sc_a(ss);
-                    const uint8_t *sb_u8 = sc_b(ss);
-                    const bool ue8 = args.scale_ue8m0 != 0;
-                    for (int bi = 0; bi < nblk_stage; ++bi, ++pq) {
-                        const int p = pq % C::NP;
-                        if (!warp_wait(&p_full[p], (pq / C::NP) & 1, kErrTimeoutEpilogue, abort_flag)) {
-                            ok = false;
-                            break;
+                    tc_fence_after();
+                    const float sa = ue8 ? ue8m0_to_f32(sa_u8[bi * BM + row_in_tile]) : sa_tile[bi * BM + row_in_tile];
+                    const float4 *sb4 = reinterpret_cast<const float4 *>(sb_tile + bi * BN + cs * 64);
+                    const uchar4 *sb4u = reinterpret_cast<const uchar4 *>(sb_u8 + bi * BN + cs * 64);
+                    const uint32_t ta = tmem_base + p * BN + cs * 64 + lane_addr;
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(ta + 32 * half, r);
+                        tmem_wait_ld();
+                        if (half == 1) {
+                            // partial buffer p read: the MMAs may refill it
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&p_empty[p]);
                         }
-                        tc_fence_after();
-                        const float sa = ue8 ? ue8m0_to_f32(sa_u8[bi * BM + row_in_tile])
-                                             : sa_tile[bi * BM + row_in_tile];
-                        const float4 *sb4 = reinterpret_cast<const float4 *>(sb_tile + bi * BN + h * 64);
-                        const uchar4 *sb4u = reinterpret_cast<const uchar4 *>(sb_u8 + bi * BN + h * 64);
-                        const uint32_t ta = tmem_base + p * BN + h * 64 + lane_addr;
 #pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            uint32_t r[32];
-                            tmem_ld_32x32b_x32(ta + 32 * half, r);
-                            tmem_wait_ld();
-                            if (half == 1) {
-                                tc_fence_before();
-                                __syncwarp();
-                                if (lane == 0) mbar_arrive(&p_empty[p]);
+                        for (int c4 = 0; c4 < 8; ++c4) {
+                            float4 sb;
+                            if (ue8) {
+                                const uchar4 e = sb4u[8 * half + c4];
+                                sb = make_float4(ue8m0_to_f32(e.x), ue8m0_to_f32(e.y), ue8m0_to_f32(e.z),
+                                                 ue8m0_to_f32(e.w));
+                            } else {
+                                sb = sb4[8 * half + c4];
                             }
-#pragma unroll
-                            for (int c4 = 0; c4 < 8; ++c4) {
-                                float4 sb;
-                                if (ue8) {
-                                    const uchar4 e = sb4u[8 * half + c4];
-                                    sb = make_float4(ue8m0_to_f32(e.x), ue8m0_to_f32(e.y), ue8m0_to_f32(e.z),
-                                                     ue8m0_to_f32(e.w));
-                                } else {
-                                    sb = sb4[8 * half + c4];
-                                }
-                                float *ac = acc + 32 * half + 4 * c4;
-                                ac[0] = __fmaf_rn(__fmul_rn(sa, sb.x), __uint_as_float(r[4 * c4 + 0]), ac[0]);
-                                ac[1] = __fmaf_rn(__fmul_rn(sa, sb.y), __uint_as_float(r[4 * c4 + 1]), ac[1]);
-                                ac[2] = __fmaf_rn(__fmul_rn(sa, sb.z), __uint_as_float(r[4 * c4 + 2]), ac[2]);
-                                ac[3] = __fmaf_rn(__fmul_rn(sa, sb.w), __uint_as_float(r[4 * c4 + 3]), ac[3]);
-                            }
+                            float *ac = acc + 32 * half + 4 * c4;
+                            ac[0] = __fmaf_rn(__fmul_rn(sa, sb.x), __uint_as_float(r[4 * c4 + 0]), ac[0]);
+                            ac[1] = __fmaf_rn(__fmul_rn(sa, sb.y), __uint_as_float(r[4 * c4 + 1]), ac[1]);
+                            ac[2] = __fmaf_rn(__fmul_rn(sa, sb.z), __uint_as_float(r[4 * c4 + 2]), ac[2]);
+                            ac[3] = __fmaf_rn(__fmul_rn(sa, sb.w), __uint_as_float(r[4 * c4 + 3]), ac[3]);
                         }
                     }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sc_empty[ss]);
                 }
-                if (!ok) break;
-                const int64_t row = tl.m0 + row_in_tile;
-                if (row < tl.g.m) {
-                    const int64_t col0 = tl.n0 + h * 64;
-                    float *dst = args.c + (tl.g.c_row + row) * args.ldc + tl.g.c_col + col0;
-                    const bool vec = (col0 + 64 <= tl.g.n) &&
-                                     ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
-                    if (vec) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sc_empty[ss]);
+            }
+            if (!ok) break;
+            const int64_t row = tl.m0 + row_in_tile;
+            if (row < tl.g.m) {
+                const int64_t col0 = tl.n0 + 64 * cs;
+                float *dst = args.c + (tl.g.c_row + row) * args.ldc + tl.g.c_col + col0;
+                const bool vec = (col0 + 64 <= tl.g.n) && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
+                if (vec) {
 #pragma unroll
-                        for (int i = 0; i < 64; i += 4)
-                            *reinterpret_cast<float4 *>(dst + i) =
-                                make_float4(acc[i] * mult, acc[i + 1] * mult, acc[i + 2] * mult,
-                                            acc[i + 3] * mult);
-                    } else {
+                    for (int i = 0; i < 64; i += 4)
+                        *reinterpret_cast<float4 *>(dst + i) =
+                            make_float4(acc[i] * mult, acc[i + 1] * mult, acc[i + 2] * mult, acc[i + 3] * mult);
+                } else {
 #pragma unroll
-                        for (int i = 0; i < 64; ++i)
-                            if (col0 + i < tl.g.n) dst[i] = acc[i] * mult;
-                    }
+                    for (int i = 0; i < 64; ++i)
+                        if (col0 + i < tl.g.n) dst[i] = acc[i] * mult;
                 }
             }
         }
     }
 
     tc_fence_before();
-    if constexpr (kPair) cluster_sync();
-    else __syncthreads();
+    __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        if constexpr (kPair) tmem_dealloc_pair(tmem_base, Lay::kTmemCols);
-        else tmem_dealloc(tmem_base, Lay::kTmemCols);
+        tmem_dealloc(tmem_base, C::kTmemCols);
     }
 }
 
 // ---------------------------------------------------------------------------
-// Native block-scaled FP4 path for two-level scales (modes 3 and 4).
+// Native block-scaled FP4 path for two-level scales, one CTA per tile (mode 3).
 //
 // kind::mxf4nvf4 multiplies E2M1 operands scaled per 16 elements by UE4M3
 // factors, which is exactly an E2M1 operand under the two-level scales (the
@@ -733,10 +538,7 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
 // same scale factors, the raw code tiles used as they arrived and only the
 // correction planes written by the transform warps (a per-byte bit function).
 //
-// Tiles: 128 x 192 on one CTA (mode 3) or 256 x 192 on a CTA pair with
-// cta_group::2 MMAs (mode 4): rank r of the pair stages A rows [128 r, +128)
-// and B rows [96 r, +96) of the tile, holds accumulator rows [128 r, +128),
-// and both ranks hold the scale factors of all 192 B rows.  192 columns let
+// Tiles: 128 x 192 on one CTA.  192 columns let
 // two accumulators share TMEM with one scale-factor slot per TMA stage, so the
 // epilogue of one tile overlaps the MMAs of the next and the transform runs
 // ahead of the MMAs as far as the TMA ring allows.  A stage covers 128 K elements
@@ -754,11 +556,11 @@ __global__ void __launch_bounds__(Layout<MODE>::kThreads, 1)
 // factors and built planes use two-slot rings, refilled once the MMAs two
 // stages back have completed.  The epilogue stages 128 x 32 fp32 chunks in
 // shared memory and writes them with coalesced 16-byte stores.
-template <int GRID, int CG, bool CIN>
+template <int GRID, bool CIN>
 struct Fp4Cfg {
     static constexpr int BN = kNativeTileN;         // tile columns (B rows)
-    static constexpr int BNh = BN / CG;             // B code rows staged per CTA
-    static constexpr int TM = BM * CG;              // tile rows
+    static constexpr int BNh = BN;                  // B code rows staged per CTA
+    static constexpr int TM = BM;                   // tile rows
     static constexpr int BKE = 128;                 // K elements per stage
     static constexpr int kRow = BKE / 2;            // code bytes per row per stage
     static constexpr int KST = BKE / 64;            // MMA K steps per stage
@@ -810,9 +612,9 @@ struct Fp4Cfg {
     static constexpr int o_scr = o_out + kOutChunk;
     static constexpr int o_raw = o_scr + kScr;
     static constexpr int o_bar = o_raw + NSF * kRawSlot;
-    // code ring: full, empty, cfull; scale-factor ring: sfull, sraw_free,
-    // sf_ready, tdone; acc_full[2], acc_empty[2], edone, drain
-    static constexpr int kNumBars = 3 * NS + 4 * NSF + 6;
+    // code ring: full, empty; scale-factor ring: sfull, sraw_free, sf_ready;
+    // acc_full[2], acc_empty[2], drain
+    static constexpr int kNumBars = 2 * NS + 3 * NSF + 5;
     static constexpr int o_misc = o_bar + kNumBars * 8;
     static constexpr int kAlloc = o_misc + 64 + 1024;
     // producer, MMA issuer, transform warps, epilogue warps, scale producer
@@ -823,7 +625,7 @@ struct Fp4Cfg {
     static_assert(kAlloc <= 232448, "shared memory budget");
     static_assert(o_corr % 1024 == 0 && o_out % 1024 == 0, "swizzle alignment");
     static_assert(BN % 32 == 0 && BN > 128 && BN <= 256, "two SFB row groups, 32-column chunks");
-    static_assert((BN / CG) % 8 == 0, "B rows per CTA");
+    static_assert(BN % 8 == 0, "B rows per CTA");
 };
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -843,54 +645,27 @@ __device__ __forceinline__ void transpose4x4(uint32_t w0, uint32_t w1, uint32_t 
     o[3] = prmt(t1, t3, 0x7632u);
 }
 
-// Arrive on the barrier at the same offset in CTA 0 of the cluster (plain
-// local arrive when this CTA is CTA 0 or there is no cluster).
-template <int CG>
-__device__ __forceinline__ void arrive_leader(uint64_t *bar, uint32_t rank) {
-    if (CG == 1 || rank == 0) mbar_arrive(bar);
-    else mbar_arrive_remote(bar, 0);
-}
-
-template <int CG>
-__device__ __forceinline__ void umma_fp4_bs_cg(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc,
-                                               uint32_t sfa, uint32_t sfb, uint32_t acc) {
-    if constexpr (CG == 1) umma_fp4_bs(d, ad, bd, idesc, sfa, sfb, acc);
-    else umma_fp4_bs_pair(d, ad, bd, idesc, sfa, sfb, acc);
-}
-
-// Completion of this thread's MMAs arrives on the barrier in every CTA of
-// the pair (or in this CTA).
-template <int CG>
-__device__ __forceinline__ void umma_commit_cg(uint64_t *bar) {
-    if constexpr (CG == 1) umma_commit(bar);
-    else umma_commit_pair_mc(bar, 0x3);
-}
-
-template <int GRID, int CG, bool CIN>
-__global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
+template <int GRID, bool CIN>
+__global__ void __launch_bounds__(Fp4Cfg<GRID, CIN>::kThreads, 1)
     gemm_fp4_kernel(const __grid_constant__ GemmArgs args) {
-    using C = Fp4Cfg<GRID, CG, CIN>;
+    using C = Fp4Cfg<GRID, CIN>;
     constexpr int BN = C::BN;
     constexpr int TM = C::TM;
     constexpr int NS = C::NS;
     constexpr int NSF = C::NSF;
-    constexpr bool kPair = CG == 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     // code ring (index s = it % NS)
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::o_bar);   // code tiles landed
     uint64_t *empty = full + NS;          // MMAs done with the stage (multicast commit)
-    uint64_t *cfull = empty + NS;         // pairs, in CTA 0: CTA 1's code tiles landed
     // scale-factor ring (index j = it % NSF)
-    uint64_t *sfull = cfull + NS;         // raw scale factors landed
+    uint64_t *sfull = empty + NS;         // raw scale factors landed
     uint64_t *sraw_free = sfull + NSF;    // transform read the raw slot
     uint64_t *sf_ready = sraw_free + NSF; // in CTA 0: factors in TMEM (all CTAs)
-    uint64_t *tdone = sf_ready + NSF;     // this CTA's transform warps done (pairs)
-    uint64_t *acc_full = tdone + NSF;     // [2]
+    uint64_t *acc_full = sf_ready + NSF;  // [2]
     uint64_t *acc_empty = acc_full + 2;   // [2], in CTA 0: accumulator drained (all CTAs)
-    uint64_t *edone = acc_empty + 2;      // this CTA's epilogue warps drained (pairs)
-    uint64_t *drain = edone + 1;
+    uint64_t *drain = acc_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::o_misc);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::o_misc + 4);
     auto stage = [&](int s) { return smem + s * C::kStage; };
@@ -900,27 +675,23 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
     const int lane = threadIdx.x & 31;
     const int blk = args.block;                       // 16 or 32
     const int nraw = C::BKE / blk;                    // raw scale rows per stage
-    const uint32_t rank = kPair ? cluster_ctarank() : 0u;
-    const int64_t unit = kPair ? (blockIdx.x >> 1) : blockIdx.x;
-    const int64_t nunits = kPair ? (gridDim.x >> 1) : gridDim.x;
+    const int64_t unit = blockIdx.x;
+    const int64_t nunits = gridDim.x;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
-            mbar_init(&cfull[i], 1);
         }
         for (int i = 0; i < NSF; ++i) {
             mbar_init(&sfull[i], 1);
             mbar_init(&sraw_free[i], C::kGroupWarps);
-            mbar_init(&sf_ready[i], kPair ? CG : C::kGroupWarps);
-            mbar_init(&tdone[i], C::kGroupWarps);
+            mbar_init(&sf_ready[i], C::kGroupWarps);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], kPair ? CG : C::NE);
+            mbar_init(&acc_empty[i], C::NE);
         }
-        mbar_init(edone, C::NE);
         mbar_init(drain, 1);
         *abort_flag = 0u;
         fence_barrier_init();
@@ -935,13 +706,9 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
             tma_prefetch_desc(&args.tm_b_corr);
         }
     }
-    if (warp == 1) {
-        if constexpr (kPair) tmem_alloc_pair(tmem_slot, 512);
-        else tmem_alloc(tmem_slot, 512);
-    }
+    if (warp == 1) tmem_alloc(tmem_slot, 512);
     tc_fence_before();
-    if constexpr (kPair) cluster_sync();
-    else __syncthreads();
+    __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int64_t ntiles = total_tiles<TM, BN>(args);
@@ -955,7 +722,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
             for (int64_t t = unit; t < ntiles && ok; t += nunits) {
                 const Tile tl = get_tile<TM, BN>(args, t);
                 const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
-                const int32_t arow = static_cast<int32_t>(tl.g.a_row + tl.m0 + BM * rank);
+                const int32_t arow = static_cast<int32_t>(tl.g.a_row + tl.m0);
                 const int32_t brow = static_cast<int32_t>(tl.g.b_row + tl.n0);
                 for (int ks = 0; ks < nks; ++ks, ++it) {
                     const int s = it % NS;
@@ -973,7 +740,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                         tma_load_2d_hint(rs + C::o_raw_b, &args.tm_b_scales, &sfull[s], brow, bcol / blk, pol);
                     }
                     mbar_arrive_expect_tx(&full[s], C::kIn * (C::kCodesA + C::kCodesB));
-                    const int32_t brow_h = brow + C::BNh * static_cast<int32_t>(rank);
+                    const int32_t brow_h = brow;
                     // Operand tiles are read by many CTAs: keep them in L2
                     // ahead of the streamed output.
                     if (CIN && args.planes3d) {
@@ -1003,32 +770,11 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ UMMA issuer (CTA 0)
-        if constexpr (kPair) {
-            // CTA 1: relay each stage's landed code tiles to CTA 0's MMAs.
-            if (lane == 0 && rank == 1) {
-                uint32_t it = 0;
-                bool ok = true;
-                for (int64_t t = unit; t < ntiles && ok; t += nunits) {
-                    const Tile tl = get_tile<TM, BN>(args, t);
-                    const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
-                    for (int ks = 0; ks < nks; ++ks, ++it) {
-                        const int s = it % NS;
-                        if (!mbar_wait(&full[s], (it / NS) & 1, kErrTimeoutMma, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        fence_proxy_async_cluster();
-                        mbar_arrive_remote(&cfull[s], 0);
-                    }
-                }
-            }
-        }
-        if (lane == 0 && rank == 0) {
+        // ------------------------------------------------------------ UMMA issuer
+        if (lane == 0) {
             constexpr uint32_t idesc = umma_idesc_fp4_bs(TM, BN);
             auto wait_any = [&](uint64_t *bar, uint32_t parity) {
-                return kPair ? mbar_wait_cluster(bar, parity, kErrTimeoutMma, abort_flag)
-                             : mbar_wait(bar, parity, kErrTimeoutMma, abort_flag);
+                return mbar_wait(bar, parity, kErrTimeoutMma, abort_flag);
             };
             uint32_t it = 0, tcount = 0;
             bool ok = true;
@@ -1043,11 +789,9 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                 for (int ks = 0; ks < nks && ok; ++ks, ++it) {
                     const int s = it % NS;
                     const int j = it % NSF;
-                    // factors in TMEM (with pairs: both CTAs'), then the code
-                    // tiles (with pairs: CTA 1's relayed by its idle MMA warp)
+                    // factors in TMEM, then the code tiles
                     if (!wait_any(&sf_ready[j], (it / NSF) & 1) ||
-                        !mbar_wait(&full[s], (it / NS) & 1, kErrTimeoutMma, abort_flag) ||
-                        (kPair && !wait_any(&cfull[s], (it / NS) & 1))) {
+                        !mbar_wait(&full[s], (it / NS) & 1, kErrTimeoutMma, abort_flag)) {
                         ok = false;
                         break;
                     }
@@ -1067,25 +811,24 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                     for (int j = 0; j < steps; ++j) {
                         const uint32_t sfa = sf0 + 12 * j, sfb = sfa + 4;
                         const uint32_t dk = 32 * j;
-                        umma_fp4_bs_cg<CG>(d_tmem, umma_desc_sw64(a0 + dk), umma_desc_sw64(b0 + dk), idesc,
+                        umma_fp4_bs(d_tmem, umma_desc_sw64(a0 + dk), umma_desc_sw64(b0 + dk), idesc,
                                            sfa, sfb, first ? 0u : 1u);
                         first = false;
                         if (GRID == 0) {
-                            umma_fp4_bs_cg<CG>(d_tmem, umma_desc_sw64(a0 + dk), umma_desc_sw64(bc + dk),
+                            umma_fp4_bs(d_tmem, umma_desc_sw64(a0 + dk), umma_desc_sw64(bc + dk),
                                                idesc, sfa, sfb, 1u);
-                            umma_fp4_bs_cg<CG>(d_tmem, umma_desc_sw64(ac + dk), umma_desc_sw64(b0 + dk),
+                            umma_fp4_bs(d_tmem, umma_desc_sw64(ac + dk), umma_desc_sw64(b0 + dk),
                                                idesc, sfa, sfb, 1u);
-                            umma_fp4_bs_cg<CG>(d_tmem, umma_desc_sw64(ac + dk), umma_desc_sw64(bc + dk),
+                            umma_fp4_bs(d_tmem, umma_desc_sw64(ac + dk), umma_desc_sw64(bc + dk),
                                                idesc, sfa, sfb, 1u);
                         }
                     }
-                    umma_commit_cg<CG>(&empty[s]);
+                    umma_commit(&empty[s]);
                 }
-                if (ok) umma_commit_cg<CG>(&acc_full[ab]);
+                if (ok) umma_commit(&acc_full[ab]);
             }
             // Drain: every MMA issued here completes before TMEM is freed.
-            if constexpr (kPair) umma_commit_pair(drain);
-            else umma_commit(drain);
+            umma_commit(drain);
             uint32_t dummy = 0;
             mbar_wait(drain, 0, kErrTimeoutDrain, reinterpret_cast<volatile uint32_t *>(&dummy));
         }
@@ -1202,25 +945,9 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                 tmem_wait_st();
                 __syncwarp();
                 tc_fence_before();
-                if constexpr (kPair) {
-                    // The MMAs of CTA 0 read this CTA's tiles: one relay
-                    // arrive per CTA after all warps of the group.
-                    fence_proxy_async_cluster();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&tdone[j]);
-                    if (gt == 0) {
-                        if (!mbar_wait(&tdone[j], jph, kErrTimeoutTransform, abort_flag)) {
-                            ok = false;
-                        } else {
-                            arrive_leader<CG>(&sf_ready[j], rank);
-                        }
-                    }
-                    __syncwarp();
-                } else {
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sf_ready[j]);
-                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_ready[j]);
             }
         }
     } else if (warp < 2 + C::NT + C::NE) {
@@ -1234,7 +961,6 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
         const int et = threadIdx.x - 32 * (2 + C::NT);   // 0 .. 127
         const int row_in_tile = 32 * q + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-        const bool elected = et == 0;
         constexpr uint32_t kEpiThreads = 32 * C::NE;
         uint8_t *buf = smem + C::o_out;
         // E1M2 operands carry k = 4 * level on both sides: 1/16 (exact).
@@ -1248,7 +974,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
             // one decision for the four epilogue warps (they share barrier 1)
             if (named_bar_or(1, kEpiThreads, !ok)) break;
             tc_fence_after();
-            const int64_t m0 = tl.m0 + BM * rank;     // this CTA's accumulator rows
+            const int64_t m0 = tl.m0;                 // accumulator rows of the tile
             const int64_t row = m0 + row_in_tile;
             const bool row_ok = row < tl.g.m;
             float *crow = args.c + (tl.g.c_row + row) * args.ldc + tl.g.c_col + tl.n0;
@@ -1263,16 +989,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
                     // accumulator drained: the MMAs of tile t + 2 may start
                     tc_fence_before();
                     __syncwarp();
-                    if constexpr (kPair) {
-                        if (lane == 0) mbar_arrive(edone);
-                        if (elected) {
-                            if (mbar_wait(edone, tcount & 1, kErrTimeoutEpilogue, abort_flag))
-                                arrive_leader<CG>(&acc_empty[ab], rank);
-                        }
-                        __syncwarp();
-                    } else {
-                        if (lane == 0) mbar_arrive(&acc_empty[ab]);
-                    }
+                    if (lane == 0) mbar_arrive(&acc_empty[ab]);
                 }
                 const int64_t col0 = tl.n0 + 32 * c;
                 if (col0 >= tl.g.n) continue;             // the same for all threads
@@ -1325,7 +1042,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
             for (int64_t t = unit; t < ntiles && ok; t += nunits) {
                 const Tile tl = get_tile<TM, BN>(args, t);
                 const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
-                const int32_t arow = static_cast<int32_t>(tl.g.a_row + tl.m0 + BM * rank);
+                const int32_t arow = static_cast<int32_t>(tl.g.a_row + tl.m0);
                 const int32_t brow = static_cast<int32_t>(tl.g.b_row + tl.n0);
                 for (int ks = 0; ks < nks; ++ks, ++it) {
                     const int j = it % NSF;
@@ -1354,12 +1071,10 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CG, CIN>::kThreads, 1)
     }
 
     tc_fence_before();
-    if constexpr (kPair) cluster_sync();
-    else __syncthreads();
+    __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        if constexpr (kPair) tmem_dealloc_pair(tmem_base, 512);
-        else tmem_dealloc(tmem_base, 512);
+        tmem_dealloc(tmem_base, 512);
     }
 }
 
@@ -1409,7 +1124,6 @@ struct PairCfg {
     static constexpr int kRawB = 256 * kRawRows;
     static constexpr int kStage = (kCodeBytes + kRawA + kRawB + 1023) / 1024 * 1024;
     static constexpr int kAtoms = 3 * KST;          // SFA, SFB rows 0-127, SFB rows 128-255 per K step
-    static constexpr int kAtomX = 64 * KST;         // u64 units of one stage's atoms along K (ATOMS)
     static constexpr int kScr = ATOMS ? 0 : 4 * kAtoms * 512;   // one atom scratch per factor warp
     static constexpr int kOutChunk = 128 * 32 * 4;  // epilogue staging: 128 rows x 32 fp32
     static constexpr int kOutBufs = 2;              // staging buffers (bulk stores in flight)
@@ -1579,9 +1293,11 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
                         // factor atoms of this CTA's A rows and of all 256 B rows, with the
                         // code tiles on the leader's barrier: 128 K elements per box
                         if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (C::kCodeBytes + C::kRawA + C::kRawB));
-                        const int32_t ax = static_cast<int32_t>(C::kAtomX * ks);
+                        // 64 u64 per atom of kAtomK K elements (dense problems: acol = bcol)
+                        constexpr int kAtomK = C::kMx ? 128 : 64;
+                        const int32_t ax = 64 * (acol / kAtomK), bx = 64 * (bcol / kAtomK);
                         tma_load_2d_pair(st + C::o_raw_a, &args.tm_a_atoms, fb, ax, arow / 128, pol);
-                        tma_load_2d_pair(st + C::o_raw_b, &args.tm_b_atoms, fb, ax, brow / 128, pol);
+                        tma_load_2d_pair(st + C::o_raw_b, &args.tm_b_atoms, fb, bx, brow / 128, pol);
                     } else {
                         // this CTA's raw factors
                         mbar_arrive_expect_tx(&sfull[s], (128 + 256) * nraw);
@@ -1662,22 +1378,21 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
                                            first ? 0u : 1u);
                             first = false;
                         }
-                        umma_commit_pair_mc(&empty[s], 0x3);
-                        continue;
-                    }
-                    for (int j = 0; j < steps; ++j) {
-                        const uint32_t sfa = sf0 + 12 * j, sfb = sfa + 4;
-                        const uint32_t dk = 32 * j;
-                        umma_fp4_bs_pair(tmem_base, umma_desc_sw64(a0 + dk), umma_desc_sw64(b0 + dk), idesc, sfa,
-                                         sfb, first ? 0u : 1u);
-                        first = false;
-                        if (GRID == 0) {
-                            umma_fp4_bs_pair(tmem_base, umma_desc_sw64(a0 + dk), umma_desc_sw64(bc + dk), idesc,
-                                             sfa, sfb, 1u);
-                            umma_fp4_bs_pair(tmem_base, umma_desc_sw64(ac + dk), umma_desc_sw64(b0 + dk), idesc,
-                                             sfa, sfb, 1u);
-                            umma_fp4_bs_pair(tmem_base, umma_desc_sw64(ac + dk), umma_desc_sw64(bc + dk), idesc,
-                                             sfa, sfb, 1u);
+                    } else {
+                        for (int j = 0; j < steps; ++j) {
+                            const uint32_t sfa = sf0 + 12 * j, sfb = sfa + 4;
+                            const uint32_t dk = 32 * j;
+                            umma_fp4_bs_pair(tmem_base, umma_desc_sw64(a0 + dk), umma_desc_sw64(b0 + dk), idesc,
+                                             sfa, sfb, first ? 0u : 1u);
+                            first = false;
+                            if (GRID == 0) {
+                                umma_fp4_bs_pair(tmem_base, umma_desc_sw64(a0 + dk), umma_desc_sw64(bc + dk), idesc,
+                                                 sfa, sfb, 1u);
+                                umma_fp4_bs_pair(tmem_base, umma_desc_sw64(ac + dk), umma_desc_sw64(b0 + dk), idesc,
+                                                 sfa, sfb, 1u);
+                                umma_fp4_bs_pair(tmem_base, umma_desc_sw64(ac + dk), umma_desc_sw64(bc + dk), idesc,
+                                                 sfa, sfb, 1u);
+                            }
                         }
                     }
                     umma_commit_pair_mc(&empty[s], 0x3);
@@ -1919,69 +1634,46 @@ cudaError_t launch_pair(const GemmArgs &args, int num_sms, cudaStream_t stream) 
     return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<GRID, ATOMS>, args);
 }
 
-template <int GRID, int CG, bool CIN>
+template <int GRID, bool CIN>
 cudaError_t launch_fp4(const GemmArgs &args, int num_sms, cudaStream_t stream) {
-    using C = Fp4Cfg<GRID, CG, CIN>;
+    using C = Fp4Cfg<GRID, CIN>;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_fp4_kernel<GRID, CG, CIN>,
+        cudaError_t e = cudaFuncSetAttribute(gemm_fp4_kernel<GRID, CIN>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc);
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    int units = num_sms / CG;
+    int units = num_sms;
     if (args.groups == nullptr) {
         const GemmGroup &g = args.single;
         const int64_t tiles = ((g.m + C::TM - 1) / C::TM) * ((g.n + C::BN - 1) / C::BN);
         if (tiles < units) units = static_cast<int>(tiles);
     }
     if (units <= 0) return cudaSuccess;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(units * CG, 1, 1);
-    cfg.blockDim = dim3(C::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = C::kAlloc;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CG;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_fp4_kernel<GRID, CG, CIN>, args);
+    gemm_fp4_kernel<GRID, CIN><<<units, C::kThreads, C::kAlloc, stream>>>(args);
+    return cudaGetLastError();
 }
 
-template <int MODE, int GRID>
-cudaError_t launch_impl(const GemmArgs &args, int num_sms, cudaStream_t stream) {
-    using Lay = Layout<MODE>;
-    using C = Cfg<MODE>;
+template <int GRID>
+cudaError_t launch_f32s(const GemmArgs &args, int num_sms, cudaStream_t stream) {
+    using C = F32sCfg;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tn_kernel<MODE, GRID>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
+        cudaError_t e = cudaFuncSetAttribute(gemm_f32s_kernel<GRID>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kAlloc);
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    int units = num_sms / C::CG;
+    int units = num_sms;
     if (args.groups == nullptr) {
         const GemmGroup &g = args.single;
         const int64_t tiles = ((g.m + C::TM - 1) / C::TM) * ((g.n + C::TN - 1) / C::TN);
         if (tiles < units) units = static_cast<int>(tiles);
     }
     if (units <= 0) return cudaSuccess;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(units * C::CG, 1, 1);
-    cfg.blockDim = dim3(Lay::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = Lay::kAlloc;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C::CG;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tn_kernel<MODE, GRID>, args);
+    gemm_f32s_kernel<GRID><<<units, C::kThreads, C::kAlloc, stream>>>(args);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -1990,18 +1682,10 @@ cudaError_t launch_gemm(const GemmArgs &args, int mode, int grid_kind, int num_s
                         cudaStream_t stream) {
     switch (mode) {
         case 0:
-            return grid_kind == 0 ? launch_impl<0, 0>(args, num_sms, stream)
-                                  : launch_impl<0, 1>(args, num_sms, stream);
-        case 1:
-            return grid_kind == 0 ? launch_impl<1, 0>(args, num_sms, stream)
-                                  : launch_impl<1, 1>(args, num_sms, stream);
-        case 2:
-            return grid_kind == 0 ? launch_impl<2, 0>(args, num_sms, stream)
-                                  : launch_impl<2, 1>(args, num_sms, stream);
+            return grid_kind == 0 ? launch_f32s<0>(args, num_sms, stream) : launch_f32s<1>(args, num_sms, stream);
         case 3:
-            if (grid_kind == 1) return launch_fp4<1, 1, false>(args, num_sms, stream);
-            return args.corr_in ? launch_fp4<0, 1, true>(args, num_sms, stream)
-                                : launch_fp4<0, 1, false>(args, num_sms, stream);
+            if (grid_kind == 1) return launch_fp4<1, false>(args, num_sms, stream);
+            return args.corr_in ? launch_fp4<0, true>(args, num_sms, stream) : launch_fp4<0, false>(args, num_sms, stream);
         case 5:
             if (args.atoms)
                 return grid_kind == 1 ? launch_pair<1, true>(args, num_sms, stream)
@@ -2011,9 +1695,7 @@ cudaError_t launch_gemm(const GemmArgs &args, int mode, int grid_kind, int num_s
         case 6:
             return args.atoms ? launch_pair<3, true>(args, num_sms, stream) : launch_pair<3, false>(args, num_sms, stream);
         default:
-            if (grid_kind == 1) return launch_fp4<1, 2, false>(args, num_sms, stream);
-            return args.corr_in ? launch_fp4<0, 2, true>(args, num_sms, stream)
-                                : launch_fp4<0, 2, false>(args, num_sms, stream);
+            return cudaErrorInvalidValue;
     }
 }
 

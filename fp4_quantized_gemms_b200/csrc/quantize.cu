@@ -828,6 +828,11 @@ __device__ __forceinline__ void unit_part(const QuantArgs &q, const uint8_t *til
 //           column-wise into `a` as AXIS 1, then row-wise into `a2` (thread t
 //           takes row t & 63 of box t >> 6: 64 columns of one input row).
 //           One read of the tensor serves both of its GEMM operands.
+// Limit of the producer's wait for a free stage (ns).  Only test support
+// lowers it, to make that bounded wait run out on purpose; the drain and the
+// compute warps keep the normal bound.
+static __device__ uint64_t g_producer_wait_limit_ns = kWaitLimitNs;
+
 template <int AXIS, int NH, int BLK, int GRID, int RND, bool AMAX_ONLY>
 __global__ void __launch_bounds__(kCtaThreads, kCtasPerSm)
     rht_quantize_kernel(const __grid_constant__ QuantArgs a, const __grid_constant__ QuantArgs a2,
@@ -888,8 +893,8 @@ __global__ void __launch_bounds__(kCtaThreads, kCtasPerSm)
             uint32_t it = 0;
             for (int64_t u = u0; u < nunits; u += gridDim.x, ++it) {
                 const int s = it % kStages;
-                if (it >= kStages &&
-                    !mbar_wait(&empty[s], ((it / kStages) - 1) & 1, kErrTimeoutProducer, abort_flag))
+                if (it >= kStages && !mbar_wait(&empty[s], ((it / kStages) - 1) & 1, kErrTimeoutProducer,
+                                                abort_flag, g_producer_wait_limit_ns))
                     break;
                 issue(u, s);
             }
@@ -1184,6 +1189,11 @@ cudaError_t launch_rht_bf16(QuantArgs a, int hadamard_n, uint16_t *y, int64_t ld
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
+}
+
+cudaError_t quantize_set_producer_wait_limit(uint64_t limit_ns) {
+    const uint64_t v = limit_ns == 0 ? kWaitLimitNs : limit_ns;
+    return cudaMemcpyToSymbol(g_producer_wait_limit_ns, &v, sizeof(v));
 }
 
 cudaError_t quantize_read_and_clear_error_word(uint32_t *out) {

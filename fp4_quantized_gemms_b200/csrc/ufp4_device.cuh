@@ -79,25 +79,18 @@ __device__ __forceinline__ uint32_t e1m2_correction(uint32_t w) {
 // Only the pipelined GEMM translation unit includes this section.
 static __device__ uint32_t g_error_word = 0;
 
-enum : uint32_t {
-    kErrTimeoutProducer = 1u << 0,
-    kErrTimeoutTransform = 1u << 1,
-    kErrTimeoutMma = 1u << 2,
-    kErrTimeoutEpilogue = 1u << 3,
-    kErrTimeoutDrain = 1u << 4,
-};
 
 // Waits for the phase with the given parity to complete.  Gives up after
 // kWaitLimitNs (or at once when *abort is set by another role of the CTA),
 // records `err` in the device error word and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t err,
-                                          volatile uint32_t *abort) {
+                                          volatile uint32_t *abort, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             atomicOr(&g_error_word, err);
             *abort = 1u;
             return false;

@@ -9,6 +9,21 @@
 
 namespace ufp4 {
 
+// Bits of the device error word: a bounded wait of that role gave up
+// (kernels OR them in; the host reads and clears the word in
+// ufp4_check_device_status).
+enum : uint32_t {
+    kErrTimeoutProducer = 1u << 0,
+    kErrTimeoutTransform = 1u << 1,
+    kErrTimeoutMma = 1u << 2,
+    kErrTimeoutEpilogue = 1u << 3,
+    kErrTimeoutDrain = 1u << 4,
+};
+
+}  // namespace ufp4
+
+namespace ufp4 {
+
 // The ten round keys of a Philox4x32-10 key: (x, y)_r = key + r * (the two
 // Weyl constants), the schedule of Salmon et al. (SC'11).
 struct PhiloxKeys {
@@ -102,7 +117,7 @@ struct GemmArgs {
     CUtensorMap tm_a_e8, tm_b_e8;         // MX path: E4M3 element planes [rows][kpad]
     int c_tma;                            // tm_c valid: single problem, c_vec, c_col == 0
     CUtensorMap tm_a_atoms, tm_b_atoms;   // factor atoms as u64 [row groups][64 atoms_k]
-    int atoms;                            // both operands carry factor atoms (pair kernels)
+    int atoms;                            // both operands carry factor atoms (pair kernels, dense)
 };
 
 // Tile columns (B rows) of the native block-scaled FP4 kernels (modes 3, 4).

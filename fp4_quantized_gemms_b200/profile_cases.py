@@ -4,6 +4,7 @@ launch ends quickly.  Each case runs its kernel twice: a warm-up launch and
 the launch to capture.
 
     python -m fp4_quantized_gemms_b200.profile_cases gemm --m 4096 --n 4096 --k 2048 --grid e1m2
+    python -m fp4_quantized_gemms_b200.profile_cases gemm --m 4096 --n 8192 --k 8192 --mx
     python -m fp4_quantized_gemms_b200.profile_cases quantize --rows 8192 --cols 8192 --axis rows --sr
     python -m fp4_quantized_gemms_b200.profile_cases quantize --rows 8192 --cols 2048 --dual
     python -m fp4_quantized_gemms_b200.profile_cases stats --rows 8192 --cols 8192 --axis rows
@@ -23,10 +24,14 @@ def _dev(bits: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def gemm_case(m: int, n: int, k: int, grid: int, path: int) -> None:
-    """Quantize X [m, k] and W [n, k] (two-level scales, RHT16, block 16),
+def gemm_case(m: int, n: int, k: int, grid: int, path: int, mx: bool = False) -> None:
+    """Quantize X [m, k] and W [n, k] (RHT16; two-level scales with block 16,
+    or with `mx` UE8M0 scales with block 32 and the E4M3 element planes),
     then run the FPROP GEMM twice."""
-    cfg = ufp4.QuantConfig(grid=grid, hadamard_n=16, block=16, scale_fmt=ufp4.SCALE_E4M3_X_FP32)
+    if mx:
+        cfg = ufp4.QuantConfig(grid=grid, hadamard_n=16, block=32, scale_fmt=ufp4.SCALE_UE8M0)
+    else:
+        cfg = ufp4.QuantConfig(grid=grid, hadamard_n=16, block=16, scale_fmt=ufp4.SCALE_E4M3_X_FP32)
     qx = ufp4.rht_quantize(_dev(wl.normal(m, k, 1.0, 1)), ufp4.ALONG_COLS, cfg)
     qw = ufp4.rht_quantize(_dev(wl.normal(n, k, 0.02, 2)), ufp4.ALONG_COLS, cfg)
     ufp4.set_two_level_gemm_path(path)
@@ -79,6 +84,7 @@ def main() -> None:
     g.add_argument("--k", type=int, default=2048)
     g.add_argument("--grid", choices=["e1m2", "e2m1"], default="e1m2")
     g.add_argument("--path", type=int, default=ufp4.GEMM_PATH_AUTO)
+    g.add_argument("--mx", action="store_true", help="UE8M0 block-32 scales (the MX path)")
     q = sub.add_parser("quantize")
     q.add_argument("--rows", type=int, default=8192)
     q.add_argument("--cols", type=int, default=8192)
@@ -92,7 +98,7 @@ def main() -> None:
     t.add_argument("--axis", choices=["cols", "rows"], default="rows")
     a = ap.parse_args()
     if a.case == "gemm":
-        gemm_case(a.m, a.n, a.k, ufp4.GRID_E1M2 if a.grid == "e1m2" else ufp4.GRID_E2M1, a.path)
+        gemm_case(a.m, a.n, a.k, ufp4.GRID_E1M2 if a.grid == "e1m2" else ufp4.GRID_E2M1, a.path, a.mx)
     elif a.case == "stats":
         stats_case(a.rows, a.cols, ufp4.ALONG_COLS if a.axis == "cols" else ufp4.ALONG_ROWS)
     else:

@@ -32,7 +32,7 @@ EXPORTED = [
     "ufp4_status_string", "ufp4_version", "ufp4_set_two_level_gemm_path",
     "ufp4_get_two_level_gemm_path", "ufp4_rht_quantize_dual", "ufp4_rht_amax_dual",
     "ufp4_quant_stats", "ufp4_qstats_summarize", "ufp4_sqnr_sums", "ufp4_rht_bf16",
-    "ufp4_sf_atoms_layout",
+    "ufp4_sf_atoms_layout", "ufp4_test_set_quantize_wait_limit",
 ]
 
 
@@ -120,6 +120,11 @@ def lib() -> ctypes.CDLL:
                                         i32, P, i64, P]
         L.ufp4_check_device_status.restype = st
         L.ufp4_check_device_status.argtypes = []
+        L.ufp4_sf_atoms_layout.restype = st
+        L.ufp4_sf_atoms_layout.argtypes = [i64, i64, ctypes.POINTER(QuantCfgC), ctypes.POINTER(i64),
+                                           ctypes.POINTER(ctypes.c_size_t)]
+        L.ufp4_test_set_quantize_wait_limit.restype = st
+        L.ufp4_test_set_quantize_wait_limit.argtypes = [u64]
         L.ufp4_set_two_level_gemm_path.restype = st
         L.ufp4_set_two_level_gemm_path.argtypes = [i32]
         L.ufp4_get_two_level_gemm_path.restype = i32
@@ -440,9 +445,7 @@ def grouped_gemm(a: QTensor, b: QTensor, groups: torch.Tensor, out: torch.Tensor
     return out
 
 
-GEMM_PATH_AUTO, GEMM_PATH_FP16, GEMM_PATH_FP16_PAIR, GEMM_PATH_NATIVE_FP4 = 0, 1, 2, 3
-GEMM_PATH_NATIVE_FP4_PAIR = 4
-GEMM_PATH_NATIVE_FP4_PAIR256 = 5
+GEMM_PATH_AUTO, GEMM_PATH_NATIVE_FP4, GEMM_PATH_NATIVE_FP4_PAIR256 = 0, 3, 5
 
 
 def set_two_level_gemm_path(path: int) -> None:
@@ -457,3 +460,8 @@ def get_two_level_gemm_path() -> int:
 def check_device_status() -> int:
     """Reads and clears the kernels' device error word (synchronises)."""
     return lib().ufp4_check_device_status()
+
+
+def set_quantize_wait_limit_for_tests(limit_ns: int) -> None:
+    """Test support: the quantizer producer's wait limit in ns (0: default)."""
+    _check(lib().ufp4_test_set_quantize_wait_limit(limit_ns), "ufp4_test_set_quantize_wait_limit")

@@ -308,7 +308,9 @@ ufp4_status_t ufp4_gemm_wgrad(const ufp4_qtensor_t *dytq, const ufp4_qtensor_t *
  * per-expert token windows along K (WGRAD, segments zero-padded to 64).
  * Requirements checked on the device: k, a_col, b_col multiples of 64; a_row,
  * b_row multiples of 16; a group that violates them is skipped and writes
- * nothing.  Reads outside an operand return zeros.  The caller guarantees that
+ * nothing.  Factor atoms (sf_atoms) are not read here: the grouped kernels
+ * build the factors from the block-major scales.  Reads outside an operand
+ * return zeros.  The caller guarantees that
  * every group's output window lies inside c_dev [..][ldc] and that groups do
  * not overlap.  Errors: INVALID_ARG, ALIGNMENT, OPERAND_MISMATCH, CUDA. */
 ufp4_status_t ufp4_grouped_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
@@ -316,34 +318,26 @@ ufp4_status_t ufp4_grouped_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b
                                 float *c_dev, int64_t ldc, void *stream);
 
 /* Kernel family for GEMMs whose operands carry two-level (E4M3 x fp32)
- * scales.  Every family computes the same contraction (the quantized values
- * are exact in each operand format and products accumulate in fp32); they
- * differ in how the tensor core is fed:
- *   UFP4_GEMM_PATH_FP16       scales folded into exact fp16 operands,
- *                             kind::f16 MMA, one CTA per 128 x 256 tile;
- *   UFP4_GEMM_PATH_FP16_PAIR  the same on a CTA pair (256 x 256 tiles);
- *   UFP4_GEMM_PATH_NATIVE_FP4 block-scaled FP4 MMA (kind::mxf4nvf4, UE4M3
- *                             factors per 16 elements); E1M2 codes are split
- *                             exactly into two E2M1 planes (four MMAs); one
- *                             CTA per 128 x 192 tile;
- *   UFP4_GEMM_PATH_NATIVE_FP4_PAIR  the same on CTA pairs (cta_group::2,
- *                             256 x 192 tiles);
- *   UFP4_GEMM_PATH_NATIVE_FP4_PAIR256  block-scaled FP4 MMA on CTA pairs with
- *                             256 x 256 tiles (half the operand bytes per
- *                             flop of one CTA); needs E2M1 operands, or E1M2
- *                             operands whose correction planes follow their
- *                             codes in one allocation (else the one-CTA path);
+ * scales.  Both families run the block-scaled FP4 MMA (kind::mxf4nvf4, UE4M3
+ * factors per 16 elements), with E1M2 codes split exactly into two E2M1
+ * planes (four MMAs per K step), and compute the same contraction:
+ *   UFP4_GEMM_PATH_NATIVE_FP4 one CTA per 128 x 192 tile, two accumulators
+ *                             (the epilogue overlaps the next tile);
+ *   UFP4_GEMM_PATH_NATIVE_FP4_PAIR256  CTA pairs (cta_group::2) with 256 x 256
+ *                             tiles (half the operand bytes per flop of one
+ *                             CTA); needs E2M1 operands, or E1M2 operands whose
+ *                             correction planes follow their codes in one
+ *                             allocation (else the one-CTA path);
  *   UFP4_GEMM_PATH_AUTO       the library's choice (default; currently the
  *                             256 x 256 CTA-pair path where it applies, else
- *                             the one-CTA native FP4 path).
- * The setting is process-wide and read at each GEMM call; fp32 and UE8M0
- * block scales are unaffected (they always run the fp32-scale kernel).  Errors: INVALID_ARG for an unknown path. */
+ *                             the one-CTA path).
+ * Values 1, 2 and 4 named kernel families that are no longer built.  The
+ * setting is process-wide and read at each GEMM call; fp32 and UE8M0 block
+ * scales are unaffected (fp32-scale kernel, or the MX path).  Errors:
+ * INVALID_ARG for any other value. */
 typedef enum {
     UFP4_GEMM_PATH_AUTO = 0,
-    UFP4_GEMM_PATH_FP16 = 1,
-    UFP4_GEMM_PATH_FP16_PAIR = 2,
     UFP4_GEMM_PATH_NATIVE_FP4 = 3,
-    UFP4_GEMM_PATH_NATIVE_FP4_PAIR = 4,
     UFP4_GEMM_PATH_NATIVE_FP4_PAIR256 = 5
 } ufp4_gemm_path_t;
 ufp4_status_t ufp4_set_two_level_gemm_path(int32_t path);
@@ -415,6 +409,16 @@ ufp4_status_t ufp4_sqnr_sums(const float *ref_dev, int64_t ld_ref, const float *
  * bounded pipeline wait gives up (synchronises the current device).
  * Returns UFP4_OK or UFP4_ERR_DEVICE_TIMEOUT (or UFP4_ERR_CUDA). */
 ufp4_status_t ufp4_check_device_status(void);
+
+/* Test support (no counterpart in the pages): sets the time limit of the
+ * quantizer's producer-side wait for a free pipeline stage, in ns, for the
+ * current device; 0 restores the default (2 s).  A limit far below one
+ * stage's compute time makes that wait give up during a call: the kernel
+ * stops issuing loads, lets every issued load land (the drain keeps its
+ * normal bound), unwinds, and the next ufp4_check_device_status() reports
+ * UFP4_ERR_DEVICE_TIMEOUT once.  Outputs of such a call are incomplete.
+ * Synchronous; not for concurrent use with quantize calls.  Errors: CUDA. */
+ufp4_status_t ufp4_test_set_quantize_wait_limit(uint64_t limit_ns);
 
 /* Human-readable name of a status code (static string). */
 const char *ufp4_status_string(ufp4_status_t status);

@@ -226,11 +226,10 @@ def test_two_level_gemm_path_selector(L):
     """The path setting is host state: it round-trips and rejects unknown values."""
     old = ufp4.get_two_level_gemm_path()
     try:
-        for p in (ufp4.GEMM_PATH_NATIVE_FP4, ufp4.GEMM_PATH_FP16, ufp4.GEMM_PATH_FP16_PAIR,
-                  ufp4.GEMM_PATH_NATIVE_FP4_PAIR, ufp4.GEMM_PATH_NATIVE_FP4_PAIR256, ufp4.GEMM_PATH_AUTO):
+        for p in (ufp4.GEMM_PATH_NATIVE_FP4, ufp4.GEMM_PATH_NATIVE_FP4_PAIR256, ufp4.GEMM_PATH_AUTO):
             ufp4.set_two_level_gemm_path(p)
             assert ufp4.get_two_level_gemm_path() == p
-        for bad in (-1, 6, 99):
+        for bad in (-1, 1, 2, 4, 6, 99):   # 1, 2, 4: removed kernel families
             with pytest.raises(ufp4.UFP4Error):
                 ufp4.set_two_level_gemm_path(bad)
         assert ufp4.get_two_level_gemm_path() == ufp4.GEMM_PATH_AUTO

@@ -161,8 +161,7 @@ def test_large_config_sampled(gemm, fmt, grid):
              block=32 if fmt == ufp4.SCALE_UE8M0 else 16)
 
 
-@pytest.mark.parametrize("path", [ufp4.GEMM_PATH_NATIVE_FP4, ufp4.GEMM_PATH_NATIVE_FP4_PAIR, ufp4.GEMM_PATH_NATIVE_FP4_PAIR256,
-                                  ufp4.GEMM_PATH_FP16])
+@pytest.mark.parametrize("path", [ufp4.GEMM_PATH_NATIVE_FP4, ufp4.GEMM_PATH_NATIVE_FP4_PAIR256])
 @pytest.mark.parametrize("corr", [True, False])
 @pytest.mark.parametrize("grid", [ufp4.GRID_E1M2, ufp4.GRID_E2M1, ufp4.GRID_E2M1_MAX2])
 def test_two_level_kernel_families(path, corr, grid):
