@@ -133,7 +133,12 @@ __device__ int64_t total_tiles(const GemmArgs &a) {
     return t;
 }
 
-// Tile t of the concatenated schedule (groups in order, M fastest inside).
+// Tile t of the concatenated schedule (groups in order).  Inside a problem
+// the M tiles go in bands of a.band rows of tiles, each band swept across all
+// of N with M fastest inside it: the tiles in flight at once (one per SM or
+// SM pair) then share a few operand panels in L2, and a panel is read from
+// HBM about once per band instead of once per column of tiles.  In a step
+// that runs at the power cap the saved DRAM traffic is clock headroom.
 template <int TM, int TN>
 __device__ Tile get_tile(const GemmArgs &a, int64_t t) {
     const int ng = a.groups == nullptr ? 1 : a.num_groups;
@@ -143,9 +148,17 @@ __device__ Tile get_tile(const GemmArgs &a, int64_t t) {
         const int64_t nt = tiles_of<TM, TN>(g);
         if (t < nt) {
             const int64_t mt = (g.m + TM - 1) / TM;
+            int64_t mi = t % mt, ni = t / mt;
+            if (a.band > 0 && mt > a.band) {
+                const int64_t per = static_cast<int64_t>(a.band) * (nt / mt);   // tiles of a full band
+                const int64_t b = t / per, r = t - b * per;
+                const int64_t h = min(static_cast<int64_t>(a.band), mt - b * a.band);   // rows of tiles in band b
+                mi = b * a.band + r % h;
+                ni = r / h;
+            }
             tl.g = g;
-            tl.m0 = (t % mt) * TM;
-            tl.n0 = (t / mt) * TN;
+            tl.m0 = mi * TM;
+            tl.n0 = ni * TN;
             tl.nks = static_cast<int>(g.k / BK);
             return tl;
         }

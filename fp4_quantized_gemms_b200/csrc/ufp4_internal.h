@@ -118,10 +118,12 @@ struct GemmArgs {
     int c_tma;                            // tm_c valid: single problem, c_vec, c_col == 0
     CUtensorMap tm_a_atoms, tm_b_atoms;   // factor atoms as u64 [row groups][64 atoms_k]
     int atoms;                            // both operands carry factor atoms (pair kernels, dense)
+    int band;                             // tile order: rows of tiles per band (0: M fastest)
 };
 
 // Tile columns (B rows) of the native block-scaled FP4 kernels (modes 3, 4).
 constexpr int kNativeTileN = 192;
+constexpr int kTileBand = 8;   // rows of output tiles per band of the GEMM tile order
 
 // mode 0: fp32 block scales (per-block partial products, CUDA-core scaling)
 // mode 1: E4M3 x fp32 two-level scales (scales folded into fp16 operands)

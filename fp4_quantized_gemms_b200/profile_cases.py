@@ -5,6 +5,8 @@ the launch to capture.
 
     python -m fp4_quantized_gemms_b200.profile_cases gemm --m 4096 --n 4096 --k 2048 --grid e1m2
     python -m fp4_quantized_gemms_b200.profile_cases gemm --m 4096 --n 8192 --k 8192 --mx
+    python -m fp4_quantized_gemms_b200.profile_cases gemm --m 4096 --n 4096 --k 2048 --fp32-scales
+    python -m fp4_quantized_gemms_b200.profile_cases grouped --tokens 4096
     python -m fp4_quantized_gemms_b200.profile_cases quantize --rows 8192 --cols 8192 --axis rows --sr
     python -m fp4_quantized_gemms_b200.profile_cases quantize --rows 8192 --cols 2048 --dual
     python -m fp4_quantized_gemms_b200.profile_cases stats --rows 8192 --cols 8192 --axis rows
@@ -24,12 +26,14 @@ def _dev(bits: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
-def gemm_case(m: int, n: int, k: int, grid: int, path: int, mx: bool = False) -> None:
+def gemm_case(m: int, n: int, k: int, grid: int, path: int, mx: bool = False, fp32: bool = False) -> None:
     """Quantize X [m, k] and W [n, k] (RHT16; two-level scales with block 16,
-    or with `mx` UE8M0 scales with block 32 and the E4M3 element planes),
-    then run the FPROP GEMM twice."""
+    or with `mx` UE8M0 scales with block 32 and the E4M3 element planes, or
+    with `fp32` fp32 scales with block 16), then run the FPROP GEMM twice."""
     if mx:
         cfg = ufp4.QuantConfig(grid=grid, hadamard_n=16, block=32, scale_fmt=ufp4.SCALE_UE8M0)
+    elif fp32:
+        cfg = ufp4.QuantConfig(grid=grid, hadamard_n=16, block=16, scale_fmt=ufp4.SCALE_FP32)
     else:
         cfg = ufp4.QuantConfig(grid=grid, hadamard_n=16, block=16, scale_fmt=ufp4.SCALE_E4M3_X_FP32)
     qx = ufp4.rht_quantize(_dev(wl.normal(m, k, 1.0, 1)), ufp4.ALONG_COLS, cfg)
@@ -38,6 +42,31 @@ def gemm_case(m: int, n: int, k: int, grid: int, path: int, mx: bool = False) ->
     out = torch.empty((m, n), dtype=torch.float32, device="cuda")
     for _ in range(2):
         ufp4.gemm_fprop(qx, qw, out)
+    torch.cuda.synchronize()
+    if ufp4.check_device_status() != ufp4.OK:
+        raise RuntimeError("device error word set")
+
+
+def grouped_case(tokens: int, experts: int, hidden: int, ffn: int) -> None:
+    """The gate/up FPROP of a mixture-of-experts layer: tokens x top-6 routed
+    rows in Zipf(1.2) expert segments (zero-padded to 64 rows), two-level
+    scales, one grouped GEMM over the device group table, twice."""
+    shp = wl.MoEShape(tokens=tokens, hidden=hidden, ffn=ffn, experts=experts, topk=6, zipf_s=1.2)
+    counts = wl.moe_expert_counts(shp)
+    starts, _, total = wl.padded_offsets(counts, 64)
+    x = wl.normal(total, hidden, 1.0, 1)
+    mask = np.zeros(total, dtype=bool)
+    for s0, c in zip(starts, counts):
+        mask[s0:s0 + c] = True
+    x[~mask] = 0
+    cfg = ufp4.QuantConfig(grid=ufp4.GRID_E1M2, hadamard_n=16, block=16, scale_fmt=ufp4.SCALE_E4M3_X_FP32)
+    qx = ufp4.rht_quantize(_dev(x), ufp4.ALONG_COLS, cfg)
+    qw = ufp4.rht_quantize(_dev(wl.normal(experts * 2 * ffn, hidden, 0.02, 2)), ufp4.ALONG_COLS, cfg)
+    groups = [(counts[e], 2 * ffn, hidden, starts[e], 0, e * 2 * ffn, 0, starts[e], 0) for e in range(experts)]
+    g = torch.tensor(np.array(groups, dtype=np.int64), device="cuda")
+    out = torch.empty((total, 2 * ffn), dtype=torch.float32, device="cuda")
+    for _ in range(2):
+        ufp4.grouped_gemm(qx, qw, g, out)
     torch.cuda.synchronize()
     if ufp4.check_device_status() != ufp4.OK:
         raise RuntimeError("device error word set")
@@ -85,6 +114,12 @@ def main() -> None:
     g.add_argument("--grid", choices=["e1m2", "e2m1"], default="e1m2")
     g.add_argument("--path", type=int, default=ufp4.GEMM_PATH_AUTO)
     g.add_argument("--mx", action="store_true", help="UE8M0 block-32 scales (the MX path)")
+    g.add_argument("--fp32-scales", action="store_true", help="fp32 block-16 scales (the fp32-scale kernel)")
+    m = sub.add_parser("grouped")
+    m.add_argument("--tokens", type=int, default=4096)
+    m.add_argument("--experts", type=int, default=64)
+    m.add_argument("--hidden", type=int, default=2048)
+    m.add_argument("--ffn", type=int, default=1408)
     q = sub.add_parser("quantize")
     q.add_argument("--rows", type=int, default=8192)
     q.add_argument("--cols", type=int, default=8192)
@@ -98,7 +133,10 @@ def main() -> None:
     t.add_argument("--axis", choices=["cols", "rows"], default="rows")
     a = ap.parse_args()
     if a.case == "gemm":
-        gemm_case(a.m, a.n, a.k, ufp4.GRID_E1M2 if a.grid == "e1m2" else ufp4.GRID_E2M1, a.path, a.mx)
+        gemm_case(a.m, a.n, a.k, ufp4.GRID_E1M2 if a.grid == "e1m2" else ufp4.GRID_E2M1, a.path, a.mx,
+                  a.fp32_scales)
+    elif a.case == "grouped":
+        grouped_case(a.tokens, a.experts, a.hidden, a.ffn)
     elif a.case == "stats":
         stats_case(a.rows, a.cols, ufp4.ALONG_COLS if a.axis == "cols" else ufp4.ALONG_ROWS)
     else:
