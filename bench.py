@@ -604,6 +604,14 @@ def run_e2e(step: LayerStep, host_inputs, args, device):
             "steps": n}
 
 
+# DRAM bytes (read + write) per launch of the large layer's three GEMMs with
+# two-level E1M2 operands, from one ncu capture of the bench's own launches
+# (dram__bytes_read.sum + dram__bytes_write.sum, a one-pass metric set): the
+# CTA-pair kernel with factor atoms and the banded tile order.  Valid only for
+# that kernel and workload; re-capture when either changes.
+LARGE_E1M2_GEMM_DRAM_BYTES = {"fprop": 3.027e9 + 1.854e9, "dgrad": 5.455e9 + 0.524e9, "wgrad": 4.685e9 + 0.923e9}
+
+
 def gemm_roofline(g_ms, shape, peaks, peak_kind, two: bool, grid: int) -> dict:
     """Roofline of the dominant (slowest) GEMM of a step: useful flops 2MNK
     over its CUDA-event time, against the peak of the MMA kind it runs on."""
@@ -632,8 +640,14 @@ def gemm_roofline(g_ms, shape, peaks, peak_kind, two: bool, grid: int) -> dict:
         r["ceiling_note"] = ("an exact E1M2 product needs four FP4 MMAs per K step (no native uniform-grid "
                              "kind), so its ceiling is the FP4 rate / 4 = the bf16 rate")
         r["issued_fp4_TFLOPs"] = round(4 * tf[dom], 1)
-    r["traffic_note"] = ("null: a full-size launch is outside the ncu capture-size rule and its DRAM "
-                         "bytes do not scale from a small capture (operands are re-read from L2)")
+    name = ("fprop", "dgrad", "wgrad")[dom]
+    if two and grid == 0 and shape is wl.LARGE:
+        r["traffic"] = LARGE_E1M2_GEMM_DRAM_BYTES[name]
+        r["traffic_note"] = ("DRAM bytes read + written per launch from one ncu capture of these launches at "
+                             "full size; algorithmic bytes (operands + output) are 2.30 / 1.03 / 1.61 GB for "
+                             "FPROP / DGRAD / WGRAD")
+    else:
+        r["traffic_note"] = "null: no capture of this kernel at this size"
     return r
 
 
