@@ -452,7 +452,7 @@ def run_f32s(step: LayerStep, peaks: dict, reps: int = 3) -> dict:
     bf16 = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     return {"fprop_ms": round(t_g, 4), "fprop_TFLOPs": round(tf, 1),
             "frac_of_bf16": round(tf / bf16, 4),
-            "kernel": "gemm_f32s_kernel (fp16-expanded codes, K = 16 kind::f16 partials, f32x2 scaled accumulate)"}
+            "kernel": "gemm_f32s_kernel (fp16-expanded codes, K = 16 kind::f16 partials, s_a * s_b * partial accumulated in fp32 registers)"}
 
 
 def run_moe(device, two_level: bool, reps: int = 10):

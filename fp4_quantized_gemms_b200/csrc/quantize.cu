@@ -20,11 +20,12 @@
 //
 // Exactness.  The butterflies are the same fp32 adds in the same stage order
 // as the definition.  Codes come from an fp32 estimate of u / s that is
-// certified: every decision whose estimate lies within 2^-16 grid steps of a
-// boundary (and every block whose step is subnormal or could saturate) sends
-// the thread's 64 elements to the exact path, which decides each element by
-// fma sign tests against exact thresholds, so codes always equal the
-// exact-quotient rule bit for bit.
+// certified: every decision whose estimate lies within 2^-18 grid steps of a
+// boundary (the estimate's error is below 2^-19 steps), and every block whose
+// step is subnormal or could saturate, sends the thread's 64 elements to the
+// exact path, which the warp runs cooperatively and which decides each
+// element by fma sign tests against exact thresholds, so codes always equal
+// the exact-quotient rule bit for bit.
 
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -141,7 +142,7 @@ __device__ __forceinline__ int round_sr(float au, float m1, float b, float inv, 
 
 
 // Reciprocal for the fp32 estimate only (every decision it feeds is either
-// certified by the 2^-16 margin or re-decided exactly): rcp.approx has at
+// certified by the 2^-18 margin or re-decided exactly): rcp.approx has at
 // most 1 ulp error; a subnormal argument flushes to zero and gives +inf,
 // which sends the block to the exact path.
 __device__ __forceinline__ float approx_rcp(float x) {
