@@ -119,14 +119,16 @@ def _cfgs(fmt, grid=0):
 SMALL = wl.MoEShape(tokens=512, hidden=256, ffn=192, experts=8, topk=2, zipf_s=1.2)
 
 
-@pytest.mark.parametrize("fmt", [ufp4.SCALE_FP32, ufp4.SCALE_E4M3_X_FP32])
+@pytest.mark.parametrize("fmt,grid", [(ufp4.SCALE_FP32, ufp4.GRID_E1M2), (ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E1M2),
+                                      (ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E2M1)])
 @pytest.mark.parametrize("name", ["fprop", "dgrad", "wgrad"])
-def test_grouped_small(fmt, name):
-    """8 experts, ragged counts (one expert empty), every group checked."""
+def test_grouped_small(fmt, grid, name):
+    """8 experts, ragged counts (one expert empty), every group checked, for
+    fp32 scales and for two-level scales on both grids."""
     counts = wl.moe_expert_counts(SMALL)
     counts[3] = 0                             # an expert with no tokens
     d = _moe(SMALL, counts)
-    _run_gemm(name, d, _cfgs(fmt), SMALL, range(SMALL.experts), per_group=40)
+    _run_gemm(name, d, _cfgs(fmt, grid), SMALL, range(SMALL.experts), per_group=40)
 
 
 _FULL = {}
