@@ -139,35 +139,62 @@ __device__ int64_t total_tiles(const GemmArgs &a) {
 // SM pair) then share a few operand panels in L2, and a panel is read from
 // HBM about once per band instead of once per column of tiles.  In a step
 // that runs at the power cap the saved DRAM traffic is clock headroom.
+// Tile t (of nt) of one problem g.
+template <int TM, int TN>
+__device__ __forceinline__ Tile tile_in_group(const GemmArgs &a, const GemmGroup &g, int64_t t, int64_t nt) {
+    Tile tl;
+    const int64_t mt = (g.m + TM - 1) / TM;
+    int64_t mi = t % mt, ni = t / mt;
+    if (a.band > 0 && mt > a.band) {
+        const int64_t per = static_cast<int64_t>(a.band) * (nt / mt);   // tiles of a full band
+        const int64_t b = t / per, r = t - b * per;
+        const int64_t h = min(static_cast<int64_t>(a.band), mt - b * a.band);   // rows of tiles in band b
+        mi = b * a.band + r % h;
+        ni = r / h;
+    }
+    tl.g = g;
+    tl.m0 = mi * TM;
+    tl.n0 = ni * TN;
+    tl.nks = static_cast<int>(g.k / BK);
+    return tl;
+}
+
 template <int TM, int TN>
 __device__ Tile get_tile(const GemmArgs &a, int64_t t) {
     const int ng = a.groups == nullptr ? 1 : a.num_groups;
-    Tile tl;
     for (int i = 0; i < ng; ++i) {
         const GemmGroup g = load_group(a, i);
         const int64_t nt = tiles_of<TM, TN>(g);
-        if (t < nt) {
-            const int64_t mt = (g.m + TM - 1) / TM;
-            int64_t mi = t % mt, ni = t / mt;
-            if (a.band > 0 && mt > a.band) {
-                const int64_t per = static_cast<int64_t>(a.band) * (nt / mt);   // tiles of a full band
-                const int64_t b = t / per, r = t - b * per;
-                const int64_t h = min(static_cast<int64_t>(a.band), mt - b * a.band);   // rows of tiles in band b
-                mi = b * a.band + r % h;
-                ni = r / h;
-            }
-            tl.g = g;
-            tl.m0 = mi * TM;
-            tl.n0 = ni * TN;
-            tl.nks = static_cast<int>(g.k / BK);
-            return tl;
-        }
+        if (t < nt) return tile_in_group<TM, TN>(a, g, t, nt);
         t -= nt;
     }
+    Tile tl;
     tl.g = a.single;
     tl.m0 = tl.n0 = 0;
     tl.nks = 0;
     return tl;
+}
+
+// A grouped schedule precomputed in shared memory: order[r] is the group
+// scheduled r-th and cum[r] the number of tiles of the groups before it
+// (cum[ng] = all tiles).  Tile t is found by binary search.
+struct GroupSchedule {
+    const uint16_t *order;
+    const int64_t *cum;
+    int ng;
+};
+
+template <int TM, int TN>
+__device__ Tile get_tile(const GemmArgs &a, int64_t t, const GroupSchedule &gs) {
+    if (gs.order == nullptr) return get_tile<TM, TN>(a, t);
+    int lo = 0, hi = gs.ng;              // largest r with cum[r] <= t
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (gs.cum[mid] <= t) lo = mid;
+        else hi = mid;
+    }
+    const GemmGroup g = load_group(a, gs.order[lo]);
+    return tile_in_group<TM, TN>(a, g, t - gs.cum[lo], gs.cum[lo + 1] - gs.cum[lo]);
 }
 
 // ---------------------------------------------------------------------------
@@ -1153,7 +1180,10 @@ struct PairCfg {
     // acc_empty, drain
     static constexpr int kNumBars = 5 * NS + 3;
     static constexpr int o_misc = o_bar + kNumBars * 8;
-    static constexpr int kAlloc = o_misc + 64 + 1024;
+    static constexpr int kMaxOrder = 256;           // grouped problems: a schedule of up to 256 groups
+    static constexpr int o_cum = o_misc + 64;       // int64 [kMaxOrder + 1]
+    static constexpr int o_order = o_cum + 8 * (kMaxOrder + 1);   // u16 [kMaxOrder]
+    static constexpr int kAlloc = o_order + 2 * kMaxOrder + 1024;
     static constexpr int kThreads = 32 * 12;
     static_assert(NS >= 4, "pipeline depth");
     static_assert(kAlloc <= 232448, "shared memory budget");
@@ -1273,11 +1303,39 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
         tma_prefetch_desc(ATOMS ? &args.tm_b_atoms : &args.tm_b_scales);
     }
     if (warp == 1) tmem_alloc_pair(tmem_slot, 512);
+    // Grouped problems: the schedule goes group by group in decreasing K
+    // (ties by index), so the longest tiles start first and the persistent
+    // CTA pairs finish together (ragged K per group, as in an expert WGRAD),
+    // and the tile -> group lookup is a binary search over prefix counts in
+    // shared memory.  Every CTA builds the same schedule: group g's rank
+    // counts the groups scheduled before it.
+    uint16_t *order_s = reinterpret_cast<uint16_t *>(smem + C::o_order);
+    int64_t *cum_s = reinterpret_cast<int64_t *>(smem + C::o_cum);
+    const bool scheduled = args.groups != nullptr && args.num_groups <= C::kMaxOrder;
+    if (scheduled) {
+        if (static_cast<int>(threadIdx.x) < args.num_groups) {
+            const int gi = threadIdx.x;
+            const GemmGroup g = load_group(args, gi);
+            int rankv = 0;
+            for (int j = 0; j < args.num_groups; ++j) {
+                const int64_t kj = load_group(args, j).k;
+                rankv += (kj > g.k || (kj == g.k && j < gi)) ? 1 : 0;
+            }
+            order_s[rankv] = static_cast<uint16_t>(gi);
+            cum_s[rankv + 1] = tiles_of<TM, BN>(g);      // tiles of the rank-th group, summed below
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            cum_s[0] = 0;
+            for (int r = 1; r <= args.num_groups; ++r) cum_s[r] += cum_s[r - 1];
+        }
+    }
+    const GroupSchedule sched{scheduled ? order_s : nullptr, cum_s, args.num_groups};
     tc_fence_before();
     cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int64_t ntiles = total_tiles<TM, BN>(args);
+    const int64_t ntiles = scheduled ? cum_s[args.num_groups] : total_tiles<TM, BN>(args);
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -1286,7 +1344,7 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int64_t t = unit; t < ntiles && ok; t += nunits) {
-                const Tile tl = get_tile<TM, BN>(args, t);
+                const Tile tl = get_tile<TM, BN>(args, t, sched);
                 const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
                 const int32_t arow = static_cast<int32_t>(tl.g.a_row + tl.m0 + 128 * rank);
                 const int32_t brow = static_cast<int32_t>(tl.g.b_row + tl.n0);
@@ -1351,7 +1409,7 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
             uint32_t it = 0, tcount = 0;
             bool ok = true;
             for (int64_t t = unit; t < ntiles && ok; t += nunits, ++tcount) {
-                const Tile tl = get_tile<TM, BN>(args, t);
+                const Tile tl = get_tile<TM, BN>(args, t, sched);
                 const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
                 if (!mbar_wait_cluster(acc_empty, (tcount & 1) ^ 1, kErrTimeoutMma, abort_flag)) break;
                 tc_fence_after();
@@ -1426,7 +1484,7 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int64_t t = unit; t < ntiles && ok; t += nunits) {
-                const Tile tl = get_tile<TM, BN>(args, t);
+                const Tile tl = get_tile<TM, BN>(args, t, sched);
                 const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
                 for (int ks = 0; ks < nks; ++ks, ++it) {
                     const int s = it % NS;
@@ -1447,7 +1505,7 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
         uint32_t it = 0;
         bool ok = true;
         for (int64_t t = unit; t < ntiles && ok; t += nunits) {
-            const Tile tl = get_tile<TM, BN>(args, t);
+            const Tile tl = get_tile<TM, BN>(args, t, sched);
             const int nks = static_cast<int>((tl.g.k + C::BKE - 1) / C::BKE);
             for (int ks = 0; ks < nks; ++ks, ++it) {
                 const int s = it % NS;
@@ -1525,7 +1583,7 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
                                               args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f));
         uint32_t tcount = 0, piece = 0;
         for (int64_t t = unit; t < ntiles; t += nunits, ++tcount) {
-            const Tile tl = get_tile<TM, BN>(args, t);
+            const Tile tl = get_tile<TM, BN>(args, t, sched);
             const bool ok = warp_wait(acc_full, tcount & 1, kErrTimeoutEpilogue, abort_flag);
             if (named_bar_or(1, kEpiThreads, !ok)) break;
             tc_fence_after();
