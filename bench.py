@@ -179,26 +179,29 @@ class LayerStep:
         self.qwt = E(s.K, s.N, self.c_rtne, device)       # DGRAD B
         self.qdyt = E(s.N, s.M, self.c_sr1, device)       # WGRAD A
         self.qxt = E(s.K, s.M, self.c_rtne, device)       # WGRAD B
-        # Each tensor feeds two GEMMs, one along each axis.  X and W go
-        # through the dual-output quantizer (one read, both results); dY
-        # through one call per axis.  The rotated amaxes of all six operands
-        # come from one dual pass per tensor.
-        self.dual = [(self.X, self.qx, self.qxt), (self.W, self.qw, self.qwt)]
-        self.single = [(self.dY, C, self.qdy), (self.dY, R, self.qdyt)]
+        # Each tensor feeds two GEMMs, one along each axis: one quantization
+        # call per operand (two single-output calls measured faster than the
+        # dual-output pass at these sizes).  The rotated amaxes of all six
+        # operands come from one dual amax pass per tensor.
+        self.ops = self._ops()
         self.amax = torch.zeros(6, dtype=torch.float32, device=device)   # [cols, rows] per tensor
         self.Y = torch.empty((s.M, s.N), dtype=torch.float32, device=device)
         self.dX = torch.empty((s.M, s.K), dtype=torch.float32, device=device)
         self.dW = torch.empty((s.N, s.K), dtype=torch.float32, device=device)
-        self.launches = (3 if two else 0) + len(self.dual) + len(self.single) + 3
+        self.launches = (3 if two else 0) + len(self.ops) + 3
         self.tensor_elems = self.X.numel() + self.W.numel() + self.dY.numel()
         self.quant_elems = 2 * self.tensor_elems         # elements quantized per step
 
+    def _ops(self):
+        """(input, axis, output, amax slot) of the six quantizations."""
+        C, R = self.u.ALONG_COLS, self.u.ALONG_ROWS
+        return [(self.X, C, self.qx, 0), (self.X, R, self.qxt, 1), (self.W, C, self.qw, 2),
+                (self.W, R, self.qwt, 3), (self.dY, C, self.qdy, 4), (self.dY, R, self.qdyt, 5)]
+
     def bind(self, X, W, dY, Y, dX, dW):
         """Point the step at other input / output buffers of the same shapes."""
-        C, R = self.u.ALONG_COLS, self.u.ALONG_ROWS
         self.X, self.W, self.dY, self.Y, self.dX, self.dW = X, W, dY, Y, dX, dW
-        self.dual = [(self.X, self.qx, self.qxt), (self.W, self.qw, self.qwt)]
-        self.single = [(self.dY, C, self.qdy), (self.dY, R, self.qdyt)]
+        self.ops = self._ops()
 
     def quantize_all(self):
         u = self.u
@@ -206,11 +209,8 @@ class LayerStep:
         if self.two:
             for i, x in enumerate((self.X, self.W, self.dY)):
                 u.rht_amax_dual(x, 16, sm, out=self.amax[2 * i:2 * i + 2])
-        for i, (x, qc, qr) in enumerate(self.dual):
-            am = self.amax[2 * i:2 * i + 2] if self.two else None
-            u.rht_quantize_dual(x, qc.cfg, qr.cfg, tensor_amax=am, out=(qc, qr))
-        for j, (x, axis, q) in enumerate(self.single):
-            am = self.amax[4 + j:5 + j] if self.two else None
+        for x, axis, q, slot in self.ops:
+            am = self.amax[slot:slot + 1] if self.two else None
             u.rht_quantize(x, axis, q.cfg, tensor_amax=am, out=q)
 
     def gemms(self, events=None):
@@ -240,14 +240,13 @@ class LayerStep:
 
 def quant_bytes(step: LayerStep) -> float:
     """Algorithmic bytes of the step's quantization: each quantized element
-    writes its code and its share of a block scale (fp32, or E4M3); bf16 inputs
-    are read once per dual call and once per single call; with two-level
-    scales the dual amax pass reads each tensor once more.  The E1M2
-    correction planes the GEMM reads are not counted."""
+    writes its code and its share of a block scale (fp32, or E4M3); every
+    quantization call reads its bf16 input once; with two-level scales the
+    dual amax pass reads each tensor once more.  The E1M2 correction planes
+    the GEMM reads are not counted."""
     out_per = 0.5 + (4 / 16 if not step.two else 1 / 16)
     total = step.quant_elems * out_per
-    total += sum(x.numel() for x, _, _ in step.dual) * 2
-    total += sum(x.numel() for x, _, _ in step.single) * 2
+    total += sum(x.numel() for x, _, _, _ in step.ops) * 2
     if step.two:
         total += step.tensor_elems * 2
     return total

@@ -18,7 +18,7 @@ BUILD_DIR = os.path.join(PKG, "_build")
 SOURCES = ["api.cu", "quantize.cu", "gemm.cu", "diag.cu"]
 NVCC = os.environ.get("NVCC", "nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-split-compile=0", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", f"-I{INCLUDE}", f"-I{CSRC}"]
 
 

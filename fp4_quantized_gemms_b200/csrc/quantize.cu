@@ -6,13 +6,12 @@
 // gist.science "Efficiëntie" (RHT fused with the quantizer).
 //
 // Work decomposition.  A persistent CTA (8 compute warps + one TMA producer
-// warp) takes units of 256 output rows x 64 K elements whose bf16 tile a TMA
-// copy stages in shared memory (128-byte swizzle, 3-stage ring).  Every
-// compute thread quantizes 64 elements of a unit as 32 "entries", each a pair
-// of fp32 values held as the two lanes of an fp32x2 register: lane x and lane
-// y are two 32-long runs along K that share their D signs position by
-// position, so the butterflies, the rounding estimate and the packing run two
-// elements per instruction:
+// warp) takes units of 256 output rows x 64 K elements whose bf16 tile a TMA copy stages in shared memory (3-stage
+// ring).  Every compute thread quantizes 64 elements of a unit as 32
+// "entries", each a pair of fp32 values held as the two lanes of an fp32x2
+// register: lane x and lane y are two 32-long runs along K that share their
+// D signs position by position, so the butterflies, the rounding estimate and
+// the packing run two elements per instruction:
 //   row map   (K contiguous)  one output row, K [0, 32) in x, [32, 64) in y;
 //   col2 map  (K strided, n <= 32)  two adjacent output rows (input columns
 //             c, c + 1: one 32-bit shared load gives both), 32 K each;
@@ -298,9 +297,17 @@ __device__ __forceinline__ GridK grid_constants(int grid) {
     return GridK{2.0f, 2.0f, 4.0f, 1.0f, 1};                    // E2M1, max_fpx 2: k / 2
 }
 
-// block_scale with the grid taken at run time: the same operations as the
-// templated version, so the stored scales and steps are identical.
-__device__ __forceinline__ ScaleOut block_scale_rt(float amax, int scale_fmt, float S, float G, const GridK &gk) {
+// block_scale with the grid taken at run time: the same stored scales and
+// steps as the templated version.  For two-level scales the quotient amax / G
+// comes from rG = RN(1 / G) (one product, within 2 ulp of the exact quotient,
+// 2.5 ulp of its rounding) instead of a division; the E4M3 byte depends only
+// on the side of the quotient's rounding midpoints (fraction bits below the
+// third = 1000...0) it falls on, so a product within 4 ulp of a midpoint, or
+// below the smallest normal E4M3 value (2^-6, where the midpoints are spaced
+// differently), sets `risky` and the exact path decides the block (so does
+// a NaN product, e.g. amax = 0 times an infinite rG).
+__device__ __forceinline__ ScaleOut block_scale_rt(float amax, int scale_fmt, float S, float G, float rG,
+                                                   const GridK &gk, bool &risky) {
     ScaleOut o;
     if (scale_fmt == 2) {
         int X = -127;
@@ -325,7 +332,8 @@ __device__ __forceinline__ ScaleOut block_scale_rt(float amax, int scale_fmt, fl
         o.inv = o.zero ? 0.0f : approx_rcp(s);
         o.stored = __float_as_uint(s);
     } else {
-        const float q = __fdiv_rn(amax, G);
+        const float q = __fmul_rn(amax, rG);
+        risky |= (__float_as_uint(q) & 0xFFFFFu) - 0x7FFFCu < 9u || !(q >= 0.015625f || q == 0.0f);
         const __nv_fp8_storage_t e8 = __nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3);
         const float e = e4m3_to_f32(e8);
         o.m1 = e;
@@ -340,13 +348,12 @@ __device__ __forceinline__ ScaleOut block_scale_rt(float amax, int scale_fmt, fl
 // ---------------------------------------------------------------------------
 // Work unit and thread maps.
 constexpr int kComputeWarps = 8;
-constexpr int kThreads = kComputeWarps * 32;
-constexpr int kCtaThreads = kThreads + 32;        // + one producer warp
 constexpr int kUnitRows = 256;
 constexpr int kStageBytes = kUnitRows * 64 * 2;   // 32 KB of bf16
 constexpr int kStages = 3;
 constexpr int kCtasPerSm = 2;
-constexpr int kQuantSmem = kStages * kStageBytes + 1024 + 128;
+constexpr int kCtaThreads = 32 * (kComputeWarps + 1);   // + one producer warp
+constexpr int kQuantSmem = kStages * kStageBytes + 8 * 2 * kStages + 16 + 1024;   // + barriers, abort word, alignment
 
 enum { MAP_ROW = 0, MAP_COL2 = 1, MAP_COL1 = 2 };
 
@@ -362,7 +369,9 @@ struct Src {
 };
 
 // Output rows and first output column of the lane-x and lane-y runs
-// (callers validate rows and kpad below 2^31).
+// (callers validate rows and kpad below 2^31).  Either row_y = row_x and
+// k_y = k_x + 32 (row and col1 maps) or row_y = row_x + 1 and k_y = k_x
+// (col2 map).
 struct Site {
     int32_t row_x, row_y, k_x, k_y;
 };
@@ -435,20 +444,23 @@ __device__ __forceinline__ void rht_entries(float2 (&v)[ENT]) {
     }
 }
 
-// Block amaxes of both lanes: am[b] lane x, am[NB + b] lane y.
+// Block amaxes of both lanes: am[b] lane x, am[NB + b] lane y (two partial
+// maxima per lane: shorter dependency chains).
 template <int BLK, int ENT>
 __device__ __forceinline__ void block_amax(const float2 (&v)[ENT], float (&am)[2 * ENT / BLK]) {
     constexpr int NB = ENT / BLK;
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-        float mx = 0.0f, my = 0.0f;
+        float mx0 = 0.0f, my0 = 0.0f, mx1 = 0.0f, my1 = 0.0f;
 #pragma unroll
-        for (int i = b * BLK; i < (b + 1) * BLK; i += 2) {
-            mx = max3(mx, fabsf(v[i].x), fabsf(v[i + 1].x));
-            my = max3(my, fabsf(v[i].y), fabsf(v[i + 1].y));
+        for (int i = b * BLK; i < (b + 1) * BLK; i += 4) {
+            mx0 = max3(mx0, fabsf(v[i].x), fabsf(v[i + 1].x));
+            my0 = max3(my0, fabsf(v[i].y), fabsf(v[i + 1].y));
+            mx1 = max3(mx1, fabsf(v[i + 2].x), fabsf(v[i + 3].x));
+            my1 = max3(my1, fabsf(v[i + 2].y), fabsf(v[i + 3].y));
         }
-        am[b] = mx;
-        am[NB + b] = my;
+        am[b] = fmaxf(mx0, mx1);
+        am[NB + b] = fmaxf(my0, my1);
     }
 }
 
@@ -640,24 +652,26 @@ constexpr float kE2m1Eps = 1.0f / 1048576.0f;
 constexpr float kPackBase = 8423560.0f;
 
 // One thread's 64 elements: load, rotate, block scales, certified fast
-// rounding, packing, stores (or the exact path).  GRID 0 = the uniform grids
-// (E1M2, restricted E2M1; a.grid picks the constants), GRID 1 = E2M1.
+// rounding and packing into cw (codes: lane x words 0..3, lane y words 4..7)
+// and st (stored scales: lane x, then lane y).  Returns whether a decision
+// is not certified (the warp then decides the thread's elements again on the
+// exact path).  GRID 0 = the uniform grids (E1M2, restricted E2M1; a.grid
+// picks the constants), GRID 1 = E2M1.
 template <int MAP, bool SWZ, int NH, int BLK, int GRID, int RND>
 __device__ __forceinline__ bool quant_thread(const QuantArgs &a, const Src &src, const Site &site, float S,
-                                             float G, const GridK &gk) {
+                                             float G, float rG, const GridK &gk, uint32_t (&cw)[8],
+                                             uint32_t (&st)[64 / BLK]) {
     constexpr int ENT = ent_of<NH, BLK>();
     constexpr int NBP = ENT / BLK;          // blocks per lane in a pass
     constexpr int NB = 32 / BLK;            // blocks per lane run
-    uint32_t cw[8];                         // codes: lane x words 0..3, lane y words 4..7
-    uint32_t st[2 * NB];                    // stored scales: lane x, then lane y
     bool risky = (GRID == 1 && RND == 1);   // E2M1 SR: exact path
-    uint64_t gx = 0, gy = 0;
-    if (RND == 1 && GRID == 0) {
+    // Philox counter of the runs' first 8 elements; lane y's is a fixed
+    // distance away (the next 32 K of the row, or the next row).
+    uint64_t gx = 0;
+    if (RND == 1 && GRID == 0)
         gx = (static_cast<uint64_t>(site.row_x) * static_cast<uint64_t>(a.kpad) +
               static_cast<uint64_t>(site.k_x)) >> 3;
-        gy = (static_cast<uint64_t>(site.row_y) * static_cast<uint64_t>(a.kpad) +
-              static_cast<uint64_t>(site.k_y)) >> 3;
-    }
+    const uint64_t dgy = MAP == MAP_COL2 ? static_cast<uint64_t>(a.kpad) >> 3 : 4u;
 #pragma unroll
     for (int p = 0; p < 32 / ENT; ++p) {
         float2 v[ENT];
@@ -669,7 +683,7 @@ __device__ __forceinline__ bool quant_thread(const QuantArgs &a, const Src &src,
         float inv[2 * NBP];
 #pragma unroll
         for (int j = 0; j < 2 * NBP; ++j) {
-            const ScaleOut sc = block_scale_rt(am[j], a.scale_fmt, S, G, gk);
+            const ScaleOut sc = block_scale_rt(am[j], a.scale_fmt, S, G, rG, gk, risky);
             st[(j / NBP) * NB + p * NBP + (j % NBP)] = sc.stored;
             const float iv = sc.zero ? 0.0f : (GRID == 1 ? sc.inv : sc.inv * gk.unit);
             inv[j] = iv;
@@ -716,12 +730,16 @@ __device__ __forceinline__ bool quant_thread(const QuantArgs &a, const Src &src,
             float2 acc[ENT / 4];
 #pragma unroll
             for (int j = 0; j < ENT / 4; ++j) acc[j] = make_float2(kPackBase, kPackBase);
-            float dev = 0.0f;
+            // Distance maximum: two chains for RTNE (shorter dependency
+            // chain); one for SR, whose Philox words already crowd the
+            // register file.
+            constexpr int NDEV = RND == 0 ? 2 : 1;
+            float dev[2] = {0.0f, 0.0f};
 #pragma unroll
             for (int j = 0; j < ENT / 8; ++j) {
                 uint4 rx = make_uint4(0u, 0u, 0u, 0u), ry = rx;
                 if (RND == 1) {
-                    const uint64_t cx = gx + p * (ENT / 8) + j, cy = gy + p * (ENT / 8) + j;
+                    const uint64_t cx = gx + p * (ENT / 8) + j, cy = cx + dgy;
                     rx = philox4x32_10(make_uint4(static_cast<uint32_t>(cx), static_cast<uint32_t>(cx >> 32),
                                                   a.stream, 0u), a.keys);
                     ry = philox4x32_10(make_uint4(static_cast<uint32_t>(cy), static_cast<uint32_t>(cy >> 32),
@@ -751,12 +769,12 @@ __device__ __forceinline__ bool quant_thread(const QuantArgs &a, const Src &src,
                     const float2 f = __fadd2_rn(t, kR2);
                     const float2 g = __fadd2_rn(f, kRn2);
                     const float2 d = __ffma2_rn(g, m1, t);
-                    dev = max3(dev, fabsf(d.x), fabsf(d.y));
+                    dev[e % NDEV] = max3(dev[e % NDEV], fabsf(d.x), fabsf(d.y));
                     const float wgt = static_cast<float>(1 << (4 * (i & 3)));
                     acc[i >> 2] = __ffma2_rn(g, make_float2(wgt, wgt), acc[i >> 2]);
                 }
             }
-            risky |= dev > 0.5f - kMargin;
+            risky |= fmaxf(dev[0], dev[1]) > 0.5f - kMargin;
 #pragma unroll
             for (int j = 0; j < ENT / 8; ++j) {
                 cw[p * (ENT / 8) + j] = offset_to_sign_magnitude(
@@ -766,10 +784,7 @@ __device__ __forceinline__ bool quant_thread(const QuantArgs &a, const Src &src,
             }
         }
     }
-    if (risky) return true;        // decided again by the warp (coop_exact)
-    store_run<BLK>(a, site.row_x, site.k_x, cw, st);
-    store_run<BLK>(a, site.row_y, site.k_y, cw + 4, st + NB);
-    return false;
+    return risky;
 }
 
 template <int MAP, bool SWZ, int NH>
@@ -789,11 +804,13 @@ __device__ __forceinline__ float amax_thread(const QuantArgs &a, const Src &src)
 }
 
 // Two-level tensor scale of one output: S maps the rotated tensor amax to
-// gmax * 448 (the top of E4M3), G = gmax * S is the block-scale divisor.
-__device__ __forceinline__ void tensor_scale(const QuantArgs &q, const GridK &gk, float &S, float &G) {
+// gmax * 448 (the top of E4M3), G = gmax * S is the block-scale divisor and
+// rG = RN(1 / G) its reciprocal for the certified quotient estimate.
+__device__ __forceinline__ void tensor_scale(const QuantArgs &q, const GridK &gk, float &S, float &G, float &rG) {
     const float amax_t = *q.amax_t;
     S = amax_t > 0.0f ? __fdiv_rn(amax_t, gk.gmax * 448.0f) : 1.0f;
     G = __fmul_rn(gk.gmax, S);
+    rG = __frcp_rn(G);
     if (blockIdx.x == 0 && threadIdx.x == 0 && q.S_out) *q.S_out = S;
 }
 
@@ -802,11 +819,16 @@ __device__ __forceinline__ void tensor_scale(const QuantArgs &q, const GridK &gk
 // are decided again by the whole warp.
 template <int MAP, bool SWZ, int NH, int BLK, int GRID, int RND, bool AMAX_ONLY>
 __device__ __forceinline__ void unit_part(const QuantArgs &q, const uint8_t *tile, const Src &src, const Site &site,
-                                          float S, float G, const GridK &gk, float &amax_acc) {
+                                          float S, float G, float rG, const GridK &gk, float &amax_acc) {
     if constexpr (AMAX_ONLY) {
         amax_acc = fmaxf(amax_acc, amax_thread<MAP, SWZ, NH>(q, src));
     } else {
-        const bool risky = quant_thread<MAP, SWZ, NH, BLK, GRID, RND>(q, src, site, S, G, gk);
+        uint32_t cw[8], st[64 / BLK];
+        const bool risky = quant_thread<MAP, SWZ, NH, BLK, GRID, RND>(q, src, site, S, G, rG, gk, cw, st);
+        if (!risky) {
+            store_run<BLK>(q, site.row_x, site.k_x, cw, st);
+            store_run<BLK>(q, site.row_y, site.k_y, cw + 4, st + 32 / BLK);
+        }
         const uint32_t owners = __ballot_sync(0xFFFFFFFFu, risky);
         if (owners != 0u) {
             const uint32_t pofs = static_cast<uint32_t>(src.p - tile);
@@ -829,6 +851,27 @@ __device__ __forceinline__ void unit_part(const QuantArgs &q, const uint8_t *til
 //           column-wise into `a` as AXIS 1, then row-wise into `a2` (thread t
 //           takes row t & 63 of box t >> 6: 64 columns of one input row).
 //           One read of the tensor serves both of its GEMM operands.
+
+// A CTA's walk over a grid of `slow` x `fast` units (fast fastest), visiting
+// units blockIdx.x, blockIdx.x + gridDim.x, ...: advanced without a division.
+struct UnitWalk {
+    int32_t slow, fast, dslow, dfast, nfast;
+    __device__ UnitWalk(uint32_t first, uint32_t step, int32_t nfast_)
+        : slow(static_cast<int32_t>(first / static_cast<uint32_t>(nfast_))),
+          fast(static_cast<int32_t>(first % static_cast<uint32_t>(nfast_))),
+          dslow(static_cast<int32_t>(step / static_cast<uint32_t>(nfast_))),
+          dfast(static_cast<int32_t>(step % static_cast<uint32_t>(nfast_))),
+          nfast(nfast_) {}
+    __device__ __forceinline__ void next() {
+        fast += dfast;
+        slow += dslow;
+        if (fast >= nfast) {
+            fast -= nfast;
+            ++slow;
+        }
+    }
+};
+
 // Limit of the producer's wait for a free stage (ns).  Only test support
 // lowers it, to make that bounded wait run out on purpose; the drain and the
 // compute warps keep the normal bound.
@@ -848,33 +891,28 @@ __global__ void __launch_bounds__(kCtaThreads, kCtasPerSm)
     const int t = threadIdx.x;
     const int lane = t & 31;
     const int warp = t >> 5;
-    const int64_t nseg = a.kpad / 64;
-    const int64_t nrb = (a.out_rows + kUnitRows - 1) / kUnitRows;
-    const int64_t nunits = nseg * nrb;
+    const int32_t nseg = static_cast<int32_t>(a.kpad / 64);
+    const int32_t nrb = static_cast<int32_t>((a.out_rows + kUnitRows - 1) / kUnitRows);
     constexpr bool kSwz = AXIS != 1;
-
-    auto unit_coords = [&](int64_t u, int64_t &rb, int64_t &seg) {
-        if (AXIS == 0) {
-            rb = u / nseg;
-            seg = u % nseg;
-        } else {
-            seg = u / nrb;
-            rb = u % nrb;
-        }
+    // Units in order (row block major for AXIS 0, K segment major otherwise).
+    const UnitWalk walk0(blockIdx.x, gridDim.x, AXIS == 0 ? nseg : nrb);
+    const int32_t nslow = AXIS == 0 ? nrb : nseg;
+    auto coords = [&](const UnitWalk &w, int32_t &rb, int32_t &seg) {
+        rb = AXIS == 0 ? w.slow : w.fast;
+        seg = AXIS == 0 ? w.fast : w.slow;
     };
-    auto issue = [&](int64_t u, int s) {
-        int64_t rb, seg;
-        unit_coords(u, rb, seg);
+
+    auto issue = [&](const UnitWalk &w, int s) {
+        int32_t rb, seg;
+        coords(w, rb, seg);
         uint8_t *dst = smem + s * kStageBytes;
         mbar_arrive_expect_tx(&full[s], kStageBytes);
         if (AXIS == 0) {
-            tma_load_2d(dst, &tmap, &full[s], static_cast<int32_t>(seg * 64),
-                        static_cast<int32_t>(rb * kUnitRows));
+            tma_load_2d(dst, &tmap, &full[s], seg * 64, rb * kUnitRows);
         } else {
 #pragma unroll
             for (int b = 0; b < 4; ++b)
-                tma_load_2d(dst + b * 8192, &tmap, &full[s], static_cast<int32_t>(rb * kUnitRows + 64 * b),
-                            static_cast<int32_t>(seg * 64));
+                tma_load_2d(dst + b * 8192, &tmap, &full[s], rb * kUnitRows + 64 * b, seg * 64);
         }
     };
 
@@ -887,17 +925,16 @@ __global__ void __launch_bounds__(kCtaThreads, kCtasPerSm)
         fence_barrier_init();
     }
     __syncthreads();
-    const int64_t u0 = blockIdx.x;
     if (warp == kComputeWarps) {
         // Producer warp: refills a stage once every compute warp released it.
         if (lane == 0) {
             uint32_t it = 0;
-            for (int64_t u = u0; u < nunits; u += gridDim.x, ++it) {
+            for (UnitWalk w = walk0; w.slow < nslow; w.next(), ++it) {
                 const int s = it % kStages;
                 if (it >= kStages && !mbar_wait(&empty[s], ((it / kStages) - 1) & 1, kErrTimeoutProducer,
                                                 abort_flag, g_producer_wait_limit_ns))
                     break;
-                issue(u, s);
+                issue(w, s);
             }
             // Drain: the last copies have landed before the CTA exits.
             for (uint32_t d = 0; d < kStages && d < it; ++d) {
@@ -909,11 +946,10 @@ __global__ void __launch_bounds__(kCtaThreads, kCtasPerSm)
         }
         return;
     }
-
     const GridK gk = grid_constants(a.grid);
-    float S = 1.0f, G = 0.0f, S2 = 1.0f, G2 = 0.0f;
-    if (!AMAX_ONLY && a.scale_fmt == 1) tensor_scale(a, gk, S, G);
-    if (AXIS == 2 && !AMAX_ONLY && a2.scale_fmt == 1) tensor_scale(a2, gk, S2, G2);
+    float S = 1.0f, G = 0.0f, rG = 0.0f, S2 = 1.0f, G2 = 0.0f, rG2 = 0.0f;
+    if (!AMAX_ONLY && a.scale_fmt == 1) tensor_scale(a, gk, S, G, rG);
+    if (AXIS == 2 && !AMAX_ONLY && a2.scale_fmt == 1) tensor_scale(a2, gk, S2, G2, rG2);
     float amax_acc = 0.0f, amax_acc2 = 0.0f;
 
     // Column maps: byte offsets of the thread's column(s) within a K row r
@@ -930,48 +966,45 @@ __global__ void __launch_bounds__(kCtaThreads, kCtasPerSm)
                            : static_cast<uint32_t>(((((t & 63) >> 3) ^ jj) << 4) + 2 * (t & 7));
     }
     uint32_t it = 0;
-    for (int64_t u = u0; u < nunits; u += gridDim.x, ++it) {
+    for (UnitWalk w = walk0; w.slow < nslow; w.next(), ++it) {
         const int s = it % kStages;
         if (!warp_wait(&full[s], (it / kStages) & 1, kErrTimeoutTransform, abort_flag)) break;
-        int64_t rb, seg;
-        unit_coords(u, rb, seg);
+        int32_t rb, seg;
+        coords(w, rb, seg);
         const uint8_t *tile = smem + s * kStageBytes;
         if (AXIS == 0) {
             Src src;
             src.p = tile + t * 128;
             src.off8[0] = static_cast<uint32_t>(t & 7);
-            const int32_t row = static_cast<int32_t>(rb * kUnitRows + t);
-            const int32_t k0 = static_cast<int32_t>(seg * 64);
+            const int32_t row = rb * kUnitRows + t, k0 = seg * 64;
             const Site site{row, row, k0, k0 + 32};
-            unit_part<MAP_ROW, true, NH, BLK, GRID, RND, AMAX_ONLY>(a, tile, src, site, S, G, gk, amax_acc);
+            unit_part<MAP_ROW, true, NH, BLK, GRID, RND, AMAX_ONLY>(a, tile, src, site, S, G, rG, gk, amax_acc);
         } else {
             Src src = csrc;
             Site site;
             if (CMAP == MAP_COL2) {
                 const int box = warp & 3, half = warp >> 2;
                 src.p = tile + box * 8192 + half * 32 * 128;
-                const int32_t row = static_cast<int32_t>(rb * kUnitRows + 64 * box + 2 * lane);
-                const int32_t k0 = static_cast<int32_t>(seg * 64 + 32 * half);
+                const int32_t row = rb * kUnitRows + 64 * box + 2 * lane, k0 = seg * 64 + 32 * half;
                 site = Site{row, row + 1, k0, k0};
             } else {
                 src.p = tile + (t >> 6) * 8192;
-                const int32_t row = static_cast<int32_t>(rb * kUnitRows + t);
-                const int32_t k0 = static_cast<int32_t>(seg * 64);
+                const int32_t row = rb * kUnitRows + t, k0 = seg * 64;
                 site = Site{row, row, k0, k0 + 32};
             }
-            unit_part<CMAP, kSwz, NH, BLK, GRID, RND, AMAX_ONLY>(a, tile, src, site, S, G, gk, amax_acc);
+            unit_part<CMAP, kSwz, NH, BLK, GRID, RND, AMAX_ONLY>(a, tile, src, site, S, G, rG, gk, amax_acc);
             if (AXIS == 2) {
                 // Row-wise output: input row 64 seg + (t & 63), K columns from
                 // 256 rb + 64 (t >> 6).  Boxes past the padded K (the last
                 // column block of a ragged width) are skipped, per warp.
-                const int64_t k0 = rb * kUnitRows + 64 * (t >> 6);
+                const int64_t k0 = static_cast<int64_t>(rb) * kUnitRows + 64 * (t >> 6);
                 if (k0 < a2.kpad) {
                     Src rs;
                     rs.p = tile + (t >> 6) * 8192 + (t & 63) * 128;
                     rs.off8[0] = static_cast<uint32_t>(t & 7);
-                    const int32_t row = static_cast<int32_t>(seg * 64 + (t & 63));
+                    const int32_t row = seg * 64 + (t & 63);
                     const Site rsite{row, row, static_cast<int32_t>(k0), static_cast<int32_t>(k0 + 32)};
-                    unit_part<MAP_ROW, true, NH, BLK, GRID, RND, AMAX_ONLY>(a2, tile, rs, rsite, S2, G2, gk,
+                    unit_part<MAP_ROW, true, NH, BLK, GRID, RND, AMAX_ONLY>(a2, tile, rs, rsite, S2, G2, rG2, gk,
                                                                              amax_acc2);
                 }
             }
@@ -1072,7 +1105,8 @@ cudaError_t launch_one(const QuantArgs &a, const QuantArgs &a2, const CUtensorMa
     const int64_t cap = static_cast<int64_t>(num_sms) * kCtasPerSm;
     const int grid = static_cast<int>(nunits < cap ? nunits : cap);
     if (grid <= 0) return cudaSuccess;
-    rht_quantize_kernel<AXIS, NH, BLK, GRID, RND, AMAX_ONLY><<<grid, kCtaThreads, kQuantSmem, stream>>>(a, a2, tmap);
+    rht_quantize_kernel<AXIS, NH, BLK, GRID, RND, AMAX_ONLY>
+        <<<grid, kCtaThreads, kQuantSmem, stream>>>(a, a2, tmap);
     return cudaGetLastError();
 }
 
