@@ -251,7 +251,7 @@ __device__ __forceinline__ float ue8m0_to_f32(uint32_t e) {
     return __uint_as_float(e ? (e << 23) : 0x00400000u);
 }
 
-template <int GRID>
+template <int GRID, bool UE8>
 __global__ void __launch_bounds__(F32sCfg::kThreads, 1)
     gemm_f32s_kernel(const __grid_constant__ GemmArgs args) {
     using C = F32sCfg;
@@ -474,14 +474,13 @@ __global__ void __launch_bounds__(F32sCfg::kThreads, 1)
         const int row_in_tile = 32 * q + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
         const float mult = args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f);
-        const bool ue8 = args.scale_ue8m0 != 0;
         uint32_t it = 0, pq = 0;
         bool ok = true;
         for (int64_t t = unit; t < ntiles && ok; t += nunits) {
             const Tile tl = get_tile<TM, TN>(args, t);
-            float acc[64];
+            float2 acc[32];   // columns 2i, 2i + 1 of the warp's 64
 #pragma unroll
-            for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
             for (int ks = 0; ks < tl.nks && ok; ++ks, ++it) {
                 const int ss = it % C::NS;
                 if (!warp_wait(&sc_full[ss], (it / C::NS) & 1, kErrTimeoutEpilogue, abort_flag)) {
@@ -500,37 +499,38 @@ __global__ void __launch_bounds__(F32sCfg::kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const float sa = ue8 ? ue8m0_to_f32(sa_u8[bi * BM + row_in_tile]) : sa_tile[bi * BM + row_in_tile];
+                    const float sa = UE8 ? ue8m0_to_f32(sa_u8[bi * BM + row_in_tile]) : sa_tile[bi * BM + row_in_tile];
+                    const float2 sa2 = make_float2(sa, sa);
                     const float4 *sb4 = reinterpret_cast<const float4 *>(sb_tile + bi * BN + cs * 64);
                     const uchar4 *sb4u = reinterpret_cast<const uchar4 *>(sb_u8 + bi * BN + cs * 64);
                     const uint32_t ta = tmem_base + p * BN + cs * 64 + lane_addr;
+                    uint32_t r[2][32];
+                    tmem_ld_32x32b_x32(ta, r[0]);
+                    tmem_ld_32x32b_x32(ta + 32, r[1]);
+                    tmem_wait_ld();
+                    // partial buffer p read: the MMAs may refill it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&p_empty[p]);
+                    // Two columns per packed fp32x2 operation: the same
+                    // per-lane IEEE product s_a s_b and fused accumulate.
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        uint32_t r[32];
-                        tmem_ld_32x32b_x32(ta + 32 * half, r);
-                        tmem_wait_ld();
-                        if (half == 1) {
-                            // partial buffer p read: the MMAs may refill it
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(&p_empty[p]);
+                    for (int c4 = 0; c4 < 16; ++c4) {
+                        float4 sb;
+                        if constexpr (UE8) {
+                            const uchar4 e = sb4u[c4];
+                            sb = make_float4(ue8m0_to_f32(e.x), ue8m0_to_f32(e.y), ue8m0_to_f32(e.z),
+                                             ue8m0_to_f32(e.w));
+                        } else {
+                            sb = sb4[c4];
                         }
-#pragma unroll
-                        for (int c4 = 0; c4 < 8; ++c4) {
-                            float4 sb;
-                            if (ue8) {
-                                const uchar4 e = sb4u[8 * half + c4];
-                                sb = make_float4(ue8m0_to_f32(e.x), ue8m0_to_f32(e.y), ue8m0_to_f32(e.z),
-                                                 ue8m0_to_f32(e.w));
-                            } else {
-                                sb = sb4[8 * half + c4];
-                            }
-                            float *ac = acc + 32 * half + 4 * c4;
-                            ac[0] = __fmaf_rn(__fmul_rn(sa, sb.x), __uint_as_float(r[4 * c4 + 0]), ac[0]);
-                            ac[1] = __fmaf_rn(__fmul_rn(sa, sb.y), __uint_as_float(r[4 * c4 + 1]), ac[1]);
-                            ac[2] = __fmaf_rn(__fmul_rn(sa, sb.z), __uint_as_float(r[4 * c4 + 2]), ac[2]);
-                            ac[3] = __fmaf_rn(__fmul_rn(sa, sb.w), __uint_as_float(r[4 * c4 + 3]), ac[3]);
-                        }
+                        const uint32_t *rr = r[c4 >> 3] + 4 * (c4 & 7);
+                        const float2 s01 = __fmul2_rn(sa2, make_float2(sb.x, sb.y));
+                        const float2 s23 = __fmul2_rn(sa2, make_float2(sb.z, sb.w));
+                        acc[2 * c4] = __ffma2_rn(s01, make_float2(__uint_as_float(rr[0]), __uint_as_float(rr[1])),
+                                                 acc[2 * c4]);
+                        acc[2 * c4 + 1] = __ffma2_rn(
+                            s23, make_float2(__uint_as_float(rr[2]), __uint_as_float(rr[3])), acc[2 * c4 + 1]);
                     }
                 }
                 __syncwarp();
@@ -544,13 +544,13 @@ __global__ void __launch_bounds__(F32sCfg::kThreads, 1)
                 const bool vec = (col0 + 64 <= tl.g.n) && ((reinterpret_cast<uintptr_t>(dst) & 15u) == 0);
                 if (vec) {
 #pragma unroll
-                    for (int i = 0; i < 64; i += 4)
-                        *reinterpret_cast<float4 *>(dst + i) =
-                            make_float4(acc[i] * mult, acc[i + 1] * mult, acc[i + 2] * mult, acc[i + 3] * mult);
+                    for (int i = 0; i < 32; i += 2)
+                        *reinterpret_cast<float4 *>(dst + 2 * i) = make_float4(
+                            acc[i].x * mult, acc[i].y * mult, acc[i + 1].x * mult, acc[i + 1].y * mult);
                 } else {
 #pragma unroll
                     for (int i = 0; i < 64; ++i)
-                        if (col0 + i < tl.g.n) dst[i] = acc[i] * mult;
+                        if (col0 + i < tl.g.n) dst[i] = (i & 1 ? acc[i >> 1].y : acc[i >> 1].x) * mult;
                 }
             }
         }
@@ -1726,12 +1726,12 @@ cudaError_t launch_fp4(const GemmArgs &args, int num_sms, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-template <int GRID>
-cudaError_t launch_f32s(const GemmArgs &args, int num_sms, cudaStream_t stream) {
+template <int GRID, bool UE8>
+cudaError_t launch_f32s_fmt(const GemmArgs &args, int num_sms, cudaStream_t stream) {
     using C = F32sCfg;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_f32s_kernel<GRID>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(gemm_f32s_kernel<GRID, UE8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kAlloc);
         if (e != cudaSuccess) return e;
         configured = true;
@@ -1743,8 +1743,15 @@ cudaError_t launch_f32s(const GemmArgs &args, int num_sms, cudaStream_t stream) 
         if (tiles < units) units = static_cast<int>(tiles);
     }
     if (units <= 0) return cudaSuccess;
-    gemm_f32s_kernel<GRID><<<units, C::kThreads, C::kAlloc, stream>>>(args);
+    gemm_f32s_kernel<GRID, UE8><<<units, C::kThreads, C::kAlloc, stream>>>(args);
     return cudaGetLastError();
+}
+
+// fp32 or UE8M0 block scales: the scale decode is a compile-time choice.
+template <int GRID>
+cudaError_t launch_f32s(const GemmArgs &args, int num_sms, cudaStream_t stream) {
+    return args.scale_ue8m0 ? launch_f32s_fmt<GRID, true>(args, num_sms, stream)
+                            : launch_f32s_fmt<GRID, false>(args, num_sms, stream);
 }
 
 }  // namespace
