@@ -135,14 +135,12 @@ ufp4_status_t check_pair(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b, bool 
 
 std::atomic<int32_t> g_two_level_path{UFP4_GEMM_PATH_AUTO};
 
-ufp4_status_t encode_operand_maps(const ufp4_qtensor_t *q, int code_rows, int scale_rows, int mode,
+ufp4_status_t encode_operand_maps(const ufp4_qtensor_t *q, int code_rows, int scale_rows, int mode, int k_stage,
                                   CUtensorMap *codes, CUtensorMap *scales) {
     const int64_t rows_t = q->rows > 0 ? q->rows : 1;
-    // The FP4 kernels (modes >= 3) stage 128 K elements per step (64-byte
-    // code rows, 64-byte swizzle), the fp32-scale kernel 64 (32-byte rows,
-    // 32-byte swizzle).
-    const bool native = mode >= 3;
-    const int k_stage = native ? 128 : 64;
+    // Code rows of k_stage / 2 bytes per pipeline stage, swizzled by their
+    // width: the fp32-scale kernel stages 64 K elements (32-byte rows), the
+    // FP4 kernels 128 (64-byte rows) or 256 (128-byte rows).
     const uint32_t row_bytes = static_cast<uint32_t>(k_stage / 2);
     const CUtensorMapSwizzle swz = row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                    : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -228,9 +226,20 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
         case 6: bn = 128; bscale = 256; break;
         default: bn = bscale = 128; break;
     }
-    s = encode_operand_maps(a, 128, 128, mode, &args.tm_a_codes, &args.tm_a_scales);
+    // Dense problems on the CTA-pair kernels whose operands both carry factor
+    // atoms: each stage's atoms come with its code tiles and the MMA issuer
+    // copies them into tensor memory.  Grouped problems keep the
+    // factor-building warps (measured faster there: short K per tile, ragged
+    // groups).
+    const bool use_atoms = (mode == 5 || mode == 6) && groups_dev == nullptr && a->sf_atoms != nullptr &&
+                           b->sf_atoms != nullptr && a->rows > 0 && b->rows > 0;
+    // The restricted E2M1 grid stores E2M1 codes (0..4): the E2M1 kernels.
+    const int grid_kind = a->cfg.grid == UFP4_GRID_E1M2 ? 0 : 1;
+    // K elements per pipeline stage of the chosen kernel.
+    const int k_stage = mode == 0 ? 64 : (mode == 5 ? pair_stage_k(grid_kind, use_atoms) : 128);
+    s = encode_operand_maps(a, 128, 128, mode, k_stage, &args.tm_a_codes, &args.tm_a_scales);
     if (s != UFP4_OK) return s;
-    s = encode_operand_maps(b, bn, bscale, mode, &args.tm_b_codes, &args.tm_b_scales);
+    s = encode_operand_maps(b, bn, bscale, mode, k_stage, &args.tm_b_codes, &args.tm_b_scales);
     if (s != UFP4_OK) return s;
     if (mode == 6) {   // E4M3 element planes: 128-byte rows (128 K per stage), 128-byte swizzle
         const int64_t ra = a->rows > 0 ? a->rows : 1, rb = b->rows > 0 ? b->rows : 1;
@@ -281,23 +290,18 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
             ac.codes = a->corr;
             bc.codes = b->corr;
             CUtensorMap scratch;
-            s = encode_operand_maps(&ac, 128, 128, mode, &args.tm_a_corr, &scratch);
+            s = encode_operand_maps(&ac, 128, 128, mode, k_stage, &args.tm_a_corr, &scratch);
             if (s != UFP4_OK) return s;
-            s = encode_operand_maps(&bc, bn, bscale, mode, &args.tm_b_corr, &scratch);
+            s = encode_operand_maps(&bc, bn, bscale, mode, k_stage, &args.tm_b_corr, &scratch);
             if (s != UFP4_OK) return s;
         }
         args.corr_in = 1;
     }
-    // Dense problems on the CTA-pair kernels whose operands both carry factor
-    // atoms: each stage's atoms come with its code tiles (one u64 box of 128 K
-    // elements per 128-row group: two atoms of E4M3 factors, one of UE8M0)
-    // and the MMA issuer copies them into tensor memory.  Grouped problems
-    // keep the factor-building warps (measured faster there: short K per
-    // tile, ragged groups).
-    if ((mode == 5 || mode == 6) && groups_dev == nullptr && a->sf_atoms != nullptr && b->sf_atoms != nullptr &&
-        a->rows > 0 && b->rows > 0) {
+    // Factor atoms: one u64 box of a stage's K elements per 128-row group
+    // (k_stage / 64 atoms of E4M3 factors, k_stage / 128 of UE8M0).
+    if (use_atoms) {
         const int64_t ak = atoms_k_of(a->kpad, a->cfg), bk = atoms_k_of(b->kpad, b->cfg);
-        const uint32_t box_k = static_cast<uint32_t>(64 * (128 / (4 * atom_slot(a->cfg))));
+        const uint32_t box_k = static_cast<uint32_t>(64 * (k_stage / (4 * atom_slot(a->cfg))));
         CUresult r = encode_tensor_map_2d(&args.tm_a_atoms, CU_TENSOR_MAP_DATA_TYPE_UINT64, a->sf_atoms,
                                           static_cast<uint64_t>(64 * ak), static_cast<uint64_t>((a->rows + 127) / 128),
                                           static_cast<uint64_t>(ak) * 512, box_k, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -323,8 +327,6 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
         if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
         args.c_tma = 1;
     }
-    // The restricted E2M1 grid stores E2M1 codes (0..4): the E2M1 kernels.
-    const int grid_kind = a->cfg.grid == UFP4_GRID_E1M2 ? 0 : 1;
     cudaError_t e = launch_gemm(args, mode, grid_kind, sm_count(), st);
     return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
 }

@@ -1149,7 +1149,7 @@ struct PairCfg {
     static constexpr bool kMx = GRID == 3;
     static constexpr int TM = 256;
     static constexpr int BN = 256;
-    static constexpr int BKE = 128;                 // K elements per stage
+    static constexpr int BKE = kMx ? 128 : pair_stage_k(GRID, ATOMS);   // K elements per stage
     static constexpr int KST = kMx ? 1 : BKE / 64;  // factor atom groups per stage
     static constexpr int kRow = kMx ? BKE : BKE / 2;   // operand bytes per row per stage
     static constexpr int kPlanes = GRID == 0 ? 2 : 1;
@@ -1450,19 +1450,20 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
                             first = false;
                         }
                     } else {
+                        // code rows of 64 bytes (64-byte swizzle) or, for 256-K stages, 128 bytes
+                        auto desc = [](uint32_t addr) {
+                            return C::kRow == 128 ? umma_desc_sw128(addr) : umma_desc_sw64(addr);
+                        };
                         for (int j = 0; j < steps; ++j) {
                             const uint32_t sfa = sf0 + 12 * j, sfb = sfa + 4;
                             const uint32_t dk = 32 * j;
-                            umma_fp4_bs_pair(tmem_base, umma_desc_sw64(a0 + dk), umma_desc_sw64(b0 + dk), idesc,
-                                             sfa, sfb, first ? 0u : 1u);
+                            umma_fp4_bs_pair(tmem_base, desc(a0 + dk), desc(b0 + dk), idesc, sfa, sfb,
+                                             first ? 0u : 1u);
                             first = false;
                             if (GRID == 0) {
-                                umma_fp4_bs_pair(tmem_base, umma_desc_sw64(a0 + dk), umma_desc_sw64(bc + dk), idesc,
-                                                 sfa, sfb, 1u);
-                                umma_fp4_bs_pair(tmem_base, umma_desc_sw64(ac + dk), umma_desc_sw64(b0 + dk), idesc,
-                                                 sfa, sfb, 1u);
-                                umma_fp4_bs_pair(tmem_base, umma_desc_sw64(ac + dk), umma_desc_sw64(bc + dk), idesc,
-                                                 sfa, sfb, 1u);
+                                umma_fp4_bs_pair(tmem_base, desc(a0 + dk), desc(bc + dk), idesc, sfa, sfb, 1u);
+                                umma_fp4_bs_pair(tmem_base, desc(ac + dk), desc(b0 + dk), idesc, sfa, sfb, 1u);
+                                umma_fp4_bs_pair(tmem_base, desc(ac + dk), desc(bc + dk), idesc, sfa, sfb, 1u);
                             }
                         }
                     }

@@ -124,6 +124,10 @@ struct GemmArgs {
 // Tile columns (B rows) of the native block-scaled FP4 kernels (modes 3, 4).
 constexpr int kNativeTileN = 192;
 constexpr int kTileBand = 8;   // rows of output tiles per band of the GEMM tile order
+// K elements per pipeline stage of the CTA-pair kernels: 256 for E2M1
+// operands with factor atoms (one MMA per 64 K: a longer stage spreads the
+// issuer's per-stage waits, fences and commits over more MMAs), else 128.
+constexpr int pair_stage_k(int grid_kind, bool atoms) { return (grid_kind == 1 && atoms) ? 256 : 128; }
 
 // mode 0: fp32 block scales (per-block partial products, CUDA-core scaling)
 // mode 1: E4M3 x fp32 two-level scales (scales folded into fp16 operands)
