@@ -198,7 +198,7 @@ def test_factor_atoms_path_equals_factor_warps(grid, fmt, block):
     copies them into tensor memory) give bit-for-bit the output of the same
     kernel building the factors from the block-major scales, and the
     oracle's result; partial 256-wide tiles, one-row operands, K tails of 64
-    and of 128 + 64."""
+    and of 128 + 64 (E2M1 stages 256 K: tails of 64, 192 and 256)."""
     import dataclasses
     cfg = _cfg(grid=grid, fmt=fmt, block=block)
     for (M, N, K) in [(520, 700, 448), (130, 230, 200), (1, 1, 8), (300, 513, 1000)]:
