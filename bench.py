@@ -934,6 +934,15 @@ def cpu_baseline(scale: str, shape, budget_s: float = 10.0) -> dict:
     oracle.gemm_tn(qa, qb)
     t2 = time.perf_counter()
     tiny_gflops = 2 * t.M * t.N * t.K / (t2 - t1) / 1e9
+    # the quantizer sweep's largest tensor (32768 x 16384 ~0.1 Student-t(4)),
+    # recipe configuration (E1M2 RTNE, n 16, block 16, fp32 scales): full-K
+    # rows quantized along the columns (rows are independent with fp32 scales)
+    sweep_rows = min(4096, 256 * cores)
+    Xs = wl.student_t(sweep_rows, 16384, seed=5)
+    t3 = time.perf_counter()
+    oracle.quantize(Xs, 0, oracle.QuantCfg(grid=0, hadamard_n=16, block=16, sign_mask=OracleSample.MASK))
+    t4 = time.perf_counter()
+    sweep_gbps = sweep_rows * 16384 * (2 + 0.5 + 4 / 16) / (t4 - t3) / 1e9
     return {"value": fig["value"], "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": (f"{n} sampled steps of the large layer ({secs:.1f} s of CPU work): {n_rows} output rows "
                        f"of each of the 6 quantized operands (full K) and a {n_rows}x{n_rows} block of each "
@@ -942,7 +951,10 @@ def cpu_baseline(scale: str, shape, budget_s: float = 10.0) -> dict:
             "quantize_GBps": round(fig["quantize_GBps"], 4),
             "gemm_GFLOPs": round(fig["gemm_GFLOPs"], 3),
             "tiny_fprop_full": {"shape": [t.M, t.K, t.N], "gemm_GFLOPs": round(tiny_gflops, 3),
-                                "quantize_ms": round((t1 - t0) * 1e3, 2)}}
+                                "quantize_ms": round((t1 - t0) * 1e3, 2)},
+            "quantize_sweep_tensor": {"shape": [32768, 16384], "sample_rows": sweep_rows,
+                                      "recipe": "E1M2 RTNE, RHT16, block 16, fp32 scales, along columns",
+                                      "GBps": round(sweep_gbps, 4), "seconds": round(t4 - t3, 2)}}
 
 
 def main():
