@@ -1138,8 +1138,11 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CIN>::kThreads, 1)
 //              transposes and store them with tcgen05.st;
 //   warps 8-11 epilogue: TMEM -> registers -> x S_a S_b / (16 n) -> staged
 //              in shared memory -> coalesced 16-byte stores.
-// One accumulator per CTA: the epilogue of a tile (about 2% of a K = 8192
-// main loop) runs before the next tile's MMAs start.
+// One accumulator per CTA.  Without factor atoms the epilogue reads TMEM in
+// 32-column pieces between its stores, and the next tile's MMAs wait for the
+// last piece.  With factor atoms (no factor writers) warps 4-11 drain the
+// accumulator into registers, 128 columns each, release TMEM at once and
+// then scale and store while the next tile's MMAs run.
 // GRID 3 is the MX path: E1M2 operands as their E4M3 element planes (one
 // byte per element, 128-byte rows, 128-byte swizzle), UE8M0 factors per 32
 // elements applied in the MMA (kind::mxf8f6f4, K = 32 per MMA, four MMAs per
@@ -1268,7 +1271,7 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
     uint64_t *sfready = sfull + NS;       // leader: factors of stage s in both CTAs' TMEM
     uint64_t *sflocal = sfready + NS;     // peer: its four factor warps wrote stage s
     uint64_t *acc_full = sflocal + NS;    // accumulator complete (commit to both CTAs)
-    uint64_t *acc_empty = acc_full + 1;   // leader: both CTAs' epilogues drained TMEM (8 warps)
+    uint64_t *acc_empty = acc_full + 1;   // leader: both CTAs' epilogues drained TMEM (8 or 16 warps)
     uint64_t *drain = acc_empty + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::o_misc);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::o_misc + 4);
@@ -1291,7 +1294,7 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
             mbar_init(&sflocal[i], 4);
         }
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 8);
+        mbar_init(acc_empty, ATOMS ? 16 : 8);
         mbar_init(drain, 1);
         *abort_flag = 0u;
         fence_barrier_init();
@@ -1496,6 +1499,84 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
                     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
                                      ready + static_cast<uint32_t>(s) * 8u)
                                  : "memory");
+                }
+            }
+        }
+    } else if (ATOMS && warp >= 4) {
+        // ------------------------------------------------------------ epilogue (factor atoms)
+        // No factor writers: eight warps drain the accumulator, warp w reads
+        // TMEM lane quarter w % 4, columns [128 h, +128) with h = (w - 4) / 4.
+        // All 128 columns go to registers first and TMEM is released at once,
+        // so the next tile's MMAs overlap this tile's scaling and stores.
+        // Each 32 x 32 piece is transposed through a per-warp 4 KB buffer
+        // (16-byte units XORed with the row mod 8) so that eight lanes write
+        // one row's 128 bytes per store.
+        const int q = warp & 3;
+        const int h = (warp - 4) >> 2;
+        const uint32_t lane_addr = (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(128 * h);
+        const uint32_t empty_acc = cluster_addr(acc_empty, 0);
+        uint8_t *buf = smem + C::o_out + (warp - 4) * 4096;
+        const float mult = C::kMx ? args.inv_n
+                                  : __fmul_rn(__fmul_rn(*args.a_S, *args.b_S),
+                                              args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f));
+        uint32_t tcount = 0;
+        for (int64_t t = unit; t < ntiles; t += nunits, ++tcount) {
+            const Tile tl = get_tile<TM, BN>(args, t, sched);
+            if (!warp_wait(acc_full, tcount & 1, kErrTimeoutEpilogue, abort_flag)) break;
+            tc_fence_after();
+            uint32_t r[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tmem_base + lane_addr + 32 * c, r[c]);
+            tmem_wait_ld();
+            // accumulator drained by this warp: the next tile's MMAs may start
+            // once all sixteen warps of the pair have arrived
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(empty_acc)
+                             : "memory");
+            const int64_t m0 = tl.m0 + 128 * rank + 32 * q;   // this warp's accumulator rows
+            const bool vec_tile = args.c_vec && (tl.g.c_col & 3) == 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int64_t col0 = tl.n0 + 128 * h + 32 * c;
+                if (col0 >= tl.g.n) break;                // the same for the whole warp
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    v[i] = tl.g.k > 0 ? __fmul_rn(__uint_as_float(r[c][i]), mult) : 0.0f;
+                if (vec_tile) {
+                    uint8_t *rowp = buf + lane * 128;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch)
+                        *reinterpret_cast<float4 *>(rowp + ((ch ^ (lane & 7)) << 4)) =
+                            make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
+                    __syncwarp();
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int rr = 4 * k + (lane >> 3), c16 = lane & 7;
+                        const float4 val =
+                            *reinterpret_cast<const float4 *>(buf + rr * 128 + ((c16 ^ (rr & 7)) << 4));
+                        const int64_t grow = m0 + rr;
+                        const int64_t gcol = col0 + 4 * c16;
+                        if (grow < tl.g.m && gcol < tl.g.n) {
+                            float *dst = args.c + (tl.g.c_row + grow) * args.ldc + tl.g.c_col + gcol;
+                            if (gcol + 4 <= tl.g.n) {
+                                __stcs(reinterpret_cast<float4 *>(dst), val);   // streamed: evict first
+                            } else {
+                                const float e4[4] = {val.x, val.y, val.z, val.w};
+                                for (int e = 0; e < 4 && gcol + e < tl.g.n; ++e) dst[e] = e4[e];
+                            }
+                        }
+                    }
+                    __syncwarp();                         // buffer read out before the next piece
+                } else {
+                    const int64_t row = m0 + lane;
+                    if (row < tl.g.m) {
+                        float *dst = args.c + (tl.g.c_row + row) * args.ldc + tl.g.c_col + col0;
+                        for (int i = 0; i < 32; ++i)
+                            if (col0 + i < tl.g.n) dst[i] = v[i];
+                    }
                 }
             }
         }
