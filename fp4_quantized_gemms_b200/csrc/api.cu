@@ -318,15 +318,6 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
     args.band = kTileBand;
     // Native kernels store 16-byte pieces when the output allows it.
     args.c_vec = (aligned16(c) && ldc % 4 == 0) ? 1 : 0;
-    // The CTA-pair kernel writes whole 128 x 32 output pieces with TMA bulk
-    // stores (clipped at m and n) when the output is a single dense problem.
-    if ((mode == 5 || mode == 6) && groups_dev == nullptr && args.c_vec) {
-        CUresult r = encode_tensor_map_2d(&args.tm_c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c, static_cast<uint64_t>(n),
-                                          static_cast<uint64_t>(m), static_cast<uint64_t>(ldc) * 4, 32, 128,
-                                          CU_TENSOR_MAP_SWIZZLE_128B);
-        if (r != CUDA_SUCCESS) return UFP4_ERR_CUDA;
-        args.c_tma = 1;
-    }
     cudaError_t e = launch_gemm(args, mode, grid_kind, sm_count(), st);
     return e == cudaSuccess ? UFP4_OK : UFP4_ERR_CUDA;
 }

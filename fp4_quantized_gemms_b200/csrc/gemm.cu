@@ -1168,16 +1168,15 @@ struct PairCfg {
     static constexpr int kStage = (kCodeBytes + kRawA + kRawB + 1023) / 1024 * 1024;
     static constexpr int kAtoms = 3 * KST;          // SFA, SFB rows 0-127, SFB rows 128-255 per K step
     static constexpr int kScr = ATOMS ? 0 : 4 * kAtoms * 512;   // one atom scratch per factor warp
-    static constexpr int kOutChunk = 128 * 32 * 4;  // epilogue staging: 128 rows x 32 fp32
-    static constexpr int kOutBufs = 2;              // staging buffers (bulk stores in flight)
+    static constexpr int kOutBytes = (ATOMS ? 8 : 4) * 4096;   // epilogue staging: 4 KB per epilogue warp
     static constexpr int kSfBase = 256;             // TMEM column of the first factor slot
     static constexpr int kSfCols = 12 * KST;        // TMEM columns of one stage's factors
     static constexpr int kNsTmem = (512 - kSfBase) / kSfCols;
     static constexpr int kBudget = 232448 - 2048;
-    static constexpr int kNsSmem = (kBudget - kScr - kOutBufs * kOutChunk) / kStage;
+    static constexpr int kNsSmem = (kBudget - kScr - kOutBytes) / kStage;
     static constexpr int NS = kNsSmem < kNsTmem ? kNsSmem : kNsTmem;
     static constexpr int o_out = NS * kStage;
-    static constexpr int o_scr = o_out + kOutBufs * kOutChunk;
+    static constexpr int o_scr = o_out + kOutBytes;
     static constexpr int o_bar = o_scr + kScr;
     // full[NS], empty[NS], sfull[NS], sfready[NS], sflocal[NS], acc_full,
     // acc_empty, drain
@@ -1255,6 +1254,52 @@ __host__ __device__ constexpr uint32_t umma_idesc_mxf8(int M, int N, uint32_t sf
            | (1u << 23)                               // factor format UE8M0
            | (static_cast<uint32_t>(M >> 4) << 24)    // M / 16
            | (sf_id << 29);                           // A factor byte
+}
+
+// Epilogue piece of one warp: accumulator rows m0 + lane (thread = row) x
+// columns [col0, col0 + 32), scaled by mult (zero: the group has k = 0 and
+// no MMA wrote the accumulator) and written to C.  With 16-byte aligned rows
+// the piece is transposed through the warp's 4 KB buffer (16-byte units
+// XORed with the row mod 8, conflict-free both ways) so that eight lanes
+// write one row's 128 bytes per store.
+__device__ __forceinline__ void store_piece(const GemmArgs &args, const Tile &tl, uint8_t *buf, int lane,
+                                            int64_t m0, int64_t col0, uint32_t (&r)[32], float mult, bool zero,
+                                            bool vec_tile) {
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = zero ? 0.0f : __fmul_rn(__uint_as_float(r[i]), mult);
+    if (vec_tile) {
+        uint8_t *rowp = buf + lane * 128;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+            *reinterpret_cast<float4 *>(rowp + ((ch ^ (lane & 7)) << 4)) =
+                make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int rr = 4 * k + (lane >> 3), c16 = lane & 7;
+            const float4 val = *reinterpret_cast<const float4 *>(buf + rr * 128 + ((c16 ^ (rr & 7)) << 4));
+            const int64_t grow = m0 + rr;
+            const int64_t gcol = col0 + 4 * c16;
+            if (grow < tl.g.m && gcol < tl.g.n) {
+                float *dst = args.c + (tl.g.c_row + grow) * args.ldc + tl.g.c_col + gcol;
+                if (gcol + 4 <= tl.g.n) {
+                    __stcs(reinterpret_cast<float4 *>(dst), val);   // streamed: evict first
+                } else {
+                    const float e4[4] = {val.x, val.y, val.z, val.w};
+                    for (int e = 0; e < 4 && gcol + e < tl.g.n; ++e) dst[e] = e4[e];
+                }
+            }
+        }
+        __syncwarp();                                 // buffer read out before the next piece
+    } else {
+        const int64_t row = m0 + lane;
+        if (row < tl.g.m) {
+            float *dst = args.c + (tl.g.c_row + row) * args.ldc + tl.g.c_col + col0;
+            for (int i = 0; i < 32; ++i)
+                if (col0 + i < tl.g.n) dst[i] = v[i];
+        }
+    }
 }
 
 template <int GRID, bool ATOMS>
@@ -1502,84 +1547,6 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
                 }
             }
         }
-    } else if (ATOMS && warp >= 4) {
-        // ------------------------------------------------------------ epilogue (factor atoms)
-        // No factor writers: eight warps drain the accumulator, warp w reads
-        // TMEM lane quarter w % 4, columns [128 h, +128) with h = (w - 4) / 4.
-        // All 128 columns go to registers first and TMEM is released at once,
-        // so the next tile's MMAs overlap this tile's scaling and stores.
-        // Each 32 x 32 piece is transposed through a per-warp 4 KB buffer
-        // (16-byte units XORed with the row mod 8) so that eight lanes write
-        // one row's 128 bytes per store.
-        const int q = warp & 3;
-        const int h = (warp - 4) >> 2;
-        const uint32_t lane_addr = (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(128 * h);
-        const uint32_t empty_acc = cluster_addr(acc_empty, 0);
-        uint8_t *buf = smem + C::o_out + (warp - 4) * 4096;
-        const float mult = C::kMx ? args.inv_n
-                                  : __fmul_rn(__fmul_rn(*args.a_S, *args.b_S),
-                                              args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f));
-        uint32_t tcount = 0;
-        for (int64_t t = unit; t < ntiles; t += nunits, ++tcount) {
-            const Tile tl = get_tile<TM, BN>(args, t, sched);
-            if (!warp_wait(acc_full, tcount & 1, kErrTimeoutEpilogue, abort_flag)) break;
-            tc_fence_after();
-            uint32_t r[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tmem_base + lane_addr + 32 * c, r[c]);
-            tmem_wait_ld();
-            // accumulator drained by this warp: the next tile's MMAs may start
-            // once all sixteen warps of the pair have arrived
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(empty_acc)
-                             : "memory");
-            const int64_t m0 = tl.m0 + 128 * rank + 32 * q;   // this warp's accumulator rows
-            const bool vec_tile = args.c_vec && (tl.g.c_col & 3) == 0;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int64_t col0 = tl.n0 + 128 * h + 32 * c;
-                if (col0 >= tl.g.n) break;                // the same for the whole warp
-                float v[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    v[i] = tl.g.k > 0 ? __fmul_rn(__uint_as_float(r[c][i]), mult) : 0.0f;
-                if (vec_tile) {
-                    uint8_t *rowp = buf + lane * 128;
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch)
-                        *reinterpret_cast<float4 *>(rowp + ((ch ^ (lane & 7)) << 4)) =
-                            make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
-                    __syncwarp();
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const int rr = 4 * k + (lane >> 3), c16 = lane & 7;
-                        const float4 val =
-                            *reinterpret_cast<const float4 *>(buf + rr * 128 + ((c16 ^ (rr & 7)) << 4));
-                        const int64_t grow = m0 + rr;
-                        const int64_t gcol = col0 + 4 * c16;
-                        if (grow < tl.g.m && gcol < tl.g.n) {
-                            float *dst = args.c + (tl.g.c_row + grow) * args.ldc + tl.g.c_col + gcol;
-                            if (gcol + 4 <= tl.g.n) {
-                                __stcs(reinterpret_cast<float4 *>(dst), val);   // streamed: evict first
-                            } else {
-                                const float e4[4] = {val.x, val.y, val.z, val.w};
-                                for (int e = 0; e < 4 && gcol + e < tl.g.n; ++e) dst[e] = e4[e];
-                            }
-                        }
-                    }
-                    __syncwarp();                         // buffer read out before the next piece
-                } else {
-                    const int64_t row = m0 + lane;
-                    if (row < tl.g.m) {
-                        float *dst = args.c + (tl.g.c_row + row) * args.ldc + tl.g.c_col + col0;
-                        for (int i = 0; i < 32; ++i)
-                            if (col0 + i < tl.g.n) dst[i] = v[i];
-                    }
-                }
-            }
-        }
     } else if (!ATOMS && warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ factor writers
         uint8_t *scr = smem + C::o_scr + (warp - 4) * (C::kAtoms * 512);
@@ -1642,109 +1609,59 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
                 if (lane == 0) mbar_arrive(rank == 0 ? &sfready[s] : &sflocal[s]);
             }
         }
-    } else if (warp >= 8) {
+    } else if (ATOMS ? warp >= 4 : warp >= 8) {
         // ------------------------------------------------------------ epilogue
-        // Thread = accumulator row.  Each 128 x 32 fp32 piece is staged in
-        // shared memory in the 128-byte-swizzled layout (16-byte units XORed
-        // with the row mod 8) and, for a single dense output, written by one
-        // TMA bulk store while the warps move on (two staging buffers); TMEM
-        // is released right after the last piece is read.  Grouped outputs
-        // (windows of a larger matrix) use coalesced 16-byte stores.
+        // Warp w reads TMEM lane quarter w % 4 (accumulator rows 32 (w % 4) +
+        // lane of this CTA's 128).  With factor atoms (no factor writers)
+        // warps 4-11 drain the accumulator, 128 columns each (h = (w - 4) / 4
+        // picks the half): all of them go to registers and TMEM is released
+        // at once, so the next tile's MMAs overlap this tile's scaling and
+        // stores.  Otherwise warps 8-11 take both halves, one after the
+        // other, and release TMEM once the second half is in registers.
         const int q = warp & 3;
-        const int et = threadIdx.x - 32 * 8;            // 0 .. 127
-        const int row_in_tile = 32 * q + lane;
+        const int h0 = ATOMS ? (warp - 4) >> 2 : 0;
+        constexpr int kHalves = ATOMS ? 1 : 2;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-        constexpr uint32_t kEpiThreads = 128;
-        const bool elected = et == 0;
         const uint32_t empty_acc = cluster_addr(acc_empty, 0);
+        uint8_t *buf = smem + C::o_out + (warp - (ATOMS ? 4 : 8)) * 4096;
         // E1M2 operands carry k = 4 * level on both sides: 1/16 (exact).  The
         // MX path's E4M3 elements are the levels and its factors are in the
         // MMA: only 1/n.
         const float mult = C::kMx ? args.inv_n
                                   : __fmul_rn(__fmul_rn(*args.a_S, *args.b_S),
                                               args.inv_n * (GRID == 0 ? (1.0f / 16.0f) : 1.0f));
-        uint32_t tcount = 0, piece = 0;
+        uint32_t tcount = 0;
         for (int64_t t = unit; t < ntiles; t += nunits, ++tcount) {
             const Tile tl = get_tile<TM, BN>(args, t, sched);
-            const bool ok = warp_wait(acc_full, tcount & 1, kErrTimeoutEpilogue, abort_flag);
-            if (named_bar_or(1, kEpiThreads, !ok)) break;
+            if (!warp_wait(acc_full, tcount & 1, kErrTimeoutEpilogue, abort_flag)) break;
             tc_fence_after();
-            const int64_t m0 = tl.m0 + 128 * rank;       // this CTA's accumulator rows
-            const int64_t row = m0 + row_in_tile;
-            const bool row_ok = row < tl.g.m;
-            float *crow = args.c + (tl.g.c_row + row) * args.ldc + tl.g.c_col + tl.n0;
-            const bool tma_tile = args.c_tma != 0;
+            const int64_t m0 = tl.m0 + 128 * rank + 32 * q;   // this warp's accumulator rows
             const bool vec_tile = args.c_vec && (tl.g.c_col & 3) == 0;
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c, ++piece) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem_base + lane_addr + 32 * c, r);
+            const bool zero = tl.g.k == 0;             // no MMA wrote the accumulator
+#pragma unroll
+            for (int hh = 0; hh < kHalves; ++hh) {
+                const int h = h0 + hh;
+                uint32_t r[4][32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tmem_base + lane_addr + 128 * h + 32 * c, r[c]);
                 tmem_wait_ld();
-                if (c == BN / 32 - 1) {
-                    // accumulator drained: the next tile's MMAs may start
+                if (hh == kHalves - 1) {
+                    // accumulator drained by this warp: the next tile's MMAs
+                    // may start once every epilogue warp of the pair arrived
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0)
                         asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(empty_acc)
                                      : "memory");
                 }
-                const int64_t col0 = tl.n0 + 32 * c;
-                if (col0 >= tl.g.n) continue;             // the same for all threads
-                float v[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    v[i] = tl.g.k > 0 ? __fmul_rn(__uint_as_float(r[i]), mult) : 0.0f;
-                if (tma_tile || vec_tile) {
-                    uint8_t *buf = smem + C::o_out + (piece & 1) * C::kOutChunk;
-                    // the bulk store issued from this buffer two pieces ago has read it
-                    if (tma_tile && elected && piece >= 2)
-                        asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-                    named_bar_sync(1, kEpiThreads);
-                    uint8_t *rowp = buf + row_in_tile * 128;
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch)
-                        *reinterpret_cast<float4 *>(rowp + ((ch ^ (row_in_tile & 7)) << 4)) =
-                            make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
-                    if (tma_tile) fence_proxy_async_smem();
-                    named_bar_sync(1, kEpiThreads);          // piece staged
-                    if (tma_tile) {
-                        if (elected) {
-                            asm volatile(
-                                "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
-                                    reinterpret_cast<uint64_t>(&args.tm_c)),
-                                "r"(static_cast<int32_t>(col0)), "r"(static_cast<int32_t>(m0)), "r"(smem_addr(buf))
-                                : "memory");
-                            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-                        }
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const int p = et + 128 * k;
-                            const int rr = p >> 3, c16 = p & 7;
-                            const float4 val =
-                                *reinterpret_cast<const float4 *>(buf + rr * 128 + ((c16 ^ (rr & 7)) << 4));
-                            const int64_t grow = m0 + rr;
-                            const int64_t gcol = col0 + 4 * c16;
-                            if (grow < tl.g.m && gcol < tl.g.n) {
-                                float *dst = args.c + (tl.g.c_row + grow) * args.ldc + tl.g.c_col + gcol;
-                                if (gcol + 4 <= tl.g.n) {
-                                    __stcs(reinterpret_cast<float4 *>(dst), val);   // streamed: evict first
-                                } else {
-                                    const float e4[4] = {val.x, val.y, val.z, val.w};
-                                    for (int e = 0; e < 4 && gcol + e < tl.g.n; ++e) dst[e] = e4[e];
-                                }
-                            }
-                        }
-                    }
-                } else if (row_ok) {
-                    float *dst = crow + 32 * c;
-                    for (int i = 0; i < 32; ++i)
-                        if (col0 + i < tl.g.n) dst[i] = v[i];
+                for (int c = 0; c < 4; ++c) {
+                    const int64_t col0 = tl.n0 + 128 * h + 32 * c;
+                    if (col0 >= tl.g.n) break;            // the same for the whole warp
+                    store_piece(args, tl, buf, lane, m0, col0, r[c], mult, zero, vec_tile);
                 }
             }
         }
-        // every bulk store has completed before the CTA exits
-        if (elected) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     }
 
     tc_fence_before();

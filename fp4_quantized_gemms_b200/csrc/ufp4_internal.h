@@ -113,9 +113,7 @@ struct GemmArgs {
     int corr_in;                          // both operands carry correction planes
     int scale_ue8m0;                      // mode 0: scales are UE8M0 exponent bytes
     int planes3d;                         // corr = codes + rows * kpad / 2 for both
-    CUtensorMap tm_c;                     // fp32 output [m][n], box 32 x 128, 128-byte swizzle
     CUtensorMap tm_a_e8, tm_b_e8;         // MX path: E4M3 element planes [rows][kpad]
-    int c_tma;                            // tm_c valid: single problem, c_vec, c_col == 0
     CUtensorMap tm_a_atoms, tm_b_atoms;   // factor atoms as u64 [row groups][64 atoms_k]
     int atoms;                            // both operands carry factor atoms (pair kernels, dense)
     int band;                             // tile order: rows of tiles per band (0: M fastest)
