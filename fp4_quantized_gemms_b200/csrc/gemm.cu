@@ -1284,7 +1284,7 @@ __device__ __forceinline__ void store_piece(const GemmArgs &args, const Tile &tl
             if (grow < tl.g.m && gcol < tl.g.n) {
                 float *dst = args.c + (tl.g.c_row + grow) * args.ldc + tl.g.c_col + gcol;
                 if (gcol + 4 <= tl.g.n) {
-                    __stcs(reinterpret_cast<float4 *>(dst), val);   // streamed: evict first
+                    *reinterpret_cast<float4 *>(dst) = val;   // default L2 policy: fewer operand re-reads than evict-first
                 } else {
                     const float e4[4] = {val.x, val.y, val.z, val.w};
                     for (int e = 0; e < 4 && gcol + e < tl.g.n; ++e) dst[e] = e4[e];
