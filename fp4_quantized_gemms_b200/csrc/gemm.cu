@@ -1161,8 +1161,11 @@ struct PairCfg {
     static constexpr int o_b = kPlanes * kTile;     // [codes | corr] of this CTA's B half
     static constexpr int kCodeBytes = 2 * kPlanes * kTile;   // per CTA per stage
     static constexpr int kRawRows = kMx ? BKE / 32 : BKE / 16;   // factor rows per stage (most)
+    // E1M2 with factor atoms: the A factors of a stage arrive as one
+    // per-lane tile (4 KB) and leave for TMEM in one copy.
+    static constexpr bool kLaneA = GRID == 0 && ATOMS;
     static constexpr int o_raw_a = kCodeBytes;      // raw factors: [blocks][128 rows]
-    static constexpr int kRawA = 128 * kRawRows;
+    static constexpr int kRawA = kLaneA ? kLaneTileBytes : 128 * kRawRows;
     static constexpr int o_raw_b = o_raw_a + kRawA; // [blocks][256 rows]
     static constexpr int kRawB = 256 * kRawRows;
     static constexpr int kStage = (kCodeBytes + kRawA + kRawB + 1023) / 1024 * 1024;
@@ -1171,6 +1174,7 @@ struct PairCfg {
     static constexpr int kOutBytes = (ATOMS ? 8 : 4) * 4096;   // epilogue staging: 4 KB per epilogue warp
     static constexpr int kSfBase = 256;             // TMEM column of the first factor slot
     static constexpr int kSfCols = 12 * KST;        // TMEM columns of one stage's factors
+    static_assert(!kLaneA || (BKE == kLaneK && 8 + 8 * KST <= kSfCols), "per-lane A factors: one tile per stage");
     static constexpr int kNsTmem = (512 - kSfBase) / kSfCols;
     static constexpr int kBudget = 232448 - 2048;
     static constexpr int kNsSmem = (kBudget - kScr - kOutBytes) / kStage;
@@ -1201,6 +1205,18 @@ __device__ __forceinline__ void tmem_cp_atom_pair(uint32_t taddr, uint32_t smem_
     const uint64_t d = static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFFu) |
                        (static_cast<uint64_t>(128u >> 4) << 32) | (static_cast<uint64_t>(1u) << 46);
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
+}
+
+// Copy of one per-lane factor tile (128 lanes x 32 bytes, two 2048-byte halves
+// of 16 bytes per lane) into TMEM columns [taddr, taddr + 8) of both CTAs of
+// the pair.  Descriptor: no swizzle, K-major, core matrices of 8 rows x 16
+// bytes at a stride of 128 bytes (SBO) along the lanes and 2048 bytes (LBO)
+// between the two halves.
+__device__ __forceinline__ void tmem_cp_lanes_pair(uint32_t taddr, uint32_t smem_byte_addr) {
+    const uint64_t d = static_cast<uint64_t>((smem_byte_addr >> 4) & 0x3FFFu) |
+                       (static_cast<uint64_t>(2048u >> 4) << 16) | (static_cast<uint64_t>(128u >> 4) << 32) |
+                       (static_cast<uint64_t>(1u) << 46);
+    asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
 }
 
 // TMA tile loads whose completion is counted on a barrier of the leader CTA
@@ -1415,7 +1431,11 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
                         // 64 u64 per atom of kAtomK K elements (dense problems: acol = bcol)
                         constexpr int kAtomK = C::kMx ? 128 : 64;
                         const int32_t ax = 64 * (acol / kAtomK), bx = 64 * (bcol / kAtomK);
-                        tma_load_2d_pair(st + C::o_raw_a, &args.tm_a_atoms, fb, ax, arow / 128, pol);
+                        if constexpr (C::kLaneA)   // this CTA's 128 A rows: the stage's per-lane tile
+                            tma_load_3d_pair(st + C::o_raw_a, &args.tm_a_atoms, fb, 0, 0,
+                                             (arow / 128) * args.lane_groups + acol / kLaneK, pol);
+                        else
+                            tma_load_2d_pair(st + C::o_raw_a, &args.tm_a_atoms, fb, ax, arow / 128, pol);
                         tma_load_2d_pair(st + C::o_raw_b, &args.tm_b_atoms, fb, bx, brow / 128, pol);
                     } else {
                         // this CTA's raw factors
@@ -1476,11 +1496,23 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
                         // the stage's factor atoms into TMEM slot s of both CTAs (each from its
                         // own shared memory; the copies run before the MMAs issued after them,
                         // and after the MMAs that last read the slot)
+                        if constexpr (C::kLaneA) {
+                            // A: columns sf0 + 4 j + q (K step j, lane quarter q); B of K step j:
+                            // columns sf0 + 8 + 8 j (rows 0-127) and + 4 (rows 128-255)
+                            tmem_cp_lanes_pair(sf0, smem_addr(st + C::o_raw_a));
 #pragma unroll
-                        for (int j = 0; j < C::KST; ++j) {
-                            tmem_cp_atom_pair(sf0 + 12 * j, smem_addr(st + C::o_raw_a + 512 * j));
-                            tmem_cp_atom_pair(sf0 + 12 * j + 4, smem_addr(st + C::o_raw_b + 512 * j));
-                            tmem_cp_atom_pair(sf0 + 12 * j + 8, smem_addr(st + C::o_raw_b + 512 * (C::KST + j)));
+                            for (int j = 0; j < C::KST; ++j) {
+                                tmem_cp_atom_pair(sf0 + 8 + 8 * j, smem_addr(st + C::o_raw_b + 512 * j));
+                                tmem_cp_atom_pair(sf0 + 12 + 8 * j, smem_addr(st + C::o_raw_b + 512 * (C::KST + j)));
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < C::KST; ++j) {
+                                tmem_cp_atom_pair(sf0 + 12 * j, smem_addr(st + C::o_raw_a + 512 * j));
+                                tmem_cp_atom_pair(sf0 + 12 * j + 4, smem_addr(st + C::o_raw_b + 512 * j));
+                                tmem_cp_atom_pair(sf0 + 12 * j + 8,
+                                                  smem_addr(st + C::o_raw_b + 512 * (C::KST + j)));
+                            }
                         }
                     }
                     const int64_t rem = tl.g.k - static_cast<int64_t>(ks) * C::BKE;
@@ -1503,7 +1535,8 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
                             return C::kRow == 128 ? umma_desc_sw128(addr) : umma_desc_sw64(addr);
                         };
                         for (int j = 0; j < steps; ++j) {
-                            const uint32_t sfa = sf0 + 12 * j, sfb = sfa + 4;
+                            const uint32_t sfa = C::kLaneA ? sf0 + 4 * j : sf0 + 12 * j;
+                            const uint32_t sfb = C::kLaneA ? sf0 + 8 + 8 * j : sfa + 4;
                             const uint32_t dk = 32 * j;
                             umma_fp4_bs_pair(tmem_base, desc(a0 + dk), desc(b0 + dk), idesc, sfa, sfb,
                                              first ? 0u : 1u);

@@ -496,11 +496,44 @@ __device__ __forceinline__ void store_atom(const QuantArgs &a, int32_t row, int3
         *reinterpret_cast<uint16_t *>(atom_byte(a, row, 2 * blk_idx)) = static_cast<uint16_t>(b | (b << 8));
 }
 
+// Per-lane factor tiles (E1M2 operands with E4M3 factors): the factor of
+// 16-element slot s of row r sits in tile (r / 128, s / 8), half
+// j = (s / 4) % 2 (the K step), lane L = r % 128, byte 4 (L / 32) + s % 4 of
+// the lane's 16 bytes: byte 2048 j + 16 L + 4 (L / 32) + s % 4.
+__device__ __forceinline__ uint8_t *lane_byte(const QuantArgs &a, int32_t row, int32_t slot) {
+    const int32_t L = row & 127;
+    return a.sf_lanes + (static_cast<int64_t>(row >> 7) * a.lane_groups + (slot >> 3)) * kLaneTileBytes +
+           2048 * ((slot >> 2) & 1) + 16 * L + 4 * (L >> 5) + (slot & 3);
+}
+
+template <int BLK>
+__device__ __forceinline__ void store_lanes(const QuantArgs &a, int32_t row, int32_t blk_idx, uint32_t sv) {
+    const uint32_t b = sv & 0xFFu;
+    if (BLK == 16)
+        *lane_byte(a, row, blk_idx) = static_cast<uint8_t>(b);
+    else
+        *reinterpret_cast<uint16_t *>(lane_byte(a, row, 2 * blk_idx)) = static_cast<uint16_t>(b | (b << 8));
+}
+
 // Stores the 16 code bytes (and the E1M2 correction plane, the MX element
 // plane) and the block scales (and factor atoms) of one lane run.
+// The whole 16-byte lane record of row `row` for the K step at k0 (a
+// multiple of 64): the step's four factors at bytes 4 (L / 32) .. + 3, zeros
+// elsewhere, one full-sector-friendly store.  st: the two runs' stored
+// scales (lane x, then lane y).
+template <int BLK>
+__device__ __forceinline__ void store_lane_record(const QuantArgs &a, int32_t row, int32_t k0, const uint32_t *st) {
+    const uint32_t f = BLK == 16 ? ((st[0] & 0xFFu) | ((st[1] & 0xFFu) << 8) | ((st[2] & 0xFFu) << 16) |
+                                    ((st[3] & 0xFFu) << 24))
+                                 : ((st[0] & 0xFFu) * 0x0101u) | (((st[1] & 0xFFu) * 0x0101u) << 16);
+    const int q = (row & 127) >> 5;
+    uint4 v = make_uint4(q == 0 ? f : 0u, q == 1 ? f : 0u, q == 2 ? f : 0u, q == 3 ? f : 0u);
+    *reinterpret_cast<uint4 *>(lane_byte(a, row, k0 / 16) - 4 * q) = v;
+}
+
 template <int BLK>
 __device__ __forceinline__ void store_run(const QuantArgs &a, int32_t row, int32_t k0, const uint32_t *w,
-                                          const uint32_t *st) {
+                                          const uint32_t *st, bool lane_bytes = true) {
     if (row >= a.out_rows) return;
     const int64_t off = static_cast<int64_t>(row) * (a.kpad / 2) + k0 / 2;
     *reinterpret_cast<uint4 *>(a.codes + off) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -528,6 +561,13 @@ __device__ __forceinline__ void store_run(const QuantArgs &a, int32_t row, int32
                 static_cast<uint16_t>((st[0] & 0xFFu) | ((st[1] & 0xFFu) << 8));
         else
             store_atom<BLK>(a, row, k0 / BLK, st[0]);
+    }
+    if (a.sf_lanes != nullptr && lane_bytes) {
+        if (BLK == 16)   // the run's two adjacent 16-slots: one 16-bit store
+            *reinterpret_cast<uint16_t *>(lane_byte(a, row, k0 / 16)) =
+                static_cast<uint16_t>((st[0] & 0xFFu) | ((st[1] & 0xFFu) << 8));
+        else
+            store_lanes<BLK>(a, row, k0 / BLK, st[0]);
     }
 }
 
@@ -640,6 +680,7 @@ __device__ __forceinline__ void coop_exact(const QuantArgs &a, const uint8_t *ti
                 if (a.scale_fmt == 0) reinterpret_cast<uint32_t *>(a.scales)[at] = stv[ln];
                 else reinterpret_cast<uint8_t *>(a.scales)[at] = static_cast<uint8_t>(stv[ln]);
                 if (a.sf_atoms != nullptr) store_atom<BLK>(a, row, k0 / BLK + lane / BLK, stv[ln]);
+                if (a.sf_lanes != nullptr) store_lanes<BLK>(a, row, k0 / BLK + lane / BLK, stv[ln]);
             }
         }
     }
@@ -826,8 +867,13 @@ __device__ __forceinline__ void unit_part(const QuantArgs &q, const uint8_t *til
         uint32_t cw[8], st[64 / BLK];
         const bool risky = quant_thread<MAP, SWZ, NH, BLK, GRID, RND>(q, src, site, S, G, rG, gk, cw, st);
         if (!risky) {
-            store_run<BLK>(q, site.row_x, site.k_x, cw, st);
-            store_run<BLK>(q, site.row_y, site.k_y, cw + 4, st + 32 / BLK);
+            // Row map: both runs are one K step of one row, so the thread
+            // writes that row's whole per-lane factor record at once.
+            constexpr bool kRecord = MAP == MAP_ROW;
+            store_run<BLK>(q, site.row_x, site.k_x, cw, st, !kRecord);
+            store_run<BLK>(q, site.row_y, site.k_y, cw + 4, st + 32 / BLK, !kRecord);
+            if (kRecord && q.sf_lanes != nullptr && site.row_x < q.out_rows)
+                store_lane_record<BLK>(q, site.row_x, site.k_x, st);
         }
         const uint32_t owners = __ballot_sync(0xFFFFFFFFu, risky);
         if (owners != 0u) {

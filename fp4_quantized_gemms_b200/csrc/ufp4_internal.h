@@ -41,6 +41,8 @@ struct QuantArgs {
     uint8_t *elems8;     // E4M3 element plane [out_rows][kpad] (MX path), or nullptr
     uint8_t *sf_atoms;   // factor atoms [ceil(out_rows/128)][atoms_k][512], or nullptr
     int64_t atoms_k;     // atoms along K (kpad / 64 for E4M3 factors, kpad / 128 rounded up for UE8M0)
+    uint8_t *sf_lanes;   // per-lane factor tiles [ceil(out_rows/128)][lane_groups][4096], or nullptr
+    int64_t lane_groups; // 128-K groups along K (ceil(kpad / 128))
     void *scales;        // block-major [kpad/B][scale_ld], fp32 or E4M3
     float *S_out;        // two-level: receives S
     const float *amax_t; // two-level: rotated tensor amax
@@ -114,7 +116,10 @@ struct GemmArgs {
     int scale_ue8m0;                      // mode 0: scales are UE8M0 exponent bytes
     int planes3d;                         // corr = codes + rows * kpad / 2 for both
     CUtensorMap tm_a_e8, tm_b_e8;         // MX path: E4M3 element planes [rows][kpad]
-    CUtensorMap tm_a_atoms, tm_b_atoms;   // factor atoms as u64 [row groups][64 atoms_k]
+    CUtensorMap tm_a_atoms, tm_b_atoms;   // factor atoms as u64 [row groups][64 atoms_k]; for
+                                          // E1M2 the A map covers the per-lane tiles instead
+                                          // (u64 [tiles][2][256])
+    int32_t lane_groups;                  // per-lane tiles per 128-row group of A (E1M2)
     int atoms;                            // both operands carry factor atoms (pair kernels, dense)
     int band;                             // tile order: rows of tiles per band (0: M fastest)
 };
@@ -122,6 +127,18 @@ struct GemmArgs {
 // Tile columns (B rows) of the native block-scaled FP4 kernels (modes 3, 4).
 constexpr int kNativeTileN = 192;
 constexpr int kTileBand = 8;   // rows of output tiles per band of the GEMM tile order
+// Per-lane factor tiles (E1M2 operands with E4M3 factors): the A-operand
+// factors of 128 rows x 128 K in the image of one 128-lane x 256-bit tensor
+// memory copy.  Each 32-lane quarter q of the block-scaled MMA reads the
+// factors of its rows from column (factor base + q), and the factor base is
+// a multiple of 4 columns; with bases c and c + 4 for K steps 0 and 1, lane
+// L (row L of the group, q = L / 32) holds the four factors of K step j in
+// column c + 4 j + q.  One copy then serves both K steps, where the
+// factor atoms (32 rows, copied to every quarter) take one copy each.
+// Tile layout: two halves of 2048 bytes (K steps 0 and 1), lane L's 16
+// bytes of a half at 16 L, the factors at bytes 4 q .. 4 q + 3 of them.
+constexpr int kLaneK = 128;
+constexpr int kLaneTileBytes = 4096;
 // K elements per pipeline stage of the CTA-pair kernels: 256 for E2M1
 // operands with factor atoms (one MMA per 64 K: a longer stage spreads the
 // issuer's per-stage waits, fences and commits over more MMAs), else 128.
@@ -139,6 +156,10 @@ CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, const
                               uint64_t inner, uint64_t outer, uint64_t row_bytes,
                               uint32_t box_inner, uint32_t box_outer,
                               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE);
+// 3-D map without swizzle: dims innermost first, strides of dims 1 and 2 in bytes.
+CUresult encode_tensor_map_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base,
+                              const cuuint64_t (&dims)[3], const cuuint64_t (&strides)[2],
+                              const cuuint32_t (&box)[3]);
 // u8 planes [planes][outer][inner] (plane_bytes apart), boxes of every plane.
 CUresult encode_tensor_map_planes(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
                                   uint64_t planes, uint64_t plane_bytes, uint32_t box_inner,

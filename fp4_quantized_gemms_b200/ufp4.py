@@ -195,7 +195,8 @@ class QTensor:
     cfg: QuantConfig
     corr: torch.Tensor | None = None    # uint8 [rows, kpad/2]: E1M2 correction plane
     elems8: torch.Tensor | None = None  # uint8 [rows, kpad]: E4M3 element plane (MX path)
-    sf_atoms: torch.Tensor | None = None  # uint8 [ceil(rows/128), atoms_k, 512]: factor atoms
+    sf_atoms: torch.Tensor | None = None  # uint8 [bytes]: factor atoms [ceil(rows/128), atoms_k, 512]
+                                          # (E1M2 with E4M3 factors: then per-lane tiles)
 
     def c(self) -> QTensorC:
         return QTensorC(self.codes.data_ptr(), self.scales.data_ptr(),
@@ -256,8 +257,8 @@ def empty_qtensor(rows: int, k: int, cfg: QuantConfig, device="cuda",
         with_atoms = wants_atoms(cfg)
     atoms = None
     if with_atoms:
-        ak, _ = sf_atoms_layout(rows, k, cfg)
-        atoms = torch.empty(((rows + 127) // 128, ak, 512), dtype=torch.uint8, device=device)
+        _, nbytes = sf_atoms_layout(rows, k, cfg)
+        atoms = torch.empty(nbytes, dtype=torch.uint8, device=device)
     return QTensor(codes, scales, ts, rows, k, kpad, sld, cfg, corr, e8, atoms)
 
 

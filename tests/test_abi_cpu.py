@@ -98,18 +98,22 @@ def test_layout(L, k, block, fmt, kpad, codes, scales):
     assert ufp4.layout(300, 64, cfg)[1] == 320
 
 
-@pytest.mark.parametrize("rows,k,block,fmt,atoms_k,nbytes", [
-    (256, 512, 16, ufp4.SCALE_E4M3_X_FP32, 8, 2 * 8 * 512),
-    (300, 200, 32, ufp4.SCALE_E4M3_X_FP32, 4, 3 * 4 * 512),     # kpad 256: 16 slots of 16
-    (129, 1000, 32, ufp4.SCALE_UE8M0, 8, 2 * 8 * 512),          # kpad 1024: 32 slots of 32
-    (1, 136, 32, ufp4.SCALE_UE8M0, 2, 1 * 2 * 512),             # kpad 192: 6 slots, 2 atoms
-    (0, 64, 16, ufp4.SCALE_E4M3_X_FP32, 1, 0),
+@pytest.mark.parametrize("rows,k,block,fmt,grid,atoms_k,nbytes", [
+    # E1M2 with E4M3 factors: atoms, then ceil(rows/128) x ceil(kpad/128) per-lane factor tiles of 4096 bytes
+    (256, 512, 16, ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E1M2, 8, 2 * 8 * 512 + 2 * 4 * 4096),
+    (300, 200, 32, ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E1M2, 4, 3 * 4 * 512 + 3 * 2 * 4096),   # kpad 256
+    (130, 64, 16, ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E1M2, 1, 2 * 1 * 512 + 2 * 1 * 4096),    # kpad 64: half a tile
+    (256, 512, 16, ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E2M1, 8, 2 * 8 * 512),                  # E2M1: atoms only
+    (129, 1000, 32, ufp4.SCALE_UE8M0, ufp4.GRID_E1M2, 8, 2 * 8 * 512),          # kpad 1024: 32 slots of 32
+    (1, 136, 32, ufp4.SCALE_UE8M0, ufp4.GRID_E1M2, 2, 1 * 2 * 512),             # kpad 192: 6 slots, 2 atoms
+    (0, 64, 16, ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E1M2, 1, 0),
 ])
-def test_sf_atoms_layout(L, rows, k, block, fmt, atoms_k, nbytes):
+def test_sf_atoms_layout(L, rows, k, block, fmt, grid, atoms_k, nbytes):
     """Factor-atom plane size: ceil(rows/128) row groups x ceil(kpad / 4W)
-    atoms of 512 bytes (W = 16 for E4M3 factors, 32 for UE8M0); none for
-    fp32 scales."""
-    cfg = ufp4.QuantConfig(block=block, scale_fmt=fmt)
+    atoms of 512 bytes (W = 16 for E4M3 factors, 32 for UE8M0), followed for
+    E1M2 operands with E4M3 factors by ceil(rows/128) x ceil(kpad/128)
+    per-lane factor tiles of 4096 bytes; none for fp32 scales."""
+    cfg = ufp4.QuantConfig(block=block, scale_fmt=fmt, grid=grid)
     assert ufp4.sf_atoms_layout(rows, k, cfg) == (atoms_k, nbytes)
     c = ufp4.QuantConfig(scale_fmt=ufp4.SCALE_FP32).c()
     assert L.ufp4_sf_atoms_layout(64, 64, ctypes.byref(c), None, None) == ufp4.ERR_UNSUPPORTED
