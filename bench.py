@@ -173,12 +173,13 @@ class LayerStep:
         self.X, self.W, self.dY = inputs
         C, R = ufp4.ALONG_COLS, ufp4.ALONG_ROWS
         E = ufp4.empty_qtensor
-        self.qx = E(s.M, s.K, self.c_rtne, device)        # FPROP A
-        self.qw = E(s.N, s.K, self.c_rtne, device)        # FPROP B
-        self.qdy = E(s.M, s.N, self.c_sr0, device)        # DGRAD A
-        self.qwt = E(s.K, s.N, self.c_rtne, device)       # DGRAD B
-        self.qdyt = E(s.N, s.M, self.c_sr1, device)       # WGRAD A
-        self.qxt = E(s.K, s.M, self.c_rtne, device)       # WGRAD B
+        # Per-lane factor tiles only on the GEMMs' first operands.
+        self.qx = E(s.M, s.K, self.c_rtne, device)                    # FPROP A
+        self.qw = E(s.N, s.K, self.c_rtne, device, with_lanes=False)  # FPROP B
+        self.qdy = E(s.M, s.N, self.c_sr0, device)                    # DGRAD A
+        self.qwt = E(s.K, s.N, self.c_rtne, device, with_lanes=False)  # DGRAD B
+        self.qdyt = E(s.N, s.M, self.c_sr1, device)                   # WGRAD A
+        self.qxt = E(s.K, s.M, self.c_rtne, device, with_lanes=False)  # WGRAD B
         # Each tensor feeds two GEMMs, one along each axis: one quantization
         # call per operand (two single-output calls measured faster than the
         # dual-output pass at these sizes).  The rotated amaxes of all six

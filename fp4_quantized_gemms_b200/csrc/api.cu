@@ -84,15 +84,15 @@ int64_t atoms_k_of(int64_t kpad, const ufp4_quant_cfg_t &c) {
     return (kpad + w - 1) / w;
 }
 
-// E1M2 operands with E4M3 factors carry per-lane factor tiles after their
-// factor atoms (the A-operand factor layout of the CTA-pair kernel).
+// E1M2 operands with E4M3 factors may carry per-lane factor tiles (the
+// A-operand factor layout of the CTA-pair kernel).
 bool has_lane_tiles(const ufp4_quant_cfg_t &c) {
     return c.grid == UFP4_GRID_E1M2 && c.scale_fmt == UFP4_SCALE_E4M3_X_FP32;
 }
 
 int64_t lane_groups_of(int64_t kpad) { return (kpad + kLaneK - 1) / kLaneK; }
 
-// Bytes of the factor atoms proper (the per-lane tiles follow them).
+// Bytes of the factor atoms.
 int64_t atom_bytes_of(int64_t rows, int64_t kpad, const ufp4_quant_cfg_t &c) {
     return (rows + 127) / 128 * atoms_k_of(kpad, c) * 512;
 }
@@ -120,6 +120,10 @@ ufp4_status_t check_qtensor(const ufp4_qtensor_t *q) {
     if (q->sf_atoms != nullptr) {   // factor atoms: byte block scales only
         if (atom_slot(q->cfg) == 0) return UFP4_ERR_INVALID_ARG;
         if (!aligned16(q->sf_atoms)) return UFP4_ERR_ALIGNMENT;
+    }
+    if (q->sf_lanes != nullptr) {   // per-lane factor tiles: E1M2 with E4M3 factors only
+        if (!has_lane_tiles(q->cfg)) return UFP4_ERR_INVALID_ARG;
+        if (!aligned16(q->sf_lanes)) return UFP4_ERR_ALIGNMENT;
     }
     if (q->rows > (int64_t(1) << 31) || q->kpad > (int64_t(1) << 31)) return UFP4_ERR_UNSUPPORTED;
     return UFP4_OK;
@@ -316,16 +320,17 @@ ufp4_status_t run_gemm(const ufp4_qtensor_t *a, const ufp4_qtensor_t *b,
         const int64_t ak = atoms_k_of(a->kpad, a->cfg), bk = atoms_k_of(b->kpad, b->cfg);
         const uint32_t box_k = static_cast<uint32_t>(64 * (k_stage / (4 * atom_slot(a->cfg))));
         CUresult r;
-        if (mode == 5 && grid_kind == 0) {
-            // E1M2: the A factors come as per-lane tiles (one 4 KB box per
-            // 128 rows and 128 K), u64 [tiles][2 halves][256]
+        if (mode == 5 && grid_kind == 0 && a->sf_lanes != nullptr) {
+            // E1M2 with per-lane tiles on A: one 4 KB box per 128 rows and
+            // 128 K, u64 [tiles][2 halves][256]
             const int64_t sg = lane_groups_of(a->kpad);
-            const uint8_t *base = static_cast<const uint8_t *>(a->sf_atoms) + atom_bytes_of(a->rows, a->kpad, a->cfg);
+            const uint8_t *base = static_cast<const uint8_t *>(a->sf_lanes);
             const cuuint64_t dims[3] = {256, 2, static_cast<cuuint64_t>((a->rows + 127) / 128 * sg)};
             const cuuint64_t strides[2] = {2048, kLaneTileBytes};
             const cuuint32_t box[3] = {256, 2, 1};
             r = encode_tensor_map_3d(&args.tm_a_atoms, CU_TENSOR_MAP_DATA_TYPE_UINT64, base, dims, strides, box);
             args.lane_groups = static_cast<int32_t>(sg);
+            args.lanes = 1;
         } else {
             r = encode_tensor_map_2d(&args.tm_a_atoms, CU_TENSOR_MAP_DATA_TYPE_UINT64, a->sf_atoms,
                                      static_cast<uint64_t>(64 * ak), static_cast<uint64_t>((a->rows + 127) / 128),
@@ -385,8 +390,8 @@ ufp4_status_t fill_quant_args(const void *x_dev, int64_t rows, int64_t cols, int
     a->elems8 = static_cast<uint8_t *>(out->elems8);
     a->sf_atoms = static_cast<uint8_t *>(out->sf_atoms);
     a->atoms_k = out->sf_atoms != nullptr ? atoms_k_of(out->kpad, out->cfg) : 0;
-    if (out->sf_atoms != nullptr && has_lane_tiles(out->cfg)) {
-        a->sf_lanes = static_cast<uint8_t *>(out->sf_atoms) + atom_bytes_of(out_rows, out->kpad, out->cfg);
+    if (out->sf_lanes != nullptr) {
+        a->sf_lanes = static_cast<uint8_t *>(out->sf_lanes);
         a->lane_groups = lane_groups_of(out->kpad);
     }
     a->scales = out->scales;
@@ -481,10 +486,14 @@ ufp4_status_t ufp4_sf_atoms_layout(int64_t rows, int64_t k, const ufp4_quant_cfg
     if (atom_slot(*cfg) == 0) return UFP4_ERR_UNSUPPORTED;
     const int64_t ak = atoms_k_of(round_up(k, kKAlign), *cfg);
     if (atoms_k) *atoms_k = ak;
-    const int64_t kp = round_up(k, kKAlign);
-    int64_t nb = atom_bytes_of(rows, kp, *cfg);
-    if (has_lane_tiles(*cfg)) nb += (rows + 127) / 128 * lane_groups_of(kp) * kLaneTileBytes;
-    if (bytes) *bytes = static_cast<size_t>(nb);
+    if (bytes) *bytes = static_cast<size_t>(atom_bytes_of(rows, round_up(k, kKAlign), *cfg));
+    return UFP4_OK;
+}
+
+ufp4_status_t ufp4_sf_lanes_layout(int64_t rows, int64_t k, const ufp4_quant_cfg_t *cfg, size_t *bytes) {
+    if (cfg == nullptr || bytes == nullptr || rows < 0 || k < 0 || !cfg_valid(*cfg)) return UFP4_ERR_INVALID_ARG;
+    if (!has_lane_tiles(*cfg)) return UFP4_ERR_UNSUPPORTED;
+    *bytes = static_cast<size_t>((rows + 127) / 128 * lane_groups_of(round_up(k, kKAlign)) * kLaneTileBytes);
     return UFP4_OK;
 }
 

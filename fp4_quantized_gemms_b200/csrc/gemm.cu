@@ -1147,7 +1147,7 @@ __global__ void __launch_bounds__(Fp4Cfg<GRID, CIN>::kThreads, 1)
 // byte per element, 128-byte rows, 128-byte swizzle), UE8M0 factors per 32
 // elements applied in the MMA (kind::mxf8f6f4, K = 32 per MMA, four MMAs per
 // stage picking byte j of the same factor atom).
-template <int GRID, bool ATOMS>
+template <int GRID, bool ATOMS, bool LANES = false>
 struct PairCfg {
     static constexpr bool kMx = GRID == 3;
     static constexpr int TM = 256;
@@ -1161,9 +1161,9 @@ struct PairCfg {
     static constexpr int o_b = kPlanes * kTile;     // [codes | corr] of this CTA's B half
     static constexpr int kCodeBytes = 2 * kPlanes * kTile;   // per CTA per stage
     static constexpr int kRawRows = kMx ? BKE / 32 : BKE / 16;   // factor rows per stage (most)
-    // E1M2 with factor atoms: the A factors of a stage arrive as one
-    // per-lane tile (4 KB) and leave for TMEM in one copy.
-    static constexpr bool kLaneA = GRID == 0 && ATOMS;
+    // E1M2 with factor atoms and per-lane tiles on A: the A factors of a
+    // stage arrive as one per-lane tile (4 KB) and leave for TMEM in one copy.
+    static constexpr bool kLaneA = GRID == 0 && ATOMS && LANES;
     static constexpr int o_raw_a = kCodeBytes;      // raw factors: [blocks][128 rows]
     static constexpr int kRawA = kLaneA ? kLaneTileBytes : 128 * kRawRows;
     static constexpr int o_raw_b = o_raw_a + kRawA; // [blocks][256 rows]
@@ -1318,10 +1318,10 @@ __device__ __forceinline__ void store_piece(const GemmArgs &args, const Tile &tl
     }
 }
 
-template <int GRID, bool ATOMS>
-__global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
+template <int GRID, bool ATOMS, bool LANES>
+__global__ void __launch_bounds__(PairCfg<GRID, ATOMS, LANES>::kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ GemmArgs args) {
-    using C = PairCfg<GRID, ATOMS>;
+    using C = PairCfg<GRID, ATOMS, LANES>;
     constexpr int TM = C::TM, BN = C::BN, NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -1705,12 +1705,12 @@ __global__ void __launch_bounds__(PairCfg<GRID, ATOMS>::kThreads, 1)
     }
 }
 
-template <int GRID, bool ATOMS>
+template <int GRID, bool ATOMS, bool LANES = false>
 cudaError_t launch_pair(const GemmArgs &args, int num_sms, cudaStream_t stream) {
-    using C = PairCfg<GRID, ATOMS>;
+    using C = PairCfg<GRID, ATOMS, LANES>;
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<GRID, ATOMS>,
+        cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<GRID, ATOMS, LANES>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc);
         if (e != cudaSuccess) return e;
         configured = true;
@@ -1734,7 +1734,7 @@ cudaError_t launch_pair(const GemmArgs &args, int num_sms, cudaStream_t stream) 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<GRID, ATOMS>, args);
+    return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<GRID, ATOMS, LANES>, args);
 }
 
 template <int GRID, bool CIN>
@@ -1799,7 +1799,8 @@ cudaError_t launch_gemm(const GemmArgs &args, int mode, int grid_kind, int num_s
         case 5:
             if (args.atoms)
                 return grid_kind == 1 ? launch_pair<1, true>(args, num_sms, stream)
-                                      : launch_pair<0, true>(args, num_sms, stream);
+                                      : (args.lanes ? launch_pair<0, true, true>(args, num_sms, stream)
+                                                    : launch_pair<0, true, false>(args, num_sms, stream));
             return grid_kind == 1 ? launch_pair<1, false>(args, num_sms, stream)
                                   : launch_pair<0, false>(args, num_sms, stream);
         case 6:

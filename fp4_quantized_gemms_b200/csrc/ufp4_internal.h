@@ -120,6 +120,7 @@ struct GemmArgs {
                                           // E1M2 the A map covers the per-lane tiles instead
                                           // (u64 [tiles][2][256])
     int32_t lane_groups;                  // per-lane tiles per 128-row group of A (E1M2)
+    int lanes;                            // A carries per-lane factor tiles (E1M2 pair kernel)
     int atoms;                            // both operands carry factor atoms (pair kernels, dense)
     int band;                             // tile order: rows of tiles per band (0: M fastest)
 };

@@ -32,7 +32,7 @@ EXPORTED = [
     "ufp4_status_string", "ufp4_version", "ufp4_set_two_level_gemm_path",
     "ufp4_get_two_level_gemm_path", "ufp4_rht_quantize_dual", "ufp4_rht_amax_dual",
     "ufp4_quant_stats", "ufp4_qstats_summarize", "ufp4_sqnr_sums", "ufp4_rht_bf16",
-    "ufp4_sf_atoms_layout", "ufp4_test_set_quantize_wait_limit",
+    "ufp4_sf_atoms_layout", "ufp4_sf_lanes_layout", "ufp4_test_set_quantize_wait_limit",
 ]
 
 
@@ -54,7 +54,7 @@ class QTensorC(ctypes.Structure):
                 ("tensor_scale", ctypes.c_void_p), ("rows", ctypes.c_int64),
                 ("k", ctypes.c_int64), ("kpad", ctypes.c_int64), ("scale_ld", ctypes.c_int64),
                 ("cfg", QuantCfgC), ("corr", ctypes.c_void_p), ("elems8", ctypes.c_void_p),
-                ("sf_atoms", ctypes.c_void_p)]
+                ("sf_atoms", ctypes.c_void_p), ("sf_lanes", ctypes.c_void_p)]
 
 
 class GroupC(ctypes.Structure):
@@ -123,6 +123,8 @@ def lib() -> ctypes.CDLL:
         L.ufp4_sf_atoms_layout.restype = st
         L.ufp4_sf_atoms_layout.argtypes = [i64, i64, ctypes.POINTER(QuantCfgC), ctypes.POINTER(i64),
                                            ctypes.POINTER(ctypes.c_size_t)]
+        L.ufp4_sf_lanes_layout.restype = st
+        L.ufp4_sf_lanes_layout.argtypes = [i64, i64, ctypes.POINTER(QuantCfgC), ctypes.POINTER(ctypes.c_size_t)]
         L.ufp4_test_set_quantize_wait_limit.restype = st
         L.ufp4_test_set_quantize_wait_limit.argtypes = [u64]
         L.ufp4_set_two_level_gemm_path.restype = st
@@ -195,8 +197,9 @@ class QTensor:
     cfg: QuantConfig
     corr: torch.Tensor | None = None    # uint8 [rows, kpad/2]: E1M2 correction plane
     elems8: torch.Tensor | None = None  # uint8 [rows, kpad]: E4M3 element plane (MX path)
-    sf_atoms: torch.Tensor | None = None  # uint8 [bytes]: factor atoms [ceil(rows/128), atoms_k, 512]
-                                          # (E1M2 with E4M3 factors: then per-lane tiles)
+    sf_atoms: torch.Tensor | None = None  # uint8 [ceil(rows/128), atoms_k, 512]: factor atoms
+    sf_lanes: torch.Tensor | None = None  # uint8 [ceil(rows/128), ceil(kpad/128), 4096]: per-lane
+                                          # factor tiles of a first GEMM operand (E1M2, E4M3 factors)
 
     def c(self) -> QTensorC:
         return QTensorC(self.codes.data_ptr(), self.scales.data_ptr(),
@@ -204,7 +207,8 @@ class QTensor:
                         self.rows, self.k, self.kpad, self.scale_ld, self.cfg.c(),
                         self.corr.data_ptr() if self.corr is not None else None,
                         self.elems8.data_ptr() if self.elems8 is not None else None,
-                        self.sf_atoms.data_ptr() if self.sf_atoms is not None else None)
+                        self.sf_atoms.data_ptr() if self.sf_atoms is not None else None,
+                        self.sf_lanes.data_ptr() if self.sf_lanes is not None else None)
 
 
 def wants_corr(cfg: QuantConfig) -> bool:
@@ -223,6 +227,21 @@ def wants_atoms(cfg: QuantConfig) -> bool:
     return cfg.scale_fmt != SCALE_FP32
 
 
+def wants_lanes(cfg: QuantConfig) -> bool:
+    """E1M2 operands with E4M3 factors: per-lane factor tiles save the
+    CTA-pair GEMM a tensor-memory copy per stage when the operand is its
+    first (A) operand."""
+    return cfg.grid == GRID_E1M2 and cfg.scale_fmt == SCALE_E4M3_X_FP32
+
+
+def sf_lanes_layout(rows: int, k: int, cfg: QuantConfig) -> int:
+    """Bytes of the per-lane factor tiles of a [rows, k] operand."""
+    nb = ctypes.c_size_t()
+    c = cfg.c()
+    _check(lib().ufp4_sf_lanes_layout(rows, k, ctypes.byref(c), ctypes.byref(nb)), "ufp4_sf_lanes_layout")
+    return nb.value
+
+
 def sf_atoms_layout(rows: int, k: int, cfg: QuantConfig) -> tuple[int, int]:
     """(atoms_k, bytes) of the factor-atom plane of a [rows, k] operand."""
     ak, nb = ctypes.c_int64(), ctypes.c_size_t()
@@ -234,7 +253,12 @@ def sf_atoms_layout(rows: int, k: int, cfg: QuantConfig) -> tuple[int, int]:
 
 def empty_qtensor(rows: int, k: int, cfg: QuantConfig, device="cuda",
                   with_corr: bool | None = None, with_elems8: bool | None = None,
-                  with_atoms: bool | None = None) -> QTensor:
+                  with_atoms: bool | None = None, with_lanes: bool | None = None) -> QTensor:
+    """Device buffers of a quantized operand.  The optional planes default
+    to what the GEMMs use: the correction plane and per-lane factor tiles
+    for E1M2 operands with two-level scales, the element plane for MX
+    operands, factor atoms for byte block scales.  Pass with_lanes=False for
+    an operand that is only ever a GEMM's second operand."""
     kpad, sld, _, _ = layout(rows, k, cfg)
     nblk = kpad // cfg.block
     if with_corr is None:
@@ -257,9 +281,15 @@ def empty_qtensor(rows: int, k: int, cfg: QuantConfig, device="cuda",
         with_atoms = wants_atoms(cfg)
     atoms = None
     if with_atoms:
-        _, nbytes = sf_atoms_layout(rows, k, cfg)
-        atoms = torch.empty(nbytes, dtype=torch.uint8, device=device)
-    return QTensor(codes, scales, ts, rows, k, kpad, sld, cfg, corr, e8, atoms)
+        ak, _ = sf_atoms_layout(rows, k, cfg)
+        atoms = torch.empty(((rows + 127) // 128, ak, 512), dtype=torch.uint8, device=device)
+    if with_lanes is None:
+        with_lanes = wants_lanes(cfg) and atoms is not None
+    lanes = None
+    if with_lanes:
+        lanes = torch.empty(((rows + 127) // 128, -(-kpad // 128), 4096), dtype=torch.uint8, device=device)
+        assert lanes.numel() == sf_lanes_layout(rows, k, cfg)
+    return QTensor(codes, scales, ts, rows, k, kpad, sld, cfg, corr, e8, atoms, lanes)
 
 
 # ---------------------------------------------------------------- entry points
@@ -295,18 +325,19 @@ def rht_bf16(x: torch.Tensor, hadamard_n: int, sign_mask: int = DEFAULT_SIGN_MAS
 def rht_quantize(x: torch.Tensor, axis: int, cfg: QuantConfig,
                  tensor_amax: torch.Tensor | None = None, out: QTensor | None = None,
                  with_corr: bool | None = None, with_elems8: bool | None = None,
-                 with_atoms: bool | None = None) -> QTensor:
+                 with_atoms: bool | None = None, with_lanes: bool | None = None) -> QTensor:
     """Fused RHT + block scale + 4-bit rounding + packing of a bf16 operand
     (plus the E1M2 correction plane when with_corr, by default for E1M2
     operands with two-level scales; the MX element plane; factor atoms, by
-    default for byte block scales)."""
+    default for byte block scales; per-lane factor tiles, by default with
+    the correction plane's operands)."""
     _require_cuda(x, tensor_amax)
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     rows, cols = x.shape
     orows, k = (rows, cols) if axis == ALONG_COLS else (cols, rows)
     if out is None:
         out = empty_qtensor(orows, k, cfg, device=x.device, with_corr=with_corr, with_elems8=with_elems8,
-                            with_atoms=with_atoms)
+                            with_atoms=with_atoms, with_lanes=with_lanes)
     if cfg.scale_fmt == SCALE_E4M3_X_FP32 and tensor_amax is None:
         tensor_amax = rht_amax(x, axis, cfg.hadamard_n, cfg.rht_sign_mask)
     qc = out.c()

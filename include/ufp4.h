@@ -81,20 +81,28 @@
  *             ceil(kpad / (4 W)); byte 16 (r % 32) + 4 ((r / 32) % 4) + s % 4
  *             of atom (r / 128, s / 4) holds the factor of slot s of row r.
  *             Bytes of rows >= rows and of slots at or beyond kpad / W are
- *             not written and feed no stored GEMM output.  E1M2 operands
- *             with E4M3 factors carry, right after the atoms, the same
- *             factors as per-lane tiles: u8 [ceil(rows/128)][ceil(kpad/128)]
- *             [4096], the factor of slot s of row r at byte
- *             2048 ((s / 4) % 2) + 16 L + 4 (L / 32) + s % 4 of tile
- *             (r / 128, s / 8) with L = r % 128 (the tensor-memory image of
- *             one 128-lane copy that holds the factors of two K steps, which
- *             the CTA-pair GEMM uses for its first operand); other bytes are
- *             not written and not read by the MMA.  ufp4_sf_atoms_layout gives atoms_k and the size
- *             of both parts.  ufp4_rht_quantize writes it when
+ *             not written and feed no stored GEMM output.  ufp4_sf_atoms_layout
+ *             gives atoms_k and the size.  ufp4_rht_quantize writes it when
  *             non-NULL; when both operands of a dense GEMM on a CTA-pair path
  *             carry one, the MMA issuer copies each stage's factors into
  *             tensor memory itself (no factor-building warps).  Must be NULL
  *             for fp32 scales.  16-byte aligned.
+ *   sf_lanes  optional, E1M2 with E4M3 x fp32 scales only: the same factors
+ *             once more, as per-lane tiles for the first operand (A) of a
+ *             CTA-pair GEMM: u8 [ceil(rows/128)][ceil(kpad/128)][4096], the
+ *             factor of slot s (16 elements) of row r at byte
+ *             2048 ((s / 4) % 2) + 16 L + 4 (L / 32) + s % 4 of tile
+ *             (r / 128, s / 8), L = r % 128.  A tile is the tensor-memory
+ *             image of one 128-lane copy holding the factors of two 64-K
+ *             steps (a hardware layout, not part of the method); the other
+ *             bytes of a lane's 16 are zero or not written.  Factor atoms
+ *             reach each 32-lane quarter by a broadcast copy per K step, so
+ *             an A operand that carries these tiles saves one copy per stage.
+ *             ufp4_rht_quantize writes it when non-NULL (with sf_atoms, it
+ *             costs a few percent of a quantization); a dense GEMM uses it
+ *             when A carries it and both operands carry factor atoms, and
+ *             ignores it on B.  ufp4_sf_lanes_layout gives the size.  16-byte
+ *             aligned.
  */
 #ifndef UFP4_H
 #define UFP4_H
@@ -174,6 +182,7 @@ typedef struct {
     void *corr;             /* device u8 [rows][kpad/2] or NULL, see above   */
     void *elems8;           /* device u8 [rows][kpad] or NULL, see above     */
     void *sf_atoms;         /* device u8 factor atoms or NULL, see above     */
+    void *sf_lanes;         /* device u8 per-lane factor tiles or NULL, see above */
 } ufp4_qtensor_t;
 
 /* One sub-problem of ufp4_grouped_gemm:
@@ -199,13 +208,17 @@ ufp4_status_t ufp4_qtensor_layout(int64_t rows, int64_t k, const ufp4_quant_cfg_
 
 /* Size of the optional factor-atom plane (sf_atoms) of a quantized operand:
  * atoms_k = ceil(kpad / (4 W)) atoms along K (W = 16 for E4M3 x fp32 scales,
- * 32 for UE8M0), bytes = ceil(rows / 128) * atoms_k * 512, plus
- * ceil(rows / 128) * ceil(kpad / 128) * 4096 for the per-lane tiles of E1M2
- * operands with E4M3 factors.  Either output may
+ * 32 for UE8M0), bytes = ceil(rows / 128) * atoms_k * 512.  Either output may
  * be NULL.  Errors: INVALID_ARG (rows < 0, k < 0, bad cfg), UNSUPPORTED (fp32
  * scales: no atoms). */
 ufp4_status_t ufp4_sf_atoms_layout(int64_t rows, int64_t k, const ufp4_quant_cfg_t *cfg, int64_t *atoms_k,
                                    size_t *bytes);
+
+/* Size of the optional per-lane factor tiles (sf_lanes) of an E1M2 operand
+ * with E4M3 x fp32 scales: bytes = ceil(rows / 128) * ceil(kpad / 128) * 4096.
+ * Errors: INVALID_ARG (rows < 0, k < 0, bad cfg, bytes NULL), UNSUPPORTED
+ * (another grid or scale format: no tiles). */
+ufp4_status_t ufp4_sf_lanes_layout(int64_t rows, int64_t k, const ufp4_quant_cfg_t *cfg, size_t *bytes);
 
 /* Absolute maximum of the rotated operand, max |H_n D x| over all elements
  * (the tensor amax that the two-level scale S is derived from; [PL] §2

@@ -91,25 +91,21 @@ def atoms_logical(q: ufp4.QTensor, rows=None) -> np.ndarray:
     w = 32 if q.cfg.scale_fmt == ufp4.SCALE_UE8M0 else 16
     slots = q.kpad // w
     r = np.arange(q.rows) if rows is None else np.asarray(rows)
-    ak = -(-q.kpad // (4 * w))
-    a = q.sf_atoms.cpu().numpy()[:((q.rows + 127) // 128) * ak * 512].reshape(-1, ak, 512)
+    a = q.sf_atoms.cpu().numpy()
     s = np.arange(slots)
     byte = (16 * (r % 32) + 4 * ((r // 32) % 4))[:, None] + (s % 4)[None, :]
     return a[(r // 128)[:, None], (s // 4)[None, :], byte]
 
 
 def lane_tiles_logical(q: ufp4.QTensor, rows=None) -> np.ndarray:
-    """Per-lane factor tiles of an E1M2 operand with E4M3 factors (after the
-    atoms: [ceil(rows/128)][ceil(kpad/128)][4096]) -> [rows, slots]: the
+    """Per-lane factor tiles of an E1M2 operand with E4M3 factors
+    ([ceil(rows/128)][ceil(kpad/128)][4096]) -> [rows, slots]: the
     factor of 16-slot s of row r is byte 2048 ((s / 4) % 2) + 16 L + 4 (L / 32)
     + s % 4 of tile (r / 128, s / 8), L = r % 128 (tensor-memory column
     4 ((s / 4) % 2) + L / 32 of lane L after one 128-lane copy)."""
     slots = q.kpad // 16
     r = np.arange(q.rows) if rows is None else np.asarray(rows)
-    ak = -(-q.kpad // 64)
-    groups = -(-q.kpad // 128)
-    nrb = (q.rows + 127) // 128
-    t = q.sf_atoms.cpu().numpy()[nrb * ak * 512:].reshape(nrb, groups, 4096)
+    t = q.sf_lanes.cpu().numpy()
     s = np.arange(slots)
     L = (r % 128)[:, None]
     byte = 2048 * ((s // 4) % 2)[None, :] + 16 * L + 4 * (L // 32) + (s % 4)[None, :]
@@ -149,13 +145,14 @@ def assert_quant_equal(q: ufp4.QTensor, ref: oracle.QTensor, rows=None):
             r, c = bad[0]
             raise AssertionError(f"{len(bad)} factor-atom bytes differ; first at (row {r}, slot {c}): gpu "
                                  f"{got_a[r, c]:#x} expected {want_a[r, c]:#x}")
-        if q.cfg.grid == ufp4.GRID_E1M2 and q.cfg.scale_fmt == ufp4.SCALE_E4M3_X_FP32:
-            got_s = lane_tiles_logical(q, rows)
-            if not np.array_equal(got_s, want_a):
-                bad = np.argwhere(got_s != want_a)
-                r, c = bad[0]
-                raise AssertionError(f"{len(bad)} per-lane tile factor bytes differ; first at (row {r}, slot {c}): "
-                                     f"gpu {got_s[r, c]:#x} expected {want_a[r, c]:#x}")
+    if q.sf_lanes is not None:
+        want_l = ref.escales[:, (np.arange(q.kpad // 16) * 16) // q.cfg.block]
+        got_l = lane_tiles_logical(q, rows)
+        if not np.array_equal(got_l, want_l):
+            bad = np.argwhere(got_l != want_l)
+            r, c = bad[0]
+            raise AssertionError(f"{len(bad)} per-lane tile factor bytes differ; first at (row {r}, slot {c}): "
+                                 f"gpu {got_l[r, c]:#x} expected {want_l[r, c]:#x}")
     sc = logical_scales(q, rows)
     if ref.scales is not None:
         assert np.array_equal(sc.view(np.uint32), ref.scales.view(np.uint32)), "fp32 scales differ"

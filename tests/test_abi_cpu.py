@@ -51,9 +51,10 @@ def test_struct_layouts_match_header(tmp_path):
 int main(void) {
   printf("%zu %zu %zu %zu %zu\\n", sizeof(ufp4_quant_cfg_t), offsetof(ufp4_quant_cfg_t, sr_seed),
          offsetof(ufp4_quant_cfg_t, rht_sign_mask), offsetof(ufp4_quant_cfg_t, scale_fmt), 0);
-  printf("%zu %zu %zu %zu %zu %zu %zu\\n", sizeof(ufp4_qtensor_t), offsetof(ufp4_qtensor_t, rows),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(ufp4_qtensor_t), offsetof(ufp4_qtensor_t, rows),
          offsetof(ufp4_qtensor_t, scale_ld), offsetof(ufp4_qtensor_t, cfg),
-         offsetof(ufp4_qtensor_t, corr), offsetof(ufp4_qtensor_t, elems8), offsetof(ufp4_qtensor_t, sf_atoms));
+         offsetof(ufp4_qtensor_t, corr), offsetof(ufp4_qtensor_t, elems8), offsetof(ufp4_qtensor_t, sf_atoms),
+         offsetof(ufp4_qtensor_t, sf_lanes));
   printf("%zu %zu\\n", sizeof(ufp4_group_t), offsetof(ufp4_group_t, c_col));
   printf("%zu %zu %zu %zu %zu\\n", sizeof(ufp4_qstats_t), offsetof(ufp4_qstats_t, level_n),
          offsetof(ufp4_qstats_t, code_count), offsetof(ufp4_qstats_t, underflow),
@@ -74,7 +75,7 @@ int main(void) {
                   ctypes.sizeof(Sm)]
     assert c1[:4] == [ctypes.sizeof(Q), Q.sr_seed.offset, Q.rht_sign_mask.offset, Q.scale_fmt.offset]
     assert c2 == [ctypes.sizeof(T), T.rows.offset, T.scale_ld.offset, T.cfg.offset, T.corr.offset,
-                  T.elems8.offset, T.sf_atoms.offset]
+                  T.elems8.offset, T.sf_atoms.offset, T.sf_lanes.offset]
     assert c3 == [ctypes.sizeof(G), G.c_col.offset]
 
 
@@ -98,28 +99,49 @@ def test_layout(L, k, block, fmt, kpad, codes, scales):
     assert ufp4.layout(300, 64, cfg)[1] == 320
 
 
-@pytest.mark.parametrize("rows,k,block,fmt,grid,atoms_k,nbytes", [
-    # E1M2 with E4M3 factors: atoms, then ceil(rows/128) x ceil(kpad/128) per-lane factor tiles of 4096 bytes
-    (256, 512, 16, ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E1M2, 8, 2 * 8 * 512 + 2 * 4 * 4096),
-    (300, 200, 32, ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E1M2, 4, 3 * 4 * 512 + 3 * 2 * 4096),   # kpad 256
-    (130, 64, 16, ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E1M2, 1, 2 * 1 * 512 + 2 * 1 * 4096),    # kpad 64: half a tile
-    (256, 512, 16, ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E2M1, 8, 2 * 8 * 512),                  # E2M1: atoms only
-    (129, 1000, 32, ufp4.SCALE_UE8M0, ufp4.GRID_E1M2, 8, 2 * 8 * 512),          # kpad 1024: 32 slots of 32
-    (1, 136, 32, ufp4.SCALE_UE8M0, ufp4.GRID_E1M2, 2, 1 * 2 * 512),             # kpad 192: 6 slots, 2 atoms
-    (0, 64, 16, ufp4.SCALE_E4M3_X_FP32, ufp4.GRID_E1M2, 1, 0),
+@pytest.mark.parametrize("rows,k,block,fmt,atoms_k,nbytes", [
+    (256, 512, 16, ufp4.SCALE_E4M3_X_FP32, 8, 2 * 8 * 512),
+    (300, 200, 32, ufp4.SCALE_E4M3_X_FP32, 4, 3 * 4 * 512),     # kpad 256: 16 slots of 16
+    (129, 1000, 32, ufp4.SCALE_UE8M0, 8, 2 * 8 * 512),          # kpad 1024: 32 slots of 32
+    (1, 136, 32, ufp4.SCALE_UE8M0, 2, 1 * 2 * 512),             # kpad 192: 6 slots, 2 atoms
+    (0, 64, 16, ufp4.SCALE_E4M3_X_FP32, 1, 0),
 ])
-def test_sf_atoms_layout(L, rows, k, block, fmt, grid, atoms_k, nbytes):
+def test_sf_atoms_layout(L, rows, k, block, fmt, atoms_k, nbytes):
     """Factor-atom plane size: ceil(rows/128) row groups x ceil(kpad / 4W)
-    atoms of 512 bytes (W = 16 for E4M3 factors, 32 for UE8M0), followed for
-    E1M2 operands with E4M3 factors by ceil(rows/128) x ceil(kpad/128)
-    per-lane factor tiles of 4096 bytes; none for fp32 scales."""
-    cfg = ufp4.QuantConfig(block=block, scale_fmt=fmt, grid=grid)
+    atoms of 512 bytes (W = 16 for E4M3 factors, 32 for UE8M0); none for
+    fp32 scales."""
+    cfg = ufp4.QuantConfig(block=block, scale_fmt=fmt)
     assert ufp4.sf_atoms_layout(rows, k, cfg) == (atoms_k, nbytes)
     c = ufp4.QuantConfig(scale_fmt=ufp4.SCALE_FP32).c()
     assert L.ufp4_sf_atoms_layout(64, 64, ctypes.byref(c), None, None) == ufp4.ERR_UNSUPPORTED
     c = cfg.c()
     assert L.ufp4_sf_atoms_layout(-1, 64, ctypes.byref(c), None, None) == ufp4.ERR_INVALID_ARG
     assert L.ufp4_sf_atoms_layout(64, 64, None, None, None) == ufp4.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("rows,k,block,grid,fmt,nbytes", [
+    (256, 512, 16, ufp4.GRID_E1M2, ufp4.SCALE_E4M3_X_FP32, 2 * 4 * 4096),
+    (300, 200, 32, ufp4.GRID_E1M2, ufp4.SCALE_E4M3_X_FP32, 3 * 2 * 4096),   # kpad 256
+    (130, 64, 16, ufp4.GRID_E1M2, ufp4.SCALE_E4M3_X_FP32, 2 * 1 * 4096),    # kpad 64: half a tile used
+    (0, 64, 16, ufp4.GRID_E1M2, ufp4.SCALE_E4M3_X_FP32, 0),
+    (256, 512, 16, ufp4.GRID_E2M1, ufp4.SCALE_E4M3_X_FP32, None),           # other grids: no tiles
+    (256, 512, 32, ufp4.GRID_E1M2, ufp4.SCALE_UE8M0, None),
+    (256, 512, 16, ufp4.GRID_E1M2, ufp4.SCALE_FP32, None),
+])
+def test_sf_lanes_layout(L, rows, k, block, grid, fmt, nbytes):
+    """Per-lane factor tiles: ceil(rows/128) x ceil(kpad/128) tiles of 4096
+    bytes, E1M2 operands with E4M3 x fp32 scales only (else UNSUPPORTED)."""
+    cfg = ufp4.QuantConfig(grid=grid, block=block, scale_fmt=fmt)
+    c = cfg.c()
+    nb = ctypes.c_size_t()
+    st = L.ufp4_sf_lanes_layout(rows, k, ctypes.byref(c), ctypes.byref(nb))
+    if nbytes is None:
+        assert st == ufp4.ERR_UNSUPPORTED
+    else:
+        assert st == ufp4.OK and nb.value == nbytes
+        assert ufp4.sf_lanes_layout(rows, k, cfg) == nbytes
+    assert L.ufp4_sf_lanes_layout(rows, k, ctypes.byref(c), None) == ufp4.ERR_INVALID_ARG
+    assert L.ufp4_sf_lanes_layout(-1, k, ctypes.byref(c), ctypes.byref(nb)) == ufp4.ERR_INVALID_ARG
 
 
 def _q(rows=128, k=256, **kw):

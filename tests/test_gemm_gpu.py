@@ -198,7 +198,9 @@ def test_factor_atoms_path_equals_factor_warps(grid, fmt, block):
     copies them into tensor memory) give bit-for-bit the output of the same
     kernel building the factors from the block-major scales, and the
     oracle's result; partial 256-wide tiles, one-row operands, K tails of 64
-    and of 128 + 64 (E2M1 stages 256 K: tails of 64, 192 and 256)."""
+    and of 128 + 64 (E2M1 stages 256 K: tails of 64, 192 and 256).  E1M2
+    operands also carry per-lane factor tiles, which the kernel uses for A:
+    A with and without them gives the same bits too."""
     import dataclasses
     cfg = _cfg(grid=grid, fmt=fmt, block=block)
     for (M, N, K) in [(520, 700, 448), (130, 230, 200), (1, 1, 8), (300, 513, 1000)]:
@@ -210,6 +212,10 @@ def test_factor_atoms_path_equals_factor_warps(grid, fmt, block):
         _check_full(qx, rx, qw, rw, ufp4.gemm_fprop)
         with_atoms = ufp4.gemm_fprop(qx, qw)
         plain = ufp4.gemm_fprop(dataclasses.replace(qx, sf_atoms=None), dataclasses.replace(qw, sf_atoms=None))
+        if qx.sf_lanes is not None:
+            no_lanes = ufp4.gemm_fprop(dataclasses.replace(qx, sf_lanes=None), qw)
+            torch.cuda.synchronize()
+            assert torch.equal(with_atoms, no_lanes), (M, N, K)
         torch.cuda.synchronize()
         assert ufp4.check_device_status() == ufp4.OK
         assert torch.equal(with_atoms, plain), (M, N, K)
